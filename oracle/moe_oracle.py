@@ -1,0 +1,407 @@
+"""Oracle: a plain, slow, fp64 CPU statement of the batch-invariant MoE layer forward.
+
+TEST INFRASTRUCTURE ONLY.  Nothing on the product path may import, call or
+execute this module: only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` use it.  It shares
+no code with the CUDA library and does not import it.
+
+Every step follows a passage of the source pages, cited by page title and
+section.  The pages (web articles, quoted here by short name):
+
+* [FW]  "MoE 模型中的訓練與推論一致性：數值漂移發生之處" -- a translation of the
+        Fireworks AI post on train/inference parity in MoE models
+        (easyvibecoding.app/curated/746).
+* [LC]  "美团把训练和推理的概率做到逐位相同:分歧藏在一个加法顺序里"
+        (bbs.huaweicloud.com/blogs/524918).
+* [DS]  "6 基建与训练稳定性优化" -- DeepSeek V4 infrastructure notes
+        (liyongzhi.xyz/files/deepseek_v4/sections/06-infra.html).
+* [LD]  The linux.do post on MoE FLOPs, parameters and variants
+        (feedbbs.com/linuxdo/72580).
+* [V4]  The nxmr.cn article on a "V4" MoE model (nxmr.cn/news/146660).
+
+The layer, in order:
+  1. input RMSNorm                       [LD] "RMSNorm before up-projection"
+  2. router logits  l = xn W_r^T         [DS] §6.3 "普通路由" (scores = W·h);
+                                          [V4] §2.2 (a Linear layer, logits per expert)
+  3. scores + top-k                      softmax [V4] §2.2; sigmoid + per-expert
+                                          bias [DS] §6.3 (upper layers), [LD] "QB"
+                                          (s + b > tau); hash [DS] §6.3
+  4. expert histogram, no capacity       [LD] "MoE是如何影响输出确定性的" (token
+                                          dropping is batch dependent: none here)
+  5. stable permute (dispatch)           [DS] §6.1 (dispatch -> compute -> combine)
+  6. routed + shared SwiGLU experts      [DS] §6.5, [LD] "SiTU-GLU" (SwiGLU form),
+                                          [LD] "共享专家"
+  7. weighted combine in fp32, one cast  [FW] Trap 3 and the case study ("standard
+                                          path": all k contributions kept in fp32,
+                                          weighted sum, one final cast)
+  8. residual add + RMSNorm epilogue     [FW] Trap 2 / Trap 3 (rmsnorm(full_out + residual))
+  9. fixed r0..r7 partial reduction      [FW] Trap 1 (Lamport kernel order)
+
+Precision.  Every floating-point step runs in fp64, on the bf16-rounded values
+the GPU path reads (x, residual, weights, xn between steps 1 and 2/6, h between
+the two expert matmuls).  Rounding to bf16 is done directly from fp64 (round to
+nearest, ties to even), never through fp32.  The one exception is step 9: the
+pages fix its precision (both all-reduce orders accumulate in FP32, [FW] Trap
+1), so the partial sums are emulated in IEEE fp32, left to right.
+
+Readings of points the pages leave open (each is also listed in the design
+notes): epsilon inside the square root; gains g_in = g_out = 1 unless given;
+ties in top-k go to the lower expert index and slots are ordered by
+descending key; the sigmoid bias only selects (weights use the unbiased
+score); a softmax logit bias, when given, is added to the logits before the
+softmax; hash routing takes e_0 = ((id * mult) mod 2^32) mod E and
+e_j = (e_0 + j) mod E with weight 1/k; the clamp bounds the gate from above
+only and the up branch on both sides; routed weights are multiplied by
+``routed_scale``; the routed sum is taken in slot order, then the shared
+experts in index order, then the residual is added.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+ROUTER_SOFTMAX, ROUTER_SIGMOID_BIAS, ROUTER_HASH = 0, 1, 2
+
+# Multiply-adds performed by expert matmuls since the last reset (FLOP pin).
+MAC_COUNTER = [0]
+
+
+# ----------------------------------------------------------------- bf16 data
+def bf16_bits_to_f64(bits) -> np.ndarray:
+    """Exact value of bf16 bit patterns."""
+    b = np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16
+    return b.view(np.float32).astype(np.float64)
+
+
+def round_bf16(a) -> np.ndarray:
+    """Round fp64 values to the nearest bf16 value, ties to even (fp64 result).
+
+    bf16 keeps 8 significant bits and fp32's exponent range.  Writing
+    a = m * 2^e with 0.5 <= |m| < 1, the rounding quantum is 2^(e-8), but
+    never finer than the subnormal spacing 2^-133.  np.rint rounds half to
+    even and the power-of-two scalings are exact, so this is one rounding.
+    """
+    a = np.asarray(a, dtype=np.float64)
+    _, e = np.frexp(a)
+    q = np.maximum(e.astype(np.int64) - 8, -133)
+    r = np.ldexp(np.rint(np.ldexp(a, -q)), q)
+    big = np.abs(r) > 3.3895313892515355e38  # (2 - 2^-7) * 2^127, the largest bf16
+    return np.where(big, np.copysign(np.inf, a), r)
+
+
+def f64_to_bf16_bits(a) -> np.ndarray:
+    """bf16 bit pattern of values that are already bf16-representable."""
+    f = np.asarray(a, dtype=np.float64).astype(np.float32)
+    return (f.view(np.uint32) >> 16).astype(np.uint16)
+
+
+# -------------------------------------------------------------- 1. RMSNorm
+def rmsnorm(x, g, eps: float) -> np.ndarray:
+    """RMSNorm(x) = g * x / sqrt(mean(x^2) + eps), over the last axis, fp64.
+
+    [LD] "RMSNorm before up-projection": RMS(x) = sqrt((1/d) sum x_i^2 + eps),
+    x_hat = x / RMS(x), y = g * x_hat (the epsilon sits inside the root).
+    """
+    x = np.asarray(x, dtype=np.float64)
+    ms = np.mean(x * x, axis=-1, keepdims=True)
+    return np.asarray(g, dtype=np.float64) * (x / np.sqrt(ms + eps))
+
+
+# ------------------------------------------------------- 2-3. router, top-k
+def router_logits(xn, w_router) -> np.ndarray:
+    """l[t, e] = sum_d xn[t, d] * W_r[e, d]: the router Linear ([V4] §2.2;
+    [DS] §6.3 "scores = W·h"), full K accumulated at once."""
+    return np.asarray(xn, np.float64) @ np.asarray(w_router, np.float64).T
+
+
+def topk_desc(keys, k: int) -> np.ndarray:
+    """Indices of the k largest keys per row, largest first; equal keys go to
+    the lower index; NaN ranks below every number.  (A stable sort of the
+    negated keys keeps equal keys in ascending index order.)"""
+    keys = np.asarray(keys, np.float64)
+    neg = np.where(np.isnan(keys), np.inf, -keys)
+    return np.argsort(neg, axis=-1, kind="stable")[..., :k].astype(np.int64)
+
+
+def softmax(z) -> np.ndarray:
+    z = np.asarray(z, np.float64)
+    m = np.max(z, axis=-1, keepdims=True)
+    p = np.exp(z - m)
+    return p / np.sum(p, axis=-1, keepdims=True)
+
+
+def sigmoid(z) -> np.ndarray:
+    return 1.0 / (1.0 + np.exp(-np.asarray(z, np.float64)))
+
+
+def route_softmax(logits, k: int, renormalize: bool, routed_scale: float, logit_bias=None):
+    """Softmax router ([V4] §2.2: Linear -> logits -> softmax weights -> top-k).
+
+    Optional logit bias b (a per-expert offset added to the logits, used for
+    the skewed workload).  Keys are the probabilities p; weights are p_j,
+    divided by the sum over the chosen k when ``renormalize``, times
+    ``routed_scale``.  Returns (idx [T,k], w [T,k], keys [T,E]).
+    """
+    z = np.asarray(logits, np.float64)
+    if logit_bias is not None:
+        z = z + np.asarray(logit_bias, np.float64)
+    p = softmax(z)
+    idx = topk_desc(p, k)
+    w = np.take_along_axis(p, idx, axis=-1)
+    if renormalize:
+        w = w / np.sum(w, axis=-1, keepdims=True)
+    return idx, w * routed_scale, p
+
+
+def route_sigmoid_bias(logits, bias, k: int, renormalize: bool, routed_scale: float):
+    """Sigmoid scores with a per-expert balancing bias ([DS] §6.3: upper layers
+    keep "sigmoid + balance"; [LD] "QuantileBalancing": expert e enters token
+    t's top-k when s_{t,e} + b_e exceeds the boundary).
+
+    The bias only selects: keys are s + b, weights are the unbiased s_j,
+    normalised over the chosen k when ``renormalize``, times ``routed_scale``.
+    """
+    s = sigmoid(logits)
+    keys = s + (0.0 if bias is None else np.asarray(bias, np.float64))
+    idx = topk_desc(keys, k)
+    w = np.take_along_axis(s, idx, axis=-1)
+    if renormalize:
+        w = w / np.sum(w, axis=-1, keepdims=True)
+    return idx, w * routed_scale, keys
+
+
+def hash_expert0(token_ids, E: int, mult: int) -> np.ndarray:
+    """[DS] §6.3 "Hash Routing": expert_id = hash(token_id) % n_experts, with
+    the multiplicative hash h(id) = (id * mult) mod 2^32."""
+    ids = np.asarray(token_ids, np.int64).astype(np.uint64)
+    h = (ids * np.uint64(mult)) & np.uint64(0xFFFFFFFF)
+    return (h % np.uint64(E)).astype(np.int64)
+
+
+def route_hash(token_ids, E: int, k: int, mult: int, routed_scale: float):
+    """Hash routing with k experts: e_j = (e_0 + j) mod E (distinct experts), no
+    router parameters, equal weights 1/k times ``routed_scale``."""
+    e0 = hash_expert0(token_ids, E, mult)
+    idx = (e0[:, None] + np.arange(k)[None, :]) % E
+    w = np.full(idx.shape, routed_scale / k, np.float64)
+    return idx.astype(np.int64), w, None
+
+
+def route(cfg, logits, bias, token_ids):
+    """Dispatch on the router variant; returns (idx, w, keys)."""
+    if cfg.router == ROUTER_SOFTMAX:
+        return route_softmax(logits, cfg.k, bool(cfg.renormalize), cfg.routed_scale, bias)
+    if cfg.router == ROUTER_SIGMOID_BIAS:
+        return route_sigmoid_bias(logits, bias, cfg.k, bool(cfg.renormalize), cfg.routed_scale)
+    if cfg.router == ROUTER_HASH:
+        return route_hash(token_ids, cfg.E, cfg.k, cfg.hash_mult, cfg.routed_scale)
+    raise ValueError(f"unknown router {cfg.router}")
+
+
+def topk_margin(keys, k: int) -> np.ndarray:
+    """key of the k-th chosen expert minus the (k+1)-th largest key: the
+    boundary tau_t of [LD] "QuantileBalancing" seen from the chosen side.
+    A token whose margin is tiny can flip experts under any perturbation
+    ([LD] "MoE是如何影响输出确定性的")."""
+    if keys is None:
+        return None
+    keys = np.asarray(keys, np.float64)
+    if k >= keys.shape[-1]:
+        return np.full(keys.shape[0], np.inf)
+    s = -np.sort(-np.where(np.isnan(keys), -np.inf, keys), axis=-1)
+    return s[:, k - 1] - s[:, k]
+
+
+# --------------------------------------------------- 4-5. histogram, permute
+def expert_histogram(idx, E: int) -> np.ndarray:
+    """counts[e] = number of (token, slot) pairs routed to e.  Dropless: no
+    capacity, so no token depends on the rest of the batch."""
+    return np.bincount(np.asarray(idx).ravel(), minlength=E).astype(np.int64)
+
+
+def stable_permute(idx, E: int):
+    """Group (token, slot) pairs by expert; inside expert e's segment the rows
+    are in ascending token order (a token picks an expert at most once).
+
+    Returns offsets [E+1] (exclusive prefix of the histogram), perm_token and
+    perm_slot [T*k] (row p of the grouped order holds token perm_token[p],
+    slot perm_slot[p]) and pos [T, k] (the inverse map).
+    """
+    idx = np.asarray(idx, np.int64)
+    T, k = idx.shape
+    counts = expert_histogram(idx, E)
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int64)
+    flat = idx.ravel()                       # flat position f = t*k + j
+    order = np.argsort(flat, kind="stable")  # by expert, then by f (i.e. by t)
+    perm_token = order // k
+    perm_slot = order % k
+    pos = np.empty(T * k, np.int64)
+    pos[order] = np.arange(T * k)
+    return offsets, perm_token, perm_slot, pos.reshape(T, k)
+
+
+# -------------------------------------------------------------- 6. experts
+def swiglu(g, u, gate_clamp_max: float = np.inf, up_clamp: float = np.inf) -> np.ndarray:
+    """SwiGLU(x) = SiLU(W_g x) * (W_u x) with Swish(a) = a * sigmoid(a)
+    ([LD] "SiTU-GLU", SwiGLU form); with the clamp of [DS] §6.5,
+    SiLU(clamp(W_g x, max=c_g)) * clamp(W_u x, -c_u, c_u)."""
+    g = np.minimum(np.asarray(g, np.float64), gate_clamp_max)
+    u = np.clip(np.asarray(u, np.float64), -up_clamp, up_clamp)
+    return g * sigmoid(g) * u
+
+
+def expert_ffn(xn_rows, w_gate, w_up, w_down, gate_clamp_max=np.inf, up_clamp=np.inf):
+    """One SwiGLU expert on a block of rows: g = xn W_g^T, u = xn W_u^T (full
+    K = D), h = bf16(SwiGLU(g, u)), y = h W_d^T (full K = I).  Returns (h, y)."""
+    x = np.asarray(xn_rows, np.float64)
+    Wg = np.asarray(w_gate, np.float64)
+    Wu = np.asarray(w_up, np.float64)
+    Wd = np.asarray(w_down, np.float64)
+    n, D = x.shape
+    I = Wg.shape[0]
+    MAC_COUNTER[0] += n * (2 * D * I + I * Wd.shape[0])
+    h = round_bf16(swiglu(x @ Wg.T, x @ Wu.T, gate_clamp_max, up_clamp))
+    return h, h @ Wd.T
+
+
+# --------------------------------------------- 7-8. combine + residual + norm
+def combine(w, y_slots, y_shared) -> np.ndarray:
+    """acc[t] = sum_j w[t,j] * y[t,j] (slot order) + sum_s y_shared[s,t]
+    ([FW] Trap 3, unfused path: moe_finalize, then += shared_expert; the
+    case study's standard path keeps all k contributions and sums them in
+    one weighted sum before a single cast)."""
+    acc = np.einsum("tj,tjd->td", np.asarray(w, np.float64), np.asarray(y_slots, np.float64))
+    if y_shared is not None and len(y_shared):
+        acc = acc + np.sum(np.asarray(y_shared, np.float64), axis=0)
+    return acc
+
+
+def residual_rmsnorm(acc, residual, g_out, eps: float):
+    """r = full_out + residual; returns (bf16(RMSNorm(r)), bf16(r), r)
+    ([FW] Trap 2 / Trap 3: normed, residual = rmsnorm(full_out + residual))."""
+    r = np.asarray(acc, np.float64) + np.asarray(residual, np.float64)
+    return round_bf16(rmsnorm(r, g_out, eps)), round_bf16(r), r
+
+
+# ------------------------------------------------ 9. partial-sum epilogue
+def allreduce_fixed_order_f32(partials) -> np.ndarray:
+    """r0 + r1 + ... + r_{P-1}, left to right, every element, IEEE fp32
+    ([FW] Trap 1: the Lamport kernel's uniform r0..r7 order, FP32 accumulation)."""
+    parts = np.asarray(partials, dtype=np.float32)
+    acc = parts[0].copy()
+    for p in range(1, parts.shape[0]):
+        acc = np.add(acc, parts[p], dtype=np.float32)
+    return acc
+
+
+def allreduce_ring_order_f32(partials) -> np.ndarray:
+    """The NCCL ring reduce-scatter order ([FW] Trap 1): the hidden vector is cut
+    into P contiguous chunks; chunk c starts from its owner r_c and then adds
+    r_{c-1}, r_{c-2}, ... around the ring, in fp32.  Used only to show that a
+    different order changes bits."""
+    parts = np.asarray(partials, dtype=np.float32)
+    P, D = parts.shape[0], parts.shape[-1]
+    bounds = [(c * D) // P for c in range(P + 1)]
+    out = np.empty(parts.shape[1:], np.float32)
+    for c in range(P):
+        sl = slice(bounds[c], bounds[c + 1])
+        acc = parts[c][..., sl].copy()
+        for step in range(1, P):
+            acc = np.add(acc, parts[(c - step) % P][..., sl], dtype=np.float32)
+        out[..., sl] = acc
+    return out
+
+
+def reduce_partials(partials, residual, g, eps: float):
+    """The tensor-parallel epilogue simulated on one GPU: r = (r0 + ... + r7) +
+    residual, all in fp32 (the sum in fixed order), then RMSNorm in fp64 on that
+    fp32 r.  Returns (bf16(RMSNorm(r)), bf16(r), r as fp32)."""
+    s = allreduce_fixed_order_f32(partials)
+    r = np.add(s, np.asarray(residual, np.float32), dtype=np.float32)
+    out_residual = round_bf16(r.astype(np.float64))
+    out_norm = round_bf16(rmsnorm(r.astype(np.float64), g, eps))
+    return out_norm, out_residual, r
+
+
+# ------------------------------------------------------------- the layer
+class Weights:
+    """In-memory weights (fp64 arrays holding bf16 values).  Any object with the
+    same attributes and ``routed(e)`` / ``shared(s)`` methods will do, e.g. one
+    that regenerates a single expert on demand."""
+
+    def __init__(self, w_router, router_bias, w_gate, w_up, w_down, ws_gate, ws_up, ws_down,
+                 g_in, g_out):
+        self.w_router = w_router
+        self.router_bias = router_bias
+        self.w_gate, self.w_up, self.w_down = w_gate, w_up, w_down
+        self.ws_gate, self.ws_up, self.ws_down = ws_gate, ws_up, ws_down
+        self.g_in, self.g_out = g_in, g_out
+
+    def routed(self, e):
+        return self.w_gate[e], self.w_up[e], self.w_down[e]
+
+    def shared(self, s):
+        return self.ws_gate[s], self.ws_up[s], self.ws_down[s]
+
+
+def moe_layer(cfg, W, x, residual, token_ids=None, rows=None) -> dict:
+    """The whole layer.  Routing, histogram and permutation are computed for
+    every token; the experts, combine and epilogue for ``rows`` (all tokens
+    when None).  ``cfg`` carries D, E, k, I, n_shared, I_shared, router,
+    renormalize, routed_scale, gate_clamp_max, up_clamp, eps, hash_mult."""
+    x = np.asarray(x, np.float64)
+    T = x.shape[0]
+    rows = np.arange(T) if rows is None else np.asarray(rows, np.int64)
+    xn = round_bf16(rmsnorm(x, W.g_in, cfg.eps))
+    logits = None
+    if cfg.router != ROUTER_HASH:
+        logits = router_logits(xn, W.w_router)
+    idx, w, keys = route(cfg, logits, W.router_bias, token_ids)
+    margin = topk_margin(keys, cfg.k)
+    counts = expert_histogram(idx, cfg.E)
+    offsets, perm_token, perm_slot, pos = stable_permute(idx, cfg.E)
+
+    # Expert compute for the selected rows, grouped by expert.
+    n, k = len(rows), cfg.k
+    y_slots = np.zeros((n, k, cfg.D))
+    sel = idx[rows]                                   # [n, k]
+    for e in np.unique(sel):
+        rr, jj = np.nonzero(sel == e)
+        Wg, Wu, Wd = W.routed(int(e))
+        _, y = expert_ffn(xn[rows[rr]], Wg, Wu, Wd, cfg.gate_clamp_max, cfg.up_clamp)
+        y_slots[rr, jj] = y
+    y_shared = np.zeros((cfg.n_shared, n, cfg.D))
+    for s in range(cfg.n_shared):
+        Wg, Wu, Wd = W.shared(s)
+        # The clamp is a property of the SwiGLU unit and applies to shared experts too.
+        _, y_shared[s] = expert_ffn(xn[rows], Wg, Wu, Wd, cfg.gate_clamp_max, cfg.up_clamp)
+    acc = combine(w[rows], y_slots, y_shared)
+    out_norm, out_residual, r = residual_rmsnorm(acc, np.asarray(residual, np.float64)[rows],
+                                                 W.g_out, cfg.eps)
+    return dict(rows=rows, xn=xn, logits=logits, keys=keys, idx=idx, w=w, margin=margin,
+                counts=counts, offsets=offsets, perm_token=perm_token, perm_slot=perm_slot,
+                pos=pos, y_slots=y_slots, y_shared=y_shared, acc=acc, r=r,
+                out_norm=out_norm, out_residual=out_residual)
+
+
+def moe_layer_dense_masked(cfg, W, x, residual, token_ids=None) -> dict:
+    """Cross-check of the routed path: run every expert on every token, weight
+    each output by the token's routing weight for that expert (0 when not
+    chosen) and sum over all experts.  Mathematically equal to ``moe_layer``."""
+    x = np.asarray(x, np.float64)
+    T = x.shape[0]
+    xn = round_bf16(rmsnorm(x, W.g_in, cfg.eps))
+    logits = None if cfg.router == ROUTER_HASH else router_logits(xn, W.w_router)
+    idx, w, _ = route(cfg, logits, W.router_bias, token_ids)
+    mask = np.zeros((T, cfg.E))
+    np.put_along_axis(mask, idx, w, axis=-1)
+    acc = np.zeros((T, cfg.D))
+    for e in range(cfg.E):
+        Wg, Wu, Wd = W.routed(e)
+        _, y = expert_ffn(xn, Wg, Wu, Wd, cfg.gate_clamp_max, cfg.up_clamp)
+        acc += mask[:, e:e + 1] * y
+    for s in range(cfg.n_shared):
+        Wg, Wu, Wd = W.shared(s)
+        _, y = expert_ffn(xn, Wg, Wu, Wd, cfg.gate_clamp_max, cfg.up_clamp)
+        acc += y
+    out_norm, out_residual, r = residual_rmsnorm(acc, residual, W.g_out, cfg.eps)
+    return dict(acc=acc, r=r, out_norm=out_norm, out_residual=out_residual, idx=idx, w=w)

@@ -1,0 +1,361 @@
+"""Pins for the oracle: checks against what the pages and the mathematics fix.
+
+Each ``pin_*`` takes the oracle module ``O`` and raises AssertionError when the
+oracle disagrees with its pin.  ``test_oracle_pins.py`` runs them on the real
+oracle; ``test_oracle_mutations.py`` runs them on copies with planted mistakes
+and requires every mistake to trip at least one pin.
+
+Pins use worked examples printed on the pages (``tests/golden``), closed
+forms derived by hand for tiny inputs, brute force, invariants, and library
+routines on special cases (torch's fp32 -> bf16 rounding).
+"""
+from __future__ import annotations
+
+import json
+import math
+import os
+import types
+
+import numpy as np
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def _cfg(**kw):
+    base = dict(D=2, E=2, k=1, I=2, n_shared=0, I_shared=2, router=0, renormalize=0,
+                routed_scale=1.0, gate_clamp_max=math.inf, up_clamp=math.inf, eps=1e-6,
+                hash_mult=2654435761)
+    base.update(kw)
+    return types.SimpleNamespace(**base)
+
+
+def _torch_bf16(v):
+    """Library routine: torch's fp32 -> bf16 conversion (round to nearest even)."""
+    import torch
+    return torch.tensor(np.asarray(v, np.float32)).to(torch.bfloat16).to(torch.float64).numpy()
+
+
+# ------------------------------------------------------------------ bf16
+def pin_round_bf16(O):
+    # Ties go to even: 1 + 2^-8 lies halfway between 1 and 1 + 2^-7.
+    assert O.round_bf16(1 + 2.0 ** -8) == 1.0
+    assert O.round_bf16(1 + 3 * 2.0 ** -8) == 1 + 2.0 ** -6
+    assert O.round_bf16(-(1 + 2.0 ** -8)) == -1.0
+    # Just above a tie rounds up; rounding through fp32 first would land on
+    # the tie and round down (double rounding), so this pins one rounding.
+    assert O.round_bf16(1 + 2.0 ** -8 + 2.0 ** -40) == 1 + 2.0 ** -7
+    # 3/sqrt(12.5) = 0.84852...: quantum 2^-9 in [0.5, 1), 434.45 -> 434.
+    assert O.round_bf16(3 / math.sqrt(12.5)) == 434 * 2.0 ** -9
+    # fp32-representable values: agree with torch's RNE conversion.
+    rng = np.random.default_rng(5)
+    v = np.concatenate([rng.standard_normal(20000) * 10.0 ** rng.integers(-30, 30, 20000),
+                        [0.0, -0.0, 1e-40, -3e-39, 3.3e38]]).astype(np.float32).astype(np.float64)
+    assert np.array_equal(O.round_bf16(v), _torch_bf16(v))
+
+
+# --------------------------------------------------------------- RMSNorm
+def pin_rmsnorm_worked_example(O):
+    g = golden("rmsnorm_worked_example.json")
+    x = np.array([g["x"]])
+    y = O.rmsnorm(x, np.ones(2), 1e-6)[0]
+    tol = 0.5 * 10.0 ** -g["printed_decimals"] + 1e-6
+    rms = math.sqrt((3.0 ** 2 + 4.0 ** 2) / 2)  # the page's RMS, 3.536
+    assert abs(rms - g["rms_printed"]) <= tol
+    assert np.allclose(y, g["normalized_printed"], atol=tol, rtol=0)
+    assert abs(math.sqrt(np.mean(y * y)) - g["rms_of_output_printed"]) <= tol
+    # The epsilon sits inside the root: with eps = 1, RMS = sqrt(12.5 + 1).
+    y1 = O.rmsnorm(x, np.ones(2), 1.0)[0]
+    assert np.allclose(y1, [3 / math.sqrt(13.5), 4 / math.sqrt(13.5)], rtol=1e-15, atol=0)
+    # Gains multiply element-wise after the normalisation.
+    y2 = O.rmsnorm(x, np.array([2.0, -0.5]), 0.0)[0]
+    assert np.allclose(y2, [2 * 3 / math.sqrt(12.5), -0.5 * 4 / math.sqrt(12.5)], rtol=1e-15)
+
+
+def pin_rmsnorm_scale_invariance(O):
+    g = golden("rmsnorm_scale_invariance.json")
+    u = np.random.default_rng(1).standard_normal((4, 64))
+    a = O.rmsnorm(u, np.ones(64), 0.0)
+    b = O.rmsnorm(g["scale"] * u, np.ones(64), 0.0)
+    assert np.allclose(a, b, rtol=1e-13, atol=0)
+    # Each normalised row has RMS 1 (eps = 0).
+    assert np.allclose(np.sqrt(np.mean(a * a, axis=-1)), 1.0, rtol=1e-13)
+
+
+# ------------------------------------------------------------------ SwiGLU
+def pin_swish_example(O):
+    g = golden("swish_worked_example.json")
+    v = float(O.swiglu(g["gate"], g["up"]))
+    assert abs(v - g["printed"]) <= 1e-3 * g["printed"]
+    # Closed form: Swish(20) * 30 = 600 / (1 + e^-20).
+    assert abs(v - 600.0 / (1.0 + math.exp(-20.0))) <= 1e-12 * 600
+    # Swish(a) = a * sigmoid(a): Swish(0) = 0 and Swish(-a) = Swish(a) - a.
+    assert float(O.swiglu(0.0, 5.0)) == 0.0
+    a = 1.7
+    assert abs(float(O.swiglu(-a, 1.0)) - (float(O.swiglu(a, 1.0)) - a)) < 1e-15
+
+
+def pin_swiglu_clamp(O):
+    g = golden("swiglu_clamp.json")
+    cg, cu = g["gate_clamp_max"], g["up_clamp"]
+    silu10 = 10.0 / (1.0 + math.exp(-10.0))
+    # Large inputs: SiLU(10) * 10, below 10 * 10.
+    assert abs(float(O.swiglu(20.0, 30.0, cg, cu)) - silu10 * 10) < 1e-12
+    assert float(O.swiglu(20.0, 30.0, cg, cu)) < 100.0
+    assert abs(float(O.swiglu(20.0, -30.0, cg, cu)) + silu10 * 10) < 1e-12
+    # The gate has no lower bound: SiLU(-20) * (-10), not SiLU(-10) * (-10).
+    want = (-20.0 / (1.0 + math.exp(20.0))) * -10.0
+    assert abs(float(O.swiglu(-20.0, -30.0, cg, cu)) - want) < 1e-18
+    # Inside the bounds the clamp changes nothing.
+    rng = np.random.default_rng(2)
+    gg, uu = rng.uniform(-9.9, 9.9, 1000), rng.uniform(-9.9, 9.9, 1000)
+    assert np.array_equal(O.swiglu(gg, uu, cg, cu), O.swiglu(gg, uu))
+    # Bound over any input: |out| <= SiLU(10) * 10.
+    big = rng.standard_normal((2, 10000)) * 50
+    assert np.max(np.abs(O.swiglu(big[0], big[1], cg, cu))) <= silu10 * 10 + 1e-12
+
+
+# ------------------------------------------------------------------ top-k
+def _brute_topk(row, k):
+    order = sorted(range(len(row)), key=lambda e: (-row[e], e))
+    return order[:k]
+
+
+def pin_topk_bruteforce(O):
+    rng = np.random.default_rng(3)
+    for E, k in [(8, 2), (64, 6), (256, 8), (5, 5), (7, 1)]:
+        keys = np.round(rng.standard_normal((50, E)), 1)  # rounding makes many ties
+        got = O.topk_desc(keys, k)
+        for t in range(50):
+            assert list(got[t]) == _brute_topk(list(keys[t]), k), (E, k, t)
+    # All equal: the lowest indices, in order.
+    assert list(O.topk_desc(np.zeros((1, 6)), 3)[0]) == [0, 1, 2]
+
+
+def pin_margin(O):
+    keys = np.array([[0.1, 0.5, 0.3, 0.45]])
+    assert abs(O.topk_margin(keys, 2)[0] - (0.45 - 0.3)) < 1e-15
+    assert abs(O.topk_margin(keys, 1)[0] - (0.5 - 0.45)) < 1e-15
+    assert O.topk_margin(keys, 4)[0] == np.inf
+
+
+# ------------------------------------------------------------------ routers
+def pin_softmax_router(O):
+    # E = 2, k = 1: the chosen weight is p_max = sigmoid(l_max - l_min).
+    logits = np.array([[0.2, 1.1], [3.0, -1.0]])
+    idx, w, _ = O.route_softmax(logits, 1, False, 1.0)
+    assert list(idx[:, 0]) == [1, 0]
+    assert abs(w[0, 0] - 1 / (1 + math.exp(-0.9))) < 1e-15
+    assert abs(w[1, 0] - 1 / (1 + math.exp(-4.0))) < 1e-15
+    # Renormalised weights sum to routed_scale; plain ones are the probabilities.
+    rng = np.random.default_rng(4)
+    L = rng.standard_normal((20, 64))
+    idx, w, p = O.route_softmax(L, 6, True, 1.0)
+    assert np.allclose(w.sum(-1), 1.0, rtol=1e-14)
+    idx2, w2, _ = O.route_softmax(L, 6, False, 1.0)
+    assert np.array_equal(idx, idx2)
+    assert np.allclose(w2.sum(-1), np.sort(p, -1)[:, -6:].sum(-1), rtol=1e-14)
+    assert np.all(w2.sum(-1) < 1.0)
+    # A logit bias is added before the softmax.
+    idx3, w3, _ = O.route_softmax(np.array([[0.0, 0.0]]), 1, False, 1.0, np.array([0.0, math.log(3)]))
+    assert idx3[0, 0] == 1 and abs(w3[0, 0] - 0.75) < 1e-15
+
+
+def pin_sigmoid_router(O):
+    # The bias moves selection but not the weights: expert 0 has the larger
+    # score, expert 1 wins on score + bias, and its weight uses its own score.
+    logits = np.array([[1.0, 0.5, -2.0]])
+    bias = np.array([0.0, 0.2, 0.0])
+    s = [1 / (1 + math.exp(-v)) for v in logits[0]]
+    idx, w, _ = O.route_sigmoid_bias(logits, bias, 1, False, 1.0)
+    assert idx[0, 0] == 1 and abs(w[0, 0] - s[1]) < 1e-15
+    idx, w, _ = O.route_sigmoid_bias(logits, bias, 2, True, 2.5)
+    assert list(idx[0]) == [1, 0]
+    assert abs(w[0, 0] - 2.5 * s[1] / (s[0] + s[1])) < 1e-15
+    rng = np.random.default_rng(6)
+    L = rng.standard_normal((30, 256)) * 1.7
+    _, w, _ = O.route_sigmoid_bias(L, rng.standard_normal(256) * 0.01, 8, True, 2.5)
+    assert np.allclose(w.sum(-1), 2.5, rtol=1e-14)
+
+
+def pin_hash(O):
+    g = golden("hash_routing.json")
+    for c in g["cases"]:
+        assert int(O.hash_expert0(np.array([c["id"]]), c["E"], g["mult"])[0]) == c["expert"], c
+    idx, w, _ = O.route_hash(np.array([1, 2]), 128, 8, g["mult"], 1.0)
+    assert list(idx[0]) == [(49 + j) % 128 for j in range(8)]
+    assert list(idx[1]) == [(98 + j) % 128 for j in range(8)]
+    assert np.all(w == 1.0 / 8)
+    # Wrap-around keeps the k experts distinct.
+    idx, _, _ = O.route_hash(np.array([1]), 50, 8, g["mult"], 1.0)  # e0 = 2654435761 % 50 = 11
+    assert list(idx[0]) == list(range(11, 19))
+    idx, _, _ = O.route_hash(np.array([3]), 8, 8, g["mult"], 1.0)   # e0 = 0xDAA66D13 % 8 = 3
+    assert sorted(idx[0]) == list(range(8)) and idx[0, 0] == 3
+
+
+# -------------------------------------------------------- histogram/permute
+def pin_histogram_permute_bruteforce(O):
+    rng = np.random.default_rng(7)
+    for T, E, k in [(40, 8, 2), (100, 16, 4), (33, 5, 5), (1, 8, 3)]:
+        idx = np.stack([rng.permutation(E)[:k] for _ in range(T)])
+        counts = O.expert_histogram(idx, E)
+        offsets, ptok, pslot, pos = O.stable_permute(idx, E)
+        want_counts = [sum(1 for t in range(T) for j in range(k) if idx[t, j] == e) for e in range(E)]
+        assert list(counts) == want_counts
+        rows = []
+        for e in range(E):
+            seg = sorted((t, j) for t in range(T) for j in range(k) if idx[t, j] == e)
+            assert offsets[e] == len(rows)
+            rows += seg
+        assert offsets[E] == T * k
+        assert list(zip(ptok.tolist(), pslot.tolist())) == rows
+        for p, (t, j) in enumerate(rows):
+            assert pos[t, j] == p
+
+
+# ---------------------------------------------------- partial-sum epilogue
+def pin_fixed_vs_ring_order(O):
+    # Non-associativity (the pages' (a + b) + c != a + (b + c)), by hand in
+    # fp32 with three partials and one element per chunk:
+    #   fixed, every element: (1 + 2^-24) + 2^-24 = 1 + 2^-24 -> 1 (tie, even), then 1.
+    #   ring, chunk 2 (owner r2): (2^-24 + 2^-24) + 1 = 2^-23 + 1, representable.
+    r = np.zeros((3, 3), np.float32)
+    r[0, :] = 1.0
+    r[1, :] = 2.0 ** -24
+    r[2, :] = 2.0 ** -24
+    assert np.array_equal(O.allreduce_fixed_order_f32(r), np.float32([1, 1, 1]))
+    assert np.array_equal(O.allreduce_ring_order_f32(r), np.float32([1, 1, 1 + 2.0 ** -23]))
+    # Chunk ownership follows the ring (chunk c: r_c, r_{c-1}, ...).  P = 4,
+    # r0 = r1 = 2^-24, r2 = 2, r3 = -2; fp32 ulp is 2^-23 in [1,2), 2^-22 in [2,4):
+    #   fixed, every element: ((2^-23) + 2) -> tie -> 2 ; - 2 = 0.
+    #   chunk 0: r0 + r3 = -(2 - 2^-24) -> tie -> -2 ; + 2 = 0 ; + 2^-24 = 2^-24.
+    #   chunk 1: r1 + r0 = 2^-23 ; - 2 = -(2 - 2^-23), exact ; + 2 = 2^-23.
+    #   chunk 2: r2 + r1 -> 2 ; + r0 -> 2 ; - 2 = 0.
+    #   chunk 3: r3 + r2 = 0 ; + 2^-24 ; + 2^-24 = 2^-23.
+    q = np.zeros((4, 4), np.float32)
+    q[0, :] = 2.0 ** -24
+    q[1, :] = 2.0 ** -24
+    q[2, :] = 2.0
+    q[3, :] = -2.0
+    assert np.array_equal(O.allreduce_fixed_order_f32(q), np.float32([0, 0, 0, 0]))
+    assert np.array_equal(O.allreduce_ring_order_f32(q),
+                          np.float32([2.0 ** -24, 2.0 ** -23, 0, 2.0 ** -23]))
+    # Random case: both orders stay within the fp32 error bound of the exact sum.
+    rng = np.random.default_rng(8)
+    parts = (rng.standard_normal((8, 4, 512)) / 8).astype(np.float32)
+    exact = parts.astype(np.float64).sum(0)
+    bound = 7 * 2.0 ** -24 * np.abs(parts.astype(np.float64)).sum(0) * 1.0001
+    for got in (O.allreduce_fixed_order_f32(parts), O.allreduce_ring_order_f32(parts)):
+        assert np.all(np.abs(got.astype(np.float64) - exact) <= bound)
+    assert not np.array_equal(O.allreduce_fixed_order_f32(parts), O.allreduce_ring_order_f32(parts))
+
+
+def pin_reduce_partials(O):
+    # r = fixed-order sum + residual in fp32; one element by hand:
+    # partials 0.5, 0.25, 2^-30 ... sum = 0.75 (2^-30 lost), + residual 1.0 = 1.75.
+    parts = np.zeros((3, 1, 2), np.float32)
+    parts[:, 0, 0] = [0.5, 0.25, 2.0 ** -30]
+    parts[:, 0, 1] = [-1.0, 0.0, 0.0]
+    res = np.array([[1.0, 0.0]], np.float32)
+    out_norm, out_res, r = O.reduce_partials(parts, res, np.ones(2), 0.0)
+    assert r[0, 0] == np.float32(1.75) and r[0, 1] == np.float32(-1.0)
+    assert np.array_equal(out_res[0], [1.75, -1.0])
+    rms = math.sqrt((1.75 ** 2 + 1.0) / 2)
+    assert np.allclose(out_norm[0], _torch_bf16([1.75 / rms, -1.0 / rms]), rtol=0, atol=0)
+
+
+# --------------------------------------------------------- closed-form layer
+def closed_form_case():
+    """T=1, D=2, I=2, E=2, top-1 softmax, one shared expert, chosen so every
+    step can be done by hand."""
+    cfg = _cfg(D=2, E=2, k=1, I=2, n_shared=1, I_shared=2)
+    Z = np.zeros((2, 2))
+    w_router = np.array([[1.0, 0.0], [0.0, 1.0]])            # logits = xn
+    w_gate = np.stack([Z, [[1.0, 0.0], [0.0, 0.0]]])          # g = [xn0, 0]
+    w_up = np.stack([Z, [[0.0, 1.0], [1.0, 0.0]]])            # u = [xn1, xn0]
+    w_down = np.stack([Z, [[1.0, 0.0], [-1.0, 0.0]]])         # y = [h0, -h0]
+    ws_gate = np.array([[[0.0, 1.0], [0.0, 0.0]]])            # gs = [xn1, 0]
+    ws_up = np.array([[[1.0, 0.0], [0.0, 0.0]]])              # us = [xn0, 0]
+    ws_down = np.array([[[0.0, 0.0], [1.0, 0.0]]])            # ys = [0, hs0]
+    W = types.SimpleNamespace(w_router=w_router, router_bias=None, g_in=np.ones(2),
+                              g_out=np.ones(2))
+    W.routed = lambda e: (w_gate[e], w_up[e], w_down[e])
+    W.shared = lambda s: (ws_gate[s], ws_up[s], ws_down[s])
+    x = np.array([[3.0, 4.0]])
+    residual = np.array([[0.5, -0.25]])
+    return cfg, W, x, residual
+
+
+def pin_closed_form_layer(O):
+    cfg, W, x, residual = closed_form_case()
+    out = O.moe_layer(cfg, W, x, residual)
+    # By hand.  RMS([3,4]) = sqrt(12.5 + 1e-6); xn = bf16(3/RMS, 4/RMS):
+    # 0.848528 -> 434 * 2^-9 = 0.84765625 ; 1.131371 -> 145 * 2^-7 = 1.1328125.
+    xn0, xn1 = 434 * 2.0 ** -9, 145 * 2.0 ** -7
+    assert np.array_equal(out["xn"][0], [xn0, xn1])
+    # Router: logits = xn; expert 1 wins; weight = p_1 = 1/(1 + e^-(xn1 - xn0)).
+    assert out["idx"][0, 0] == 1
+    w = 1.0 / (1.0 + math.exp(-(xn1 - xn0)))
+    assert abs(out["w"][0, 0] - w) < 1e-15
+    silu = lambda a: a / (1.0 + math.exp(-a))  # noqa: E731
+    h0 = float(_torch_bf16(silu(xn0) * xn1))      # gate = xn0, up = xn1
+    hs0 = float(_torch_bf16(silu(xn1) * xn0))     # shared: gate = xn1, up = xn0
+    r = np.array([w * h0 + 0.5, -w * h0 + hs0 - 0.25])
+    assert np.allclose(out["r"][0], r, rtol=1e-15, atol=1e-16)
+    rms = math.sqrt((r[0] ** 2 + r[1] ** 2) / 2 + 1e-6)
+    assert np.array_equal(out["out_residual"][0], _torch_bf16(r))
+    assert np.array_equal(out["out_norm"][0], _torch_bf16(r / rms))
+    # Counts / permutation of the single routed row.
+    assert list(out["counts"]) == [0, 1] and list(out["offsets"]) == [0, 0, 1]
+
+
+# ---------------------------------------------------------- dense cross-check
+def small_random_case(O, router=0, T=24, D=64, E=8, k=2, I=32, S=1, seed=9, **kw):
+    rng = np.random.default_rng(seed)
+    bf = lambda a: O.round_bf16(a)  # noqa: E731
+    cfg = _cfg(D=D, E=E, k=k, I=I, n_shared=S, I_shared=I, router=router, **kw)
+    W = O.Weights(
+        w_router=bf(rng.standard_normal((E, D)) * 0.3),
+        router_bias=(rng.standard_normal(E) * 0.01) if router == 1 else None,
+        w_gate=bf(rng.standard_normal((E, I, D)) * 0.1), w_up=bf(rng.standard_normal((E, I, D)) * 0.1),
+        w_down=bf(rng.standard_normal((E, D, I)) * 0.1),
+        ws_gate=bf(rng.standard_normal((S, I, D)) * 0.1), ws_up=bf(rng.standard_normal((S, I, D)) * 0.1),
+        ws_down=bf(rng.standard_normal((S, D, I)) * 0.1),
+        g_in=bf(1 + 0.1 * rng.standard_normal(D)), g_out=bf(1 + 0.1 * rng.standard_normal(D)))
+    x = bf(rng.standard_normal((T, D)))
+    res = bf(rng.standard_normal((T, D)))
+    ids = rng.integers(0, 128000, T)
+    return cfg, W, x, res, ids
+
+
+def pin_dense_masked(O):
+    for router, extra in [(0, {}), (0, {"renormalize": 1}), (1, {"renormalize": 1, "routed_scale": 2.5,
+                                                                     "gate_clamp_max": 0.3, "up_clamp": 0.3}),
+                          (2, {})]:
+        cfg, W, x, res, ids = small_random_case(O, router=router, **extra)
+        a = O.moe_layer(cfg, W, x, res, ids)
+        b = O.moe_layer_dense_masked(cfg, W, x, res, ids)
+        assert np.allclose(a["r"], b["r"], rtol=1e-12, atol=1e-12), router
+        assert np.array_equal(a["idx"], b["idx"])
+        # Sampled rows give the same rows as the full run.
+        rows = np.array([3, 0, 17])
+        c = O.moe_layer(cfg, W, x, res, ids, rows=rows)
+        assert np.array_equal(c["out_norm"], a["out_norm"][rows])
+
+
+def pin_mac_count(O):
+    # [LD] "FLOPs与参数量": an MoE with k active experts costs k times one expert;
+    # a SwiGLU expert multiplies by three D x I matrices, so the expert matmuls
+    # perform T*k*3*D*I + T*S*3*D*I_s multiply-adds.
+    for S in (0, 1, 2):
+        cfg, W, x, res, ids = small_random_case(O, S=S, T=10, D=64, E=8, k=3, I=32)
+        O.MAC_COUNTER[0] = 0
+        O.moe_layer(cfg, W, x, res, ids)
+        assert O.MAC_COUNTER[0] == 10 * 3 * 3 * 64 * 32 + 10 * S * 3 * 64 * 32
+
+
+ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

@@ -1,0 +1,74 @@
+"""Plant plausible mistakes in copies of the oracle and require a pin to catch each.
+
+The mistakes are planted on the CPU, in a private copy of the oracle's source;
+the real oracle is never modified.
+"""
+import os
+import types
+
+import pytest
+
+import oracle_pins as P
+
+SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                   "oracle", "moe_oracle.py")
+
+MUTATIONS = {
+    "eps_outside_sqrt": ("x / np.sqrt(ms + eps)", "x / (np.sqrt(ms) + eps)"),
+    "gain_dropped": ("return np.asarray(g, dtype=np.float64) * (x / np.sqrt(ms + eps))",
+                     "return (x / np.sqrt(ms + eps))"),
+    "double_rounding_via_fp32": ("a = np.asarray(a, dtype=np.float64)\n    _, e",
+                                 "a = np.asarray(a, dtype=np.float64).astype(np.float32).astype(np.float64)\n    _, e"),
+    "topk_ascending": ("neg = np.where(np.isnan(keys), np.inf, -keys)",
+                       "neg = np.where(np.isnan(keys), np.inf, keys)"),
+    "topk_ties_to_higher_index": ('return np.argsort(neg, axis=-1, kind="stable")[..., :k].astype(np.int64)',
+                                  'return (neg.shape[-1] - 1 - np.argsort(neg[..., ::-1], axis=-1, kind="stable"))[..., :k].astype(np.int64)'),
+    "softmax_no_renorm": ("    if renormalize:\n        w = w / np.sum(w, axis=-1, keepdims=True)\n    return idx, w * routed_scale, p",
+                          "    return idx, w * routed_scale, p"),
+    "sigmoid_weights_use_bias": ("w = np.take_along_axis(s, idx, axis=-1)",
+                                 "w = np.take_along_axis(keys, idx, axis=-1)"),
+    "hash_without_multiply": ("h = (ids * np.uint64(mult)) & np.uint64(0xFFFFFFFF)",
+                              "h = ids & np.uint64(0xFFFFFFFF)"),
+    "gate_up_swapped": ("swiglu(x @ Wg.T, x @ Wu.T,", "swiglu(x @ Wu.T, x @ Wg.T,"),
+    "down_not_transposed": ("return h, h @ Wd.T", "return h, h @ Wd"),
+    "silu_sign": ("return g * sigmoid(g) * u", "return g * sigmoid(-g) * u"),
+    "gate_clamped_both_sides": ("g = np.minimum(np.asarray(g, np.float64), gate_clamp_max)",
+                                "g = np.clip(np.asarray(g, np.float64), -gate_clamp_max, gate_clamp_max)"),
+    "shared_dropped": ("        acc = acc + np.sum(np.asarray(y_shared, np.float64), axis=0)",
+                       "        acc = acc"),
+    "residual_after_norm": ("r = np.asarray(acc, np.float64) + np.asarray(residual, np.float64)\n    return round_bf16(rmsnorm(r, g_out, eps))",
+                            "r = np.asarray(acc, np.float64) + np.asarray(residual, np.float64)\n    return round_bf16(rmsnorm(acc, g_out, eps) + residual)"),
+    "slot_weights_reversed": ('acc = np.einsum("tj,tjd->td", np.asarray(w, np.float64)',
+                              'acc = np.einsum("tj,tjd->td", np.asarray(w, np.float64)[:, ::-1]'),
+    "permute_unstable_desc_token": ('order = np.argsort(flat, kind="stable")',
+                                    'order = (len(flat) - 1 - np.argsort(flat[::-1], kind="stable"))'),
+    "ring_order_used_as_fixed": ("    acc = parts[0].copy()\n    for p in range(1, parts.shape[0]):",
+                                 "    return allreduce_ring_order_f32(partials)\n    acc = parts[0].copy()\n    for p in range(1, parts.shape[0]):"),
+    "fixed_order_reversed": ("    acc = parts[0].copy()\n    for p in range(1, parts.shape[0]):\n        acc = np.add(acc, parts[p], dtype=np.float32)",
+                             "    acc = parts[-1].copy()\n    for p in range(parts.shape[0] - 2, -1, -1):\n        acc = np.add(acc, parts[p], dtype=np.float32)"),
+    "partials_residual_in_fp64": ("r = np.add(s, np.asarray(residual, np.float32), dtype=np.float32)",
+                                  "r = s.astype(np.float64) + np.asarray(residual, np.float64) + 2.0 ** -30"),
+    "histogram_off_by_one": ("return np.bincount(np.asarray(idx).ravel(), minlength=E).astype(np.int64)",
+                             "return np.bincount(np.asarray(idx).ravel() % max(E - 1, 1), minlength=E).astype(np.int64)"),
+}
+
+
+def mutated_module(name):
+    old, new = MUTATIONS[name]
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"mutation {name}: anchor not found once in the oracle"
+    mod = types.ModuleType(f"oracle_mutant_{name}")
+    exec(compile(src.replace(old, new), f"<mutant {name}>", "exec"), mod.__dict__)
+    return mod
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_planted_mistake_is_caught(name):
+    M = mutated_module(name)
+    caught = []
+    for pin in P.ALL_PINS:
+        try:
+            pin(M)
+        except Exception as e:  # AssertionError, or a shape error from a wrong operand
+            caught.append((pin.__name__, type(e).__name__))
+    assert caught, f"no pin caught the planted mistake {name}"
