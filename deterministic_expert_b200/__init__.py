@@ -1,0 +1,214 @@
+"""Batch-invariant MoE layer forward for B200 (sm_100a): Python binding of libmoe.so.
+
+This module only marshals arguments: every step of the layer runs in the CUDA
+kernels of ``libmoe.so`` (built from ``csrc/`` by ``__graft_entry__.build()``).
+There is no fallback: importing the binding without the built library, or
+calling it without a CUDA device, raises.
+
+PyTorch supplies device memory and streams; tensors are passed to the C ABI
+as raw pointers (bf16 tensors as their bit patterns).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe.so")
+HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "moe.h")
+
+MOE_OK, MOE_EINVAL, MOE_ETOOBIG, MOE_EWORKSPACE, MOE_EUNSUPPORTED, MOE_ECUDA, MOE_ETIMEOUT = (
+    0, -1, -2, -3, -4, -5, -6)
+ROUTER_SOFTMAX, ROUTER_SIGMOID_BIAS, ROUTER_HASH = 0, 1, 2
+NUM_STAGES = 10
+STAGE_NAMES = ("rmsnorm_in", "router_gemm", "router_topk", "dispatch_count", "dispatch_scan",
+               "dispatch_scatter", "gather_rows", "gemm_gateup_swiglu", "gemm_down", "combine_norm")
+
+
+class MoEError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {status_string(status)} ({status})")
+        self.status = status
+
+
+class moe_config(ctypes.Structure):
+    _fields_ = [("D", ctypes.c_int), ("E", ctypes.c_int), ("k", ctypes.c_int), ("I", ctypes.c_int),
+                ("n_shared", ctypes.c_int), ("I_shared", ctypes.c_int), ("T_max", ctypes.c_int),
+                ("router", ctypes.c_int), ("renormalize", ctypes.c_int),
+                ("routed_scale", ctypes.c_float), ("gate_clamp_max", ctypes.c_float),
+                ("up_clamp", ctypes.c_float), ("eps", ctypes.c_float), ("hash_mult", ctypes.c_uint32)]
+
+
+class moe_weights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("w_router", "router_bias", "w_gate", "w_up", "w_down",
+                                               "ws_gate", "ws_up", "ws_down", "g_in", "g_out")]
+
+
+class moe_views(ctypes.Structure):
+    _fields_ = [("xn", ctypes.c_void_p), ("logits", ctypes.c_void_p), ("E_pad", ctypes.c_int),
+                ("topk_idx", ctypes.c_void_p), ("topk_w", ctypes.c_void_p), ("counts", ctypes.c_void_p),
+                ("offsets", ctypes.c_void_p), ("src_token", ctypes.c_void_p),
+                ("dest_row", ctypes.c_void_p), ("h_routed", ctypes.c_void_p),
+                ("h_shared", ctypes.c_void_p), ("y_slot", ctypes.c_void_p),
+                ("y_shared", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libmoe.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with __graft_entry__.build()")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i, sz, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_float
+        L.moe_init.argtypes = [ctypes.POINTER(moe_config), ctypes.POINTER(moe_weights), ctypes.POINTER(vp)]
+        L.moe_workspace_size.argtypes = [vp, i]
+        L.moe_workspace_size.restype = sz
+        L.moe_invariance_workspace_size.argtypes = [vp, i]
+        L.moe_invariance_workspace_size.restype = sz
+        L.moe_layer_forward.argtypes = [vp, i, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.moe_get_device_error.argtypes = [vp, vp, vp]
+        L.moe_reduce_partials.argtypes = [i, ctypes.POINTER(vp), vp, vp, vp, vp, i, i, f, vp]
+        L.moe_check_invariance.argtypes = [vp, i, vp, vp, vp, i, vp, i, vp, sz,
+                                           ctypes.POINTER(ctypes.c_ulonglong), vp]
+        L.moe_workspace_views.argtypes = [vp, i, vp, ctypes.POINTER(moe_views)]
+        L.moe_profile_enable.argtypes = [vp, i]
+        L.moe_profile_read.argtypes = [vp, ctypes.POINTER(f), ctypes.POINTER(i)]
+        L.moe_forward_launch_count.argtypes = [vp, i]
+        L.moe_selftest_wait_timeout.argtypes = [i, vp]
+        L.moe_destroy.argtypes = [vp]
+        L.moe_status_string.argtypes = [i]
+        L.moe_status_string.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().moe_status_string(status).decode()
+
+
+def _check(status: int, what: str) -> None:
+    if status != MOE_OK:
+        raise MoEError(status, what)
+
+
+def _ptr(t) -> int | None:
+    return None if t is None else int(t.data_ptr())
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        import torch
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+
+
+@dataclass
+class LayerConfig:
+    D: int
+    E: int
+    k: int
+    I: int
+    n_shared: int = 0
+    I_shared: int = 0
+    T_max: int = 8192
+    router: int = ROUTER_SOFTMAX
+    renormalize: int = 0
+    routed_scale: float = 1.0
+    gate_clamp_max: float = float("inf")
+    up_clamp: float = float("inf")
+    eps: float = 1e-6
+    hash_mult: int = 2654435761
+
+    def to_c(self) -> moe_config:
+        return moe_config(self.D, self.E, self.k, self.I, self.n_shared,
+                          self.I_shared if self.n_shared else self.I, self.T_max, self.router,
+                          self.renormalize, self.routed_scale, self.gate_clamp_max, self.up_clamp,
+                          self.eps, self.hash_mult)
+
+
+class MoELayer:
+    """A handle over caller-owned device weights (torch tensors, bf16 unless
+    noted).  ``weights`` maps the moe_weights field names to tensors; the
+    tensors must outlive the layer."""
+
+    def __init__(self, cfg: LayerConfig, weights: dict):
+        self.cfg = cfg
+        self._keep = dict(weights)
+        w = moe_weights(*[_ptr(weights.get(n)) for n, _ in moe_weights._fields_])
+        h = ctypes.c_void_p()
+        _check(lib().moe_init(ctypes.byref(cfg.to_c()), ctypes.byref(w), ctypes.byref(h)), "moe_init")
+        self.handle = h
+
+    def close(self):
+        if getattr(self, "handle", None):
+            lib().moe_destroy(self.handle)
+            self.handle = None
+
+    __del__ = close
+
+    def workspace_size(self, T: int) -> int:
+        return int(lib().moe_workspace_size(self.handle, T))
+
+    def invariance_workspace_size(self, T: int) -> int:
+        return int(lib().moe_invariance_workspace_size(self.handle, T))
+
+    def forward(self, x, residual, out_norm, out_residual, workspace, token_ids=None,
+                out_topk_idx=None, out_topk_w=None, out_counts=None, stream=None) -> None:
+        T = int(x.shape[0])
+        _check(lib().moe_layer_forward(self.handle, T, _ptr(x), _ptr(residual), _ptr(token_ids),
+                                       _ptr(out_norm), _ptr(out_residual), _ptr(out_topk_idx),
+                                       _ptr(out_topk_w), _ptr(out_counts), _ptr(workspace),
+                                       workspace.numel() * workspace.element_size() if workspace is not None else 0,
+                                       _stream(stream)),
+               "moe_layer_forward")
+
+    def device_error(self, workspace, stream=None) -> int:
+        return int(lib().moe_get_device_error(self.handle, _ptr(workspace), _stream(stream)))
+
+    def check_invariance(self, x, residual, workspace, token_ids=None, n_splits=0, perm=None,
+                         repeats=0, stream=None) -> int:
+        out = ctypes.c_ulonglong(0)
+        _check(lib().moe_check_invariance(self.handle, int(x.shape[0]), _ptr(x), _ptr(residual),
+                                          _ptr(token_ids), n_splits, _ptr(perm), repeats,
+                                          _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                          ctypes.byref(out), _stream(stream)),
+               "moe_check_invariance")
+        return int(out.value)
+
+    def views(self, T: int, workspace) -> moe_views:
+        v = moe_views()
+        _check(lib().moe_workspace_views(self.handle, T, _ptr(workspace), ctypes.byref(v)),
+               "moe_workspace_views")
+        return v
+
+    def profile_enable(self, on: bool = True) -> None:
+        _check(lib().moe_profile_enable(self.handle, int(on)), "moe_profile_enable")
+
+    def profile_read(self):
+        ms = (ctypes.c_float * NUM_STAGES)()
+        n = (ctypes.c_int * NUM_STAGES)()
+        _check(lib().moe_profile_read(self.handle, ms, n), "moe_profile_read")
+        return list(ms), list(n)
+
+    def launch_count(self, T: int) -> int:
+        return int(lib().moe_forward_launch_count(self.handle, T))
+
+
+def reduce_partials(partials, residual, g, out_norm, out_residual, eps: float = 1e-6,
+                    stream=None) -> None:
+    """Fixed r0..r7 order partial reduction + residual + RMSNorm (P <= 8 bf16 tensors)."""
+    P = len(partials)
+    arr = (ctypes.c_void_p * P)(*[_ptr(p) for p in partials])
+    T, D = int(residual.shape[0]), int(residual.shape[1])
+    _check(lib().moe_reduce_partials(P, arr, _ptr(residual), _ptr(g), _ptr(out_norm),
+                                     _ptr(out_residual), T, D, eps, _stream(stream)),
+           "moe_reduce_partials")
+
+
+def selftest_wait_timeout(limit_us: int, stream=None) -> int:
+    return int(lib().moe_selftest_wait_timeout(limit_us, _stream(stream)))

@@ -1,0 +1,597 @@
+// The C ABI of libmoe.so (declared in include/moe.h): argument checks, the
+// workspace layout, TMA descriptor encoding and the launch sequence of one
+// layer forward.  Everything here runs on the host; every step of the layer
+// runs in the kernels of the other translation units.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "common.cuh"
+#include "moe_internal.h"
+
+using namespace moe;
+
+struct moe_handle {
+  moe_config cfg;
+  moe_weights w;
+  int S = 0, G = 0, E_pad = 0, bn_gu = 0, bn_dn = 0, num_sms = 0, device = 0;
+  uint16_t* w_router_pad = nullptr;  // [E_pad, D], rows >= E zero
+  CUtensorMap map_router, map_wg, map_wu, map_wd, map_wsg, map_wsu, map_wsd;
+  unsigned long long timeout_ns = 2000ull * 1000 * 1000;
+  // Per-stage timing (moe_profile_*).
+  bool prof_on = false;
+  int prof_fwd = 0;
+  std::vector<cudaEvent_t> ev;  // [kProfFwd][MOE_NUM_STAGES][2]
+  int prof_launches[MOE_NUM_STAGES] = {0};
+};
+
+namespace {
+
+constexpr int kProfFwd = 256;
+
+size_t align256(size_t b) { return (b + 255) & ~static_cast<size_t>(255); }
+
+struct Layout {
+  size_t err, xn, logits, tidx, tw, bcount, bbase, counts, offsets, tiles_gu, tiles_dn, dest, src,
+      xp, h, hs, y, ys, total;
+};
+
+Layout layout(const moe_handle* h, int T) {
+  const moe_config& c = h->cfg;
+  const size_t Tz = static_cast<size_t>(T), nb = (Tz + kDispatchRows - 1) / kDispatchRows;
+  Layout L;
+  size_t off = 0;
+  auto take = [&](size_t bytes) { const size_t o = off; off += align256(bytes); return o; };
+  L.err = take(256);
+  L.xn = take(Tz * c.D * 2);
+  L.logits = take(c.router == MOE_ROUTER_HASH ? 0 : Tz * h->E_pad * 4);
+  L.tidx = take(Tz * c.k * 4);
+  L.tw = take(Tz * c.k * 4);
+  L.bcount = take(nb * c.E * 4);
+  L.bbase = take(nb * c.E * 4);
+  L.counts = take(static_cast<size_t>(c.E) * 4);
+  L.offsets = take(static_cast<size_t>(c.E + 1) * 4);
+  L.tiles_gu = take(static_cast<size_t>(h->G + 1) * 4);
+  L.tiles_dn = take(static_cast<size_t>(h->G + 1) * 4);
+  L.dest = take(Tz * c.k * 4);
+  L.src = take(Tz * c.k * 4);
+  L.xp = take(Tz * c.k * c.D * 2);
+  L.h = take(Tz * c.k * c.I * 2);
+  L.hs = take(static_cast<size_t>(h->S) * Tz * c.I_shared * 2);
+  L.y = take(Tz * c.k * c.D * 4);
+  L.ys = take(static_cast<size_t>(h->S) * Tz * c.D * 4);
+  L.total = off;
+  return L;
+}
+
+struct InvLayout {
+  size_t ref_n, ref_r, tst_n, tst_r, xp, rp, ip, cnt, errs, total;
+};
+constexpr int kMaxInvRuns = 64;
+
+InvLayout inv_layout(const moe_handle* h, int T, size_t base) {
+  const size_t rowb = static_cast<size_t>(T) * h->cfg.D * 2;
+  InvLayout L;
+  size_t off = base;
+  auto take = [&](size_t bytes) { const size_t o = off; off += align256(bytes); return o; };
+  L.ref_n = take(rowb); L.ref_r = take(rowb); L.tst_n = take(rowb); L.tst_r = take(rowb);
+  L.xp = take(rowb); L.rp = take(rowb); L.ip = take(static_cast<size_t>(T) * 4);
+  L.cnt = take(8); L.errs = take(kMaxInvRuns * 4);
+  L.total = off;
+  return L;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2D bf16 tensor map over a row-major [rows, inner] matrix; box = 64 columns
+// (128 bytes, the 128-byte swizzle span) x box_rows rows.  Rows past the end
+// read as zeros.  An empty matrix leaves the map zeroed (never loaded).
+bool make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t rows, uint32_t box_rows) {
+  std::memset(m, 0, sizeof(*m));
+  if (rows == 0 || ptr == nullptr) return true;
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {inner * 2};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK), box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int validate_config(const moe_config* c, const moe_weights* w) {
+  if (!c || !w) return MOE_EINVAL;
+  if (c->router < 0 || c->router > 2 || c->D <= 0 || c->E <= 0 || c->k <= 0 || c->I <= 0 ||
+      c->n_shared < 0 || c->T_max <= 0 || !(c->eps >= 0.f) || !(c->routed_scale == c->routed_scale) ||
+      !(c->gate_clamp_max == c->gate_clamp_max) || !(c->up_clamp >= 0.f))
+    return MOE_EINVAL;
+  if (c->n_shared > 0 && c->I_shared <= 0) return MOE_EINVAL;
+  if (c->D % 64 || c->I % 64 || (c->n_shared > 0 && c->I_shared % 64)) return MOE_EUNSUPPORTED;
+  if (c->D > 16384 || c->E > 256 || c->k > c->E || c->k > 16 || c->n_shared > 8 || c->T_max > (1 << 20))
+    return MOE_EUNSUPPORTED;
+  const long long rows = static_cast<long long>(c->T_max) * std::max(c->k, c->n_shared);
+  if (rows * std::max(c->D, std::max(c->I, c->I_shared)) >= (1ll << 31)) return MOE_EUNSUPPORTED;
+  if (!w->w_gate || !w->w_up || !w->w_down || !w->g_in || !w->g_out) return MOE_EINVAL;
+  if (c->router != MOE_ROUTER_HASH && !w->w_router) return MOE_EINVAL;
+  if (c->n_shared > 0 && (!w->ws_gate || !w->ws_up || !w->ws_down)) return MOE_EINVAL;
+  const void* ptrs[] = {w->w_router, w->w_gate, w->w_up, w->w_down, w->ws_gate, w->ws_up,
+                        w->ws_down, w->g_in, w->g_out, w->router_bias};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return MOE_EINVAL;
+  return MOE_OK;
+}
+
+int gemm_grid(const moe_handle* h, int tiles_bound) {
+  return std::max(1, std::min(h->num_sms, tiles_bound));
+}
+
+struct Prof {
+  moe_handle* h;
+  cudaStream_t s;
+  int f;
+  void begin(int stage) {
+    if (f >= 0) cudaEventRecord(h->ev[(static_cast<size_t>(f) * MOE_NUM_STAGES + stage) * 2], s);
+  }
+  void end(int stage) {
+    if (f >= 0) {
+      cudaEventRecord(h->ev[(static_cast<size_t>(f) * MOE_NUM_STAGES + stage) * 2 + 1], s);
+      h->prof_launches[stage] += 1;
+    }
+  }
+};
+
+#define MOE_TRY(expr)                            \
+  do {                                           \
+    if ((expr) != cudaSuccess) return MOE_ECUDA; \
+  } while (0)
+
+// Upper bound on the tiles of the routed + shared expert GEMMs for T rows:
+// sum_e ceil(c_e / 128) <= T*k/128 + (number of non-empty experts).
+int expert_tile_bound(const moe_handle* h, int T, int nt_routed, int nt_shared) {
+  const moe_config& c = h->cfg;
+  const long long tk = static_cast<long long>(T) * c.k;
+  const long long mt = (tk + kBM - 1) / kBM + std::min<long long>(c.E, tk);
+  const long long b = mt * nt_routed + static_cast<long long>(h->S) * ((T + kBM - 1) / kBM) * nt_shared;
+  return static_cast<int>(std::min<long long>(b, 1 << 30));
+}
+
+int forward_impl(moe_handle* h, int T, const uint16_t* x, const uint16_t* residual,
+                 const int32_t* token_ids, uint16_t* out_norm, uint16_t* out_residual,
+                 int32_t* out_idx, float* out_w, int32_t* out_counts, uint8_t* ws,
+                 cudaStream_t s) {
+  const moe_config& c = h->cfg;
+  const Layout L = layout(h, T);
+  int* err = reinterpret_cast<int*>(ws + L.err);
+  uint16_t* xn = reinterpret_cast<uint16_t*>(ws + L.xn);
+  float* logits = reinterpret_cast<float*>(ws + L.logits);
+  int32_t* tidx = reinterpret_cast<int32_t*>(ws + L.tidx);
+  float* tw = reinterpret_cast<float*>(ws + L.tw);
+  int32_t* offsets = reinterpret_cast<int32_t*>(ws + L.offsets);
+  int32_t* tiles_gu = reinterpret_cast<int32_t*>(ws + L.tiles_gu);
+  int32_t* tiles_dn = reinterpret_cast<int32_t*>(ws + L.tiles_dn);
+  int32_t* dest = reinterpret_cast<int32_t*>(ws + L.dest);
+  int32_t* src = reinterpret_cast<int32_t*>(ws + L.src);
+  uint16_t* xp = reinterpret_cast<uint16_t*>(ws + L.xp);
+  uint16_t* hb = reinterpret_cast<uint16_t*>(ws + L.h);
+  uint16_t* hsb = reinterpret_cast<uint16_t*>(ws + L.hs);
+  float* y = reinterpret_cast<float*>(ws + L.y);
+  float* ys = reinterpret_cast<float*>(ws + L.ys);
+  const int TK = T * c.k;
+
+  Prof prof{h, s, -1};
+  if (h->prof_on && h->prof_fwd < kProfFwd) prof.f = h->prof_fwd++;
+
+  // 0. input RMSNorm (also clears the device error word)
+  prof.begin(0);
+  MOE_TRY(launch_rmsnorm_rows(x, h->w.g_in, xn, T, c.D, c.eps, err, s));
+  prof.end(0);
+
+  // 1. router logits on the tensor cores
+  if (c.router != MOE_ROUTER_HASH) {
+    GemmArgs g;
+    std::memset(&g, 0, sizeof(g));
+    if (!make_map(&g.mapA[0], xn, c.D, T, kBM)) return MOE_ECUDA;
+    g.mapB[0] = h->map_router;
+    g.T = T;
+    g.n_kind[0] = h->E_pad;
+    g.k_kind[0] = c.D;
+    g.BN = h->E_pad;
+    g.router_tiles = (T + kBM - 1) / kBM;
+    g.out[0] = logits;
+    g.ld_out[0] = h->E_pad;
+    g.err = err;
+    g.timeout_ns = h->timeout_ns;
+    prof.begin(1);
+    MOE_TRY(launch_grouped_gemm(kRouter, g, gemm_grid(h, g.router_tiles), s));
+    prof.end(1);
+  }
+
+  // 2. scores, top-k, weights
+  RouterArgs ra;
+  ra.logits = logits; ra.E_pad = h->E_pad; ra.bias = h->w.router_bias; ra.token_ids = token_ids;
+  ra.router = c.router; ra.E = c.E; ra.k = c.k; ra.renormalize = c.renormalize;
+  ra.routed_scale = c.routed_scale; ra.hash_mult = c.hash_mult; ra.idx = tidx; ra.w = tw; ra.T = T;
+  prof.begin(2);
+  MOE_TRY(launch_router_topk(ra, s));
+  prof.end(2);
+  if (out_idx) MOE_TRY(cudaMemcpyAsync(out_idx, tidx, static_cast<size_t>(TK) * 4, cudaMemcpyDeviceToDevice, s));
+  if (out_w) MOE_TRY(cudaMemcpyAsync(out_w, tw, static_cast<size_t>(TK) * 4, cudaMemcpyDeviceToDevice, s));
+
+  // 3-5. histogram, scan (+ tile lists), stable scatter
+  DispatchArgs da;
+  da.idx = tidx; da.T = T; da.k = c.k; da.E = c.E; da.S = h->S;
+  da.block_counts = reinterpret_cast<int32_t*>(ws + L.bcount);
+  da.block_base = reinterpret_cast<int32_t*>(ws + L.bbase);
+  da.counts = reinterpret_cast<int32_t*>(ws + L.counts);
+  da.offsets = offsets; da.user_counts = out_counts; da.tiles_gu = tiles_gu; da.tiles_dn = tiles_dn;
+  da.gu_ntiles_routed = c.I / h->bn_gu;
+  da.gu_ntiles_shared = h->S > 0 ? c.I_shared / h->bn_gu : 0;
+  da.dn_ntiles = c.D / h->bn_dn;
+  da.dest_row = dest; da.src_token = src;
+  prof.begin(3);
+  MOE_TRY(launch_dispatch_count(da, s));
+  prof.end(3);
+  prof.begin(4);
+  MOE_TRY(launch_dispatch_scan(da, s));
+  prof.end(4);
+  prof.begin(5);
+  MOE_TRY(launch_dispatch_scatter(da, s));
+  prof.end(5);
+
+  // 6. grouped A rows of the routed experts
+  prof.begin(6);
+  MOE_TRY(launch_gather_rows(xn, src, TK, c.D, xp, s));
+  prof.end(6);
+
+  // 7. gate/up + SwiGLU(+clamp): routed groups read xp, shared groups read xn
+  {
+    GemmArgs g;
+    std::memset(&g, 0, sizeof(g));
+    if (!make_map(&g.mapA[0], xp, c.D, TK, kBM)) return MOE_ECUDA;
+    if (h->S > 0 && !make_map(&g.mapA[1], xn, c.D, T, kBM)) return MOE_ECUDA;
+    g.mapB[0] = h->map_wg; g.mapB[1] = h->map_wu; g.mapB[2] = h->map_wsg; g.mapB[3] = h->map_wsu;
+    g.offsets = offsets; g.tile_start = tiles_gu; g.G = h->G; g.E = c.E; g.T = T;
+    g.n_kind[0] = c.I; g.n_kind[1] = c.I_shared;
+    g.k_kind[0] = c.D; g.k_kind[1] = c.D;
+    g.BN = h->bn_gu;
+    g.shared_a_stride = 0;
+    g.out[0] = hb; g.ld_out[0] = c.I;
+    g.out[1] = hsb; g.ld_out[1] = c.I_shared;
+    g.shared_out_stride = T;
+    g.gate_clamp = c.gate_clamp_max; g.up_clamp = c.up_clamp;
+    g.err = err; g.timeout_ns = h->timeout_ns;
+    const int bound = expert_tile_bound(h, T, da.gu_ntiles_routed, da.gu_ntiles_shared);
+    prof.begin(7);
+    MOE_TRY(launch_grouped_gemm(kGateUp, g, gemm_grid(h, bound), s));
+    prof.end(7);
+  }
+
+  // 8. down: routed rows scatter to their (token, slot) row of y
+  {
+    GemmArgs g;
+    std::memset(&g, 0, sizeof(g));
+    if (!make_map(&g.mapA[0], hb, c.I, TK, kBM)) return MOE_ECUDA;
+    if (h->S > 0 && !make_map(&g.mapA[1], hsb, c.I_shared, static_cast<uint64_t>(h->S) * T, kBM))
+      return MOE_ECUDA;
+    g.mapB[0] = h->map_wd; g.mapB[2] = h->map_wsd;
+    g.offsets = offsets; g.tile_start = tiles_dn; g.G = h->G; g.E = c.E; g.T = T;
+    g.n_kind[0] = c.D; g.n_kind[1] = c.D;
+    g.k_kind[0] = c.I; g.k_kind[1] = c.I_shared;
+    g.BN = h->bn_dn;
+    g.shared_a_stride = T;
+    g.out[0] = y; g.ld_out[0] = c.D;
+    g.out[1] = ys; g.ld_out[1] = c.D;
+    g.shared_out_stride = T;
+    g.dest_row = dest;
+    g.err = err; g.timeout_ns = h->timeout_ns;
+    const int bound = expert_tile_bound(h, T, da.dn_ntiles, da.dn_ntiles);
+    prof.begin(8);
+    MOE_TRY(launch_grouped_gemm(kDown, g, gemm_grid(h, bound), s));
+    prof.end(8);
+  }
+
+  // 9. fixed-order combine + residual + RMSNorm
+  prof.begin(9);
+  MOE_TRY(launch_combine_norm(y, tw, ys, c.k, h->S, residual, h->w.g_out, out_norm, out_residual, T,
+                              c.D, c.eps, s));
+  prof.end(9);
+  return MOE_OK;
+}
+
+int check_forward_args(const moe_handle* h, int T, const void* x, const void* residual,
+                       const void* token_ids, const void* out_norm, const void* out_residual,
+                       const void* workspace, size_t ws_bytes, size_t need) {
+  if (!h || T < 0) return MOE_EINVAL;
+  if (T > h->cfg.T_max) return MOE_ETOOBIG;
+  if (T == 0) return MOE_OK;
+  if (!x || !residual || !out_norm || !out_residual || !workspace) return MOE_EINVAL;
+  if (h->cfg.router == MOE_ROUTER_HASH && !token_ids) return MOE_EINVAL;
+  if (!aligned16(x) || !aligned16(residual) || !aligned16(out_norm) || !aligned16(out_residual))
+    return MOE_EINVAL;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MOE_EINVAL;
+  if (ws_bytes < need) return MOE_EWORKSPACE;
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int moe_init(const moe_config* cfg, const moe_weights* w, moe_handle** out) {
+  if (!out) return MOE_EINVAL;
+  *out = nullptr;
+  const int v = validate_config(cfg, w);
+  if (v != MOE_OK) return v;
+  moe_handle* h = new (std::nothrow) moe_handle();
+  if (!h) return MOE_ECUDA;
+  h->cfg = *cfg;
+  h->w = *w;
+  h->S = cfg->n_shared;
+  if (h->S == 0) h->cfg.I_shared = cfg->I;  // unused; keeps the shapes well defined
+  h->G = cfg->E + h->S;
+  h->E_pad = (cfg->E + 15) / 16 * 16;
+  // One GEMM configuration per layer shape, never per T.
+  h->bn_gu = (cfg->I % 128 == 0 && h->cfg.I_shared % 128 == 0) ? 128 : 64;
+  h->bn_dn = (cfg->D % 256 == 0) ? 256 : (cfg->D % 128 == 0 ? 128 : 64);
+  auto fail = [&](int code) { moe_destroy(h); return code; };
+  if (cudaGetDevice(&h->device) != cudaSuccess) return fail(MOE_ECUDA);
+  if (cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, h->device) != cudaSuccess)
+    return fail(MOE_ECUDA);
+  gemm_prepare();
+  const moe_config& c = h->cfg;
+  if (c.router != MOE_ROUTER_HASH) {
+    const size_t row = static_cast<size_t>(c.D) * 2;
+    if (cudaMalloc(&h->w_router_pad, static_cast<size_t>(h->E_pad) * row) != cudaSuccess) return fail(MOE_ECUDA);
+    if (cudaMemset(h->w_router_pad, 0, static_cast<size_t>(h->E_pad) * row) != cudaSuccess) return fail(MOE_ECUDA);
+    if (cudaMemcpy(h->w_router_pad, w->w_router, static_cast<size_t>(c.E) * row, cudaMemcpyDeviceToDevice) != cudaSuccess)
+      return fail(MOE_ECUDA);
+  }
+  bool ok = make_map(&h->map_router, h->w_router_pad, c.D, h->w_router_pad ? h->E_pad : 0, h->E_pad) &&
+            make_map(&h->map_wg, w->w_gate, c.D, static_cast<uint64_t>(c.E) * c.I, h->bn_gu) &&
+            make_map(&h->map_wu, w->w_up, c.D, static_cast<uint64_t>(c.E) * c.I, h->bn_gu) &&
+            make_map(&h->map_wd, w->w_down, c.I, static_cast<uint64_t>(c.E) * c.D, h->bn_dn) &&
+            make_map(&h->map_wsg, w->ws_gate, c.D, static_cast<uint64_t>(h->S) * c.I_shared, h->bn_gu) &&
+            make_map(&h->map_wsu, w->ws_up, c.D, static_cast<uint64_t>(h->S) * c.I_shared, h->bn_gu) &&
+            make_map(&h->map_wsd, w->ws_down, c.I_shared, static_cast<uint64_t>(h->S) * c.D, h->bn_dn);
+  if (!ok) return fail(MOE_ECUDA);
+  *out = h;
+  return MOE_OK;
+}
+
+size_t moe_workspace_size(const moe_handle* h, int T) {
+  if (!h || T <= 0 || T > h->cfg.T_max) return 0;
+  return layout(h, T).total;
+}
+
+int moe_layer_forward(moe_handle* h, int T, const moe_bf16* x, const moe_bf16* residual,
+                      const int32_t* token_ids, moe_bf16* out_norm, moe_bf16* out_residual,
+                      int32_t* out_topk_idx, float* out_topk_w, int32_t* out_counts,
+                      void* workspace, size_t ws_bytes, void* stream) {
+  const size_t need = (h && T > 0 && T <= h->cfg.T_max) ? layout(h, T).total : 0;
+  const int v = check_forward_args(h, T, x, residual, token_ids, out_norm, out_residual, workspace,
+                                   ws_bytes, need);
+  if (v != MOE_OK || T == 0) return v;
+  return forward_impl(h, T, x, residual, token_ids, out_norm, out_residual, out_topk_idx, out_topk_w,
+                      out_counts, static_cast<uint8_t*>(workspace), static_cast<cudaStream_t>(stream));
+}
+
+int moe_get_device_error(moe_handle* h, void* workspace, void* stream) {
+  if (!h || !workspace) return MOE_EINVAL;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int e = 0;
+  if (cudaMemcpyAsync(&e, workspace, 4, cudaMemcpyDeviceToHost, s) != cudaSuccess) return MOE_ECUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ECUDA;
+  if (cudaMemsetAsync(workspace, 0, 4, s) != cudaSuccess) return MOE_ECUDA;
+  return e == kDevOk ? MOE_OK : MOE_ETIMEOUT;
+}
+
+int moe_reduce_partials(int P, const moe_bf16* const* partials, const moe_bf16* residual,
+                        const moe_bf16* g, moe_bf16* out_norm, moe_bf16* out_residual, int T, int D,
+                        float eps, void* stream) {
+  if (P < 1 || P > 8 || !partials || T < 0 || D <= 0 || !(eps >= 0.f)) return MOE_EINVAL;
+  if (D % 64 || D > 16384) return MOE_EUNSUPPORTED;
+  if (T == 0) return MOE_OK;
+  if (!residual || !g || !out_norm || !out_residual) return MOE_EINVAL;
+  PartialPtrs pp;
+  for (int p = 0; p < 8; ++p) pp.p[p] = nullptr;
+  for (int p = 0; p < P; ++p) {
+    if (!partials[p] || !aligned16(partials[p])) return MOE_EINVAL;
+    pp.p[p] = partials[p];
+  }
+  if (!aligned16(residual) || !aligned16(out_norm) || !aligned16(out_residual)) return MOE_EINVAL;
+  return launch_reduce_partials(pp, P, residual, g, out_norm, out_residual, T, D, eps,
+                                static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? MOE_OK
+             : MOE_ECUDA;
+}
+
+size_t moe_invariance_workspace_size(const moe_handle* h, int T) {
+  if (!h || T <= 0 || T > h->cfg.T_max) return 0;
+  const size_t base = layout(h, T).total;
+  return inv_layout(h, T, base).total;
+}
+
+int moe_check_invariance(moe_handle* h, int T, const moe_bf16* x, const moe_bf16* residual,
+                         const int32_t* token_ids, int n_splits, const int32_t* perm, int repeats,
+                         void* workspace, size_t ws_bytes, unsigned long long* out_mismatched_elems,
+                         void* stream) {
+  if (!h || !out_mismatched_elems || T <= 0 || n_splits < 0 || repeats < 0) return MOE_EINVAL;
+  if (T > h->cfg.T_max) return MOE_ETOOBIG;
+  if (n_splits > T || 2 + n_splits + repeats > kMaxInvRuns) return MOE_EINVAL;
+  if (!x || !residual || !workspace) return MOE_EINVAL;
+  if (h->cfg.router == MOE_ROUTER_HASH && !token_ids) return MOE_EINVAL;
+  const size_t base = layout(h, T).total;
+  const InvLayout V = inv_layout(h, T, base);
+  if (ws_bytes < V.total) return MOE_EWORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MOE_EINVAL;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int D = h->cfg.D;
+  auto P16 = [&](size_t off) { return reinterpret_cast<uint16_t*>(ws + off); };
+  unsigned long long* cnt = reinterpret_cast<unsigned long long*>(ws + V.cnt);
+  int* errs = reinterpret_cast<int*>(ws + V.errs);
+  int nrun = 0;
+  if (cudaMemsetAsync(cnt, 0, 8, s) != cudaSuccess) return MOE_ECUDA;
+  if (cudaMemsetAsync(errs, 0, kMaxInvRuns * 4, s) != cudaSuccess) return MOE_ECUDA;
+  auto run = [&](int n, const uint16_t* xx, const uint16_t* rr, const int32_t* ii, uint16_t* on,
+                 uint16_t* orr) -> int {
+    const int r = forward_impl(h, n, xx, rr, ii, on, orr, nullptr, nullptr, nullptr, ws, s);
+    if (r != MOE_OK) return r;
+    if (cudaMemcpyAsync(errs + nrun++, ws, 4, cudaMemcpyDeviceToDevice, s) != cudaSuccess) return MOE_ECUDA;
+    return MOE_OK;
+  };
+  auto compare = [&](const int32_t* rowmap) -> int {
+    if (launch_bitcompare(P16(V.tst_n), P16(V.ref_n), rowmap, T, D, cnt, s) != cudaSuccess) return MOE_ECUDA;
+    if (launch_bitcompare(P16(V.tst_r), P16(V.ref_r), rowmap, T, D, cnt, s) != cudaSuccess) return MOE_ECUDA;
+    return MOE_OK;
+  };
+  int r = run(T, x, residual, token_ids, P16(V.ref_n), P16(V.ref_r));
+  if (r != MOE_OK) return r;
+  if (n_splits > 0) {
+    for (int i = 0; i < n_splits; ++i) {
+      const int r0 = static_cast<int>(static_cast<long long>(T) * i / n_splits);
+      const int r1 = static_cast<int>(static_cast<long long>(T) * (i + 1) / n_splits);
+      if (r1 == r0) continue;
+      const size_t o = static_cast<size_t>(r0) * D;
+      r = run(r1 - r0, x + o, residual + o, token_ids ? token_ids + r0 : nullptr, P16(V.tst_n) + o,
+              P16(V.tst_r) + o);
+      if (r != MOE_OK) return r;
+    }
+    if ((r = compare(nullptr)) != MOE_OK) return r;
+  }
+  if (perm) {
+    int32_t* ip = reinterpret_cast<int32_t*>(ws + V.ip);
+    if (launch_permute_inputs(x, residual, token_ids, perm, T, D, P16(V.xp), P16(V.rp),
+                              token_ids ? ip : nullptr, s) != cudaSuccess)
+      return MOE_ECUDA;
+    r = run(T, P16(V.xp), P16(V.rp), token_ids ? ip : nullptr, P16(V.tst_n), P16(V.tst_r));
+    if (r != MOE_OK) return r;
+    if ((r = compare(perm)) != MOE_OK) return r;
+  }
+  for (int i = 0; i < repeats; ++i) {
+    r = run(T, x, residual, token_ids, P16(V.tst_n), P16(V.tst_r));
+    if (r != MOE_OK) return r;
+    if ((r = compare(nullptr)) != MOE_OK) return r;
+  }
+  int herr[kMaxInvRuns];
+  if (cudaMemcpyAsync(out_mismatched_elems, cnt, 8, cudaMemcpyDeviceToHost, s) != cudaSuccess) return MOE_ECUDA;
+  if (cudaMemcpyAsync(herr, errs, kMaxInvRuns * 4, cudaMemcpyDeviceToHost, s) != cudaSuccess) return MOE_ECUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ECUDA;
+  for (int i = 0; i < nrun; ++i)
+    if (herr[i] != kDevOk) return MOE_ETIMEOUT;
+  return MOE_OK;
+}
+
+int moe_workspace_views(const moe_handle* h, int T, void* workspace, moe_views* out) {
+  if (!h || !workspace || !out || T <= 0 || T > h->cfg.T_max) return MOE_EINVAL;
+  const Layout L = layout(h, T);
+  const uint8_t* ws = static_cast<const uint8_t*>(workspace);
+  out->xn = reinterpret_cast<const moe_bf16*>(ws + L.xn);
+  out->logits = h->cfg.router == MOE_ROUTER_HASH ? nullptr : reinterpret_cast<const float*>(ws + L.logits);
+  out->E_pad = h->E_pad;
+  out->topk_idx = reinterpret_cast<const int32_t*>(ws + L.tidx);
+  out->topk_w = reinterpret_cast<const float*>(ws + L.tw);
+  out->counts = reinterpret_cast<const int32_t*>(ws + L.counts);
+  out->offsets = reinterpret_cast<const int32_t*>(ws + L.offsets);
+  out->src_token = reinterpret_cast<const int32_t*>(ws + L.src);
+  out->dest_row = reinterpret_cast<const int32_t*>(ws + L.dest);
+  out->h_routed = reinterpret_cast<const moe_bf16*>(ws + L.h);
+  out->h_shared = reinterpret_cast<const moe_bf16*>(ws + L.hs);
+  out->y_slot = reinterpret_cast<const float*>(ws + L.y);
+  out->y_shared = reinterpret_cast<const float*>(ws + L.ys);
+  return MOE_OK;
+}
+
+int moe_profile_enable(moe_handle* h, int on) {
+  if (!h) return MOE_EINVAL;
+  if (on && h->ev.empty()) {
+    h->ev.resize(static_cast<size_t>(kProfFwd) * MOE_NUM_STAGES * 2);
+    for (auto& e : h->ev)
+      if (cudaEventCreate(&e) != cudaSuccess) return MOE_ECUDA;
+  }
+  h->prof_on = on != 0;
+  h->prof_fwd = 0;
+  for (int i = 0; i < MOE_NUM_STAGES; ++i) h->prof_launches[i] = 0;
+  return MOE_OK;
+}
+
+int moe_profile_read(moe_handle* h, float* ms, int* launches) {
+  if (!h || !ms || !launches) return MOE_EINVAL;
+  for (int i = 0; i < MOE_NUM_STAGES; ++i) { ms[i] = 0.f; launches[i] = h->prof_launches[i]; }
+  for (int f = 0; f < h->prof_fwd; ++f) {
+    for (int st = 0; st < MOE_NUM_STAGES; ++st) {
+      cudaEvent_t a = h->ev[(static_cast<size_t>(f) * MOE_NUM_STAGES + st) * 2];
+      cudaEvent_t b = h->ev[(static_cast<size_t>(f) * MOE_NUM_STAGES + st) * 2 + 1];
+      if (cudaEventQuery(b) == cudaErrorNotReady && cudaEventSynchronize(b) != cudaSuccess) return MOE_ECUDA;
+      float t = 0.f;
+      if (cudaEventElapsedTime(&t, a, b) == cudaSuccess) ms[st] += t;
+      else cudaGetLastError();  // stage not recorded in this forward (e.g. no router GEMM)
+    }
+  }
+  h->prof_fwd = 0;
+  for (int i = 0; i < MOE_NUM_STAGES; ++i) h->prof_launches[i] = 0;
+  return MOE_OK;
+}
+
+int moe_forward_launch_count(const moe_handle* h, int T) {
+  if (!h || T < 0) return -1;
+  if (T == 0) return 0;
+  return h->cfg.router == MOE_ROUTER_HASH ? MOE_NUM_STAGES - 1 : MOE_NUM_STAGES;
+}
+
+int moe_selftest_wait_timeout(int limit_us, void* stream) {
+  if (limit_us < 1 || limit_us > 1000000) return MOE_EINVAL;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int* buf = nullptr;
+  if (cudaMalloc(&buf, 8) != cudaSuccess) return MOE_ECUDA;
+  int res = MOE_ECUDA;
+  int host[2] = {0, 0};
+  if (cudaMemsetAsync(buf, 0, 8, s) == cudaSuccess &&
+      launch_wait_selftest(buf, buf + 1, static_cast<unsigned long long>(limit_us) * 1000ull, s) == cudaSuccess &&
+      cudaMemcpyAsync(host, buf, 8, cudaMemcpyDeviceToHost, s) == cudaSuccess &&
+      cudaStreamSynchronize(s) == cudaSuccess)
+    res = host[1] == kDevTimeout ? MOE_ETIMEOUT : MOE_OK;
+  cudaFree(buf);
+  return res;
+}
+
+int moe_destroy(moe_handle* h) {
+  if (!h) return MOE_EINVAL;
+  for (auto& e : h->ev)
+    if (e) cudaEventDestroy(e);
+  if (h->w_router_pad) cudaFree(h->w_router_pad);
+  delete h;
+  return MOE_OK;
+}
+
+const char* moe_status_string(int status) {
+  switch (status) {
+    case MOE_OK: return "ok";
+    case MOE_EINVAL: return "invalid argument";
+    case MOE_ETOOBIG: return "T exceeds T_max";
+    case MOE_EWORKSPACE: return "workspace too small";
+    case MOE_EUNSUPPORTED: return "unsupported shape";
+    case MOE_ECUDA: return "CUDA error";
+    case MOE_ETIMEOUT: return "device wait timed out";
+    default: return "unknown status";
+  }
+}
+
+}  // extern "C"

@@ -1,0 +1,112 @@
+// Internal declarations shared by the library's translation units.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "../../include/moe.h"
+
+namespace moe {
+
+// ------------------------------------------------------------ grouped GEMM
+// One persistent, warp-specialised tcgen05 GEMM serves the router (one group
+// of T rows), gate/up + SwiGLU (E routed groups + S shared groups) and down
+// (same groups).  Tiles are BM = 128 rows x BN columns with the whole K
+// reduced in one TMEM accumulator (no split-K), K walked in 64-wide steps in
+// the same order for every tile.
+constexpr int kBM = 128;
+constexpr int kBK = 64;
+constexpr int kStages = 4;
+constexpr int kGemmThreads = 192;  // warp 0: TMA, warp 1: MMA, warps 2-5: epilogue
+constexpr int kSmemA = kBM * kBK * 2;
+constexpr int kSmemBMax = 256 * kBK * 2;
+constexpr int kGemmSmem = 1024 + kStages * (kSmemA + kSmemBMax) + 256;
+
+enum GemmMode : int { kGateUp = 0, kDown = 1, kRouter = 2 };
+
+struct GemmArgs {
+  CUtensorMap mapA[2];    // A operand per group kind: 0 routed, 1 shared
+  CUtensorMap mapB[4];    // B operands: [kind * 2 + 0] first (gate / down / router),
+                          //             [kind * 2 + 1] second (up; gate/up only)
+  const int* offsets;     // [E + 1] grouped-row offsets of the routed groups
+  const int* tile_start;  // [G + 1] first tile of each group; NULL: one group of T rows
+  int G, E, T;
+  int n_kind[2];          // B rows per expert (N extent) per kind
+  int k_kind[2];          // K extent per kind
+  int BN;
+  int shared_a_stride;    // A rows between consecutive shared experts (0: all read row 0..T)
+  int router_tiles;       // tile count when tile_start is NULL
+  void* out[2];           // output base per kind
+  int ld_out[2];          // output row pitch (elements) per kind
+  int shared_out_stride;  // output rows between consecutive shared experts
+  const int* dest_row;    // down, routed: grouped row -> output row
+  float gate_clamp, up_clamp;
+  int* err;               // device error word
+  unsigned long long timeout_ns;
+};
+
+void gemm_prepare();  // sets the dynamic shared memory limit once per device
+cudaError_t launch_grouped_gemm(int mode, const GemmArgs& a, int grid, cudaStream_t s);
+
+// --------------------------------------------------------------- row ops
+cudaError_t launch_rmsnorm_rows(const uint16_t* x, const uint16_t* g, uint16_t* y, int T, int D,
+                                float eps, int* err_to_clear, cudaStream_t s);
+cudaError_t launch_combine_norm(const float* y_slot, const float* topk_w, const float* y_shared,
+                                int k, int S, const uint16_t* residual, const uint16_t* g,
+                                uint16_t* out_norm, uint16_t* out_residual, int T, int D,
+                                float eps, cudaStream_t s);
+struct PartialPtrs {
+  const uint16_t* p[8];
+};
+cudaError_t launch_reduce_partials(const PartialPtrs& parts, int P, const uint16_t* residual,
+                                   const uint16_t* g, uint16_t* out_norm, uint16_t* out_residual,
+                                   int T, int D, float eps, cudaStream_t s);
+cudaError_t launch_bitcompare(const uint16_t* a, const uint16_t* b, const int32_t* b_row_of_a,
+                              int rows, int D, unsigned long long* count, cudaStream_t s);
+cudaError_t launch_permute_inputs(const uint16_t* x, const uint16_t* res, const int32_t* ids,
+                                  const int32_t* perm, int T, int D, uint16_t* xo, uint16_t* ro,
+                                  int32_t* io, cudaStream_t s);
+
+// ------------------------------------------------------------- routing
+struct RouterArgs {
+  const float* logits;      // [T, E_pad]
+  int E_pad;
+  const float* bias;        // [E] or NULL
+  const int32_t* token_ids; // hash routing
+  int router, E, k, renormalize;
+  float routed_scale;
+  uint32_t hash_mult;
+  int32_t* idx;             // [T, k]
+  float* w;                 // [T, k]
+  int T;
+};
+cudaError_t launch_router_topk(const RouterArgs& a, cudaStream_t s);
+
+// ------------------------------------------------------------ dispatch
+constexpr int kDispatchRows = 256;  // tokens per dispatch block
+struct DispatchArgs {
+  const int32_t* idx;   // [T, k]
+  int T, k, E, S;
+  int32_t* block_counts;  // [nb, E]
+  int32_t* block_base;    // [nb, E]
+  int32_t* counts;        // [E]
+  int32_t* offsets;       // [E + 1]
+  int32_t* user_counts;   // [E] or NULL
+  int32_t* tiles_gu;      // [E + S + 1]
+  int32_t* tiles_dn;      // [E + S + 1]
+  int gu_ntiles_routed, gu_ntiles_shared, dn_ntiles;
+  int32_t* dest_row;      // [T * k]
+  int32_t* src_token;     // [T * k]
+};
+cudaError_t launch_dispatch_count(const DispatchArgs& a, cudaStream_t s);
+cudaError_t launch_dispatch_scan(const DispatchArgs& a, cudaStream_t s);
+cudaError_t launch_dispatch_scatter(const DispatchArgs& a, cudaStream_t s);
+cudaError_t launch_gather_rows(const uint16_t* src, const int32_t* src_row, int rows, int D,
+                               uint16_t* dst, cudaStream_t s);
+
+// ------------------------------------------------------------ self test
+cudaError_t launch_wait_selftest(int* flag, int* err, unsigned long long limit_ns,
+                                 cudaStream_t s);
+
+}  // namespace moe

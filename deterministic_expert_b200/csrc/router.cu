@@ -1,0 +1,140 @@
+// Router scores and top-k, one warp per token.
+//
+//   softmax  keys = l (+ logit bias b), p = exp(l + b - max) / sum over all E
+//            (nxmr.cn "V4" article, §2.2: Linear -> logits -> softmax -> top-k)
+//   sigmoid  s = 1 / (1 + exp(-l)), keys = s + b, the bias only selects
+//            (DeepSeek V4 infra notes §6.3: upper layers use sigmoid + balancing;
+//            linux.do post, "QuantileBalancing": expert e enters when s + b > tau)
+//   hash     e_0 = ((id * mult) mod 2^32) mod E, e_j = (e_0 + j) mod E, w = 1/k
+//            (DeepSeek V4 infra notes §6.3 "Hash Routing", no router parameters)
+//
+// Selection is deterministic: k rounds of a warp arg-max under the total
+// order (key descending, expert index ascending), so equal keys go to the
+// lower index and slot j holds the j-th best expert.  Lane l always owns
+// experts l, l + 32, ... and every sum runs in a fixed order (per lane in
+// index order, then a 5-step butterfly), so a token's routing does not
+// depend on T.  Keys that are NaN rank below every number.  Softmax selects on
+// the logits themselves (the softmax is monotone), weights use the
+// probabilities; renormalised weights divide by their sum in slot order.
+#include <cfloat>
+
+#include "common.cuh"
+#include "moe_internal.h"
+
+namespace moe {
+namespace {
+
+constexpr int kMaxPerLane = 8;  // E <= 256
+
+__device__ __forceinline__ bool better(float k1, int e1, float k2, int e2) {
+  return k1 > k2 || (k1 == k2 && e1 < e2);
+}
+
+__global__ void __launch_bounds__(256) k_router_topk(const RouterArgs a) {
+  const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (t >= a.T) return;
+  const int k = a.k, E = a.E;
+
+  if (a.router == MOE_ROUTER_HASH) {
+    if (lane < k) {
+      const uint32_t h = static_cast<uint32_t>(a.token_ids[t]) * a.hash_mult;  // mod 2^32
+      const int e0 = static_cast<int>(h % static_cast<uint32_t>(E));
+      a.idx[t * k + lane] = (e0 + lane) % E;
+      a.w[t * k + lane] = a.routed_scale / static_cast<float>(k);
+    }
+    return;
+  }
+
+  const float* lr = a.logits + static_cast<size_t>(t) * a.E_pad;
+  float key[kMaxPerLane], val[kMaxPerLane];
+  float zmax = -FLT_MAX;
+#pragma unroll
+  for (int i = 0; i < kMaxPerLane; ++i) {
+    const int e = lane + 32 * i;
+    key[i] = -INFINITY;
+    val[i] = 0.f;
+    if (e < E) {
+      const float l = lr[e];
+      const float b = a.bias ? a.bias[e] : 0.f;
+      if (a.router == MOE_ROUTER_SOFTMAX) {
+        key[i] = l + b;
+        zmax = fmaxf(zmax, key[i]);
+      } else {
+        val[i] = 1.0f / (1.0f + expf(-l));
+        key[i] = val[i] + b;
+      }
+      if (isnan(key[i])) key[i] = -INFINITY;
+    }
+  }
+  float denom = 1.f;
+  if (a.router == MOE_ROUTER_SOFTMAX) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) zmax = fmaxf(zmax, __shfl_xor_sync(0xffffffffu, zmax, o));
+    float s = 0.f;
+#pragma unroll
+    for (int i = 0; i < kMaxPerLane; ++i) {
+      const int e = lane + 32 * i;
+      if (e < E) {
+        val[i] = expf(key[i] - zmax);
+        s += val[i];
+      }
+    }
+    s += __shfl_xor_sync(0xffffffffu, s, 16);
+    s += __shfl_xor_sync(0xffffffffu, s, 8);
+    s += __shfl_xor_sync(0xffffffffu, s, 4);
+    s += __shfl_xor_sync(0xffffffffu, s, 2);
+    s += __shfl_xor_sync(0xffffffffu, s, 1);
+    denom = s;
+  }
+
+  uint32_t taken = 0;
+  float chosen_v[16];
+  int chosen_e[16];
+  for (int j = 0; j < k; ++j) {
+    float bk = -INFINITY;
+    int be = 0x7fffffff, bi = -1;
+#pragma unroll
+    for (int i = 0; i < kMaxPerLane; ++i) {
+      const int e = lane + 32 * i;
+      if (e < E && !(taken & (1u << i)) && better(key[i], e, bk, be)) { bk = key[i]; be = e; bi = i; }
+    }
+    float bv = bi >= 0 ? val[bi] : 0.f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ok = __shfl_xor_sync(0xffffffffu, bk, o);
+      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      if (better(ok, oe, bk, be)) { bk = ok; be = oe; bv = ov; }
+    }
+    if ((be & 31) == lane) taken |= 1u << (be >> 5);
+    chosen_e[j] = be;
+    chosen_v[j] = bv;
+  }
+
+  float norm = denom;
+  if (a.renormalize) {
+    norm = 0.f;
+    for (int j = 0; j < k; ++j) norm += chosen_v[j];
+  }
+  for (int j = lane; j < k; j += 32) {
+    float w = 0.f;
+    int e = 0;
+    for (int q = 0; q < k; ++q)
+      if (q == j) { w = chosen_v[q]; e = chosen_e[q]; }
+    a.idx[t * k + j] = e;
+    const float wn = (a.router == MOE_ROUTER_SOFTMAX || a.renormalize) ? w / norm : w;
+    a.w[t * k + j] = wn * a.routed_scale;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_router_topk(const RouterArgs& a, cudaStream_t s) {
+  if (a.T <= 0) return cudaSuccess;
+  const int warps_per_block = 8;
+  k_router_topk<<<(a.T + warps_per_block - 1) / warps_per_block, 32 * warps_per_block, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

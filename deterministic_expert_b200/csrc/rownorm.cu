@@ -1,0 +1,268 @@
+// Row kernels with a fixed thread layout: one CTA of 256 threads per token
+// row, thread i always owning the 4-element chunks i, i + 256, i + 512, ...
+// of the row.  The sum of squares for RMSNorm goes through the fixed tree of
+// block_sum_fixed (per-thread sum in element order, a 5-step butterfly with
+// masks 16..1, warp partials added left to right), the layout the Fireworks
+// parity post (Chinese translation), Trap 2, says must not change with the
+// launch shape.  Nothing here depends on T.
+//
+//   rmsnorm_rows     xn = bf16(x * rsqrt(mean(x^2) + eps) * g)
+//                    (linux.do post on MoE variants, "RMSNorm before up-projection")
+//   combine_norm     acc = sum_j w_j y_j (slot order) + sum_s y_s; r = acc + residual;
+//                    out_residual = bf16(r); out_norm = bf16(RMSNorm(r) * g)
+//                    (Fireworks post, Trap 3 unfused chain and case-study "standard path":
+//                    fp32 weighted sum, one cast; no atomics)
+//   reduce_partials  r = ((p0 + p1) + ... + p_{P-1}) + residual in fp32, every element,
+//                    then the same norm (Fireworks post, Trap 1: the r0..r7 order)
+#include "common.cuh"
+#include "moe_internal.h"
+
+namespace moe {
+namespace {
+
+constexpr int kMaxChunks = 16;  // D <= 4 * 256 * 16 = 16384
+
+__device__ __forceinline__ float4 ld_bf16x4(const uint16_t* p) {
+  const uint2 v = *reinterpret_cast<const uint2*>(p);
+  return make_float4(bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y));
+}
+
+__device__ __forceinline__ void st_bf16x4(uint16_t* p, float a, float b, float c, float d) {
+  *reinterpret_cast<uint2*>(p) = make_uint2(pack_bf16x2(a, b), pack_bf16x2(c, d));
+}
+
+__device__ __forceinline__ float sumsq4(float s, float4 v) {
+  s = fmaf(v.x, v.x, s);
+  s = fmaf(v.y, v.y, s);
+  s = fmaf(v.z, v.z, s);
+  s = fmaf(v.w, v.w, s);
+  return s;
+}
+
+__device__ __forceinline__ float inv_rms(float ss, int D, float eps) {
+  return 1.0f / sqrtf(ss / static_cast<float>(D) + eps);
+}
+
+__global__ void __launch_bounds__(kRowThreads) k_rmsnorm_rows(const uint16_t* __restrict__ x,
+                                                              const uint16_t* __restrict__ g,
+                                                              uint16_t* __restrict__ y, int D,
+                                                              float eps, int* err) {
+  __shared__ float red[kRowThreads / 32 + 1];
+  if (err != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *err = kDevOk;
+  const size_t row = blockIdx.x;
+  const int nch = D / 4;
+  const uint16_t* xr = x + row * D;
+  float4 v[kMaxChunks];
+  float ss = 0.f;
+#pragma unroll
+  for (int i = 0; i < kMaxChunks; ++i) {
+    const int c = threadIdx.x + i * kRowThreads;
+    if (c < nch) {
+      v[i] = ld_bf16x4(xr + 4 * c);
+      ss = sumsq4(ss, v[i]);
+    }
+  }
+  const float inv = inv_rms(block_sum_fixed(ss, red), D, eps);
+  uint16_t* yr = y + row * D;
+#pragma unroll
+  for (int i = 0; i < kMaxChunks; ++i) {
+    const int c = threadIdx.x + i * kRowThreads;
+    if (c < nch) {
+      const float4 gg = ld_bf16x4(g + 4 * c);
+      st_bf16x4(yr + 4 * c, v[i].x * inv * gg.x, v[i].y * inv * gg.y, v[i].z * inv * gg.z,
+                v[i].w * inv * gg.w);
+    }
+  }
+}
+
+// Shared tail of the two epilogues: r (kept in registers) -> out_residual,
+// out_norm.
+__device__ __forceinline__ void norm_store(const float4 (&r)[kMaxChunks], float ss, float* red,
+                                           const uint16_t* __restrict__ g, uint16_t* on,
+                                           int D, float eps) {
+  const int nch = D / 4;
+  const float inv = inv_rms(block_sum_fixed(ss, red), D, eps);
+#pragma unroll
+  for (int i = 0; i < kMaxChunks; ++i) {
+    const int c = threadIdx.x + i * kRowThreads;
+    if (c < nch) {
+      const float4 gg = ld_bf16x4(g + 4 * c);
+      st_bf16x4(on + 4 * c, r[i].x * inv * gg.x, r[i].y * inv * gg.y, r[i].z * inv * gg.z,
+                r[i].w * inv * gg.w);
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kRowThreads) k_combine_norm(
+    const float* __restrict__ y_slot, const float* __restrict__ topk_w,
+    const float* __restrict__ y_shared, int k, int S, const uint16_t* __restrict__ residual,
+    const uint16_t* __restrict__ g, uint16_t* __restrict__ out_norm,
+    uint16_t* __restrict__ out_residual, int T, int D, float eps) {
+  __shared__ float red[kRowThreads / 32 + 1];
+  __shared__ float w_s[16];
+  const size_t t = blockIdx.x;
+  if (threadIdx.x < k) w_s[threadIdx.x] = topk_w[t * k + threadIdx.x];
+  __syncthreads();
+  const int nch = D / 4;
+  float4 r[kMaxChunks];
+  float ss = 0.f;
+#pragma unroll
+  for (int i = 0; i < kMaxChunks; ++i) {
+    const int c = threadIdx.x + i * kRowThreads;
+    if (c < nch) {
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int j = 0; j < k; ++j) {  // routed, slot order
+        const float4 y = *reinterpret_cast<const float4*>(y_slot + (t * k + j) * D + 4 * c);
+        const float w = w_s[j];
+        acc.x = fmaf(w, y.x, acc.x); acc.y = fmaf(w, y.y, acc.y);
+        acc.z = fmaf(w, y.z, acc.z); acc.w = fmaf(w, y.w, acc.w);
+      }
+      for (int s = 0; s < S; ++s) {  // shared, index order
+        const float4 y = *reinterpret_cast<const float4*>(y_shared + (s * static_cast<size_t>(T) + t) * D + 4 * c);
+        acc.x += y.x; acc.y += y.y; acc.z += y.z; acc.w += y.w;
+      }
+      const float4 res = ld_bf16x4(residual + t * D + 4 * c);
+      r[i] = make_float4(acc.x + res.x, acc.y + res.y, acc.z + res.z, acc.w + res.w);
+      st_bf16x4(out_residual + t * D + 4 * c, r[i].x, r[i].y, r[i].z, r[i].w);
+      ss = sumsq4(ss, r[i]);
+    }
+  }
+  norm_store(r, ss, red, g, out_norm + t * D, D, eps);
+}
+
+__global__ void __launch_bounds__(kRowThreads) k_reduce_partials(
+    const PartialPtrs parts, int P, const uint16_t* __restrict__ residual,
+    const uint16_t* __restrict__ g, uint16_t* __restrict__ out_norm,
+    uint16_t* __restrict__ out_residual, int D, float eps) {
+  __shared__ float red[kRowThreads / 32 + 1];
+  const size_t t = blockIdx.x;
+  const int nch = D / 4;
+  float4 r[kMaxChunks];
+  float ss = 0.f;
+#pragma unroll
+  for (int i = 0; i < kMaxChunks; ++i) {
+    const int c = threadIdx.x + i * kRowThreads;
+    if (c < nch) {
+      const size_t off = t * D + 4 * c;
+      float4 acc = ld_bf16x4(parts.p[0] + off);
+      for (int p = 1; p < P; ++p) {  // r0 + r1 + ... + r_{P-1}, left to right
+        const float4 v = ld_bf16x4(parts.p[p] + off);
+        acc.x = __fadd_rn(acc.x, v.x); acc.y = __fadd_rn(acc.y, v.y);
+        acc.z = __fadd_rn(acc.z, v.z); acc.w = __fadd_rn(acc.w, v.w);
+      }
+      const float4 res = ld_bf16x4(residual + off);
+      r[i] = make_float4(__fadd_rn(acc.x, res.x), __fadd_rn(acc.y, res.y),
+                         __fadd_rn(acc.z, res.z), __fadd_rn(acc.w, res.w));
+      st_bf16x4(out_residual + off, r[i].x, r[i].y, r[i].z, r[i].w);
+      ss = sumsq4(ss, r[i]);
+    }
+  }
+  norm_store(r, ss, red, g, out_norm + t * D, D, eps);
+}
+
+// Count bf16 elements of a whose bits differ from the matching row of b
+// (b row = b_row_of_a[row], or row itself when NULL).
+__global__ void k_bitcompare(const uint16_t* __restrict__ a, const uint16_t* __restrict__ b,
+                             const int32_t* __restrict__ b_row_of_a, int rows, int D,
+                             unsigned long long* count) {
+  const int per_row = D / 8;
+  const size_t n = static_cast<size_t>(rows) * per_row;
+  unsigned long long mism = 0;
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const size_t row = i / per_row, col = (i % per_row) * 8;
+    const size_t brow = b_row_of_a ? static_cast<size_t>(b_row_of_a[row]) : row;
+    const uint4 va = *reinterpret_cast<const uint4*>(a + row * D + col);
+    const uint4 vb = *reinterpret_cast<const uint4*>(b + brow * D + col);
+    const uint32_t xa[4] = {va.x, va.y, va.z, va.w}, xb[4] = {vb.x, vb.y, vb.z, vb.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint32_t d = xa[q] ^ xb[q];
+      mism += ((d & 0xFFFFu) != 0) + ((d >> 16) != 0);
+    }
+  }
+  for (int o = 16; o > 0; o >>= 1) mism += __shfl_xor_sync(0xffffffffu, mism, o);
+  if ((threadIdx.x & 31) == 0 && mism) atomicAdd(count, mism);
+}
+
+// xo[i] = x[perm[i]], ro[i] = res[perm[i]], io[i] = ids[perm[i]]: one warp per row.
+__global__ void k_permute_inputs(const uint16_t* __restrict__ x, const uint16_t* __restrict__ res,
+                                 const int32_t* __restrict__ ids, const int32_t* __restrict__ perm,
+                                 int T, int D, uint16_t* __restrict__ xo, uint16_t* __restrict__ ro,
+                                 int32_t* __restrict__ io) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  if (warp >= T) return;
+  const size_t src = perm[warp];
+  const uint4* xs = reinterpret_cast<const uint4*>(x + src * D);
+  const uint4* rs = reinterpret_cast<const uint4*>(res + src * D);
+  uint4* xd = reinterpret_cast<uint4*>(xo + static_cast<size_t>(warp) * D);
+  uint4* rd = reinterpret_cast<uint4*>(ro + static_cast<size_t>(warp) * D);
+  for (int c = lane; c < D / 8; c += 32) { xd[c] = xs[c]; rd[c] = rs[c]; }
+  if (lane == 0 && ids != nullptr) io[warp] = ids[src];
+}
+
+// One thread waits on a flag nothing sets, bounded by limit_ns.
+__global__ void k_wait_selftest(volatile int* flag, int* err, unsigned long long limit_ns) {
+  const uint64_t t0 = globaltimer_ns();
+  while (*flag == 0) {
+    if (globaltimer_ns() - t0 > limit_ns) {
+      atomicExch(err, kDevTimeout);
+      return;
+    }
+    __nanosleep(1000);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_rmsnorm_rows(const uint16_t* x, const uint16_t* g, uint16_t* y, int T, int D,
+                                float eps, int* err_to_clear, cudaStream_t s) {
+  if (T <= 0) return cudaSuccess;
+  k_rmsnorm_rows<<<T, kRowThreads, 0, s>>>(x, g, y, D, eps, err_to_clear);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine_norm(const float* y_slot, const float* topk_w, const float* y_shared,
+                                int k, int S, const uint16_t* residual, const uint16_t* g,
+                                uint16_t* out_norm, uint16_t* out_residual, int T, int D,
+                                float eps, cudaStream_t s) {
+  if (T <= 0) return cudaSuccess;
+  k_combine_norm<<<T, kRowThreads, 0, s>>>(y_slot, topk_w, y_shared, k, S, residual, g, out_norm,
+                                          out_residual, T, D, eps);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_reduce_partials(const PartialPtrs& parts, int P, const uint16_t* residual,
+                                   const uint16_t* g, uint16_t* out_norm, uint16_t* out_residual,
+                                   int T, int D, float eps, cudaStream_t s) {
+  if (T <= 0) return cudaSuccess;
+  k_reduce_partials<<<T, kRowThreads, 0, s>>>(parts, P, residual, g, out_norm, out_residual, D, eps);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bitcompare(const uint16_t* a, const uint16_t* b, const int32_t* b_row_of_a,
+                              int rows, int D, unsigned long long* count, cudaStream_t s) {
+  if (rows <= 0) return cudaSuccess;
+  const size_t n = static_cast<size_t>(rows) * (D / 8);
+  int grid = static_cast<int>((n + 255) / 256);
+  if (grid > 148 * 8) grid = 148 * 8;
+  k_bitcompare<<<grid, 256, 0, s>>>(a, b, b_row_of_a, rows, D, count);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_permute_inputs(const uint16_t* x, const uint16_t* res, const int32_t* ids,
+                                  const int32_t* perm, int T, int D, uint16_t* xo, uint16_t* ro,
+                                  int32_t* io, cudaStream_t s) {
+  if (T <= 0) return cudaSuccess;
+  const int warps_per_block = 8;
+  k_permute_inputs<<<(T + warps_per_block - 1) / warps_per_block, 32 * warps_per_block, 0, s>>>(
+      x, res, ids, perm, T, D, xo, ro, io);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_wait_selftest(int* flag, int* err, unsigned long long limit_ns, cudaStream_t s) {
+  k_wait_selftest<<<1, 1, 0, s>>>(flag, err, limit_ns);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,222 @@
+/*
+ * moe.h -- C ABI of libmoe.so: a batch-invariant Mixture-of-Experts FFN layer
+ * forward for NVIDIA B200 (sm_100a).
+ *
+ * The layer (one token row t at a time; nothing depends on other rows):
+ *   xn    = bf16(RMSNorm(x_t) * g_in)                 RMSNorm, epsilon inside the root
+ *   l     = xn W_r^T                                   router Linear, fp32, full K
+ *   idx,w = top-k of softmax(l [+ b]) | sigmoid(l) + b | hash(token id)
+ *   h     = bf16(SiLU(min(xn W_g^T, c_g)) * clamp(xn W_u^T, -c_u, c_u))   per chosen expert
+ *   y     = h W_d^T                                    fp32, full K
+ *   acc   = sum_j w_j y_j (slot order) + sum_s y_s (shared, index order), fp32
+ *   r     = acc + residual_t;  out_residual = bf16(r);  out_norm = bf16(RMSNorm(r) * g_out)
+ * Passages (web pages on MoE numerics, cited by title and section):
+ *   RMSNorm ............ linux.do post on MoE variants, "RMSNorm before up-projection"
+ *   router ............. nxmr.cn "V4" article, §2.2 (Linear -> softmax -> top-k);
+ *                        DeepSeek V4 infra notes §6.3 (sigmoid + balance upper layers,
+ *                        hash routing expert = hash(token_id) % n_experts)
+ *   selection bias ..... linux.do post, "QuantileBalancing" (s + b > tau)
+ *   SwiGLU + clamp ..... DeepSeek V4 infra notes §6.5 "SwiGLU Clamping"
+ *   shared experts ..... linux.do post, "共享专家" (always active, added to the routed sum)
+ *   combine ............ Fireworks parity post (Chinese translation), Trap 3 and the
+ *                        Qwen3.5-MoE case study: all k contributions in fp32, one cast
+ *   residual + norm .... same post, Trap 2 (normed, residual = rmsnorm(full_out, residual))
+ *   r0..r7 reduction ... same post, Trap 1 (the uniform r0 + r1 + ... + r7 order, fp32)
+ *   full-K GEMMs ....... Meituan LongCat parity article, "为什么会不一致" (a full-K
+ *                        computation instead of summing split partial results)
+ *
+ * Determinism contract.  For every row t, out_norm[t], out_residual[t],
+ * out_topk_idx[t] and out_topk_w[t] are bit-identical whatever T is, where
+ * the row sits in the batch, what the other rows hold, and how often the
+ * call is repeated.  No kernel picks its tiling, split or reduction order
+ * from T; there is no split-K and no floating-point atomic.
+ *
+ * Conventions.
+ *  - "bf16" buffers hold raw bfloat16 bit patterns (moe_bf16 = uint16_t).
+ *  - All tensor arguments are DEVICE pointers, row-major, densely packed,
+ *    16-byte aligned, owned by the caller; the library never frees them.
+ *    Weight pointers given to moe_init must stay valid until moe_destroy.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *  - Every call is asynchronous on `stream` unless its comment says it
+ *    synchronises.  Nothing throws or aborts across the ABI: every call
+ *    returns a moe_status.
+ *  - Limits: D % 64 == 0, I % 64 == 0, I_shared % 64 == 0, 1 <= E <= 256,
+ *    1 <= k <= min(E, 16), 0 <= n_shared <= 8, 1 <= T_max <= 2^20,
+ *    T * max(k, n_shared) * max(D, I) < 2^31.
+ */
+#ifndef MOE_H_
+#define MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t moe_bf16;
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_EINVAL = -1,        /* bad argument: NULL pointer, negative size, bad enum    */
+  MOE_ETOOBIG = -2,       /* T > T_max of the handle                                */
+  MOE_EWORKSPACE = -3,    /* workspace smaller than moe_workspace_size()            */
+  MOE_EUNSUPPORTED = -4,  /* shape outside the limits above                         */
+  MOE_ECUDA = -5,         /* a CUDA runtime call failed (launch, copy, allocation)  */
+  MOE_ETIMEOUT = -6       /* a device-side wait gave up (see moe_get_device_error)  */
+} moe_status;
+
+typedef enum {
+  MOE_ROUTER_SOFTMAX = 0,       /* keys = logits (+ optional per-expert logit bias);
+                                   w_j = softmax prob, / sum over chosen if renormalize */
+  MOE_ROUTER_SIGMOID_BIAS = 1,  /* s = sigmoid(logit); keys = s + bias (selection only);
+                                   w_j = s_j, / sum over chosen if renormalize          */
+  MOE_ROUTER_HASH = 2           /* e_0 = ((id * hash_mult) mod 2^32) mod E,
+                                   e_j = (e_0 + j) mod E, w_j = 1/k                     */
+} moe_router;
+
+typedef struct moe_config {
+  int D;               /* hidden size                                                  */
+  int E;               /* routed experts                                               */
+  int k;               /* experts per token                                            */
+  int I;               /* routed expert intermediate size                              */
+  int n_shared;        /* always-active shared experts (0 allowed)                     */
+  int I_shared;        /* shared expert intermediate size                              */
+  int T_max;           /* largest T any call will pass                                 */
+  int router;          /* moe_router                                                   */
+  int renormalize;     /* 1: divide chosen weights by their sum (softmax / sigmoid)    */
+  float routed_scale;  /* multiplies every routed weight (1.0 = none)                  */
+  float gate_clamp_max;/* SwiGLU gate upper bound (+INF = off); the gate has no lower  */
+  float up_clamp;      /* SwiGLU up branch clipped to [-up_clamp, up_clamp] (+INF = off)*/
+  float eps;           /* RMSNorm epsilon, inside the square root                      */
+  uint32_t hash_mult;  /* multiplicative hash constant for MOE_ROUTER_HASH             */
+} moe_config;
+
+typedef struct moe_weights {      /* device pointers, caller-owned                   */
+  const moe_bf16* w_router;       /* [E, D]      (unused for hash routing)            */
+  const float* router_bias;       /* [E] fp32 or NULL: logit bias (softmax) or
+                                     selection bias (sigmoid)                         */
+  const moe_bf16* w_gate;         /* [E, I, D]                                        */
+  const moe_bf16* w_up;           /* [E, I, D]                                        */
+  const moe_bf16* w_down;         /* [E, D, I]                                        */
+  const moe_bf16* ws_gate;        /* [S, I_shared, D]  (NULL when n_shared == 0)      */
+  const moe_bf16* ws_up;          /* [S, I_shared, D]                                 */
+  const moe_bf16* ws_down;        /* [S, D, I_shared]                                 */
+  const moe_bf16* g_in;           /* [D] input RMSNorm gain                           */
+  const moe_bf16* g_out;          /* [D] output RMSNorm gain                          */
+} moe_weights;
+
+typedef struct moe_handle moe_handle;
+
+/* Number of kernel stages moe_profile_read reports, in launch order:
+ * 0 rmsnorm_in, 1 router_gemm, 2 router_topk, 3 dispatch_count, 4 dispatch_scan,
+ * 5 dispatch_scatter, 6 gather_rows, 7 gemm_gateup_swiglu, 8 gemm_down, 9 combine_norm. */
+#define MOE_NUM_STAGES 10
+
+/* Validate `cfg`, keep the weight pointers and build the weight TMA
+ * descriptors on the current CUDA device.  Allocates one small handle-owned
+ * device buffer (the router weights zero-padded to a multiple of 16 rows).
+ * Returns MOE_EINVAL / MOE_EUNSUPPORTED for bad configs (checked before any
+ * CUDA call), MOE_ECUDA when a CUDA call fails.  *out is NULL on failure. */
+int moe_init(const moe_config* cfg, const moe_weights* w, moe_handle** out);
+
+/* Bytes of device workspace moe_layer_forward needs for T rows (0 < T <= T_max).
+ * Returns 0 for a NULL handle or T outside (0, T_max]. */
+size_t moe_workspace_size(const moe_handle* h, int T);
+
+/* One layer forward over T rows.
+ *   x, residual       [T, D] bf16
+ *   token_ids         [T] int32, required for hash routing, else may be NULL
+ *   out_norm          [T, D] bf16   bf16(RMSNorm(r) * g_out)
+ *   out_residual      [T, D] bf16   bf16(r)
+ *   out_topk_idx      [T, k] int32 or NULL: chosen experts, slot order (descending key,
+ *                     ties to the lower index)
+ *   out_topk_w        [T, k] fp32 or NULL: their weights
+ *   out_counts        [E] int32 or NULL: tokens per expert (dropless; no capacity)
+ *   workspace         device buffer of >= moe_workspace_size(h, T) bytes, 256-byte
+ *                     aligned, not used by any other call in flight
+ * T == 0 returns MOE_OK and launches nothing.  Errors: MOE_EINVAL, MOE_ETOOBIG,
+ * MOE_EWORKSPACE, MOE_ECUDA (launch failure).  A device-side wait that times
+ * out is reported later by moe_get_device_error. */
+int moe_layer_forward(moe_handle* h, int T, const moe_bf16* x, const moe_bf16* residual,
+                      const int32_t* token_ids, moe_bf16* out_norm, moe_bf16* out_residual,
+                      int32_t* out_topk_idx, float* out_topk_w, int32_t* out_counts,
+                      void* workspace, size_t ws_bytes, void* stream);
+
+/* Read and clear the device error word the last forward on `workspace` left:
+ * MOE_OK, or MOE_ETIMEOUT when a bounded device wait gave up.  Synchronises
+ * `stream`. */
+int moe_get_device_error(moe_handle* h, void* workspace, void* stream);
+
+/* The tensor-parallel epilogue on one GPU (Fireworks parity post, Trap 1 + 2):
+ *   r = ((((p_0 + p_1) + p_2) + ...) + p_{P-1}) + residual   every element, fp32,
+ *   out_residual = bf16(r), out_norm = bf16(RMSNorm(r) * g).
+ * partials: HOST array of P device pointers, each [T, D] bf16; 1 <= P <= 8.
+ * residual [T, D] bf16, g [D] bf16, outputs [T, D] bf16.  D % 64 == 0.
+ * Needs no handle and no workspace.  Errors: MOE_EINVAL, MOE_EUNSUPPORTED, MOE_ECUDA. */
+int moe_reduce_partials(int P, const moe_bf16* const* partials, const moe_bf16* residual,
+                        const moe_bf16* g, moe_bf16* out_norm, moe_bf16* out_residual, int T,
+                        int D, float eps, void* stream);
+
+/* Bytes of device workspace moe_check_invariance needs for T rows. */
+size_t moe_invariance_workspace_size(const moe_handle* h, int T);
+
+/* The bitwise invariance test of the Meituan parity article ("逐 token logprob
+ * 一致": compare bit patterns, change one configuration axis at a time):
+ * run the forward on all T rows (the reference), then
+ *   - on n_splits contiguous chunks (sizes differ by at most one row),
+ *   - on the rows in the order perm (perm[i] = source row of row i; NULL = skip),
+ *   - `repeats` more times on all T rows,
+ * and count output elements (out_norm and out_residual) whose bits differ from
+ * the reference.  Synchronises `stream`; writes the count to
+ * *out_mismatched_elems.  Returns MOE_ETIMEOUT if any run hit a device timeout. */
+int moe_check_invariance(moe_handle* h, int T, const moe_bf16* x, const moe_bf16* residual,
+                         const int32_t* token_ids, int n_splits, const int32_t* perm,
+                         int repeats, void* workspace, size_t ws_bytes,
+                         unsigned long long* out_mismatched_elems, void* stream);
+
+/* Device pointers into a forward's workspace, for stage-by-stage checks.
+ * Valid after a forward with the same T and workspace has completed. */
+typedef struct moe_views {
+  const moe_bf16* xn;          /* [T, D]          normalised input                   */
+  const float* logits;         /* [T, E_pad]      router logits (NULL for hash)      */
+  int E_pad;                   /* row pitch of logits (E rounded up to 16)           */
+  const int32_t* topk_idx;     /* [T, k]          copy used inside the layer         */
+  const float* topk_w;         /* [T, k]                                             */
+  const int32_t* counts;       /* [E]                                                */
+  const int32_t* offsets;      /* [E + 1]         exclusive prefix of counts         */
+  const int32_t* src_token;    /* [T * k]         grouped row p -> token             */
+  const int32_t* dest_row;     /* [T * k]         grouped row p -> t * k + slot      */
+  const moe_bf16* h_routed;    /* [T * k, I]      grouped order                      */
+  const moe_bf16* h_shared;    /* [S, T, I_shared]                                   */
+  const float* y_slot;         /* [T, k, D]       routed expert outputs, slot order  */
+  const float* y_shared;       /* [S, T, D]                                          */
+} moe_views;
+
+int moe_workspace_views(const moe_handle* h, int T, void* workspace, moe_views* out);
+
+/* Per-stage device timing.  While enabled, every forward records a CUDA event
+ * pair around each of its MOE_NUM_STAGES launches on the forward's stream.
+ * moe_profile_read synchronises, adds each stage's elapsed time over all
+ * forwards since the last read into ms[MOE_NUM_STAGES] (milliseconds) and
+ * launches[MOE_NUM_STAGES] (kernels launched per stage), then resets.
+ * At most 256 forwards are recorded between reads; later ones are not timed. */
+int moe_profile_enable(moe_handle* h, int on);
+int moe_profile_read(moe_handle* h, float* ms, int* launches);
+
+/* Kernels launched by one forward with this T (for launch accounting). */
+int moe_forward_launch_count(const moe_handle* h, int T);
+
+/* Fault path check: launch one CTA that waits on a flag nothing sets, with a
+ * time limit of `limit_us` microseconds (1..1000000).  Returns MOE_ETIMEOUT
+ * when the wait gave up as designed (the CUDA context stays usable), MOE_OK
+ * if the flag was seen, MOE_EINVAL / MOE_ECUDA otherwise.  Synchronises `stream`. */
+int moe_selftest_wait_timeout(int limit_us, void* stream);
+
+int moe_destroy(moe_handle* h);
+const char* moe_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_H_ */

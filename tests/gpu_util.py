@@ -1,0 +1,116 @@
+"""Helpers for the GPU tests: run the layer through the C ABI on a workload and
+compare with the oracle.  Inputs come from the seeded generator twins; no
+oracle input or expected value comes from the CUDA path."""
+from __future__ import annotations
+
+import numpy as np
+
+import oracle as O
+from synth import device as SD
+from synth import workloads as W
+
+TOL_MAX = 2e-2     # max |gpu - oracle| / max(1, |oracle|) per element
+TOL_MEAN = 4e-3    # mean of the same
+NEAR_TIE = 1e-5    # routing margin below which a token may route differently
+
+
+def layer_config(cfg, T_max):
+    import deterministic_expert_b200 as moe
+    return moe.LayerConfig(D=cfg.D, E=cfg.E, k=cfg.k, I=cfg.I, n_shared=cfg.n_shared,
+                           I_shared=cfg.I_shared, T_max=T_max, router=cfg.router,
+                           renormalize=cfg.renormalize, routed_scale=cfg.routed_scale,
+                           gate_clamp_max=cfg.gate_clamp_max, up_clamp=cfg.up_clamp, eps=cfg.eps,
+                           hash_mult=cfg.hash_mult)
+
+
+class Run:
+    """One configured layer on the device with its inputs and outputs."""
+
+    def __init__(self, cfg, T=None, T_max=None, weights=None, device="cuda"):
+        import torch
+        import deterministic_expert_b200 as moe
+        self.cfg = cfg
+        self.T = cfg.T if T is None else T
+        self.T_max = T_max or max(self.T, 1)
+        self.w = weights if weights is not None else SD.device_weights(cfg, device=device)
+        self.layer = moe.MoELayer(layer_config(cfg, self.T_max), self.w)
+        self.device = device
+
+    def inputs(self, T=None):
+        return SD.device_inputs(self.cfg, T=self.T if T is None else T, device=self.device)
+
+    def forward(self, x, r, ids, ws=None):
+        import torch
+        T = int(x.shape[0])
+        if ws is None:
+            ws = torch.empty(max(self.layer.workspace_size(T), 256), dtype=torch.uint8, device=self.device)
+        on = torch.empty((T, self.cfg.D), dtype=torch.bfloat16, device=self.device)
+        orr = torch.empty_like(on)
+        idx = torch.empty((T, self.cfg.k), dtype=torch.int32, device=self.device)
+        tw = torch.empty((T, self.cfg.k), dtype=torch.float32, device=self.device)
+        cnt = torch.empty(self.cfg.E, dtype=torch.int32, device=self.device)
+        self.layer.forward(x, r, on, orr, ws, token_ids=ids, out_topk_idx=idx, out_topk_w=tw,
+                           out_counts=cnt)
+        torch.cuda.synchronize()
+        assert self.layer.device_error(ws) == 0, "device wait timed out"
+        return dict(out_norm=on, out_residual=orr, idx=idx, w=tw, counts=cnt, ws=ws)
+
+
+def np64(t):
+    import torch
+    return t.to(torch.float32).cpu().numpy().astype(np.float64)
+
+
+def rel_err(gpu, ref):
+    return np.abs(gpu - ref) / np.maximum(1.0, np.abs(ref))
+
+
+def check_outputs(out, ref, rows=None, same_rows=None):
+    """Tolerance check of out_norm / out_residual on the rows whose routing
+    matches the oracle (``same_rows``: boolean over ``rows``)."""
+    rows = np.arange(out["out_norm"].shape[0]) if rows is None else np.asarray(rows)
+    stats = {}
+    for name in ("out_norm", "out_residual"):
+        g = np64(out[name])[rows]
+        o = ref[name]
+        if same_rows is not None:
+            g, o = g[same_rows], o[same_rows]
+        e = rel_err(g, o)
+        stats[name] = (float(e.max()) if e.size else 0.0, float(e.mean()) if e.size else 0.0)
+        assert e.size == 0 or e.max() <= TOL_MAX, (name, stats[name])
+        assert e.size == 0 or e.mean() <= TOL_MEAN, (name, stats[name])
+    return stats
+
+
+def check_routing(out, ref):
+    """Indices must equal the oracle's except on near-tie tokens (margin below
+    1e-5 in the oracle's key space); a near-tie token must still have picked a
+    valid top-k under the oracle's keys (its keys within the margin of the
+    k-th).  Returns the boolean mask of rows that route exactly like the oracle."""
+    gi = out["idx"].cpu().numpy()
+    same = np.all(gi == ref["idx"], axis=1)
+    if ref["margin"] is None:  # hash routing: exact
+        assert np.all(same)
+        return same
+    bad = ~same & ~(ref["margin"] < NEAR_TIE)
+    assert not np.any(bad), f"routing differs on tokens {np.nonzero(bad)[0][:10]} (margins " \
+                            f"{ref['margin'][bad][:10]})"
+    for t in np.nonzero(~same)[0]:
+        keys = ref["keys"][t]
+        kth = np.sort(keys)[-cfg_k(ref)]
+        assert np.all(keys[gi[t]] >= kth - NEAR_TIE), t
+    return same
+
+
+def cfg_k(ref):
+    return ref["idx"].shape[1]
+
+
+def oracle_full(cfg, T=None, rows=None):
+    """Oracle on the workload's inputs (all T rows routed; experts for ``rows``)."""
+    T = cfg.T if T is None else T
+    hw = SD.HostWeights(cfg)
+    x = SD.host_rows(cfg, "x", range(T), T=T)
+    r = SD.host_rows(cfg, "residual", range(T), T=T)
+    ids = W.host_token_ids(cfg, T)
+    return O.moe_layer(cfg, hw, x, r, ids, rows=rows), hw

@@ -1,0 +1,71 @@
+"""The C ABI without a GPU: the library loads, exports every declared entry
+point, and rejects bad arguments before touching CUDA."""
+import ctypes
+import re
+
+import pytest
+
+import deterministic_expert_b200 as moe
+
+
+def declared_functions():
+    src = open(moe.HEADER_PATH).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:int|size_t|const char\*)\s+(moe_\w+)\s*\(", src, flags=re.M)))
+
+
+def test_every_declared_symbol_is_exported():
+    names = declared_functions()
+    assert len(names) >= 14
+    lib = moe.lib()
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings():
+    assert moe.status_string(0) == "ok"
+    assert "timed out" in moe.status_string(moe.MOE_ETIMEOUT)
+    assert moe.status_string(12345) == "unknown status"
+
+
+def _init(**kw):
+    base = dict(D=256, E=8, k=2, I=128, n_shared=1, I_shared=128, T_max=64)
+    base.update(kw)
+    cfg = moe.LayerConfig(**base).to_c()
+    fake = 1 << 20  # never dereferenced: validation fails first
+    w = moe.moe_weights(*[fake] * 10)
+    h = ctypes.c_void_p()
+    return moe.lib().moe_init(ctypes.byref(cfg), ctypes.byref(w), ctypes.byref(h)), h
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(D=100), moe.MOE_EUNSUPPORTED), (dict(I=96), moe.MOE_EUNSUPPORTED),
+    (dict(E=300), moe.MOE_EUNSUPPORTED), (dict(k=9), moe.MOE_EUNSUPPORTED),
+    (dict(k=0), moe.MOE_EINVAL), (dict(T_max=0), moe.MOE_EINVAL), (dict(router=7), moe.MOE_EINVAL),
+    (dict(n_shared=9), moe.MOE_EUNSUPPORTED), (dict(eps=-1.0), moe.MOE_EINVAL),
+    (dict(D=32768), moe.MOE_EUNSUPPORTED), (dict(T_max=1 << 21), moe.MOE_EUNSUPPORTED),
+])
+def test_init_rejects_bad_configs_without_cuda(kw, status):
+    rc, h = _init(**kw)
+    assert rc == status and not h.value
+
+
+def test_init_rejects_missing_weights():
+    cfg = moe.LayerConfig(D=256, E=8, k=2, I=128).to_c()
+    w = moe.moe_weights()
+    h = ctypes.c_void_p()
+    assert moe.lib().moe_init(ctypes.byref(cfg), ctypes.byref(w), ctypes.byref(h)) == moe.MOE_EINVAL
+    assert moe.lib().moe_init(None, ctypes.byref(w), ctypes.byref(h)) == moe.MOE_EINVAL
+
+
+def test_calls_reject_null_handles():
+    L = moe.lib()
+    assert L.moe_workspace_size(None, 4) == 0
+    assert L.moe_layer_forward(None, 4, *[None] * 9, 0, None) == moe.MOE_EINVAL
+    assert L.moe_destroy(None) == moe.MOE_EINVAL
+    assert L.moe_forward_launch_count(None, 1) == -1
+    assert L.moe_reduce_partials(0, None, None, None, None, None, 1, 64, 1e-6, None) == moe.MOE_EINVAL
+    arr = (ctypes.c_void_p * 1)(1 << 20)
+    assert L.moe_reduce_partials(1, arr, 1 << 20, 1 << 20, 1 << 20, 1 << 20, 4, 100, 1e-6, None) \
+        == moe.MOE_EUNSUPPORTED
+    assert L.moe_selftest_wait_timeout(0, None) == moe.MOE_EINVAL

@@ -1,0 +1,68 @@
+"""Bitwise batch invariance on the GPU (the GPU against itself; no oracle).
+
+The Meituan parity article ("逐 token logprob 一致") asks for bit-pattern
+comparison, one configuration axis at a time: here the batch is split into
+chunks, permuted, and re-run, and every output bit must match the full-batch
+run.  The decode sweep checks that a token's output is the same bits whether
+it runs alone, in a batch of 8 .. 512, or inside the 8192-row batch.
+"""
+import dataclasses
+
+import numpy as np
+import pytest
+
+from gpu_util import Run
+from synth import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def torch_cuda():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    return torch
+
+
+@pytest.mark.parametrize("name,splits", [("tiny", 7), ("fine_grained", 4), ("skew_hash", 3)])
+def test_splits_permutation_repeats(torch_cuda, name, splits):
+    torch = torch_cuda
+    cfg = W.CONFIGS[name]
+    if name == "skew_hash":
+        cfg = dataclasses.replace(cfg, T=4096)
+    run = Run(cfg)
+    x, r, ids = run.inputs()
+    perm = torch.from_numpy(W.token_permutation(cfg.T).astype(np.int32)).cuda()
+    ws = torch.empty(run.layer.invariance_workspace_size(cfg.T), dtype=torch.uint8, device="cuda")
+    mism = run.layer.check_invariance(x, r, ws, token_ids=ids, n_splits=splits, perm=perm, repeats=2)
+    assert mism == 0
+
+
+def test_decode_sweep_matches_full_batch(torch_cuda):
+    """Each decode batch (first T rows, and a random subset of T rows, of the
+    8192-row input) must reproduce those rows of the 8192-row run bit for bit."""
+    torch = torch_cuda
+    cfg = W.C2.with_T(W.C4_SOURCE_T)
+    run = Run(cfg, T_max=W.C4_SOURCE_T)
+    x, r, ids = run.inputs()
+    full = run.forward(x, r, ids)
+    for T in W.C4_T:
+        for rows in (np.arange(T), W.decode_subset(T)):
+            ri = torch.from_numpy(rows).cuda()
+            out = run.forward(x[ri].contiguous(), r[ri].contiguous(), ids[ri].contiguous())
+            for key in ("out_norm", "out_residual", "idx", "w"):
+                a = out[key].view(torch.int16) if out[key].dtype == torch.bfloat16 else out[key]
+                b = full[key][ri]
+                b = b.view(torch.int16) if b.dtype == torch.bfloat16 else b
+                assert torch.equal(a, b), (T, key)
+
+
+def test_repeat_runs_same_bits_v3_shape_small(torch_cuda):
+    torch = torch_cuda
+    cfg = dataclasses.replace(W.C3, T=512)
+    run = Run(cfg)
+    x, r, ids = run.inputs()
+    ws = torch.empty(run.layer.invariance_workspace_size(cfg.T), dtype=torch.uint8, device="cuda")
+    perm = torch.from_numpy(W.token_permutation(cfg.T, salt=3).astype(np.int32)).cuda()
+    assert run.layer.check_invariance(x, r, ws, token_ids=ids, n_splits=5, perm=perm, repeats=1) == 0
