@@ -1,0 +1,398 @@
+#!/usr/bin/env python
+"""Throughput of the batch-invariant MoE layer forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl b200|reference]
+
+One step is one full layer forward (all ten kernels: RMSNorm, router GEMM,
+top-k, histogram / scan / stable scatter, row gather, gate/up + SwiGLU GEMM,
+down GEMM, fixed-order combine + residual + RMSNorm) over one batch of the
+fine-grained workload (T=4096 tokens, D=2048, 64 experts top-6 softmax
+renormalised, I=1408, 2 shared experts of 1408) with seeded synthetic inputs
+and random weights of that architecture.  The L2 cache is flushed (a 512 MiB
+write) before every timed step; each step is timed with CUDA events on the
+launching stream.  N > 1 (torchrun, one rank per GPU) runs independent
+replicas on disjoint token batches: the layer shards by token with no data
+exchange, so scaling is weak and `value` = all ranks' tokens / the slowest
+rank's time.
+
+Printed by rank 0 as one JSON line: tokens/s, the roofline of the dominant
+kernel (the gate/up + SwiGLU grouped GEMM, tensor-bound), the end-to-end
+number through the public API with host buffers, SM clocks sampled during the
+timed region, and the fp64 CPU oracle timed on a bounded sample
+(`cpu_baseline`).  `--impl reference` times only that oracle.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE layer tokens/sec at 1 B200; % bf16 TC peak (prefill) / % HBM BW (decode)"
+UNIT = "tokens/s"
+GATEUP_STAGE = 7
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic_gemm_gateup_swiglu_fine_grained.json")
+GEMM_SOURCES = [os.path.join(ROOT, "deterministic_expert_b200", "csrc", n)
+                for n in ("grouped_gemm.cu", "common.cuh", "moe_internal.h")]
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", default="b200", choices=["b200", "reference"])
+    p.add_argument("--workload", default="fine_grained")
+    p.add_argument("--T", type=int, default=None, help="override the workload's batch size")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    a = p.parse_args()
+    a.warmup = max(a.warmup, 3)
+    return a
+
+
+def workload(a):
+    from synth import workloads as W
+    cfg = W.CONFIGS[a.workload]
+    return cfg.with_T(a.T) if a.T else cfg
+
+
+def describe(cfg):
+    from synth import workloads as W
+    return {"workload": W.pretty(cfg), "T": cfg.T, "D": cfg.D, "E": cfg.E, "k": cfg.k, "I": cfg.I,
+            "n_shared": cfg.n_shared, "I_shared": cfg.I_shared,
+            "router": {0: "softmax", 1: "sigmoid+bias", 2: "hash"}[cfg.router],
+            "renormalize": bool(cfg.renormalize)}
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d["bf16_tflops"], d["hbm_gbs"], "measured"
+    return 1590.0, 6650.0, "fallback"
+
+
+def gemm_source_hash():
+    h = hashlib.sha256()
+    for p in GEMM_SOURCES:
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def ncu_traffic(cfg):
+    """DRAM bytes per launch of the gate/up GEMM from the committed ncu summary,
+    or None when the kernel source changed since the counters were taken."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    with open(TRAFFIC_FILE) as f:
+        d = json.load(f)
+    if d.get("source_sha256") != gemm_source_hash() or d.get("T") != cfg.T or d.get("workload") != cfg.name:
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    def __init__(self, index):
+        self.file = tempfile.NamedTemporaryFile(prefix="clocks", suffix=".csv", delete=False)
+        q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(index), f"--query-gpu={q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.file, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.file.close()
+        rows = []
+        with open(self.file.name) as f:
+            for line in f:
+                parts = [s.strip() for s in line.split(",")]
+                if len(parts) >= 8:
+                    rows.append(parts)
+        os.unlink(self.file.name)
+        if not rows:
+            return None
+        sm = [float(r[0]) for r in rows if r[0].replace(".", "").isdigit()]
+        mx = max(float(r[1]) for r in rows if r[1].replace(".", "").isdigit())
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[4 + i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ oracle
+def oracle_sample(cfg, budget_s=12.0, chunk=256):
+    """Time the fp64 oracle (as it stands) on chunks of the workload's tokens
+    until about budget_s of CPU work has run.  Weight generation is not timed."""
+    import numpy as np
+    from threadpoolctl import threadpool_info
+
+    import oracle as O
+    from synth import device as SD
+    hw = SD.HostWeights(cfg)
+    for e in range(cfg.E):
+        hw.routed(e)
+    for s in range(cfg.n_shared):
+        hw.shared(s)
+    from synth import workloads as W
+    tokens, spent, chunks = 0, 0.0, 0
+    while spent < budget_s and tokens < cfg.T:
+        rows = np.arange(tokens, min(cfg.T, tokens + chunk))
+        x = SD.host_rows(cfg, "x", rows, T=cfg.T)
+        r = SD.host_rows(cfg, "residual", rows, T=cfg.T)
+        ids = W.host_token_ids(cfg, cfg.T)[rows]
+        t0 = time.perf_counter()
+        O.moe_layer(cfg, hw, x, r, ids)
+        spent += time.perf_counter() - t0
+        tokens += len(rows)
+        chunks += 1
+    cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    return {"value": tokens / spent, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{tokens} of {cfg.T} tokens ({chunks} chunks of {chunk}), full layer in fp64, "
+                      f"{spent:.1f} s of oracle time; weight generation not timed"}
+
+
+def run_reference(a):
+    """--impl reference: the oracle on the same workload, rank 0 only."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    cfg = workload(a)
+    import numpy as np
+    from threadpoolctl import threadpool_info
+
+    import oracle as O
+    from synth import device as SD
+    from synth import workloads as W
+    hw = SD.HostWeights(cfg)
+    for e in range(cfg.E):
+        hw.routed(e)
+    for s in range(cfg.n_shared):
+        hw.shared(s)
+    chunk = 128
+    ids_all = W.host_token_ids(cfg, cfg.T)
+    times = []
+    for step in range(a.warmup + a.steps):
+        r0 = (step * chunk) % cfg.T
+        rows = np.arange(r0, min(cfg.T, r0 + chunk))
+        x = SD.host_rows(cfg, "x", rows, T=cfg.T)
+        r = SD.host_rows(cfg, "residual", rows, T=cfg.T)
+        t0 = time.perf_counter()
+        O.moe_layer(cfg, hw, x, r, ids_all[rows])
+        dt = time.perf_counter() - t0
+        if step >= a.warmup:
+            times.append((dt, len(rows)))
+    secs = sum(t for t, _ in times)
+    toks = sum(n for _, n in times)
+    value = toks / secs
+    cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": a.gpus,
+        "steps": a.steps, "warmup": a.warmup, "ms_per_step": 1e3 * secs / len(times),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded counter-based generator; random weights of the workload's shape)",
+        "config": describe(cfg),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"each step: {chunk} tokens of the {cfg.T}-token batch, full layer in fp64"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+# --------------------------------------------------------------- b200 arm
+def main():
+    a = parse()
+    if a.impl == "reference":
+        run_reference(a)
+        return
+    import torch
+    import torch.distributed as dist
+
+    import deterministic_expert_b200 as moe
+    from synth import device as SD
+    from synth import workloads as W
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != a.gpus:
+        a.gpus = world
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    cfg = workload(a)
+    T = cfg.T
+    stream = torch.cuda.current_stream()
+
+    w = SD.device_weights(cfg, device=dev)
+    # Each rank takes its own T rows of a world*T-row batch (disjoint tokens).
+    xa, ra, ida = SD.device_inputs(cfg, T=T * world, device=dev)
+    x, r, ids = (xa[rank * T:(rank + 1) * T].contiguous(), ra[rank * T:(rank + 1) * T].contiguous(),
+                 ida[rank * T:(rank + 1) * T].contiguous())
+    del xa, ra, ida
+    lc = moe.LayerConfig(D=cfg.D, E=cfg.E, k=cfg.k, I=cfg.I, n_shared=cfg.n_shared,
+                         I_shared=cfg.I_shared, T_max=T, router=cfg.router,
+                         renormalize=cfg.renormalize, routed_scale=cfg.routed_scale,
+                         gate_clamp_max=cfg.gate_clamp_max, up_clamp=cfg.up_clamp, eps=cfg.eps,
+                         hash_mult=cfg.hash_mult)
+    layer = moe.MoELayer(lc, w)
+    ws = torch.empty(layer.workspace_size(T), dtype=torch.uint8, device=dev)
+    on = torch.empty((T, cfg.D), dtype=torch.bfloat16, device=dev)
+    orr = torch.empty_like(on)
+    cnt = torch.empty(cfg.E, dtype=torch.int32, device=dev)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    use_ids = ids if cfg.router == W.ROUTER_HASH else None
+
+    def step(timed_events=None):
+        flush.fill_(1)
+        if timed_events:
+            timed_events[0].record(stream)
+        layer.forward(x, r, on, orr, ws, token_ids=use_ids, out_counts=cnt, stream=stream)
+        if timed_events:
+            timed_events[1].record(stream)
+
+    for _ in range(a.warmup):
+        step()
+    torch.cuda.synchronize()
+    if layer.device_error(ws) != moe.MOE_OK:
+        raise RuntimeError("device wait timed out during warm-up")
+
+    # ------------------------------------------------ timed region (value)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(a.steps)]
+    clocks = ClockSampler(local) if rank == 0 else None
+    layer.profile_enable([GATEUP_STAGE])
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for i in range(a.steps):
+        step(evs[i])
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop() if clocks else None
+    ms_steps = [e0.elapsed_time(e1) for e0, e1 in evs]
+    stage_ms, stage_n = layer.profile_read()
+    layer.profile_enable([])
+    if layer.device_error(ws) != moe.MOE_OK:
+        raise RuntimeError("device wait timed out in the timed region")
+    ms_total = torch.tensor([sum(ms_steps)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(ms_total, op=dist.ReduceOp.MAX)
+    ms_per_step = float(ms_total.item()) / a.steps
+    value = world * T / (ms_per_step / 1e3)
+    distinct = int((cnt > 0).sum().item())
+
+    # --------------------------------------------- per-stage breakdown (untimed)
+    layer.profile_enable(None)
+    for _ in range(3):
+        step()
+    all_ms, all_n = layer.profile_read()
+    layer.profile_enable([])
+    stage_avg = {moe.STAGE_NAMES[i]: round(all_ms[i] / all_n[i] * 1e3, 2) if all_n[i] else None
+                 for i in range(moe.NUM_STAGES)}
+
+    # ------------------------------------------------------- e2e (host buffers)
+    xh, rh = x.cpu().pin_memory(), r.cpu().pin_memory()
+    idh = ids.cpu().pin_memory()
+    onh = torch.empty(on.shape, dtype=on.dtype).pin_memory()
+    orh = torch.empty_like(onh).pin_memory()
+    h2d = xh.numel() * 2 + rh.numel() * 2 + (idh.numel() * 4 if use_ids is not None else 0)
+    d2h = onh.numel() * 2 + orh.numel() * 2
+
+    def e2e_step(ev=None):
+        flush.fill_(1)
+        if ev:
+            ev[0].record(stream)
+        x.copy_(xh, non_blocking=True)
+        r.copy_(rh, non_blocking=True)
+        if use_ids is not None:
+            ids.copy_(idh, non_blocking=True)
+        layer.forward(x, r, on, orr, ws, token_ids=use_ids, stream=stream)
+        onh.copy_(on, non_blocking=True)
+        orh.copy_(orr, non_blocking=True)
+        if ev:
+            ev[1].record(stream)
+
+    for _ in range(a.warmup):
+        e2e_step()
+    ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(a.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for i in range(a.steps):
+        e2e_step(ev2[i])
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e2e_ms = torch.tensor([sum(e0.elapsed_time(e1) for e0, e1 in ev2)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
+    e2e_value = world * T / (float(e2e_ms.item()) / a.steps / 1e3)
+
+    if rank == 0:
+        tc_peak, hbm_peak, peak_kind = peaks()
+        fl = W.moe_flops(cfg)
+        gate_ms = stage_ms[GATEUP_STAGE] / max(stage_n[GATEUP_STAGE], 1)
+        achieved = fl["gateup"] / (gate_ms / 1e3) / 1e12
+        traffic = ncu_traffic(cfg)
+        roof = {"bound": "tensor", "kernel": "gemm_gateup_swiglu", "achieved": round(achieved, 1),
+                "peak": tc_peak, "unit": "TFLOP/s", "frac": round(achieved / tc_peak, 4),
+                "traffic": traffic, "peak_source": f"{peak_kind} bf16 (burst)",
+                "flops_per_launch": fl["gateup"], "avg_launch_ms": round(gate_ms, 4)}
+        layer_tflops = fl["total"] / (ms_per_step / 1e3) / 1e12
+        cpu = None
+        if world == 1 and not a.no_cpu_baseline:
+            cpu = oracle_sample(cfg)
+        line = {
+            "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+            "steps": a.steps, "warmup": a.warmup, "ms_per_step": round(ms_per_step, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded counter-based generator; random weights of the workload's shape)",
+            "config": {**describe(cfg), "l2": "flushed before every step (512 MiB write, untimed)",
+                       "parallelism": f"replicas x{world} (token-sharded, no collective)"},
+            "roofline": roof,
+            "layer": {"tflops": round(layer_tflops, 1), "frac_of_tc_peak": round(layer_tflops / tc_peak, 4),
+                      "flops_per_step": fl["total"], "distinct_experts": distinct,
+                      "algorithmic_bytes": W.layer_bytes(cfg, T, distinct)},
+            "stage_us": stage_avg,
+            "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": a.steps * layer.launch_count(T),
+            "clocks": clk,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    layer.close()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -186,8 +186,13 @@ class MoELayer:
                "moe_workspace_views")
         return v
 
-    def profile_enable(self, on: bool = True) -> None:
-        _check(lib().moe_profile_enable(self.handle, int(on)), "moe_profile_enable")
+    def profile_enable(self, stages=None) -> None:
+        """Time the given stage indices (all when None; [] turns timing off)."""
+        stages = range(NUM_STAGES) if stages is None else stages
+        mask = 0
+        for s_ in stages:
+            mask |= 1 << int(s_)
+        _check(lib().moe_profile_enable(self.handle, mask), "moe_profile_enable")
 
     def profile_read(self):
         ms = (ctypes.c_float * NUM_STAGES)()

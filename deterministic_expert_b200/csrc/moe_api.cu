@@ -22,7 +22,7 @@ struct moe_handle {
   CUtensorMap map_router, map_wg, map_wu, map_wd, map_wsg, map_wsu, map_wsd;
   unsigned long long timeout_ns = 2000ull * 1000 * 1000;
   // Per-stage timing (moe_profile_*).
-  bool prof_on = false;
+  int prof_mask = 0;
   int prof_fwd = 0;
   std::vector<cudaEvent_t> ev;  // [kProfFwd][MOE_NUM_STAGES][2]
   int prof_launches[MOE_NUM_STAGES] = {0};
@@ -146,11 +146,12 @@ struct Prof {
   moe_handle* h;
   cudaStream_t s;
   int f;
+  bool on(int stage) const { return f >= 0 && ((h->prof_mask >> stage) & 1); }
   void begin(int stage) {
-    if (f >= 0) cudaEventRecord(h->ev[(static_cast<size_t>(f) * MOE_NUM_STAGES + stage) * 2], s);
+    if (on(stage)) cudaEventRecord(h->ev[(static_cast<size_t>(f) * MOE_NUM_STAGES + stage) * 2], s);
   }
   void end(int stage) {
-    if (f >= 0) {
+    if (on(stage)) {
       cudaEventRecord(h->ev[(static_cast<size_t>(f) * MOE_NUM_STAGES + stage) * 2 + 1], s);
       h->prof_launches[stage] += 1;
     }
@@ -196,7 +197,7 @@ int forward_impl(moe_handle* h, int T, const uint16_t* x, const uint16_t* residu
   const int TK = T * c.k;
 
   Prof prof{h, s, -1};
-  if (h->prof_on && h->prof_fwd < kProfFwd) prof.f = h->prof_fwd++;
+  if (h->prof_mask && h->prof_fwd < kProfFwd) prof.f = h->prof_fwd++;
 
   // 0. input RMSNorm (also clears the device error word)
   prof.begin(0);
@@ -519,14 +520,14 @@ int moe_workspace_views(const moe_handle* h, int T, void* workspace, moe_views* 
   return MOE_OK;
 }
 
-int moe_profile_enable(moe_handle* h, int on) {
-  if (!h) return MOE_EINVAL;
-  if (on && h->ev.empty()) {
+int moe_profile_enable(moe_handle* h, int stage_mask) {
+  if (!h || stage_mask < 0 || stage_mask >= (1 << MOE_NUM_STAGES)) return MOE_EINVAL;
+  if (stage_mask && h->ev.empty()) {
     h->ev.resize(static_cast<size_t>(kProfFwd) * MOE_NUM_STAGES * 2);
     for (auto& e : h->ev)
       if (cudaEventCreate(&e) != cudaSuccess) return MOE_ECUDA;
   }
-  h->prof_on = on != 0;
+  h->prof_mask = stage_mask;
   h->prof_fwd = 0;
   for (int i = 0; i < MOE_NUM_STAGES; ++i) h->prof_launches[i] = 0;
   return MOE_OK;
@@ -537,6 +538,7 @@ int moe_profile_read(moe_handle* h, float* ms, int* launches) {
   for (int i = 0; i < MOE_NUM_STAGES; ++i) { ms[i] = 0.f; launches[i] = h->prof_launches[i]; }
   for (int f = 0; f < h->prof_fwd; ++f) {
     for (int st = 0; st < MOE_NUM_STAGES; ++st) {
+      if (!((h->prof_mask >> st) & 1)) continue;
       cudaEvent_t a = h->ev[(static_cast<size_t>(f) * MOE_NUM_STAGES + st) * 2];
       cudaEvent_t b = h->ev[(static_cast<size_t>(f) * MOE_NUM_STAGES + st) * 2 + 1];
       if (cudaEventQuery(b) == cudaErrorNotReady && cudaEventSynchronize(b) != cudaSuccess) return MOE_ECUDA;

@@ -195,13 +195,15 @@ typedef struct moe_views {
 
 int moe_workspace_views(const moe_handle* h, int T, void* workspace, moe_views* out);
 
-/* Per-stage device timing.  While enabled, every forward records a CUDA event
- * pair around each of its MOE_NUM_STAGES launches on the forward's stream.
+/* Per-stage device timing.  stage_mask selects stages (bit s = stage s;
+ * 0 = off; (1 << MOE_NUM_STAGES) - 1 = all).  While enabled, every forward
+ * records a CUDA event pair on its stream around each selected stage's launch.
  * moe_profile_read synchronises, adds each stage's elapsed time over all
  * forwards since the last read into ms[MOE_NUM_STAGES] (milliseconds) and
- * launches[MOE_NUM_STAGES] (kernels launched per stage), then resets.
- * At most 256 forwards are recorded between reads; later ones are not timed. */
-int moe_profile_enable(moe_handle* h, int on);
+ * launches[MOE_NUM_STAGES] (kernels launched per stage, selected stages only),
+ * then resets.  At most 256 forwards are recorded between reads; later ones
+ * are not timed. */
+int moe_profile_enable(moe_handle* h, int stage_mask);
 int moe_profile_read(moe_handle* h, float* ms, int* launches);
 
 /* Kernels launched by one forward with this T (for launch accounting). */

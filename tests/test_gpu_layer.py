@@ -17,6 +17,12 @@ from synth import workloads as W
 
 pytestmark = pytest.mark.gpu
 
+# Routing weights (in [0, 1]) inherit the logit differences of xn elements that
+# the fp32 kernel and the fp64 oracle round to neighbouring bf16 values: one
+# bf16 ulp (<= 2^-7 relative) times a router weight (|w| ~ 0.02 * 6 sigma)
+# per flipped element moves a logit by ~1e-3 at most, and a weight by less.
+W_TOL = 2e-3
+
 
 @pytest.fixture(scope="module")
 def torch_cuda():
@@ -104,7 +110,7 @@ def test_tiny_layer_parity_with_stages(torch_cuda):
     assert np.array_equal(out["counts"].cpu().numpy(), O.expert_histogram(out["idx"].cpu().numpy(), cfg.E))
     check_outputs(out, ref, same_rows=same)
     w = out["w"].cpu().numpy().astype(np.float64)
-    assert np.abs(w[same] - ref["w"][same]).max() < 1e-5
+    assert np.abs(w[same] - ref["w"][same]).max() < W_TOL
     _stage_checks(run, out, ref, hw, torch_cuda)
 
 
@@ -116,7 +122,7 @@ def test_fine_grained_layer_parity(torch_cuda):
     same = check_routing(out, ref)
     check_outputs(out, ref, same_rows=same)
     w = out["w"].cpu().numpy().astype(np.float64)
-    assert np.abs(w[same] - ref["w"][same]).max() < 1e-5
+    assert np.abs(w[same] - ref["w"][same]).max() < W_TOL
     assert np.allclose(w.sum(1), 1.0, atol=1e-5)  # renormalised
     _stage_checks(run, out, ref, hw, torch_cuda)
 

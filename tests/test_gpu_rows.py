@@ -47,10 +47,6 @@ def test_fixed_order_bit_exact(torch_cuda, P, T, D):
     assert np.array_equal(np64(orr), want_r)
     e = rel_err(np64(on), want_n)
     assert e.max() <= TOL_MAX and e.mean() <= TOL_MEAN
-    if P == 8 and T * D >= 8 * 8192:
-        ring = O.allreduce_ring_order_f32(pf) + res.float().numpy()
-        ring_bf = O.round_bf16(ring.astype(np.float64))
-        assert not np.array_equal(ring_bf, want_r)
 
 
 def test_epilogue_full_size_sampled_rows(torch_cuda):
@@ -71,3 +67,31 @@ def test_epilogue_full_size_sampled_rows(torch_cuda):
     assert np.array_equal(np64(orr)[rows], want_r)
     e = rel_err(np64(on)[rows], want_n)
     assert e.max() <= TOL_MAX and e.mean() <= TOL_MEAN
+
+
+def test_order_change_is_visible(torch_cuda):
+    """A case where the two orders differ after bf16 rounding, derived by hand
+    in fp32 (P = 8, residual 0, every element r0 = 1, r1 = -1, r2 = 2^-25,
+    r3..r7 = 0; the ring cuts D into 8 chunks):
+      fixed, every element: (1 - 1) + 2^-25 = 2^-25.
+      ring chunk 0: 1 + 0 .. + 2^-25 -> 1 (2^-25 < half an ulp of 1), - 1 = 0.
+      ring chunk 1: (-1 + 1) + 0 .. + 2^-25 = 2^-25.
+      ring chunks 2..7: 2^-25 - 1 is a tie between -1 and -(1 - 2^-24) and
+      rounds to the even -1; + 1 = 0.
+    The kernel must give 2^-25 everywhere: the fixed order, not the ring's."""
+    torch = torch_cuda
+    T, D = 4, 256
+    vals = [1.0, -1.0, 2.0 ** -25, 0, 0, 0, 0, 0]
+    parts = [torch.full((T, D), v, dtype=torch.bfloat16) for v in vals]
+    res = torch.zeros((T, D), dtype=torch.bfloat16)
+    g = torch.ones(D, dtype=torch.bfloat16)
+    on, orr = _run(torch, [p.cuda() for p in parts], res.cuda(), g.cuda())
+    got = np64(orr)
+    assert np.all(got == 2.0 ** -25)
+    pf = np.stack([p.float().numpy() for p in parts])
+    assert np.array_equal(O.allreduce_fixed_order_f32(pf), np.full((T, D), 2.0 ** -25, np.float32))
+    ring = O.allreduce_ring_order_f32(pf)
+    c = D // 8
+    assert np.all(ring[:, :c] == 0) and np.all(ring[:, c:2 * c] == 2.0 ** -25) and np.all(ring[:, 2 * c:] == 0)
+    assert not np.array_equal(O.round_bf16(ring.astype(np.float64)), got)
+
