@@ -217,3 +217,18 @@ def reduce_partials(partials, residual, g, out_norm, out_residual, eps: float = 
 
 def selftest_wait_timeout(limit_us: int, stream=None) -> int:
     return int(lib().moe_selftest_wait_timeout(limit_us, _stream(stream)))
+
+
+def forward_noalloc(layer: MoELayer, x, residual, out_norm, out_residual, token_ids=None,
+                    out_topk_idx=None, out_topk_w=None, out_counts=None, stream=None) -> None:
+    """moe_layer_forward_noalloc: the layer forward for decode-sized batches
+    without a caller workspace (scratch in a static 32 MiB device array), for
+    callers that cannot allocate device memory.  See include/moe.h."""
+    L = lib()
+    fn = L.moe_layer_forward_noalloc
+    vp = ctypes.c_void_p
+    fn.argtypes = [vp, ctypes.c_int, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+    _check(fn(layer.handle, int(x.shape[0]), _ptr(x), _ptr(residual), _ptr(token_ids),
+              _ptr(out_norm), _ptr(out_residual), _ptr(out_topk_idx), _ptr(out_topk_w),
+              _ptr(out_counts), _stream(stream)),
+           "moe_layer_forward_noalloc")

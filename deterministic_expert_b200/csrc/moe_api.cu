@@ -597,3 +597,52 @@ const char* moe_status_string(int status) {
 }
 
 }  // extern "C"
+
+// ------------------------------------------------- no-allocation forward
+// The workspace of moe_layer_forward_noalloc: one static device array per GPU
+// (held by every GPU that loads the library until the process exits).  Host
+// code only knows a host-side stand-in for its name, so its device address is
+// looked up once per device with cudaGetSymbolAddress and cached.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[MOE_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {nullptr};
+
+// Device address of g_noalloc_scratch on the current device (nullptr on failure).
+void* noalloc_scratch() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    g_noalloc_ptr[dev] = p;
+  }
+  return g_noalloc_ptr[dev];
+}
+}  // namespace
+
+extern "C" int moe_layer_forward_noalloc(moe_handle* h, int T, const moe_bf16* x,
+                                         const moe_bf16* residual, const int32_t* token_ids,
+                                         moe_bf16* out_norm, moe_bf16* out_residual,
+                                         int32_t* out_topk_idx, float* out_topk_w,
+                                         int32_t* out_counts, void* stream) {
+  if (!h || T < 0) return MOE_EINVAL;
+  if (T > h->cfg.T_max) return MOE_ETOOBIG;
+  if (T == 0) return MOE_OK;
+  const size_t need = layout(h, T).total;
+  if (need > MOE_NOALLOC_SCRATCH_BYTES) return MOE_EWORKSPACE;
+  void* ws = noalloc_scratch();
+  if (!ws) return MOE_ECUDA;
+  const int v = check_forward_args(h, T, x, residual, token_ids, out_norm, out_residual, ws,
+                                   MOE_NOALLOC_SCRATCH_BYTES, need);
+  if (v != MOE_OK) return v;
+  return forward_impl(h, T, x, residual, token_ids, out_norm, out_residual, out_topk_idx,
+                      out_topk_w, out_counts, static_cast<uint8_t*>(ws),
+                      static_cast<cudaStream_t>(stream));
+}

@@ -215,6 +215,31 @@ int moe_forward_launch_count(const moe_handle* h, int T);
  * if the flag was seen, MOE_EINVAL / MOE_ECUDA otherwise.  Synchronises `stream`. */
 int moe_selftest_wait_timeout(int limit_us, void* stream);
 
+/* Forward without any allocation, for callers that cannot call cudaMalloc:
+ * a plugin or custom-op enqueue path that must not allocate, a process whose
+ * own allocator already holds all free device memory, or a latency-critical
+ * path that cannot afford cudaMalloc's device-wide synchronisation.  (The
+ * source pages have no counterpart of this entry point.)
+ * Same arguments and results as moe_layer_forward, minus the workspace: the
+ * scratch is one static device array of MOE_NOALLOC_SCRATCH_BYTES (32 MiB)
+ * that every GPU loading the library holds until the process exits.  T must
+ * satisfy moe_workspace_size(h, T) <= MOE_NOALLOC_SCRATCH_BYTES (decode-sized
+ * batches: about 280 tokens for D=2048, top-6, I=1408, 2 shared experts);
+ * larger T returns MOE_EWORKSPACE and launches nothing.
+ * The first call on each device looks up the array's device address with that
+ * device current; make that first call before any stream capture.
+ * Every call shares the array and it keeps the last call's contents; the
+ * only value that must start at zero (the device error word) is cleared by
+ * the call's first kernel.  Calls whose kernels overlap on the GPU (other
+ * streams, or another thread's call) race on the array: serialise them.
+ * A device-side wait time-out is recorded in the array's error word and is
+ * not reported to the caller. */
+#define MOE_NOALLOC_SCRATCH_BYTES (32u << 20)
+int moe_layer_forward_noalloc(moe_handle* h, int T, const moe_bf16* x, const moe_bf16* residual,
+                              const int32_t* token_ids, moe_bf16* out_norm,
+                              moe_bf16* out_residual, int32_t* out_topk_idx, float* out_topk_w,
+                              int32_t* out_counts, void* stream);
+
 int moe_destroy(moe_handle* h);
 const char* moe_status_string(int status);
 
