@@ -82,6 +82,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
   uint64_t* tfull = bars + 2 * kStages;
   uint64_t* tempty = tfull + 2;
   uint64_t* tdone = tempty + 2;
+  uint8_t* epi = reinterpret_cast<uint8_t*>(bars) + 256;  // 4 warps x 32 x kEpiStride words
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
 
@@ -181,8 +182,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
     }
   } else {
     // --------------------------------------------------------- epilogue
+    // Each warp owns 32 accumulator rows (one TMEM lane quarter).  It reads 32
+    // columns per tcgen05.ld (lane i = row i), stages the 32 x 32 block in its
+    // own shared buffer, and stores it back so that every store instruction
+    // writes whole 128-byte row segments (8 lanes per row, 4 rows at a time).
     const int q = warp & 3;           // TMEM lane quarter this warp may access
     const int row = q * 32 + lane;    // accumulator row = TMEM lane
+    uint32_t* stage_w = reinterpret_cast<uint32_t*>(epi) + (warp - 2) * (32 * kEpiStride);
+    const int sr = lane >> 3, sc = lane & 7;  // store phase: row offset 0..3, 16-byte column 0..7
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x) {
@@ -193,18 +200,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
       tc_fence_after();
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                           static_cast<uint32_t>(acc) * acc_stride;
-      const int grow = ti.m * kBM + row;
-      const bool valid = grow < ti.rows;
+      const int grow0 = ti.m * kBM + q * 32;   // first group row of this warp's block
+      const int nvalid = max(0, min(32, ti.rows - grow0));
       if (MODE == kGateUp) {
-        const int orow = (ti.kind == 0 ? ti.a_row0 : ti.idx * a.shared_out_stride) + grow;
-        uint16_t* out = static_cast<uint16_t*>(a.out[ti.kind]) +
-                        static_cast<size_t>(orow) * a.ld_out[ti.kind] + ti.n * BN;
-        for (int c = 0; c < BN; c += 32) {
-          uint32_t g[32], u[32];
-          tmem_ld32(tb + c, g);
-          tmem_ld32(tb + BN + c, u);
-          tmem_ld_wait();
-          if (valid) {
+        // 64 output columns (128 bytes of bf16) per staged block.
+        const int orow0 = (ti.kind == 0 ? ti.a_row0 : ti.idx * a.shared_out_stride) + grow0;
+        uint8_t* out0 = reinterpret_cast<uint8_t*>(static_cast<uint16_t*>(a.out[ti.kind]) + ti.n * BN);
+        const size_t ld_bytes = static_cast<size_t>(a.ld_out[ti.kind]) * 2;
+        for (int c = 0; c < BN; c += 64) {
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            uint32_t g[32], u[32];
+            tmem_ld32(tb + c + 32 * half, g);
+            tmem_ld32(tb + BN + c + 32 * half, u);
+            tmem_ld_wait();
             uint32_t p[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i)
@@ -213,28 +222,53 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
                                        a.gate_clamp, a.up_clamp),
                   silu_clamped_product(__uint_as_float(g[2 * i + 1]), __uint_as_float(u[2 * i + 1]),
                                        a.gate_clamp, a.up_clamp));
-            uint4* dst = reinterpret_cast<uint4*>(out + c);
+            uint4* dst = reinterpret_cast<uint4*>(stage_w + lane * kEpiStride + 16 * half);
 #pragma unroll
             for (int i = 0; i < 4; ++i) dst[i] = make_uint4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
           }
+          __syncwarp();
+#pragma unroll
+          for (int s8 = 0; s8 < 8; ++s8) {
+            const int r = 4 * s8 + sr;
+            if (r < nvalid) {
+              const uint4 v = *reinterpret_cast<const uint4*>(stage_w + r * kEpiStride + 4 * sc);
+              *reinterpret_cast<uint4*>(out0 + static_cast<size_t>(orow0 + r) * ld_bytes + c * 2 + 16 * sc) = v;
+            }
+          }
+          __syncwarp();
         }
       } else {
-        float* out;
-        if (MODE == kDown && ti.kind == 0) {
-          const int drow = valid ? a.dest_row[ti.a_row0 + grow] : 0;
-          out = static_cast<float*>(a.out[0]) + static_cast<size_t>(drow) * a.ld_out[0];
-        } else {
-          const int orow = (ti.kind == 0 ? ti.a_row0 : ti.idx * a.shared_out_stride) + grow;
-          out = static_cast<float*>(a.out[ti.kind]) + static_cast<size_t>(orow) * a.ld_out[ti.kind];
-        }
-        out += ti.n * BN;
+        // fp32 output, 32 columns (128 bytes) per staged block.
+        const bool scatter = (MODE == kDown && ti.kind == 0);
+        const int my_dest = (scatter && lane < nvalid) ? a.dest_row[ti.a_row0 + grow0 + lane] : 0;
+        const int orow0 = (ti.kind == 0 ? ti.a_row0 : ti.idx * a.shared_out_stride) + grow0;
+        float* out0 = static_cast<float*>(a.out[ti.kind]) + ti.n * BN;
+        const size_t ld = static_cast<size_t>(a.ld_out[ti.kind]);
         for (int c = 0; c < BN; c += 32) {
           uint32_t v[32];
           tmem_ld32(tb + c, v);
           tmem_ld_wait();
-          if (valid) {
-            const int nq = min(32, BN - c) / 4;
-            float4* dst = reinterpret_cast<float4*>(out + c);
+          if (BN - c >= 32) {
+            uint4* dst = reinterpret_cast<uint4*>(stage_w + lane * kEpiStride);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) dst[i] = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+            __syncwarp();
+#pragma unroll
+            for (int s8 = 0; s8 < 8; ++s8) {
+              const int r = 4 * s8 + sr;
+              const int drow = __shfl_sync(0xffffffffu, my_dest, r);
+              if (r < nvalid) {
+                const uint4 val = *reinterpret_cast<const uint4*>(stage_w + r * kEpiStride + 4 * sc);
+                const size_t orow = scatter ? static_cast<size_t>(drow) : static_cast<size_t>(orow0 + r);
+                *reinterpret_cast<uint4*>(out0 + orow * ld + c + 4 * sc) = val;
+              }
+            }
+            __syncwarp();
+          } else if (lane < nvalid) {
+            // Narrow tail (router with fewer than 32 columns left): direct stores.
+            const size_t orow = scatter ? static_cast<size_t>(my_dest) : static_cast<size_t>(orow0 + lane);
+            float4* dst = reinterpret_cast<float4*>(out0 + orow * ld + c);
+            const int nq = (BN - c) / 4;
 #pragma unroll
             for (int i = 0; i < 8; ++i)
               if (i < nq)

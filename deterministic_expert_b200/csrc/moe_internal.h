@@ -21,7 +21,8 @@ constexpr int kStages = 4;
 constexpr int kGemmThreads = 192;  // warp 0: TMA, warp 1: MMA, warps 2-5: epilogue
 constexpr int kSmemA = kBM * kBK * 2;
 constexpr int kSmemBMax = 256 * kBK * 2;
-constexpr int kGemmSmem = 1024 + kStages * (kSmemA + kSmemBMax) + 256;
+constexpr int kEpiStride = 36;  // words per staged epilogue row (128 B + 16 B pad)
+constexpr int kGemmSmem = 1024 + kStages * (kSmemA + kSmemBMax) + 256 + 4 * 32 * kEpiStride * 4;
 
 enum GemmMode : int { kGateUp = 0, kDown = 1, kRouter = 2 };
 

@@ -22,6 +22,16 @@ namespace {
 
 constexpr int kMaxChunks = 16;  // D <= 4 * 256 * 16 = 16384
 
+// Chunks per thread for a row of D elements: the smallest of 1, 2, 4, 8, 16
+// with 4 * 256 * NC >= D.  It depends on D only, so thread i owns the same
+// chunks i, i + 256, ... whatever T is; the template bound only trims
+// registers (kernels for small D keep fewer live values).
+inline int chunks_for(int D) {
+  int nc = 1;
+  while (nc < kMaxChunks && 4 * kRowThreads * nc < D) nc *= 2;
+  return nc;
+}
+
 __device__ __forceinline__ float4 ld_bf16x4(const uint16_t* p) {
   const uint2 v = *reinterpret_cast<const uint2*>(p);
   return make_float4(bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y));
@@ -43,6 +53,7 @@ __device__ __forceinline__ float inv_rms(float ss, int D, float eps) {
   return 1.0f / sqrtf(ss / static_cast<float>(D) + eps);
 }
 
+template <int NC>
 __global__ void __launch_bounds__(kRowThreads) k_rmsnorm_rows(const uint16_t* __restrict__ x,
                                                               const uint16_t* __restrict__ g,
                                                               uint16_t* __restrict__ y, int D,
@@ -52,10 +63,10 @@ __global__ void __launch_bounds__(kRowThreads) k_rmsnorm_rows(const uint16_t* __
   const size_t row = blockIdx.x;
   const int nch = D / 4;
   const uint16_t* xr = x + row * D;
-  float4 v[kMaxChunks];
+  float4 v[NC];
   float ss = 0.f;
 #pragma unroll
-  for (int i = 0; i < kMaxChunks; ++i) {
+  for (int i = 0; i < NC; ++i) {
     const int c = threadIdx.x + i * kRowThreads;
     if (c < nch) {
       v[i] = ld_bf16x4(xr + 4 * c);
@@ -65,7 +76,7 @@ __global__ void __launch_bounds__(kRowThreads) k_rmsnorm_rows(const uint16_t* __
   const float inv = inv_rms(block_sum_fixed(ss, red), D, eps);
   uint16_t* yr = y + row * D;
 #pragma unroll
-  for (int i = 0; i < kMaxChunks; ++i) {
+  for (int i = 0; i < NC; ++i) {
     const int c = threadIdx.x + i * kRowThreads;
     if (c < nch) {
       const float4 gg = ld_bf16x4(g + 4 * c);
@@ -77,13 +88,14 @@ __global__ void __launch_bounds__(kRowThreads) k_rmsnorm_rows(const uint16_t* __
 
 // Shared tail of the two epilogues: r (kept in registers) -> out_residual,
 // out_norm.
-__device__ __forceinline__ void norm_store(const float4 (&r)[kMaxChunks], float ss, float* red,
+template <int NC>
+__device__ __forceinline__ void norm_store(const float4 (&r)[NC], float ss, float* red,
                                            const uint16_t* __restrict__ g, uint16_t* on,
                                            int D, float eps) {
   const int nch = D / 4;
   const float inv = inv_rms(block_sum_fixed(ss, red), D, eps);
 #pragma unroll
-  for (int i = 0; i < kMaxChunks; ++i) {
+  for (int i = 0; i < NC; ++i) {
     const int c = threadIdx.x + i * kRowThreads;
     if (c < nch) {
       const float4 gg = ld_bf16x4(g + 4 * c);
@@ -93,6 +105,7 @@ __device__ __forceinline__ void norm_store(const float4 (&r)[kMaxChunks], float 
   }
 }
 
+template <int NC>
 __global__ void __launch_bounds__(kRowThreads) k_combine_norm(
     const float* __restrict__ y_slot, const float* __restrict__ topk_w,
     const float* __restrict__ y_shared, int k, int S, const uint16_t* __restrict__ residual,
@@ -104,10 +117,10 @@ __global__ void __launch_bounds__(kRowThreads) k_combine_norm(
   if (threadIdx.x < k) w_s[threadIdx.x] = topk_w[t * k + threadIdx.x];
   __syncthreads();
   const int nch = D / 4;
-  float4 r[kMaxChunks];
+  float4 r[NC];
   float ss = 0.f;
 #pragma unroll
-  for (int i = 0; i < kMaxChunks; ++i) {
+  for (int i = 0; i < NC; ++i) {
     const int c = threadIdx.x + i * kRowThreads;
     if (c < nch) {
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -130,6 +143,7 @@ __global__ void __launch_bounds__(kRowThreads) k_combine_norm(
   norm_store(r, ss, red, g, out_norm + t * D, D, eps);
 }
 
+template <int NC>
 __global__ void __launch_bounds__(kRowThreads) k_reduce_partials(
     const PartialPtrs parts, int P, const uint16_t* __restrict__ residual,
     const uint16_t* __restrict__ g, uint16_t* __restrict__ out_norm,
@@ -137,10 +151,10 @@ __global__ void __launch_bounds__(kRowThreads) k_reduce_partials(
   __shared__ float red[kRowThreads / 32 + 1];
   const size_t t = blockIdx.x;
   const int nch = D / 4;
-  float4 r[kMaxChunks];
+  float4 r[NC];
   float ss = 0.f;
 #pragma unroll
-  for (int i = 0; i < kMaxChunks; ++i) {
+  for (int i = 0; i < NC; ++i) {
     const int c = threadIdx.x + i * kRowThreads;
     if (c < nch) {
       const size_t off = t * D + 4 * c;
@@ -218,7 +232,13 @@ __global__ void k_wait_selftest(volatile int* flag, int* err, unsigned long long
 cudaError_t launch_rmsnorm_rows(const uint16_t* x, const uint16_t* g, uint16_t* y, int T, int D,
                                 float eps, int* err_to_clear, cudaStream_t s) {
   if (T <= 0) return cudaSuccess;
-  k_rmsnorm_rows<<<T, kRowThreads, 0, s>>>(x, g, y, D, eps, err_to_clear);
+  switch (chunks_for(D)) {
+    case 1: k_rmsnorm_rows<1><<<T, kRowThreads, 0, s>>>(x, g, y, D, eps, err_to_clear); break;
+    case 2: k_rmsnorm_rows<2><<<T, kRowThreads, 0, s>>>(x, g, y, D, eps, err_to_clear); break;
+    case 4: k_rmsnorm_rows<4><<<T, kRowThreads, 0, s>>>(x, g, y, D, eps, err_to_clear); break;
+    case 8: k_rmsnorm_rows<8><<<T, kRowThreads, 0, s>>>(x, g, y, D, eps, err_to_clear); break;
+    default: k_rmsnorm_rows<16><<<T, kRowThreads, 0, s>>>(x, g, y, D, eps, err_to_clear); break;
+  }
   return cudaGetLastError();
 }
 
@@ -227,8 +247,17 @@ cudaError_t launch_combine_norm(const float* y_slot, const float* topk_w, const 
                                 uint16_t* out_norm, uint16_t* out_residual, int T, int D,
                                 float eps, cudaStream_t s) {
   if (T <= 0) return cudaSuccess;
-  k_combine_norm<<<T, kRowThreads, 0, s>>>(y_slot, topk_w, y_shared, k, S, residual, g, out_norm,
-                                          out_residual, T, D, eps);
+#define MOE_COMBINE(NC)                                                                          \
+  k_combine_norm<NC><<<T, kRowThreads, 0, s>>>(y_slot, topk_w, y_shared, k, S, residual, g,     \
+                                              out_norm, out_residual, T, D, eps)
+  switch (chunks_for(D)) {
+    case 1: MOE_COMBINE(1); break;
+    case 2: MOE_COMBINE(2); break;
+    case 4: MOE_COMBINE(4); break;
+    case 8: MOE_COMBINE(8); break;
+    default: MOE_COMBINE(16); break;
+  }
+#undef MOE_COMBINE
   return cudaGetLastError();
 }
 
@@ -236,7 +265,16 @@ cudaError_t launch_reduce_partials(const PartialPtrs& parts, int P, const uint16
                                    const uint16_t* g, uint16_t* out_norm, uint16_t* out_residual,
                                    int T, int D, float eps, cudaStream_t s) {
   if (T <= 0) return cudaSuccess;
-  k_reduce_partials<<<T, kRowThreads, 0, s>>>(parts, P, residual, g, out_norm, out_residual, D, eps);
+#define MOE_REDUCE(NC) \
+  k_reduce_partials<NC><<<T, kRowThreads, 0, s>>>(parts, P, residual, g, out_norm, out_residual, D, eps)
+  switch (chunks_for(D)) {
+    case 1: MOE_REDUCE(1); break;
+    case 2: MOE_REDUCE(2); break;
+    case 4: MOE_REDUCE(4); break;
+    case 8: MOE_REDUCE(8); break;
+    default: MOE_REDUCE(16); break;
+  }
+#undef MOE_REDUCE
   return cudaGetLastError();
 }
 
