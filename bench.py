@@ -379,7 +379,10 @@ def main():
             "roofline": roof,
             "layer": {"tflops": round(layer_tflops, 1), "frac_of_tc_peak": round(layer_tflops / tc_peak, 4),
                       "flops_per_step": fl["total"], "distinct_experts": distinct,
-                      "algorithmic_bytes": W.layer_bytes(cfg, T, distinct)},
+                      "algorithmic_bytes": W.layer_bytes(cfg, T, distinct),
+                      "hbm_gbs": round(W.layer_bytes(cfg, T, distinct) / (ms_per_step / 1e3) / 1e9, 1),
+                      "frac_of_hbm": round(W.layer_bytes(cfg, T, distinct) / (ms_per_step / 1e3) / 1e9
+                                           / hbm_peak, 4)},
             "stage_us": stage_avg,
             "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},

@@ -55,6 +55,29 @@ __device__ __forceinline__ float block_sum_fixed(float v, float* smem_warps /*[k
   return smem_warps[kRowThreads / 32];
 }
 
+// The same fixed tree in fp64 (used for the input RMSNorm's sum of squares,
+// whose bf16 output feeds the router: with an fp64 sum the fp32 scale is the
+// correctly rounded value of 1/sqrt(mean + eps) whatever the summation order,
+// so the bf16 code of every element is decided from a well-defined fp32 scale).
+__device__ __forceinline__ double block_sum_fixed_f64(double v, double* smem_warps) {
+  v += __shfl_xor_sync(0xffffffffu, v, 16);
+  v += __shfl_xor_sync(0xffffffffu, v, 8);
+  v += __shfl_xor_sync(0xffffffffu, v, 4);
+  v += __shfl_xor_sync(0xffffffffu, v, 2);
+  v += __shfl_xor_sync(0xffffffffu, v, 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) smem_warps[warp] = v;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double s = smem_warps[0];
+#pragma unroll
+    for (int w = 1; w < kRowThreads / 32; ++w) s += smem_warps[w];
+    smem_warps[kRowThreads / 32] = s;
+  }
+  __syncthreads();
+  return smem_warps[kRowThreads / 32];
+}
+
 // --------------------------------------------------------------- mbarrier
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

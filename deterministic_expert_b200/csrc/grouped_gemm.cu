@@ -187,7 +187,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
     // own shared buffer, and stores it back so that every store instruction
     // writes whole 128-byte row segments (8 lanes per row, 4 rows at a time).
     const int q = warp & 3;           // TMEM lane quarter this warp may access
-    const int row = q * 32 + lane;    // accumulator row = TMEM lane
     uint32_t* stage_w = reinterpret_cast<uint32_t*>(epi) + (warp - 2) * (32 * kEpiStride);
     const int sr = lane >> 3, sc = lane & 7;  // store phase: row offset 0..3, 16-byte column 0..7
     int acc = 0;

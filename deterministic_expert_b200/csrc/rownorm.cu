@@ -6,8 +6,10 @@
 // parity post (Chinese translation), Trap 2, says must not change with the
 // launch shape.  Nothing here depends on T.
 //
-//   rmsnorm_rows     xn = bf16(x * rsqrt(mean(x^2) + eps) * g)
-//                    (linux.do post on MoE variants, "RMSNorm before up-projection")
+//   rmsnorm_rows     xn = bf16((x * s) * g), s = fp32(1 / sqrt(mean(x^2) + eps)) from an
+//                    fp64 sum of squares (same fixed tree) so that the bf16 code of
+//                    xn, which decides the routing, is fixed by a well-defined fp32
+//                    scale (linux.do post on MoE variants, "RMSNorm before up-projection")
 //   combine_norm     acc = sum_j w_j y_j (slot order) + sum_s y_s; r = acc + residual;
 //                    out_residual = bf16(r); out_norm = bf16(RMSNorm(r) * g)
 //                    (Fireworks post, Trap 3 unfused chain and case-study "standard path":
@@ -58,22 +60,29 @@ __global__ void __launch_bounds__(kRowThreads) k_rmsnorm_rows(const uint16_t* __
                                                               const uint16_t* __restrict__ g,
                                                               uint16_t* __restrict__ y, int D,
                                                               float eps, int* err) {
-  __shared__ float red[kRowThreads / 32 + 1];
+  __shared__ double red[kRowThreads / 32 + 1];
   if (err != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *err = kDevOk;
   const size_t row = blockIdx.x;
   const int nch = D / 4;
   const uint16_t* xr = x + row * D;
   float4 v[NC];
-  float ss = 0.f;
+  double ss = 0.0;
 #pragma unroll
   for (int i = 0; i < NC; ++i) {
     const int c = threadIdx.x + i * kRowThreads;
     if (c < nch) {
       v[i] = ld_bf16x4(xr + 4 * c);
-      ss = sumsq4(ss, v[i]);
+      ss = fma(static_cast<double>(v[i].x), static_cast<double>(v[i].x), ss);
+      ss = fma(static_cast<double>(v[i].y), static_cast<double>(v[i].y), ss);
+      ss = fma(static_cast<double>(v[i].z), static_cast<double>(v[i].z), ss);
+      ss = fma(static_cast<double>(v[i].w), static_cast<double>(v[i].w), ss);
     }
   }
-  const float inv = inv_rms(block_sum_fixed(ss, red), D, eps);
+  // The squares of bf16 values are exact in fp64 and the fp64 sum is exact to
+  // ~2^-52, so the scale below is the correctly rounded fp32 value of
+  // 1 / sqrt(mean(x^2) + eps); xn = bf16((x * scale) * g) in fp32.
+  const double ms = block_sum_fixed_f64(ss, red) / static_cast<double>(D);
+  const float inv = static_cast<float>(1.0 / sqrt(ms + static_cast<double>(eps)));
   uint16_t* yr = y + row * D;
 #pragma unroll
   for (int i = 0; i < NC; ++i) {

@@ -40,9 +40,11 @@ The layer, in order:
 Precision.  Every floating-point step runs in fp64, on the bf16-rounded values
 the GPU path reads (x, residual, weights, xn between steps 1 and 2/6, h between
 the two expert matmuls).  Rounding to bf16 is done directly from fp64 (round to
-nearest, ties to even), never through fp32.  The one exception is step 9: the
-pages fix its precision (both all-reduce orders accumulate in FP32, [FW] Trap
-1), so the partial sums are emulated in IEEE fp32, left to right.
+nearest, ties to even), never through fp32.  Two exceptions: step 9, whose
+precision the pages fix (both all-reduce orders accumulate in FP32, [FW] Trap
+1), is emulated in IEEE fp32 left to right; and the bf16 code of xn, which
+decides the routing (an integer), is decided in the kernel's precision
+(``rmsnorm_bf16_code``).
 
 Readings of points the pages leave open (each is also listed in the design
 notes): epsilon inside the square root; gains g_in = g_out = 1 unless given;
@@ -104,6 +106,23 @@ def rmsnorm(x, g, eps: float) -> np.ndarray:
     x = np.asarray(x, dtype=np.float64)
     ms = np.mean(x * x, axis=-1, keepdims=True)
     return np.asarray(g, dtype=np.float64) * (x / np.sqrt(ms + eps))
+
+
+def rmsnorm_bf16_code(x, g, eps: float) -> np.ndarray:
+    """xn = bf16(RMSNorm(x) * g), with the bf16 code decided in the kernel's
+    precision.  The code of xn decides the routing (an integer), so both
+    sides decide it the same way: the mean of squares in fp64 (exact to
+    ~2^-52 for bf16 inputs), the scale s = 1/sqrt(mean + eps) rounded once to
+    fp32, then y = (x * s) * g with two fp32 products (round to nearest), then
+    round to nearest even bf16.  eps is the fp32 value the kernel receives.
+    Away from bf16 rounding boundaries this equals round_bf16(rmsnorm(...)),
+    the plain fp64 definition ([LD] "RMSNorm before up-projection")."""
+    x = np.asarray(x, np.float64)
+    ms = np.mean(x * x, axis=-1, keepdims=True)
+    s = (1.0 / np.sqrt(ms + float(np.float32(eps)))).astype(np.float32)
+    y = np.multiply(x.astype(np.float32), s, dtype=np.float32)
+    y = np.multiply(y, np.asarray(g, np.float64).astype(np.float32), dtype=np.float32)
+    return round_bf16(y.astype(np.float64))
 
 
 # ------------------------------------------------------- 2-3. router, top-k
@@ -351,7 +370,7 @@ def moe_layer(cfg, W, x, residual, token_ids=None, rows=None) -> dict:
     x = np.asarray(x, np.float64)
     T = x.shape[0]
     rows = np.arange(T) if rows is None else np.asarray(rows, np.int64)
-    xn = round_bf16(rmsnorm(x, W.g_in, cfg.eps))
+    xn = rmsnorm_bf16_code(x, W.g_in, cfg.eps)
     logits = None
     if cfg.router != ROUTER_HASH:
         logits = router_logits(xn, W.w_router)
@@ -389,7 +408,7 @@ def moe_layer_dense_masked(cfg, W, x, residual, token_ids=None) -> dict:
     chosen) and sum over all experts.  Mathematically equal to ``moe_layer``."""
     x = np.asarray(x, np.float64)
     T = x.shape[0]
-    xn = round_bf16(rmsnorm(x, W.g_in, cfg.eps))
+    xn = rmsnorm_bf16_code(x, W.g_in, cfg.eps)
     logits = None if cfg.router == ROUTER_HASH else router_logits(xn, W.w_router)
     idx, w, _ = route(cfg, logits, W.router_bias, token_ids)
     mask = np.zeros((T, cfg.E))

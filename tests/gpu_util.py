@@ -82,23 +82,42 @@ def check_outputs(out, ref, rows=None, same_rows=None):
     return stats
 
 
-def check_routing(out, ref):
-    """Indices must equal the oracle's except on near-tie tokens (margin below
-    1e-5 in the oracle's key space); a near-tie token must still have picked a
-    valid top-k under the oracle's keys (its keys within the margin of the
-    k-th).  Returns the boolean mask of rows that route exactly like the oracle."""
+def routing_consistent(gi, keys, tol=NEAR_TIE):
+    """Is ``gi`` (one token's GPU slots) a top-k of ``keys`` (the oracle's fp64
+    keys) up to near ties?  Every chosen expert must be within ``tol`` of the
+    oracle's k-th key, every expert left out must not beat the chosen ones by
+    more than ``tol``, and consecutive slots must descend up to ``tol``."""
+    k = len(gi)
+    if len(set(gi.tolist())) != k:
+        return False
+    kth = np.sort(keys)[-k]
+    chosen = keys[gi]
+    if np.any(chosen < kth - tol):
+        return False
+    rest = np.delete(keys, gi)
+    if rest.size and rest.max() > chosen.min() + tol:
+        return False
+    return bool(np.all(chosen[:-1] >= chosen[1:] - tol))
+
+
+def check_routing(out, ref, report=None):
+    """Top-k indices must equal the oracle's (set and slot order) except on
+    near-tie tokens: where the oracle's keys of the experts that differ lie
+    within 1e-5 (at the k-th/(k+1)-th boundary, or between adjacent slots).
+    Those tokens must still hold a valid top-k of the oracle's keys up to
+    1e-5; they are counted (``report``) and left out of the value comparison.
+    Returns the boolean mask of rows that route exactly like the oracle."""
     gi = out["idx"].cpu().numpy()
     same = np.all(gi == ref["idx"], axis=1)
-    if ref["margin"] is None:  # hash routing: exact
+    if ref["keys"] is None:  # hash routing: exact
         assert np.all(same)
         return same
-    bad = ~same & ~(ref["margin"] < NEAR_TIE)
-    assert not np.any(bad), f"routing differs on tokens {np.nonzero(bad)[0][:10]} (margins " \
-                            f"{ref['margin'][bad][:10]})"
-    for t in np.nonzero(~same)[0]:
-        keys = ref["keys"][t]
-        kth = np.sort(keys)[-cfg_k(ref)]
-        assert np.all(keys[gi[t]] >= kth - NEAR_TIE), t
+    bad = [t for t in np.nonzero(~same)[0] if not routing_consistent(gi[t], ref["keys"][t])]
+    assert not bad, f"routing differs beyond near ties on tokens {bad[:10]}"
+    if report is not None:
+        report["near_tie_tokens"] = int((~same).sum())
+    if (~same).any():
+        print(f"near-tie tokens (routing differs within 1e-5 of the oracle's keys): {int((~same).sum())}")
     return same
 
 

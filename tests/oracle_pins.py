@@ -86,6 +86,28 @@ def pin_rmsnorm_scale_invariance(O):
     assert np.allclose(np.sqrt(np.mean(a * a, axis=-1)), 1.0, rtol=1e-13)
 
 
+def pin_rmsnorm_bf16_code(O):
+    # By hand: [3,4], eps 1e-6: 3/sqrt(12.5) = 0.848528 -> 434 * 2^-9; 4/sqrt(12.5) = 1.131371 -> 145 * 2^-7.
+    assert np.array_equal(O.rmsnorm_bf16_code(np.array([[3.0, 4.0]]), np.ones(2), 1e-6)[0],
+                          [434 * 2.0 ** -9, 145 * 2.0 ** -7])
+    # eps = 1 sits inside the root: 3/sqrt(13.5) = 0.816497 -> 418 * 2^-9; 4/sqrt(13.5) = 1.088662 -> 139 * 2^-7.
+    assert np.array_equal(O.rmsnorm_bf16_code(np.array([[3.0, 4.0]]), np.ones(2), 1.0)[0],
+                          [418 * 2.0 ** -9, 139 * 2.0 ** -7])
+    # Gains after the scale: 2 * 0.848528 = 1.697056 -> 217 * 2^-7; -0.5 * 1.131371 = -0.565685 -> -290 * 2^-9.
+    assert np.array_equal(O.rmsnorm_bf16_code(np.array([[3.0, 4.0]]), np.array([2.0, -0.5]), 0.0)[0],
+                          [217 * 2.0 ** -7, -290 * 2.0 ** -9])
+    # Random rows: equal to the plain fp64 definition rounded once, except for
+    # rare values next to a bf16 rounding boundary, which differ by one bf16 step.
+    rng = np.random.default_rng(11)
+    x = O.round_bf16(rng.standard_normal((64, 2048)))
+    g = O.round_bf16(1 + 0.1 * rng.standard_normal(2048))
+    a = O.rmsnorm_bf16_code(x, g, 1e-6)
+    b = O.round_bf16(O.rmsnorm(x, g, float(np.float32(1e-6))))
+    d = a != b
+    assert d.mean() < 1e-3
+    assert np.all(np.abs(a[d] - b[d]) <= np.abs(b[d]) * 2.0 ** -7 * 1.0001)
+
+
 # ------------------------------------------------------------------ SwiGLU
 def pin_swish_example(O):
     g = golden("swish_worked_example.json")

@@ -17,6 +17,10 @@ MUTATIONS = {
     "eps_outside_sqrt": ("x / np.sqrt(ms + eps)", "x / (np.sqrt(ms) + eps)"),
     "gain_dropped": ("return np.asarray(g, dtype=np.float64) * (x / np.sqrt(ms + eps))",
                      "return (x / np.sqrt(ms + eps))"),
+    "code_eps_outside_sqrt": ("s = (1.0 / np.sqrt(ms + float(np.float32(eps)))).astype(np.float32)",
+                              "s = (1.0 / (np.sqrt(ms) + float(np.float32(eps)))).astype(np.float32)"),
+    "code_gain_dropped": ("    y = np.multiply(y, np.asarray(g, np.float64).astype(np.float32), dtype=np.float32)\n",
+                          ""),
     "double_rounding_via_fp32": ("a = np.asarray(a, dtype=np.float64)\n    _, e",
                                  "a = np.asarray(a, dtype=np.float64).astype(np.float32).astype(np.float64)\n    _, e"),
     "topk_ascending": ("neg = np.where(np.isnan(keys), np.inf, -keys)",
