@@ -18,8 +18,9 @@
 //   warp 0   one thread issues TMA loads of A and B tiles into a 4-stage ring
 //   warp 1   allocates 512 TMEM columns; one thread issues tcgen05.mma and
 //            commits stage releases / accumulator-ready signals to mbarriers
-//   warps 2-5 epilogue: tcgen05.ld the accumulator (one TMEM lane = one row per
-//            thread), apply SwiGLU or scatter, store to global memory
+//   warps 2-9 epilogue: tcgen05.ld the accumulator (one TMEM lane = one row per
+//            thread; two warps per lane quarter split the columns), apply SwiGLU
+//            or scatter, store to global memory
 // Two accumulator buffers let the epilogue of tile i overlap the MMAs of i+1.
 // Every mbarrier wait is bounded in time; on time-out the CTA records an error
 // word, drains its own TMA copies and MMAs (bounded), frees TMEM and exits.
@@ -63,10 +64,12 @@ __device__ __forceinline__ void decode_tile(const GemmArgs& a, int t, Tile& ti) 
   ti.m = local - ti.n * mt;
 }
 
+// SiLU(min(g, c_g)) * clamp(u, -c_u, c_u) in fp32 with the fast exponential
+// and division (deterministic; about 2 ulp, far below the bf16 rounding of h).
 __device__ __forceinline__ float silu_clamped_product(float g, float u, float cg, float cu) {
   g = fminf(g, cg);
   u = fminf(fmaxf(u, -cu), cu);
-  return g / (1.0f + __expf(-g)) * u;
+  return __fdividef(g, 1.0f + __expf(-g)) * u;
 }
 
 template <int MODE>
@@ -82,14 +85,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
   uint64_t* tfull = bars + 2 * kStages;
   uint64_t* tempty = tfull + 2;
   uint64_t* tdone = tempty + 2;
-  uint8_t* epi = reinterpret_cast<uint8_t*>(bars) + 256;  // 4 warps x 32 x kEpiStride words
+  uint8_t* epi = reinterpret_cast<uint8_t*>(bars) + 256;  // kEpiWarps x kEpiBytes
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-    for (int b = 0; b < 2; ++b) { mbar_init(&tfull[b], 1); mbar_init(&tempty[b], 4); }
+    for (int b = 0; b < 2; ++b) { mbar_init(&tfull[b], 1); mbar_init(&tempty[b], kEpiWarps); }
     mbar_init(tdone, 1);
     abort_flag = 0;
     fence_barrier_init();
@@ -143,7 +146,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
   } else if (warp == 1) {
     // ------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(kBM, BN);
+      // Gate/up: the gate tile (BN rows) and the up tile (BN rows) sit back to
+      // back in shared memory, so one N = 2*BN MMA reads A once and writes the
+      // gate accumulator to columns [0, BN) and the up accumulator to [BN, 2*BN).
+      const uint32_t idesc = idesc_bf16_f32(kBM, MODE == kGateUp ? 2 * BN : BN);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -166,8 +172,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
             const uint64_t ad = sw128_kmajor_desc(a_addr + kk * 32);
             const uint32_t accum = (kb | kk) != 0 ? 1u : 0u;
             umma_bf16(d0, ad, sw128_kmajor_desc(b_addr + kk * 32), idesc, accum);
-            if (MODE == kGateUp)
-              umma_bf16(d0 + BN, ad, sw128_kmajor_desc(b_addr + bytesB + kk * 32), idesc, accum);
           }
           umma_commit(&empty[stage]);
           if (++stage == kStages) { stage = 0; phase ^= 1u; }
@@ -182,13 +186,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
     }
   } else {
     // --------------------------------------------------------- epilogue
-    // Each warp owns 32 accumulator rows (one TMEM lane quarter).  It reads 32
-    // columns per tcgen05.ld (lane i = row i), stages the 32 x 32 block in its
-    // own shared buffer, and stores it back so that every store instruction
-    // writes whole 128-byte row segments (8 lanes per row, 4 rows at a time).
-    const int q = warp & 3;           // TMEM lane quarter this warp may access
-    uint32_t* stage_w = reinterpret_cast<uint32_t*>(epi) + (warp - 2) * (32 * kEpiStride);
-    const int sr = lane >> 3, sc = lane & 7;  // store phase: row offset 0..3, 16-byte column 0..7
+    // Two warps per TMEM lane quarter (32 accumulator rows each) split the
+    // tile's columns: half 0 takes blocks 0, 2, 4, ..., half 1 blocks 1, 3, ...
+    // (64 columns per block for gate/up, 32 otherwise).  Each block is read with
+    // tcgen05.ld (lane i = row i), staged in the warp's own 4 KB buffer, and
+    // stored back so that every store instruction writes whole 128-byte row
+    // segments (8 lanes per row, 4 rows at a time).  The buffer holds 32 rows
+    // of 128 bytes; 16-byte chunk m of row r sits at chunk m ^ (r & 7), so both
+    // the row-wise writes and the column-wise reads are free of bank conflicts.
+    const int q = warp & 3;                  // TMEM lane quarter this warp may access
+    const int half = (warp - 2) >> 2;        // which column blocks
+    uint8_t* stage_w = epi + (warp - 2) * kEpiBytes;
+    const int sr = lane >> 3, sc = lane & 7; // store phase: row offset 0..3, 16-byte chunk 0..7
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x) {
@@ -202,16 +211,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
       const int grow0 = ti.m * kBM + q * 32;   // first group row of this warp's block
       const int nvalid = max(0, min(32, ti.rows - grow0));
       if (MODE == kGateUp) {
-        // 64 output columns (128 bytes of bf16) per staged block.
         const int orow0 = (ti.kind == 0 ? ti.a_row0 : ti.idx * a.shared_out_stride) + grow0;
         uint8_t* out0 = reinterpret_cast<uint8_t*>(static_cast<uint16_t*>(a.out[ti.kind]) + ti.n * BN);
         const size_t ld_bytes = static_cast<size_t>(a.ld_out[ti.kind]) * 2;
-        for (int c = 0; c < BN; c += 64) {
+        for (int c = 64 * half; c < BN; c += 128) {
 #pragma unroll
-          for (int half = 0; half < 2; ++half) {
+          for (int hb = 0; hb < 2; ++hb) {
             uint32_t g[32], u[32];
-            tmem_ld32(tb + c + 32 * half, g);
-            tmem_ld32(tb + BN + c + 32 * half, u);
+            tmem_ld32(tb + c + 32 * hb, g);
+            tmem_ld32(tb + BN + c + 32 * hb, u);
             tmem_ld_wait();
             uint32_t p[16];
 #pragma unroll
@@ -221,43 +229,47 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
                                        a.gate_clamp, a.up_clamp),
                   silu_clamped_product(__uint_as_float(g[2 * i + 1]), __uint_as_float(u[2 * i + 1]),
                                        a.gate_clamp, a.up_clamp));
-            uint4* dst = reinterpret_cast<uint4*>(stage_w + lane * kEpiStride + 16 * half);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) dst[i] = make_uint4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
+            for (int i = 0; i < 4; ++i) {
+              const int m = 4 * hb + i;
+              *reinterpret_cast<uint4*>(stage_w + lane * 128 + ((m ^ (lane & 7)) << 4)) =
+                  make_uint4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
+            }
           }
           __syncwarp();
 #pragma unroll
           for (int s8 = 0; s8 < 8; ++s8) {
             const int r = 4 * s8 + sr;
             if (r < nvalid) {
-              const uint4 v = *reinterpret_cast<const uint4*>(stage_w + r * kEpiStride + 4 * sc);
+              const uint4 v = *reinterpret_cast<const uint4*>(stage_w + r * 128 + ((sc ^ (r & 7)) << 4));
               *reinterpret_cast<uint4*>(out0 + static_cast<size_t>(orow0 + r) * ld_bytes + c * 2 + 16 * sc) = v;
             }
           }
           __syncwarp();
         }
       } else {
-        // fp32 output, 32 columns (128 bytes) per staged block.
+        // fp32 output, 32 columns (128 bytes) per block.
         const bool scatter = (MODE == kDown && ti.kind == 0);
         const int my_dest = (scatter && lane < nvalid) ? a.dest_row[ti.a_row0 + grow0 + lane] : 0;
         const int orow0 = (ti.kind == 0 ? ti.a_row0 : ti.idx * a.shared_out_stride) + grow0;
         float* out0 = static_cast<float*>(a.out[ti.kind]) + ti.n * BN;
         const size_t ld = static_cast<size_t>(a.ld_out[ti.kind]);
-        for (int c = 0; c < BN; c += 32) {
+        for (int c = 32 * half; c < BN; c += 64) {
           uint32_t v[32];
           tmem_ld32(tb + c, v);
           tmem_ld_wait();
           if (BN - c >= 32) {
-            uint4* dst = reinterpret_cast<uint4*>(stage_w + lane * kEpiStride);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) dst[i] = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+            for (int m = 0; m < 8; ++m)
+              *reinterpret_cast<uint4*>(stage_w + lane * 128 + ((m ^ (lane & 7)) << 4)) =
+                  make_uint4(v[4 * m], v[4 * m + 1], v[4 * m + 2], v[4 * m + 3]);
             __syncwarp();
 #pragma unroll
             for (int s8 = 0; s8 < 8; ++s8) {
               const int r = 4 * s8 + sr;
               const int drow = __shfl_sync(0xffffffffu, my_dest, r);
               if (r < nvalid) {
-                const uint4 val = *reinterpret_cast<const uint4*>(stage_w + r * kEpiStride + 4 * sc);
+                const uint4 val = *reinterpret_cast<const uint4*>(stage_w + r * 128 + ((sc ^ (r & 7)) << 4));
                 const size_t orow = scatter ? static_cast<size_t>(drow) : static_cast<size_t>(orow0 + r);
                 *reinterpret_cast<uint4*>(out0 + orow * ld + c + 4 * sc) = val;
               }

@@ -18,11 +18,12 @@ namespace moe {
 constexpr int kBM = 128;
 constexpr int kBK = 64;
 constexpr int kStages = 4;
-constexpr int kGemmThreads = 192;  // warp 0: TMA, warp 1: MMA, warps 2-5: epilogue
+constexpr int kEpiWarps = 8;       // two per TMEM lane quarter, splitting the columns
+constexpr int kGemmThreads = 64 + 32 * kEpiWarps;  // warp 0: TMA, warp 1: MMA, warps 2-9: epilogue
 constexpr int kSmemA = kBM * kBK * 2;
 constexpr int kSmemBMax = 256 * kBK * 2;
-constexpr int kEpiStride = 36;  // words per staged epilogue row (128 B + 16 B pad)
-constexpr int kGemmSmem = 1024 + kStages * (kSmemA + kSmemBMax) + 256 + 4 * 32 * kEpiStride * 4;
+constexpr int kEpiBytes = 32 * 128;  // per epilogue warp: 32 rows x 128 B, XOR-swizzled
+constexpr int kGemmSmem = 1024 + kStages * (kSmemA + kSmemBMax) + 256 + kEpiWarps * kEpiBytes;
 
 enum GemmMode : int { kGateUp = 0, kDown = 1, kRouter = 2 };
 
