@@ -49,12 +49,12 @@ __global__ void __launch_bounds__(256) k_dispatch_scan(const DispatchArgs a) {
     for (int q = 0; q < a.E; ++q) { offs[q] = run; run += total[q]; }
     offs[a.E] = run;
     // Tile lists: routed groups first (experts in index order), then shared.
-    const int mt_shared = (a.T + kBM - 1) / kBM;
+    const int mt_shared = (a.T + a.tile_m - 1) / a.tile_m;
     int gu = 0, dn = 0;
     for (int q = 0; q < a.E; ++q) {
       a.tiles_gu[q] = gu;
       a.tiles_dn[q] = dn;
-      const int mt = (total[q] + kBM - 1) / kBM;
+      const int mt = (total[q] + a.tile_m - 1) / a.tile_m;
       gu += mt * a.gu_ntiles_routed;
       dn += mt * a.dn_ntiles;
     }

@@ -10,20 +10,30 @@
 // the whole K of a dot product in one accumulation instead of summing split
 // partial results).  Every output element is one TMEM accumulator that walks
 // all of K in 64-wide steps, 16 per MMA, in the same order for every tile;
-// the tile shape (128 x BN) is fixed per layer shape and never chosen from T;
-// rows of a tile never mix (a row's result depends only on its own A row), so
-// padding rows and rows of a neighbouring group are computed and discarded.
+// the tile shape is fixed per layer shape and never chosen from T; rows of a
+// tile never mix (a row's result depends only on its own A row), so padding
+// rows and rows of a neighbouring group are computed and discarded.
 //
-// Structure (one CTA per SM, persistent over a device-built tile list):
-//   warp 0   one thread issues TMA loads of A and B tiles into a 4-stage ring
-//   warp 1   allocates 512 TMEM columns; one thread issues tcgen05.mma and
-//            commits stage releases / accumulator-ready signals to mbarriers
+// Two variants, persistent over a device-built tile list:
+//   CG = 1  one CTA per 128-row tile (the router GEMM).
+//   CG = 2  a CTA pair (cluster of 2) per 256-row tile with cta_group::2 MMAs
+//           (the expert GEMMs): each CTA loads its own 128 A rows and half of
+//           the B tile (gate/up: the even CTA the gate rows, the odd CTA the up
+//           rows; down: one half of the BN output columns each), so each SM's
+//           shared memory receives and feeds half the B bytes of a 1-CTA tile.
+//           The even CTA issues the MMAs; its commits reach both CTAs.
+// Roles in each CTA:
+//   warp 0    one thread issues the TMA loads of its CTA into a stage ring
+//   warp 1    allocates 512 TMEM columns; in the (even) issuing CTA one thread
+//             issues tcgen05.mma and commits stage releases / accumulator-ready
 //   warps 2-9 epilogue: tcgen05.ld the accumulator (one TMEM lane = one row per
-//            thread; two warps per lane quarter split the columns), apply SwiGLU
-//            or scatter, store to global memory
+//             thread; two warps per lane quarter split the columns), apply
+//             SwiGLU or scatter, store to global memory
 // Two accumulator buffers let the epilogue of tile i overlap the MMAs of i+1.
 // Every mbarrier wait is bounded in time; on time-out the CTA records an error
 // word, drains its own TMA copies and MMAs (bounded), frees TMEM and exits.
+#include <algorithm>
+
 #include "common.cuh"
 #include "moe_internal.h"
 
@@ -33,6 +43,14 @@ namespace {
 constexpr uint32_t kTmemCols = 512;
 constexpr unsigned long long kDrainNs = 200ull * 1000 * 1000;  // 200 ms
 
+template <int CG>
+struct Cfg {
+  static constexpr int kTileM = 128 * CG;                                 // rows per tile (pair)
+  static constexpr int kSmemB = CG == 1 ? 256 * kBK * 2 : 128 * kBK * 2;  // B bytes per CTA stage
+  static constexpr int kStage = kSmemA + kSmemB;
+  static constexpr int kStagesN = (kStages * (kSmemA + kSmemBMax)) / kStage;  // 4 or 6
+};
+
 struct Tile {
   int kind;   // 0 routed, 1 shared
   int idx;    // expert index within its kind
@@ -41,6 +59,7 @@ struct Tile {
   int m, n;   // tile coordinates within the group
 };
 
+template <int CG>
 __device__ __forceinline__ void decode_tile(const GemmArgs& a, int t, Tile& ti) {
   if (a.tile_start == nullptr) {
     ti.kind = 0; ti.idx = 0; ti.rows = a.T; ti.a_row0 = 0; ti.m = t; ti.n = 0;
@@ -59,7 +78,7 @@ __device__ __forceinline__ void decode_tile(const GemmArgs& a, int t, Tile& ti) 
   } else {
     ti.kind = 1; ti.idx = lo - a.E; ti.rows = a.T; ti.a_row0 = ti.idx * a.shared_a_stride;
   }
-  const int mt = (ti.rows + kBM - 1) / kBM;
+  const int mt = (ti.rows + Cfg<CG>::kTileM - 1) / Cfg<CG>::kTileM;
   ti.n = local / mt;
   ti.m = local - ti.n * mt;
 }
@@ -72,17 +91,19 @@ __device__ __forceinline__ float silu_clamped_product(float g, float u, float cg
   return __fdividef(g, 1.0f + __expf(-g)) * u;
 }
 
-template <int MODE>
+template <int MODE, int CG>
 __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_constant__ GemmArgs a) {
+  using C = Cfg<CG>;
+  constexpr int S = C::kStagesN;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint8_t* sA = smem;
-  uint8_t* sB = smem + kStages * kSmemA;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + kStages * kSmemBMax);
+  uint8_t* sA = smem;                              // S x kSmemA
+  uint8_t* sB = smem + S * kSmemA;                 // S x kSmemB
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * (kSmemA + kSmemBMax));
   uint64_t* full = bars;
-  uint64_t* empty = bars + kStages;
-  uint64_t* tfull = bars + 2 * kStages;
+  uint64_t* empty = bars + S;
+  uint64_t* tfull = bars + 2 * S;
   uint64_t* tempty = tfull + 2;
   uint64_t* tdone = tempty + 2;
   uint8_t* epi = reinterpret_cast<uint8_t*>(bars) + 256;  // kEpiWarps x kEpiBytes
@@ -90,74 +111,97 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
   __shared__ int abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = CG == 2 ? cluster_ctarank() : 0;   // 0 = the MMA-issuing CTA
+  const bool leader = rank == 0;
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-    for (int b = 0; b < 2; ++b) { mbar_init(&tfull[b], 1); mbar_init(&tempty[b], kEpiWarps); }
+    for (int s = 0; s < S; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    for (int b = 0; b < 2; ++b) { mbar_init(&tfull[b], 1); mbar_init(&tempty[b], CG * kEpiWarps); }
     mbar_init(tdone, 1);
     abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 1) tmem_alloc(&tmem_slot, kTmemCols);
+  if (warp == 1) {
+    if (CG == 2) tmem_alloc_pair(&tmem_slot, kTmemCols);
+    else tmem_alloc(&tmem_slot, kTmemCols);
+  }
   tc_fence_before();
-  __syncthreads();
+  if (CG == 2) cluster_sync(); else __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = tmem_slot;
   volatile int* abort = &abort_flag;
 
+  const int cluster_id = blockIdx.x / CG, n_clusters = gridDim.x / CG;
   const int total = (a.tile_start == nullptr) ? a.router_tiles : a.tile_start[a.G];
-  const int BN = a.BN;
-  const uint32_t bytesB = static_cast<uint32_t>(BN) * kBK * 2;
-  constexpr int kNB = (MODE == kGateUp) ? 2 : 1;
-  const uint32_t stage_bytes = kSmemA + bytesB * kNB;
-  const uint32_t acc_stride = static_cast<uint32_t>(BN * kNB);  // TMEM columns per buffer
+  const int BN = a.BN;                                    // output columns per tile (per matrix)
+  const int n_mma = MODE == kGateUp ? 2 * BN : BN;        // N of one MMA
+  // B rows each CTA loads per stage (per matrix for gate/up).
+  const uint32_t b_rows = static_cast<uint32_t>(MODE == kGateUp ? BN : BN / CG);
+  const uint32_t stage_bytes = kSmemA + b_rows * kBK * 2 * (MODE == kGateUp && CG == 1 ? 2 : 1);
+  const uint32_t acc_stride = static_cast<uint32_t>(n_mma);  // TMEM columns per buffer
+  // Barriers the pair shares live in the even CTA.
+  const uint32_t full0 = CG == 2 ? mapa_shared(full, 0) : 0;
+  const uint32_t tempty0 = CG == 2 ? mapa_shared(tempty, 0) : 0;
 
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
-      int issued[kStages];
-      for (int s = 0; s < kStages; ++s) issued[s] = -1;
+      int issued[S];
+      for (int s = 0; s < S; ++s) issued[s] = -1;
       bool ok = true;
-      for (int t = blockIdx.x; ok && t < total; t += gridDim.x) {
+      for (int t = cluster_id; ok && t < total; t += n_clusters) {
         Tile ti;
-        decode_tile(a, t, ti);
+        decode_tile<CG>(a, t, ti);
         const int nkb = a.k_kind[ti.kind] / kBK;
-        const int a_y = ti.a_row0 + ti.m * kBM;
-        const int b_y = ti.idx * a.n_kind[ti.kind] + ti.n * BN;
+        const int a_y = ti.a_row0 + ti.m * C::kTileM + static_cast<int>(rank) * 128;
+        int b_y = ti.idx * a.n_kind[ti.kind] + ti.n * BN;
+        const CUtensorMap* bmap = &a.mapB[ti.kind * 2];
+        if (CG == 2) {
+          if (MODE == kGateUp) bmap += rank;                          // gate | up
+          else b_y += static_cast<int>(rank) * (BN / 2);             // lower | upper half
+        }
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort, a.err, a.timeout_ns)) { ok = false; break; }
-          mbar_arrive_expect_tx(&full[stage], stage_bytes);
-          tma_load_2d(sA + stage * kSmemA, &a.mapA[ti.kind], kb * kBK, a_y, &full[stage]);
-          uint8_t* b0 = sB + stage * kSmemBMax;
-          tma_load_2d(b0, &a.mapB[ti.kind * 2], kb * kBK, b_y, &full[stage]);
-          if (MODE == kGateUp)
-            tma_load_2d(b0 + bytesB, &a.mapB[ti.kind * 2 + 1], kb * kBK, b_y, &full[stage]);
+          uint8_t* b0 = sB + stage * C::kSmemB;
+          if (CG == 1) {
+            mbar_arrive_expect_tx(&full[stage], stage_bytes);
+            tma_load_2d(sA + stage * kSmemA, &a.mapA[ti.kind], kb * kBK, a_y, &full[stage]);
+            tma_load_2d(b0, bmap, kb * kBK, b_y, &full[stage]);
+            if (MODE == kGateUp)
+              tma_load_2d(b0 + b_rows * kBK * 2, bmap + 1, kb * kBK, b_y, &full[stage]);
+          } else {
+            // The even CTA expects the bytes of both CTAs on its barrier.
+            if (leader) mbar_arrive_expect_tx(&full[stage], 2 * stage_bytes);
+            tma_load_2d_pair(sA + stage * kSmemA, &a.mapA[ti.kind], kb * kBK, a_y, full0 + 8 * stage);
+            tma_load_2d_pair(b0, bmap, kb * kBK, b_y, full0 + 8 * stage);
+          }
           issued[stage] = static_cast<int>(phase);
-          if (++stage == kStages) { stage = 0; phase ^= 1u; }
+          if (++stage == S) { stage = 0; phase ^= 1u; }
         }
       }
-      if (!ok) {
+      if (!ok && (CG == 1 || leader)) {
         // Let the copies already in flight land before the CTA goes away.
-        for (int s = 0; s < kStages; ++s)
+        for (int s = 0; s < S; ++s)
           if (issued[s] >= 0) mbar_wait_drain(&full[s], static_cast<uint32_t>(issued[s]), kDrainNs);
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      // Gate/up: the gate tile (BN rows) and the up tile (BN rows) sit back to
-      // back in shared memory, so one N = 2*BN MMA reads A once and writes the
-      // gate accumulator to columns [0, BN) and the up accumulator to [BN, 2*BN).
-      const uint32_t idesc = idesc_bf16_f32(kBM, MODE == kGateUp ? 2 * BN : BN);
+    if (lane == 0 && leader) {
+      // Gate/up: the gate tile and the up tile sit back to back in shared
+      // memory (CG = 1) or in the two CTAs of the pair (CG = 2), so one
+      // N = 2*BN MMA reads A once and writes the gate accumulator to columns
+      // [0, BN) and the up accumulator to [BN, 2*BN).
+      const uint32_t idesc = idesc_bf16_f32(C::kTileM, n_mma);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      for (int t = blockIdx.x; ok && t < total; t += gridDim.x) {
+      for (int t = cluster_id; ok && t < total; t += n_clusters) {
         Tile ti;
-        decode_tile(a, t, ti);
+        decode_tile<CG>(a, t, ti);
         const int nkb = a.k_kind[ti.kind] / kBK;
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort, a.err, a.timeout_ns)) break;
         tc_fence_after();
@@ -166,22 +210,27 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
           if (!mbar_wait(&full[stage], phase, abort, a.err, a.timeout_ns)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a_addr = smem_u32(sA + stage * kSmemA);
-          const uint32_t b_addr = smem_u32(sB + stage * kSmemBMax);
+          const uint32_t b_addr = smem_u32(sB + stage * C::kSmemB);
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk) {
             const uint64_t ad = sw128_kmajor_desc(a_addr + kk * 32);
+            const uint64_t bd = sw128_kmajor_desc(b_addr + kk * 32);
             const uint32_t accum = (kb | kk) != 0 ? 1u : 0u;
-            umma_bf16(d0, ad, sw128_kmajor_desc(b_addr + kk * 32), idesc, accum);
+            if (CG == 2) umma_bf16_pair(d0, ad, bd, idesc, accum);
+            else umma_bf16(d0, ad, bd, idesc, accum);
           }
-          umma_commit(&empty[stage]);
-          if (++stage == kStages) { stage = 0; phase ^= 1u; }
+          if (CG == 2) umma_commit_pair_mc(&empty[stage], 0x3);
+          else umma_commit(&empty[stage]);
+          if (++stage == S) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
-        umma_commit(&tfull[acc]);
+        if (CG == 2) umma_commit_pair_mc(&tfull[acc], 0x3);
+        else umma_commit(&tfull[acc]);
         if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
       }
       // Every MMA issued above has finished before TMEM is released.
-      umma_commit(tdone);
+      if (CG == 2) umma_commit_pair_mc(tdone, 0x1);
+      else umma_commit(tdone);
       mbar_wait_drain(tdone, 0, kDrainNs);
     }
   } else {
@@ -200,15 +249,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
     const int sr = lane >> 3, sc = lane & 7; // store phase: row offset 0..3, 16-byte chunk 0..7
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int t = blockIdx.x; t < total; t += gridDim.x) {
+    for (int t = cluster_id; t < total; t += n_clusters) {
       Tile ti;
-      decode_tile(a, t, ti);
+      decode_tile<CG>(a, t, ti);
       bool ok = mbar_wait(&tfull[acc], acc_phase, abort, a.err, a.timeout_ns);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                           static_cast<uint32_t>(acc) * acc_stride;
-      const int grow0 = ti.m * kBM + q * 32;   // first group row of this warp's block
+      const int grow0 = ti.m * C::kTileM + static_cast<int>(rank) * 128 + q * 32;
       const int nvalid = max(0, min(32, ti.rows - grow0));
       if (MODE == kGateUp) {
         const int orow0 = (ti.kind == 0 ? ti.a_row0 : ti.idx * a.shared_out_stride) + grow0;
@@ -290,18 +339,52 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[acc]);
+      if (lane == 0) {
+        if (CG == 2) mbar_arrive_cluster(tempty0 + 8 * acc);   // the even CTA's barrier
+        else mbar_arrive(&tempty[acc]);
+      }
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
     }
   }
 
+  // Neither CTA of a pair leaves while the other may still signal it.
   tc_fence_before();
-  __syncthreads();
+  if (CG == 2) cluster_sync(); else __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, kTmemCols);
+    if (CG == 2) tmem_dealloc_pair(tmem_base, kTmemCols);
+    else tmem_dealloc(tmem_base, kTmemCols);
   }
 }
+
+cudaLaunchConfig_t pair_config(int grid, cudaStream_t s, cudaLaunchAttribute* attr) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+  cfg.blockDim = dim3(kGemmThreads, 1, 1);
+  cfg.dynamicSmemBytes = kGemmSmem;
+  cfg.stream = s;
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cfg;
+}
+
+template <int MODE, int CG>
+cudaError_t launch_one(const GemmArgs& a, int grid, cudaStream_t s) {
+  if constexpr (CG == 1) {
+    k_grouped_gemm<MODE, 1><<<grid, kGemmThreads, kGemmSmem, s>>>(a);
+    return cudaGetLastError();
+  } else {
+    cudaLaunchAttribute attr[1];
+    const cudaLaunchConfig_t cfg = pair_config(grid, s, attr);
+    return cudaLaunchKernelEx(&cfg, k_grouped_gemm<MODE, 2>, a);
+  }
+}
+
+int g_pair_clusters[64] = {0};
 
 }  // namespace
 
@@ -310,20 +393,34 @@ void gemm_prepare() {
   int dev = 0;
   cudaGetDevice(&dev);
   if (done_dev == dev) return;
-  cudaFuncSetAttribute(k_grouped_gemm<kGateUp>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem);
-  cudaFuncSetAttribute(k_grouped_gemm<kDown>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem);
-  cudaFuncSetAttribute(k_grouped_gemm<kRouter>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem);
+  cudaFuncSetAttribute(k_grouped_gemm<kGateUp, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem);
+  cudaFuncSetAttribute(k_grouped_gemm<kDown, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem);
+  cudaFuncSetAttribute(k_grouped_gemm<kRouter, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem);
+  // How many CTA pairs fit on the device at once: the persistent pair grid is
+  // never larger, so no pair waits for another to finish before it starts.
+  int n_gu = 0, n_dn = 0;
+  cudaLaunchAttribute attr[1];
+  cudaLaunchConfig_t cfg = pair_config(2, nullptr, attr);
+  if (cudaOccupancyMaxActiveClusters(&n_gu, k_grouped_gemm<kGateUp, 2>, &cfg) != cudaSuccess) n_gu = 0;
+  if (cudaOccupancyMaxActiveClusters(&n_dn, k_grouped_gemm<kDown, 2>, &cfg) != cudaSuccess) n_dn = 0;
+  cudaGetLastError();
+  if (dev >= 0 && dev < 64) g_pair_clusters[dev] = std::min(n_gu, n_dn);
   done_dev = dev;
+}
+
+int gemm_max_pairs() {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  return (dev >= 0 && dev < 64) ? g_pair_clusters[dev] : 0;
 }
 
 cudaError_t launch_grouped_gemm(int mode, const GemmArgs& a, int grid, cudaStream_t s) {
   if (grid <= 0) return cudaSuccess;
   switch (mode) {
-    case kGateUp: k_grouped_gemm<kGateUp><<<grid, kGemmThreads, kGemmSmem, s>>>(a); break;
-    case kDown: k_grouped_gemm<kDown><<<grid, kGemmThreads, kGemmSmem, s>>>(a); break;
-    default: k_grouped_gemm<kRouter><<<grid, kGemmThreads, kGemmSmem, s>>>(a); break;
+    case kGateUp: return launch_one<kGateUp, 2>(a, grid, s);
+    case kDown: return launch_one<kDown, 2>(a, grid, s);
+    default: return launch_one<kRouter, 1>(a, grid, s);
   }
-  return cudaGetLastError();
 }
 
 }  // namespace moe

@@ -17,7 +17,7 @@ using namespace moe;
 struct moe_handle {
   moe_config cfg;
   moe_weights w;
-  int S = 0, G = 0, E_pad = 0, bn_gu = 0, bn_dn = 0, num_sms = 0, device = 0;
+  int S = 0, G = 0, E_pad = 0, bn_gu = 0, bn_dn = 0, num_sms = 0, device = 0, max_pairs = 0;
   uint16_t* w_router_pad = nullptr;  // [E_pad, D], rows >= E zero
   CUtensorMap map_router, map_wg, map_wu, map_wd, map_wsg, map_wsu, map_wsd;
   unsigned long long timeout_ns = 2000ull * 1000 * 1000;
@@ -165,12 +165,19 @@ struct Prof {
 
 // Upper bound on the tiles of the routed + shared expert GEMMs for T rows:
 // sum_e ceil(c_e / 128) <= T*k/128 + (number of non-empty experts).
+// sum_e ceil(c_e / 256) <= T*k/256 + (number of non-empty experts), in pair tiles.
 int expert_tile_bound(const moe_handle* h, int T, int nt_routed, int nt_shared) {
   const moe_config& c = h->cfg;
   const long long tk = static_cast<long long>(T) * c.k;
-  const long long mt = (tk + kBM - 1) / kBM + std::min<long long>(c.E, tk);
-  const long long b = mt * nt_routed + static_cast<long long>(h->S) * ((T + kBM - 1) / kBM) * nt_shared;
-  return static_cast<int>(std::min<long long>(b, 1 << 30));
+  const long long mt = (tk + kPairTileM - 1) / kPairTileM + std::min<long long>(c.E, tk);
+  const long long b = mt * nt_routed +
+                      static_cast<long long>(h->S) * ((T + kPairTileM - 1) / kPairTileM) * nt_shared;
+  return static_cast<int>(std::min<long long>(b, 1 << 29));
+}
+
+// CTA-pair grid: two CTAs per tile, at most one CTA per SM.
+int pair_grid(const moe_handle* h, int tiles_bound) {
+  return 2 * std::max(1, std::min(h->max_pairs, tiles_bound));
 }
 
 int forward_impl(moe_handle* h, int T, const uint16_t* x, const uint16_t* residual,
@@ -246,6 +253,7 @@ int forward_impl(moe_handle* h, int T, const uint16_t* x, const uint16_t* residu
   da.gu_ntiles_shared = h->S > 0 ? c.I_shared / h->bn_gu : 0;
   da.dn_ntiles = c.D / h->bn_dn;
   da.dest_row = dest; da.src_token = src;
+  da.tile_m = kPairTileM;
   prof.begin(3);
   MOE_TRY(launch_dispatch_count(da, s));
   prof.end(3);
@@ -280,7 +288,7 @@ int forward_impl(moe_handle* h, int T, const uint16_t* x, const uint16_t* residu
     g.err = err; g.timeout_ns = h->timeout_ns;
     const int bound = expert_tile_bound(h, T, da.gu_ntiles_routed, da.gu_ntiles_shared);
     prof.begin(7);
-    MOE_TRY(launch_grouped_gemm(kGateUp, g, gemm_grid(h, bound), s));
+    MOE_TRY(launch_grouped_gemm(kGateUp, g, pair_grid(h, bound), s));
     prof.end(7);
   }
 
@@ -304,7 +312,7 @@ int forward_impl(moe_handle* h, int T, const uint16_t* x, const uint16_t* residu
     g.err = err; g.timeout_ns = h->timeout_ns;
     const int bound = expert_tile_bound(h, T, da.dn_ntiles, da.dn_ntiles);
     prof.begin(8);
-    MOE_TRY(launch_grouped_gemm(kDown, g, gemm_grid(h, bound), s));
+    MOE_TRY(launch_grouped_gemm(kDown, g, pair_grid(h, bound), s));
     prof.end(8);
   }
 
@@ -348,7 +356,9 @@ int moe_init(const moe_config* cfg, const moe_weights* w, moe_handle** out) {
   if (h->S == 0) h->cfg.I_shared = cfg->I;  // unused; keeps the shapes well defined
   h->G = cfg->E + h->S;
   h->E_pad = (cfg->E + 15) / 16 * 16;
-  // One GEMM configuration per layer shape, never per T.
+  // One GEMM configuration per layer shape, never per T.  The expert GEMMs run
+  // on CTA pairs: each CTA loads the gate or the up tile (bn_gu rows) or half
+  // of a down tile (bn_dn / 2 rows).
   h->bn_gu = (cfg->I % 128 == 0 && h->cfg.I_shared % 128 == 0) ? 128 : 64;
   h->bn_dn = (cfg->D % 256 == 0) ? 256 : (cfg->D % 128 == 0 ? 128 : 64);
   auto fail = [&](int code) { moe_destroy(h); return code; };
@@ -356,6 +366,8 @@ int moe_init(const moe_config* cfg, const moe_weights* w, moe_handle** out) {
   if (cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, h->device) != cudaSuccess)
     return fail(MOE_ECUDA);
   gemm_prepare();
+  h->max_pairs = gemm_max_pairs();
+  if (h->max_pairs <= 0) h->max_pairs = h->num_sms / 2;
   const moe_config& c = h->cfg;
   if (c.router != MOE_ROUTER_HASH) {
     const size_t row = static_cast<size_t>(c.D) * 2;
@@ -367,10 +379,10 @@ int moe_init(const moe_config* cfg, const moe_weights* w, moe_handle** out) {
   bool ok = make_map(&h->map_router, h->w_router_pad, c.D, h->w_router_pad ? h->E_pad : 0, h->E_pad) &&
             make_map(&h->map_wg, w->w_gate, c.D, static_cast<uint64_t>(c.E) * c.I, h->bn_gu) &&
             make_map(&h->map_wu, w->w_up, c.D, static_cast<uint64_t>(c.E) * c.I, h->bn_gu) &&
-            make_map(&h->map_wd, w->w_down, c.I, static_cast<uint64_t>(c.E) * c.D, h->bn_dn) &&
+            make_map(&h->map_wd, w->w_down, c.I, static_cast<uint64_t>(c.E) * c.D, h->bn_dn / 2) &&
             make_map(&h->map_wsg, w->ws_gate, c.D, static_cast<uint64_t>(h->S) * c.I_shared, h->bn_gu) &&
             make_map(&h->map_wsu, w->ws_up, c.D, static_cast<uint64_t>(h->S) * c.I_shared, h->bn_gu) &&
-            make_map(&h->map_wsd, w->ws_down, c.I_shared, static_cast<uint64_t>(h->S) * c.D, h->bn_dn);
+            make_map(&h->map_wsd, w->ws_down, c.I_shared, static_cast<uint64_t>(h->S) * c.D, h->bn_dn / 2);
   if (!ok) return fail(MOE_ECUDA);
   *out = h;
   return MOE_OK;

@@ -15,7 +15,8 @@ namespace moe {
 // (same groups).  Tiles are BM = 128 rows x BN columns with the whole K
 // reduced in one TMEM accumulator (no split-K), K walked in 64-wide steps in
 // the same order for every tile.
-constexpr int kBM = 128;
+constexpr int kBM = 128;        // rows per CTA of a tile
+constexpr int kPairTileM = 256; // rows per tile of the expert GEMMs (a CTA pair)
 constexpr int kBK = 64;
 constexpr int kStages = 4;
 constexpr int kEpiWarps = 8;       // two per TMEM lane quarter, splitting the columns
@@ -48,7 +49,8 @@ struct GemmArgs {
   unsigned long long timeout_ns;
 };
 
-void gemm_prepare();  // sets the dynamic shared memory limit once per device
+void gemm_prepare();    // shared memory limit + pair occupancy, once per device
+int gemm_max_pairs();   // CTA pairs of the expert GEMMs resident at once (0 = unknown)
 cudaError_t launch_grouped_gemm(int mode, const GemmArgs& a, int grid, cudaStream_t s);
 
 // --------------------------------------------------------------- row ops
@@ -98,6 +100,7 @@ struct DispatchArgs {
   int32_t* tiles_gu;      // [E + S + 1]
   int32_t* tiles_dn;      // [E + S + 1]
   int gu_ntiles_routed, gu_ntiles_shared, dn_ntiles;
+  int tile_m;             // rows per expert-GEMM tile (256: a CTA pair)
   int32_t* dest_row;      // [T * k]
   int32_t* src_token;     // [T * k]
 };
