@@ -3,9 +3,9 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl b200|reference]
 
-One step is one full layer forward (all ten kernels: RMSNorm, router GEMM,
-top-k, histogram / scan / stable scatter, row gather, gate/up + SwiGLU GEMM,
-down GEMM, fixed-order combine + residual + RMSNorm) over one batch of the
+One step is one full layer forward (all eight kernels: RMSNorm, router GEMM,
+top-k with the expert histogram, offsets + stable scatter, row gather,
+gate/up + SwiGLU GEMM, down GEMM, fixed-order combine + residual + RMSNorm) over one batch of the
 fine-grained workload (T=4096 tokens, D=2048, 64 experts top-6 softmax
 renormalised, I=1408, 2 shared experts of 1408) with seeded synthetic inputs
 and random weights of that architecture.  The L2 cache is flushed (a 512 MiB
@@ -38,7 +38,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "MoE layer tokens/sec at 1 B200; % bf16 TC peak (prefill) / % HBM BW (decode)"
 UNIT = "tokens/s"
-GATEUP_STAGE = 7
+GATEUP_STAGE = 5
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic_gemm_gateup_swiglu_fine_grained.json")
 GEMM_SOURCES = [os.path.join(ROOT, "deterministic_expert_b200", "csrc", n)
                 for n in ("grouped_gemm.cu", "common.cuh", "moe_internal.h")]

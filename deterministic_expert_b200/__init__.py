@@ -21,9 +21,9 @@ HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "moe.h")
 MOE_OK, MOE_EINVAL, MOE_ETOOBIG, MOE_EWORKSPACE, MOE_EUNSUPPORTED, MOE_ECUDA, MOE_ETIMEOUT = (
     0, -1, -2, -3, -4, -5, -6)
 ROUTER_SOFTMAX, ROUTER_SIGMOID_BIAS, ROUTER_HASH = 0, 1, 2
-NUM_STAGES = 10
-STAGE_NAMES = ("rmsnorm_in", "router_gemm", "router_topk", "dispatch_count", "dispatch_scan",
-               "dispatch_scatter", "gather_rows", "gemm_gateup_swiglu", "gemm_down", "combine_norm")
+NUM_STAGES = 8
+STAGE_NAMES = ("rmsnorm_in", "router_gemm", "router_topk", "dispatch", "gather_rows",
+               "gemm_gateup_swiglu", "gemm_down", "combine_norm")
 
 
 class MoEError(RuntimeError):

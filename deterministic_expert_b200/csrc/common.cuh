@@ -18,6 +18,16 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
+// ------------------------------------------------- programmatic launch
+// Every kernel of the layer is launched with programmatic stream
+// serialisation and calls griddep_wait() before its first global-memory
+// access, so it still sees all of the previous kernel's writes (the wait
+// returns once that grid has completed and flushed); what overlaps is only
+// the launch and the prologue.  griddep_launch() lets the next kernel of the
+// stream start launching.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch() { asm volatile("griddepcontrol.launch_dependents;" :::); }
+
 // ------------------------------------------------------------------- bf16
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }

@@ -129,6 +129,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
   tc_fence_after();
   const uint32_t tmem_base = tmem_slot;
   volatile int* abort = &abort_flag;
+  // The prologue above touches no global memory; wait for the previous kernel
+  // of the stream before reading the tile list or any operand.
+  griddep_wait();
+  griddep_launch();
 
   const int cluster_id = blockIdx.x / CG, n_clusters = gridDim.x / CG;
   const int total = (a.tile_start == nullptr) ? a.router_tiles : a.tile_start[a.G];
@@ -374,14 +378,7 @@ cudaLaunchConfig_t pair_config(int grid, cudaStream_t s, cudaLaunchAttribute* at
 
 template <int MODE, int CG>
 cudaError_t launch_one(const GemmArgs& a, int grid, cudaStream_t s) {
-  if constexpr (CG == 1) {
-    k_grouped_gemm<MODE, 1><<<grid, kGemmThreads, kGemmSmem, s>>>(a);
-    return cudaGetLastError();
-  } else {
-    cudaLaunchAttribute attr[1];
-    const cudaLaunchConfig_t cfg = pair_config(grid, s, attr);
-    return cudaLaunchKernelEx(&cfg, k_grouped_gemm<MODE, 2>, a);
-  }
+  return launch_k(k_grouped_gemm<MODE, CG>, dim3(grid), dim3(kGemmThreads), kGemmSmem, s, CG == 2, a);
 }
 
 int g_pair_clusters[64] = {0};

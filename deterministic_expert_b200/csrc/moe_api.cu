@@ -35,7 +35,7 @@ constexpr int kProfFwd = 256;
 size_t align256(size_t b) { return (b + 255) & ~static_cast<size_t>(255); }
 
 struct Layout {
-  size_t err, xn, logits, tidx, tw, bcount, bbase, counts, offsets, tiles_gu, tiles_dn, dest, src,
+  size_t err, xn, logits, tidx, tw, bcount, counts, offsets, tiles_gu, tiles_dn, dest, src,
       xp, h, hs, y, ys, total;
 };
 
@@ -51,7 +51,6 @@ Layout layout(const moe_handle* h, int T) {
   L.tidx = take(Tz * c.k * 4);
   L.tw = take(Tz * c.k * 4);
   L.bcount = take(nb * c.E * 4);
-  L.bbase = take(nb * c.E * 4);
   L.counts = take(static_cast<size_t>(c.E) * 4);
   L.offsets = take(static_cast<size_t>(c.E + 1) * 4);
   L.tiles_gu = take(static_cast<size_t>(h->G + 1) * 4);
@@ -206,9 +205,11 @@ int forward_impl(moe_handle* h, int T, const uint16_t* x, const uint16_t* residu
   Prof prof{h, s, -1};
   if (h->prof_mask && h->prof_fwd < kProfFwd) prof.f = h->prof_fwd++;
 
-  // 0. input RMSNorm (also clears the device error word)
+  // 0. input RMSNorm (also clears the device error word and the histogram)
+  int32_t* bcount = reinterpret_cast<int32_t*>(ws + L.bcount);
+  const int nblk = (T + kDispatchRows - 1) / kDispatchRows;
   prof.begin(0);
-  MOE_TRY(launch_rmsnorm_rows(x, h->w.g_in, xn, T, c.D, c.eps, err, s));
+  MOE_TRY(launch_rmsnorm_rows(x, h->w.g_in, xn, T, c.D, c.eps, err, bcount, nblk * c.E, s));
   prof.end(0);
 
   // 1. router logits on the tensor cores
@@ -231,22 +232,22 @@ int forward_impl(moe_handle* h, int T, const uint16_t* x, const uint16_t* residu
     prof.end(1);
   }
 
-  // 2. scores, top-k, weights
+  // 2. scores, top-k, weights, and each 128-token block's expert histogram
   RouterArgs ra;
   ra.logits = logits; ra.E_pad = h->E_pad; ra.bias = h->w.router_bias; ra.token_ids = token_ids;
   ra.router = c.router; ra.E = c.E; ra.k = c.k; ra.renormalize = c.renormalize;
-  ra.routed_scale = c.routed_scale; ra.hash_mult = c.hash_mult; ra.idx = tidx; ra.w = tw; ra.T = T;
+  ra.routed_scale = c.routed_scale; ra.hash_mult = c.hash_mult; ra.idx = tidx; ra.w = tw;
+  ra.block_counts = bcount; ra.T = T;
   prof.begin(2);
   MOE_TRY(launch_router_topk(ra, s));
   prof.end(2);
   if (out_idx) MOE_TRY(cudaMemcpyAsync(out_idx, tidx, static_cast<size_t>(TK) * 4, cudaMemcpyDeviceToDevice, s));
   if (out_w) MOE_TRY(cudaMemcpyAsync(out_w, tw, static_cast<size_t>(TK) * 4, cudaMemcpyDeviceToDevice, s));
 
-  // 3-5. histogram, scan (+ tile lists), stable scatter
+  // 3. offsets, stable scatter and the expert-GEMM tile lists
   DispatchArgs da;
   da.idx = tidx; da.T = T; da.k = c.k; da.E = c.E; da.S = h->S;
-  da.block_counts = reinterpret_cast<int32_t*>(ws + L.bcount);
-  da.block_base = reinterpret_cast<int32_t*>(ws + L.bbase);
+  da.block_counts = bcount;
   da.counts = reinterpret_cast<int32_t*>(ws + L.counts);
   da.offsets = offsets; da.user_counts = out_counts; da.tiles_gu = tiles_gu; da.tiles_dn = tiles_dn;
   da.gu_ntiles_routed = c.I / h->bn_gu;
@@ -255,21 +256,15 @@ int forward_impl(moe_handle* h, int T, const uint16_t* x, const uint16_t* residu
   da.dest_row = dest; da.src_token = src;
   da.tile_m = kPairTileM;
   prof.begin(3);
-  MOE_TRY(launch_dispatch_count(da, s));
+  MOE_TRY(launch_dispatch(da, s));
   prof.end(3);
+
+  // 4. grouped A rows of the routed experts
   prof.begin(4);
-  MOE_TRY(launch_dispatch_scan(da, s));
-  prof.end(4);
-  prof.begin(5);
-  MOE_TRY(launch_dispatch_scatter(da, s));
-  prof.end(5);
-
-  // 6. grouped A rows of the routed experts
-  prof.begin(6);
   MOE_TRY(launch_gather_rows(xn, src, TK, c.D, xp, s));
-  prof.end(6);
+  prof.end(4);
 
-  // 7. gate/up + SwiGLU(+clamp): routed groups read xp, shared groups read xn
+  // 5. gate/up + SwiGLU(+clamp): routed groups read xp, shared groups read xn
   {
     GemmArgs g;
     std::memset(&g, 0, sizeof(g));
@@ -287,12 +282,12 @@ int forward_impl(moe_handle* h, int T, const uint16_t* x, const uint16_t* residu
     g.gate_clamp = c.gate_clamp_max; g.up_clamp = c.up_clamp;
     g.err = err; g.timeout_ns = h->timeout_ns;
     const int bound = expert_tile_bound(h, T, da.gu_ntiles_routed, da.gu_ntiles_shared);
-    prof.begin(7);
+    prof.begin(5);
     MOE_TRY(launch_grouped_gemm(kGateUp, g, pair_grid(h, bound), s));
-    prof.end(7);
+    prof.end(5);
   }
 
-  // 8. down: routed rows scatter to their (token, slot) row of y
+  // 6. down: routed rows scatter to their (token, slot) row of y
   {
     GemmArgs g;
     std::memset(&g, 0, sizeof(g));
@@ -311,16 +306,16 @@ int forward_impl(moe_handle* h, int T, const uint16_t* x, const uint16_t* residu
     g.dest_row = dest;
     g.err = err; g.timeout_ns = h->timeout_ns;
     const int bound = expert_tile_bound(h, T, da.dn_ntiles, da.dn_ntiles);
-    prof.begin(8);
+    prof.begin(6);
     MOE_TRY(launch_grouped_gemm(kDown, g, pair_grid(h, bound), s));
-    prof.end(8);
+    prof.end(6);
   }
 
-  // 9. fixed-order combine + residual + RMSNorm
-  prof.begin(9);
+  // 7. fixed-order combine + residual + RMSNorm
+  prof.begin(7);
   MOE_TRY(launch_combine_norm(y, tw, ys, c.k, h->S, residual, h->w.g_out, out_norm, out_residual, T,
                               c.D, c.eps, s));
-  prof.end(9);
+  prof.end(7);
   return MOE_OK;
 }
 
@@ -567,7 +562,7 @@ int moe_profile_read(moe_handle* h, float* ms, int* launches) {
 int moe_forward_launch_count(const moe_handle* h, int T) {
   if (!h || T < 0) return -1;
   if (T == 0) return 0;
-  return h->cfg.router == MOE_ROUTER_HASH ? MOE_NUM_STAGES - 1 : MOE_NUM_STAGES;
+  return h->cfg.router == MOE_ROUTER_HASH ? MOE_NUM_STAGES - 1 : MOE_NUM_STAGES;  // no router GEMM
 }
 
 int moe_selftest_wait_timeout(int limit_us, void* stream) {

@@ -9,6 +9,32 @@
 
 namespace moe {
 
+// Launch `kernel` on `s` with programmatic stream serialisation (and a cluster
+// of 2 CTAs when pair is true).  See griddep_wait() in common.cuh.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                     bool pair, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  int n = 1;
+  if (pair) {
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = 2;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    n = 2;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 // ------------------------------------------------------------ grouped GEMM
 // One persistent, warp-specialised tcgen05 GEMM serves the router (one group
 // of T rows), gate/up + SwiGLU (E routed groups + S shared groups) and down
@@ -54,8 +80,10 @@ int gemm_max_pairs();   // CTA pairs of the expert GEMMs resident at once (0 = u
 cudaError_t launch_grouped_gemm(int mode, const GemmArgs& a, int grid, cudaStream_t s);
 
 // --------------------------------------------------------------- row ops
+// Also clears the device error word and zeroes `zero_words` int32 at `zero`.
 cudaError_t launch_rmsnorm_rows(const uint16_t* x, const uint16_t* g, uint16_t* y, int T, int D,
-                                float eps, int* err_to_clear, cudaStream_t s);
+                                float eps, int* err_to_clear, int32_t* zero, int zero_words,
+                                cudaStream_t s);
 cudaError_t launch_combine_norm(const float* y_slot, const float* topk_w, const float* y_shared,
                                 int k, int S, const uint16_t* residual, const uint16_t* g,
                                 uint16_t* out_norm, uint16_t* out_residual, int T, int D,
@@ -83,17 +111,17 @@ struct RouterArgs {
   uint32_t hash_mult;
   int32_t* idx;             // [T, k]
   float* w;                 // [T, k]
+  int32_t* block_counts;    // [ceil(T / 128), E], zeroed beforehand
   int T;
 };
 cudaError_t launch_router_topk(const RouterArgs& a, cudaStream_t s);
 
 // ------------------------------------------------------------ dispatch
-constexpr int kDispatchRows = 256;  // tokens per dispatch block
+constexpr int kDispatchRows = 128;  // tokens per dispatch block (= one router GEMM tile)
 struct DispatchArgs {
   const int32_t* idx;   // [T, k]
   int T, k, E, S;
-  int32_t* block_counts;  // [nb, E]
-  int32_t* block_base;    // [nb, E]
+  const int32_t* block_counts;  // [nb, E] expert counts of each 128-token block
   int32_t* counts;        // [E]
   int32_t* offsets;       // [E + 1]
   int32_t* user_counts;   // [E] or NULL
@@ -104,9 +132,7 @@ struct DispatchArgs {
   int32_t* dest_row;      // [T * k]
   int32_t* src_token;     // [T * k]
 };
-cudaError_t launch_dispatch_count(const DispatchArgs& a, cudaStream_t s);
-cudaError_t launch_dispatch_scan(const DispatchArgs& a, cudaStream_t s);
-cudaError_t launch_dispatch_scatter(const DispatchArgs& a, cudaStream_t s);
+cudaError_t launch_dispatch(const DispatchArgs& a, cudaStream_t s);
 cudaError_t launch_gather_rows(const uint16_t* src, const int32_t* src_row, int rows, int D,
                                uint16_t* dst, cudaStream_t s);
 

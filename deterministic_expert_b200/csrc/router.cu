@@ -10,7 +10,9 @@
 //
 // Selection is deterministic: k rounds of a warp arg-max under the total
 // order (key descending, expert index ascending), so equal keys go to the
-// lower index and slot j holds the j-th best expert.  Lane l always owns
+// lower index and slot j holds the j-th best expert.  Each token also adds its
+// k experts to the histogram of its 128-token block (integer atomics into a
+// buffer the input RMSNorm zeroed; the counts do not depend on the order).  Lane l always owns
 // experts l, l + 32, ... and every sum runs in a fixed order (per lane in
 // index order, then a 5-step butterfly), so a token's routing does not
 // depend on T.  Keys that are NaN rank below every number.  Softmax selects on
@@ -31,10 +33,13 @@ __device__ __forceinline__ bool better(float k1, int e1, float k2, int e2) {
 }
 
 __global__ void __launch_bounds__(256) k_router_topk(const RouterArgs a) {
+  griddep_wait();
+  griddep_launch();
   const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (t >= a.T) return;
   const int k = a.k, E = a.E;
+  int32_t* hist = a.block_counts + static_cast<size_t>(t / kDispatchRows) * E;
 
   if (a.router == MOE_ROUTER_HASH) {
     if (lane < k) {
@@ -42,6 +47,7 @@ __global__ void __launch_bounds__(256) k_router_topk(const RouterArgs a) {
       const int e0 = static_cast<int>(h % static_cast<uint32_t>(E));
       a.idx[t * k + lane] = (e0 + lane) % E;
       a.w[t * k + lane] = a.routed_scale / static_cast<float>(k);
+      atomicAdd(hist + (e0 + lane) % E, 1);
     }
     return;
   }
@@ -123,6 +129,7 @@ __global__ void __launch_bounds__(256) k_router_topk(const RouterArgs a) {
     for (int q = 0; q < k; ++q)
       if (q == j) { w = chosen_v[q]; e = chosen_e[q]; }
     a.idx[t * k + j] = e;
+    atomicAdd(hist + e, 1);
     const float wn = (a.router == MOE_ROUTER_SOFTMAX || a.renormalize) ? w / norm : w;
     a.w[t * k + j] = wn * a.routed_scale;
   }
@@ -133,8 +140,8 @@ __global__ void __launch_bounds__(256) k_router_topk(const RouterArgs a) {
 cudaError_t launch_router_topk(const RouterArgs& a, cudaStream_t s) {
   if (a.T <= 0) return cudaSuccess;
   const int warps_per_block = 8;
-  k_router_topk<<<(a.T + warps_per_block - 1) / warps_per_block, 32 * warps_per_block, 0, s>>>(a);
-  return cudaGetLastError();
+  return launch_k(k_router_topk, dim3((a.T + warps_per_block - 1) / warps_per_block),
+                  dim3(32 * warps_per_block), 0, s, false, a);
 }
 
 }  // namespace moe

@@ -6,7 +6,7 @@
 // parity post (Chinese translation), Trap 2, says must not change with the
 // launch shape.  Nothing here depends on T.
 //
-//   rmsnorm_rows     xn = bf16((x * s) * g), s = fp32(1 / sqrt(mean(x^2) + eps)) from an
+//   rmsnorm_rows     (also zeroes the routing histogram) xn = bf16((x * s) * g), s = fp32(1 / sqrt(mean(x^2) + eps)) from an
 //                    fp64 sum of squares (same fixed tree) so that the bf16 code of
 //                    xn, which decides the routing, is fixed by a well-defined fp32
 //                    scale (linux.do post on MoE variants, "RMSNorm before up-projection")
@@ -59,9 +59,14 @@ template <int NC>
 __global__ void __launch_bounds__(kRowThreads) k_rmsnorm_rows(const uint16_t* __restrict__ x,
                                                               const uint16_t* __restrict__ g,
                                                               uint16_t* __restrict__ y, int D,
-                                                              float eps, int* err) {
+                                                              float eps, int* err, int32_t* zero,
+                                                              int zero_words) {
   __shared__ double red[kRowThreads / 32 + 1];
+  griddep_wait();
+  griddep_launch();
   if (err != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *err = kDevOk;
+  for (int i = blockIdx.x * kRowThreads + threadIdx.x; i < zero_words; i += gridDim.x * kRowThreads)
+    zero[i] = 0;
   const size_t row = blockIdx.x;
   const int nch = D / 4;
   const uint16_t* xr = x + row * D;
@@ -122,6 +127,8 @@ __global__ void __launch_bounds__(kRowThreads) k_combine_norm(
     uint16_t* __restrict__ out_residual, int T, int D, float eps) {
   __shared__ float red[kRowThreads / 32 + 1];
   __shared__ float w_s[16];
+  griddep_wait();
+  griddep_launch();
   const size_t t = blockIdx.x;
   if (threadIdx.x < k) w_s[threadIdx.x] = topk_w[t * k + threadIdx.x];
   __syncthreads();
@@ -158,6 +165,8 @@ __global__ void __launch_bounds__(kRowThreads) k_reduce_partials(
     const uint16_t* __restrict__ g, uint16_t* __restrict__ out_norm,
     uint16_t* __restrict__ out_residual, int D, float eps) {
   __shared__ float red[kRowThreads / 32 + 1];
+  griddep_wait();
+  griddep_launch();
   const size_t t = blockIdx.x;
   const int nch = D / 4;
   float4 r[NC];
@@ -188,6 +197,8 @@ __global__ void __launch_bounds__(kRowThreads) k_reduce_partials(
 __global__ void k_bitcompare(const uint16_t* __restrict__ a, const uint16_t* __restrict__ b,
                              const int32_t* __restrict__ b_row_of_a, int rows, int D,
                              unsigned long long* count) {
+  griddep_wait();
+  griddep_launch();
   const int per_row = D / 8;
   const size_t n = static_cast<size_t>(rows) * per_row;
   unsigned long long mism = 0;
@@ -213,6 +224,8 @@ __global__ void k_permute_inputs(const uint16_t* __restrict__ x, const uint16_t*
                                  const int32_t* __restrict__ ids, const int32_t* __restrict__ perm,
                                  int T, int D, uint16_t* __restrict__ xo, uint16_t* __restrict__ ro,
                                  int32_t* __restrict__ io) {
+  griddep_wait();
+  griddep_launch();
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   if (warp >= T) return;
   const size_t src = perm[warp];
@@ -239,16 +252,20 @@ __global__ void k_wait_selftest(volatile int* flag, int* err, unsigned long long
 }  // namespace
 
 cudaError_t launch_rmsnorm_rows(const uint16_t* x, const uint16_t* g, uint16_t* y, int T, int D,
-                                float eps, int* err_to_clear, cudaStream_t s) {
+                                float eps, int* err_to_clear, int32_t* zero, int zero_words,
+                                cudaStream_t s) {
   if (T <= 0) return cudaSuccess;
+  auto go = [&](auto kernel) {
+    return launch_k(kernel, dim3(T), dim3(kRowThreads), 0, s, false, x, g, y, D, eps, err_to_clear,
+                    zero, zero_words);
+  };
   switch (chunks_for(D)) {
-    case 1: k_rmsnorm_rows<1><<<T, kRowThreads, 0, s>>>(x, g, y, D, eps, err_to_clear); break;
-    case 2: k_rmsnorm_rows<2><<<T, kRowThreads, 0, s>>>(x, g, y, D, eps, err_to_clear); break;
-    case 4: k_rmsnorm_rows<4><<<T, kRowThreads, 0, s>>>(x, g, y, D, eps, err_to_clear); break;
-    case 8: k_rmsnorm_rows<8><<<T, kRowThreads, 0, s>>>(x, g, y, D, eps, err_to_clear); break;
-    default: k_rmsnorm_rows<16><<<T, kRowThreads, 0, s>>>(x, g, y, D, eps, err_to_clear); break;
+    case 1: return go(k_rmsnorm_rows<1>);
+    case 2: return go(k_rmsnorm_rows<2>);
+    case 4: return go(k_rmsnorm_rows<4>);
+    case 8: return go(k_rmsnorm_rows<8>);
+    default: return go(k_rmsnorm_rows<16>);
   }
-  return cudaGetLastError();
 }
 
 cudaError_t launch_combine_norm(const float* y_slot, const float* topk_w, const float* y_shared,
@@ -256,35 +273,34 @@ cudaError_t launch_combine_norm(const float* y_slot, const float* topk_w, const 
                                 uint16_t* out_norm, uint16_t* out_residual, int T, int D,
                                 float eps, cudaStream_t s) {
   if (T <= 0) return cudaSuccess;
-#define MOE_COMBINE(NC)                                                                          \
-  k_combine_norm<NC><<<T, kRowThreads, 0, s>>>(y_slot, topk_w, y_shared, k, S, residual, g,     \
-                                              out_norm, out_residual, T, D, eps)
+  auto go = [&](auto kernel) {
+    return launch_k(kernel, dim3(T), dim3(kRowThreads), 0, s, false, y_slot, topk_w, y_shared, k, S,
+                    residual, g, out_norm, out_residual, T, D, eps);
+  };
   switch (chunks_for(D)) {
-    case 1: MOE_COMBINE(1); break;
-    case 2: MOE_COMBINE(2); break;
-    case 4: MOE_COMBINE(4); break;
-    case 8: MOE_COMBINE(8); break;
-    default: MOE_COMBINE(16); break;
+    case 1: return go(k_combine_norm<1>);
+    case 2: return go(k_combine_norm<2>);
+    case 4: return go(k_combine_norm<4>);
+    case 8: return go(k_combine_norm<8>);
+    default: return go(k_combine_norm<16>);
   }
-#undef MOE_COMBINE
-  return cudaGetLastError();
 }
 
 cudaError_t launch_reduce_partials(const PartialPtrs& parts, int P, const uint16_t* residual,
                                    const uint16_t* g, uint16_t* out_norm, uint16_t* out_residual,
                                    int T, int D, float eps, cudaStream_t s) {
   if (T <= 0) return cudaSuccess;
-#define MOE_REDUCE(NC) \
-  k_reduce_partials<NC><<<T, kRowThreads, 0, s>>>(parts, P, residual, g, out_norm, out_residual, D, eps)
+  auto go = [&](auto kernel) {
+    return launch_k(kernel, dim3(T), dim3(kRowThreads), 0, s, false, parts, P, residual, g, out_norm,
+                    out_residual, D, eps);
+  };
   switch (chunks_for(D)) {
-    case 1: MOE_REDUCE(1); break;
-    case 2: MOE_REDUCE(2); break;
-    case 4: MOE_REDUCE(4); break;
-    case 8: MOE_REDUCE(8); break;
-    default: MOE_REDUCE(16); break;
+    case 1: return go(k_reduce_partials<1>);
+    case 2: return go(k_reduce_partials<2>);
+    case 4: return go(k_reduce_partials<4>);
+    case 8: return go(k_reduce_partials<8>);
+    default: return go(k_reduce_partials<16>);
   }
-#undef MOE_REDUCE
-  return cudaGetLastError();
 }
 
 cudaError_t launch_bitcompare(const uint16_t* a, const uint16_t* b, const int32_t* b_row_of_a,
@@ -293,8 +309,7 @@ cudaError_t launch_bitcompare(const uint16_t* a, const uint16_t* b, const int32_
   const size_t n = static_cast<size_t>(rows) * (D / 8);
   int grid = static_cast<int>((n + 255) / 256);
   if (grid > 148 * 8) grid = 148 * 8;
-  k_bitcompare<<<grid, 256, 0, s>>>(a, b, b_row_of_a, rows, D, count);
-  return cudaGetLastError();
+  return launch_k(k_bitcompare, dim3(grid), dim3(256), 0, s, false, a, b, b_row_of_a, rows, D, count);
 }
 
 cudaError_t launch_permute_inputs(const uint16_t* x, const uint16_t* res, const int32_t* ids,
@@ -302,9 +317,8 @@ cudaError_t launch_permute_inputs(const uint16_t* x, const uint16_t* res, const 
                                   int32_t* io, cudaStream_t s) {
   if (T <= 0) return cudaSuccess;
   const int warps_per_block = 8;
-  k_permute_inputs<<<(T + warps_per_block - 1) / warps_per_block, 32 * warps_per_block, 0, s>>>(
-      x, res, ids, perm, T, D, xo, ro, io);
-  return cudaGetLastError();
+  return launch_k(k_permute_inputs, dim3((T + warps_per_block - 1) / warps_per_block),
+                  dim3(32 * warps_per_block), 0, s, false, x, res, ids, perm, T, D, xo, ro, io);
 }
 
 cudaError_t launch_wait_selftest(int* flag, int* err, unsigned long long limit_ns, cudaStream_t s) {

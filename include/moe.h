@@ -108,10 +108,13 @@ typedef struct moe_weights {      /* device pointers, caller-owned              
 
 typedef struct moe_handle moe_handle;
 
-/* Number of kernel stages moe_profile_read reports, in launch order:
- * 0 rmsnorm_in, 1 router_gemm, 2 router_topk, 3 dispatch_count, 4 dispatch_scan,
- * 5 dispatch_scatter, 6 gather_rows, 7 gemm_gateup_swiglu, 8 gemm_down, 9 combine_norm. */
-#define MOE_NUM_STAGES 10
+/* Kernel stages of one forward, in launch order (one kernel each), as
+ * moe_profile_read reports them:
+ * 0 rmsnorm_in, 1 router_gemm (not launched for MOE_ROUTER_HASH), 2 router_topk
+ * (scores, top-k, weights, per-128-token expert histogram), 3 dispatch (offsets
+ * and stable scatter), 4 gather_rows, 5 gemm_gateup_swiglu, 6 gemm_down,
+ * 7 combine_norm. */
+#define MOE_NUM_STAGES 8
 
 /* Validate `cfg`, keep the weight pointers and build the weight TMA
  * descriptors on the current CUDA device.  Allocates one small handle-owned
