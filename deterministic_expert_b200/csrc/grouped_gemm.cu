@@ -18,10 +18,13 @@
 //   CG = 1  one CTA per 128-row tile (the router GEMM).
 //   CG = 2  a CTA pair (cluster of 2) per 256-row tile with cta_group::2 MMAs
 //           (the expert GEMMs): each CTA loads its own 128 A rows and half of
-//           the B tile (gate/up: the even CTA the gate rows, the odd CTA the up
-//           rows; down: one half of the BN output columns each), so each SM's
+//           the B tile (one half of the output columns: gate/up as [gate | up]
+//           rows for those columns, down as those rows of W_d), so each SM's
 //           shared memory receives and feeds half the B bytes of a 1-CTA tile.
-//           The even CTA issues the MMAs; its commits reach both CTAs.
+//           The even CTA issues the MMAs; its commits reach both CTAs.  A
+//           group's last tile runs as a 128-row pair tile (M = 128, 64 rows per
+//           CTA) when no more than 128 rows remain, so the padding of a group is
+//           under 128 rows, not 256.
 // Roles in each CTA:
 //   warp 0    one thread issues the TMA loads of its CTA into a stage ring
 //   warp 1    allocates 512 TMEM columns; in the (even) issuing CTA one thread
@@ -57,12 +60,13 @@ struct Tile {
   int rows;   // rows of the group
   int a_row0; // first A row of the group
   int m, n;   // tile coordinates within the group
+  bool small; // pair tile with 128 rows (M = 128): the group's last <= 128 rows
 };
 
 template <int CG>
 __device__ __forceinline__ void decode_tile(const GemmArgs& a, int t, Tile& ti) {
   if (a.tile_start == nullptr) {
-    ti.kind = 0; ti.idx = 0; ti.rows = a.T; ti.a_row0 = 0; ti.m = t; ti.n = 0;
+    ti.kind = 0; ti.idx = 0; ti.rows = a.T; ti.a_row0 = 0; ti.m = t; ti.n = 0; ti.small = false;
     return;
   }
   // Largest g with tile_start[g] <= t; tile_start[0] = 0 <= t < tile_start[G].
@@ -81,6 +85,7 @@ __device__ __forceinline__ void decode_tile(const GemmArgs& a, int t, Tile& ti) 
   const int mt = (ti.rows + Cfg<CG>::kTileM - 1) / Cfg<CG>::kTileM;
   ti.n = local / mt;
   ti.m = local - ti.n * mt;
+  ti.small = CG == 2 && ti.rows - ti.m * Cfg<CG>::kTileM <= 128;
 }
 
 // SiLU(min(g, c_g)) * clamp(u, -c_u, c_u) in fp32 with the fast exponential
@@ -138,9 +143,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
   const int total = (a.tile_start == nullptr) ? a.router_tiles : a.tile_start[a.G];
   const int BN = a.BN;                                    // output columns per tile (per matrix)
   const int n_mma = MODE == kGateUp ? 2 * BN : BN;        // N of one MMA
-  // B rows each CTA loads per stage (per matrix for gate/up).
-  const uint32_t b_rows = static_cast<uint32_t>(MODE == kGateUp ? BN : BN / CG);
-  const uint32_t stage_bytes = kSmemA + b_rows * kBK * 2 * (MODE == kGateUp && CG == 1 ? 2 : 1);
+  // B rows each CTA loads per stage, per matrix (gate and up each for gate/up).
+  const uint32_t b_rows = static_cast<uint32_t>(BN / CG);
+  const uint32_t stage_bytes = kSmemA + b_rows * kBK * 2 * (MODE == kGateUp ? 2 : 1);
   const uint32_t acc_stride = static_cast<uint32_t>(n_mma);  // TMEM columns per buffer
   // Barriers the pair shares live in the even CTA.
   const uint32_t full0 = CG == 2 ? mapa_shared(full, 0) : 0;
@@ -158,13 +163,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
         Tile ti;
         decode_tile<CG>(a, t, ti);
         const int nkb = a.k_kind[ti.kind] / kBK;
-        const int a_y = ti.a_row0 + ti.m * C::kTileM + static_cast<int>(rank) * 128;
+        // A: this CTA's rows of the tile (128, or 64 in a 128-row pair tile).
+        const int a_y = ti.a_row0 + ti.m * C::kTileM + static_cast<int>(rank) * (ti.small ? 64 : 128);
         int b_y = ti.idx * a.n_kind[ti.kind] + ti.n * BN;
         const CUtensorMap* bmap = &a.mapB[ti.kind * 2];
-        if (CG == 2) {
-          if (MODE == kGateUp) bmap += rank;                          // gate | up
-          else b_y += static_cast<int>(rank) * (BN / 2);             // lower | upper half
-        }
+        // Pair B halves: gate/up - the CTA of rank r loads gate rows and up rows
+        // [r*BN/2, (r+1)*BN/2) of the tile (interleaved [gate | up] per half, so
+        // each accumulator lane holds matching gate and up columns); down - rows
+        // [r*BN/2, (r+1)*BN/2) of the tile's output columns.
+        if (CG == 2) b_y += static_cast<int>(rank) * (BN / 2);
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort, a.err, a.timeout_ns)) { ok = false; break; }
           uint8_t* b0 = sB + stage * C::kSmemB;
@@ -179,6 +186,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
             if (leader) mbar_arrive_expect_tx(&full[stage], 2 * stage_bytes);
             tma_load_2d_pair(sA + stage * kSmemA, &a.mapA[ti.kind], kb * kBK, a_y, full0 + 8 * stage);
             tma_load_2d_pair(b0, bmap, kb * kBK, b_y, full0 + 8 * stage);
+            if (MODE == kGateUp)
+              tma_load_2d_pair(b0 + (BN / 2) * kBK * 2, bmap + 1, kb * kBK, b_y, full0 + 8 * stage);
           }
           issued[stage] = static_cast<int>(phase);
           if (++stage == S) { stage = 0; phase ^= 1u; }
@@ -197,7 +206,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
       // memory (CG = 1) or in the two CTAs of the pair (CG = 2), so one
       // N = 2*BN MMA reads A once and writes the gate accumulator to columns
       // [0, BN) and the up accumulator to [BN, 2*BN).
-      const uint32_t idesc = idesc_bf16_f32(C::kTileM, n_mma);
+      const uint32_t idesc_full = idesc_bf16_f32(C::kTileM, n_mma);
+      const uint32_t idesc_small = idesc_bf16_f32(128, n_mma);  // pair tile of 128 rows
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -210,6 +220,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort, a.err, a.timeout_ns)) break;
         tc_fence_after();
         const uint32_t d0 = tmem_base + static_cast<uint32_t>(acc) * acc_stride;
+        const uint32_t idesc = ti.small ? idesc_small : idesc_full;
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(&full[stage], phase, abort, a.err, a.timeout_ns)) { ok = false; break; }
           tc_fence_after();
@@ -261,18 +272,33 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
       tc_fence_after();
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                           static_cast<uint32_t>(acc) * acc_stride;
-      const int grow0 = ti.m * C::kTileM + static_cast<int>(rank) * 128 + q * 32;
+      // Rows and columns this warp owns.  A 256-row pair tile (and every CG = 1
+      // tile) keeps row i of the CTA's 128 in TMEM lane i with all n_mma
+      // columns.  A 128-row pair tile keeps the CTA's 64 rows twice: lanes 0-63
+      // hold output columns [0, n_mma/2) and lanes 64-127 hold [n_mma/2, n_mma),
+      // both in TMEM columns [0, n_mma/2).
+      const bool small = ti.small;
+      const int row_in_cta = small ? (q & 1) * 32 : q * 32;
+      const int colhalf = small ? (q >> 1) : 0;           // which half of the columns (small)
+      const int grow0 = ti.m * C::kTileM + static_cast<int>(rank) * (small ? 64 : 128) + row_in_cta;
       const int nvalid = max(0, min(32, ti.rows - grow0));
       if (MODE == kGateUp) {
+        // Output block b covers columns [b*G, b*G + G) with its gate values in
+        // TMEM columns [2bG, 2bG + G) and up values in [2bG + G, 2bG + 2G), G = BN/2.
+        const int G = BN / 2;
         const int orow0 = (ti.kind == 0 ? ti.a_row0 : ti.idx * a.shared_out_stride) + grow0;
         uint8_t* out0 = reinterpret_cast<uint8_t*>(static_cast<uint16_t*>(a.out[ti.kind]) + ti.n * BN);
         const size_t ld_bytes = static_cast<size_t>(a.ld_out[ti.kind]) * 2;
-        for (int c = 64 * half; c < BN; c += 128) {
-#pragma unroll
-          for (int hb = 0; hb < 2; ++hb) {
+        const int nchunk = G / 8;                  // 16-byte chunks per staged row (4 or 8)
+        const int rows_per_st = 32 / nchunk;
+        // 256-row tiles: half h takes block h; 128-row tiles: block colhalf, half 0 only.
+        const int blk = small ? colhalf : half;
+        if (!small || half == 0) {
+          const int tcol = small ? 0 : blk * 2 * G;
+          for (int c = 0; c < G; c += 32) {
             uint32_t g[32], u[32];
-            tmem_ld32(tb + c + 32 * hb, g);
-            tmem_ld32(tb + BN + c + 32 * hb, u);
+            tmem_ld32(tb + tcol + c, g);
+            tmem_ld32(tb + tcol + G + c, u);
             tmem_ld_wait();
             uint32_t p[16];
 #pragma unroll
@@ -284,18 +310,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
                                        a.gate_clamp, a.up_clamp));
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-              const int m = 4 * hb + i;
+              const int m = c / 8 + i;
               *reinterpret_cast<uint4*>(stage_w + lane * 128 + ((m ^ (lane & 7)) << 4)) =
                   make_uint4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
             }
           }
           __syncwarp();
-#pragma unroll
-          for (int s8 = 0; s8 < 8; ++s8) {
-            const int r = 4 * s8 + sr;
+          for (int s8 = 0; s8 < nchunk; ++s8) {
+            const int r = s8 * rows_per_st + lane / nchunk, cc = lane % nchunk;
             if (r < nvalid) {
-              const uint4 v = *reinterpret_cast<const uint4*>(stage_w + r * 128 + ((sc ^ (r & 7)) << 4));
-              *reinterpret_cast<uint4*>(out0 + static_cast<size_t>(orow0 + r) * ld_bytes + c * 2 + 16 * sc) = v;
+              const uint4 v = *reinterpret_cast<const uint4*>(stage_w + r * 128 + ((cc ^ (r & 7)) << 4));
+              *reinterpret_cast<uint4*>(out0 + static_cast<size_t>(orow0 + r) * ld_bytes + blk * G * 2 + 16 * cc) = v;
             }
           }
           __syncwarp();
@@ -305,13 +330,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
         const bool scatter = (MODE == kDown && ti.kind == 0);
         const int my_dest = (scatter && lane < nvalid) ? a.dest_row[ti.a_row0 + grow0 + lane] : 0;
         const int orow0 = (ti.kind == 0 ? ti.a_row0 : ti.idx * a.shared_out_stride) + grow0;
-        float* out0 = static_cast<float*>(a.out[ti.kind]) + ti.n * BN;
+        float* out0 = static_cast<float*>(a.out[ti.kind]) + ti.n * BN + colhalf * (BN / 2);
         const size_t ld = static_cast<size_t>(a.ld_out[ti.kind]);
-        for (int c = 32 * half; c < BN; c += 64) {
+        const int ncols = small ? BN / 2 : BN;
+        for (int c = 32 * half; c < ncols; c += 64) {
           uint32_t v[32];
           tmem_ld32(tb + c, v);
           tmem_ld_wait();
-          if (BN - c >= 32) {
+          if (ncols - c >= 32) {
 #pragma unroll
             for (int m = 0; m < 8; ++m)
               *reinterpret_cast<uint4*>(stage_w + lane * 128 + ((m ^ (lane & 7)) << 4)) =
@@ -332,7 +358,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
             // Narrow tail (router with fewer than 32 columns left): direct stores.
             const size_t orow = scatter ? static_cast<size_t>(my_dest) : static_cast<size_t>(orow0 + lane);
             float4* dst = reinterpret_cast<float4*>(out0 + orow * ld + c);
-            const int nq = (BN - c) / 4;
+            const int nq = (ncols - c) / 4;
 #pragma unroll
             for (int i = 0; i < 8; ++i)
               if (i < nq)

@@ -352,8 +352,8 @@ int moe_init(const moe_config* cfg, const moe_weights* w, moe_handle** out) {
   h->G = cfg->E + h->S;
   h->E_pad = (cfg->E + 15) / 16 * 16;
   // One GEMM configuration per layer shape, never per T.  The expert GEMMs run
-  // on CTA pairs: each CTA loads the gate or the up tile (bn_gu rows) or half
-  // of a down tile (bn_dn / 2 rows).
+  // on CTA pairs: each CTA loads half of a gate/up tile (bn_gu / 2 gate rows and
+  // bn_gu / 2 up rows) or half of a down tile (bn_dn / 2 rows).
   h->bn_gu = (cfg->I % 128 == 0 && h->cfg.I_shared % 128 == 0) ? 128 : 64;
   h->bn_dn = (cfg->D % 256 == 0) ? 256 : (cfg->D % 128 == 0 ? 128 : 64);
   auto fail = [&](int code) { moe_destroy(h); return code; };
@@ -372,11 +372,11 @@ int moe_init(const moe_config* cfg, const moe_weights* w, moe_handle** out) {
       return fail(MOE_ECUDA);
   }
   bool ok = make_map(&h->map_router, h->w_router_pad, c.D, h->w_router_pad ? h->E_pad : 0, h->E_pad) &&
-            make_map(&h->map_wg, w->w_gate, c.D, static_cast<uint64_t>(c.E) * c.I, h->bn_gu) &&
-            make_map(&h->map_wu, w->w_up, c.D, static_cast<uint64_t>(c.E) * c.I, h->bn_gu) &&
+            make_map(&h->map_wg, w->w_gate, c.D, static_cast<uint64_t>(c.E) * c.I, h->bn_gu / 2) &&
+            make_map(&h->map_wu, w->w_up, c.D, static_cast<uint64_t>(c.E) * c.I, h->bn_gu / 2) &&
             make_map(&h->map_wd, w->w_down, c.I, static_cast<uint64_t>(c.E) * c.D, h->bn_dn / 2) &&
-            make_map(&h->map_wsg, w->ws_gate, c.D, static_cast<uint64_t>(h->S) * c.I_shared, h->bn_gu) &&
-            make_map(&h->map_wsu, w->ws_up, c.D, static_cast<uint64_t>(h->S) * c.I_shared, h->bn_gu) &&
+            make_map(&h->map_wsg, w->ws_gate, c.D, static_cast<uint64_t>(h->S) * c.I_shared, h->bn_gu / 2) &&
+            make_map(&h->map_wsu, w->ws_up, c.D, static_cast<uint64_t>(h->S) * c.I_shared, h->bn_gu / 2) &&
             make_map(&h->map_wsd, w->ws_down, c.I_shared, static_cast<uint64_t>(h->S) * c.D, h->bn_dn / 2);
   if (!ok) return fail(MOE_ECUDA);
   *out = h;
