@@ -145,11 +145,16 @@ class MoELayer:
         self.handle = h
 
     def close(self):
-        if getattr(self, "handle", None):
-            lib().moe_destroy(self.handle)
+        h = getattr(self, "handle", None)
+        if h:
             self.handle = None
+            lib().moe_destroy(h)
 
-    __del__ = close
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:  # interpreter shutdown: the library may already be unloaded
+            pass
 
     def workspace_size(self, T: int) -> int:
         return int(lib().moe_workspace_size(self.handle, T))
