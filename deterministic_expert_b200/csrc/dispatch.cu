@@ -6,8 +6,9 @@
 // dependence).  Integer-only; the result is unique.
 //
 //   dispatch  block b (128 tokens) reads the per-block expert counts the router
-//             wrote, forms the exclusive prefix over experts (offsets) and over
-//             the blocks before it, then ranks each of its (token, slot) pairs
+//             wrote (all blocks' rows at once, 16-byte loads), forms the exclusive
+//             prefix over experts (offsets, a block scan) and over the blocks
+//             before it, then ranks each of its (token, slot) pairs
 //             among the block's earlier tokens that chose the same expert (a
 //             token bitmask per expert + popcount): grouped row
 //             p = offsets[e] + (pairs of e in earlier tokens).  Block 0 also
@@ -19,74 +20,126 @@
 namespace moe {
 namespace {
 
+// Exclusive prefix sum of in[0..n) into out[0..n], out[n] = total, by the
+// kDispatchRows threads of the block (n <= kDispatchRows * kScanPer): thread i
+// scans a run of consecutive items, a warp scan and the warp totals (left to
+// right) give the run's base.  Integer only, so the order is immaterial.
+constexpr int kScanPer = 3;
+__device__ __forceinline__ void block_exclusive_scan(const int* in, int* out, int n, int* warp_tot) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int per = (n + kDispatchRows - 1) / kDispatchRows;
+  const int i0 = tid * per;
+  int v[kScanPer];
+  int run = 0;
+#pragma unroll
+  for (int u = 0; u < kScanPer; ++u) {
+    v[u] = (u < per && i0 + u < n) ? in[i0 + u] : 0;
+    run += v[u];
+  }
+  int incl = run;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) warp_tot[warp] = incl;
+  __syncthreads();
+  int base = incl - run;
+  int all = 0;
+#pragma unroll
+  for (int w = 0; w < kDispatchRows / 32; ++w) {
+    if (w < warp) base += warp_tot[w];
+    all += warp_tot[w];
+  }
+#pragma unroll
+  for (int u = 0; u < kScanPer; ++u)
+    if (u < per && i0 + u < n) { out[i0 + u] = base; base += v[u]; }
+  if (tid == 0) out[n] = all;
+  __syncthreads();
+}
+
 __global__ void __launch_bounds__(kDispatchRows) k_dispatch(const DispatchArgs a) {
   constexpr int kWords = kDispatchRows / 32;
-  __shared__ int base[256];    // offsets[e] + pairs of e in blocks before this one
+  constexpr int kMaxG = 256 + 8;
+  __shared__ int before[256];  // pairs of e in the blocks before this one
   __shared__ int total[256];
   __shared__ int offs[257];
+  __shared__ int cnt[kMaxG], tstart[kMaxG + 1];
+  __shared__ int warp_tot[kDispatchRows / 32];
   __shared__ uint32_t mask[256][kWords];
+  const int tid = threadIdx.x;
+  const int b = blockIdx.x;
+  const int nb = (a.T + kDispatchRows - 1) / kDispatchRows;
+  for (int e = tid; e < a.E; e += kDispatchRows) { before[e] = 0; total[e] = 0; }
+  for (int i = tid; i < a.E * kWords; i += kDispatchRows) mask[i / kWords][i % kWords] = 0;
   griddep_wait();
   griddep_launch();
-  const int nb = (a.T + kDispatchRows - 1) / kDispatchRows;
-  const int b = blockIdx.x;
-  for (int e = threadIdx.x; e < a.E; e += blockDim.x) {
-    int before = 0, all = 0;
-    for (int q = 0; q < nb; ++q) {
-      const int c = a.block_counts[q * a.E + e];
-      if (q < b) before += c;
-      all += c;
-    }
-    base[e] = before;
-    total[e] = all;
-  }
-  for (int i = threadIdx.x; i < a.E * kWords; i += blockDim.x) mask[i / kWords][i % kWords] = 0;
   __syncthreads();
-  if (threadIdx.x == 0) {
-    int run = 0;
-    for (int q = 0; q < a.E; ++q) { offs[q] = run; run += total[q]; }
-    offs[a.E] = run;
+  // Column sums of the [nb, E4] block counts, 16-byte loads eight at a time.
+  {
+    const int row4 = a.E4 / 4;
+    const int n4 = nb * row4;
+    const int4* bc4 = reinterpret_cast<const int4*>(a.block_counts);
+    for (int f0 = tid; f0 < n4; f0 += 8 * kDispatchRows) {
+      int4 v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int f = f0 + u * kDispatchRows;
+        v[u] = f < n4 ? bc4[f] : make_int4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int f = f0 + u * kDispatchRows;
+        if (f >= n4) continue;
+        const int q = f / row4, e = (f - q * row4) * 4;
+        const int c[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+        for (int z = 0; z < 4; ++z) {
+          if (c[z] == 0 || e + z >= a.E) continue;
+          atomicAdd(&total[e + z], c[z]);
+          if (q < b) atomicAdd(&before[e + z], c[z]);
+        }
+      }
+    }
   }
-  const int tl = threadIdx.x;
-  const int t = b * kDispatchRows + tl;
+  __syncthreads();
+  block_exclusive_scan(total, offs, a.E, warp_tot);
+
+  const int t = b * kDispatchRows + tid;
   if (t < a.T)
-    for (int j = 0; j < a.k; ++j) atomicOr(&mask[a.idx[t * a.k + j]][tl >> 5], 1u << (tl & 31));
+    for (int j = 0; j < a.k; ++j) atomicOr(&mask[a.idx[t * a.k + j]][tid >> 5], 1u << (tid & 31));
   __syncthreads();
   if (t < a.T) {
     for (int j = 0; j < a.k; ++j) {
       const int e = a.idx[t * a.k + j];
-      int rank = __popc(mask[e][tl >> 5] & ((1u << (tl & 31)) - 1u));
-      for (int w = 0; w < (tl >> 5); ++w) rank += __popc(mask[e][w]);
-      const int p = offs[e] + base[e] + rank;
+      int rank = __popc(mask[e][tid >> 5] & ((1u << (tid & 31)) - 1u));
+      for (int w = 0; w < (tid >> 5); ++w) rank += __popc(mask[e][w]);
+      const int p = offs[e] + before[e] + rank;
       a.dest_row[p] = t * a.k + j;
       a.src_token[p] = t;
     }
   }
   if (b == 0) {
-    for (int q = threadIdx.x; q <= a.E; q += blockDim.x) a.offsets[q] = offs[q];
-    for (int e = threadIdx.x; e < a.E; e += blockDim.x) {
+    for (int q = tid; q <= a.E; q += kDispatchRows) a.offsets[q] = offs[q];
+    for (int e = tid; e < a.E; e += kDispatchRows) {
       a.counts[e] = total[e];
       if (a.user_counts) a.user_counts[e] = total[e];
     }
-    if (threadIdx.x == 0) {
-      // Tile lists: routed groups first (experts in index order), then shared.
-      const int mt_shared = (a.T + a.tile_m - 1) / a.tile_m;
-      int gu = 0, dn = 0;
-      for (int q = 0; q < a.E; ++q) {
-        a.tiles_gu[q] = gu;
-        a.tiles_dn[q] = dn;
-        const int mt = (total[q] + a.tile_m - 1) / a.tile_m;
-        gu += mt * a.gu_ntiles_routed;
-        dn += mt * a.dn_ntiles;
-      }
-      for (int s = 0; s < a.S; ++s) {
-        a.tiles_gu[a.E + s] = gu;
-        a.tiles_dn[a.E + s] = dn;
-        gu += mt_shared * a.gu_ntiles_shared;
-        dn += mt_shared * a.dn_ntiles;
-      }
-      a.tiles_gu[a.E + a.S] = gu;
-      a.tiles_dn[a.E + a.S] = dn;
-    }
+    // Tile lists: routed groups first (experts in index order), then shared.
+    const int G = a.E + a.S;
+    const int mt_shared = (a.T + a.tile_m - 1) / a.tile_m;
+    for (int g = tid; g < G; g += kDispatchRows)
+      cnt[g] = (g < a.E ? (total[g] + a.tile_m - 1) / a.tile_m * a.gu_ntiles_routed
+                        : mt_shared * a.gu_ntiles_shared);
+    __syncthreads();
+    block_exclusive_scan(cnt, tstart, G, warp_tot);
+    for (int g = tid; g <= G; g += kDispatchRows) a.tiles_gu[g] = tstart[g];
+    __syncthreads();
+    for (int g = tid; g < G; g += kDispatchRows)
+      cnt[g] = (g < a.E ? (total[g] + a.tile_m - 1) / a.tile_m : mt_shared) * a.dn_ntiles;
+    __syncthreads();
+    block_exclusive_scan(cnt, tstart, G, warp_tot);
+    for (int g = tid; g <= G; g += kDispatchRows) a.tiles_dn[g] = tstart[g];
   }
 }
 

@@ -44,6 +44,8 @@ namespace moe {
 namespace {
 
 constexpr uint32_t kTmemCols = 512;
+constexpr int kRingBytes = kStages * (kSmemA + kSmemBMax);  // shared memory of the stage ring
+constexpr int kRingMax = 8;                                 // most stages any variant uses
 constexpr unsigned long long kDrainNs = 200ull * 1000 * 1000;  // 200 ms
 
 template <int CG>
@@ -51,7 +53,7 @@ struct Cfg {
   static constexpr int kTileM = 128 * CG;                                 // rows per tile (pair)
   static constexpr int kSmemB = CG == 1 ? 256 * kBK * 2 : 128 * kBK * 2;  // B bytes per CTA stage
   static constexpr int kStage = kSmemA + kSmemB;
-  static constexpr int kStagesN = (kStages * (kSmemA + kSmemBMax)) / kStage;  // 4 or 6
+  static constexpr int kStagesN = kRingBytes / kStage;  // 4 or 6
 };
 
 struct Tile {
@@ -99,16 +101,21 @@ __device__ __forceinline__ float silu_clamped_product(float g, float u, float cg
 template <int MODE, int CG>
 __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_constant__ GemmArgs a) {
   using C = Cfg<CG>;
-  constexpr int S = C::kStagesN;
+  // Stage ring.  The expert GEMMs use C::kStagesN stages of kSmemA + C::kSmemB
+  // bytes; the router, whose B tile is only E_pad rows, packs as many stages of
+  // kSmemA + E_pad * 128 bytes as fit (up to kRingMax), so one CTA walking the
+  // whole K keeps more loads in flight.  The stage count never changes a result.
+  const int sb_bytes = MODE == kRouter ? a.BN * kBK * 2 : C::kSmemB;
+  const int S = MODE == kRouter ? min(kRingMax, kRingBytes / (kSmemA + sb_bytes)) : C::kStagesN;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sA = smem;                              // S x kSmemA
-  uint8_t* sB = smem + S * kSmemA;                 // S x kSmemB
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * (kSmemA + kSmemBMax));
+  uint8_t* sB = smem + S * kSmemA;                 // S x sb_bytes
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kRingBytes);
   uint64_t* full = bars;
-  uint64_t* empty = bars + S;
-  uint64_t* tfull = bars + 2 * S;
+  uint64_t* empty = bars + kRingMax;
+  uint64_t* tfull = bars + 2 * kRingMax;
   uint64_t* tempty = tfull + 2;
   uint64_t* tdone = tempty + 2;
   uint8_t* epi = reinterpret_cast<uint8_t*>(bars) + 256;  // kEpiWarps x kEpiBytes
@@ -156,7 +163,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
-      int issued[S];
+      int issued[kRingMax];
       for (int s = 0; s < S; ++s) issued[s] = -1;
       bool ok = true;
       for (int t = cluster_id; ok && t < total; t += n_clusters) {
@@ -174,7 +181,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
         if (CG == 2) b_y += static_cast<int>(rank) * (BN / 2);
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort, a.err, a.timeout_ns)) { ok = false; break; }
-          uint8_t* b0 = sB + stage * C::kSmemB;
+          uint8_t* b0 = sB + stage * sb_bytes;
           if (CG == 1) {
             mbar_arrive_expect_tx(&full[stage], stage_bytes);
             tma_load_2d(sA + stage * kSmemA, &a.mapA[ti.kind], kb * kBK, a_y, &full[stage]);
@@ -225,7 +232,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
           if (!mbar_wait(&full[stage], phase, abort, a.err, a.timeout_ns)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a_addr = smem_u32(sA + stage * kSmemA);
-          const uint32_t b_addr = smem_u32(sB + stage * C::kSmemB);
+          const uint32_t b_addr = smem_u32(sB + stage * sb_bytes);
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk) {
             const uint64_t ad = sw128_kmajor_desc(a_addr + kk * 32);

@@ -50,7 +50,7 @@ Layout layout(const moe_handle* h, int T) {
   L.logits = take(c.router == MOE_ROUTER_HASH ? 0 : Tz * h->E_pad * 4);
   L.tidx = take(Tz * c.k * 4);
   L.tw = take(Tz * c.k * 4);
-  L.bcount = take(nb * c.E * 4);
+  L.bcount = take(nb * ((c.E + 3) / 4 * 4) * 4);
   L.counts = take(static_cast<size_t>(c.E) * 4);
   L.offsets = take(static_cast<size_t>(c.E + 1) * 4);
   L.tiles_gu = take(static_cast<size_t>(h->G + 1) * 4);
@@ -208,8 +208,9 @@ int forward_impl(moe_handle* h, int T, const uint16_t* x, const uint16_t* residu
   // 0. input RMSNorm (also clears the device error word and the histogram)
   int32_t* bcount = reinterpret_cast<int32_t*>(ws + L.bcount);
   const int nblk = (T + kDispatchRows - 1) / kDispatchRows;
+  const int E4 = (c.E + 3) / 4 * 4;
   prof.begin(0);
-  MOE_TRY(launch_rmsnorm_rows(x, h->w.g_in, xn, T, c.D, c.eps, err, bcount, nblk * c.E, s));
+  MOE_TRY(launch_rmsnorm_rows(x, h->w.g_in, xn, T, c.D, c.eps, err, bcount, nblk * E4, s));
   prof.end(0);
 
   // 1. router logits on the tensor cores
@@ -237,17 +238,15 @@ int forward_impl(moe_handle* h, int T, const uint16_t* x, const uint16_t* residu
   ra.logits = logits; ra.E_pad = h->E_pad; ra.bias = h->w.router_bias; ra.token_ids = token_ids;
   ra.router = c.router; ra.E = c.E; ra.k = c.k; ra.renormalize = c.renormalize;
   ra.routed_scale = c.routed_scale; ra.hash_mult = c.hash_mult; ra.idx = tidx; ra.w = tw;
-  ra.block_counts = bcount; ra.T = T;
+  ra.block_counts = bcount; ra.E4 = E4; ra.user_idx = out_idx; ra.user_w = out_w; ra.T = T;
   prof.begin(2);
   MOE_TRY(launch_router_topk(ra, s));
   prof.end(2);
-  if (out_idx) MOE_TRY(cudaMemcpyAsync(out_idx, tidx, static_cast<size_t>(TK) * 4, cudaMemcpyDeviceToDevice, s));
-  if (out_w) MOE_TRY(cudaMemcpyAsync(out_w, tw, static_cast<size_t>(TK) * 4, cudaMemcpyDeviceToDevice, s));
 
   // 3. offsets, stable scatter and the expert-GEMM tile lists
   DispatchArgs da;
   da.idx = tidx; da.T = T; da.k = c.k; da.E = c.E; da.S = h->S;
-  da.block_counts = bcount;
+  da.block_counts = bcount; da.E4 = E4;
   da.counts = reinterpret_cast<int32_t*>(ws + L.counts);
   da.offsets = offsets; da.user_counts = out_counts; da.tiles_gu = tiles_gu; da.tiles_dn = tiles_dn;
   da.gu_ntiles_routed = c.I / h->bn_gu;

@@ -111,7 +111,10 @@ struct RouterArgs {
   uint32_t hash_mult;
   int32_t* idx;             // [T, k]
   float* w;                 // [T, k]
-  int32_t* block_counts;    // [ceil(T / 128), E], zeroed beforehand
+  int32_t* block_counts;    // [ceil(T / 128), E4], zeroed beforehand
+  int E4;                   // row stride of block_counts: E rounded up to 4
+  int32_t* user_idx;        // [T, k] copy of idx for the caller, or NULL
+  float* user_w;            // [T, k] copy of w for the caller, or NULL
   int T;
 };
 cudaError_t launch_router_topk(const RouterArgs& a, cudaStream_t s);
@@ -121,7 +124,8 @@ constexpr int kDispatchRows = 128;  // tokens per dispatch block (= one router G
 struct DispatchArgs {
   const int32_t* idx;   // [T, k]
   int T, k, E, S;
-  const int32_t* block_counts;  // [nb, E] expert counts of each 128-token block
+  const int32_t* block_counts;  // [nb, E4] expert counts of each 128-token block
+  int E4;                       // row stride of block_counts (E rounded up to 4)
   int32_t* counts;        // [E]
   int32_t* offsets;       // [E + 1]
   int32_t* user_counts;   // [E] or NULL

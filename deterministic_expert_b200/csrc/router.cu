@@ -39,15 +39,19 @@ __global__ void __launch_bounds__(256) k_router_topk(const RouterArgs a) {
   const int lane = threadIdx.x & 31;
   if (t >= a.T) return;
   const int k = a.k, E = a.E;
-  int32_t* hist = a.block_counts + static_cast<size_t>(t / kDispatchRows) * E;
+  int32_t* hist = a.block_counts + static_cast<size_t>(t / kDispatchRows) * a.E4;
 
   if (a.router == MOE_ROUTER_HASH) {
     if (lane < k) {
       const uint32_t h = static_cast<uint32_t>(a.token_ids[t]) * a.hash_mult;  // mod 2^32
       const int e0 = static_cast<int>(h % static_cast<uint32_t>(E));
-      a.idx[t * k + lane] = (e0 + lane) % E;
-      a.w[t * k + lane] = a.routed_scale / static_cast<float>(k);
-      atomicAdd(hist + (e0 + lane) % E, 1);
+      const int e = (e0 + lane) % E;
+      const float w = a.routed_scale / static_cast<float>(k);
+      a.idx[t * k + lane] = e;
+      a.w[t * k + lane] = w;
+      if (a.user_idx) a.user_idx[t * k + lane] = e;
+      if (a.user_w) a.user_w[t * k + lane] = w;
+      atomicAdd(hist + e, 1);
     }
     return;
   }
@@ -94,44 +98,60 @@ __global__ void __launch_bounds__(256) k_router_topk(const RouterArgs a) {
     denom = s;
   }
 
+  // k rounds of a warp arg-max; the loops run to the compile-time bound 16 so
+  // the chosen values stay in registers.
   uint32_t taken = 0;
   float chosen_v[16];
   int chosen_e[16];
-  for (int j = 0; j < k; ++j) {
-    float bk = -INFINITY;
-    int be = 0x7fffffff, bi = -1;
 #pragma unroll
-    for (int i = 0; i < kMaxPerLane; ++i) {
-      const int e = lane + 32 * i;
-      if (e < E && !(taken & (1u << i)) && better(key[i], e, bk, be)) { bk = key[i]; be = e; bi = i; }
-    }
-    float bv = bi >= 0 ? val[bi] : 0.f;
+  for (int j = 0; j < 16; ++j) {
+    chosen_v[j] = 0.f;
+    chosen_e[j] = 0;
+    if (j < k) {
+      float bk = -INFINITY;
+      int be = 0x7fffffff, bi = -1;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ok = __shfl_xor_sync(0xffffffffu, bk, o);
-      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      if (better(ok, oe, bk, be)) { bk = ok; be = oe; bv = ov; }
+      for (int i = 0; i < kMaxPerLane; ++i) {
+        const int e = lane + 32 * i;
+        if (e < E && !(taken & (1u << i)) && better(key[i], e, bk, be)) { bk = key[i]; be = e; bi = i; }
+      }
+      float bv = 0.f;
+#pragma unroll
+      for (int i = 0; i < kMaxPerLane; ++i)
+        if (i == bi) bv = val[i];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ok = __shfl_xor_sync(0xffffffffu, bk, o);
+        const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        if (better(ok, oe, bk, be)) { bk = ok; be = oe; bv = ov; }
+      }
+      if ((be & 31) == lane) taken |= 1u << (be >> 5);
+      chosen_e[j] = be;
+      chosen_v[j] = bv;
     }
-    if ((be & 31) == lane) taken |= 1u << (be >> 5);
-    chosen_e[j] = be;
-    chosen_v[j] = bv;
   }
 
   float norm = denom;
   if (a.renormalize) {
     norm = 0.f;
-    for (int j = 0; j < k; ++j) norm += chosen_v[j];
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+      if (j < k) norm += chosen_v[j];
   }
-  for (int j = lane; j < k; j += 32) {
-    float w = 0.f;
-    int e = 0;
-    for (int q = 0; q < k; ++q)
-      if (q == j) { w = chosen_v[q]; e = chosen_e[q]; }
-    a.idx[t * k + j] = e;
+  // Lane j < k writes slot j.
+  float w = 0.f;
+  int e = 0;
+#pragma unroll
+  for (int q = 0; q < 16; ++q)
+    if (q == lane) { w = chosen_v[q]; e = chosen_e[q]; }
+  if (lane < k) {
+    const float wn = ((a.router == MOE_ROUTER_SOFTMAX || a.renormalize) ? w / norm : w) * a.routed_scale;
+    a.idx[t * k + lane] = e;
+    a.w[t * k + lane] = wn;
+    if (a.user_idx) a.user_idx[t * k + lane] = e;
+    if (a.user_w) a.user_w[t * k + lane] = wn;
     atomicAdd(hist + e, 1);
-    const float wn = (a.router == MOE_ROUTER_SOFTMAX || a.renormalize) ? w / norm : w;
-    a.w[t * k + j] = wn * a.routed_scale;
   }
 }
 

@@ -1,6 +1,8 @@
 // Row kernels with a fixed thread layout: one CTA of 256 threads per token
-// row, thread i always owning the 4-element chunks i, i + 256, i + 512, ...
-// of the row.  The sum of squares for RMSNorm goes through the fixed tree of
+// row, thread i always owning the chunks i, i + 256, i + 512, ... of the row
+// (8 elements per chunk for the input norm and the partial reduce, whose
+// operands are bf16 and load as 16 bytes; 4 for the combine, whose fp32 slot
+// rows load as 16 bytes).  The sum of squares for RMSNorm goes through the fixed tree of
 // block_sum_fixed (per-thread sum in element order, a 5-step butterfly with
 // masks 16..1, warp partials added left to right), the layout the Fireworks
 // parity post (Chinese translation), Trap 2, says must not change with the
@@ -24,14 +26,31 @@ namespace {
 
 constexpr int kMaxChunks = 16;  // D <= 4 * 256 * 16 = 16384
 
-// Chunks per thread for a row of D elements: the smallest of 1, 2, 4, 8, 16
-// with 4 * 256 * NC >= D.  It depends on D only, so thread i owns the same
-// chunks i, i + 256, ... whatever T is; the template bound only trims
-// registers (kernels for small D keep fewer live values).
-inline int chunks_for(int D) {
+// Chunks per thread for a row of D elements in chunks of W elements: the
+// smallest of 1, 2, 4, 8, 16 with W * 256 * NC >= D.  It depends on D only, so
+// thread i owns the same chunks i, i + 256, ... whatever T is; the template
+// bound only trims registers (kernels for small D keep fewer live values).
+inline int chunks_for(int D, int W = 4) {
   int nc = 1;
-  while (nc < kMaxChunks && 4 * kRowThreads * nc < D) nc *= 2;
+  while (nc < kMaxChunks && W * kRowThreads * nc < D) nc *= 2;
   return nc;
+}
+
+struct f8 {
+  float v[8];
+};
+
+__device__ __forceinline__ f8 ld_bf16x8(const uint16_t* p) {
+  const uint4 u = *reinterpret_cast<const uint4*>(p);
+  f8 r;
+  r.v[0] = bf16_lo(u.x); r.v[1] = bf16_hi(u.x); r.v[2] = bf16_lo(u.y); r.v[3] = bf16_hi(u.y);
+  r.v[4] = bf16_lo(u.z); r.v[5] = bf16_hi(u.z); r.v[6] = bf16_lo(u.w); r.v[7] = bf16_hi(u.w);
+  return r;
+}
+
+__device__ __forceinline__ void st_bf16x8(uint16_t* p, const float (&v)[8]) {
+  *reinterpret_cast<uint4*>(p) = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+                                            pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
 }
 
 __device__ __forceinline__ float4 ld_bf16x4(const uint16_t* p) {
@@ -68,19 +87,22 @@ __global__ void __launch_bounds__(kRowThreads) k_rmsnorm_rows(const uint16_t* __
   for (int i = blockIdx.x * kRowThreads + threadIdx.x; i < zero_words; i += gridDim.x * kRowThreads)
     zero[i] = 0;
   const size_t row = blockIdx.x;
-  const int nch = D / 4;
+  const int nch = D / 8;
   const uint16_t* xr = x + row * D;
-  float4 v[NC];
+  f8 v[NC];
   double ss = 0.0;
 #pragma unroll
   for (int i = 0; i < NC; ++i) {
     const int c = threadIdx.x + i * kRowThreads;
+    if (c < nch) v[i] = ld_bf16x8(xr + 8 * c);
+  }
+#pragma unroll
+  for (int i = 0; i < NC; ++i) {
+    const int c = threadIdx.x + i * kRowThreads;
     if (c < nch) {
-      v[i] = ld_bf16x4(xr + 4 * c);
-      ss = fma(static_cast<double>(v[i].x), static_cast<double>(v[i].x), ss);
-      ss = fma(static_cast<double>(v[i].y), static_cast<double>(v[i].y), ss);
-      ss = fma(static_cast<double>(v[i].z), static_cast<double>(v[i].z), ss);
-      ss = fma(static_cast<double>(v[i].w), static_cast<double>(v[i].w), ss);
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        ss = fma(static_cast<double>(v[i].v[q]), static_cast<double>(v[i].v[q]), ss);
     }
   }
   // The squares of bf16 values are exact in fp64 and the fp64 sum is exact to
@@ -93,9 +115,11 @@ __global__ void __launch_bounds__(kRowThreads) k_rmsnorm_rows(const uint16_t* __
   for (int i = 0; i < NC; ++i) {
     const int c = threadIdx.x + i * kRowThreads;
     if (c < nch) {
-      const float4 gg = ld_bf16x4(g + 4 * c);
-      st_bf16x4(yr + 4 * c, v[i].x * inv * gg.x, v[i].y * inv * gg.y, v[i].z * inv * gg.z,
-                v[i].w * inv * gg.w);
+      const f8 gg = ld_bf16x8(g + 8 * c);
+      float o[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) o[q] = v[i].v[q] * inv * gg.v[q];
+      st_bf16x8(yr + 8 * c, o);
     }
   }
 }
@@ -168,28 +192,56 @@ __global__ void __launch_bounds__(kRowThreads) k_reduce_partials(
   griddep_wait();
   griddep_launch();
   const size_t t = blockIdx.x;
-  const int nch = D / 4;
-  float4 r[NC];
+  const int nch = D / 8;
+  f8 r[NC];
   float ss = 0.f;
 #pragma unroll
   for (int i = 0; i < NC; ++i) {
     const int c = threadIdx.x + i * kRowThreads;
     if (c < nch) {
-      const size_t off = t * D + 4 * c;
-      float4 acc = ld_bf16x4(parts.p[0] + off);
-      for (int p = 1; p < P; ++p) {  // r0 + r1 + ... + r_{P-1}, left to right
-        const float4 v = ld_bf16x4(parts.p[p] + off);
-        acc.x = __fadd_rn(acc.x, v.x); acc.y = __fadd_rn(acc.y, v.y);
-        acc.z = __fadd_rn(acc.z, v.z); acc.w = __fadd_rn(acc.w, v.w);
+      const size_t off = t * D + 8 * c;
+      // Issue every partial's load before the first add.
+      uint4 raw[8];
+#pragma unroll
+      for (int p = 0; p < 8; ++p)
+        if (p < P) raw[p] = *reinterpret_cast<const uint4*>(parts.p[p] + off);
+      const f8 res = ld_bf16x8(residual + off);
+      const uint32_t* w0 = reinterpret_cast<const uint32_t*>(&raw[0]);
+      float acc[8];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) { acc[2 * q] = bf16_lo(w0[q]); acc[2 * q + 1] = bf16_hi(w0[q]); }
+#pragma unroll
+      for (int p = 1; p < 8; ++p) {  // r0 + r1 + ... + r_{P-1}, left to right
+        if (p < P) {
+          const uint32_t* wp = reinterpret_cast<const uint32_t*>(&raw[p]);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            acc[2 * q] = __fadd_rn(acc[2 * q], bf16_lo(wp[q]));
+            acc[2 * q + 1] = __fadd_rn(acc[2 * q + 1], bf16_hi(wp[q]));
+          }
+        }
       }
-      const float4 res = ld_bf16x4(residual + off);
-      r[i] = make_float4(__fadd_rn(acc.x, res.x), __fadd_rn(acc.y, res.y),
-                         __fadd_rn(acc.z, res.z), __fadd_rn(acc.w, res.w));
-      st_bf16x4(out_residual + off, r[i].x, r[i].y, r[i].z, r[i].w);
-      ss = sumsq4(ss, r[i]);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        r[i].v[q] = __fadd_rn(acc[q], res.v[q]);
+        ss = fmaf(r[i].v[q], r[i].v[q], ss);
+      }
+      st_bf16x8(out_residual + off, r[i].v);
     }
   }
-  norm_store(r, ss, red, g, out_norm + t * D, D, eps);
+  const float inv = inv_rms(block_sum_fixed(ss, red), D, eps);
+  uint16_t* on = out_norm + t * D;
+#pragma unroll
+  for (int i = 0; i < NC; ++i) {
+    const int c = threadIdx.x + i * kRowThreads;
+    if (c < nch) {
+      const f8 gg = ld_bf16x8(g + 8 * c);
+      float o[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) o[q] = r[i].v[q] * inv * gg.v[q];
+      st_bf16x8(on + 8 * c, o);
+    }
+  }
 }
 
 // Count bf16 elements of a whose bits differ from the matching row of b
@@ -259,7 +311,7 @@ cudaError_t launch_rmsnorm_rows(const uint16_t* x, const uint16_t* g, uint16_t* 
     return launch_k(kernel, dim3(T), dim3(kRowThreads), 0, s, false, x, g, y, D, eps, err_to_clear,
                     zero, zero_words);
   };
-  switch (chunks_for(D)) {
+  switch (chunks_for(D, 8)) {
     case 1: return go(k_rmsnorm_rows<1>);
     case 2: return go(k_rmsnorm_rows<2>);
     case 4: return go(k_rmsnorm_rows<4>);
@@ -294,7 +346,7 @@ cudaError_t launch_reduce_partials(const PartialPtrs& parts, int P, const uint16
     return launch_k(kernel, dim3(T), dim3(kRowThreads), 0, s, false, parts, P, residual, g, out_norm,
                     out_residual, D, eps);
   };
-  switch (chunks_for(D)) {
+  switch (chunks_for(D, 8)) {
     case 1: return go(k_reduce_partials<1>);
     case 2: return go(k_reduce_partials<2>);
     case 4: return go(k_reduce_partials<4>);
