@@ -170,8 +170,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
         Tile ti;
         decode_tile<CG>(a, t, ti);
         const int nkb = a.k_kind[ti.kind] / kBK;
-        // A: this CTA's rows of the tile (128, or 64 in a 128-row pair tile).
+        // A: this CTA's rows of the tile (128, or 64 in a 128-row pair tile,
+        // loaded with the 64-row box so no unused rows cross into shared memory).
         const int a_y = ti.a_row0 + ti.m * C::kTileM + static_cast<int>(rank) * (ti.small ? 64 : 128);
+        const CUtensorMap* amap = (CG == 2 && ti.small) ? &a.mapA64[ti.kind] : &a.mapA[ti.kind];
+        const uint32_t tx = (CG == 2 && ti.small) ? stage_bytes - kSmemA / 2 : stage_bytes;
         int b_y = ti.idx * a.n_kind[ti.kind] + ti.n * BN;
         const CUtensorMap* bmap = &a.mapB[ti.kind * 2];
         // Pair B halves: gate/up - the CTA of rank r loads gate rows and up rows
@@ -190,8 +193,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
               tma_load_2d(b0 + b_rows * kBK * 2, bmap + 1, kb * kBK, b_y, &full[stage]);
           } else {
             // The even CTA expects the bytes of both CTAs on its barrier.
-            if (leader) mbar_arrive_expect_tx(&full[stage], 2 * stage_bytes);
-            tma_load_2d_pair(sA + stage * kSmemA, &a.mapA[ti.kind], kb * kBK, a_y, full0 + 8 * stage);
+            if (leader) mbar_arrive_expect_tx(&full[stage], 2 * tx);
+            tma_load_2d_pair(sA + stage * kSmemA, amap, kb * kBK, a_y, full0 + 8 * stage);
             tma_load_2d_pair(b0, bmap, kb * kBK, b_y, full0 + 8 * stage);
             if (MODE == kGateUp)
               tma_load_2d_pair(b0 + (BN / 2) * kBK * 2, bmap + 1, kb * kBK, b_y, full0 + 8 * stage);
