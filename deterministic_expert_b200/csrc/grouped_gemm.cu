@@ -63,12 +63,16 @@ struct Tile {
   int a_row0; // first A row of the group
   int m, n;   // tile coordinates within the group
   bool small; // pair tile with 128 rows (M = 128): the group's last <= 128 rows
+  bool swap;  // operand-swapped pair tile: weights are the M = 256 operand, the
+              // group's last r < 256 rows the N = nt operand (nt = r rounded up to 16)
+  int nt;
 };
 
 template <int CG>
 __device__ __forceinline__ void decode_tile(const GemmArgs& a, int t, Tile& ti) {
   if (a.tile_start == nullptr) {
     ti.kind = 0; ti.idx = 0; ti.rows = a.T; ti.a_row0 = 0; ti.m = t; ti.n = 0; ti.small = false;
+    ti.swap = false; ti.nt = 0;
     return;
   }
   // Largest g with tile_start[g] <= t; tile_start[0] = 0 <= t < tile_start[G].
@@ -87,7 +91,10 @@ __device__ __forceinline__ void decode_tile(const GemmArgs& a, int t, Tile& ti) 
   const int mt = (ti.rows + Cfg<CG>::kTileM - 1) / Cfg<CG>::kTileM;
   ti.n = local / mt;
   ti.m = local - ti.n * mt;
-  ti.small = CG == 2 && ti.rows - ti.m * Cfg<CG>::kTileM <= 128;
+  const int r = ti.rows - ti.m * Cfg<CG>::kTileM;
+  ti.swap = CG == 2 && a.swap_ok && r < 256;
+  ti.nt = ti.swap ? (r + 15) & ~15 : 0;
+  ti.small = CG == 2 && !ti.swap && r <= 128;
 }
 
 // SiLU(min(g, c_g)) * clamp(u, -c_u, c_u) in fp32 with the fast exponential
@@ -118,6 +125,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
   uint64_t* tfull = bars + 2 * kRingMax;
   uint64_t* tempty = tfull + 2;
   uint64_t* tdone = tempty + 2;
+  uint64_t* xfull = tdone + 1;   // [4] swapped gate/up tiles: up values staged for the gate warp
+  uint64_t* xempty = xfull + 4;  // [4] ... and read back
   uint8_t* epi = reinterpret_cast<uint8_t*>(bars) + 256;  // kEpiWarps x kEpiBytes
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
@@ -129,6 +138,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
     for (int s = 0; s < S; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
     for (int b = 0; b < 2; ++b) { mbar_init(&tfull[b], 1); mbar_init(&tempty[b], CG * kEpiWarps); }
     mbar_init(tdone, 1);
+    for (int p = 0; p < 4; ++p) { mbar_init(&xfull[p], 1); mbar_init(&xempty[p], 1); }
     abort_flag = 0;
     fence_barrier_init();
   }
@@ -172,9 +182,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
         const int nkb = a.k_kind[ti.kind] / kBK;
         // A: this CTA's rows of the tile (128, or 64 in a 128-row pair tile,
         // loaded with the 64-row box so no unused rows cross into shared memory).
-        const int a_y = ti.a_row0 + ti.m * C::kTileM + static_cast<int>(rank) * (ti.small ? 64 : 128);
-        const CUtensorMap* amap = (CG == 2 && ti.small) ? &a.mapA64[ti.kind] : &a.mapA[ti.kind];
-        const uint32_t tx = (CG == 2 && ti.small) ? stage_bytes - kSmemA / 2 : stage_bytes;
+        // Swapped tile: this CTA's nt / 2 token rows (the B operand's half).
+        const int a_rows = ti.swap ? ti.nt / 2 : (ti.small ? 64 : 128);
+        const int a_y = ti.a_row0 + ti.m * C::kTileM + static_cast<int>(rank) * a_rows;
+        const bool box64 = CG == 2 && a_rows <= 64;
+        const CUtensorMap* amap = box64 ? &a.mapA64[ti.kind] : &a.mapA[ti.kind];
+        const uint32_t tx = box64 ? stage_bytes - kSmemA / 2 : stage_bytes;
         int b_y = ti.idx * a.n_kind[ti.kind] + ti.n * BN;
         const CUtensorMap* bmap = &a.mapB[ti.kind * 2];
         // Pair B halves: gate/up - the CTA of rank r loads gate rows and up rows
@@ -230,12 +243,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort, a.err, a.timeout_ns)) break;
         tc_fence_after();
         const uint32_t d0 = tmem_base + static_cast<uint32_t>(acc) * acc_stride;
-        const uint32_t idesc = ti.small ? idesc_small : idesc_full;
+        // Swapped tiles are one M = 256 pair MMA per step: 128 weight rows per CTA
+        // (gate/up: the 64 gate rows then the 64 up rows of its output columns).
+        const uint32_t idesc = ti.swap ? idesc_bf16_f32(256, ti.nt) : (ti.small ? idesc_small : idesc_full);
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(&full[stage], phase, abort, a.err, a.timeout_ns)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t a_addr = smem_u32(sA + stage * kSmemA);
-          const uint32_t b_addr = smem_u32(sB + stage * sb_bytes);
+          // A swapped tile reads the weight rows as its A operand and the token
+          // rows as its B operand (the same K order, so the same bits per element).
+          const uint32_t tok_addr = smem_u32(sA + stage * kSmemA);
+          const uint32_t w_addr = smem_u32(sB + stage * sb_bytes);
+          const uint32_t a_addr = ti.swap ? w_addr : tok_addr;
+          const uint32_t b_addr = ti.swap ? tok_addr : w_addr;
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk) {
             const uint64_t ad = sw128_kmajor_desc(a_addr + kk * 32);
@@ -274,6 +293,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
     const int sr = lane >> 3, sc = lane & 7; // store phase: row offset 0..3, 16-byte chunk 0..7
     int acc = 0;
     uint32_t acc_phase = 0;
+    uint32_t xph = 0;  // phase of this warp's exchange channel (swapped gate/up tiles)
     for (int t = cluster_id; t < total; t += n_clusters) {
       Tile ti;
       decode_tile<CG>(a, t, ti);
@@ -282,6 +302,77 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
       tc_fence_after();
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                           static_cast<uint32_t>(acc) * acc_stride;
+      if (CG == 2 && ti.swap) {
+        // Operand-swapped tile: TMEM lanes are output columns, TMEM columns are
+        // the tile's tokens (rows m * 256 + j of the group, j < r valid).
+        const int r = min(256, ti.rows - ti.m * C::kTileM);
+        const int trow0 = ti.m * C::kTileM;
+        if (MODE == kGateUp) {
+          // Lanes 0-63 hold the gate rows and lanes 64-127 the up rows of the CTA's
+          // 64 output columns; TMEM columns are tokens.  The up warp of each lane
+          // quarter pair stages its values in its buffer (4-byte word j of lane l
+          // at l * 32 + (j ^ l): conflict-free both ways) and the gate warp of the
+          // same columns reads them, both under bounded mbarrier waits.
+          const bool gate_warp = q < 2;
+          const int pch = (q & 1) + 2 * half;  // exchange channel of this warp pair
+          uint32_t* xbuf = reinterpret_cast<uint32_t*>(gate_warp ? stage_w - 2 * kEpiBytes : stage_w);
+          const int col = ti.n * BN + static_cast<int>(rank) * (BN / 2) + 32 * (q & 1) + lane;
+          uint16_t* outb = static_cast<uint16_t*>(a.out[ti.kind]);
+          const size_t ld = static_cast<size_t>(a.ld_out[ti.kind]);
+          const int orow0 = (ti.kind == 0 ? ti.a_row0 : ti.idx * a.shared_out_stride) + trow0;
+          for (int c = 32 * half; c < ti.nt && ok; c += 64) {
+            uint32_t v[32];
+            tmem_ld32(tb + c, v);
+            tmem_ld_wait();
+            if (!gate_warp) {
+              ok = mbar_wait(&xempty[pch], xph ^ 1u, abort, a.err, a.timeout_ns);
+              if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+#pragma unroll
+              for (int j = 0; j < 32; ++j) xbuf[lane * 32 + (j ^ lane)] = v[j];
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&xfull[pch]);
+            } else {
+              ok = mbar_wait(&xfull[pch], xph, abort, a.err, a.timeout_ns);
+              if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+              uint32_t u[32];
+#pragma unroll
+              for (int j = 0; j < 32; ++j) u[j] = xbuf[lane * 32 + (j ^ lane)];
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&xempty[pch]);
+#pragma unroll
+              for (int j = 0; j < 32; ++j) {
+                if (c + j < r) {
+                  const float hv = silu_clamped_product(__uint_as_float(v[j]), __uint_as_float(u[j]),
+                                                        a.gate_clamp, a.up_clamp);
+                  outb[static_cast<size_t>(orow0 + c + j) * ld + col] =
+                      static_cast<uint16_t>(pack_bf16x2(hv, 0.f) & 0xFFFFu);
+                }
+              }
+            }
+            xph ^= 1u;
+          }
+        } else {
+          // One M = 256 pair MMA: lane i = output column n * BN + 128 * rank + i.
+          const bool scatter = (MODE == kDown && ti.kind == 0);
+          const int col = ti.n * BN + static_cast<int>(rank) * (BN / 2) + 32 * q + lane;
+          float* outb = static_cast<float*>(a.out[ti.kind]);
+          const size_t ld = static_cast<size_t>(a.ld_out[ti.kind]);
+          const int orow0 = (ti.kind == 0 ? ti.a_row0 : ti.idx * a.shared_out_stride) + trow0;
+          for (int c = 32 * half; c < ti.nt; c += 64) {
+            uint32_t v[32];
+            tmem_ld32(tb + c, v);
+            tmem_ld_wait();
+            const int my_tok = c + lane;  // this lane fetches the output row of token c + lane
+            int my_row = 0;
+            if (my_tok < r) my_row = scatter ? a.dest_row[ti.a_row0 + trow0 + my_tok] : orow0 + my_tok;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const int orow = __shfl_sync(0xffffffffu, my_row, j);
+              if (c + j < r) outb[static_cast<size_t>(orow) * ld + col] = __uint_as_float(v[j]);
+            }
+          }
+        }
+      } else {
       // Rows and columns this warp owns.  A 256-row pair tile (and every CG = 1
       // tile) keeps row i of the CTA's 128 in TMEM lane i with all n_mma
       // columns.  A 128-row pair tile keeps the CTA's 64 rows twice: lanes 0-63
@@ -377,6 +468,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
           }
         }
       }
+      }  // not swapped
+      if (!ok) break;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {

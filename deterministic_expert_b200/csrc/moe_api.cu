@@ -276,6 +276,7 @@ int forward_impl(moe_handle* h, int T, const uint16_t* x, const uint16_t* residu
     g.n_kind[0] = c.I; g.n_kind[1] = c.I_shared;
     g.k_kind[0] = c.D; g.k_kind[1] = c.D;
     g.BN = h->bn_gu;
+    g.swap_ok = h->bn_gu == 128;
     g.shared_a_stride = 0;
     g.out[0] = hb; g.ld_out[0] = c.I;
     g.out[1] = hsb; g.ld_out[1] = c.I_shared;
@@ -303,6 +304,7 @@ int forward_impl(moe_handle* h, int T, const uint16_t* x, const uint16_t* residu
     g.n_kind[0] = c.D; g.n_kind[1] = c.D;
     g.k_kind[0] = c.I; g.k_kind[1] = c.I_shared;
     g.BN = h->bn_dn;
+    g.swap_ok = h->bn_dn == 256;
     g.shared_a_stride = T;
     g.out[0] = y; g.ld_out[0] = c.D;
     g.out[1] = ys; g.ld_out[1] = c.D;

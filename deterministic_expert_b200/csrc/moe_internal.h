@@ -65,6 +65,8 @@ struct GemmArgs {
   int n_kind[2];          // B rows per expert (N extent) per kind
   int k_kind[2];          // K extent per kind
   int BN;
+  int swap_ok;            // expert GEMMs: a group's last partial tile may run operand-swapped
+                          // (needs 128 weight rows per CTA: gate/up BN = 128, down BN = 256)
   int shared_a_stride;    // A rows between consecutive shared experts (0: all read row 0..T)
   int router_tiles;       // tile count when tile_start is NULL
   void* out[2];           // output base per kind
