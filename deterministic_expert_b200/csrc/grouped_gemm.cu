@@ -185,9 +185,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
         // Swapped tile: this CTA's nt / 2 token rows (the B operand's half).
         const int a_rows = ti.swap ? ti.nt / 2 : (ti.small ? 64 : 128);
         const int a_y = ti.a_row0 + ti.m * C::kTileM + static_cast<int>(rank) * a_rows;
-        const bool box64 = CG == 2 && a_rows <= 64;
-        const CUtensorMap* amap = box64 ? &a.mapA64[ti.kind] : &a.mapA[ti.kind];
-        const uint32_t tx = box64 ? stage_bytes - kSmemA / 2 : stage_bytes;
+        const int box = CG == 2 ? (a_rows <= 16 ? 16 : (a_rows <= 64 ? 64 : 128)) : 128;
+        const CUtensorMap* amap =
+            box == 16 ? &a.mapA16[ti.kind] : (box == 64 ? &a.mapA64[ti.kind] : &a.mapA[ti.kind]);
+        const uint32_t tx = stage_bytes - kSmemA + static_cast<uint32_t>(box) * kBK * 2;
         int b_y = ti.idx * a.n_kind[ti.kind] + ti.n * BN;
         const CUtensorMap* bmap = &a.mapB[ti.kind * 2];
         // Pair B halves: gate/up - the CTA of rank r loads gate rows and up rows

@@ -269,8 +269,10 @@ int forward_impl(moe_handle* h, int T, const uint16_t* x, const uint16_t* residu
     std::memset(&g, 0, sizeof(g));
     if (!make_map(&g.mapA[0], xp, c.D, TK, kBM)) return MOE_ECUDA;
     if (!make_map(&g.mapA64[0], xp, c.D, TK, kBM / 2)) return MOE_ECUDA;
+    if (!make_map(&g.mapA16[0], xp, c.D, TK, 16)) return MOE_ECUDA;
     if (h->S > 0 && !make_map(&g.mapA[1], xn, c.D, T, kBM)) return MOE_ECUDA;
     if (h->S > 0 && !make_map(&g.mapA64[1], xn, c.D, T, kBM / 2)) return MOE_ECUDA;
+    if (h->S > 0 && !make_map(&g.mapA16[1], xn, c.D, T, 16)) return MOE_ECUDA;
     g.mapB[0] = h->map_wg; g.mapB[1] = h->map_wu; g.mapB[2] = h->map_wsg; g.mapB[3] = h->map_wsu;
     g.offsets = offsets; g.tile_start = tiles_gu; g.G = h->G; g.E = c.E; g.T = T;
     g.n_kind[0] = c.I; g.n_kind[1] = c.I_shared;
@@ -295,9 +297,12 @@ int forward_impl(moe_handle* h, int T, const uint16_t* x, const uint16_t* residu
     std::memset(&g, 0, sizeof(g));
     if (!make_map(&g.mapA[0], hb, c.I, TK, kBM)) return MOE_ECUDA;
     if (!make_map(&g.mapA64[0], hb, c.I, TK, kBM / 2)) return MOE_ECUDA;
+    if (!make_map(&g.mapA16[0], hb, c.I, TK, 16)) return MOE_ECUDA;
     if (h->S > 0 && !make_map(&g.mapA[1], hsb, c.I_shared, static_cast<uint64_t>(h->S) * T, kBM))
       return MOE_ECUDA;
     if (h->S > 0 && !make_map(&g.mapA64[1], hsb, c.I_shared, static_cast<uint64_t>(h->S) * T, kBM / 2))
+      return MOE_ECUDA;
+    if (h->S > 0 && !make_map(&g.mapA16[1], hsb, c.I_shared, static_cast<uint64_t>(h->S) * T, 16))
       return MOE_ECUDA;
     g.mapB[0] = h->map_wd; g.mapB[2] = h->map_wsd;
     g.offsets = offsets; g.tile_start = tiles_dn; g.G = h->G; g.E = c.E; g.T = T;

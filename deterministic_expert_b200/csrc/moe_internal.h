@@ -57,6 +57,7 @@ enum GemmMode : int { kGateUp = 0, kDown = 1, kRouter = 2 };
 struct GemmArgs {
   CUtensorMap mapA[2];    // A operand per group kind: 0 routed, 1 shared
   CUtensorMap mapA64[2];  // the same A operands with a 64-row box (128-row pair tiles)
+  CUtensorMap mapA16[2];  // ... and a 16-row box (swapped tiles of up to 32 tokens)
   CUtensorMap mapB[4];    // B operands: [kind * 2 + 0] first (gate / down / router),
                           //             [kind * 2 + 1] second (up; gate/up only)
   const int* offsets;     // [E + 1] grouped-row offsets of the routed groups

@@ -32,14 +32,12 @@ __device__ __forceinline__ bool better(float k1, int e1, float k2, int e2) {
   return k1 > k2 || (k1 == k2 && e1 < e2);
 }
 
-__global__ void __launch_bounds__(256) k_router_topk(const RouterArgs a) {
-  griddep_wait();
-  griddep_launch();
-  const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (t >= a.T) return;
+// Route token t (one warp; lr = its logits row, anywhere in memory; hist = the
+// histogram its experts are counted into).  Shared by the per-token kernel and
+// the single-block decode kernel, so both take the same arithmetic.
+__device__ __forceinline__ void route_token(const RouterArgs& a, int t, int lane, const float* lr,
+                                            int32_t* hist) {
   const int k = a.k, E = a.E;
-  int32_t* hist = a.block_counts + static_cast<size_t>(t / kDispatchRows) * a.E4;
 
   if (a.router == MOE_ROUTER_HASH) {
     if (lane < k) {
@@ -56,7 +54,6 @@ __global__ void __launch_bounds__(256) k_router_topk(const RouterArgs a) {
     return;
   }
 
-  const float* lr = a.logits + static_cast<size_t>(t) * a.E_pad;
   float key[kMaxPerLane], val[kMaxPerLane];
   float zmax = -FLT_MAX;
 #pragma unroll
@@ -153,6 +150,16 @@ __global__ void __launch_bounds__(256) k_router_topk(const RouterArgs a) {
     if (a.user_w) a.user_w[t * k + lane] = wn;
     atomicAdd(hist + e, 1);
   }
+}
+
+__global__ void __launch_bounds__(256) k_router_topk(const RouterArgs a) {
+  griddep_wait();
+  griddep_launch();
+  const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (t >= a.T) return;
+  route_token(a, t, lane, a.logits + static_cast<size_t>(t) * a.E_pad,
+              a.block_counts + static_cast<size_t>(t / kDispatchRows) * a.E4);
 }
 
 }  // namespace
