@@ -185,7 +185,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
         // Swapped tile: this CTA's nt / 2 token rows (the B operand's half).
         const int a_rows = ti.swap ? ti.nt / 2 : (ti.small ? 64 : 128);
         const int a_y = ti.a_row0 + ti.m * C::kTileM + static_cast<int>(rank) * a_rows;
-        const int box = CG == 2 ? (a_rows <= 16 ? 16 : (a_rows <= 64 ? 64 : 128)) : 128;
+        // Rows of A the MMA uses: a_rows (pairs), or the router tile's valid rows.
+        const int need = CG == 2 ? a_rows : min(128, ti.rows - ti.m * 128);
+        const int box = need <= 16 ? 16 : (need <= 64 ? 64 : 128);
         const CUtensorMap* amap =
             box == 16 ? &a.mapA16[ti.kind] : (box == 64 ? &a.mapA64[ti.kind] : &a.mapA[ti.kind]);
         const uint32_t tx = stage_bytes - kSmemA + static_cast<uint32_t>(box) * kBK * 2;
@@ -200,8 +202,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort, a.err, a.timeout_ns)) { ok = false; break; }
           uint8_t* b0 = sB + stage * sb_bytes;
           if (CG == 1) {
-            mbar_arrive_expect_tx(&full[stage], stage_bytes);
-            tma_load_2d(sA + stage * kSmemA, &a.mapA[ti.kind], kb * kBK, a_y, &full[stage]);
+            mbar_arrive_expect_tx(&full[stage], tx);
+            tma_load_2d(sA + stage * kSmemA, amap, kb * kBK, a_y, &full[stage]);
             tma_load_2d(b0, bmap, kb * kBK, b_y, &full[stage]);
             if (MODE == kGateUp)
               tma_load_2d(b0 + b_rows * kBK * 2, bmap + 1, kb * kBK, b_y, &full[stage]);

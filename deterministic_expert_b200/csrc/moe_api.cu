@@ -218,6 +218,8 @@ int forward_impl(moe_handle* h, int T, const uint16_t* x, const uint16_t* residu
     GemmArgs g;
     std::memset(&g, 0, sizeof(g));
     if (!make_map(&g.mapA[0], xn, c.D, T, kBM)) return MOE_ECUDA;
+    if (!make_map(&g.mapA64[0], xn, c.D, T, kBM / 2)) return MOE_ECUDA;
+    if (!make_map(&g.mapA16[0], xn, c.D, T, 16)) return MOE_ECUDA;
     g.mapB[0] = h->map_router;
     g.T = T;
     g.n_kind[0] = h->E_pad;
