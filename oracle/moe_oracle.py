@@ -30,7 +30,8 @@ The layer, in order:
                                           dropping is batch dependent: none here)
   5. stable permute (dispatch)           [DS] §6.1 (dispatch -> compute -> combine)
   6. routed + shared SwiGLU experts      [DS] §6.5, [LD] "SiTU-GLU" (SwiGLU form),
-                                          [LD] "共享专家"
+                                          [LD] "共享专家"; or SiTU-GLU experts
+                                          ([LD] "SiTU-GLU", beta 4 / 25)
   7. weighted combine in fp32, one cast  [FW] Trap 3 and the case study ("standard
                                           path": all k contributions kept in fp32,
                                           weighted sum, one final cast)
@@ -268,9 +269,41 @@ def swiglu(g, u, gate_clamp_max: float = np.inf, up_clamp: float = np.inf) -> np
     return g * sigmoid(g) * u
 
 
-def expert_ffn(xn_rows, w_gate, w_up, w_down, gate_clamp_max=np.inf, up_clamp=np.inf):
-    """One SwiGLU expert on a block of rows: g = xn W_g^T, u = xn W_u^T (full
-    K = D), h = bf16(SwiGLU(g, u)), y = h W_d^T (full K = I).  Returns (h, y)."""
+ACT_SWIGLU = 0
+ACT_SITU_GLU = 1
+
+
+def situ_glu(g, u, beta_g: float = 4.0, beta_u: float = 25.0) -> np.ndarray:
+    """SiTU-GLU ([LD] "SiTU-GLU", the K3 report's formula as the post quotes
+    it): [beta_g tanh(W_g x / beta_g) * Sigmoid(W_g x)] * [beta_u tanh(W_u x /
+    beta_u)], a soft cap on both branches (the post gives beta_g = 4 for the
+    gate and beta_u = 25 for the up branch), so |h| < beta_g * beta_u."""
+    g = np.asarray(g, np.float64)
+    u = np.asarray(u, np.float64)
+    return (beta_g * np.tanh(g / beta_g) * sigmoid(g)) * (beta_u * np.tanh(u / beta_u))
+
+
+def glu_unit(g, u, act: int = ACT_SWIGLU, gate_clamp_max: float = np.inf, up_clamp: float = np.inf,
+             beta_g: float = 4.0, beta_u: float = 25.0) -> np.ndarray:
+    """The expert's gated unit: SwiGLU (with the optional clamp) or SiTU-GLU."""
+    if act == ACT_SITU_GLU:
+        return situ_glu(g, u, beta_g, beta_u)
+    return swiglu(g, u, gate_clamp_max, up_clamp)
+
+
+def unit_args(cfg) -> dict:
+    """glu_unit keyword arguments of a layer configuration (SwiGLU when the
+    configuration names no activation)."""
+    return dict(act=getattr(cfg, "activation", ACT_SWIGLU), gate_clamp_max=cfg.gate_clamp_max,
+                up_clamp=cfg.up_clamp, beta_g=getattr(cfg, "situ_beta_gate", 4.0),
+                beta_u=getattr(cfg, "situ_beta_up", 25.0))
+
+
+def expert_ffn(xn_rows, w_gate, w_up, w_down, gate_clamp_max=np.inf, up_clamp=np.inf,
+               act: int = ACT_SWIGLU, beta_g: float = 4.0, beta_u: float = 25.0):
+    """One gated expert on a block of rows: g = xn W_g^T, u = xn W_u^T (full
+    K = D), h = bf16(unit(g, u)) with the SwiGLU or SiTU-GLU unit, y = h W_d^T
+    (full K = I).  Returns (h, y)."""
     x = np.asarray(xn_rows, np.float64)
     Wg = np.asarray(w_gate, np.float64)
     Wu = np.asarray(w_up, np.float64)
@@ -278,7 +311,7 @@ def expert_ffn(xn_rows, w_gate, w_up, w_down, gate_clamp_max=np.inf, up_clamp=np
     n, D = x.shape
     I = Wg.shape[0]
     MAC_COUNTER[0] += n * (2 * D * I + I * Wd.shape[0])
-    h = round_bf16(swiglu(x @ Wg.T, x @ Wu.T, gate_clamp_max, up_clamp))
+    h = round_bf16(glu_unit(x @ Wg.T, x @ Wu.T, act, gate_clamp_max, up_clamp, beta_g, beta_u))
     return h, h @ Wd.T
 
 
@@ -366,7 +399,8 @@ def moe_layer(cfg, W, x, residual, token_ids=None, rows=None) -> dict:
     """The whole layer.  Routing, histogram and permutation are computed for
     every token; the experts, combine and epilogue for ``rows`` (all tokens
     when None).  ``cfg`` carries D, E, k, I, n_shared, I_shared, router,
-    renormalize, routed_scale, gate_clamp_max, up_clamp, eps, hash_mult."""
+    renormalize, routed_scale, gate_clamp_max, up_clamp, eps, hash_mult and
+    optionally activation, situ_beta_gate, situ_beta_up (SiTU-GLU experts)."""
     x = np.asarray(x, np.float64)
     T = x.shape[0]
     rows = np.arange(T) if rows is None else np.asarray(rows, np.int64)
@@ -386,13 +420,13 @@ def moe_layer(cfg, W, x, residual, token_ids=None, rows=None) -> dict:
     for e in np.unique(sel):
         rr, jj = np.nonzero(sel == e)
         Wg, Wu, Wd = W.routed(int(e))
-        _, y = expert_ffn(xn[rows[rr]], Wg, Wu, Wd, cfg.gate_clamp_max, cfg.up_clamp)
+        _, y = expert_ffn(xn[rows[rr]], Wg, Wu, Wd, **unit_args(cfg))
         y_slots[rr, jj] = y
     y_shared = np.zeros((cfg.n_shared, n, cfg.D))
     for s in range(cfg.n_shared):
         Wg, Wu, Wd = W.shared(s)
         # The clamp is a property of the SwiGLU unit and applies to shared experts too.
-        _, y_shared[s] = expert_ffn(xn[rows], Wg, Wu, Wd, cfg.gate_clamp_max, cfg.up_clamp)
+        _, y_shared[s] = expert_ffn(xn[rows], Wg, Wu, Wd, **unit_args(cfg))
     acc = combine(w[rows], y_slots, y_shared)
     out_norm, out_residual, r = residual_rmsnorm(acc, np.asarray(residual, np.float64)[rows],
                                                  W.g_out, cfg.eps)
@@ -416,11 +450,11 @@ def moe_layer_dense_masked(cfg, W, x, residual, token_ids=None) -> dict:
     acc = np.zeros((T, cfg.D))
     for e in range(cfg.E):
         Wg, Wu, Wd = W.routed(e)
-        _, y = expert_ffn(xn, Wg, Wu, Wd, cfg.gate_clamp_max, cfg.up_clamp)
+        _, y = expert_ffn(xn, Wg, Wu, Wd, **unit_args(cfg))
         acc += mask[:, e:e + 1] * y
     for s in range(cfg.n_shared):
         Wg, Wu, Wd = W.shared(s)
-        _, y = expert_ffn(xn, Wg, Wu, Wd, cfg.gate_clamp_max, cfg.up_clamp)
+        _, y = expert_ffn(xn, Wg, Wu, Wd, **unit_args(cfg))
         acc += y
     out_norm, out_residual, r = residual_rmsnorm(acc, residual, W.g_out, cfg.eps)
     return dict(acc=acc, r=r, out_norm=out_norm, out_residual=out_residual, idx=idx, w=w)

@@ -141,6 +141,41 @@ def pin_swiglu_clamp(O):
     assert np.max(np.abs(O.swiglu(big[0], big[1], cg, cu))) <= silu10 * 10 + 1e-12
 
 
+def pin_situ_glu(O):
+    """SiTU-GLU against the limits and bounds the page states, not its formula."""
+    g = golden("situ_glu.json")
+    b1, b2 = g["beta_gate"], g["beta_up"]
+
+    def situ(gg, uu):
+        return np.asarray(O.glu_unit(gg, uu, O.ACT_SITU_GLU, beta_g=b1, beta_u=b2), np.float64)
+
+    # Bounded by beta1 * beta2 (the page's 4 x 25 = 100) on any input, and the
+    # page's example (20, 30) is far below SwiGLU's ~600.
+    rng = np.random.default_rng(5)
+    big = rng.standard_normal((2, 20000)) * 200
+    assert np.max(np.abs(situ(big[0], big[1]))) <= g["bound_printed"]
+    v = float(situ(g["gate"], g["up"]))
+    assert 0.0 < v < g["bound_printed"] < float(O.swiglu(g["gate"], g["up"]))
+    # Near the origin the soft caps are the identity to second order, so the
+    # unit equals SwiGLU up to a relative O(x^2) term (the page: it keeps
+    # SwiGLU's local response).
+    for s_ in (1e-2, 1e-3):
+        gg, uu = 0.7 * s_, -0.4 * s_
+        assert abs(float(situ(gg, uu)) / float(O.swiglu(gg, uu)) - 1.0) < 2 * s_ ** 2
+    # Saturation of each branch alone: a large gate passes beta1 * u for a small
+    # up value; a large up value passes beta2 * Swish(g) for a small gate.
+    u0, g0 = 1e-4, 1e-4
+    assert abs(float(situ(60.0, u0)) / (b1 * u0) - 1.0) < 1e-6
+    assert abs(float(situ(g0, 1e4)) / (b2 * g0 / (1.0 + math.exp(-g0))) - 1.0) < 1e-6
+    # Both large: the product of the caps.
+    assert abs(float(situ(1e3, 1e4)) - b1 * b2) < 1e-9 * b1 * b2
+    # The Sigmoid of the gate closes the unit for a very negative gate,
+    # whatever the up branch.
+    assert abs(float(situ(-60.0, 1e4))) < 1e-20
+    # The up branch is odd.
+    assert float(situ(2.0, -3.0)) == -float(situ(2.0, 3.0))
+
+
 # ------------------------------------------------------------------ top-k
 def _brute_topk(row, k):
     order = sorted(range(len(row)), key=lambda e: (-row[e], e))

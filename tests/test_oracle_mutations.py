@@ -33,7 +33,14 @@ MUTATIONS = {
                                  "w = np.take_along_axis(keys, idx, axis=-1)"),
     "hash_without_multiply": ("h = (ids * np.uint64(mult)) & np.uint64(0xFFFFFFFF)",
                               "h = ids & np.uint64(0xFFFFFFFF)"),
-    "gate_up_swapped": ("swiglu(x @ Wg.T, x @ Wu.T,", "swiglu(x @ Wu.T, x @ Wg.T,"),
+    "gate_up_swapped": ("glu_unit(x @ Wg.T, x @ Wu.T,", "glu_unit(x @ Wu.T, x @ Wg.T,"),
+    "situ_betas_swapped": ("return (beta_g * np.tanh(g / beta_g) * sigmoid(g)) * (beta_u * np.tanh(u / beta_u))",
+                           "return (beta_u * np.tanh(g / beta_u) * sigmoid(g)) * (beta_g * np.tanh(u / beta_g))"),
+    "situ_sigmoid_of_up": ("return (beta_g * np.tanh(g / beta_g) * sigmoid(g)) * (beta_u * np.tanh(u / beta_u))",
+                           "return (beta_g * np.tanh(g / beta_g) * sigmoid(u)) * (beta_u * np.tanh(u / beta_u))"),
+    "situ_caps_unscaled": ("return (beta_g * np.tanh(g / beta_g) * sigmoid(g)) * (beta_u * np.tanh(u / beta_u))",
+                           "return (np.tanh(g / beta_g) * sigmoid(g)) * (np.tanh(u / beta_u))"),
+    "situ_falls_back_to_swiglu": ("    if act == ACT_SITU_GLU:\n        return situ_glu(g, u, beta_g, beta_u)\n", ""),
     "down_not_transposed": ("return h, h @ Wd.T", "return h, h @ Wd"),
     "silu_sign": ("return g * sigmoid(g) * u", "return g * sigmoid(-g) * u"),
     "gate_clamped_both_sides": ("g = np.minimum(np.asarray(g, np.float64), gate_clamp_max)",
