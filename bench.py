@@ -69,7 +69,8 @@ def describe(cfg):
     return {"workload": W.pretty(cfg), "T": cfg.T, "D": cfg.D, "E": cfg.E, "k": cfg.k, "I": cfg.I,
             "n_shared": cfg.n_shared, "I_shared": cfg.I_shared,
             "router": {0: "softmax", 1: "sigmoid+bias", 2: "hash"}[cfg.router],
-            "renormalize": bool(cfg.renormalize)}
+            "renormalize": bool(cfg.renormalize),
+            "activation": "SiTU-GLU" if cfg.activation == 1 else "SwiGLU"}
 
 
 def peaks():

@@ -21,6 +21,7 @@ HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "moe.h")
 MOE_OK, MOE_EINVAL, MOE_ETOOBIG, MOE_EWORKSPACE, MOE_EUNSUPPORTED, MOE_ECUDA, MOE_ETIMEOUT = (
     0, -1, -2, -3, -4, -5, -6)
 ROUTER_SOFTMAX, ROUTER_SIGMOID_BIAS, ROUTER_HASH = 0, 1, 2
+ACT_SWIGLU, ACT_SITU_GLU = 0, 1
 NUM_STAGES = 8
 STAGE_NAMES = ("rmsnorm_in", "router_gemm", "router_topk", "dispatch", "gather_rows",
                "gemm_gateup_swiglu", "gemm_down", "combine_norm")
@@ -37,7 +38,9 @@ class moe_config(ctypes.Structure):
                 ("n_shared", ctypes.c_int), ("I_shared", ctypes.c_int), ("T_max", ctypes.c_int),
                 ("router", ctypes.c_int), ("renormalize", ctypes.c_int),
                 ("routed_scale", ctypes.c_float), ("gate_clamp_max", ctypes.c_float),
-                ("up_clamp", ctypes.c_float), ("eps", ctypes.c_float), ("hash_mult", ctypes.c_uint32)]
+                ("up_clamp", ctypes.c_float), ("eps", ctypes.c_float), ("hash_mult", ctypes.c_uint32),
+                ("activation", ctypes.c_int), ("situ_beta_gate", ctypes.c_float),
+                ("situ_beta_up", ctypes.c_float)]
 
 
 class moe_weights(ctypes.Structure):
@@ -123,12 +126,16 @@ class LayerConfig:
     up_clamp: float = float("inf")
     eps: float = 1e-6
     hash_mult: int = 2654435761
+    activation: int = ACT_SWIGLU
+    situ_beta_gate: float = 4.0
+    situ_beta_up: float = 25.0
 
     def to_c(self) -> moe_config:
         return moe_config(self.D, self.E, self.k, self.I, self.n_shared,
                           self.I_shared if self.n_shared else self.I, self.T_max, self.router,
                           self.renormalize, self.routed_scale, self.gate_clamp_max, self.up_clamp,
-                          self.eps, self.hash_mult)
+                          self.eps, self.hash_mult, self.activation, self.situ_beta_gate,
+                          self.situ_beta_up)
 
 
 class MoELayer:

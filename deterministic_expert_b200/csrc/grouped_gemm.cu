@@ -3,6 +3,7 @@
 // Used three ways by the layer:
 //   router : logits[T, E_pad] = xn W_r^T                     one group of T rows
 //   gate/up: h = bf16(SiLU(min(g, c_g)) * clamp(u, +-c_u)),  g = A W_g^T, u = A W_u^T,
+//            (or the SiTU-GLU unit [b_g tanh(g/b_g) sigmoid(g)] * [b_u tanh(u/b_u)])
 //            per routed expert (A = its grouped rows of xn) and per shared expert (A = xn)
 //   down   : y = h W_d^T in fp32, routed rows scattered to their (token, slot) row
 //
@@ -105,7 +106,33 @@ __device__ __forceinline__ float silu_clamped_product(float g, float u, float cg
   return __fdividef(g, 1.0f + __expf(-g)) * u;
 }
 
-template <int MODE, int CG>
+// tanh(z) = sign(z) (1 - e^{-2|z|}) / (1 + e^{-2|z|}), each step an explicitly
+// rounded fp32 operation or an intrinsic, none of which the compiler may fuse
+// or reorder, so the result is the same bits wherever it is inlined.  Error
+// about 1e-7 absolute (the exponential's), far below the bf16 rounding of h.
+__device__ __forceinline__ float tanh_rn(float z) {
+  const float e = __expf(__fmul_rn(-2.0f, fabsf(z)));
+  return copysignf(__fdividef(__fsub_rn(1.0f, e), __fadd_rn(1.0f, e)), z);
+}
+
+// SiTU-GLU: [bg tanh(g / bg) * sigmoid(g)] * [bu tanh(u / bu)] in fp32 (the
+// linux.do post on MoE variants, "SiTU-GLU": soft caps on both branches);
+// ibg = 1 / bg and ibu = 1 / bu are rounded once on the host.
+__device__ __forceinline__ float situ_glu_product(float g, float u, float bg, float bu, float ibg,
+                                                  float ibu) {
+  const float sig = __fdividef(1.0f, __fadd_rn(1.0f, __expf(-g)));
+  const float gate = __fmul_rn(__fmul_rn(bg, tanh_rn(__fmul_rn(g, ibg))), sig);
+  return __fmul_rn(gate, __fmul_rn(bu, tanh_rn(__fmul_rn(u, ibu))));
+}
+
+// The experts' gated unit (the same function in every tile shape).
+template <int ACT>
+__device__ __forceinline__ float glu_unit(float g, float u, const GemmArgs& a) {
+  if (ACT == MOE_ACT_SITU_GLU) return situ_glu_product(g, u, a.beta_g, a.beta_u, a.inv_beta_g, a.inv_beta_u);
+  return silu_clamped_product(g, u, a.gate_clamp, a.up_clamp);
+}
+
+template <int MODE, int CG, int ACT>
 __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_constant__ GemmArgs a) {
   using C = Cfg<CG>;
   // Stage ring.  The expert GEMMs use C::kStagesN stages of kSmemA + C::kSmemB
@@ -345,14 +372,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
 #pragma unroll
               for (int j = 0; j < 32; ++j) {
                 if (c + j < r) {
-                  const float hv = silu_clamped_product(__uint_as_float(v[j]), __uint_as_float(u[j]),
-                                                        a.gate_clamp, a.up_clamp);
+                  const float hv = glu_unit<ACT>(__uint_as_float(v[j]), __uint_as_float(u[j]), a);
                   outb[static_cast<size_t>(orow0 + c + j) * ld + col] =
                       static_cast<uint16_t>(pack_bf16x2(hv, 0.f) & 0xFFFFu);
                 }
               }
             }
             xph ^= 1u;
+          }
+          // The up warp's buffer is its own staging area in row tiles: do not
+          // leave the tile before the gate warp has read the last block.
+          if (!gate_warp && ok) {
+            ok = mbar_wait(&xempty[pch], xph ^ 1u, abort, a.err, a.timeout_ns);
+            ok = __all_sync(0xffffffffu, ok);
           }
         } else {
           // One M = 256 pair MMA: lane i = output column n * BN + 128 * rank + i.
@@ -407,11 +439,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
             uint32_t p[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i)
-              p[i] = pack_bf16x2(
-                  silu_clamped_product(__uint_as_float(g[2 * i]), __uint_as_float(u[2 * i]),
-                                       a.gate_clamp, a.up_clamp),
-                  silu_clamped_product(__uint_as_float(g[2 * i + 1]), __uint_as_float(u[2 * i + 1]),
-                                       a.gate_clamp, a.up_clamp));
+              p[i] = pack_bf16x2(glu_unit<ACT>(__uint_as_float(g[2 * i]), __uint_as_float(u[2 * i]), a),
+                                 glu_unit<ACT>(__uint_as_float(g[2 * i + 1]), __uint_as_float(u[2 * i + 1]), a));
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               const int m = c / 8 + i;
@@ -508,9 +537,9 @@ cudaLaunchConfig_t pair_config(int grid, cudaStream_t s, cudaLaunchAttribute* at
   return cfg;
 }
 
-template <int MODE, int CG>
+template <int MODE, int CG, int ACT = MOE_ACT_SWIGLU>
 cudaError_t launch_one(const GemmArgs& a, int grid, cudaStream_t s) {
-  return launch_k(k_grouped_gemm<MODE, CG>, dim3(grid), dim3(kGemmThreads), kGemmSmem, s, CG == 2, a);
+  return launch_k(k_grouped_gemm<MODE, CG, ACT>, dim3(grid), dim3(kGemmThreads), kGemmSmem, s, CG == 2, a);
 }
 
 int g_pair_clusters[64] = {0};
@@ -522,16 +551,22 @@ void gemm_prepare() {
   int dev = 0;
   cudaGetDevice(&dev);
   if (done_dev == dev) return;
-  cudaFuncSetAttribute(k_grouped_gemm<kGateUp, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem);
-  cudaFuncSetAttribute(k_grouped_gemm<kDown, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem);
-  cudaFuncSetAttribute(k_grouped_gemm<kRouter, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem);
+  cudaFuncSetAttribute(k_grouped_gemm<kGateUp, 2, MOE_ACT_SWIGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       kGemmSmem);
+  cudaFuncSetAttribute(k_grouped_gemm<kGateUp, 2, MOE_ACT_SITU_GLU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       kGemmSmem);
+  cudaFuncSetAttribute(k_grouped_gemm<kDown, 2, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem);
+  cudaFuncSetAttribute(k_grouped_gemm<kRouter, 1, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem);
   // How many CTA pairs fit on the device at once: the persistent pair grid is
   // never larger, so no pair waits for another to finish before it starts.
   int n_gu = 0, n_dn = 0;
   cudaLaunchAttribute attr[1];
   cudaLaunchConfig_t cfg = pair_config(2, nullptr, attr);
-  if (cudaOccupancyMaxActiveClusters(&n_gu, k_grouped_gemm<kGateUp, 2>, &cfg) != cudaSuccess) n_gu = 0;
-  if (cudaOccupancyMaxActiveClusters(&n_dn, k_grouped_gemm<kDown, 2>, &cfg) != cudaSuccess) n_dn = 0;
+  int n_gs = 0;
+  if (cudaOccupancyMaxActiveClusters(&n_gu, k_grouped_gemm<kGateUp, 2, 0>, &cfg) != cudaSuccess) n_gu = 0;
+  if (cudaOccupancyMaxActiveClusters(&n_gs, k_grouped_gemm<kGateUp, 2, 1>, &cfg) != cudaSuccess) n_gs = 0;
+  if (cudaOccupancyMaxActiveClusters(&n_dn, k_grouped_gemm<kDown, 2, 0>, &cfg) != cudaSuccess) n_dn = 0;
+  n_gu = std::min(n_gu, n_gs);
   cudaGetLastError();
   if (dev >= 0 && dev < 64) g_pair_clusters[dev] = std::min(n_gu, n_dn);
   done_dev = dev;
@@ -546,7 +581,9 @@ int gemm_max_pairs() {
 cudaError_t launch_grouped_gemm(int mode, const GemmArgs& a, int grid, cudaStream_t s) {
   if (grid <= 0) return cudaSuccess;
   switch (mode) {
-    case kGateUp: return launch_one<kGateUp, 2>(a, grid, s);
+    case kGateUp:
+      return a.act == MOE_ACT_SITU_GLU ? launch_one<kGateUp, 2, MOE_ACT_SITU_GLU>(a, grid, s)
+                                       : launch_one<kGateUp, 2>(a, grid, s);
     case kDown: return launch_one<kDown, 2>(a, grid, s);
     default: return launch_one<kRouter, 1>(a, grid, s);
   }

@@ -122,6 +122,11 @@ int validate_config(const moe_config* c, const moe_weights* w) {
       !(c->gate_clamp_max == c->gate_clamp_max) || !(c->up_clamp >= 0.f))
     return MOE_EINVAL;
   if (c->n_shared > 0 && c->I_shared <= 0) return MOE_EINVAL;
+  if (c->activation != MOE_ACT_SWIGLU && c->activation != MOE_ACT_SITU_GLU) return MOE_EINVAL;
+  if (c->activation == MOE_ACT_SITU_GLU &&
+      !(c->situ_beta_gate > 0.f && c->situ_beta_gate < 3.0e38f && c->situ_beta_up > 0.f &&
+        c->situ_beta_up < 3.0e38f))
+    return MOE_EINVAL;
   if (c->D % 64 || c->I % 64 || (c->n_shared > 0 && c->I_shared % 64)) return MOE_EUNSUPPORTED;
   if (c->D > 16384 || c->E > 256 || c->k > c->E || c->k > 16 || c->n_shared > 8 || c->T_max > (1 << 20))
     return MOE_EUNSUPPORTED;
@@ -286,6 +291,8 @@ int forward_impl(moe_handle* h, int T, const uint16_t* x, const uint16_t* residu
     g.out[1] = hsb; g.ld_out[1] = c.I_shared;
     g.shared_out_stride = T;
     g.gate_clamp = c.gate_clamp_max; g.up_clamp = c.up_clamp;
+    g.act = c.activation; g.beta_g = c.situ_beta_gate; g.beta_u = c.situ_beta_up;
+    g.inv_beta_g = 1.0f / c.situ_beta_gate; g.inv_beta_u = 1.0f / c.situ_beta_up;
     g.err = err; g.timeout_ns = h->timeout_ns;
     const int bound = expert_tile_bound(h, T, da.gu_ntiles_routed, da.gu_ntiles_shared);
     prof.begin(5);

@@ -75,6 +75,9 @@ struct GemmArgs {
   int shared_out_stride;  // output rows between consecutive shared experts
   const int* dest_row;    // down, routed: grouped row -> output row
   float gate_clamp, up_clamp;
+  int act;                // moe_activation
+  float beta_g, beta_u;   // SiTU-GLU caps
+  float inv_beta_g, inv_beta_u;  // their reciprocals (rounded once)
   int* err;               // device error word
   unsigned long long timeout_ns;
 };

@@ -75,6 +75,15 @@ typedef enum {
                                    e_j = (e_0 + j) mod E, w_j = 1/k                     */
 } moe_router;
 
+/* The experts' gated unit. */
+typedef enum moe_activation {
+  MOE_ACT_SWIGLU = 0,    /* SiLU(min(g, gate_clamp_max)) * clamp(u, +-up_clamp)
+                            (DeepSeek V4 infra notes §6.5; the clamps may be +INF)  */
+  MOE_ACT_SITU_GLU = 1   /* [bg tanh(g / bg) * sigmoid(g)] * [bu tanh(u / bu)],
+                            bg = situ_beta_gate, bu = situ_beta_up (linux.do post on
+                            MoE variants, "SiTU-GLU": 4 and 25); clamps unused    */
+} moe_activation;
+
 typedef struct moe_config {
   int D;               /* hidden size                                                  */
   int E;               /* routed experts                                               */
@@ -90,6 +99,9 @@ typedef struct moe_config {
   float up_clamp;      /* SwiGLU up branch clipped to [-up_clamp, up_clamp] (+INF = off)*/
   float eps;           /* RMSNorm epsilon, inside the square root                      */
   uint32_t hash_mult;  /* multiplicative hash constant for MOE_ROUTER_HASH             */
+  int activation;      /* moe_activation of routed and shared experts                  */
+  float situ_beta_gate;/* SiTU-GLU gate cap (> 0, finite; read for MOE_ACT_SITU_GLU)    */
+  float situ_beta_up;  /* SiTU-GLU up cap (> 0, finite)                                 */
 } moe_config;
 
 typedef struct moe_weights {      /* device pointers, caller-owned                   */

@@ -57,6 +57,9 @@ class MoEConfig:
     weight_sigma: float = 0.02
     x_sigma: float = 1.0
     token_id_range: int = 128000
+    activation: int = 0             # 0 SwiGLU (+ clamp), 1 SiTU-GLU
+    situ_beta_gate: float = 4.0
+    situ_beta_up: float = 25.0
 
     def with_T(self, T: int) -> "MoEConfig":
         return dataclasses.replace(self, T=T)
@@ -80,13 +83,16 @@ C5 = MoEConfig("skew_zipf", T=16384, D=4096, E=128, k=8, I=1024, n_shared=0, I_s
                bias="zipf")
 # Hash-routing variant of the skewed workload.
 C5H = dataclasses.replace(C5, name="skew_hash", router=ROUTER_HASH, bias="none")
+# SiTU-GLU experts (the linux.do post on MoE variants, "SiTU-GLU": caps 4 and
+# 25) on the fine-grained shapes.
+C2S = dataclasses.replace(C2, name="fine_grained_situ", activation=1)
 # The 8-partial fixed-order reduce + residual + RMSNorm epilogue of that workload.
 EPILOGUE_P = 8
 EPILOGUE_T = 16384
 EPILOGUE_D = 4096
 EPILOGUE_SIGMA = 1.0 / 8.0
 
-CONFIGS = {c.name: c for c in (C1, C2, C3, C5, C5H)}
+CONFIGS = {c.name: c for c in (C1, C2, C3, C5, C5H, C2S)}
 
 _ZIPF_FILE = os.path.join(os.path.dirname(os.path.abspath(__file__)), "zipf_beta.json")
 ZIPF_S = 1.2
@@ -213,9 +219,10 @@ def layer_bytes(cfg: MoEConfig, T: int, distinct_experts: int) -> int:
 
 def pretty(cfg: MoEConfig) -> str:
     r = {0: "softmax", 1: "sigmoid+bias", 2: "hash"}[cfg.router]
+    act = "" if cfg.activation == 0 else f" SiTU-GLU({cfg.situ_beta_gate:g},{cfg.situ_beta_up:g})"
     return (f"{cfg.name}: T={cfg.T} D={cfg.D} E={cfg.E} top-{cfg.k} {r} I={cfg.I} "
-            f"shared={cfg.n_shared}x{cfg.I_shared}")
+            f"shared={cfg.n_shared}x{cfg.I_shared}{act}")
 
 
-__all__ = ["MoEConfig", "C1", "C2", "C3", "C4_T", "C5", "C5H", "CONFIGS", "STREAM", "SEED",
+__all__ = ["MoEConfig", "C1", "C2", "C2S", "C3", "C4_T", "C5", "C5H", "CONFIGS", "STREAM", "SEED",
            "host_bf16", "host_router_bias", "host_token_ids", "moe_flops", "math"]

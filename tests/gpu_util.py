@@ -20,7 +20,8 @@ def layer_config(cfg, T_max):
                            I_shared=cfg.I_shared, T_max=T_max, router=cfg.router,
                            renormalize=cfg.renormalize, routed_scale=cfg.routed_scale,
                            gate_clamp_max=cfg.gate_clamp_max, up_clamp=cfg.up_clamp, eps=cfg.eps,
-                           hash_mult=cfg.hash_mult)
+                           hash_mult=cfg.hash_mult, activation=cfg.activation,
+                           situ_beta_gate=cfg.situ_beta_gate, situ_beta_up=cfg.situ_beta_up)
 
 
 class Run:

@@ -25,7 +25,8 @@ def torch_cuda():
     return torch
 
 
-@pytest.mark.parametrize("name,splits", [("tiny", 7), ("fine_grained", 4), ("skew_hash", 3)])
+@pytest.mark.parametrize("name,splits", [("tiny", 7), ("fine_grained", 4), ("skew_hash", 3),
+                                         ("fine_grained_situ", 5)])
 def test_splits_permutation_repeats(torch_cuda, name, splits):
     torch = torch_cuda
     cfg = W.CONFIGS[name]

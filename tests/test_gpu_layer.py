@@ -133,7 +133,8 @@ def test_ragged_and_tiny_batches(torch_cuda, T):
     check_outputs(out, ref, same_rows=same)
 
 
-@pytest.mark.parametrize("variant", ["all_experts", "no_shared", "hash_small", "sigmoid_clamp", "k1"])
+@pytest.mark.parametrize("variant", ["all_experts", "no_shared", "hash_small", "sigmoid_clamp", "k1",
+                                     "situ_caps", "situ_tight_caps"])
 def test_layer_variants(torch_cuda, variant):
     base = dataclasses.replace(W.C1, T=300)
     cfg = {
@@ -144,7 +145,25 @@ def test_layer_variants(torch_cuda, variant):
                                              routed_scale=2.5, gate_clamp_max=0.05, up_clamp=0.05,
                                              bias="normal", bias_sigma=0.01),
         "k1": dataclasses.replace(base, k=1, E=16, n_shared=2, I=192, I_shared=64),
+        # SiTU-GLU experts.  Weights N(0, 0.15) drive the gate past its cap of 4
+        # on about 1 element in 10 while the layer's outputs stay near the scale
+        # the tolerance is stated for (at N(0, 0.5) outputs in the hundreds
+        # cancel, and a one-ulp flip of a bf16 h moves them past it); tight
+        # caps saturate both branches on the default weights.
+        "situ_caps": dataclasses.replace(base, activation=1, weight_sigma=0.15, name="situ_caps"),
+        "situ_tight_caps": dataclasses.replace(base, activation=1, situ_beta_gate=0.25,
+                                               situ_beta_up=0.5, name="situ_tight"),
     }[variant]
+    run = Run(cfg)
+    out = run.forward(*run.inputs())
+    ref, _ = oracle_full(cfg)
+    same = check_routing(out, ref)
+    check_outputs(out, ref, same_rows=same)
+
+
+def test_fine_grained_situ_parity(torch_cuda):
+    """SiTU-GLU experts on the fine-grained shapes (a 512-token batch)."""
+    cfg = dataclasses.replace(W.C2S, T=512)
     run = Run(cfg)
     out = run.forward(*run.inputs())
     ref, _ = oracle_full(cfg)
