@@ -37,6 +37,11 @@ The layer, in order:
                                           weighted sum, one final cast)
   8. residual add + RMSNorm epilogue     [FW] Trap 2 / Trap 3 (rmsnorm(full_out + residual))
   9. fixed r0..r7 partial reduction      [FW] Trap 1 (Lamport kernel order)
+  Latent MoE (optional)                  [LD] "潜在MoE (Latent MoE)", K3 flow: the
+                                          router and routed experts read
+                                          z = bf16(xn W_down^T); their weighted
+                                          sum is cast once and projected back by
+                                          W_up; shared experts stay at full width
 
 Precision.  Every floating-point step runs in fp64, on the bf16-rounded values
 the GPU path reads (x, residual, weights, xn between steps 1 and 2/6, h between
@@ -315,6 +320,26 @@ def expert_ffn(xn_rows, w_gate, w_up, w_down, gate_clamp_max=np.inf, up_clamp=np
     return h, h @ Wd.T
 
 
+# ------------------------------------------------------------ latent MoE
+def latent_down(xn, w_proj_down) -> np.ndarray:
+    """z = bf16(xn W_down^T): the down-projection W_down of [LD] "潜在MoE (Latent
+    MoE)" / "K3 的 Stable Latent MoE" (input -> down-projection -> choose the
+    experts -> each expert's GLU in the latent space of width l -> weighted sum
+    -> up-projection -> back to the hidden space).  z is an activation between
+    two matmuls, so it is a bf16 value like xn and h."""
+    return round_bf16(np.asarray(xn, np.float64) @ np.asarray(w_proj_down, np.float64).T)
+
+
+def latent_up(w, y_slots, w_proj_up):
+    """s = sum_j w_j y_j (the routed experts' latent outputs, slot order),
+    a = bf16(s) (one cast; [FW] case study's standard path for the weighted
+    sum), then y = a W_up^T, the up-projection back to the hidden width ([LD]
+    "潜在MoE").  Returns (s, a, y)."""
+    s = np.einsum("tj,tjl->tl", np.asarray(w, np.float64), np.asarray(y_slots, np.float64))
+    a = round_bf16(s)
+    return s, a, a @ np.asarray(w_proj_up, np.float64).T
+
+
 # --------------------------------------------- 7-8. combine + residual + norm
 def combine(w, y_slots, y_shared) -> np.ndarray:
     """acc[t] = sum_j w[t,j] * y[t,j] (slot order) + sum_s y_shared[s,t]
@@ -381,7 +406,8 @@ class Weights:
     that regenerates a single expert on demand."""
 
     def __init__(self, w_router, router_bias, w_gate, w_up, w_down, ws_gate, ws_up, ws_down,
-                 g_in, g_out):
+                 g_in, g_out, w_proj_down=None, w_proj_up=None):
+        self.w_proj_down, self.w_proj_up = w_proj_down, w_proj_up  # latent MoE only
         self.w_router = w_router
         self.router_bias = router_bias
         self.w_gate, self.w_up, self.w_down = w_gate, w_up, w_down
@@ -400,14 +426,22 @@ def moe_layer(cfg, W, x, residual, token_ids=None, rows=None) -> dict:
     every token; the experts, combine and epilogue for ``rows`` (all tokens
     when None).  ``cfg`` carries D, E, k, I, n_shared, I_shared, router,
     renormalize, routed_scale, gate_clamp_max, up_clamp, eps, hash_mult and
-    optionally activation, situ_beta_gate, situ_beta_up (SiTU-GLU experts)."""
+    optionally activation, situ_beta_gate, situ_beta_up (SiTU-GLU experts) and
+    latent (the latent width l; 0 or absent: no latent projection).
+
+    Latent MoE ([LD] "潜在MoE" and its K3 flow): the router and the routed
+    experts read z = latent_down(xn) (width l), the routed experts' weighted sum
+    is projected back by latent_up, and the shared experts keep the full width
+    (they read xn)."""
     x = np.asarray(x, np.float64)
     T = x.shape[0]
     rows = np.arange(T) if rows is None else np.asarray(rows, np.int64)
     xn = rmsnorm_bf16_code(x, W.g_in, cfg.eps)
+    lat = int(getattr(cfg, "latent", 0) or 0)
+    xe = latent_down(xn, W.w_proj_down) if lat else xn   # what the router and routed experts read
     logits = None
     if cfg.router != ROUTER_HASH:
-        logits = router_logits(xn, W.w_router)
+        logits = router_logits(xe, W.w_router)
     idx, w, keys = route(cfg, logits, W.router_bias, token_ids)
     margin = topk_margin(keys, cfg.k)
     counts = expert_histogram(idx, cfg.E)
@@ -415,22 +449,29 @@ def moe_layer(cfg, W, x, residual, token_ids=None, rows=None) -> dict:
 
     # Expert compute for the selected rows, grouped by expert.
     n, k = len(rows), cfg.k
-    y_slots = np.zeros((n, k, cfg.D))
+    y_slots = np.zeros((n, k, lat or cfg.D))
     sel = idx[rows]                                   # [n, k]
     for e in np.unique(sel):
         rr, jj = np.nonzero(sel == e)
         Wg, Wu, Wd = W.routed(int(e))
-        _, y = expert_ffn(xn[rows[rr]], Wg, Wu, Wd, **unit_args(cfg))
+        _, y = expert_ffn(xe[rows[rr]], Wg, Wu, Wd, **unit_args(cfg))
         y_slots[rr, jj] = y
     y_shared = np.zeros((cfg.n_shared, n, cfg.D))
     for s in range(cfg.n_shared):
         Wg, Wu, Wd = W.shared(s)
         # The clamp is a property of the SwiGLU unit and applies to shared experts too.
         _, y_shared[s] = expert_ffn(xn[rows], Wg, Wu, Wd, **unit_args(cfg))
-    acc = combine(w[rows], y_slots, y_shared)
+    agg = lat_sum = None
+    if lat:
+        lat_sum, agg, y_lat = latent_up(w[rows], y_slots, W.w_proj_up)
+        acc = combine(np.ones((n, 1)), y_lat[:, None, :], y_shared)   # projected sum, then shared
+    else:
+        acc = combine(w[rows], y_slots, y_shared)
     out_norm, out_residual, r = residual_rmsnorm(acc, np.asarray(residual, np.float64)[rows],
                                                  W.g_out, cfg.eps)
-    return dict(rows=rows, xn=xn, logits=logits, keys=keys, idx=idx, w=w, margin=margin,
+    return dict(rows=rows, xn=xn, z=xe if lat else None, lat_sum=lat_sum, agg=agg, logits=logits,
+                keys=keys, idx=idx,
+                w=w, margin=margin,
                 counts=counts, offsets=offsets, perm_token=perm_token, perm_slot=perm_slot,
                 pos=pos, y_slots=y_slots, y_shared=y_shared, acc=acc, r=r,
                 out_norm=out_norm, out_residual=out_residual)
@@ -443,18 +484,24 @@ def moe_layer_dense_masked(cfg, W, x, residual, token_ids=None) -> dict:
     x = np.asarray(x, np.float64)
     T = x.shape[0]
     xn = rmsnorm_bf16_code(x, W.g_in, cfg.eps)
-    logits = None if cfg.router == ROUTER_HASH else router_logits(xn, W.w_router)
+    lat = int(getattr(cfg, "latent", 0) or 0)
+    xe = latent_down(xn, W.w_proj_down) if lat else xn
+    logits = None if cfg.router == ROUTER_HASH else router_logits(xe, W.w_router)
     idx, w, _ = route(cfg, logits, W.router_bias, token_ids)
     mask = np.zeros((T, cfg.E))
     np.put_along_axis(mask, idx, w, axis=-1)
-    acc = np.zeros((T, cfg.D))
+    acc = np.zeros((T, lat or cfg.D))
     for e in range(cfg.E):
         Wg, Wu, Wd = W.routed(e)
-        _, y = expert_ffn(xn, Wg, Wu, Wd, **unit_args(cfg))
+        _, y = expert_ffn(xe, Wg, Wu, Wd, **unit_args(cfg))
         acc += mask[:, e:e + 1] * y
+    lat_sum = None
+    if lat:
+        lat_sum = acc
+        acc = round_bf16(acc) @ np.asarray(W.w_proj_up, np.float64).T
     for s in range(cfg.n_shared):
         Wg, Wu, Wd = W.shared(s)
         _, y = expert_ffn(xn, Wg, Wu, Wd, **unit_args(cfg))
         acc += y
     out_norm, out_residual, r = residual_rmsnorm(acc, residual, W.g_out, cfg.eps)
-    return dict(acc=acc, r=r, out_norm=out_norm, out_residual=out_residual, idx=idx, w=w)
+    return dict(acc=acc, r=r, out_norm=out_norm, out_residual=out_residual, idx=idx, w=w, lat_sum=lat_sum)

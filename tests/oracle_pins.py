@@ -415,4 +415,96 @@ def pin_mac_count(O):
         assert O.MAC_COUNTER[0] == 10 * 3 * 3 * 64 * 32 + 10 * S * 3 * 64 * 32
 
 
+# ------------------------------------------------------------ latent MoE
+def pin_latent_closed_form(O):
+    """[LD] "潜在MoE": down-project, route and run the experts in the latent
+    space, sum, up-project; shared experts at full width.  T=1, D=2, l=1, two
+    routed experts (top-1, renormalised), one shared expert, by hand."""
+    bf = O.round_bf16
+    cfg = _cfg(D=2, E=2, k=1, I=1, n_shared=1, I_shared=1, renormalize=1, latent=1)
+    W = O.Weights(w_router=np.array([[1.0], [-1.0]]), router_bias=None,
+                  w_gate=np.array([[[2.0]], [[1.0]]]), w_up=np.array([[[1.0]], [[1.0]]]),
+                  w_down=np.array([[[0.375]], [[1.0]]]),
+                  ws_gate=np.array([[[0.5, 0.5]]]), ws_up=np.array([[[1.0, -0.5]]]),
+                  ws_down=np.array([[[1.0], [0.25]]]), g_in=np.ones(2), g_out=np.ones(2),
+                  w_proj_down=np.array([[129 / 256, 129 / 512]]), w_proj_up=np.array([[2.0], [-4.0]]))
+    assert np.array_equal(bf(W.w_proj_down), W.w_proj_down)
+    out = O.moe_layer(cfg, W, np.array([[1.0, 1.0]]), np.zeros((1, 2)))
+    # xn = bf16(1 / sqrt(1 + 1e-6)) = 1; z = bf16(387/512), a tie between 193/256
+    # and 194/256 that goes to the even 194/256.
+    assert np.array_equal(out["xn"][0], [1.0, 1.0])
+    z = 194 / 256
+    assert out["z"][0, 0] == z
+    # Router on z: logits [z, -z], expert 0, weight 1 after renormalising.
+    assert out["idx"][0, 0] == 0 and out["w"][0, 0] == 1.0
+    # Expert 0 in the latent space: g = 2z, u = z, h = bf16(g sigmoid(g) u).
+    g = 2 * z
+    hv = g / (1.0 + math.exp(-g)) * z
+    assert 240.5 / 256 < hv < 241.5 / 256
+    # y0 = h * 0.375 = 723/2048; a = bf16(y0) = 181/512 (723/2048 = 180.75/512).
+    assert out["lat_sum"][0, 0] == 723 / 2048
+    assert out["agg"][0, 0] == 181 / 512
+    # Shared expert on xn at full width: g = 1, u = 0.5, h = bf16(sigmoid(1) / 2) = 187/512.
+    hs = 0.5 / (1.0 + math.exp(-1.0))
+    assert 186.5 / 512 < hs < 187.5 / 512
+    acc = np.array([181 / 256 + 187 / 512, -181 / 128 + 187 / 2048])
+    assert np.array_equal(out["acc"][0], acc)
+    # out_residual = bf16(acc): 137.25/128 -> 137/128, -169.3125/128 -> -169/128.
+    assert np.array_equal(out["out_residual"][0], [137 / 128, -169 / 128])
+
+
+def _latent_case(O, l=16, router=0, S=1, seed=11, **kw):
+    cfg, W, x, res, ids = small_random_case(O, router=router, S=S, seed=seed, **kw)
+    rng = np.random.default_rng(seed + 1)
+    bf = O.round_bf16
+    E, D, I = cfg.E, cfg.D, cfg.I
+    cfg.latent = l
+    W.w_router = bf(rng.standard_normal((E, l)) * 0.3)
+    W.w_gate = bf(rng.standard_normal((E, I, l)) * 0.2)
+    W.w_up = bf(rng.standard_normal((E, I, l)) * 0.2)
+    W.w_down = bf(rng.standard_normal((E, l, I)) * 0.2)
+    W.w_proj_down = bf(rng.standard_normal((l, D)) * 0.15)
+    W.w_proj_up = bf(rng.standard_normal((D, l)) * 0.2)
+    return cfg, W, x, res, ids
+
+
+def pin_latent_dense_masked(O):
+    # The routed latent sum equals every expert run on every token's z, masked
+    # to its routing weights, and sampled rows equal the full run's rows.
+    for router, extra in [(0, {"renormalize": 1}), (1, {"renormalize": 1, "routed_scale": 2.5})]:
+        cfg, W, x, res, ids = _latent_case(O, router=router, **extra)
+        a = O.moe_layer(cfg, W, x, res, ids)
+        b = O.moe_layer_dense_masked(cfg, W, x, res, ids)
+        assert np.array_equal(a["idx"], b["idx"])
+        assert np.allclose(a["lat_sum"], b["lat_sum"], rtol=1e-12, atol=1e-13)
+        rows = np.array([5, 1])
+        c = O.moe_layer(cfg, W, x, res, ids, rows=rows)
+        assert np.array_equal(c["out_norm"], a["out_norm"][rows])
+
+
+def pin_latent_identity_projection(O):
+    # With l = D and identity projections the latent layer is the plain layer
+    # with its routed sum cast to bf16 before the shared experts are added.
+    cfg, W, x, res, ids = small_random_case(O, router=0, renormalize=1, seed=13)
+    plain = O.moe_layer(cfg, W, x, res, ids)
+    cfg_l = _cfg(**{**vars(cfg), "latent": cfg.D})
+    eye = np.eye(cfg.D)
+    W.w_proj_down, W.w_proj_up = eye, eye
+    lat = O.moe_layer(cfg_l, W, x, res, ids)
+    assert np.array_equal(lat["z"], plain["xn"]) and np.array_equal(lat["idx"], plain["idx"])
+    routed = np.einsum("tj,tjd->td", plain["w"], plain["y_slots"])
+    want = O.round_bf16(routed) + np.sum(plain["y_shared"], axis=0)
+    assert np.allclose(lat["acc"], want, rtol=1e-15, atol=1e-15)
+
+
+def pin_latent_mac_count(O):
+    # [LD] "FLOPs与参数量" with the routed experts at the latent width l: the
+    # expert matmuls perform T*k*3*l*I + T*S*3*D*I_s multiply-adds.
+    cfg, W, x, res, ids = _latent_case(O, l=16, S=1)
+    O.MAC_COUNTER[0] = 0
+    O.moe_layer(cfg, W, x, res, ids)
+    T = x.shape[0]
+    assert O.MAC_COUNTER[0] == T * cfg.k * 3 * 16 * cfg.I + T * 1 * 3 * cfg.D * cfg.I_shared
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

@@ -59,6 +59,14 @@ MUTATIONS = {
                              "    acc = parts[-1].copy()\n    for p in range(parts.shape[0] - 2, -1, -1):\n        acc = np.add(acc, parts[p], dtype=np.float32)"),
     "partials_residual_in_fp64": ("r = np.add(s, np.asarray(residual, np.float32), dtype=np.float32)",
                                   "r = s.astype(np.float64) + np.asarray(residual, np.float64) + 2.0 ** -30"),
+    "latent_z_not_rounded": ("    return round_bf16(np.asarray(xn, np.float64) @ np.asarray(w_proj_down, np.float64).T)",
+                             "    return np.asarray(xn, np.float64) @ np.asarray(w_proj_down, np.float64).T"),
+    "latent_sum_not_rounded": ("    a = round_bf16(s)\n", "    a = s\n"),
+    "latent_router_reads_xn": ("        logits = router_logits(xe, W.w_router)", "        logits = router_logits(xn, W.w_router)"),
+    "latent_experts_read_xn": ("_, y = expert_ffn(xe[rows[rr]]", "_, y = expert_ffn(xn[rows[rr]]"),
+    "latent_shared_reads_z": ("_, y_shared[s] = expert_ffn(xn[rows]", "_, y_shared[s] = expert_ffn(xe[rows]"),
+    "latent_shared_dropped": ("        acc = combine(np.ones((n, 1)), y_lat[:, None, :], y_shared)",
+                              "        acc = combine(np.ones((n, 1)), y_lat[:, None, :], None)"),
     "histogram_off_by_one": ("return np.bincount(np.asarray(idx).ravel(), minlength=E).astype(np.int64)",
                              "return np.bincount(np.asarray(idx).ravel() % max(E - 1, 1), minlength=E).astype(np.int64)"),
 }
