@@ -70,7 +70,7 @@ def describe(cfg):
             "n_shared": cfg.n_shared, "I_shared": cfg.I_shared,
             "router": {0: "softmax", 1: "sigmoid+bias", 2: "hash"}[cfg.router],
             "renormalize": bool(cfg.renormalize),
-            "activation": "SiTU-GLU" if cfg.activation == 1 else "SwiGLU"}
+            "activation": "SiTU-GLU" if cfg.activation == 1 else "SwiGLU", "latent": cfg.latent}
 
 
 def peaks():
@@ -405,11 +405,7 @@ def main():
     x, r, ids = (xa[rank * T:(rank + 1) * T].contiguous(), ra[rank * T:(rank + 1) * T].contiguous(),
                  ida[rank * T:(rank + 1) * T].contiguous())
     del xa, ra, ida
-    lc = moe.LayerConfig(D=cfg.D, E=cfg.E, k=cfg.k, I=cfg.I, n_shared=cfg.n_shared,
-                         I_shared=cfg.I_shared, T_max=T, router=cfg.router,
-                         renormalize=cfg.renormalize, routed_scale=cfg.routed_scale,
-                         gate_clamp_max=cfg.gate_clamp_max, up_clamp=cfg.up_clamp, eps=cfg.eps,
-                         hash_mult=cfg.hash_mult)
+    lc = SD.layer_config(cfg, T_max=T)
     layer = moe.MoELayer(lc, w)
     ws = torch.empty(layer.workspace_size(T), dtype=torch.uint8, device=dev)
     on = torch.empty((T, cfg.D), dtype=torch.bfloat16, device=dev)

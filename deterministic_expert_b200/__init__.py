@@ -22,9 +22,10 @@ MOE_OK, MOE_EINVAL, MOE_ETOOBIG, MOE_EWORKSPACE, MOE_EUNSUPPORTED, MOE_ECUDA, MO
     0, -1, -2, -3, -4, -5, -6)
 ROUTER_SOFTMAX, ROUTER_SIGMOID_BIAS, ROUTER_HASH = 0, 1, 2
 ACT_SWIGLU, ACT_SITU_GLU = 0, 1
-NUM_STAGES = 8
+NUM_STAGES = 11
 STAGE_NAMES = ("rmsnorm_in", "router_gemm", "router_topk", "dispatch", "gather_rows",
-               "gemm_gateup_swiglu", "gemm_down", "combine_norm")
+               "gemm_gateup_swiglu", "gemm_down", "combine_norm", "latent_down", "latent_combine",
+               "latent_up")
 
 
 class MoEError(RuntimeError):
@@ -40,12 +41,13 @@ class moe_config(ctypes.Structure):
                 ("routed_scale", ctypes.c_float), ("gate_clamp_max", ctypes.c_float),
                 ("up_clamp", ctypes.c_float), ("eps", ctypes.c_float), ("hash_mult", ctypes.c_uint32),
                 ("activation", ctypes.c_int), ("situ_beta_gate", ctypes.c_float),
-                ("situ_beta_up", ctypes.c_float)]
+                ("situ_beta_up", ctypes.c_float), ("latent", ctypes.c_int)]
 
 
 class moe_weights(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in ("w_router", "router_bias", "w_gate", "w_up", "w_down",
-                                               "ws_gate", "ws_up", "ws_down", "g_in", "g_out")]
+                                               "ws_gate", "ws_up", "ws_down", "g_in", "g_out",
+                                               "w_proj_down", "w_proj_up")]
 
 
 class moe_views(ctypes.Structure):
@@ -54,7 +56,8 @@ class moe_views(ctypes.Structure):
                 ("offsets", ctypes.c_void_p), ("src_token", ctypes.c_void_p),
                 ("dest_row", ctypes.c_void_p), ("h_routed", ctypes.c_void_p),
                 ("h_shared", ctypes.c_void_p), ("y_slot", ctypes.c_void_p),
-                ("y_shared", ctypes.c_void_p)]
+                ("y_shared", ctypes.c_void_p), ("z", ctypes.c_void_p), ("agg", ctypes.c_void_p),
+                ("y_latent", ctypes.c_void_p)]
 
 
 _lib = None
@@ -129,13 +132,36 @@ class LayerConfig:
     activation: int = ACT_SWIGLU
     situ_beta_gate: float = 4.0
     situ_beta_up: float = 25.0
+    latent: int = 0
 
     def to_c(self) -> moe_config:
         return moe_config(self.D, self.E, self.k, self.I, self.n_shared,
                           self.I_shared if self.n_shared else self.I, self.T_max, self.router,
                           self.renormalize, self.routed_scale, self.gate_clamp_max, self.up_clamp,
                           self.eps, self.hash_mult, self.activation, self.situ_beta_gate,
-                          self.situ_beta_up)
+                          self.situ_beta_up, self.latent)
+
+
+def _check_weight_sizes(cfg: LayerConfig, weights: dict) -> None:
+    """The library reads each weight through a descriptor sized from the
+    configuration, so a tensor of another size must be refused here."""
+    L = cfg.latent or cfg.D
+    S, Is = cfg.n_shared, (cfg.I_shared if cfg.n_shared else cfg.I)
+    want = {"w_router": cfg.E * L, "router_bias": cfg.E, "w_gate": cfg.E * cfg.I * L,
+            "w_up": cfg.E * cfg.I * L, "w_down": cfg.E * L * cfg.I, "ws_gate": S * Is * cfg.D,
+            "ws_up": S * Is * cfg.D, "ws_down": S * cfg.D * Is, "g_in": cfg.D, "g_out": cfg.D,
+            "w_proj_down": cfg.latent * cfg.D, "w_proj_up": cfg.D * cfg.latent}
+    for name, n in want.items():
+        t = weights.get(name)
+        if t is None:
+            continue
+        if not t.is_contiguous() or t.numel() != n:
+            raise ValueError(f"weight {name}: expected {n} contiguous elements for this configuration, "
+                             f"got {t.numel()} (contiguous={t.is_contiguous()})")
+        import torch
+        dtype = torch.float32 if name == "router_bias" else torch.bfloat16
+        if t.dtype != dtype:
+            raise ValueError(f"weight {name}: expected {dtype}, got {t.dtype}")
 
 
 class MoELayer:
@@ -145,6 +171,7 @@ class MoELayer:
 
     def __init__(self, cfg: LayerConfig, weights: dict):
         self.cfg = cfg
+        _check_weight_sizes(cfg, weights)
         self._keep = dict(weights)
         w = moe_weights(*[_ptr(weights.get(n)) for n, _ in moe_weights._fields_])
         h = ctypes.c_void_p()

@@ -136,7 +136,7 @@ __global__ void __launch_bounds__(kDispatchRows) k_dispatch(const DispatchArgs a
     for (int g = tid; g <= G; g += kDispatchRows) a.tiles_gu[g] = tstart[g];
     __syncthreads();
     for (int g = tid; g < G; g += kDispatchRows)
-      cnt[g] = (g < a.E ? (total[g] + a.tile_m - 1) / a.tile_m : mt_shared) * a.dn_ntiles;
+      cnt[g] = g < a.E ? (total[g] + a.tile_m - 1) / a.tile_m * a.dn_ntiles : mt_shared * a.dn_ntiles_shared;
     __syncthreads();
     block_exclusive_scan(cnt, tstart, G, warp_tot);
     for (int g = tid; g <= G; g += kDispatchRows) a.tiles_dn[g] = tstart[g];

@@ -71,23 +71,24 @@ struct Tile {
 
 template <int CG>
 __device__ __forceinline__ void decode_tile(const GemmArgs& a, int t, Tile& ti) {
+  int local = t;
   if (a.tile_start == nullptr) {
-    ti.kind = 0; ti.idx = 0; ti.rows = a.T; ti.a_row0 = 0; ti.m = t; ti.n = 0; ti.small = false;
-    ti.swap = false; ti.nt = 0;
-    return;
-  }
+    // One dense group of T rows (router, latent projections) of kind dense_kind.
+    ti.kind = a.dense_kind; ti.idx = 0; ti.rows = a.T; ti.a_row0 = 0;
+  } else {
   // Largest g with tile_start[g] <= t; tile_start[0] = 0 <= t < tile_start[G].
   int lo = 0, hi = a.G;
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
     if (a.tile_start[mid] <= t) lo = mid; else hi = mid;
   }
-  const int local = t - a.tile_start[lo];
+  local = t - a.tile_start[lo];
   if (lo < a.E) {
     const int o0 = a.offsets[lo];
     ti.kind = 0; ti.idx = lo; ti.rows = a.offsets[lo + 1] - o0; ti.a_row0 = o0;
   } else {
     ti.kind = 1; ti.idx = lo - a.E; ti.rows = a.T; ti.a_row0 = ti.idx * a.shared_a_stride;
+  }
   }
   const int mt = (ti.rows + Cfg<CG>::kTileM - 1) / Cfg<CG>::kTileM;
   ti.n = local / mt;
@@ -106,23 +107,27 @@ __device__ __forceinline__ float silu_clamped_product(float g, float u, float cg
   return __fdividef(g, 1.0f + __expf(-g)) * u;
 }
 
-// tanh(z) = sign(z) (1 - e^{-2|z|}) / (1 + e^{-2|z|}), each step an explicitly
-// rounded fp32 operation or an intrinsic, none of which the compiler may fuse
-// or reorder, so the result is the same bits wherever it is inlined.  Error
-// about 1e-7 absolute (the exponential's), far below the bf16 rounding of h.
-__device__ __forceinline__ float tanh_rn(float z) {
-  const float e = __expf(__fmul_rn(-2.0f, fabsf(z)));
-  return copysignf(__fdividef(__fsub_rn(1.0f, e), __fadd_rn(1.0f, e)), z);
-}
-
-// SiTU-GLU: [bg tanh(g / bg) * sigmoid(g)] * [bu tanh(u / bu)] in fp32 (the
-// linux.do post on MoE variants, "SiTU-GLU": soft caps on both branches);
-// ibg = 1 / bg and ibu = 1 / bu are rounded once on the host.
+// SiTU-GLU: [bg tanh(g / bg) * sigmoid(g)] * [bu tanh(u / bu)] (the linux.do
+// post on MoE variants, "SiTU-GLU": soft caps on both branches), written with
+// tanh(z) = sign(z) (1 - e^{-2|z|}) / (1 + e^{-2|z|}) and sigmoid(g) =
+// 1 / (1 + e^{-g}) over one common denominator:
+//   h = sign(g u) bg bu (1 - e1)(1 - e3) / ((1 + e1)(1 + e2)(1 + e3)),
+//   e1 = e^{-2|g|/bg}, e2 = e^{-g}, e3 = e^{-2|u|/bu}
+// (three exponentials, one division).  A very negative g makes e2 infinite
+// and h 0, as the closed gate should.  Every step is an explicitly rounded
+// fp32 operation or an intrinsic, which the compiler may not fuse or reorder,
+// so the result is the same bits wherever the function is inlined; the error
+// is a few ulp of fp32, far below the bf16 rounding of h.  ibg = 1 / bg,
+// ibu = 1 / bu are rounded once on the host.
 __device__ __forceinline__ float situ_glu_product(float g, float u, float bg, float bu, float ibg,
                                                   float ibu) {
-  const float sig = __fdividef(1.0f, __fadd_rn(1.0f, __expf(-g)));
-  const float gate = __fmul_rn(__fmul_rn(bg, tanh_rn(__fmul_rn(g, ibg))), sig);
-  return __fmul_rn(gate, __fmul_rn(bu, tanh_rn(__fmul_rn(u, ibu))));
+  const float e1 = __expf(__fmul_rn(__fmul_rn(-2.0f, fabsf(g)), ibg));
+  const float e2 = __expf(-g);
+  const float e3 = __expf(__fmul_rn(__fmul_rn(-2.0f, fabsf(u)), ibu));
+  const float num = __fmul_rn(__fsub_rn(1.0f, e1), __fsub_rn(1.0f, e3));
+  const float den = __fmul_rn(__fmul_rn(__fadd_rn(1.0f, e1), __fadd_rn(1.0f, e2)), __fadd_rn(1.0f, e3));
+  const float mag = __fmul_rn(__fmul_rn(bg, bu), __fdividef(num, den));
+  return (g < 0.f) != (u < 0.f) ? -mag : mag;
 }
 
 // The experts' gated unit (the same function in every tile shape).
@@ -391,6 +396,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
           const bool scatter = (MODE == kDown && ti.kind == 0);
           const int col = ti.n * BN + static_cast<int>(rank) * (BN / 2) + 32 * q + lane;
           float* outb = static_cast<float*>(a.out[ti.kind]);
+          uint16_t* outh = static_cast<uint16_t*>(a.out[ti.kind]);  // out_bf16
           const size_t ld = static_cast<size_t>(a.ld_out[ti.kind]);
           const int orow0 = (ti.kind == 0 ? ti.a_row0 : ti.idx * a.shared_out_stride) + trow0;
           for (int c = 32 * half; c < ti.nt; c += 64) {
@@ -403,7 +409,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
               const int orow = __shfl_sync(0xffffffffu, my_row, j);
-              if (c + j < r) outb[static_cast<size_t>(orow) * ld + col] = __uint_as_float(v[j]);
+              if (c + j < r) {
+                if (a.out_bf16)
+                  outh[static_cast<size_t>(orow) * ld + col] =
+                      static_cast<uint16_t>(pack_bf16x2(__uint_as_float(v[j]), 0.f) & 0xFFFFu);
+                else
+                  outb[static_cast<size_t>(orow) * ld + col] = __uint_as_float(v[j]);
+              }
             }
           }
         }
@@ -470,7 +482,30 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
           uint32_t v[32];
           tmem_ld32(tb + c, v);
           tmem_ld_wait();
-          if (ncols - c >= 32) {
+          if (ncols - c >= 32 && a.out_bf16) {
+            // bf16 output (latent down-projection): 64 bytes per row, four
+            // 16-byte chunks, staged so each store covers whole row segments.
+            uint16_t* oh = static_cast<uint16_t*>(a.out[ti.kind]) + ti.n * BN + colhalf * (BN / 2);
+#pragma unroll
+            for (int m = 0; m < 4; ++m)
+              *reinterpret_cast<uint4*>(stage_w + lane * 128 + ((m ^ (lane & 7)) << 4)) =
+                  make_uint4(pack_bf16x2(__uint_as_float(v[8 * m]), __uint_as_float(v[8 * m + 1])),
+                             pack_bf16x2(__uint_as_float(v[8 * m + 2]), __uint_as_float(v[8 * m + 3])),
+                             pack_bf16x2(__uint_as_float(v[8 * m + 4]), __uint_as_float(v[8 * m + 5])),
+                             pack_bf16x2(__uint_as_float(v[8 * m + 6]), __uint_as_float(v[8 * m + 7])));
+            __syncwarp();
+#pragma unroll
+            for (int s4 = 0; s4 < 4; ++s4) {
+              const int r = 8 * s4 + (lane >> 2), ch = lane & 3;
+              const int drow = __shfl_sync(0xffffffffu, my_dest, r);
+              if (r < nvalid) {
+                const uint4 val = *reinterpret_cast<const uint4*>(stage_w + r * 128 + ((ch ^ (r & 7)) << 4));
+                const size_t orow = scatter ? static_cast<size_t>(drow) : static_cast<size_t>(orow0 + r);
+                *reinterpret_cast<uint4*>(oh + orow * ld + c + 8 * ch) = val;
+              }
+            }
+            __syncwarp();
+          } else if (ncols - c >= 32) {
 #pragma unroll
             for (int m = 0; m < 8; ++m)
               *reinterpret_cast<uint4*>(stage_w + lane * 128 + ((m ^ (lane & 7)) << 4)) =

@@ -18,8 +18,10 @@ struct moe_handle {
   moe_config cfg;
   moe_weights w;
   int S = 0, G = 0, E_pad = 0, bn_gu = 0, bn_dn = 0, num_sms = 0, device = 0, max_pairs = 0;
-  uint16_t* w_router_pad = nullptr;  // [E_pad, D], rows >= E zero
-  CUtensorMap map_router, map_wg, map_wu, map_wd, map_wsg, map_wsu, map_wsd;
+  int L = 0;                          // width the router and routed experts read (latent or D)
+  int bn_pd = 0, bn_pu = 0;           // N tiles of the latent down / up projections
+  uint16_t* w_router_pad = nullptr;  // [E_pad, L], rows >= E zero
+  CUtensorMap map_router, map_wg, map_wu, map_wd, map_wsg, map_wsu, map_wsd, map_pd, map_pu;
   unsigned long long timeout_ns = 2000ull * 1000 * 1000;
   // Per-stage timing (moe_profile_*).
   int prof_mask = 0;
@@ -36,7 +38,7 @@ size_t align256(size_t b) { return (b + 255) & ~static_cast<size_t>(255); }
 
 struct Layout {
   size_t err, xn, logits, tidx, tw, bcount, counts, offsets, tiles_gu, tiles_dn, dest, src,
-      xp, h, hs, y, ys, total;
+      xp, h, hs, y, ys, z, agg, ylat, total;
 };
 
 Layout layout(const moe_handle* h, int T) {
@@ -57,11 +59,16 @@ Layout layout(const moe_handle* h, int T) {
   L.tiles_dn = take(static_cast<size_t>(h->G + 1) * 4);
   L.dest = take(Tz * c.k * 4);
   L.src = take(Tz * c.k * 4);
-  L.xp = take(Tz * c.k * c.D * 2);
+  const size_t Lw = static_cast<size_t>(h->L);
+  L.xp = take(Tz * c.k * Lw * 2);
   L.h = take(Tz * c.k * c.I * 2);
   L.hs = take(static_cast<size_t>(h->S) * Tz * c.I_shared * 2);
-  L.y = take(Tz * c.k * c.D * 4);
+  L.y = take(Tz * c.k * Lw * 4);
   L.ys = take(static_cast<size_t>(h->S) * Tz * c.D * 4);
+  const bool lat = c.latent > 0;
+  L.z = take(lat ? Tz * Lw * 2 : 0);
+  L.agg = take(lat ? Tz * Lw * 2 : 0);
+  L.ylat = take(lat ? Tz * c.D * 4 : 0);
   L.total = off;
   return L;
 }
@@ -122,6 +129,11 @@ int validate_config(const moe_config* c, const moe_weights* w) {
       !(c->gate_clamp_max == c->gate_clamp_max) || !(c->up_clamp >= 0.f))
     return MOE_EINVAL;
   if (c->n_shared > 0 && c->I_shared <= 0) return MOE_EINVAL;
+  if (c->latent < 0) return MOE_EINVAL;
+  if (c->latent > 0 && (c->latent % 64 || c->latent > 16384)) return MOE_EUNSUPPORTED;
+  if (c->latent > 0 && (!w->w_proj_down || !w->w_proj_up || !aligned16(w->w_proj_down) ||
+                        !aligned16(w->w_proj_up)))
+    return MOE_EINVAL;
   if (c->activation != MOE_ACT_SWIGLU && c->activation != MOE_ACT_SITU_GLU) return MOE_EINVAL;
   if (c->activation == MOE_ACT_SITU_GLU &&
       !(c->situ_beta_gate > 0.f && c->situ_beta_gate < 3.0e38f && c->situ_beta_up > 0.f &&
@@ -206,6 +218,32 @@ int forward_impl(moe_handle* h, int T, const uint16_t* x, const uint16_t* residu
   float* y = reinterpret_cast<float*>(ws + L.y);
   float* ys = reinterpret_cast<float*>(ws + L.ys);
   const int TK = T * c.k;
+  const bool lat = c.latent > 0;
+  uint16_t* zb = reinterpret_cast<uint16_t*>(ws + L.z);
+  uint16_t* aggb = reinterpret_cast<uint16_t*>(ws + L.agg);
+  float* ylat = reinterpret_cast<float*>(ws + L.ylat);
+  const int LW = h->L;
+
+  // One dense group of T rows through the CTA-pair GEMM (latent projections):
+  // out[T, N] = A[T, K] B[N, K]^T, bf16 or fp32 out.
+  auto dense_gemm = [&](const uint16_t* A, int K, const CUtensorMap& B, int N, int BN, void* out,
+                        int out_bf16) -> int {
+    GemmArgs g;
+    std::memset(&g, 0, sizeof(g));
+    if (!make_map(&g.mapA[1], A, K, T, kBM) || !make_map(&g.mapA64[1], A, K, T, kBM / 2) ||
+        !make_map(&g.mapA16[1], A, K, T, 16))
+      return MOE_ECUDA;
+    g.mapB[2] = B;
+    g.T = T; g.G = 1; g.E = 0;
+    g.n_kind[1] = N; g.k_kind[1] = K;
+    g.BN = BN;
+    g.swap_ok = BN == 256;
+    g.dense_kind = 1;
+    g.router_tiles = (T + kPairTileM - 1) / kPairTileM * (N / BN);
+    g.out[1] = out; g.ld_out[1] = N; g.out_bf16 = out_bf16;
+    g.err = err; g.timeout_ns = h->timeout_ns;
+    return launch_grouped_gemm(kDown, g, pair_grid(h, g.router_tiles), s) == cudaSuccess ? MOE_OK : MOE_ECUDA;
+  };
 
   Prof prof{h, s, -1};
   if (h->prof_mask && h->prof_fwd < kProfFwd) prof.f = h->prof_fwd++;
@@ -218,17 +256,27 @@ int forward_impl(moe_handle* h, int T, const uint16_t* x, const uint16_t* residu
   MOE_TRY(launch_rmsnorm_rows(x, h->w.g_in, xn, T, c.D, c.eps, err, bcount, nblk * E4, s));
   prof.end(0);
 
+  // Latent MoE: the router and the routed experts read z = bf16(xn W_down^T).
+  const uint16_t* xe = xn;
+  if (lat) {
+    prof.begin(8);
+    const int r = dense_gemm(xn, c.D, h->map_pd, LW, h->bn_pd, zb, 1);
+    if (r != MOE_OK) return r;
+    prof.end(8);
+    xe = zb;
+  }
+
   // 1. router logits on the tensor cores
   if (c.router != MOE_ROUTER_HASH) {
     GemmArgs g;
     std::memset(&g, 0, sizeof(g));
-    if (!make_map(&g.mapA[0], xn, c.D, T, kBM)) return MOE_ECUDA;
-    if (!make_map(&g.mapA64[0], xn, c.D, T, kBM / 2)) return MOE_ECUDA;
-    if (!make_map(&g.mapA16[0], xn, c.D, T, 16)) return MOE_ECUDA;
+    if (!make_map(&g.mapA[0], xe, LW, T, kBM)) return MOE_ECUDA;
+    if (!make_map(&g.mapA64[0], xe, LW, T, kBM / 2)) return MOE_ECUDA;
+    if (!make_map(&g.mapA16[0], xe, LW, T, 16)) return MOE_ECUDA;
     g.mapB[0] = h->map_router;
     g.T = T;
     g.n_kind[0] = h->E_pad;
-    g.k_kind[0] = c.D;
+    g.k_kind[0] = LW;
     g.BN = h->E_pad;
     g.router_tiles = (T + kBM - 1) / kBM;
     g.out[0] = logits;
@@ -258,7 +306,8 @@ int forward_impl(moe_handle* h, int T, const uint16_t* x, const uint16_t* residu
   da.offsets = offsets; da.user_counts = out_counts; da.tiles_gu = tiles_gu; da.tiles_dn = tiles_dn;
   da.gu_ntiles_routed = c.I / h->bn_gu;
   da.gu_ntiles_shared = h->S > 0 ? c.I_shared / h->bn_gu : 0;
-  da.dn_ntiles = c.D / h->bn_dn;
+  da.dn_ntiles = LW / h->bn_dn;
+  da.dn_ntiles_shared = c.D / h->bn_dn;
   da.dest_row = dest; da.src_token = src;
   da.tile_m = kPairTileM;
   prof.begin(3);
@@ -267,23 +316,23 @@ int forward_impl(moe_handle* h, int T, const uint16_t* x, const uint16_t* residu
 
   // 4. grouped A rows of the routed experts
   prof.begin(4);
-  MOE_TRY(launch_gather_rows(xn, src, TK, c.D, xp, s));
+  MOE_TRY(launch_gather_rows(xe, src, TK, LW, xp, s));
   prof.end(4);
 
   // 5. gate/up + SwiGLU(+clamp): routed groups read xp, shared groups read xn
   {
     GemmArgs g;
     std::memset(&g, 0, sizeof(g));
-    if (!make_map(&g.mapA[0], xp, c.D, TK, kBM)) return MOE_ECUDA;
-    if (!make_map(&g.mapA64[0], xp, c.D, TK, kBM / 2)) return MOE_ECUDA;
-    if (!make_map(&g.mapA16[0], xp, c.D, TK, 16)) return MOE_ECUDA;
+    if (!make_map(&g.mapA[0], xp, LW, TK, kBM)) return MOE_ECUDA;
+    if (!make_map(&g.mapA64[0], xp, LW, TK, kBM / 2)) return MOE_ECUDA;
+    if (!make_map(&g.mapA16[0], xp, LW, TK, 16)) return MOE_ECUDA;
     if (h->S > 0 && !make_map(&g.mapA[1], xn, c.D, T, kBM)) return MOE_ECUDA;
     if (h->S > 0 && !make_map(&g.mapA64[1], xn, c.D, T, kBM / 2)) return MOE_ECUDA;
     if (h->S > 0 && !make_map(&g.mapA16[1], xn, c.D, T, 16)) return MOE_ECUDA;
     g.mapB[0] = h->map_wg; g.mapB[1] = h->map_wu; g.mapB[2] = h->map_wsg; g.mapB[3] = h->map_wsu;
     g.offsets = offsets; g.tile_start = tiles_gu; g.G = h->G; g.E = c.E; g.T = T;
     g.n_kind[0] = c.I; g.n_kind[1] = c.I_shared;
-    g.k_kind[0] = c.D; g.k_kind[1] = c.D;
+    g.k_kind[0] = LW; g.k_kind[1] = c.D;
     g.BN = h->bn_gu;
     g.swap_ok = h->bn_gu == 128;
     g.shared_a_stride = 0;
@@ -315,27 +364,43 @@ int forward_impl(moe_handle* h, int T, const uint16_t* x, const uint16_t* residu
       return MOE_ECUDA;
     g.mapB[0] = h->map_wd; g.mapB[2] = h->map_wsd;
     g.offsets = offsets; g.tile_start = tiles_dn; g.G = h->G; g.E = c.E; g.T = T;
-    g.n_kind[0] = c.D; g.n_kind[1] = c.D;
+    g.n_kind[0] = LW; g.n_kind[1] = c.D;
     g.k_kind[0] = c.I; g.k_kind[1] = c.I_shared;
     g.BN = h->bn_dn;
     g.swap_ok = h->bn_dn == 256;
     g.shared_a_stride = T;
-    g.out[0] = y; g.ld_out[0] = c.D;
+    g.out[0] = y; g.ld_out[0] = LW;
     g.out[1] = ys; g.ld_out[1] = c.D;
     g.shared_out_stride = T;
     g.dest_row = dest;
     g.err = err; g.timeout_ns = h->timeout_ns;
-    const int bound = expert_tile_bound(h, T, da.dn_ntiles, da.dn_ntiles);
+    const int bound = expert_tile_bound(h, T, da.dn_ntiles, da.dn_ntiles_shared);
     prof.begin(6);
     MOE_TRY(launch_grouped_gemm(kDown, g, pair_grid(h, bound), s));
     prof.end(6);
   }
 
   // 7. fixed-order combine + residual + RMSNorm
-  prof.begin(7);
-  MOE_TRY(launch_combine_norm(y, tw, ys, c.k, h->S, residual, h->w.g_out, out_norm, out_residual, T,
-                              c.D, c.eps, s));
-  prof.end(7);
+  if (lat) {
+    // Latent MoE: a = bf16(sum_j w_j y_j) in slot order, then y = a W_up^T, which
+    // the epilogue takes as a single slot of weight 1.
+    prof.begin(9);
+    MOE_TRY(launch_combine_latent(y, tw, c.k, LW, aggb, T, s));
+    prof.end(9);
+    prof.begin(10);
+    const int r = dense_gemm(aggb, LW, h->map_pu, c.D, h->bn_pu, ylat, 0);
+    if (r != MOE_OK) return r;
+    prof.end(10);
+    prof.begin(7);
+    MOE_TRY(launch_combine_norm(ylat, nullptr, ys, 1, h->S, residual, h->w.g_out, out_norm, out_residual,
+                                T, c.D, c.eps, s));
+    prof.end(7);
+  } else {
+    prof.begin(7);
+    MOE_TRY(launch_combine_norm(y, tw, ys, c.k, h->S, residual, h->w.g_out, out_norm, out_residual, T,
+                                c.D, c.eps, s));
+    prof.end(7);
+  }
   return MOE_OK;
 }
 
@@ -374,8 +439,13 @@ int moe_init(const moe_config* cfg, const moe_weights* w, moe_handle** out) {
   // One GEMM configuration per layer shape, never per T.  The expert GEMMs run
   // on CTA pairs: each CTA loads half of a gate/up tile (bn_gu / 2 gate rows and
   // bn_gu / 2 up rows) or half of a down tile (bn_dn / 2 rows).
+  h->L = cfg->latent > 0 ? cfg->latent : cfg->D;
   h->bn_gu = (cfg->I % 128 == 0 && h->cfg.I_shared % 128 == 0) ? 128 : 64;
-  h->bn_dn = (cfg->D % 256 == 0) ? 256 : (cfg->D % 128 == 0 ? 128 : 64);
+  // The down GEMM's routed groups have N = L, its shared groups N = D.
+  auto bn_for = [](int n) { return n % 256 == 0 ? 256 : (n % 128 == 0 ? 128 : 64); };
+  h->bn_dn = std::min(bn_for(cfg->D), bn_for(h->L));
+  h->bn_pd = bn_for(h->L);   // latent down-projection: N = latent
+  h->bn_pu = bn_for(cfg->D); // latent up-projection: N = D
   auto fail = [&](int code) { moe_destroy(h); return code; };
   if (cudaGetDevice(&h->device) != cudaSuccess) return fail(MOE_ECUDA);
   if (cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, h->device) != cudaSuccess)
@@ -385,19 +455,21 @@ int moe_init(const moe_config* cfg, const moe_weights* w, moe_handle** out) {
   if (h->max_pairs <= 0) h->max_pairs = h->num_sms / 2;
   const moe_config& c = h->cfg;
   if (c.router != MOE_ROUTER_HASH) {
-    const size_t row = static_cast<size_t>(c.D) * 2;
+    const size_t row = static_cast<size_t>(h->L) * 2;
     if (cudaMalloc(&h->w_router_pad, static_cast<size_t>(h->E_pad) * row) != cudaSuccess) return fail(MOE_ECUDA);
     if (cudaMemset(h->w_router_pad, 0, static_cast<size_t>(h->E_pad) * row) != cudaSuccess) return fail(MOE_ECUDA);
     if (cudaMemcpy(h->w_router_pad, w->w_router, static_cast<size_t>(c.E) * row, cudaMemcpyDeviceToDevice) != cudaSuccess)
       return fail(MOE_ECUDA);
   }
-  bool ok = make_map(&h->map_router, h->w_router_pad, c.D, h->w_router_pad ? h->E_pad : 0, h->E_pad) &&
-            make_map(&h->map_wg, w->w_gate, c.D, static_cast<uint64_t>(c.E) * c.I, h->bn_gu / 2) &&
-            make_map(&h->map_wu, w->w_up, c.D, static_cast<uint64_t>(c.E) * c.I, h->bn_gu / 2) &&
-            make_map(&h->map_wd, w->w_down, c.I, static_cast<uint64_t>(c.E) * c.D, h->bn_dn / 2) &&
+  bool ok = make_map(&h->map_router, h->w_router_pad, h->L, h->w_router_pad ? h->E_pad : 0, h->E_pad) &&
+            make_map(&h->map_wg, w->w_gate, h->L, static_cast<uint64_t>(c.E) * c.I, h->bn_gu / 2) &&
+            make_map(&h->map_wu, w->w_up, h->L, static_cast<uint64_t>(c.E) * c.I, h->bn_gu / 2) &&
+            make_map(&h->map_wd, w->w_down, c.I, static_cast<uint64_t>(c.E) * h->L, h->bn_dn / 2) &&
             make_map(&h->map_wsg, w->ws_gate, c.D, static_cast<uint64_t>(h->S) * c.I_shared, h->bn_gu / 2) &&
             make_map(&h->map_wsu, w->ws_up, c.D, static_cast<uint64_t>(h->S) * c.I_shared, h->bn_gu / 2) &&
-            make_map(&h->map_wsd, w->ws_down, c.I_shared, static_cast<uint64_t>(h->S) * c.D, h->bn_dn / 2);
+            make_map(&h->map_wsd, w->ws_down, c.I_shared, static_cast<uint64_t>(h->S) * c.D, h->bn_dn / 2) &&
+            make_map(&h->map_pd, c.latent > 0 ? w->w_proj_down : nullptr, c.D, c.latent, h->bn_pd / 2) &&
+            make_map(&h->map_pu, c.latent > 0 ? w->w_proj_up : nullptr, h->L, c.D, h->bn_pu / 2);
   if (!ok) return fail(MOE_ECUDA);
   *out = h;
   return MOE_OK;
@@ -544,6 +616,10 @@ int moe_workspace_views(const moe_handle* h, int T, void* workspace, moe_views* 
   out->h_shared = reinterpret_cast<const moe_bf16*>(ws + L.hs);
   out->y_slot = reinterpret_cast<const float*>(ws + L.y);
   out->y_shared = reinterpret_cast<const float*>(ws + L.ys);
+  const bool lat = h->cfg.latent > 0;
+  out->z = lat ? reinterpret_cast<const moe_bf16*>(ws + L.z) : nullptr;
+  out->agg = lat ? reinterpret_cast<const moe_bf16*>(ws + L.agg) : nullptr;
+  out->y_latent = lat ? reinterpret_cast<const float*>(ws + L.ylat) : nullptr;
   return MOE_OK;
 }
 
@@ -582,7 +658,8 @@ int moe_profile_read(moe_handle* h, float* ms, int* launches) {
 int moe_forward_launch_count(const moe_handle* h, int T) {
   if (!h || T < 0) return -1;
   if (T == 0) return 0;
-  return h->cfg.router == MOE_ROUTER_HASH ? MOE_NUM_STAGES - 1 : MOE_NUM_STAGES;  // no router GEMM
+  const int base = 8 + (h->cfg.latent > 0 ? 3 : 0);  // latent: two projections and the latent sum
+  return h->cfg.router == MOE_ROUTER_HASH ? base - 1 : base;  // hash routing: no router GEMM
 }
 
 int moe_selftest_wait_timeout(int limit_us, void* stream) {

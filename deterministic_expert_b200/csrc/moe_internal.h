@@ -69,7 +69,9 @@ struct GemmArgs {
   int swap_ok;            // expert GEMMs: a group's last partial tile may run operand-swapped
                           // (needs 128 weight rows per CTA: gate/up BN = 128, down BN = 256)
   int shared_a_stride;    // A rows between consecutive shared experts (0: all read row 0..T)
-  int router_tiles;       // tile count when tile_start is NULL
+  int router_tiles;       // tile count when tile_start is NULL (M-tiles x N-tiles)
+  int dense_kind;         // kind of the single group when tile_start is NULL
+  int out_bf16;           // down-mode output as bf16 instead of fp32 (latent projection)
   void* out[2];           // output base per kind
   int ld_out[2];          // output row pitch (elements) per kind
   int shared_out_stride;  // output rows between consecutive shared experts
@@ -91,10 +93,14 @@ cudaError_t launch_grouped_gemm(int mode, const GemmArgs& a, int grid, cudaStrea
 cudaError_t launch_rmsnorm_rows(const uint16_t* x, const uint16_t* g, uint16_t* y, int T, int D,
                                 float eps, int* err_to_clear, int32_t* zero, int zero_words,
                                 cudaStream_t s);
+// topk_w == NULL: every slot weighs 1.
 cudaError_t launch_combine_norm(const float* y_slot, const float* topk_w, const float* y_shared,
                                 int k, int S, const uint16_t* residual, const uint16_t* g,
                                 uint16_t* out_norm, uint16_t* out_residual, int T, int D,
                                 float eps, cudaStream_t s);
+// agg[t] = bf16(sum_j topk_w[t, j] * y_slot[t, j, :]) over L latent columns.
+cudaError_t launch_combine_latent(const float* y_slot, const float* topk_w, int k, int L, uint16_t* agg,
+                                  int T, cudaStream_t s);
 struct PartialPtrs {
   const uint16_t* p[8];
 };
@@ -138,7 +144,7 @@ struct DispatchArgs {
   int32_t* user_counts;   // [E] or NULL
   int32_t* tiles_gu;      // [E + S + 1]
   int32_t* tiles_dn;      // [E + S + 1]
-  int gu_ntiles_routed, gu_ntiles_shared, dn_ntiles;
+  int gu_ntiles_routed, gu_ntiles_shared, dn_ntiles, dn_ntiles_shared;
   int tile_m;             // rows per expert-GEMM tile (256: a CTA pair)
   int32_t* dest_row;      // [T * k]
   int32_t* src_token;     // [T * k]

@@ -154,7 +154,7 @@ __global__ void __launch_bounds__(kRowThreads) k_combine_norm(
   griddep_wait();
   griddep_launch();
   const size_t t = blockIdx.x;
-  if (threadIdx.x < k) w_s[threadIdx.x] = topk_w[t * k + threadIdx.x];
+  if (threadIdx.x < k) w_s[threadIdx.x] = topk_w != nullptr ? topk_w[t * k + threadIdx.x] : 1.0f;
   __syncthreads();
   const int nch = D / 4;
   float4 r[NC];
@@ -181,6 +181,37 @@ __global__ void __launch_bounds__(kRowThreads) k_combine_norm(
     }
   }
   norm_store(r, ss, red, g, out_norm + t * D, D, eps);
+}
+
+// Latent MoE: a[t] = bf16(sum_j w_j y[t, j]) over the routed experts' latent
+// outputs, in slot order, fp32, one cast (the linux.do post on MoE variants,
+// "潜在MoE": the experts' weighted sum before the up-projection).  Thread i owns
+// the 4-element chunks i, i + 256, ... of the latent row.
+template <int NC>
+__global__ void __launch_bounds__(kRowThreads) k_combine_latent(const float* __restrict__ y_slot,
+                                                                const float* __restrict__ topk_w, int k,
+                                                                int L, uint16_t* __restrict__ agg) {
+  __shared__ float w_s[16];
+  griddep_wait();
+  griddep_launch();
+  const size_t t = blockIdx.x;
+  if (threadIdx.x < k) w_s[threadIdx.x] = topk_w[t * k + threadIdx.x];
+  __syncthreads();
+  const int nch = L / 4;
+#pragma unroll
+  for (int i = 0; i < NC; ++i) {
+    const int c = threadIdx.x + i * kRowThreads;
+    if (c < nch) {
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int j = 0; j < k; ++j) {
+        const float4 y = *reinterpret_cast<const float4*>(y_slot + (t * k + j) * L + 4 * c);
+        const float w = w_s[j];
+        acc.x = fmaf(w, y.x, acc.x); acc.y = fmaf(w, y.y, acc.y);
+        acc.z = fmaf(w, y.z, acc.z); acc.w = fmaf(w, y.w, acc.w);
+      }
+      st_bf16x4(agg + t * L + 4 * c, acc.x, acc.y, acc.z, acc.w);
+    }
+  }
 }
 
 template <int NC>
@@ -335,6 +366,21 @@ cudaError_t launch_combine_norm(const float* y_slot, const float* topk_w, const 
     case 4: return go(k_combine_norm<4>);
     case 8: return go(k_combine_norm<8>);
     default: return go(k_combine_norm<16>);
+  }
+}
+
+cudaError_t launch_combine_latent(const float* y_slot, const float* topk_w, int k, int L, uint16_t* agg,
+                                  int T, cudaStream_t s) {
+  if (T <= 0) return cudaSuccess;
+  auto go = [&](auto kernel) {
+    return launch_k(kernel, dim3(T), dim3(kRowThreads), 0, s, false, y_slot, topk_w, k, L, agg);
+  };
+  switch (chunks_for(L)) {
+    case 1: return go(k_combine_latent<1>);
+    case 2: return go(k_combine_latent<2>);
+    case 4: return go(k_combine_latent<4>);
+    case 8: return go(k_combine_latent<8>);
+    default: return go(k_combine_latent<16>);
   }
 }
 

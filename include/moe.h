@@ -102,20 +102,29 @@ typedef struct moe_config {
   int activation;      /* moe_activation of routed and shared experts                  */
   float situ_beta_gate;/* SiTU-GLU gate cap (> 0, finite; read for MOE_ACT_SITU_GLU)    */
   float situ_beta_up;  /* SiTU-GLU up cap (> 0, finite)                                 */
+  int latent;          /* latent MoE width l (0 = none; else a multiple of 64, at most
+                          16384): the router and the routed experts work on
+                          z = bf16(xn W_proj_down^T) of width l, their weighted sum is
+                          cast to bf16 once and projected back by W_proj_up; shared
+                          experts stay at width D (linux.do post on MoE variants,
+                          "潜在MoE (Latent MoE)" and K3's Stable Latent MoE)          */
 } moe_config;
 
-typedef struct moe_weights {      /* device pointers, caller-owned                   */
-  const moe_bf16* w_router;       /* [E, D]      (unused for hash routing)            */
+typedef struct moe_weights {      /* device pointers, caller-owned; L = latent if
+                                     latent > 0, else D                               */
+  const moe_bf16* w_router;       /* [E, L]      (unused for hash routing)            */
   const float* router_bias;       /* [E] fp32 or NULL: logit bias (softmax) or
                                      selection bias (sigmoid)                         */
-  const moe_bf16* w_gate;         /* [E, I, D]                                        */
-  const moe_bf16* w_up;           /* [E, I, D]                                        */
-  const moe_bf16* w_down;         /* [E, D, I]                                        */
+  const moe_bf16* w_gate;         /* [E, I, L]                                        */
+  const moe_bf16* w_up;           /* [E, I, L]                                        */
+  const moe_bf16* w_down;         /* [E, L, I]                                        */
   const moe_bf16* ws_gate;        /* [S, I_shared, D]  (NULL when n_shared == 0)      */
   const moe_bf16* ws_up;          /* [S, I_shared, D]                                 */
   const moe_bf16* ws_down;        /* [S, D, I_shared]                                 */
   const moe_bf16* g_in;           /* [D] input RMSNorm gain                           */
   const moe_bf16* g_out;          /* [D] output RMSNorm gain                          */
+  const moe_bf16* w_proj_down;    /* [latent, D] latent down-projection (latent > 0)  */
+  const moe_bf16* w_proj_up;      /* [D, latent] latent up-projection (latent > 0)    */
 } moe_weights;
 
 typedef struct moe_handle moe_handle;
@@ -125,8 +134,9 @@ typedef struct moe_handle moe_handle;
  * 0 rmsnorm_in, 1 router_gemm (not launched for MOE_ROUTER_HASH), 2 router_topk
  * (scores, top-k, weights, per-128-token expert histogram), 3 dispatch (offsets
  * and stable scatter), 4 gather_rows, 5 gemm_gateup_swiglu, 6 gemm_down,
- * 7 combine_norm. */
-#define MOE_NUM_STAGES 8
+ * 7 combine_norm; with a latent width also 8 latent_down (launched before
+ * stage 1), 9 latent_combine and 10 latent_up (both before stage 7). */
+#define MOE_NUM_STAGES 11
 
 /* Validate `cfg`, keep the weight pointers and build the weight TMA
  * descriptors on the current CUDA device.  Allocates one small handle-owned
@@ -204,8 +214,11 @@ typedef struct moe_views {
   const int32_t* dest_row;     /* [T * k]         grouped row p -> t * k + slot      */
   const moe_bf16* h_routed;    /* [T * k, I]      grouped order                      */
   const moe_bf16* h_shared;    /* [S, T, I_shared]                                   */
-  const float* y_slot;         /* [T, k, D]       routed expert outputs, slot order  */
+  const float* y_slot;         /* [T, k, L]       routed expert outputs, slot order  */
   const float* y_shared;       /* [S, T, D]                                          */
+  const moe_bf16* z;           /* [T, latent]     latent input (NULL unless latent)  */
+  const moe_bf16* agg;         /* [T, latent]     bf16 routed sum (NULL unless latent)*/
+  const float* y_latent;       /* [T, D]          up-projected sum (NULL unless latent)*/
 } moe_views;
 
 int moe_workspace_views(const moe_handle* h, int T, void* workspace, moe_views* out);

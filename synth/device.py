@@ -30,6 +30,18 @@ def device_bf16(cfg, name, T=None, device="cuda", stream=None):
     return t
 
 
+def layer_config(cfg, T_max=None):
+    """The library's LayerConfig for a workload (every field of the layer)."""
+    import deterministic_expert_b200 as moe
+    return moe.LayerConfig(D=cfg.D, E=cfg.E, k=cfg.k, I=cfg.I, n_shared=cfg.n_shared,
+                           I_shared=cfg.I_shared, T_max=T_max or cfg.T, router=cfg.router,
+                           renormalize=cfg.renormalize, routed_scale=cfg.routed_scale,
+                           gate_clamp_max=cfg.gate_clamp_max, up_clamp=cfg.up_clamp, eps=cfg.eps,
+                           hash_mult=cfg.hash_mult, activation=cfg.activation,
+                           situ_beta_gate=cfg.situ_beta_gate, situ_beta_up=cfg.situ_beta_up,
+                           latent=cfg.latent)
+
+
 def device_weights(cfg, device="cuda", stream=None) -> dict:
     """moe_weights field name -> device tensor."""
     import torch
@@ -37,6 +49,9 @@ def device_weights(cfg, device="cuda", stream=None) -> dict:
          for n in ("w_router", "w_gate", "w_up", "w_down", "g_in", "g_out")}
     if cfg.n_shared:
         for n in ("ws_gate", "ws_up", "ws_down"):
+            w[n] = device_bf16(cfg, n, device=device, stream=stream)
+    if cfg.latent:
+        for n in ("w_proj_down", "w_proj_up"):
             w[n] = device_bf16(cfg, n, device=device, stream=stream)
     if cfg.bias == "normal":
         b = torch.empty(cfg.E, dtype=torch.float32, device=device)
@@ -82,7 +97,10 @@ class HostWeights:
     def __init__(self, cfg, cache_experts: int = 512):
         self.cfg = cfg
         E, D, I = cfg.E, cfg.D, cfg.I
-        self.w_router = f64(W.host_bf16(cfg, "w_router")).reshape(E, D) if cfg.router != W.ROUTER_HASH else None
+        L = cfg.latent or D
+        self.w_router = f64(W.host_bf16(cfg, "w_router")).reshape(E, L) if cfg.router != W.ROUTER_HASH else None
+        self.w_proj_down = f64(W.host_bf16(cfg, "w_proj_down")).reshape(cfg.latent, D) if cfg.latent else None
+        self.w_proj_up = f64(W.host_bf16(cfg, "w_proj_up")).reshape(D, cfg.latent) if cfg.latent else None
         b = W.host_router_bias(cfg)
         self.router_bias = None if b is None else b.astype(np.float64)
         self.g_in = f64(W.host_bf16(cfg, "g_in"))
@@ -100,8 +118,9 @@ class HostWeights:
             c = self.cfg
             if len(self._cache) >= self._cap:
                 self._cache.pop(next(iter(self._cache)))
-            self._cache[key] = (self._slice("w_gate", e, c.I, c.D), self._slice("w_up", e, c.I, c.D),
-                                self._slice("w_down", e, c.D, c.I))
+            L = c.latent or c.D
+            self._cache[key] = (self._slice("w_gate", e, c.I, L), self._slice("w_up", e, c.I, L),
+                                self._slice("w_down", e, L, c.I))
         return self._cache[key]
 
     def shared(self, s):

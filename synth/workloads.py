@@ -27,7 +27,7 @@ STREAM = {
     "w_gate": 5, "w_up": 6, "w_down": 7,
     "ws_gate": 8, "ws_up": 9, "ws_down": 10,
     "g_in": 11, "g_out": 12, "token_ids": 13, "zipf_rank": 14,
-    "decode_subset": 15, "perm": 16, "PARTIAL0": 32,
+    "decode_subset": 15, "perm": 16, "w_proj_down": 17, "w_proj_up": 18, "PARTIAL0": 32,
 }
 
 ROUTER_SOFTMAX, ROUTER_SIGMOID_BIAS, ROUTER_HASH = 0, 1, 2
@@ -60,6 +60,7 @@ class MoEConfig:
     activation: int = 0             # 0 SwiGLU (+ clamp), 1 SiTU-GLU
     situ_beta_gate: float = 4.0
     situ_beta_up: float = 25.0
+    latent: int = 0                 # latent MoE width (0: none)
 
     def with_T(self, T: int) -> "MoEConfig":
         return dataclasses.replace(self, T=T)
@@ -86,13 +87,19 @@ C5H = dataclasses.replace(C5, name="skew_hash", router=ROUTER_HASH, bias="none")
 # SiTU-GLU experts (the linux.do post on MoE variants, "SiTU-GLU": caps 4 and
 # 25) on the fine-grained shapes.
 C2S = dataclasses.replace(C2, name="fine_grained_situ", activation=1)
+# Latent MoE in the K3 manner (the linux.do post on MoE variants, "潜在MoE" and
+# "K3 的 Stable Latent MoE": many small routed experts with 16 active, working
+# at a latent width, SiTU-GLU inside the experts, a full-width shared expert).
+# The post gives no sizes; these are the fine-grained shapes with l = D / 4.
+C6 = MoEConfig("latent_situ", T=4096, D=2048, E=256, k=16, I=512, n_shared=1, I_shared=2048,
+               renormalize=1, activation=1, latent=512)
 # The 8-partial fixed-order reduce + residual + RMSNorm epilogue of that workload.
 EPILOGUE_P = 8
 EPILOGUE_T = 16384
 EPILOGUE_D = 4096
 EPILOGUE_SIGMA = 1.0 / 8.0
 
-CONFIGS = {c.name: c for c in (C1, C2, C3, C5, C5H, C2S)}
+CONFIGS = {c.name: c for c in (C1, C2, C3, C5, C5H, C2S, C6)}
 
 _ZIPF_FILE = os.path.join(os.path.dirname(os.path.abspath(__file__)), "zipf_beta.json")
 ZIPF_S = 1.2
@@ -112,9 +119,11 @@ def k_(name: str, index: int = 0) -> int:
 def tensor_shape(cfg: MoEConfig, name: str, T: int | None = None):
     T = cfg.T if T is None else T
     D, E, I, S, Is = cfg.D, cfg.E, cfg.I, cfg.n_shared, cfg.I_shared
+    L = cfg.latent or D   # width the router and routed experts read
     return {
-        "x": (T, D), "residual": (T, D), "w_router": (E, D), "router_bias": (E,),
-        "w_gate": (E, I, D), "w_up": (E, I, D), "w_down": (E, D, I),
+        "x": (T, D), "residual": (T, D), "w_router": (E, L), "router_bias": (E,),
+        "w_gate": (E, I, L), "w_up": (E, I, L), "w_down": (E, L, I),
+        "w_proj_down": (cfg.latent, D), "w_proj_up": (D, cfg.latent),
         "ws_gate": (S, Is, D), "ws_up": (S, Is, D), "ws_down": (S, D, Is),
         "g_in": (D,), "g_out": (D,), "token_ids": (T,),
     }[name]
@@ -191,20 +200,23 @@ def host_partial(p: int, T: int = EPILOGUE_T, D: int = EPILOGUE_D, start: int = 
 def moe_flops(cfg: MoEConfig, T: int | None = None) -> dict:
     """Algorithmic FLOPs of one layer call: 2 per multiply-add.
 
-    routed = 2*T*k*3*D*I, shared = 2*T*S*3*D*I_s, router = 2*T*E*D (none for
-    hash routing).  Gate/up is two thirds of each expert's work.
+    routed = 2*T*k*3*L*I, shared = 2*T*S*3*D*I_s, router = 2*T*E*L (none for
+    hash routing), with L the latent width (D without one); a latent layer adds
+    its two projections, 2*2*T*D*L.  Gate/up is two thirds of each expert's work.
     """
     T = cfg.T if T is None else T
-    routed = 2 * T * cfg.k * 3 * cfg.D * cfg.I
+    L = cfg.latent or cfg.D
+    routed = 2 * T * cfg.k * 3 * L * cfg.I
     shared = 2 * T * cfg.n_shared * 3 * cfg.D * cfg.I_shared
-    router = 0 if cfg.router == ROUTER_HASH else 2 * T * cfg.E * cfg.D
-    gateup = 2 * T * (cfg.k * 2 * cfg.D * cfg.I + cfg.n_shared * 2 * cfg.D * cfg.I_shared)
-    return {"routed": routed, "shared": shared, "router": router, "total": routed + shared + router,
-            "gateup": gateup, "down": routed + shared - gateup}
+    router = 0 if cfg.router == ROUTER_HASH else 2 * T * cfg.E * L
+    proj = 2 * 2 * T * cfg.D * cfg.latent
+    gateup = 2 * T * (cfg.k * 2 * L * cfg.I + cfg.n_shared * 2 * cfg.D * cfg.I_shared)
+    return {"routed": routed, "shared": shared, "router": router, "proj": proj,
+            "total": routed + shared + router + proj, "gateup": gateup, "down": routed + shared - gateup}
 
 
 def expert_bytes(cfg: MoEConfig) -> int:
-    return 3 * cfg.D * cfg.I * 2
+    return 3 * (cfg.latent or cfg.D) * cfg.I * 2
 
 
 def layer_bytes(cfg: MoEConfig, T: int, distinct_experts: int) -> int:
@@ -212,7 +224,8 @@ def layer_bytes(cfg: MoEConfig, T: int, distinct_experts: int) -> int:
     weights, x and residual in, two bf16 outputs."""
     w = distinct_experts * expert_bytes(cfg) + cfg.n_shared * 3 * cfg.D * cfg.I_shared * 2
     if cfg.router != ROUTER_HASH:
-        w += cfg.E * cfg.D * 2
+        w += cfg.E * (cfg.latent or cfg.D) * 2
+    w += 2 * cfg.D * cfg.latent * 2   # latent projections
     act = 4 * T * cfg.D * 2
     return w + act
 
@@ -220,9 +233,10 @@ def layer_bytes(cfg: MoEConfig, T: int, distinct_experts: int) -> int:
 def pretty(cfg: MoEConfig) -> str:
     r = {0: "softmax", 1: "sigmoid+bias", 2: "hash"}[cfg.router]
     act = "" if cfg.activation == 0 else f" SiTU-GLU({cfg.situ_beta_gate:g},{cfg.situ_beta_up:g})"
-    return (f"{cfg.name}: T={cfg.T} D={cfg.D} E={cfg.E} top-{cfg.k} {r} I={cfg.I} "
+    lat = f" latent={cfg.latent}" if cfg.latent else ""
+    return (f"{cfg.name}: T={cfg.T} D={cfg.D}{lat} E={cfg.E} top-{cfg.k} {r} I={cfg.I} "
             f"shared={cfg.n_shared}x{cfg.I_shared}{act}")
 
 
-__all__ = ["MoEConfig", "C1", "C2", "C2S", "C3", "C4_T", "C5", "C5H", "CONFIGS", "STREAM", "SEED",
+__all__ = ["MoEConfig", "C1", "C2", "C2S", "C3", "C4_T", "C5", "C5H", "C6", "CONFIGS", "STREAM", "SEED",
            "host_bf16", "host_router_bias", "host_token_ids", "moe_flops", "math"]

@@ -15,13 +15,7 @@ NEAR_TIE = 1e-5    # routing margin below which a token may route differently
 
 
 def layer_config(cfg, T_max):
-    import deterministic_expert_b200 as moe
-    return moe.LayerConfig(D=cfg.D, E=cfg.E, k=cfg.k, I=cfg.I, n_shared=cfg.n_shared,
-                           I_shared=cfg.I_shared, T_max=T_max, router=cfg.router,
-                           renormalize=cfg.renormalize, routed_scale=cfg.routed_scale,
-                           gate_clamp_max=cfg.gate_clamp_max, up_clamp=cfg.up_clamp, eps=cfg.eps,
-                           hash_mult=cfg.hash_mult, activation=cfg.activation,
-                           situ_beta_gate=cfg.situ_beta_gate, situ_beta_up=cfg.situ_beta_up)
+    return SD.layer_config(cfg, T_max)
 
 
 class Run:

@@ -69,3 +69,17 @@ def test_calls_reject_null_handles():
     assert L.moe_reduce_partials(1, arr, 1 << 20, 1 << 20, 1 << 20, 1 << 20, 4, 100, 1e-6, None) \
         == moe.MOE_EUNSUPPORTED
     assert L.moe_selftest_wait_timeout(0, None) == moe.MOE_EINVAL
+
+
+def test_weight_size_mismatch_is_refused():
+    """A weight tensor sized for another configuration (e.g. full-width experts
+    under a latent configuration) is refused before the library sees it."""
+    import torch
+    import deterministic_expert_b200 as moe
+    cfg = moe.LayerConfig(D=256, E=8, k=2, I=128, latent=64)
+    w = {"w_gate": torch.empty(8 * 128 * 256, dtype=torch.bfloat16)}
+    with pytest.raises(ValueError):
+        moe.MoELayer(cfg, w)
+    w = {"router_bias": torch.empty(8, dtype=torch.bfloat16)}
+    with pytest.raises(ValueError):
+        moe.MoELayer(cfg, w)

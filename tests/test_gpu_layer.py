@@ -171,6 +171,51 @@ def test_fine_grained_situ_parity(torch_cuda):
     check_outputs(out, ref, same_rows=same)
 
 
+def _latent_parity(run, cfg, torch):
+    """Latent layers: z = bf16(xn W_down^T) is rounded from fp32 on the GPU and
+    from fp64 in the oracle, so an element may land one bf16 step apart; the
+    routing is therefore checked against the oracle's router run on the GPU's
+    own z (the step's input), and the rest of the layer against the oracle."""
+    out = run.forward(*run.inputs())
+    ref, hw = oracle_full(cfg)
+    T, c = cfg.T, cfg
+    v = run.layer.views(T, out["ws"])
+    ws = out["ws"]
+    off = v.z - ws.data_ptr()
+    z = ws[off:off + T * c.latent * 2].view(torch.bfloat16).reshape(T, c.latent)
+    zg = np64(z)
+    # Differences are single bf16 steps of the larger of the two values, or,
+    # where the dot product cancels to a tiny z, within the fp32 accumulation
+    # error of its terms (|x| ~ 1, |w| ~ 0.02, K = D).
+    dz = np.abs(zg - ref["z"])
+    big = np.maximum(np.abs(zg), np.abs(ref["z"]))
+    ulp = 2.0 ** (np.floor(np.log2(np.maximum(big, 1e-30))) - 7)
+    assert np.all(dz <= np.maximum(ulp * 1.0000001, 2.0 ** -16)), float(dz.max())
+    # The tensor cores' fp32 accumulation of the K = D products rounds about
+    # 0.1 % of z to the neighbouring bf16 value of the fp64 result.
+    print(f"z elements one bf16 step from the oracle's: {(dz > 0).mean():.2e}")
+    assert (dz > 0).mean() < 1e-2, (dz > 0).mean()
+    logits = O.router_logits(zg, hw.w_router)
+    _, _, keys = O.route(c, logits, hw.router_bias, W.host_token_ids(c, T))
+    same = check_routing(out, dict(ref, keys=keys))
+    check_outputs(out, ref, same_rows=same)
+    return out, ref
+
+
+def test_latent_tiny_parity(torch_cuda):
+    cfg = dataclasses.replace(W.C1, T=300, latent=64, name="tiny_latent")
+    run = Run(cfg)
+    _latent_parity(run, cfg, torch_cuda)
+
+
+def test_latent_situ_parity(torch_cuda):
+    """The K3-style latent workload (l = 512, 256 experts top-16, SiTU-GLU, a
+    full-width shared expert) at T=512."""
+    cfg = dataclasses.replace(W.C6, T=512)
+    run = Run(cfg)
+    _latent_parity(run, cfg, torch_cuda)
+
+
 def test_empty_batch_launches_nothing(torch_cuda):
     import deterministic_expert_b200 as moe
     run = Run(W.C1)
