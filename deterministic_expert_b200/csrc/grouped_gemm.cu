@@ -46,7 +46,8 @@ namespace {
 
 constexpr uint32_t kTmemCols = 512;
 constexpr int kRingBytes = kStages * (kSmemA + kSmemBMax);  // shared memory of the stage ring
-constexpr int kRingMax = 8;                                 // most stages any variant uses
+constexpr int kRingMax = 12;                                // most stages any variant uses
+constexpr int kBarBytes = 512;                              // mbarrier region after the ring
 constexpr unsigned long long kDrainNs = 200ull * 1000 * 1000;  // 200 ms
 
 template <int CG>
@@ -144,13 +145,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
   // bytes; the router, whose B tile is only E_pad rows, packs as many stages of
   // kSmemA + E_pad * 128 bytes as fit (up to kRingMax), so one CTA walking the
   // whole K keeps more loads in flight.  The stage count never changes a result.
+  // Batches of at most 256 tokens make every expert tile a swapped tile whose
+  // token operand is at most a_stage_bytes / 128 rows per CTA: the A slot of a
+  // stage then shrinks to that and the ring holds more stages (more weight
+  // bytes in flight per SM).  No stage layout changes a result.
+  const int sa_bytes = (MODE != kRouter && a.a_stage_bytes > 0) ? a.a_stage_bytes : kSmemA;
   const int sb_bytes = MODE == kRouter ? a.BN * kBK * 2 : C::kSmemB;
-  const int S = MODE == kRouter ? min(kRingMax, kRingBytes / (kSmemA + sb_bytes)) : C::kStagesN;
+  const int S = MODE == kRouter ? min(8, kRingBytes / (kSmemA + sb_bytes))
+                                : min(kRingMax, kRingBytes / (sa_bytes + sb_bytes));
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint8_t* sA = smem;                              // S x kSmemA
-  uint8_t* sB = smem + S * kSmemA;                 // S x sb_bytes
+  uint8_t* sA = smem;                              // S x sa_bytes
+  uint8_t* sB = smem + S * sa_bytes;               // S x sb_bytes
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kRingBytes);
   uint64_t* full = bars;
   uint64_t* empty = bars + kRingMax;
@@ -159,7 +166,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
   uint64_t* tdone = tempty + 2;
   uint64_t* xfull = tdone + 1;   // [4] swapped gate/up tiles: up values staged for the gate warp
   uint64_t* xempty = xfull + 4;  // [4] ... and read back
-  uint8_t* epi = reinterpret_cast<uint8_t*>(bars) + 256;  // kEpiWarps x kEpiBytes
+  uint8_t* epi = reinterpret_cast<uint8_t*>(bars) + kBarBytes;  // kEpiWarps x kEpiBytes
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
 
@@ -235,14 +242,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
           uint8_t* b0 = sB + stage * sb_bytes;
           if (CG == 1) {
             mbar_arrive_expect_tx(&full[stage], tx);
-            tma_load_2d(sA + stage * kSmemA, amap, kb * kBK, a_y, &full[stage]);
+            tma_load_2d(sA + stage * sa_bytes, amap, kb * kBK, a_y, &full[stage]);
             tma_load_2d(b0, bmap, kb * kBK, b_y, &full[stage]);
             if (MODE == kGateUp)
               tma_load_2d(b0 + b_rows * kBK * 2, bmap + 1, kb * kBK, b_y, &full[stage]);
           } else {
             // The even CTA expects the bytes of both CTAs on its barrier.
             if (leader) mbar_arrive_expect_tx(&full[stage], 2 * tx);
-            tma_load_2d_pair(sA + stage * kSmemA, amap, kb * kBK, a_y, full0 + 8 * stage);
+            tma_load_2d_pair(sA + stage * sa_bytes, amap, kb * kBK, a_y, full0 + 8 * stage);
             tma_load_2d_pair(b0, bmap, kb * kBK, b_y, full0 + 8 * stage);
             if (MODE == kGateUp)
               tma_load_2d_pair(b0 + (BN / 2) * kBK * 2, bmap + 1, kb * kBK, b_y, full0 + 8 * stage);
@@ -286,7 +293,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
           tc_fence_after();
           // A swapped tile reads the weight rows as its A operand and the token
           // rows as its B operand (the same K order, so the same bits per element).
-          const uint32_t tok_addr = smem_u32(sA + stage * kSmemA);
+          const uint32_t tok_addr = smem_u32(sA + stage * sa_bytes);
           const uint32_t w_addr = smem_u32(sB + stage * sb_bytes);
           const uint32_t a_addr = ti.swap ? w_addr : tok_addr;
           const uint32_t b_addr = ti.swap ? tok_addr : w_addr;

@@ -154,6 +154,16 @@ int validate_config(const moe_config* c, const moe_weights* w) {
   return MOE_OK;
 }
 
+// With T < 256 no group reaches 256 rows, so every expert tile is a swapped
+// tile with at most ceil(T rounded up to 16 / 2) token rows per CTA; the GEMM
+// then sizes its stages' A slot to the TMA box that covers them (16, 64 or 128
+// rows).  0: the default 16 KB slot.
+int small_batch_a_bytes(int T) {
+  if (T >= 256) return 0;
+  const int rows = ((T + 15) / 16 * 16) / 2;
+  return (rows <= 16 ? 16 : (rows <= 64 ? 64 : 128)) * kBK * 2;
+}
+
 int gemm_grid(const moe_handle* h, int tiles_bound) {
   return std::max(1, std::min(h->num_sms, tiles_bound));
 }
@@ -335,6 +345,7 @@ int forward_impl(moe_handle* h, int T, const uint16_t* x, const uint16_t* residu
     g.k_kind[0] = LW; g.k_kind[1] = c.D;
     g.BN = h->bn_gu;
     g.swap_ok = h->bn_gu == 128;
+    g.a_stage_bytes = g.swap_ok ? small_batch_a_bytes(T) : 0;
     g.shared_a_stride = 0;
     g.out[0] = hb; g.ld_out[0] = c.I;
     g.out[1] = hsb; g.ld_out[1] = c.I_shared;
@@ -368,6 +379,7 @@ int forward_impl(moe_handle* h, int T, const uint16_t* x, const uint16_t* residu
     g.k_kind[0] = c.I; g.k_kind[1] = c.I_shared;
     g.BN = h->bn_dn;
     g.swap_ok = h->bn_dn == 256;
+    g.a_stage_bytes = g.swap_ok ? small_batch_a_bytes(T) : 0;
     g.shared_a_stride = T;
     g.out[0] = y; g.ld_out[0] = LW;
     g.out[1] = ys; g.ld_out[1] = c.D;

@@ -50,7 +50,7 @@ constexpr int kGemmThreads = 64 + 32 * kEpiWarps;  // warp 0: TMA, warp 1: MMA, 
 constexpr int kSmemA = kBM * kBK * 2;
 constexpr int kSmemBMax = 256 * kBK * 2;
 constexpr int kEpiBytes = 32 * 128;  // per epilogue warp: 32 rows x 128 B, XOR-swizzled
-constexpr int kGemmSmem = 1024 + kStages * (kSmemA + kSmemBMax) + 256 + kEpiWarps * kEpiBytes;
+constexpr int kGemmSmem = 1024 + kStages * (kSmemA + kSmemBMax) + 512 + kEpiWarps * kEpiBytes;
 
 enum GemmMode : int { kGateUp = 0, kDown = 1, kRouter = 2 };
 
@@ -66,6 +66,8 @@ struct GemmArgs {
   int n_kind[2];          // B rows per expert (N extent) per kind
   int k_kind[2];          // K extent per kind
   int BN;
+  int a_stage_bytes;      // expert GEMMs: A bytes per stage (0 = 16 KB); set when every tile is
+                          // swapped with at most a_stage_bytes / 128 token rows per CTA
   int swap_ok;            // expert GEMMs: a group's last partial tile may run operand-swapped
                           // (needs 128 weight rows per CTA: gate/up BN = 128, down BN = 256)
   int shared_a_stride;    // A rows between consecutive shared experts (0: all read row 0..T)
