@@ -6,14 +6,18 @@
 //            (or the SiTU-GLU unit [b_g tanh(g/b_g) sigmoid(g)] * [b_u tanh(u/b_u)])
 //            per routed expert (A = its grouped rows of xn) and per shared expert (A = xn)
 //   down   : y = h W_d^T in fp32, routed rows scattered to their (token, slot) row
+//   dense  : one group of T rows with N-tiles through the down path (the latent
+//            projections; bf16 or fp32 output)
 //
 // Batch invariance (the Meituan LongCat parity article, "为什么会不一致": keep
 // the whole K of a dot product in one accumulation instead of summing split
 // partial results).  Every output element is one TMEM accumulator that walks
 // all of K in 64-wide steps, 16 per MMA, in the same order for every tile;
-// the tile shape is fixed per layer shape and never chosen from T; rows of a
-// tile never mix (a row's result depends only on its own A row), so padding
-// rows and rows of a neighbouring group are computed and discarded.
+// rows of a tile never mix (a row's result depends only on its own A row), so
+// padding rows and rows of a neighbouring group are computed and discarded.
+// The MMA accumulates an element over K in the same order whatever the tile's
+// M, N or operand roles (checked bit for bit on B200), so the tile shapes
+// below, which do depend on a group's row count, never change a result.
 //
 // Two variants, persistent over a device-built tile list:
 //   CG = 1  one CTA per 128-row tile (the router GEMM).
@@ -23,9 +27,11 @@
 //           rows for those columns, down as those rows of W_d), so each SM's
 //           shared memory receives and feeds half the B bytes of a 1-CTA tile.
 //           The even CTA issues the MMAs; its commits reach both CTAs.  A
-//           group's last tile runs as a 128-row pair tile (M = 128, 64 rows per
-//           CTA) when no more than 128 rows remain, so the padding of a group is
-//           under 128 rows, not 256.
+//           group's last r < 256 rows run operand-swapped: the CTA's 128 weight
+//           rows are the M = 256 MMA's A operand and its r/2 token rows the B
+//           operand (N = r rounded up to 16), so a group's padding is under 16
+//           rows.  (Shapes whose tiles are not 128 gate/up or 256 down columns
+//           use a 128-row pair tile, M = 128, for the last <= 128 rows.)
 // Roles in each CTA:
 //   warp 0    one thread issues the TMA loads of its CTA into a stage ring
 //   warp 1    allocates 512 TMEM columns; in the (even) issuing CTA one thread
@@ -141,10 +147,10 @@ __device__ __forceinline__ float glu_unit(float g, float u, const GemmArgs& a) {
 template <int MODE, int CG, int ACT>
 __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_constant__ GemmArgs a) {
   using C = Cfg<CG>;
-  // Stage ring.  The expert GEMMs use C::kStagesN stages of kSmemA + C::kSmemB
-  // bytes; the router, whose B tile is only E_pad rows, packs as many stages of
-  // kSmemA + E_pad * 128 bytes as fit (up to kRingMax), so one CTA walking the
-  // whole K keeps more loads in flight.  The stage count never changes a result.
+  // Stage ring.  The expert GEMMs use as many stages of kSmemA + C::kSmemB bytes
+  // as fit (6); the router, whose B tile is only E_pad rows, packs as many
+  // stages of kSmemA + E_pad * 128 bytes as fit (up to 8), so one CTA walking
+  // the whole K keeps more loads in flight.
   // Batches of at most 256 tokens make every expert tile a swapped tile whose
   // token operand is at most a_stage_bytes / 128 rows per CTA: the A slot of a
   // stage then shrinks to that and the ring holds more stages (more weight
