@@ -2,6 +2,12 @@
 """Throughput of the batch-invariant MoE layer forward on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl b200|reference]
+                    [--workload NAME] [--T TOKENS] [--no-cpu-baseline]
+
+--workload picks another workload (v3_shaped, skew_zipf, skew_hash,
+fine_grained_situ, latent_situ, tiny, or skew_epilogue for the 8-partial
+reduce + residual + RMSNorm); --T overrides the batch size (the decode sweep
+is --T 1, 8, 64, 128, 512 on the fine-grained weights).
 
 One step is one full layer forward (all eight kernels: RMSNorm, router GEMM,
 top-k with the expert histogram, offsets + stable scatter, row gather,
