@@ -281,7 +281,10 @@ def run_epilogue(a):
     """--workload skew_epilogue: the 8-partial fixed-order reduce + residual +
     RMSNorm of the skewed workload (8 bf16 buffers of [16384, 4096] N(0,1)/8),
     HBM-bound; reported as tokens/s with its share of the measured HBM copy
-    bandwidth (algorithmic bytes (P + 3) * T * D * 2 per launch)."""
+    bandwidth (algorithmic bytes (P + 3) * T * D * 2 per launch).  With N > 1
+    ranks (N dividing 8) the same job runs tensor parallel: the partials are
+    spread over the ranks and every rank reduces T / N rows over NVLink
+    (strong scaling, share of the measured peer-copy bandwidth)."""
     import torch
     import torch.distributed as dist
 
@@ -297,16 +300,29 @@ def run_epilogue(a):
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     P, T, D = W.EPILOGUE_P, W.EPILOGUE_T, W.EPILOGUE_D
-    parts = SD.device_partials(P, T, D, device=dev)
     res = SD.device_bf16(W.C5, "residual", T=T, device=dev)
     g = SD.device_bf16(W.C5, "g_out", device=dev)
-    on = torch.empty((T, D), dtype=torch.bfloat16, device=dev)
-    orr = torch.empty_like(on)
-    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
+    # N > 1 (N dividing 8): tensor parallel, as in the Fireworks parity post
+    # (Trap 1, one reduction order on every rank).  Rank r holds
+    # partials r*8/N .. (r+1)*8/N - 1 in symmetric memory; each step is one
+    # TPAllReduceNorm call (device barrier, one kernel reducing this rank's rows
+    # over every rank's partials and storing them to every rank, barrier).
+    tp = None
+    if world > 1 and P % world == 0:
+        tp = moe.TPAllReduceNorm(T, D, per_rank=P // world, device=dev)
+        for j in range(P // world):
+            SD.fill_partial(tp.partial[j], rank * (P // world) + j)
+        step = lambda: tp(res, g, stream=stream)  # noqa: E731
+    else:
+        parts = SD.device_partials(P, T, D, device=dev)
+        on = torch.empty((T, D), dtype=torch.bfloat16, device=dev)
+        orr = torch.empty_like(on)
+        step = lambda: moe.reduce_partials(parts, res, g, on, orr, stream=stream)  # noqa: E731
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
     for _ in range(a.warmup):
         flush.fill_(1)
-        moe.reduce_partials(parts, res, g, on, orr, stream=stream)
+        step()
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(a.steps)]
     clocks = ClockSampler(local) if rank == 0 else None
     if world > 1:
@@ -315,7 +331,7 @@ def run_epilogue(a):
     for e0, e1 in evs:
         flush.fill_(1)
         e0.record(stream)
-        moe.reduce_partials(parts, res, g, on, orr, stream=stream)
+        step()
         e1.record(stream)
     torch.cuda.synchronize()
     if world > 1:
@@ -326,7 +342,7 @@ def run_epilogue(a):
         dist.all_reduce(ms, op=dist.ReduceOp.MAX)
     ms_per_step = float(ms.item()) / a.steps
     e2e = None
-    if rank == 0:
+    if rank == 0 and tp is None:
         # End to end: partials and residual from pinned host memory, both outputs back.
         hp = [torch.empty((T, D), dtype=torch.bfloat16, pin_memory=True) for _ in range(P)]
         for h, d in zip(hp, parts):
@@ -353,22 +369,39 @@ def run_epilogue(a):
     cpu = None if (rank != 0 or a.no_cpu_baseline) else epilogue_oracle_sample(budget_s=12.0)
     if rank == 0:
         _, hbm_peak, peak_kind = peaks()
-        nbytes = (P + 3) * T * D * 2
-        gbs = nbytes / (ms_per_step / 1e3) / 1e9
+        wl = (f"skewed workload epilogue: {P} partial buffers [T={T}, D={D}] bf16 "
+              f"N(0,1)/8, fixed r0..r{P - 1} order + residual + RMSNorm")
+        if tp is None:
+            nbytes = (P + 3) * T * D * 2
+            gbs = nbytes / (ms_per_step / 1e3) / 1e9
+            value, scaling = world * T / (ms_per_step / 1e3), "weak"
+            roof = {"bound": "hbm", "kernel": "reduce_partials", "achieved": round(gbs, 1),
+                    "peak": hbm_peak, "unit": "GB/s", "frac": round(gbs / hbm_peak, 4), "traffic": None,
+                    "peak_source": f"{peak_kind} HBM copy", "bytes_per_launch": nbytes}
+        else:
+            # One T-row job split across the ranks.  Bytes that cross this
+            # rank's NVLink per step: the other ranks' partials for its rows
+            # in, its normalised rows for the other ranks out (both outputs).
+            rows = tp.rows
+            link = ((P - P // world) * rows * D * 2) + 2 * (world - 1) * rows * D * 2
+            gbs = link / (ms_per_step / 1e3) / 1e9
+            value, scaling = T / (ms_per_step / 1e3), "strong"
+            wl = f"tensor parallel over {world} ranks ({P // world} partials each, {rows} rows reduced per rank): " + wl
+            roof = {"bound": "nvlink", "kernel": "reduce_partials (row slice, peer loads and stores)",
+                    "achieved": round(gbs, 1), "peak": 770.0, "unit": "GB/s", "frac": round(gbs / 770.0, 4),
+                    "traffic": None, "peak_source": "measured peer copy per direction (profiling recipe)",
+                    "bytes_per_launch": link}
         print(json.dumps({
-            "metric": METRIC, "value": round(world * T / (ms_per_step / 1e3), 1), "unit": UNIT,
+            "metric": METRIC, "value": round(value, 1), "unit": UNIT,
             "n_gpus": world, "steps": a.steps, "warmup": a.warmup, "ms_per_step": round(ms_per_step, 4),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "higher_is_better": True, "scaling": scaling, "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded counter-based generator)",
-            "config": {"workload": f"skewed workload epilogue: {P} partial buffers [T={T}, D={D}] bf16 "
-                                   f"N(0,1)/8, fixed r0..r{P - 1} order + residual + RMSNorm",
-                       "l2": "flushed before every step (512 MiB write, untimed)"},
-            "roofline": {"bound": "hbm", "kernel": "reduce_partials", "achieved": round(gbs, 1),
-                         "peak": hbm_peak, "unit": "GB/s", "frac": round(gbs / hbm_peak, 4), "traffic": None,
-                         "peak_source": f"{peak_kind} HBM copy", "bytes_per_launch": nbytes},
+            "config": {"workload": wl, "l2": "flushed before every step (512 MiB write, untimed)"},
+            "roofline": roof,
             "gpu_launches": a.steps, "clocks": clk, "e2e": e2e, "cpu_baseline": cpu}), flush=True)
     if world > 1:
         dist.barrier()
+        del tp
         dist.destroy_process_group()
 
 

@@ -514,24 +514,42 @@ int moe_get_device_error(moe_handle* h, void* workspace, void* stream) {
   return e == kDevOk ? MOE_OK : MOE_ETIMEOUT;
 }
 
-int moe_reduce_partials(int P, const moe_bf16* const* partials, const moe_bf16* residual,
-                        const moe_bf16* g, moe_bf16* out_norm, moe_bf16* out_residual, int T, int D,
-                        float eps, void* stream) {
-  if (P < 1 || P > 8 || !partials || T < 0 || D <= 0 || !(eps >= 0.f)) return MOE_EINVAL;
+int moe_reduce_partials_rows(int P, const moe_bf16* const* partials, const moe_bf16* residual,
+                             const moe_bf16* g, int n_out, moe_bf16* const* out_norm,
+                             moe_bf16* const* out_residual, int row0, int rows, int D, float eps,
+                             void* stream) {
+  if (P < 1 || P > 8 || !partials || n_out < 1 || n_out > 8 || !out_norm || !out_residual || row0 < 0 ||
+      rows < 0 || D <= 0 || !(eps >= 0.f))
+    return MOE_EINVAL;
   if (D % 64 || D > 16384) return MOE_EUNSUPPORTED;
-  if (T == 0) return MOE_OK;
-  if (!residual || !g || !out_norm || !out_residual) return MOE_EINVAL;
+  if (rows == 0) return MOE_OK;
+  if (!residual || !g || !aligned16(residual)) return MOE_EINVAL;
   PartialPtrs pp;
   for (int p = 0; p < 8; ++p) pp.p[p] = nullptr;
   for (int p = 0; p < P; ++p) {
     if (!partials[p] || !aligned16(partials[p])) return MOE_EINVAL;
     pp.p[p] = partials[p];
   }
-  if (!aligned16(residual) || !aligned16(out_norm) || !aligned16(out_residual)) return MOE_EINVAL;
-  return launch_reduce_partials(pp, P, residual, g, out_norm, out_residual, T, D, eps,
+  OutPtrs op;
+  for (int d = 0; d < 8; ++d) op.norm[d] = op.res[d] = nullptr;
+  for (int d = 0; d < n_out; ++d) {
+    if (!out_norm[d] || !out_residual[d] || !aligned16(out_norm[d]) || !aligned16(out_residual[d]))
+      return MOE_EINVAL;
+    op.norm[d] = out_norm[d];
+    op.res[d] = out_residual[d];
+  }
+  return launch_reduce_partials(pp, P, residual, g, op, n_out, row0, rows, D, eps,
                                 static_cast<cudaStream_t>(stream)) == cudaSuccess
              ? MOE_OK
              : MOE_ECUDA;
+}
+
+int moe_reduce_partials(int P, const moe_bf16* const* partials, const moe_bf16* residual,
+                        const moe_bf16* g, moe_bf16* out_norm, moe_bf16* out_residual, int T, int D,
+                        float eps, void* stream) {
+  if (T < 0) return MOE_EINVAL;
+  return moe_reduce_partials_rows(P, partials, residual, g, 1, &out_norm, &out_residual, 0, T, D, eps,
+                                  stream);
 }
 
 size_t moe_invariance_workspace_size(const moe_handle* h, int T) {

@@ -106,9 +106,17 @@ cudaError_t launch_combine_latent(const float* y_slot, const float* topk_w, int 
 struct PartialPtrs {
   const uint16_t* p[8];
 };
+// Destinations of the reduced rows (n_out pairs; local or peer memory).
+struct OutPtrs {
+  uint16_t* norm[8];
+  uint16_t* res[8];
+};
+// Rows [row0, row0 + rows) of the P partial buffers (each [T, D], local or peer
+// memory) reduced in the fixed order p = 0 .. P-1, + residual, RMSNorm; written
+// to the same rows of every destination pair.
 cudaError_t launch_reduce_partials(const PartialPtrs& parts, int P, const uint16_t* residual,
-                                   const uint16_t* g, uint16_t* out_norm, uint16_t* out_residual,
-                                   int T, int D, float eps, cudaStream_t s);
+                                   const uint16_t* g, const OutPtrs& outs, int n_out, int row0, int rows,
+                                   int D, float eps, cudaStream_t s);
 cudaError_t launch_bitcompare(const uint16_t* a, const uint16_t* b, const int32_t* b_row_of_a,
                               int rows, int D, unsigned long long* count, cudaStream_t s);
 cudaError_t launch_permute_inputs(const uint16_t* x, const uint16_t* res, const int32_t* ids,

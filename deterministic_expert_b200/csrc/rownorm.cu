@@ -217,12 +217,11 @@ __global__ void __launch_bounds__(kRowThreads) k_combine_latent(const float* __r
 template <int NC>
 __global__ void __launch_bounds__(kRowThreads) k_reduce_partials(
     const PartialPtrs parts, int P, const uint16_t* __restrict__ residual,
-    const uint16_t* __restrict__ g, uint16_t* __restrict__ out_norm,
-    uint16_t* __restrict__ out_residual, int D, float eps) {
+    const uint16_t* __restrict__ g, const OutPtrs outs, int n_out, int row0, int D, float eps) {
   __shared__ float red[kRowThreads / 32 + 1];
   griddep_wait();
   griddep_launch();
-  const size_t t = blockIdx.x;
+  const size_t t = static_cast<size_t>(row0) + blockIdx.x;
   const int nch = D / 8;
   f8 r[NC];
   float ss = 0.f;
@@ -257,11 +256,12 @@ __global__ void __launch_bounds__(kRowThreads) k_reduce_partials(
         r[i].v[q] = __fadd_rn(acc[q], res.v[q]);
         ss = fmaf(r[i].v[q], r[i].v[q], ss);
       }
-      st_bf16x8(out_residual + off, r[i].v);
+#pragma unroll
+      for (int d = 0; d < 8; ++d)
+        if (d < n_out) st_bf16x8(outs.res[d] + off, r[i].v);
     }
   }
   const float inv = inv_rms(block_sum_fixed(ss, red), D, eps);
-  uint16_t* on = out_norm + t * D;
 #pragma unroll
   for (int i = 0; i < NC; ++i) {
     const int c = threadIdx.x + i * kRowThreads;
@@ -270,7 +270,9 @@ __global__ void __launch_bounds__(kRowThreads) k_reduce_partials(
       float o[8];
 #pragma unroll
       for (int q = 0; q < 8; ++q) o[q] = r[i].v[q] * inv * gg.v[q];
-      st_bf16x8(on + 8 * c, o);
+#pragma unroll
+      for (int d = 0; d < 8; ++d)
+        if (d < n_out) st_bf16x8(outs.norm[d] + t * D + 8 * c, o);
     }
   }
 }
@@ -385,12 +387,12 @@ cudaError_t launch_combine_latent(const float* y_slot, const float* topk_w, int 
 }
 
 cudaError_t launch_reduce_partials(const PartialPtrs& parts, int P, const uint16_t* residual,
-                                   const uint16_t* g, uint16_t* out_norm, uint16_t* out_residual,
-                                   int T, int D, float eps, cudaStream_t s) {
-  if (T <= 0) return cudaSuccess;
+                                   const uint16_t* g, const OutPtrs& outs, int n_out, int row0, int rows,
+                                   int D, float eps, cudaStream_t s) {
+  if (rows <= 0) return cudaSuccess;
   auto go = [&](auto kernel) {
-    return launch_k(kernel, dim3(T), dim3(kRowThreads), 0, s, false, parts, P, residual, g, out_norm,
-                    out_residual, D, eps);
+    return launch_k(kernel, dim3(rows), dim3(kRowThreads), 0, s, false, parts, P, residual, g, outs, n_out,
+                    row0, D, eps);
   };
   switch (chunks_for(D, 8)) {
     case 1: return go(k_reduce_partials<1>);

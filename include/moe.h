@@ -183,6 +183,22 @@ int moe_reduce_partials(int P, const moe_bf16* const* partials, const moe_bf16* 
                         const moe_bf16* g, moe_bf16* out_norm, moe_bf16* out_residual, int T,
                         int D, float eps, void* stream);
 
+/* The same reduction for rows [row0, row0 + rows) only, written to n_out
+ * destination pairs (1 <= n_out <= 8): the fused form of the tensor-parallel
+ * all-reduce + residual + RMSNorm over NVLink.  With P ranks, rank i passes the
+ * P ranks' partial buffers in rank order (its own and its peers', mapped into
+ * its address space, e.g. by symmetric memory), its row slice, and every rank's
+ * output buffers: each rank reads all partials of its rows with plain loads,
+ * reduces them in the fixed order p = 0 .. P-1, and stores the rows to every
+ * rank.  Every rank then holds the same bits as moe_reduce_partials over all T
+ * rows on one GPU.  The caller orders the ranks (a barrier after the partials
+ * are written, another before they are overwritten); the call itself does not
+ * synchronise.  Pointers: [T, D] buffers, 16-byte aligned.  Errors as above. */
+int moe_reduce_partials_rows(int P, const moe_bf16* const* partials, const moe_bf16* residual,
+                             const moe_bf16* g, int n_out, moe_bf16* const* out_norm,
+                             moe_bf16* const* out_residual, int row0, int rows, int D, float eps,
+                             void* stream);
+
 /* Bytes of device workspace moe_check_invariance needs for T rows. */
 size_t moe_invariance_workspace_size(const moe_handle* h, int T);
 

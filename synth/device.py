@@ -79,9 +79,14 @@ def device_partials(P=W.EPILOGUE_P, T=W.EPILOGUE_T, D=W.EPILOGUE_D, device="cuda
     out = []
     for p in range(P):
         t = torch.empty((T, D), dtype=torch.bfloat16, device=device)
-        dev_normal_bf16(W.k_("PARTIAL0", p), 0, T * D, W.EPILOGUE_SIGMA, t.data_ptr(), _stream_ptr(stream))
+        fill_partial(t, p, stream)
         out.append(t)
     return out
+
+
+def fill_partial(t, p, stream=None):
+    """Write partial buffer p of the epilogue workload into the [T, D] bf16 tensor t."""
+    dev_normal_bf16(W.k_("PARTIAL0", p), 0, t.numel(), W.EPILOGUE_SIGMA, t.data_ptr(), _stream_ptr(stream))
 
 
 # ------------------------------------------------------------------ host side

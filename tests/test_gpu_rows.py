@@ -95,3 +95,71 @@ def test_order_change_is_visible(torch_cuda):
     assert np.all(ring[:, :c] == 0) and np.all(ring[:, c:2 * c] == 2.0 ** -25) and np.all(ring[:, 2 * c:] == 0)
     assert not np.array_equal(O.round_bf16(ring.astype(np.float64)), got)
 
+
+
+def test_row_slices_to_several_destinations(torch_cuda):
+    """moe_reduce_partials_rows over three row slices, each written to two
+    destination pairs: both destinations must equal moe_reduce_partials over
+    all rows bit for bit (the form the tensor-parallel epilogue launches on
+    each rank)."""
+    import deterministic_expert_b200 as moe
+    torch = torch_cuda
+    P, T, D = 8, 301, 2048
+    gen = torch.Generator().manual_seed(77)
+    parts = [(torch.randn((T, D), generator=gen) / 8).to(torch.bfloat16).cuda() for _ in range(P)]
+    res = torch.randn((T, D), generator=gen).to(torch.bfloat16).cuda()
+    g = (1 + 0.1 * torch.randn(D, generator=gen)).to(torch.bfloat16).cuda()
+    on, orr = _run(torch, parts, res, g)
+    outs = [(torch.zeros_like(res), torch.zeros_like(res)) for _ in range(2)]
+    for row0, rows in moe.row_slices(T, 3):
+        moe.reduce_partials_rows(parts, res, g, [o[0] for o in outs], [o[1] for o in outs], row0, rows)
+    torch.cuda.synchronize()
+    for n_, r_ in outs:
+        assert torch.equal(n_.view(torch.int16), on.view(torch.int16))
+        assert torch.equal(r_.view(torch.int16), orr.view(torch.int16))
+
+
+def _tp_world1(q):
+    import os
+    import torch
+    import torch.distributed as dist
+    import deterministic_expert_b200 as moe
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(q.get()))
+    torch.cuda.set_device(0)
+    dist.init_process_group("nccl", rank=0, world_size=1, device_id=torch.device("cuda", 0))
+    try:
+        P, T, D = 8, 129, 1024
+        tp = moe.TPAllReduceNorm(T, D, per_rank=P, device="cuda")
+        gen = torch.Generator().manual_seed(5)
+        parts = [(torch.randn((T, D), generator=gen) / 8).to(torch.bfloat16).cuda() for _ in range(P)]
+        for j in range(P):
+            tp.partial[j].copy_(parts[j])
+        res = torch.randn((T, D), generator=gen).to(torch.bfloat16).cuda()
+        g = torch.ones(D, dtype=torch.bfloat16, device="cuda")
+        on, orr = tp(res, g)
+        ref_n, ref_r = torch.empty_like(res), torch.empty_like(res)
+        moe.reduce_partials(parts, res, g, ref_n, ref_r)
+        torch.cuda.synchronize()
+        q.put(bool(torch.equal(on.view(torch.int16), ref_n.view(torch.int16)) and
+                   torch.equal(orr.view(torch.int16), ref_r.view(torch.int16))))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_tp_epilogue_one_rank(torch_cuda):
+    """TPAllReduceNorm on one rank (symmetric-memory buffers, device-side
+    barriers, the row-slice kernel) equals moe_reduce_partials bit for bit."""
+    import socket
+    import torch.multiprocessing as mp
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    q.put(port)
+    p = ctx.Process(target=_tp_world1, args=(q,))
+    p.start()
+    p.join(timeout=300)
+    assert p.exitcode == 0
+    assert q.get(timeout=5) is True
