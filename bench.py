@@ -334,6 +334,8 @@ def run_epilogue(a):
         step()
         e1.record(stream)
     torch.cuda.synchronize()
+    if tp is not None:
+        tp.check()   # raises if a device barrier wait gave up
     if world > 1:
         dist.barrier()
     clk = clocks.stop() if clocks else None
@@ -398,10 +400,12 @@ def run_epilogue(a):
             "data": "synthetic (seeded counter-based generator)",
             "config": {"workload": wl, "l2": "flushed before every step (512 MiB write, untimed)"},
             "roofline": roof,
-            "gpu_launches": a.steps, "clocks": clk, "e2e": e2e, "cpu_baseline": cpu}), flush=True)
+            "gpu_launches": a.steps * (1 if tp is None else 3), "clocks": clk, "e2e": e2e,
+            "cpu_baseline": cpu}), flush=True)
     if world > 1:
         dist.barrier()
-        del tp
+        if tp is not None:
+            tp.close()
         dist.destroy_process_group()
 
 

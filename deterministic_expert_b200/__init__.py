@@ -313,56 +313,162 @@ def row_slices(T: int, world: int):
     return out
 
 
+PEER_HANDLE_BYTES = 64
+
+
+def peer_alloc(nbytes: int):
+    """moe_peer_alloc: (device address, IPC handle bytes) of a new zeroed,
+    exported allocation on the current device."""
+    L = lib()
+    ptr = ctypes.c_void_p()
+    h = (ctypes.c_ubyte * PEER_HANDLE_BYTES)()
+    L.moe_peer_alloc.argtypes = [ctypes.c_size_t, ctypes.POINTER(ctypes.c_void_p), ctypes.c_void_p]
+    _check(L.moe_peer_alloc(nbytes, ctypes.byref(ptr), h), "moe_peer_alloc")
+    return int(ptr.value), bytes(h)
+
+
+def peer_open(handle: bytes) -> int:
+    """moe_peer_open: map another process's exported allocation; its address."""
+    L = lib()
+    ptr = ctypes.c_void_p()
+    h = (ctypes.c_ubyte * PEER_HANDLE_BYTES).from_buffer_copy(handle)
+    L.moe_peer_open.argtypes = [ctypes.c_void_p, ctypes.POINTER(ctypes.c_void_p)]
+    _check(L.moe_peer_open(h, ctypes.byref(ptr)), "moe_peer_open")
+    return int(ptr.value)
+
+
+def peer_close(addr: int) -> None:
+    L = lib()
+    L.moe_peer_close.argtypes = [ctypes.c_void_p]
+    _check(L.moe_peer_close(addr), "moe_peer_close")
+
+
+def peer_free(addr: int) -> None:
+    L = lib()
+    L.moe_peer_free.argtypes = [ctypes.c_void_p]
+    _check(L.moe_peer_free(addr), "moe_peer_free")
+
+
+def peer_barrier(flags, rank: int, epoch: int, err, limit_us: int, stream=None) -> None:
+    """moe_peer_barrier over len(flags) ranks (flag-array device addresses in
+    rank order); a timed-out wait stores 1 to the device int32 tensor ``err``."""
+    L = lib()
+    arr = (ctypes.c_void_p * len(flags))(*flags)
+    L.moe_peer_barrier.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_uint32,
+                                   ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p]
+    _check(L.moe_peer_barrier(len(flags), rank, arr, epoch, _ptr(err), limit_us, _stream(stream)),
+           "moe_peer_barrier")
+
+
+class _DeviceArray:
+    """A device address exposed through __cuda_array_interface__ (int16 words),
+    so that torch can view memory this library allocated."""
+
+    def __init__(self, addr: int, n: int):
+        self.__cuda_array_interface__ = {"shape": (n,), "typestr": "<i2", "data": (addr, False),
+                                         "version": 3, "strides": None}
+
+
 class TPAllReduceNorm:
     """The tensor-parallel epilogue across GPUs (the Fireworks parity post,
     Trap 1 and Trap 2: every rank reduces r_0 + r_1 + ... in the same fixed
-    order, then residual + RMSNorm): each rank holds ``per_rank`` partial
-    buffers [T, D] in symmetric memory; a call reduces this rank's row slice by
-    reading every rank's partials over NVLink with plain loads and stores the
-    rows to every rank's outputs, in one kernel (moe_reduce_partials_rows),
-    between two device-side barriers.  Every rank ends with the bits the
-    single-GPU moe_reduce_partials gives over the same P partials.
+    order, then residual + RMSNorm).  Each rank exports one allocation
+    (moe_peer_alloc) holding its barrier flags, its ``per_rank`` partial
+    buffers [T, D] and its two outputs, and maps every other rank's
+    (moe_peer_open; handles travel over the process group).  A call is three
+    kernels on the caller's stream: a device barrier, moe_reduce_partials_rows
+    on this rank's row slice (all ranks' partials read over NVLink with plain
+    loads, the rows stored to every rank's outputs), and a second barrier.
+    Every rank ends with the bits the single-GPU moe_reduce_partials gives over
+    the same P partials.
 
-    Fill ``partial[j]`` (this rank's partial rank * per_rank + j) before the
-    call; read ``out_norm`` / ``out_residual`` after it."""
+    Fill ``partial[j]`` (partial rank * per_rank + j) before the call; read
+    ``out_norm`` / ``out_residual`` after it.  A barrier wait that gives up
+    after ``barrier_timeout_ms`` records it in a device word: ``check()``
+    raises MoEError(MOE_ETIMEOUT) if any did.  ``close()`` (collective)
+    releases the memory; the tensors are invalid after it."""
+
+    _ALIGN = 4096
 
     def __init__(self, T: int, D: int, per_rank: int = 1, group=None, device=None,
-                 barrier_timeout_ms: int = 10000):
+                 barrier_timeout_ms: int = 5000):
         import torch
         import torch.distributed as dist
-        import torch.distributed._symmetric_memory as symm
+        self.group = group
         self.world = dist.get_world_size(group)
         self.rank = dist.get_rank(group)
         if self.world * per_rank > 8:
             raise ValueError("at most 8 partials in all")
+        if not 1 <= barrier_timeout_ms <= 60000:
+            raise ValueError("barrier_timeout_ms must be in 1 .. 60000")
         self.T, self.D, self.per_rank = T, D, per_rank
-        self.timeout_ms = barrier_timeout_ms
-        gname = group.group_name if group is not None else dist.group.WORLD.group_name
-        bf = torch.bfloat16
-        self.partial = symm.empty((per_rank, T, D), dtype=bf, device=device)
-        self.out_norm = symm.empty((T, D), dtype=bf, device=device)
-        self.out_residual = symm.empty((T, D), dtype=bf, device=device)
-        self._hp = symm.rendezvous(self.partial, gname)
-        self._hn = symm.rendezvous(self.out_norm, gname)
-        self._hr = symm.rendezvous(self.out_residual, gname)
-        peer_p = [self._hp.get_buffer(r, (per_rank, T, D), bf) for r in range(self.world)]
-        self._partials = [peer_p[r][j] for r, j in partial_order(self.world, per_rank)]
-        self._outs_n = [self._hn.get_buffer(r, (T, D), bf) for r in range(self.world)]
-        self._outs_r = [self._hr.get_buffer(r, (T, D), bf) for r in range(self.world)]
+        self.limit_us = barrier_timeout_ms * 1000
+        up = lambda n: (n + self._ALIGN - 1) // self._ALIGN * self._ALIGN  # noqa: E731
+        buf = T * D * 2
+        off_part = up(4 * self.world)
+        off_norm = off_part + up(per_rank * buf)
+        off_res = off_norm + up(buf)
+        total = off_res + up(buf)
+        dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+        with torch.cuda.device(dev):
+            self._base, handle = peer_alloc(total)
+        self._opened, self._closed = [], False
+        info = [None] * self.world
+        dist.all_gather_object(info, (handle, T, D, per_rank), group=group)
+        if any(x[1:] != (T, D, per_rank) for x in info):
+            raise ValueError(f"ranks disagree on (T, D, per_rank): {[x[1:] for x in info]}")
+        bases = []
+        with torch.cuda.device(dev):
+            for r in range(self.world):
+                if r == self.rank:
+                    bases.append(self._base)
+                else:
+                    bases.append(peer_open(info[r][0]))
+                    self._opened.append(bases[-1])
+        view = lambda addr, n, shape: torch.as_tensor(  # noqa: E731
+            _DeviceArray(addr, n), device=dev).view(torch.bfloat16).view(shape)
+        self.partial = view(self._base + off_part, per_rank * T * D, (per_rank, T, D))
+        self.out_norm = view(self._base + off_norm, T * D, (T, D))
+        self.out_residual = view(self._base + off_res, T * D, (T, D))
+        self._flags = [b for b in bases]
+        self._partials = [bases[r] + off_part + j * buf for r, j in partial_order(self.world, per_rank)]
+        self._outs_n = [b + off_norm for b in bases]
+        self._outs_r = [b + off_res for b in bases]
         self.row0, self.rows = row_slices(T, self.world)[self.rank]
+        self.err = torch.zeros(1, dtype=torch.int32, device=dev)
+        self._epoch = 0
+
+    def _barrier(self, stream):
+        self._epoch += 1
+        peer_barrier(self._flags, self.rank, self._epoch, self.err, self.limit_us, stream)
 
     def __call__(self, residual, g, eps: float = 1e-6, stream=None):
-        import contextlib
-
-        import torch
-        # The barriers run on the current stream: make it the caller's.
-        ctx = torch.cuda.stream(stream) if stream is not None else contextlib.nullcontext()
-        with ctx:
-            # Every rank's partials are written before anyone reads them ...
-            self._hp.barrier(channel=0, timeout_ms=self.timeout_ms)
-            reduce_partials_rows(self._partials, residual, g, self._outs_n, self._outs_r, self.row0, self.rows,
-                                 eps, stream)
-            # ... and every rank's rows are stored before anyone reads the
-            # outputs or rewrites its partials.
-            self._hp.barrier(channel=1, timeout_ms=self.timeout_ms)
+        # Every rank's partials are written before anyone reads them ...
+        self._barrier(stream)
+        reduce_partials_rows(self._partials, residual, g, self._outs_n, self._outs_r, self.row0, self.rows,
+                             eps, stream)
+        # ... and every rank's rows are stored before anyone reads the outputs
+        # or rewrites its partials.
+        self._barrier(stream)
         return self.out_norm, self.out_residual
+
+    def check(self) -> None:
+        """Raise MoEError(MOE_ETIMEOUT) if a barrier wait gave up (synchronises)."""
+        e = int(self.err.item())
+        self.err.zero_()
+        if e:
+            raise MoEError(MOE_ETIMEOUT, "TPAllReduceNorm barrier")
+
+    def close(self) -> None:
+        """Collective: unmap the peers' memory, then free this rank's."""
+        import torch
+        import torch.distributed as dist
+        if self._closed:
+            return
+        torch.cuda.synchronize()
+        dist.barrier(group=self.group)
+        for a in self._opened:
+            peer_close(a)
+        dist.barrier(group=self.group)
+        peer_free(self._base)
+        self._closed = True

@@ -708,6 +708,65 @@ int moe_selftest_wait_timeout(int limit_us, void* stream) {
   return res;
 }
 
+int moe_peer_alloc(size_t bytes, void** dptr, unsigned char* handle) {
+  if (!dptr || !handle || bytes == 0) return MOE_EINVAL;
+  *dptr = nullptr;
+  static_assert(sizeof(cudaIpcMemHandle_t) == MOE_PEER_HANDLE_BYTES, "IPC handle size");
+  void* p = nullptr;
+  if (cudaMalloc(&p, bytes) != cudaSuccess) return MOE_ECUDA;
+  cudaIpcMemHandle_t ih;
+  if (cudaMemset(p, 0, bytes) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess ||
+      cudaIpcGetMemHandle(&ih, p) != cudaSuccess) {
+    cudaFree(p);
+    return MOE_ECUDA;
+  }
+  std::memcpy(handle, &ih, sizeof ih);
+  *dptr = p;
+  return MOE_OK;
+}
+
+int moe_peer_free(void* dptr) {
+  if (!dptr) return MOE_EINVAL;
+  return cudaFree(dptr) == cudaSuccess ? MOE_OK : MOE_ECUDA;
+}
+
+int moe_peer_open(const unsigned char* handle, void** dptr) {
+  if (!handle || !dptr) return MOE_EINVAL;
+  *dptr = nullptr;
+  cudaIpcMemHandle_t ih;
+  std::memcpy(&ih, handle, sizeof ih);
+  void* p = nullptr;
+  if (cudaIpcOpenMemHandle(&p, ih, cudaIpcMemLazyEnablePeerAccess) != cudaSuccess) {
+    cudaGetLastError();  // leave no stale error for the next runtime call
+    return MOE_ECUDA;
+  }
+  *dptr = p;
+  return MOE_OK;
+}
+
+int moe_peer_close(void* dptr) {
+  if (!dptr) return MOE_EINVAL;
+  return cudaIpcCloseMemHandle(dptr) == cudaSuccess ? MOE_OK : MOE_ECUDA;
+}
+
+int moe_peer_barrier(int world, int rank, uint32_t* const* flags, uint32_t epoch, int* err, int limit_us,
+                     void* stream) {
+  if (world < 1 || world > 8 || rank < 0 || rank >= world || !flags || !err || epoch == 0 || limit_us < 1 ||
+      limit_us > 60000000)
+    return MOE_EINVAL;
+  moe::PeerFlags f;
+  for (int r = 0; r < 8; ++r) f.p[r] = nullptr;
+  for (int r = 0; r < world; ++r) {
+    if (!flags[r] || (reinterpret_cast<uintptr_t>(flags[r]) & 3)) return MOE_EINVAL;
+    f.p[r] = flags[r];
+  }
+  const unsigned long long limit_ns = static_cast<unsigned long long>(limit_us) * 1000ull;
+  return moe::launch_peer_barrier(f, world, rank, epoch, err, limit_ns, static_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess
+             ? MOE_OK
+             : MOE_ECUDA;
+}
+
 int moe_destroy(moe_handle* h) {
   if (!h) return MOE_EINVAL;
   for (auto& e : h->ev)

@@ -167,4 +167,11 @@ cudaError_t launch_gather_rows(const uint16_t* src, const int32_t* src_row, int 
 cudaError_t launch_wait_selftest(int* flag, int* err, unsigned long long limit_ns,
                                  cudaStream_t s);
 
+// Flag arrays of the ranks of a peer barrier (addresses in this process).
+struct PeerFlags {
+  uint32_t* p[8];
+};
+cudaError_t launch_peer_barrier(const PeerFlags& f, int world, int rank, uint32_t epoch, int* err,
+                                unsigned long long limit_ns, cudaStream_t s);
+
 }  // namespace moe

@@ -187,7 +187,7 @@ int moe_reduce_partials(int P, const moe_bf16* const* partials, const moe_bf16* 
  * destination pairs (1 <= n_out <= 8): the fused form of the tensor-parallel
  * all-reduce + residual + RMSNorm over NVLink.  With P ranks, rank i passes the
  * P ranks' partial buffers in rank order (its own and its peers', mapped into
- * its address space, e.g. by symmetric memory), its row slice, and every rank's
+ * its address space, e.g. by moe_peer_open), its row slice, and every rank's
  * output buffers: each rank reads all partials of its rows with plain loads,
  * reduces them in the fixed order p = 0 .. P-1, and stores the rows to every
  * rank.  Every rank then holds the same bits as moe_reduce_partials over all T
@@ -283,6 +283,42 @@ int moe_layer_forward_noalloc(moe_handle* h, int T, const moe_bf16* x, const moe
                               const int32_t* token_ids, moe_bf16* out_norm,
                               moe_bf16* out_residual, int32_t* out_topk_idx, float* out_topk_w,
                               int32_t* out_counts, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Peer memory for the tensor-parallel epilogue (one process per GPU).
+ *
+ * moe_peer_alloc allocates `bytes` of zeroed device memory on the current
+ * device and exports it: `handle` (MOE_PEER_HANDLE_BYTES bytes, host memory the
+ * caller owns) is the CUDA IPC handle of the allocation, to be sent to the
+ * other ranks of one node by any host channel.  The allocation is 256-byte
+ * aligned and owned by the caller: release it with moe_peer_free after every
+ * rank has closed its mapping.  Errors: MOE_EINVAL (NULL or bytes == 0),
+ * MOE_ECUDA (allocation or export failed; *dptr is NULL).
+ *
+ * moe_peer_open maps another process's exported allocation into this process
+ * (on the current device, with peer access enabled) and writes its address to
+ * *dptr; moe_peer_close unmaps it.  Opening a handle of this same process is
+ * an error (MOE_ECUDA): use the exporter's own pointer.
+ *
+ * moe_peer_barrier is a device-side barrier of `world` ranks (1 <= world <= 8)
+ * on `stream`: flags[r] is the address (in this process) of rank r's array of
+ * `world` uint32 flag words, zero when allocated.  One thread per rank first
+ * makes this GPU's earlier writes (the stream's previous kernels, local and
+ * peer stores) visible at system scope, then writes `epoch` to slot `rank` of
+ * every rank's array, and waits until every slot of its own array holds a
+ * value >= epoch (wrap-around compare).  All ranks call it with the same epoch
+ * sequence, starting at 1 and growing by one per call.  Each wait gives up
+ * after `limit_us` microseconds (1..60000000): it then stores 1 to the device
+ * int *err (which the caller zeroes and reads), and returns; the CUDA context
+ * stays usable and later kernels run as usual.  Errors: MOE_EINVAL, MOE_ECUDA
+ * (launch failure).  The call does not synchronise. */
+#define MOE_PEER_HANDLE_BYTES 64
+int moe_peer_alloc(size_t bytes, void** dptr, unsigned char* handle);
+int moe_peer_free(void* dptr);
+int moe_peer_open(const unsigned char* handle, void** dptr);
+int moe_peer_close(void* dptr);
+int moe_peer_barrier(int world, int rank, uint32_t* const* flags, uint32_t epoch, int* err, int limit_us,
+                     void* stream);
 
 int moe_destroy(moe_handle* h);
 const char* moe_status_string(int status);

@@ -140,15 +140,28 @@ def _tp_world1(q):
         ref_n, ref_r = torch.empty_like(res), torch.empty_like(res)
         moe.reduce_partials(parts, res, g, ref_n, ref_r)
         torch.cuda.synchronize()
-        q.put(bool(torch.equal(on.view(torch.int16), ref_n.view(torch.int16)) and
-                   torch.equal(orr.view(torch.int16), ref_r.view(torch.int16))))
+        ok = bool(torch.equal(on.view(torch.int16), ref_n.view(torch.int16)) and
+                  torch.equal(orr.view(torch.int16), ref_r.view(torch.int16)))
+        # A second step over new partials: the barriers' epochs advance.
+        for j in range(P):
+            parts[j] = (torch.randn((T, D), generator=gen) / 8).to(torch.bfloat16).cuda()
+            tp.partial[j].copy_(parts[j])
+        on, orr = tp(res, g)
+        moe.reduce_partials(parts, res, g, ref_n, ref_r)
+        torch.cuda.synchronize()
+        tp.check()
+        ok = ok and bool(torch.equal(on.view(torch.int16), ref_n.view(torch.int16)) and
+                         torch.equal(orr.view(torch.int16), ref_r.view(torch.int16)))
+        tp.close()
+        q.put(ok)
     finally:
         dist.destroy_process_group()
 
 
 def test_tp_epilogue_one_rank(torch_cuda):
-    """TPAllReduceNorm on one rank (symmetric-memory buffers, device-side
-    barriers, the row-slice kernel) equals moe_reduce_partials bit for bit."""
+    """TPAllReduceNorm on one rank (exported peer allocation, device-side
+    barriers, the row-slice kernel) equals moe_reduce_partials bit for bit,
+    over two steps."""
     import socket
     import torch.multiprocessing as mp
     s = socket.socket()
@@ -163,3 +176,30 @@ def test_tp_epilogue_one_rank(torch_cuda):
     p.join(timeout=300)
     assert p.exitcode == 0
     assert q.get(timeout=5) is True
+
+
+def test_peer_barrier_times_out(torch_cuda):
+    """A two-rank barrier on one GPU whose second rank never signals (both flag
+    arrays are this process's memory and nothing writes slot 1): the wait gives
+    up after its limit, records the timeout in the error word, and the context
+    keeps working."""
+    import time
+
+    import deterministic_expert_b200 as moe
+    torch = torch_cuda
+    flags = torch.zeros((2, 64), dtype=torch.int32, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    t0 = time.perf_counter()
+    moe.peer_barrier([flags[0].data_ptr(), flags[1].data_ptr()], 0, 1, err, 200000)
+    torch.cuda.synchronize()
+    dt = time.perf_counter() - t0
+    assert int(err.item()) == 1
+    assert 0.15 < dt < 30.0
+    # Rank 0 signalled both arrays in slot 0 and saw its own signal.
+    assert int(flags[0, 0].item()) == 1 and int(flags[1, 0].item()) == 1 and int(flags[0, 1].item()) == 0
+    # The context is usable: a one-rank barrier passes and leaves no error.
+    err.zero_()
+    own = torch.zeros(64, dtype=torch.int32, device="cuda")
+    moe.peer_barrier([own.data_ptr()], 0, 1, err, 200000)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0 and int(own[0].item()) == 1
