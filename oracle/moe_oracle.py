@@ -37,6 +37,10 @@ The layer, in order:
                                           weighted sum, one final cast)
   8. residual add + RMSNorm epilogue     [FW] Trap 2 / Trap 3 (rmsnorm(full_out + residual))
   9. fixed r0..r7 partial reduction      [FW] Trap 1 (Lamport kernel order)
+  FP4 expert weights (optional)          [DS] §6.2 "FP4 QAT": weights FP4 (E2M1) with a
+                                          scale per block, dequantised losslessly to
+                                          FP8, FP8 x FP8 expert GEMMs (activations
+                                          E4M3 with a power-of-two scale per row)
   Latent MoE (optional)                  [LD] "潜在MoE (Latent MoE)", K3 flow: the
                                           router and routed experts read
                                           z = bf16(xn W_down^T); their weighted
@@ -320,6 +324,148 @@ def expert_ffn(xn_rows, w_gate, w_up, w_down, gate_clamp_max=np.inf, up_clamp=np
     return h, h @ Wd.T
 
 
+# ------------------------------------------- FP4 expert weights, FP8 compute
+# [DS] §6.2 "FP4 QAT": expert weights are quantised from the master weights to
+# FP4 (E2M1) with one scale factor per block; FP4 -> FP8 dequantisation is
+# lossless (the 16 FP4 values times the block's scale fit FP8 exactly); the
+# forward is an FP8 x FP8 GEMM.  Readings where the page is silent: the block
+# is 32 consecutive elements along the contraction axis (the last axis of
+# every weight here) and its scale is a power of two 2^s; the FP8 format is
+# E4M3; activations enter each expert GEMM as E4M3 with one power-of-two
+# scale per row (row-local, so batch-invariant); products accumulate exactly
+# and the row scale is applied to the sum.  Every quantisation step divides by
+# a power of two (exact) and rounds to nearest, ties to even.
+WEIGHTS_BF16, WEIGHTS_FP8 = 0, 1
+E2M1_GRID = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])   # magnitudes, code order
+FP4_BLOCK = 32
+FP4_SCALE_MIN, FP4_SCALE_MAX = -8, 6     # 2^s keeps every q * 2^s an E4M3 value
+E4M3_MAX = 448.0
+ACT_EXP_MIN, ACT_EXP_MAX = -126, 126
+
+
+def round_e2m1(x) -> np.ndarray:
+    """Nearest E2M1 value to each x (ties to the even code, i.e. the grid
+    point whose index in E2M1_GRID is even); beyond 6 the nearest is 6."""
+    x = np.asarray(x, np.float64)
+    mag = np.abs(x)
+    d = np.abs(mag[..., None] - E2M1_GRID)                 # distance to every grid point
+    best = d.min(axis=-1, keepdims=True)
+    cand = d == best                                       # one or two nearest points
+    even = cand & (np.arange(8) % 2 == 0)
+    pick = np.where(even.any(axis=-1), even.argmax(axis=-1), cand.argmax(axis=-1))
+    return np.copysign(E2M1_GRID[pick], x)
+
+
+def fp4_block_exponent(amax) -> np.ndarray:
+    """Smallest integer s with amax <= 6 * 2^s, clamped to [-8, 6] (amax = 0
+    gives -8).  Written with frexp: amax = m 2^E, m in [0.5, 1); 6 * 2^(E-3) =
+    0.75 * 2^E, so s = E - 3 when m <= 0.75, else E - 2."""
+    amax = np.asarray(amax, np.float64)
+    m, E = np.frexp(amax)
+    s = np.where(m <= 0.75, E - 3, E - 2)
+    s = np.where(amax == 0, FP4_SCALE_MIN, s)
+    return np.clip(s, FP4_SCALE_MIN, FP4_SCALE_MAX).astype(np.int64)
+
+
+def quantize_weights_fp4(w, block: int = FP4_BLOCK):
+    """Master weights -> FP4: for each block of ``block`` consecutive elements
+    of the last axis, s = fp4_block_exponent(max |w|) and q = round_e2m1(w / 2^s).
+    Returns (q, s) with s of shape [..., K / block]."""
+    w = np.asarray(w, np.float64)
+    K = w.shape[-1]
+    if K % block:
+        raise ValueError("the contraction axis must be a multiple of the block")
+    wb = w.reshape(w.shape[:-1] + (K // block, block))
+    s = fp4_block_exponent(np.abs(wb).max(axis=-1))
+    q = round_e2m1(wb / np.exp2(s)[..., None])
+    return q.reshape(w.shape), s
+
+
+def dequantize_fp4(q, s, block: int = FP4_BLOCK) -> np.ndarray:
+    """FP4 -> FP8 values: q * 2^s per block (exact; every result is an E4M3 value)."""
+    q = np.asarray(q, np.float64)
+    K = q.shape[-1]
+    qb = q.reshape(q.shape[:-1] + (K // block, block))
+    return (qb * np.exp2(np.asarray(s))[..., None]).reshape(q.shape)
+
+
+def fp4_weights_as_fp8(w, block: int = FP4_BLOCK) -> np.ndarray:
+    """The FP8 operand values the expert GEMMs read for master weights w."""
+    return dequantize_fp4(*quantize_weights_fp4(w, block), block)
+
+
+def round_e4m3(x) -> np.ndarray:
+    """Nearest E4M3 value (1 sign, 4 exponent bits with bias 7, 3 mantissa
+    bits; subnormals m/8 * 2^-6; largest finite 448), ties to even; magnitudes
+    above 448 saturate to 448."""
+    x = np.asarray(x, np.float64)
+    mag = np.abs(x)
+    _, E = np.frexp(mag)                       # mag = m 2^E, m in [0.5, 1): binade 2^(E-1)
+    e = np.maximum(E - 1, -6)                  # below 2^-6 the spacing stays 2^-9
+    ulp = np.exp2(e - 3)
+    r = np.rint(mag / ulp) * ulp               # np.rint: ties to even
+    r = np.where(mag == 0, 0.0, np.minimum(r, E4M3_MAX))
+    return np.copysign(r, x)
+
+
+def e4m3_bits(v) -> np.ndarray:
+    """uint8 code of E4M3-representable values (sign | exponent | mantissa)."""
+    v = np.asarray(v, np.float64)
+    if not np.array_equal(round_e4m3(v), v):
+        raise ValueError("not E4M3 values")
+    mag = np.abs(v)
+    _, E = np.frexp(mag)
+    sub = mag < 2.0 ** -6
+    expo = np.where(sub | (mag == 0), 0, E - 1 + 7)
+    mant = np.where(sub | (mag == 0), mag / 2.0 ** -9, (mag / np.exp2(E - 1) - 1.0) * 8)
+    code = (expo.astype(np.int64) << 3) | mant.astype(np.int64)
+    return (code | np.where(np.signbit(v), 0x80, 0)).astype(np.uint8)
+
+
+def act_row_exponent(amax) -> np.ndarray:
+    """Smallest integer e with amax <= 448 * 2^e, clamped to [-126, 126] (amax =
+    0 gives 0).  448 = 0.875 * 2^9, so with amax = m 2^E (m in [0.5, 1)):
+    e = E - 9 when m <= 0.875, else E - 8."""
+    amax = np.asarray(amax, np.float64)
+    m, E = np.frexp(amax)
+    e = np.where(m <= 0.875, E - 9, E - 8)
+    e = np.where(amax == 0, 0, e)
+    return np.clip(e, ACT_EXP_MIN, ACT_EXP_MAX).astype(np.int64)
+
+
+def quantize_act_rows(a):
+    """Per row: e = act_row_exponent(max |a|), q = round_e4m3(a / 2^e).
+    Returns (q, e); the row's value is q * 2^e."""
+    a = np.asarray(a, np.float64)
+    e = act_row_exponent(np.abs(a).max(axis=-1) if a.shape[-1] else np.zeros(a.shape[:-1]))
+    return round_e4m3(a / np.exp2(e)[..., None]), e
+
+
+def expert_ffn_fp8(xn_rows, w8_gate, w8_up, w8_down, gate_clamp_max=np.inf, up_clamp=np.inf,
+                   act: int = ACT_SWIGLU, beta_g: float = 4.0, beta_u: float = 25.0):
+    """One gated expert with FP8 weights (the values fp4_weights_as_fp8 gives)
+    and FP8 activations: xn rows -> (qx, ex); g = (qx W_g^T) 2^ex, u likewise,
+    h = bf16(unit(g, u)); h -> (qh, eh); y = (qh W_d^T) 2^eh.  The sums are of
+    exact products (E4M3 x E4M3 has at most 8 significant bits) and are taken
+    in fp64.  Returns (h, y)."""
+    qx, ex = quantize_act_rows(xn_rows)
+    Wg = np.asarray(w8_gate, np.float64)
+    Wu = np.asarray(w8_up, np.float64)
+    Wd = np.asarray(w8_down, np.float64)
+    n, D = qx.shape
+    I = Wg.shape[0]
+    MAC_COUNTER[0] += n * (2 * D * I + I * Wd.shape[0])
+    sx = np.exp2(ex)[:, None]
+    h = round_bf16(glu_unit((qx @ Wg.T) * sx, (qx @ Wu.T) * sx, act, gate_clamp_max, up_clamp, beta_g, beta_u))
+    qh, eh = quantize_act_rows(h)
+    return h, (qh @ Wd.T) * np.exp2(eh)[:, None]
+
+
+def expert_fn(cfg):
+    """expert_ffn or expert_ffn_fp8, by the configuration's weight format."""
+    return expert_ffn_fp8 if int(getattr(cfg, "weight_format", WEIGHTS_BF16)) == WEIGHTS_FP8 else expert_ffn
+
+
 # ------------------------------------------------------------ latent MoE
 def latent_down(xn, w_proj_down) -> np.ndarray:
     """z = bf16(xn W_down^T): the down-projection W_down of [LD] "潜在MoE (Latent
@@ -426,8 +572,10 @@ def moe_layer(cfg, W, x, residual, token_ids=None, rows=None) -> dict:
     every token; the experts, combine and epilogue for ``rows`` (all tokens
     when None).  ``cfg`` carries D, E, k, I, n_shared, I_shared, router,
     renormalize, routed_scale, gate_clamp_max, up_clamp, eps, hash_mult and
-    optionally activation, situ_beta_gate, situ_beta_up (SiTU-GLU experts) and
-    latent (the latent width l; 0 or absent: no latent projection).
+    optionally activation, situ_beta_gate, situ_beta_up (SiTU-GLU experts),
+    latent (the latent width l; 0 or absent: no latent projection) and
+    weight_format (WEIGHTS_FP8: the expert weights in ``W`` are FP8 values, as
+    fp4_weights_as_fp8 gives, and the experts run expert_ffn_fp8).
 
     Latent MoE ([LD] "潜在MoE" and its K3 flow): the router and the routed
     experts read z = latent_down(xn) (width l), the routed experts' weighted sum
@@ -448,19 +596,20 @@ def moe_layer(cfg, W, x, residual, token_ids=None, rows=None) -> dict:
     offsets, perm_token, perm_slot, pos = stable_permute(idx, cfg.E)
 
     # Expert compute for the selected rows, grouped by expert.
+    ffn = expert_fn(cfg)
     n, k = len(rows), cfg.k
     y_slots = np.zeros((n, k, lat or cfg.D))
     sel = idx[rows]                                   # [n, k]
     for e in np.unique(sel):
         rr, jj = np.nonzero(sel == e)
         Wg, Wu, Wd = W.routed(int(e))
-        _, y = expert_ffn(xe[rows[rr]], Wg, Wu, Wd, **unit_args(cfg))
+        _, y = ffn(xe[rows[rr]], Wg, Wu, Wd, **unit_args(cfg))
         y_slots[rr, jj] = y
     y_shared = np.zeros((cfg.n_shared, n, cfg.D))
     for s in range(cfg.n_shared):
         Wg, Wu, Wd = W.shared(s)
         # The clamp is a property of the SwiGLU unit and applies to shared experts too.
-        _, y_shared[s] = expert_ffn(xn[rows], Wg, Wu, Wd, **unit_args(cfg))
+        _, y_shared[s] = ffn(xn[rows], Wg, Wu, Wd, **unit_args(cfg))
     agg = lat_sum = None
     if lat:
         lat_sum, agg, y_lat = latent_up(w[rows], y_slots, W.w_proj_up)
@@ -491,9 +640,10 @@ def moe_layer_dense_masked(cfg, W, x, residual, token_ids=None) -> dict:
     mask = np.zeros((T, cfg.E))
     np.put_along_axis(mask, idx, w, axis=-1)
     acc = np.zeros((T, lat or cfg.D))
+    ffn = expert_fn(cfg)
     for e in range(cfg.E):
         Wg, Wu, Wd = W.routed(e)
-        _, y = expert_ffn(xe, Wg, Wu, Wd, **unit_args(cfg))
+        _, y = ffn(xe, Wg, Wu, Wd, **unit_args(cfg))
         acc += mask[:, e:e + 1] * y
     lat_sum = None
     if lat:
@@ -501,7 +651,7 @@ def moe_layer_dense_masked(cfg, W, x, residual, token_ids=None) -> dict:
         acc = round_bf16(acc) @ np.asarray(W.w_proj_up, np.float64).T
     for s in range(cfg.n_shared):
         Wg, Wu, Wd = W.shared(s)
-        _, y = expert_ffn(xn, Wg, Wu, Wd, **unit_args(cfg))
+        _, y = ffn(xn, Wg, Wu, Wd, **unit_args(cfg))
         acc += y
     out_norm, out_residual, r = residual_rmsnorm(acc, residual, W.g_out, cfg.eps)
     return dict(acc=acc, r=r, out_norm=out_norm, out_residual=out_residual, idx=idx, w=w, lat_sum=lat_sum)

@@ -507,4 +507,187 @@ def pin_latent_mac_count(O):
     assert O.MAC_COUNTER[0] == T * cfg.k * 3 * 16 * cfg.I + T * 1 * 3 * cfg.D * cfg.I_shared
 
 
+# ------------------------------------------------ FP4 weights, FP8 compute
+def _torch_e4m3(v):
+    """torch's own float8_e4m3fn cast (round to nearest even) of fp32 values."""
+    import torch
+    return torch.from_numpy(np.asarray(v, np.float32)).to(torch.float8_e4m3fn).float().numpy().astype(np.float64)
+
+
+def pin_e4m3_rounding(O):
+    """round_e4m3 / e4m3_bits against torch's float8_e4m3fn conversion (a
+    library routine): every finite code round-trips with its own bits, every
+    midpoint between neighbours goes to the even one, and random values of
+    every binade (normal and subnormal) round the same."""
+    import torch
+    codes = np.arange(256, dtype=np.uint8)
+    vals = torch.from_numpy(codes).view(torch.float8_e4m3fn).float().numpy().astype(np.float64)
+    fin = np.isfinite(vals)
+    assert fin.sum() == 254 and vals[fin].max() == O.E4M3_MAX
+    assert np.array_equal(O.round_e4m3(vals[fin]), vals[fin])
+    assert np.array_equal(O.e4m3_bits(vals[fin]), codes[fin])
+    pos = np.unique(vals[fin & (vals >= 0)])
+    mids = (pos[1:] + pos[:-1]) / 2
+    assert np.array_equal(O.round_e4m3(mids), _torch_e4m3(mids))
+    assert np.array_equal(O.round_e4m3(-mids), _torch_e4m3(-mids))
+    rng = np.random.default_rng(21)
+    r = (rng.standard_normal(50000) * np.exp2(rng.integers(-14, 9, 50000))).astype(np.float32).astype(np.float64)
+    r = r[np.abs(r) <= O.E4M3_MAX]
+    assert np.array_equal(O.round_e4m3(r), _torch_e4m3(r))
+    # Saturation instead of overflow.
+    assert float(O.round_e4m3(1e6)) == O.E4M3_MAX and float(O.round_e4m3(-500.0)) == -O.E4M3_MAX
+
+
+def pin_e2m1_grid(O):
+    """The E2M1 grid from the format's definition (1 sign, 2 exponent bits with
+    bias 1, 1 mantissa bit; exponent field 0 is subnormal), against the page's
+    facts (16 codes, largest magnitude 6), and round_e2m1 against a second,
+    binade-based rounding (spacing 0.5 below 2, 1 in [2, 4), 2 in [4, 6])."""
+    g = golden("fp4_fp8_quantisation.json")
+    vals = []
+    for sign in (1.0, -1.0):
+        for e in range(4):
+            for m in range(2):
+                vals.append(sign * ((m / 2.0) if e == 0 else (1.0 + m / 2.0) * 2.0 ** (e - 1)))
+    assert len(vals) == g["e2m1_codes"] and max(vals) == g["e2m1_max"]
+    assert np.array_equal(np.array(vals[:8]), O.E2M1_GRID)
+    x = np.concatenate([np.linspace(-7, 7, 28001), (O.E2M1_GRID[1:] + O.E2M1_GRID[:-1]) / 2])
+    mag = np.abs(x)
+    spacing = np.where(mag < 2, 0.5, np.where(mag < 4, 1.0, 2.0))
+    # Each binade starts at an even multiple of its spacing, so the even
+    # multiple (np.rint: ties to even) is the even code; above 6 the nearest is 6.
+    alt = np.minimum(np.rint(mag / spacing) * spacing, 6.0)
+    assert np.array_equal(np.abs(O.round_e2m1(x)), alt)
+    assert np.array_equal(np.signbit(O.round_e2m1(x[x != 0])), np.signbit(x[x != 0]))
+
+
+def pin_fp4_lossless(O):
+    """The page's lossless claim: every FP4 value times a block scale 2^s with
+    s in [FP4_SCALE_MIN, FP4_SCALE_MAX] is an E4M3 value (checked with torch's
+    cast), and the range is the widest for which that holds."""
+    q = np.concatenate([O.E2M1_GRID, -O.E2M1_GRID])
+    for s_ in range(O.FP4_SCALE_MIN, O.FP4_SCALE_MAX + 1):
+        v = q * 2.0 ** s_
+        assert np.array_equal(_torch_e4m3(v), v), s_
+    assert not np.array_equal(_torch_e4m3(6.0 * 2.0 ** (O.FP4_SCALE_MAX + 1)), 6.0 * 2.0 ** (O.FP4_SCALE_MAX + 1))
+    assert float(_torch_e4m3(0.5 * 2.0 ** (O.FP4_SCALE_MIN - 1))) != 0.5 * 2.0 ** (O.FP4_SCALE_MIN - 1)
+
+
+def pin_fp4_weight_blocks(O):
+    """Hand-derived FP4 quantisation of two blocks (the golden file's
+    derivation), blocks along the contraction (last) axis only, and the
+    dequantised values lying on E4M3."""
+    g = golden("fp4_fp8_quantisation.json")
+    w = np.zeros((2, 64))
+    w[0, :6] = g["weight_block"]
+    w[0, 32:36] = g["weight_block2"]
+    w[1, 40:46] = g["weight_block"]
+    q, s_ = O.quantize_weights_fp4(w)
+    assert s_.shape == (2, 2)
+    assert s_.tolist() == [[g["weight_block_scale_exp"], g["weight_block2_scale_exp"]],
+                           [O.FP4_SCALE_MIN, g["weight_block_scale_exp"]]]
+    w8 = O.dequantize_fp4(q, s_)
+    assert w8[0, :6].tolist() == g["weight_block_fp8"]
+    assert w8[0, 32:36].tolist() == g["weight_block2_fp8"]
+    assert w8[1, 40:46].tolist() == g["weight_block_fp8"]
+    assert np.count_nonzero(w8) == np.count_nonzero(w8[0, :6]) + 4 + np.count_nonzero(w8[1, 40:46])
+    assert np.array_equal(O.fp4_weights_as_fp8(w), w8)
+    # Scales outside the lossless range are clamped: a block of magnitude 1e-4
+    # would want s = -15 (6 * 2^-15 = 1.8e-4) and gets -8, so its values
+    # (1e-4 / 2^-8 = 0.0256) round to 0; a block of magnitude 1000 would want
+    # s = 8 and gets 6, so 1000 / 64 = 15.6 saturates to 6 * 64 = 384.
+    wc = np.zeros((1, 64))
+    wc[0, 0], wc[0, 32] = 1e-4, -1000.0
+    qc, sc = O.quantize_weights_fp4(wc)
+    assert sc.tolist() == [[O.FP4_SCALE_MIN, O.FP4_SCALE_MAX]] == [[-8, 6]]
+    assert O.dequantize_fp4(qc, sc)[0, [0, 32]].tolist() == [0.0, -384.0]
+    # Random weights: every value is q * 2^s with q on the grid, |w - w8| within
+    # half a grid step of the block (2^s below 2, more above), and E4M3-exact.
+    rng = np.random.default_rng(3)
+    wr = rng.standard_normal((4, 128)) * 0.02
+    q, s_ = O.quantize_weights_fp4(wr)
+    assert np.all(np.isin(np.abs(q), O.E2M1_GRID))
+    w8 = O.dequantize_fp4(q, s_)
+    assert np.array_equal(O.round_e4m3(w8), w8)
+    step = np.repeat(np.exp2(s_), 32, axis=-1)
+    assert np.all(np.abs(wr - w8) <= step)   # worst gap on the grid is 2 units (between 4 and 6)
+
+
+def pin_fp8_activation_rows(O):
+    """Hand-derived per-row activation scales and E4M3 codes, the scale being
+    the smallest power of two that brings the row into +-448."""
+    g = golden("fp4_fp8_quantisation.json")
+    q, e = O.quantize_act_rows(np.array(g["act_rows"]))
+    assert e.tolist() == g["act_row_exp"]
+    assert q.tolist() == g["act_row_q"]
+    rng = np.random.default_rng(4)
+    a = rng.standard_normal((64, 96)) * np.exp2(rng.integers(-20, 20, (64, 1)))
+    q, e = O.quantize_act_rows(a)
+    amax = np.abs(a).max(axis=1)
+    assert np.all(amax <= 448.0 * np.exp2(e)) and np.all(amax > 448.0 * np.exp2(e - 1))
+    assert np.array_equal(q, _torch_e4m3(a / np.exp2(e)[:, None]))
+
+
+def pin_fp8_expert_reduces_to_bf16(O):
+    """When quantisation is the identity -- weights already FP4 values with
+    block scale 1 (every block holds a 6 or -6) and activations E4M3 values
+    whose row maximum is 448 -- the FP8 expert equals the plain expert exactly;
+    with rows scaled by powers of two, g and u scale exactly."""
+    rng = np.random.default_rng(8)
+    D, I, n = 64, 32, 5
+    grid = np.concatenate([O.E2M1_GRID, -O.E2M1_GRID])
+    Wg, Wu, Wd = (rng.choice(grid, size=sh) for sh in ((I, D), (I, D), (D, I)))
+    for Wm in (Wg, Wu, Wd):
+        Wm[:, ::32] = 6.0
+        assert np.array_equal(O.fp4_weights_as_fp8(Wm), Wm)
+    x = _torch_e4m3(rng.standard_normal((n, D)) * 30)
+    x[:, 3] = 448.0
+    h_ref, y_ref = O.expert_ffn(x, Wg, Wu, Wd)
+    h8, y8 = O.expert_ffn_fp8(x, Wg, Wu, Wd)
+    assert np.array_equal(h8, h_ref)
+    qh, eh = O.quantize_act_rows(h_ref)
+    assert np.array_equal(y8, (qh @ Wd.T) * np.exp2(eh)[:, None])
+    # The down input is quantised: y8 differs from the unquantised down product
+    # wherever h is not an E4M3 multiple of its row scale.
+    assert not np.array_equal(y8, y_ref)
+    # Scaling a row of x by 2^j scales its gate/up sums by exactly 2^j.
+    xs = x * 2.0 ** -7
+    qx, ex = O.quantize_act_rows(xs)
+    assert np.array_equal(qx, x) and np.all(ex == -7)
+
+
+def _fp8_weights(O, W):
+    """The same layer with every expert weight replaced by its FP8 values."""
+    q = O.fp4_weights_as_fp8
+    return O.Weights(W.w_router, W.router_bias, q(W.w_gate), q(W.w_up), q(W.w_down), q(W.ws_gate),
+                     q(W.ws_up), q(W.ws_down), W.g_in, W.g_out)
+
+
+def pin_fp8_dense_masked(O):
+    """The FP8 layer's routed path against the every-expert masked sum, and
+    sampled rows against the full run."""
+    cfg, W, x, res, ids = small_random_case(O, weight_format=O.WEIGHTS_FP8, renormalize=1)
+    W8 = _fp8_weights(O, W)
+    a = O.moe_layer(cfg, W8, x, res, ids)
+    b = O.moe_layer_dense_masked(cfg, W8, x, res, ids)
+    assert np.array_equal(a["idx"], b["idx"])
+    assert np.allclose(a["r"], b["r"], rtol=1e-12, atol=1e-12)
+    rows = np.array([5, 1, 20])
+    c = O.moe_layer(cfg, W8, x, res, ids, rows=rows)
+    assert np.array_equal(c["out_norm"], a["out_norm"][rows])
+    # The layer's slot outputs are the FP8 expert's (activations quantised per
+    # row), not the plain expert's on the FP8 weights.
+    for t, j in ((0, 0), (7, 1), (23, 0)):
+        e = int(a["idx"][t, j])
+        y8 = O.expert_ffn_fp8(a["xn"][[t]], *W8.routed(e))[1][0]
+        assert np.array_equal(a["y_slots"][t, j], y8)
+        assert not np.array_equal(O.expert_ffn(a["xn"][[t]], *W8.routed(e))[1][0], y8)
+    # FP8 experts follow the bf16 layer on the master weights loosely (4-bit
+    # weights of Gaussian values with power-of-two block scales are off by about
+    # 12% in norm; two of them in series give about 20% here) and never equal it.
+    ref = O.moe_layer(types.SimpleNamespace(**{**vars(cfg), "weight_format": O.WEIGHTS_BF16}), W, x, res, ids)
+    rel = np.linalg.norm(a["acc"] - ref["acc"]) / np.linalg.norm(ref["acc"])
+    assert 1e-2 < rel < 0.5
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

@@ -63,10 +63,24 @@ MUTATIONS = {
                              "    return np.asarray(xn, np.float64) @ np.asarray(w_proj_down, np.float64).T"),
     "latent_sum_not_rounded": ("    a = round_bf16(s)\n", "    a = s\n"),
     "latent_router_reads_xn": ("        logits = router_logits(xe, W.w_router)", "        logits = router_logits(xn, W.w_router)"),
-    "latent_experts_read_xn": ("_, y = expert_ffn(xe[rows[rr]]", "_, y = expert_ffn(xn[rows[rr]]"),
-    "latent_shared_reads_z": ("_, y_shared[s] = expert_ffn(xn[rows]", "_, y_shared[s] = expert_ffn(xe[rows]"),
+    "latent_experts_read_xn": ("_, y = ffn(xe[rows[rr]]", "_, y = ffn(xn[rows[rr]]"),
+    "latent_shared_reads_z": ("_, y_shared[s] = ffn(xn[rows]", "_, y_shared[s] = ffn(xe[rows]"),
     "latent_shared_dropped": ("        acc = combine(np.ones((n, 1)), y_lat[:, None, :], y_shared)",
                               "        acc = combine(np.ones((n, 1)), y_lat[:, None, :], None)"),
+    "fp4_scale_floor": ("s = np.where(m <= 0.75, E - 3, E - 2)", "s = np.where(m <= 0.75, E - 4, E - 3)"),
+    "fp4_ties_to_odd": ("even = cand & (np.arange(8) % 2 == 0)", "even = cand & (np.arange(8) % 2 == 1)"),
+    "fp4_block_along_rows": ("    wb = w.reshape(w.shape[:-1] + (K // block, block))\n    s = fp4_block_exponent(np.abs(wb).max(axis=-1))",
+                             "    wb = w.reshape(w.shape[:-1] + (K // block, block))\n    s = np.broadcast_to(fp4_block_exponent(np.abs(wb).max(axis=(-1, 0))), wb.shape[:-1])"),
+    "fp4_scale_range_unclamped": ("return np.clip(s, FP4_SCALE_MIN, FP4_SCALE_MAX).astype(np.int64)",
+                                  "return np.clip(s, FP4_SCALE_MIN - 4, FP4_SCALE_MAX + 4).astype(np.int64)"),
+    "e4m3_no_subnormals": ("e = np.maximum(E - 1, -6)", "e = E - 1"),
+    "e4m3_ties_away": ("r = np.rint(mag / ulp) * ulp", "r = np.floor(mag / ulp + 0.5) * ulp"),
+    "act_scale_off_by_one": ("e = np.where(m <= 0.875, E - 9, E - 8)", "e = np.where(m <= 0.875, E - 8, E - 7)"),
+    "act_scale_not_applied": ("h = round_bf16(glu_unit((qx @ Wg.T) * sx, (qx @ Wu.T) * sx,",
+                              "h = round_bf16(glu_unit((qx @ Wg.T), (qx @ Wu.T),"),
+    "down_input_not_quantised": ("return h, (qh @ Wd.T) * np.exp2(eh)[:, None]", "return h, h @ Wd.T"),
+    "fp8_path_ignored": ("return expert_ffn_fp8 if int(getattr(cfg, \"weight_format\", WEIGHTS_BF16)) == WEIGHTS_FP8 else expert_ffn",
+                         "return expert_ffn"),
     "histogram_off_by_one": ("return np.bincount(np.asarray(idx).ravel(), minlength=E).astype(np.int64)",
                              "return np.bincount(np.asarray(idx).ravel() % max(E - 1, 1), minlength=E).astype(np.int64)"),
 }
