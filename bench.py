@@ -5,7 +5,7 @@
                     [--workload NAME] [--T TOKENS] [--no-cpu-baseline]
 
 --workload picks another workload (v3_shaped, skew_zipf, skew_hash,
-fine_grained_situ, latent_situ, tiny, or skew_epilogue for the 8-partial
+fine_grained_situ, latent_situ, fine_grained_fp8, tiny, tiny_fp8, or skew_epilogue for the 8-partial
 reduce + residual + RMSNorm); --T overrides the batch size (the decode sweep
 is --T 1, 8, 64, 128, 512 on the fine-grained weights).
 
@@ -76,7 +76,8 @@ def describe(cfg):
             "n_shared": cfg.n_shared, "I_shared": cfg.I_shared,
             "router": {0: "softmax", 1: "sigmoid+bias", 2: "hash"}[cfg.router],
             "renormalize": bool(cfg.renormalize),
-            "activation": "SiTU-GLU" if cfg.activation == 1 else "SwiGLU", "latent": cfg.latent}
+            "activation": "SiTU-GLU" if cfg.activation == 1 else "SwiGLU", "latent": cfg.latent,
+            "expert_weights": "FP4 values as E4M3 (E4M3 x E4M3 GEMMs)" if cfg.weight_format else "bf16"}
 
 
 def peaks():
@@ -159,6 +160,8 @@ def oracle_sample(cfg, budget_s=12.0, chunk=256):
     import oracle as O
     from synth import device as SD
     hw = SD.HostWeights(cfg)
+    if cfg.weight_format:
+        hw = O.FP4Weights(hw)   # the oracle's own FP4 quantisation of the master weights
     for e in range(cfg.E):
         hw.routed(e)
     for s in range(cfg.n_shared):
@@ -194,6 +197,8 @@ def run_reference(a):
     from synth import device as SD
     from synth import workloads as W
     hw = SD.HostWeights(cfg)
+    if cfg.weight_format:
+        hw = O.FP4Weights(hw)   # the oracle's own FP4 quantisation of the master weights
     for e in range(cfg.E):
         hw.routed(e)
     for s in range(cfg.n_shared):
@@ -443,6 +448,11 @@ def main():
     stream = torch.cuda.current_stream()
 
     w = SD.device_weights(cfg, device=dev)
+    if cfg.weight_format:
+        # FP4 expert weights: the library's quantiser turns the bf16 master
+        # weights into their E4M3 codes once, before anything is timed.
+        w = moe.quantize_expert_weights(w)
+        torch.cuda.synchronize()
     # Each rank takes its own T rows of a world*T-row batch (disjoint tokens).
     xa, ra, ida = SD.device_inputs(cfg, T=T * world, device=dev)
     x, r, ids = (xa[rank * T:(rank + 1) * T].contiguous(), ra[rank * T:(rank + 1) * T].contiguous(),
@@ -547,13 +557,18 @@ def main():
 
     if rank == 0:
         tc_peak, hbm_peak, peak_kind = peaks()
+        peak_src = f"{peak_kind} bf16 (burst)"
+        if cfg.weight_format:
+            # E4M3 x E4M3: the measured bf16 peak times the nominal dense ratio
+            # of the two formats (4.5 / 2.25 PFLOP/s).
+            tc_peak, peak_src = 2.0 * tc_peak, f"{peak_kind} bf16 (burst) x 2, nominal E4M3 / bf16 ratio"
         fl = W.moe_flops(cfg)
         gate_ms = stage_ms[GATEUP_STAGE] / max(stage_n[GATEUP_STAGE], 1)
         achieved = fl["gateup"] / (gate_ms / 1e3) / 1e12
         traffic = ncu_traffic(cfg)
         roof = {"bound": "tensor", "kernel": "gemm_gateup_swiglu", "achieved": round(achieved, 1),
                 "peak": tc_peak, "unit": "TFLOP/s", "frac": round(achieved / tc_peak, 4),
-                "traffic": traffic, "peak_source": f"{peak_kind} bf16 (burst)",
+                "traffic": traffic, "peak_source": peak_src,
                 "flops_per_launch": fl["gateup"], "avg_launch_ms": round(gate_ms, 4)}
         layer_tflops = fl["total"] / (ms_per_step / 1e3) / 1e12
         cpu = None
@@ -562,7 +577,8 @@ def main():
         line = {
             "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
             "steps": a.steps, "warmup": a.warmup, "ms_per_step": round(ms_per_step, 4),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "e4m3" if cfg.weight_format else "bf16",
             "data": "synthetic (seeded counter-based generator; random weights of the workload's shape)",
             "config": {**describe(cfg), "l2": "flushed before every step (512 MiB write, untimed)",
                        "parallelism": f"replicas x{world} (token-sharded, no collective)"},

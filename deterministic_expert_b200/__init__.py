@@ -22,10 +22,11 @@ MOE_OK, MOE_EINVAL, MOE_ETOOBIG, MOE_EWORKSPACE, MOE_EUNSUPPORTED, MOE_ECUDA, MO
     0, -1, -2, -3, -4, -5, -6)
 ROUTER_SOFTMAX, ROUTER_SIGMOID_BIAS, ROUTER_HASH = 0, 1, 2
 ACT_SWIGLU, ACT_SITU_GLU = 0, 1
-NUM_STAGES = 11
+WEIGHTS_BF16, WEIGHTS_FP8 = 0, 1
+NUM_STAGES = 12
 STAGE_NAMES = ("rmsnorm_in", "router_gemm", "router_topk", "dispatch", "gather_rows",
                "gemm_gateup_swiglu", "gemm_down", "combine_norm", "latent_down", "latent_combine",
-               "latent_up")
+               "latent_up", "quant_h")
 
 
 class MoEError(RuntimeError):
@@ -41,7 +42,7 @@ class moe_config(ctypes.Structure):
                 ("routed_scale", ctypes.c_float), ("gate_clamp_max", ctypes.c_float),
                 ("up_clamp", ctypes.c_float), ("eps", ctypes.c_float), ("hash_mult", ctypes.c_uint32),
                 ("activation", ctypes.c_int), ("situ_beta_gate", ctypes.c_float),
-                ("situ_beta_up", ctypes.c_float), ("latent", ctypes.c_int)]
+                ("situ_beta_up", ctypes.c_float), ("latent", ctypes.c_int), ("weight_format", ctypes.c_int)]
 
 
 class moe_weights(ctypes.Structure):
@@ -57,7 +58,9 @@ class moe_views(ctypes.Structure):
                 ("dest_row", ctypes.c_void_p), ("h_routed", ctypes.c_void_p),
                 ("h_shared", ctypes.c_void_p), ("y_slot", ctypes.c_void_p),
                 ("y_shared", ctypes.c_void_p), ("z", ctypes.c_void_p), ("agg", ctypes.c_void_p),
-                ("y_latent", ctypes.c_void_p)]
+                ("y_latent", ctypes.c_void_p), ("xq", ctypes.c_void_p), ("xq_exp", ctypes.c_void_p),
+                ("hq_routed", ctypes.c_void_p), ("hq_routed_exp", ctypes.c_void_p),
+                ("hq_shared", ctypes.c_void_p), ("hq_shared_exp", ctypes.c_void_p)]
 
 
 _lib = None
@@ -133,13 +136,14 @@ class LayerConfig:
     situ_beta_gate: float = 4.0
     situ_beta_up: float = 25.0
     latent: int = 0
+    weight_format: int = WEIGHTS_BF16
 
     def to_c(self) -> moe_config:
         return moe_config(self.D, self.E, self.k, self.I, self.n_shared,
                           self.I_shared if self.n_shared else self.I, self.T_max, self.router,
                           self.renormalize, self.routed_scale, self.gate_clamp_max, self.up_clamp,
                           self.eps, self.hash_mult, self.activation, self.situ_beta_gate,
-                          self.situ_beta_up, self.latent)
+                          self.situ_beta_up, self.latent, self.weight_format)
 
 
 def _check_weight_sizes(cfg: LayerConfig, weights: dict) -> None:
@@ -160,6 +164,8 @@ def _check_weight_sizes(cfg: LayerConfig, weights: dict) -> None:
                              f"got {t.numel()} (contiguous={t.is_contiguous()})")
         import torch
         dtype = torch.float32 if name == "router_bias" else torch.bfloat16
+        if cfg.weight_format == WEIGHTS_FP8 and name in ("w_gate", "w_up", "w_down", "ws_gate", "ws_up", "ws_down"):
+            dtype = torch.uint8   # E4M3 codes
         if t.dtype != dtype:
             raise ValueError(f"weight {name}: expected {dtype}, got {t.dtype}")
 
@@ -252,6 +258,40 @@ def reduce_partials(partials, residual, g, out_norm, out_residual, eps: float = 
     _check(lib().moe_reduce_partials(P, arr, _ptr(residual), _ptr(g), _ptr(out_norm),
                                      _ptr(out_residual), T, D, eps, _stream(stream)),
            "moe_reduce_partials")
+
+
+def quantize_weights_fp4(w, w8, block_exp=None, stream=None) -> None:
+    """moe_quantize_weights_fp4: bf16 master weights [..., K] -> E4M3 codes (uint8,
+    same shape) of their FP4 values, and optionally the int8 block exponents
+    [..., K / 32]."""
+    L = lib()
+    K = int(w.shape[-1])
+    rows = w.numel() // K if K else 0
+    if w8.numel() != w.numel() or w8.dtype.itemsize != 1:
+        raise ValueError("w8 must be a byte tensor with as many elements as w")
+    L.moe_quantize_weights_fp4.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                           ctypes.c_longlong, ctypes.c_int, ctypes.c_void_p]
+    _check(L.moe_quantize_weights_fp4(_ptr(w), _ptr(w8), _ptr(block_exp), rows, K, _stream(stream)),
+           "moe_quantize_weights_fp4")
+
+
+EXPERT_WEIGHTS = ("w_gate", "w_up", "w_down", "ws_gate", "ws_up", "ws_down")
+
+
+def quantize_expert_weights(weights: dict, stream=None) -> dict:
+    """A copy of a moe_weights dict whose expert matrices (bf16 master weights)
+    are replaced by their E4M3 codes from quantize_weights_fp4, for a layer
+    configured with weight_format=WEIGHTS_FP8.  Other entries are shared."""
+    import torch
+    out = dict(weights)
+    for n in EXPERT_WEIGHTS:
+        t = weights.get(n)
+        if t is None:
+            continue
+        q = torch.empty(t.shape, dtype=torch.uint8, device=t.device)
+        quantize_weights_fp4(t, q, stream=stream)
+        out[n] = q
+    return out
 
 
 def selftest_wait_timeout(limit_us: int, stream=None) -> int:

@@ -4,6 +4,7 @@
 #pragma once
 #include <cstdint>
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 
 namespace moe {
@@ -265,6 +266,14 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
          (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// Instruction descriptor, kind::f8f6f4: fp32 accumulator (bits 4-5 = 1), A and
+// B E4M3 (type code 0 at bits 7-9 and 10-12), both K-major, N >> 3 at bits
+// 17-22, M >> 4 at bits 24-28.  One MMA then walks 32 K elements (32 bytes of a
+// 128-byte swizzled row, as the bf16 form's 16).
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
+  return (1u << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
 // D[tmem] (+)= A[smem] * B[smem]^T, one M x N x 16 step, issued by one thread.
 __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                           uint32_t idesc, uint32_t accumulate) {
@@ -272,6 +281,17 @@ __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// The E4M3 form: one M x N x 32 step.
+__device__ __forceinline__ void umma_e4m3(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
@@ -296,6 +316,38 @@ __device__ __forceinline__ void umma_bf16_pair(uint32_t d_tmem, uint64_t a_desc,
       "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
+}
+
+// The E4M3 form of the pair MMA: one M x N x 32 step.
+__device__ __forceinline__ void umma_e4m3_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                               uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// 2^e as an fp32 value for -126 <= e <= 127 (exact: a normal power of two).
+__device__ __forceinline__ float exp2_int(int e) { return __int_as_float((e + 127) << 23); }
+
+// ------------------------------------------------------------ E4M3 rows
+// Per-row scale of E4M3 activations: the smallest integer e with
+// amax <= 448 * 2^e, clamped to [-126, 126]; 0 for amax = 0.  With
+// amax = m 2^E (m in [0.5, 1)) and 448 = 0.875 * 2^9, e = E - 9 when
+// m <= 0.875, else E - 8 (exact: frexpf only splits the bits).
+__device__ __forceinline__ int act_row_exp(float amax) {
+  if (!(amax > 0.f)) return 0;
+  int E = 0;
+  const float m = frexpf(amax, &E);
+  const int e = m <= 0.875f ? E - 9 : E - 8;
+  return min(max(e, -126), 126);
+}
+
+// E4M3 code of v, round to nearest even, saturating at +-448.
+__device__ __forceinline__ uint32_t e4m3_rn(float v) {
+  return static_cast<uint32_t>(__nv_cvt_float_to_fp8(v, __NV_SATFINITE, __NV_E4M3));
 }
 
 // Arrive once on `bar` (same offset) in each CTA of cta_mask when the pair's

@@ -13,7 +13,8 @@
 //             token bitmask per expert + popcount): grouped row
 //             p = offsets[e] + (pairs of e in earlier tokens).  Block 0 also
 //             writes the counts, the offsets and the two expert-GEMM tile lists.
-//   gather    xp[p] = xn[src_token[p]]  (the routed GEMM's A operand)
+//   gather    xp[p] = xn[src_token[p]]  (the routed GEMM's A operand; bf16
+//             rows, or E4M3 rows and their exponents)
 #include "common.cuh"
 #include "moe_internal.h"
 
@@ -144,15 +145,20 @@ __global__ void __launch_bounds__(kDispatchRows) k_dispatch(const DispatchArgs a
 }
 
 // dst[p] = src[src_row[p]], one warp per row, 16-byte vectors.
-__global__ void k_gather_rows(const uint16_t* __restrict__ src, const int32_t* __restrict__ src_row,
-                              int rows, int D, uint16_t* __restrict__ dst) {
+// Row p of dst = row src_row[p] of src (row_bytes each, a multiple of 16: bf16
+// rows or E4M3 rows), and with E4M3 rows also their exponents.
+__global__ void k_gather_rows(const uint8_t* __restrict__ src, const int32_t* __restrict__ src_row,
+                              int rows, int row_bytes, uint8_t* __restrict__ dst,
+                              const int8_t* __restrict__ src_exp, int8_t* __restrict__ dst_exp) {
   griddep_wait();
   griddep_launch();
   const int p = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   if (p >= rows) return;
-  const uint4* s = reinterpret_cast<const uint4*>(src + static_cast<size_t>(src_row[p]) * D);
-  uint4* d = reinterpret_cast<uint4*>(dst + static_cast<size_t>(p) * D);
-  for (int c = lane; c < D / 8; c += 32) d[c] = s[c];
+  const int from = src_row[p];
+  const uint4* s = reinterpret_cast<const uint4*>(src + static_cast<size_t>(from) * row_bytes);
+  uint4* d = reinterpret_cast<uint4*>(dst + static_cast<size_t>(p) * row_bytes);
+  for (int c = lane; c < row_bytes / 16; c += 32) d[c] = s[c];
+  if (dst_exp != nullptr && lane == 0) dst_exp[p] = src_exp[from];
 }
 
 }  // namespace
@@ -162,12 +168,13 @@ cudaError_t launch_dispatch(const DispatchArgs& a, cudaStream_t s) {
   return launch_k(k_dispatch, dim3(nb), dim3(kDispatchRows), 0, s, false, a);
 }
 
-cudaError_t launch_gather_rows(const uint16_t* src, const int32_t* src_row, int rows, int D,
-                               uint16_t* dst, cudaStream_t s) {
+cudaError_t launch_gather_rows(const void* src, const int32_t* src_row, int rows, int row_bytes, void* dst,
+                               const int8_t* src_exp, int8_t* dst_exp, cudaStream_t s) {
   if (rows <= 0) return cudaSuccess;
   const int warps_per_block = 8;
   return launch_k(k_gather_rows, dim3((rows + warps_per_block - 1) / warps_per_block),
-                  dim3(32 * warps_per_block), 0, s, false, src, src_row, rows, D, dst);
+                  dim3(32 * warps_per_block), 0, s, false, static_cast<const uint8_t*>(src), src_row, rows,
+                  row_bytes, static_cast<uint8_t*>(dst), src_exp, dst_exp);
 }
 
 }  // namespace moe

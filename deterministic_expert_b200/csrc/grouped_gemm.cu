@@ -144,9 +144,13 @@ __device__ __forceinline__ float glu_unit(float g, float u, const GemmArgs& a) {
   return silu_clamped_product(g, u, a.gate_clamp, a.up_clamp);
 }
 
-template <int MODE, int CG, int ACT>
+template <int MODE, int CG, int ACT, int F8>
 __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_constant__ GemmArgs a) {
   using C = Cfg<CG>;
+  // K elements per 128-byte operand row of a stage: 64 bf16 or 128 E4M3.  Every
+  // byte count below (stage slots, TMA boxes, descriptor steps) is the same for
+  // both; an E4M3 MMA walks 32 elements where a bf16 one walks 16.
+  constexpr int KE = F8 ? 2 * kBK : kBK;
   // Stage ring.  The expert GEMMs use as many stages of kSmemA + C::kSmemB bytes
   // as fit (6); the router, whose B tile is only E_pad rows, packs as many
   // stages of kSmemA + E_pad * 128 bytes as fit (up to 8), so one CTA walking
@@ -224,7 +228,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
       for (int t = cluster_id; ok && t < total; t += n_clusters) {
         Tile ti;
         decode_tile<CG>(a, t, ti);
-        const int nkb = a.k_kind[ti.kind] / kBK;
+        const int nkb = a.k_kind[ti.kind] / KE;
         // A: this CTA's rows of the tile (128, or 64 in a 128-row pair tile,
         // loaded with the 64-row box so no unused rows cross into shared memory).
         // Swapped tile: this CTA's nt / 2 token rows (the B operand's half).
@@ -248,17 +252,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
           uint8_t* b0 = sB + stage * sb_bytes;
           if (CG == 1) {
             mbar_arrive_expect_tx(&full[stage], tx);
-            tma_load_2d(sA + stage * sa_bytes, amap, kb * kBK, a_y, &full[stage]);
-            tma_load_2d(b0, bmap, kb * kBK, b_y, &full[stage]);
+            tma_load_2d(sA + stage * sa_bytes, amap, kb * KE, a_y, &full[stage]);
+            tma_load_2d(b0, bmap, kb * KE, b_y, &full[stage]);
             if (MODE == kGateUp)
-              tma_load_2d(b0 + b_rows * kBK * 2, bmap + 1, kb * kBK, b_y, &full[stage]);
+              tma_load_2d(b0 + b_rows * kBK * 2, bmap + 1, kb * KE, b_y, &full[stage]);
           } else {
             // The even CTA expects the bytes of both CTAs on its barrier.
             if (leader) mbar_arrive_expect_tx(&full[stage], 2 * tx);
-            tma_load_2d_pair(sA + stage * sa_bytes, amap, kb * kBK, a_y, full0 + 8 * stage);
-            tma_load_2d_pair(b0, bmap, kb * kBK, b_y, full0 + 8 * stage);
+            tma_load_2d_pair(sA + stage * sa_bytes, amap, kb * KE, a_y, full0 + 8 * stage);
+            tma_load_2d_pair(b0, bmap, kb * KE, b_y, full0 + 8 * stage);
             if (MODE == kGateUp)
-              tma_load_2d_pair(b0 + (BN / 2) * kBK * 2, bmap + 1, kb * kBK, b_y, full0 + 8 * stage);
+              tma_load_2d_pair(b0 + (BN / 2) * kBK * 2, bmap + 1, kb * KE, b_y, full0 + 8 * stage);
           }
           issued[stage] = static_cast<int>(phase);
           if (++stage == S) { stage = 0; phase ^= 1u; }
@@ -277,8 +281,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
       // memory (CG = 1) or in the two CTAs of the pair (CG = 2), so one
       // N = 2*BN MMA reads A once and writes the gate accumulator to columns
       // [0, BN) and the up accumulator to [BN, 2*BN).
-      const uint32_t idesc_full = idesc_bf16_f32(C::kTileM, n_mma);
-      const uint32_t idesc_small = idesc_bf16_f32(128, n_mma);  // pair tile of 128 rows
+      auto idesc_of = [](int M, int N) { return F8 ? idesc_e4m3_f32(M, N) : idesc_bf16_f32(M, N); };
+      const uint32_t idesc_full = idesc_of(C::kTileM, n_mma);
+      const uint32_t idesc_small = idesc_of(128, n_mma);  // pair tile of 128 rows
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -287,13 +292,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
       for (int t = cluster_id; ok && t < total; t += n_clusters) {
         Tile ti;
         decode_tile<CG>(a, t, ti);
-        const int nkb = a.k_kind[ti.kind] / kBK;
+        const int nkb = a.k_kind[ti.kind] / KE;
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort, a.err, a.timeout_ns)) break;
         tc_fence_after();
         const uint32_t d0 = tmem_base + static_cast<uint32_t>(acc) * acc_stride;
         // Swapped tiles are one M = 256 pair MMA per step: 128 weight rows per CTA
         // (gate/up: the 64 gate rows then the 64 up rows of its output columns).
-        const uint32_t idesc = ti.swap ? idesc_bf16_f32(256, ti.nt) : (ti.small ? idesc_small : idesc_full);
+        const uint32_t idesc = ti.swap ? idesc_of(256, ti.nt) : (ti.small ? idesc_small : idesc_full);
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(&full[stage], phase, abort, a.err, a.timeout_ns)) { ok = false; break; }
           tc_fence_after();
@@ -308,8 +313,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
             const uint64_t ad = sw128_kmajor_desc(a_addr + kk * 32);
             const uint64_t bd = sw128_kmajor_desc(b_addr + kk * 32);
             const uint32_t accum = (kb | kk) != 0 ? 1u : 0u;
-            if (CG == 2) umma_bf16_pair(d0, ad, bd, idesc, accum);
-            else umma_bf16(d0, ad, bd, idesc, accum);
+            if (F8) {
+              if (CG == 2) umma_e4m3_pair(d0, ad, bd, idesc, accum);
+              else umma_e4m3(d0, ad, bd, idesc, accum);
+            } else {
+              if (CG == 2) umma_bf16_pair(d0, ad, bd, idesc, accum);
+              else umma_bf16(d0, ad, bd, idesc, accum);
+            }
           }
           if (CG == 2) umma_commit_pair_mc(&empty[stage], 0x3);
           else umma_commit(&empty[stage]);
@@ -387,10 +397,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
               for (int j = 0; j < 32; ++j) u[j] = xbuf[lane * 32 + (j ^ lane)];
               __syncwarp();
               if (lane == 0) mbar_arrive(&xempty[pch]);
+              // fp8: token c + lane's row scale, handed to every lane per token.
+              float my_sc = 1.f;
+              if (F8 && c + lane < r) my_sc = exp2_int(a.a_exp[ti.kind][ti.a_row0 + trow0 + c + lane]);
 #pragma unroll
               for (int j = 0; j < 32; ++j) {
+                const float sc = F8 ? __shfl_sync(0xffffffffu, my_sc, j) : 1.f;
                 if (c + j < r) {
-                  const float hv = glu_unit<ACT>(__uint_as_float(v[j]), __uint_as_float(u[j]), a);
+                  float gv = __uint_as_float(v[j]), uv = __uint_as_float(u[j]);
+                  if (F8) { gv = __fmul_rn(gv, sc); uv = __fmul_rn(uv, sc); }
+                  const float hv = glu_unit<ACT>(gv, uv, a);
                   outb[static_cast<size_t>(orow0 + c + j) * ld + col] =
                       static_cast<uint16_t>(pack_bf16x2(hv, 0.f) & 0xFFFFu);
                 }
@@ -418,16 +434,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
             tmem_ld_wait();
             const int my_tok = c + lane;  // this lane fetches the output row of token c + lane
             int my_row = 0;
-            if (my_tok < r) my_row = scatter ? a.dest_row[ti.a_row0 + trow0 + my_tok] : orow0 + my_tok;
+            float my_sc = 1.f;
+            if (my_tok < r) {
+              my_row = scatter ? a.dest_row[ti.a_row0 + trow0 + my_tok] : orow0 + my_tok;
+              if (F8) my_sc = exp2_int(a.a_exp[ti.kind][ti.a_row0 + trow0 + my_tok]);
+            }
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
               const int orow = __shfl_sync(0xffffffffu, my_row, j);
+              const float sc = F8 ? __shfl_sync(0xffffffffu, my_sc, j) : 1.f;
               if (c + j < r) {
+                const float val = F8 ? __fmul_rn(__uint_as_float(v[j]), sc) : __uint_as_float(v[j]);
                 if (a.out_bf16)
                   outh[static_cast<size_t>(orow) * ld + col] =
-                      static_cast<uint16_t>(pack_bf16x2(__uint_as_float(v[j]), 0.f) & 0xFFFFu);
+                      static_cast<uint16_t>(pack_bf16x2(val, 0.f) & 0xFFFFu);
                 else
-                  outb[static_cast<size_t>(orow) * ld + col] = __uint_as_float(v[j]);
+                  outb[static_cast<size_t>(orow) * ld + col] = val;
               }
             }
           }
@@ -443,6 +465,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
       const int colhalf = small ? (q >> 1) : 0;           // which half of the columns (small)
       const int grow0 = ti.m * C::kTileM + static_cast<int>(rank) * (small ? 64 : 128) + row_in_cta;
       const int nvalid = max(0, min(32, ti.rows - grow0));
+      // fp8: this thread's row scale (row grow0 + lane of the group's A rows).
+      float rsc = 1.f;
+      if (F8 && lane < nvalid) rsc = exp2_int(a.a_exp[ti.kind][ti.a_row0 + grow0 + lane]);
       if (MODE == kGateUp) {
         // Output block b covers columns [b*G, b*G + G) with its gate values in
         // TMEM columns [2bG, 2bG + G) and up values in [2bG + G, 2bG + 2G), G = BN/2.
@@ -461,6 +486,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
             tmem_ld32(tb + tcol + c, g);
             tmem_ld32(tb + tcol + G + c, u);
             tmem_ld_wait();
+            if (F8) {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                g[i] = __float_as_uint(__fmul_rn(__uint_as_float(g[i]), rsc));
+                u[i] = __float_as_uint(__fmul_rn(__uint_as_float(u[i]), rsc));
+              }
+            }
             uint32_t p[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i)
@@ -495,6 +527,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
           uint32_t v[32];
           tmem_ld32(tb + c, v);
           tmem_ld_wait();
+          if (F8) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__fmul_rn(__uint_as_float(v[i]), rsc));
+          }
           if (ncols - c >= 32 && a.out_bf16) {
             // bf16 output (latent down-projection): 64 bytes per row, four
             // 16-byte chunks, staged so each store covers whole row segments.
@@ -585,9 +621,9 @@ cudaLaunchConfig_t pair_config(int grid, cudaStream_t s, cudaLaunchAttribute* at
   return cfg;
 }
 
-template <int MODE, int CG, int ACT = MOE_ACT_SWIGLU>
+template <int MODE, int CG, int ACT = MOE_ACT_SWIGLU, int F8 = 0>
 cudaError_t launch_one(const GemmArgs& a, int grid, cudaStream_t s) {
-  return launch_k(k_grouped_gemm<MODE, CG, ACT>, dim3(grid), dim3(kGemmThreads), kGemmSmem, s, CG == 2, a);
+  return launch_k(k_grouped_gemm<MODE, CG, ACT, F8>, dim3(grid), dim3(kGemmThreads), kGemmSmem, s, CG == 2, a);
 }
 
 int g_pair_clusters[64] = {0};
@@ -599,24 +635,32 @@ void gemm_prepare() {
   int dev = 0;
   cudaGetDevice(&dev);
   if (done_dev == dev) return;
-  cudaFuncSetAttribute(k_grouped_gemm<kGateUp, 2, MOE_ACT_SWIGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                       kGemmSmem);
-  cudaFuncSetAttribute(k_grouped_gemm<kGateUp, 2, MOE_ACT_SITU_GLU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                       kGemmSmem);
-  cudaFuncSetAttribute(k_grouped_gemm<kDown, 2, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem);
-  cudaFuncSetAttribute(k_grouped_gemm<kRouter, 1, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem);
+  const cudaFuncAttribute smem_attr = cudaFuncAttributeMaxDynamicSharedMemorySize;
+  cudaFuncSetAttribute(k_grouped_gemm<kGateUp, 2, MOE_ACT_SWIGLU, 0>, smem_attr, kGemmSmem);
+  cudaFuncSetAttribute(k_grouped_gemm<kGateUp, 2, MOE_ACT_SITU_GLU, 0>, smem_attr, kGemmSmem);
+  cudaFuncSetAttribute(k_grouped_gemm<kGateUp, 2, MOE_ACT_SWIGLU, 1>, smem_attr, kGemmSmem);
+  cudaFuncSetAttribute(k_grouped_gemm<kGateUp, 2, MOE_ACT_SITU_GLU, 1>, smem_attr, kGemmSmem);
+  cudaFuncSetAttribute(k_grouped_gemm<kDown, 2, 0, 0>, smem_attr, kGemmSmem);
+  cudaFuncSetAttribute(k_grouped_gemm<kDown, 2, 0, 1>, smem_attr, kGemmSmem);
+  cudaFuncSetAttribute(k_grouped_gemm<kRouter, 1, 0, 0>, smem_attr, kGemmSmem);
   // How many CTA pairs fit on the device at once: the persistent pair grid is
   // never larger, so no pair waits for another to finish before it starts.
-  int n_gu = 0, n_dn = 0;
   cudaLaunchAttribute attr[1];
   cudaLaunchConfig_t cfg = pair_config(2, nullptr, attr);
-  int n_gs = 0;
-  if (cudaOccupancyMaxActiveClusters(&n_gu, k_grouped_gemm<kGateUp, 2, 0>, &cfg) != cudaSuccess) n_gu = 0;
-  if (cudaOccupancyMaxActiveClusters(&n_gs, k_grouped_gemm<kGateUp, 2, 1>, &cfg) != cudaSuccess) n_gs = 0;
-  if (cudaOccupancyMaxActiveClusters(&n_dn, k_grouped_gemm<kDown, 2, 0>, &cfg) != cudaSuccess) n_dn = 0;
-  n_gu = std::min(n_gu, n_gs);
+  int n = 1 << 30;
+  auto occ = [&](const void* fn) {
+    int c = 0;
+    if (cudaOccupancyMaxActiveClusters(&c, fn, &cfg) != cudaSuccess) c = 0;
+    n = std::min(n, c);
+  };
+  occ(reinterpret_cast<const void*>(k_grouped_gemm<kGateUp, 2, 0, 0>));
+  occ(reinterpret_cast<const void*>(k_grouped_gemm<kGateUp, 2, 1, 0>));
+  occ(reinterpret_cast<const void*>(k_grouped_gemm<kGateUp, 2, 0, 1>));
+  occ(reinterpret_cast<const void*>(k_grouped_gemm<kGateUp, 2, 1, 1>));
+  occ(reinterpret_cast<const void*>(k_grouped_gemm<kDown, 2, 0, 0>));
+  occ(reinterpret_cast<const void*>(k_grouped_gemm<kDown, 2, 0, 1>));
   cudaGetLastError();
-  if (dev >= 0 && dev < 64) g_pair_clusters[dev] = std::min(n_gu, n_dn);
+  if (dev >= 0 && dev < 64) g_pair_clusters[dev] = n;
   done_dev = dev;
 }
 
@@ -628,11 +672,15 @@ int gemm_max_pairs() {
 
 cudaError_t launch_grouped_gemm(int mode, const GemmArgs& a, int grid, cudaStream_t s) {
   if (grid <= 0) return cudaSuccess;
+  const bool f8 = a.fp8 != 0;
   switch (mode) {
     case kGateUp:
-      return a.act == MOE_ACT_SITU_GLU ? launch_one<kGateUp, 2, MOE_ACT_SITU_GLU>(a, grid, s)
-                                       : launch_one<kGateUp, 2>(a, grid, s);
-    case kDown: return launch_one<kDown, 2>(a, grid, s);
+      if (a.act == MOE_ACT_SITU_GLU)
+        return f8 ? launch_one<kGateUp, 2, MOE_ACT_SITU_GLU, 1>(a, grid, s)
+                  : launch_one<kGateUp, 2, MOE_ACT_SITU_GLU, 0>(a, grid, s);
+      return f8 ? launch_one<kGateUp, 2, MOE_ACT_SWIGLU, 1>(a, grid, s)
+                : launch_one<kGateUp, 2, MOE_ACT_SWIGLU, 0>(a, grid, s);
+    case kDown: return f8 ? launch_one<kDown, 2, 0, 1>(a, grid, s) : launch_one<kDown, 2, 0, 0>(a, grid, s);
     default: return launch_one<kRouter, 1>(a, grid, s);
   }
 }

@@ -19,6 +19,7 @@ struct moe_handle {
   moe_weights w;
   int S = 0, G = 0, E_pad = 0, bn_gu = 0, bn_dn = 0, num_sms = 0, device = 0, max_pairs = 0;
   int L = 0;                          // width the router and routed experts read (latent or D)
+  bool fp8 = false;                   // MOE_WEIGHTS_FP8: E4M3 expert GEMMs
   int bn_pd = 0, bn_pu = 0;           // N tiles of the latent down / up projections
   uint16_t* w_router_pad = nullptr;  // [E_pad, L], rows >= E zero
   CUtensorMap map_router, map_wg, map_wu, map_wd, map_wsg, map_wsu, map_wsd, map_pd, map_pu;
@@ -38,7 +39,7 @@ size_t align256(size_t b) { return (b + 255) & ~static_cast<size_t>(255); }
 
 struct Layout {
   size_t err, xn, logits, tidx, tw, bcount, counts, offsets, tiles_gu, tiles_dn, dest, src,
-      xp, h, hs, y, ys, z, agg, ylat, total;
+      xp, h, hs, y, ys, z, agg, ylat, xq, xqe, xpe, hq, hqs, he, hse, total;
 };
 
 Layout layout(const moe_handle* h, int T) {
@@ -60,7 +61,8 @@ Layout layout(const moe_handle* h, int T) {
   L.dest = take(Tz * c.k * 4);
   L.src = take(Tz * c.k * 4);
   const size_t Lw = static_cast<size_t>(h->L);
-  L.xp = take(Tz * c.k * Lw * 2);
+  const size_t eb = h->fp8 ? 1 : 2;   // bytes per element of the expert GEMMs' inputs
+  L.xp = take(Tz * c.k * Lw * eb);
   L.h = take(Tz * c.k * c.I * 2);
   L.hs = take(static_cast<size_t>(h->S) * Tz * c.I_shared * 2);
   L.y = take(Tz * c.k * Lw * 4);
@@ -69,6 +71,15 @@ Layout layout(const moe_handle* h, int T) {
   L.z = take(lat ? Tz * Lw * 2 : 0);
   L.agg = take(lat ? Tz * Lw * 2 : 0);
   L.ylat = take(lat ? Tz * c.D * 4 : 0);
+  // E4M3 inputs of the expert GEMMs and their per-row exponents.
+  const size_t f = h->fp8 ? 1 : 0;
+  L.xq = take(f * Tz * c.D);
+  L.xqe = take(f * Tz);
+  L.xpe = take(f * Tz * c.k);
+  L.hq = take(f * Tz * c.k * c.I);
+  L.hqs = take(f * static_cast<size_t>(h->S) * Tz * c.I_shared);
+  L.he = take(f * Tz * c.k);
+  L.hse = take(f * static_cast<size_t>(h->S) * Tz);
   L.total = off;
   return L;
 }
@@ -103,19 +114,22 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 2D bf16 tensor map over a row-major [rows, inner] matrix; box = 64 columns
-// (128 bytes, the 128-byte swizzle span) x box_rows rows.  Rows past the end
-// read as zeros.  An empty matrix leaves the map zeroed (never loaded).
-bool make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t rows, uint32_t box_rows) {
+// 2D tensor map over a row-major [rows, inner] matrix of bf16 (elem_bytes 2)
+// or E4M3 bytes (elem_bytes 1); box = 128 bytes of a row (the 128-byte swizzle
+// span: 64 bf16 or 128 E4M3) x box_rows rows.  Rows past the end read as
+// zeros.  An empty matrix leaves the map zeroed (never loaded).
+bool make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t rows, uint32_t box_rows,
+              int elem_bytes = 2) {
   std::memset(m, 0, sizeof(*m));
   if (rows == 0 || ptr == nullptr) return true;
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {inner, rows};
-  cuuint64_t strides[1] = {inner * 2};
-  cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK), box_rows};
+  cuuint64_t strides[1] = {inner * static_cast<cuuint64_t>(elem_bytes)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / elem_bytes), box_rows};
   cuuint32_t estr[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+  const CUtensorMapDataType dt = elem_bytes == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  return fn(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -140,6 +154,10 @@ int validate_config(const moe_config* c, const moe_weights* w) {
         c->situ_beta_up < 3.0e38f))
     return MOE_EINVAL;
   if (c->D % 64 || c->I % 64 || (c->n_shared > 0 && c->I_shared % 64)) return MOE_EUNSUPPORTED;
+  if (c->weight_format != MOE_WEIGHTS_BF16 && c->weight_format != MOE_WEIGHTS_FP8) return MOE_EINVAL;
+  if (c->weight_format == MOE_WEIGHTS_FP8 &&
+      (c->D % 128 || c->I % 128 || (c->n_shared > 0 && c->I_shared % 128) || c->latent > 0))
+    return MOE_EUNSUPPORTED;
   if (c->D > 16384 || c->E > 256 || c->k > c->E || c->k > 16 || c->n_shared > 8 || c->T_max > (1 << 20))
     return MOE_EUNSUPPORTED;
   const long long rows = static_cast<long long>(c->T_max) * std::max(c->k, c->n_shared);
@@ -233,6 +251,15 @@ int forward_impl(moe_handle* h, int T, const uint16_t* x, const uint16_t* residu
   uint16_t* aggb = reinterpret_cast<uint16_t*>(ws + L.agg);
   float* ylat = reinterpret_cast<float*>(ws + L.ylat);
   const int LW = h->L;
+  const bool f8 = h->fp8;
+  const int eb = f8 ? 1 : 2;
+  uint8_t* xq = ws + L.xq;
+  int8_t* xqe = reinterpret_cast<int8_t*>(ws + L.xqe);
+  int8_t* xpe = reinterpret_cast<int8_t*>(ws + L.xpe);
+  uint8_t* hq = ws + L.hq;
+  uint8_t* hqs = ws + L.hqs;
+  int8_t* he = reinterpret_cast<int8_t*>(ws + L.he);
+  int8_t* hse = reinterpret_cast<int8_t*>(ws + L.hse);
 
   // One dense group of T rows through the CTA-pair GEMM (latent projections):
   // out[T, N] = A[T, K] B[N, K]^T, bf16 or fp32 out.
@@ -263,7 +290,8 @@ int forward_impl(moe_handle* h, int T, const uint16_t* x, const uint16_t* residu
   const int nblk = (T + kDispatchRows - 1) / kDispatchRows;
   const int E4 = (c.E + 3) / 4 * 4;
   prof.begin(0);
-  MOE_TRY(launch_rmsnorm_rows(x, h->w.g_in, xn, T, c.D, c.eps, err, bcount, nblk * E4, s));
+  MOE_TRY(launch_rmsnorm_rows(x, h->w.g_in, xn, T, c.D, c.eps, err, bcount, nblk * E4, f8 ? xq : nullptr,
+                              f8 ? xqe : nullptr, s));
   prof.end(0);
 
   // Latent MoE: the router and the routed experts read z = bf16(xn W_down^T).
@@ -326,19 +354,24 @@ int forward_impl(moe_handle* h, int T, const uint16_t* x, const uint16_t* residu
 
   // 4. grouped A rows of the routed experts
   prof.begin(4);
-  MOE_TRY(launch_gather_rows(xe, src, TK, LW, xp, s));
+  if (f8) MOE_TRY(launch_gather_rows(xq, src, TK, LW, xp, xqe, xpe, s));
+  else MOE_TRY(launch_gather_rows(xe, src, TK, LW * 2, xp, nullptr, nullptr, s));
   prof.end(4);
 
   // 5. gate/up + SwiGLU(+clamp): routed groups read xp, shared groups read xn
   {
     GemmArgs g;
     std::memset(&g, 0, sizeof(g));
-    if (!make_map(&g.mapA[0], xp, LW, TK, kBM)) return MOE_ECUDA;
-    if (!make_map(&g.mapA64[0], xp, LW, TK, kBM / 2)) return MOE_ECUDA;
-    if (!make_map(&g.mapA16[0], xp, LW, TK, 16)) return MOE_ECUDA;
-    if (h->S > 0 && !make_map(&g.mapA[1], xn, c.D, T, kBM)) return MOE_ECUDA;
-    if (h->S > 0 && !make_map(&g.mapA64[1], xn, c.D, T, kBM / 2)) return MOE_ECUDA;
-    if (h->S > 0 && !make_map(&g.mapA16[1], xn, c.D, T, 16)) return MOE_ECUDA;
+    // E4M3: the routed rows are the gathered E4M3 rows, the shared rows xq.
+    const void* xs = f8 ? static_cast<const void*>(xq) : static_cast<const void*>(xn);
+    if (!make_map(&g.mapA[0], xp, LW, TK, kBM, eb)) return MOE_ECUDA;
+    if (!make_map(&g.mapA64[0], xp, LW, TK, kBM / 2, eb)) return MOE_ECUDA;
+    if (!make_map(&g.mapA16[0], xp, LW, TK, 16, eb)) return MOE_ECUDA;
+    if (h->S > 0 && !make_map(&g.mapA[1], xs, c.D, T, kBM, eb)) return MOE_ECUDA;
+    if (h->S > 0 && !make_map(&g.mapA64[1], xs, c.D, T, kBM / 2, eb)) return MOE_ECUDA;
+    if (h->S > 0 && !make_map(&g.mapA16[1], xs, c.D, T, 16, eb)) return MOE_ECUDA;
+    g.fp8 = f8;
+    g.a_exp[0] = xpe; g.a_exp[1] = xqe;
     g.mapB[0] = h->map_wg; g.mapB[1] = h->map_wu; g.mapB[2] = h->map_wsg; g.mapB[3] = h->map_wsu;
     g.offsets = offsets; g.tile_start = tiles_gu; g.G = h->G; g.E = c.E; g.T = T;
     g.n_kind[0] = c.I; g.n_kind[1] = c.I_shared;
@@ -360,19 +393,28 @@ int forward_impl(moe_handle* h, int T, const uint16_t* x, const uint16_t* residu
     prof.end(5);
   }
 
+  // 5b. E4M3: h rows (routed and shared) to E4M3 with their row exponents
+  if (f8) {
+    prof.begin(11);
+    MOE_TRY(launch_quant_rows(hb, TK, c.I, hq, he, hsb, h->S * T, c.I_shared, hqs, hse, s));
+    prof.end(11);
+  }
+
   // 6. down: routed rows scatter to their (token, slot) row of y
   {
     GemmArgs g;
     std::memset(&g, 0, sizeof(g));
-    if (!make_map(&g.mapA[0], hb, c.I, TK, kBM)) return MOE_ECUDA;
-    if (!make_map(&g.mapA64[0], hb, c.I, TK, kBM / 2)) return MOE_ECUDA;
-    if (!make_map(&g.mapA16[0], hb, c.I, TK, 16)) return MOE_ECUDA;
-    if (h->S > 0 && !make_map(&g.mapA[1], hsb, c.I_shared, static_cast<uint64_t>(h->S) * T, kBM))
-      return MOE_ECUDA;
-    if (h->S > 0 && !make_map(&g.mapA64[1], hsb, c.I_shared, static_cast<uint64_t>(h->S) * T, kBM / 2))
-      return MOE_ECUDA;
-    if (h->S > 0 && !make_map(&g.mapA16[1], hsb, c.I_shared, static_cast<uint64_t>(h->S) * T, 16))
-      return MOE_ECUDA;
+    const void* ar = f8 ? static_cast<const void*>(hq) : static_cast<const void*>(hb);
+    const void* as = f8 ? static_cast<const void*>(hqs) : static_cast<const void*>(hsb);
+    const uint64_t srows = static_cast<uint64_t>(h->S) * T;
+    if (!make_map(&g.mapA[0], ar, c.I, TK, kBM, eb)) return MOE_ECUDA;
+    if (!make_map(&g.mapA64[0], ar, c.I, TK, kBM / 2, eb)) return MOE_ECUDA;
+    if (!make_map(&g.mapA16[0], ar, c.I, TK, 16, eb)) return MOE_ECUDA;
+    if (h->S > 0 && !make_map(&g.mapA[1], as, c.I_shared, srows, kBM, eb)) return MOE_ECUDA;
+    if (h->S > 0 && !make_map(&g.mapA64[1], as, c.I_shared, srows, kBM / 2, eb)) return MOE_ECUDA;
+    if (h->S > 0 && !make_map(&g.mapA16[1], as, c.I_shared, srows, 16, eb)) return MOE_ECUDA;
+    g.fp8 = f8;
+    g.a_exp[0] = he; g.a_exp[1] = hse;
     g.mapB[0] = h->map_wd; g.mapB[2] = h->map_wsd;
     g.offsets = offsets; g.tile_start = tiles_dn; g.G = h->G; g.E = c.E; g.T = T;
     g.n_kind[0] = LW; g.n_kind[1] = c.D;
@@ -452,6 +494,7 @@ int moe_init(const moe_config* cfg, const moe_weights* w, moe_handle** out) {
   // on CTA pairs: each CTA loads half of a gate/up tile (bn_gu / 2 gate rows and
   // bn_gu / 2 up rows) or half of a down tile (bn_dn / 2 rows).
   h->L = cfg->latent > 0 ? cfg->latent : cfg->D;
+  h->fp8 = cfg->weight_format == MOE_WEIGHTS_FP8;
   h->bn_gu = (cfg->I % 128 == 0 && h->cfg.I_shared % 128 == 0) ? 128 : 64;
   // The down GEMM's routed groups have N = L, its shared groups N = D.
   auto bn_for = [](int n) { return n % 256 == 0 ? 256 : (n % 128 == 0 ? 128 : 64); };
@@ -473,13 +516,14 @@ int moe_init(const moe_config* cfg, const moe_weights* w, moe_handle** out) {
     if (cudaMemcpy(h->w_router_pad, w->w_router, static_cast<size_t>(c.E) * row, cudaMemcpyDeviceToDevice) != cudaSuccess)
       return fail(MOE_ECUDA);
   }
+  const int eb = h->fp8 ? 1 : 2;   // expert weights: E4M3 or bf16
   bool ok = make_map(&h->map_router, h->w_router_pad, h->L, h->w_router_pad ? h->E_pad : 0, h->E_pad) &&
-            make_map(&h->map_wg, w->w_gate, h->L, static_cast<uint64_t>(c.E) * c.I, h->bn_gu / 2) &&
-            make_map(&h->map_wu, w->w_up, h->L, static_cast<uint64_t>(c.E) * c.I, h->bn_gu / 2) &&
-            make_map(&h->map_wd, w->w_down, c.I, static_cast<uint64_t>(c.E) * h->L, h->bn_dn / 2) &&
-            make_map(&h->map_wsg, w->ws_gate, c.D, static_cast<uint64_t>(h->S) * c.I_shared, h->bn_gu / 2) &&
-            make_map(&h->map_wsu, w->ws_up, c.D, static_cast<uint64_t>(h->S) * c.I_shared, h->bn_gu / 2) &&
-            make_map(&h->map_wsd, w->ws_down, c.I_shared, static_cast<uint64_t>(h->S) * c.D, h->bn_dn / 2) &&
+            make_map(&h->map_wg, w->w_gate, h->L, static_cast<uint64_t>(c.E) * c.I, h->bn_gu / 2, eb) &&
+            make_map(&h->map_wu, w->w_up, h->L, static_cast<uint64_t>(c.E) * c.I, h->bn_gu / 2, eb) &&
+            make_map(&h->map_wd, w->w_down, c.I, static_cast<uint64_t>(c.E) * h->L, h->bn_dn / 2, eb) &&
+            make_map(&h->map_wsg, w->ws_gate, c.D, static_cast<uint64_t>(h->S) * c.I_shared, h->bn_gu / 2, eb) &&
+            make_map(&h->map_wsu, w->ws_up, c.D, static_cast<uint64_t>(h->S) * c.I_shared, h->bn_gu / 2, eb) &&
+            make_map(&h->map_wsd, w->ws_down, c.I_shared, static_cast<uint64_t>(h->S) * c.D, h->bn_dn / 2, eb) &&
             make_map(&h->map_pd, c.latent > 0 ? w->w_proj_down : nullptr, c.D, c.latent, h->bn_pd / 2) &&
             make_map(&h->map_pu, c.latent > 0 ? w->w_proj_up : nullptr, h->L, c.D, h->bn_pu / 2);
   if (!ok) return fail(MOE_ECUDA);
@@ -650,6 +694,13 @@ int moe_workspace_views(const moe_handle* h, int T, void* workspace, moe_views* 
   out->z = lat ? reinterpret_cast<const moe_bf16*>(ws + L.z) : nullptr;
   out->agg = lat ? reinterpret_cast<const moe_bf16*>(ws + L.agg) : nullptr;
   out->y_latent = lat ? reinterpret_cast<const float*>(ws + L.ylat) : nullptr;
+  const bool f8 = h->fp8;
+  out->xq = f8 ? ws + L.xq : nullptr;
+  out->xq_exp = f8 ? reinterpret_cast<const int8_t*>(ws + L.xqe) : nullptr;
+  out->hq_routed = f8 ? ws + L.hq : nullptr;
+  out->hq_routed_exp = f8 ? reinterpret_cast<const int8_t*>(ws + L.he) : nullptr;
+  out->hq_shared = f8 ? ws + L.hqs : nullptr;
+  out->hq_shared_exp = f8 ? reinterpret_cast<const int8_t*>(ws + L.hse) : nullptr;
   return MOE_OK;
 }
 
@@ -688,7 +739,8 @@ int moe_profile_read(moe_handle* h, float* ms, int* launches) {
 int moe_forward_launch_count(const moe_handle* h, int T) {
   if (!h || T < 0) return -1;
   if (T == 0) return 0;
-  const int base = 8 + (h->cfg.latent > 0 ? 3 : 0);  // latent: two projections and the latent sum
+  const int base = 8 + (h->cfg.latent > 0 ? 3 : 0)   // latent: two projections and the latent sum
+                   + (h->fp8 ? 1 : 0);                // E4M3: quantisation of h
   return h->cfg.router == MOE_ROUTER_HASH ? base - 1 : base;  // hash routing: no router GEMM
 }
 
@@ -706,6 +758,15 @@ int moe_selftest_wait_timeout(int limit_us, void* stream) {
     res = host[1] == kDevTimeout ? MOE_ETIMEOUT : MOE_OK;
   cudaFree(buf);
   return res;
+}
+
+int moe_quantize_weights_fp4(const moe_bf16* w, uint8_t* w8, int8_t* block_exp, long long rows, int K,
+                             void* stream) {
+  if (!w || !w8 || rows < 0 || K <= 0 || K % 32 || !aligned16(w) || !aligned16(w8)) return MOE_EINVAL;
+  return launch_quant_weights_fp4(w, w8, block_exp, rows * (K / 32), static_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess
+             ? MOE_OK
+             : MOE_ECUDA;
 }
 
 int moe_peer_alloc(size_t bytes, void** dptr, unsigned char* handle) {

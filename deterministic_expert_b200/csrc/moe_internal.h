@@ -74,6 +74,9 @@ struct GemmArgs {
   int router_tiles;       // tile count when tile_start is NULL (M-tiles x N-tiles)
   int dense_kind;         // kind of the single group when tile_start is NULL
   int out_bf16;           // down-mode output as bf16 instead of fp32 (latent projection)
+  int fp8;                // expert GEMMs: A and B are E4M3 codes (kind::f8f6f4)
+  const int8_t* a_exp[2]; // fp8: per kind, power-of-two exponent of each A row; the
+                          // accumulator of row r is multiplied by 2^a_exp[kind][r]
   void* out[2];           // output base per kind
   int ld_out[2];          // output row pitch (elements) per kind
   int shared_out_stride;  // output rows between consecutive shared experts
@@ -92,9 +95,17 @@ cudaError_t launch_grouped_gemm(int mode, const GemmArgs& a, int grid, cudaStrea
 
 // --------------------------------------------------------------- row ops
 // Also clears the device error word and zeroes `zero_words` int32 at `zero`.
+// yq != NULL: also the E4M3 copy of y with one power-of-two exponent per row.
 cudaError_t launch_rmsnorm_rows(const uint16_t* x, const uint16_t* g, uint16_t* y, int T, int D,
                                 float eps, int* err_to_clear, int32_t* zero, int zero_words,
-                                cudaStream_t s);
+                                uint8_t* yq, int8_t* yq_exp, cudaStream_t s);
+// bf16 rows -> E4M3 rows + per-row exponents, two segments.
+cudaError_t launch_quant_rows(const uint16_t* a0, int rows0, int w0, uint8_t* q0, int8_t* e0,
+                              const uint16_t* a1, int rows1, int w1, uint8_t* q1, int8_t* e1,
+                              cudaStream_t s);
+// FP4 (E2M1, power-of-two scale per 32-element block) -> E4M3 weights.
+cudaError_t launch_quant_weights_fp4(const uint16_t* w, uint8_t* w8, int8_t* block_exp, long long nblocks,
+                                     cudaStream_t s);
 // topk_w == NULL: every slot weighs 1.
 cudaError_t launch_combine_norm(const float* y_slot, const float* topk_w, const float* y_shared,
                                 int k, int S, const uint16_t* residual, const uint16_t* g,
@@ -160,8 +171,8 @@ struct DispatchArgs {
   int32_t* src_token;     // [T * k]
 };
 cudaError_t launch_dispatch(const DispatchArgs& a, cudaStream_t s);
-cudaError_t launch_gather_rows(const uint16_t* src, const int32_t* src_row, int rows, int D,
-                               uint16_t* dst, cudaStream_t s);
+cudaError_t launch_gather_rows(const void* src, const int32_t* src_row, int rows, int row_bytes, void* dst,
+                               const int8_t* src_exp, int8_t* dst_exp, cudaStream_t s);
 
 // ------------------------------------------------------------ self test
 cudaError_t launch_wait_selftest(int* flag, int* err, unsigned long long limit_ns,

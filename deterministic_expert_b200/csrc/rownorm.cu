@@ -12,6 +12,8 @@
 //                    fp64 sum of squares (same fixed tree) so that the bf16 code of
 //                    xn, which decides the routing, is fixed by a well-defined fp32
 //                    scale (linux.do post on MoE variants, "RMSNorm before up-projection")
+//                    (with FP8 expert weights also an E4M3 copy of xn with one
+//                    power-of-two scale per row; quant_rows does the same for h)
 //   combine_norm     acc = sum_j w_j y_j (slot order) + sum_s y_s; r = acc + residual;
 //                    out_residual = bf16(r); out_norm = bf16(RMSNorm(r) * g)
 //                    (Fireworks post, Trap 3 unfused chain and case-study "standard path":
@@ -74,13 +76,40 @@ __device__ __forceinline__ float inv_rms(float ss, int D, float eps) {
   return 1.0f / sqrtf(ss / static_cast<float>(D) + eps);
 }
 
+// Largest value of amax over the block (max is exact, so any order gives the
+// same result); every thread receives it.
+__device__ __forceinline__ float block_max(float amax, float* redf) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  if ((threadIdx.x & 31) == 0) redf[threadIdx.x >> 5] = amax;
+  __syncthreads();
+  float m = redf[0];
+#pragma unroll
+  for (int w = 1; w < kRowThreads / 32; ++w) m = fmaxf(m, redf[w]);
+  return m;
+}
+
+// Eight E4M3 codes of v * 2^-e (exact scaling) packed into 8 bytes, element 0
+// in the lowest byte.
+__device__ __forceinline__ uint2 e4m3x8(const float (&v)[8], float inv_scale) {
+  uint32_t lo = 0, hi = 0;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    lo |= e4m3_rn(__fmul_rn(v[q], inv_scale)) << (8 * q);
+    hi |= e4m3_rn(__fmul_rn(v[q + 4], inv_scale)) << (8 * q);
+  }
+  return make_uint2(lo, hi);
+}
+
 template <int NC>
 __global__ void __launch_bounds__(kRowThreads) k_rmsnorm_rows(const uint16_t* __restrict__ x,
                                                               const uint16_t* __restrict__ g,
                                                               uint16_t* __restrict__ y, int D,
                                                               float eps, int* err, int32_t* zero,
-                                                              int zero_words) {
+                                                              int zero_words, uint8_t* __restrict__ yq,
+                                                              int8_t* __restrict__ yq_exp) {
   __shared__ double red[kRowThreads / 32 + 1];
+  __shared__ float redf[kRowThreads / 32];
   griddep_wait();
   griddep_launch();
   if (err != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *err = kDevOk;
@@ -111,6 +140,7 @@ __global__ void __launch_bounds__(kRowThreads) k_rmsnorm_rows(const uint16_t* __
   const double ms = block_sum_fixed_f64(ss, red) / static_cast<double>(D);
   const float inv = static_cast<float>(1.0 / sqrt(ms + static_cast<double>(eps)));
   uint16_t* yr = y + row * D;
+  float amax = 0.f;
 #pragma unroll
   for (int i = 0; i < NC; ++i) {
     const int c = threadIdx.x + i * kRowThreads;
@@ -120,8 +150,61 @@ __global__ void __launch_bounds__(kRowThreads) k_rmsnorm_rows(const uint16_t* __
 #pragma unroll
       for (int q = 0; q < 8; ++q) o[q] = v[i].v[q] * inv * gg.v[q];
       st_bf16x8(yr + 8 * c, o);
+      if (yq != nullptr) {
+        // Keep the bf16 values (what the expert GEMMs read) for the E4M3 copy.
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          v[i].v[q] = bf16_lo(pack_bf16x2(o[q], 0.f));
+          amax = fmaxf(amax, fabsf(v[i].v[q]));
+        }
+      }
     }
   }
+  if (yq == nullptr) return;
+  // E4M3 copy of the row with its power-of-two scale (MOE_WEIGHTS_FP8).
+  const int e = act_row_exp(block_max(amax, redf));
+  const float inv_scale = exp2_int(-e);
+  uint8_t* qr = yq + row * D;
+#pragma unroll
+  for (int i = 0; i < NC; ++i) {
+    const int c = threadIdx.x + i * kRowThreads;
+    if (c < nch) *reinterpret_cast<uint2*>(qr + 8 * c) = e4m3x8(v[i].v, inv_scale);
+  }
+  if (threadIdx.x == 0) yq_exp[row] = static_cast<int8_t>(e);
+}
+
+// Rows of h (bf16) -> E4M3 rows + per-row exponent (MOE_WEIGHTS_FP8, the down
+// GEMM's input).  One warp per row, two passes over the row (the second from
+// L2): the row's largest magnitude, then the codes.  Two segments in one
+// launch: the routed rows (rows0 x w0) and the shared experts' rows (rows1 x w1).
+__global__ void __launch_bounds__(256) k_quant_rows(const uint16_t* __restrict__ a0, int rows0, int w0,
+                                                    uint8_t* __restrict__ q0, int8_t* __restrict__ e0,
+                                                    const uint16_t* __restrict__ a1, int rows1, int w1,
+                                                    uint8_t* __restrict__ q1, int8_t* __restrict__ e1) {
+  griddep_wait();
+  griddep_launch();
+  const int r0 = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  const bool first = r0 < rows0;
+  if (!first && r0 >= rows0 + rows1) return;
+  const int r = first ? r0 : r0 - rows0;
+  const int w = first ? w0 : w1;
+  const uint16_t* ar = (first ? a0 : a1) + static_cast<size_t>(r) * w;
+  uint8_t* qr = (first ? q0 : q1) + static_cast<size_t>(r) * w;
+  float amax = 0.f;
+  for (int c = lane; c < w / 8; c += 32) {
+    const f8 v = ld_bf16x8(ar + 8 * c);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) amax = fmaxf(amax, fabsf(v.v[q]));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  const int e = act_row_exp(amax);
+  const float inv_scale = exp2_int(-e);
+  for (int c = lane; c < w / 8; c += 32) {
+    const f8 v = ld_bf16x8(ar + 8 * c);
+    *reinterpret_cast<uint2*>(qr + 8 * c) = e4m3x8(v.v, inv_scale);
+  }
+  if (lane == 0) (first ? e0 : e1)[r] = static_cast<int8_t>(e);
 }
 
 // Shared tail of the two epilogues: r (kept in registers) -> out_residual,
@@ -338,11 +421,11 @@ __global__ void k_wait_selftest(volatile int* flag, int* err, unsigned long long
 
 cudaError_t launch_rmsnorm_rows(const uint16_t* x, const uint16_t* g, uint16_t* y, int T, int D,
                                 float eps, int* err_to_clear, int32_t* zero, int zero_words,
-                                cudaStream_t s) {
+                                uint8_t* yq, int8_t* yq_exp, cudaStream_t s) {
   if (T <= 0) return cudaSuccess;
   auto go = [&](auto kernel) {
     return launch_k(kernel, dim3(T), dim3(kRowThreads), 0, s, false, x, g, y, D, eps, err_to_clear,
-                    zero, zero_words);
+                    zero, zero_words, yq, yq_exp);
   };
   switch (chunks_for(D, 8)) {
     case 1: return go(k_rmsnorm_rows<1>);
@@ -351,6 +434,15 @@ cudaError_t launch_rmsnorm_rows(const uint16_t* x, const uint16_t* g, uint16_t* 
     case 8: return go(k_rmsnorm_rows<8>);
     default: return go(k_rmsnorm_rows<16>);
   }
+}
+
+cudaError_t launch_quant_rows(const uint16_t* a0, int rows0, int w0, uint8_t* q0, int8_t* e0,
+                              const uint16_t* a1, int rows1, int w1, uint8_t* q1, int8_t* e1,
+                              cudaStream_t s) {
+  const int rows = rows0 + rows1;
+  if (rows <= 0) return cudaSuccess;
+  return launch_k(k_quant_rows, dim3((rows + 7) / 8), dim3(256), 0, s, false, a0, rows0, w0, q0, e0, a1,
+                  rows1, w1, q1, e1);
 }
 
 cudaError_t launch_combine_norm(const float* y_slot, const float* topk_w, const float* y_shared,

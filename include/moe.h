@@ -84,6 +84,23 @@ typedef enum moe_activation {
                             MoE variants, "SiTU-GLU": 4 and 25); clamps unused    */
 } moe_activation;
 
+/* Format of the expert weights (DeepSeek V4 infra notes, §6.2 FP4 QAT: expert
+ * weights are FP4 (E2M1) with one scale per block, dequantised losslessly to
+ * FP8, and the experts run FP8 x FP8 GEMMs). */
+typedef enum moe_weight_format {
+  MOE_WEIGHTS_BF16 = 0,  /* bf16 weights, bf16 x bf16 GEMMs                          */
+  MOE_WEIGHTS_FP8 = 1    /* E4M3 bytes (as moe_quantize_weights_fp4 writes them),
+                            E4M3 x E4M3 GEMMs with fp32 accumulation.  Each expert
+                            GEMM's input rows are E4M3 with one power-of-two scale
+                            per row: e = the smallest integer with max|row| <=
+                            448 * 2^e (clamped to [-126, 126]; 0 for a zero row),
+                            code = E4M3 round-to-nearest-even of value / 2^e; the
+                            row's accumulators are multiplied by 2^e.  The gate/up
+                            input is xn (after its bf16 rounding), the down input
+                            is h.  The router GEMM stays bf16.  Needs D, I and
+                            I_shared multiples of 128 and latent == 0.              */
+} moe_weight_format;
+
 typedef struct moe_config {
   int D;               /* hidden size                                                  */
   int E;               /* routed experts                                               */
@@ -108,19 +125,21 @@ typedef struct moe_config {
                           cast to bf16 once and projected back by W_proj_up; shared
                           experts stay at width D (linux.do post on MoE variants,
                           "潜在MoE (Latent MoE)" and K3's Stable Latent MoE)          */
+  int weight_format;   /* moe_weight_format of the routed and shared expert weights     */
 } moe_config;
 
 typedef struct moe_weights {      /* device pointers, caller-owned; L = latent if
-                                     latent > 0, else D                               */
+                                     latent > 0, else D.  The six expert matrices are
+                                     bf16 or E4M3 bytes, as weight_format says.       */
   const moe_bf16* w_router;       /* [E, L]      (unused for hash routing)            */
   const float* router_bias;       /* [E] fp32 or NULL: logit bias (softmax) or
                                      selection bias (sigmoid)                         */
-  const moe_bf16* w_gate;         /* [E, I, L]                                        */
-  const moe_bf16* w_up;           /* [E, I, L]                                        */
-  const moe_bf16* w_down;         /* [E, L, I]                                        */
-  const moe_bf16* ws_gate;        /* [S, I_shared, D]  (NULL when n_shared == 0)      */
-  const moe_bf16* ws_up;          /* [S, I_shared, D]                                 */
-  const moe_bf16* ws_down;        /* [S, D, I_shared]                                 */
+  const void* w_gate;             /* [E, I, L]                                        */
+  const void* w_up;               /* [E, I, L]                                        */
+  const void* w_down;             /* [E, L, I]                                        */
+  const void* ws_gate;            /* [S, I_shared, D]  (NULL when n_shared == 0)      */
+  const void* ws_up;              /* [S, I_shared, D]                                 */
+  const void* ws_down;            /* [S, D, I_shared]                                 */
   const moe_bf16* g_in;           /* [D] input RMSNorm gain                           */
   const moe_bf16* g_out;          /* [D] output RMSNorm gain                          */
   const moe_bf16* w_proj_down;    /* [latent, D] latent down-projection (latent > 0)  */
@@ -135,8 +154,9 @@ typedef struct moe_handle moe_handle;
  * (scores, top-k, weights, per-128-token expert histogram), 3 dispatch (offsets
  * and stable scatter), 4 gather_rows, 5 gemm_gateup_swiglu, 6 gemm_down,
  * 7 combine_norm; with a latent width also 8 latent_down (launched before
- * stage 1), 9 latent_combine and 10 latent_up (both before stage 7). */
-#define MOE_NUM_STAGES 11
+ * stage 1), 9 latent_combine and 10 latent_up (both before stage 7); with
+ * MOE_WEIGHTS_FP8 also 11 quant_h (h to E4M3 rows, between stages 5 and 6). */
+#define MOE_NUM_STAGES 12
 
 /* Validate `cfg`, keep the weight pointers and build the weight TMA
  * descriptors on the current CUDA device.  Allocates one small handle-owned
@@ -235,6 +255,14 @@ typedef struct moe_views {
   const moe_bf16* z;           /* [T, latent]     latent input (NULL unless latent)  */
   const moe_bf16* agg;         /* [T, latent]     bf16 routed sum (NULL unless latent)*/
   const float* y_latent;       /* [T, D]          up-projected sum (NULL unless latent)*/
+  /* MOE_WEIGHTS_FP8 only (NULL otherwise): E4M3 expert inputs and the power-of-two
+   * exponent of each row (row value = code value * 2^exp).                      */
+  const uint8_t* xq;           /* [T, D]          xn as E4M3                          */
+  const int8_t* xq_exp;        /* [T]                                                 */
+  const uint8_t* hq_routed;    /* [T * k, I]      h_routed as E4M3, grouped order     */
+  const int8_t* hq_routed_exp; /* [T * k]                                             */
+  const uint8_t* hq_shared;    /* [S, T, I_shared]                                    */
+  const int8_t* hq_shared_exp; /* [S, T]                                              */
 } moe_views;
 
 int moe_workspace_views(const moe_handle* h, int T, void* workspace, moe_views* out);
@@ -283,6 +311,22 @@ int moe_layer_forward_noalloc(moe_handle* h, int T, const moe_bf16* x, const moe
                               const int32_t* token_ids, moe_bf16* out_norm,
                               moe_bf16* out_residual, int32_t* out_topk_idx, float* out_topk_w,
                               int32_t* out_counts, void* stream);
+
+/* FP4 weight quantisation (DeepSeek V4 infra notes, §6.2 FP4 QAT: master
+ * weights -> FP4 (E2M1) with a scale per block -> lossless FP8).  `w` is a
+ * row-major [rows, K] bf16 matrix (the master weights), K a multiple of 32,
+ * the contraction axis of the GEMM that will read it.  Every block of 32
+ * consecutive elements of a row gets the power-of-two scale 2^s with s the
+ * smallest integer such that max|block| <= 6 * 2^s, clamped to [-8, 6] (-8 for
+ * an all-zero block); each element becomes q = the E2M1 value (0, 0.5, 1, 1.5,
+ * 2, 3, 4, 6, signed) nearest to w / 2^s, ties to the even code, and
+ * w8[i] = the E4M3 code of q * 2^s, which that range of s keeps exact.
+ * block_exp (NULL allowed) receives s, [rows, K / 32] int8.  Pointers are
+ * device memory the caller owns; w and w8 16-byte aligned.  Asynchronous on
+ * `stream`.  Errors: MOE_EINVAL (NULL, misaligned, rows < 0, K not a positive
+ * multiple of 32), MOE_ECUDA (launch). */
+int moe_quantize_weights_fp4(const moe_bf16* w, uint8_t* w8, int8_t* block_exp, long long rows, int K,
+                             void* stream);
 
 /* ------------------------------------------------------------------------
  * Peer memory for the tensor-parallel epilogue (one process per GPU).

@@ -567,6 +567,30 @@ class Weights:
         return self.ws_gate[s], self.ws_up[s], self.ws_down[s]
 
 
+class FP4Weights:
+    """The weights of a layer with FP4 experts ([DS] §6.2): the master weights
+    ``master`` (any Weights-like object) with every expert matrix replaced, on
+    first use, by its FP8 values fp4_weights_as_fp8(w).  Router, gains and
+    projections are the master's."""
+
+    def __init__(self, master):
+        self._master = master
+        self._cache = {}
+        for n in ("w_router", "router_bias", "g_in", "g_out", "w_proj_down", "w_proj_up"):
+            setattr(self, n, getattr(master, n, None))
+
+    def _q(self, key, mats):
+        if key not in self._cache:
+            self._cache[key] = tuple(fp4_weights_as_fp8(m) for m in mats)
+        return self._cache[key]
+
+    def routed(self, e):
+        return self._q(("r", int(e)), self._master.routed(e))
+
+    def shared(self, s):
+        return self._q(("s", int(s)), self._master.shared(s))
+
+
 def moe_layer(cfg, W, x, residual, token_ids=None, rows=None) -> dict:
     """The whole layer.  Routing, histogram and permutation are computed for
     every token; the experts, combine and epilogue for ``rows`` (all tokens

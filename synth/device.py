@@ -39,7 +39,7 @@ def layer_config(cfg, T_max=None):
                            gate_clamp_max=cfg.gate_clamp_max, up_clamp=cfg.up_clamp, eps=cfg.eps,
                            hash_mult=cfg.hash_mult, activation=cfg.activation,
                            situ_beta_gate=cfg.situ_beta_gate, situ_beta_up=cfg.situ_beta_up,
-                           latent=cfg.latent)
+                           latent=cfg.latent, weight_format=cfg.weight_format)
 
 
 def device_weights(cfg, device="cuda", stream=None) -> dict:

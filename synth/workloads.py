@@ -61,6 +61,7 @@ class MoEConfig:
     situ_beta_gate: float = 4.0
     situ_beta_up: float = 25.0
     latent: int = 0                 # latent MoE width (0: none)
+    weight_format: int = 0          # 0 bf16 experts, 1 FP4-valued experts stored as E4M3
 
     def with_T(self, T: int) -> "MoEConfig":
         return dataclasses.replace(self, T=T)
@@ -93,13 +94,18 @@ C2S = dataclasses.replace(C2, name="fine_grained_situ", activation=1)
 # The post gives no sizes; these are the fine-grained shapes with l = D / 4.
 C6 = MoEConfig("latent_situ", T=4096, D=2048, E=256, k=16, I=512, n_shared=1, I_shared=2048,
                renormalize=1, activation=1, latent=512)
+# FP4 expert weights with FP8 x FP8 expert GEMMs (the DeepSeek V4 infra notes,
+# §6.2 FP4 QAT) on the tiny and fine-grained shapes; the master weights are the
+# bf16 weights of those workloads.
+C1F = dataclasses.replace(C1, name="tiny_fp8", weight_format=1)
+C2F = dataclasses.replace(C2, name="fine_grained_fp8", weight_format=1)
 # The 8-partial fixed-order reduce + residual + RMSNorm epilogue of that workload.
 EPILOGUE_P = 8
 EPILOGUE_T = 16384
 EPILOGUE_D = 4096
 EPILOGUE_SIGMA = 1.0 / 8.0
 
-CONFIGS = {c.name: c for c in (C1, C2, C3, C5, C5H, C2S, C6)}
+CONFIGS = {c.name: c for c in (C1, C2, C3, C5, C5H, C2S, C6, C1F, C2F)}
 
 _ZIPF_FILE = os.path.join(os.path.dirname(os.path.abspath(__file__)), "zipf_beta.json")
 ZIPF_S = 1.2
@@ -215,14 +221,19 @@ def moe_flops(cfg: MoEConfig, T: int | None = None) -> dict:
             "total": routed + shared + router + proj, "gateup": gateup, "down": routed + shared - gateup}
 
 
+def weight_elem_bytes(cfg: MoEConfig) -> int:
+    """Bytes per expert weight element as the GEMMs read them (bf16 or E4M3)."""
+    return 1 if cfg.weight_format else 2
+
+
 def expert_bytes(cfg: MoEConfig) -> int:
-    return 3 * (cfg.latent or cfg.D) * cfg.I * 2
+    return 3 * (cfg.latent or cfg.D) * cfg.I * weight_elem_bytes(cfg)
 
 
 def layer_bytes(cfg: MoEConfig, T: int, distinct_experts: int) -> int:
     """Algorithmic HBM bytes: the touched routed experts, shared and router
     weights, x and residual in, two bf16 outputs."""
-    w = distinct_experts * expert_bytes(cfg) + cfg.n_shared * 3 * cfg.D * cfg.I_shared * 2
+    w = distinct_experts * expert_bytes(cfg) + cfg.n_shared * 3 * cfg.D * cfg.I_shared * weight_elem_bytes(cfg)
     if cfg.router != ROUTER_HASH:
         w += cfg.E * (cfg.latent or cfg.D) * 2
     w += 2 * cfg.D * cfg.latent * 2   # latent projections
@@ -234,9 +245,11 @@ def pretty(cfg: MoEConfig) -> str:
     r = {0: "softmax", 1: "sigmoid+bias", 2: "hash"}[cfg.router]
     act = "" if cfg.activation == 0 else f" SiTU-GLU({cfg.situ_beta_gate:g},{cfg.situ_beta_up:g})"
     lat = f" latent={cfg.latent}" if cfg.latent else ""
+    if cfg.weight_format:
+        act += " FP4 weights (E4M3 x E4M3 GEMMs)"
     return (f"{cfg.name}: T={cfg.T} D={cfg.D}{lat} E={cfg.E} top-{cfg.k} {r} I={cfg.I} "
             f"shared={cfg.n_shared}x{cfg.I_shared}{act}")
 
 
-__all__ = ["MoEConfig", "C1", "C2", "C2S", "C3", "C4_T", "C5", "C5H", "C6", "CONFIGS", "STREAM", "SEED",
+__all__ = ["MoEConfig", "C1", "C1F", "C2", "C2F", "C2S", "C3", "C4_T", "C5", "C5H", "C6", "CONFIGS", "STREAM", "SEED",
            "host_bf16", "host_router_bias", "host_token_ids", "moe_flops", "math"]

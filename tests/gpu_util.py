@@ -27,7 +27,12 @@ class Run:
         self.cfg = cfg
         self.T = cfg.T if T is None else T
         self.T_max = T_max or max(self.T, 1)
-        self.w = weights if weights is not None else SD.device_weights(cfg, device=device)
+        if weights is None:
+            weights = SD.device_weights(cfg, device=device)
+            if cfg.weight_format:
+                # FP4 expert weights: the library's own quantiser writes their E4M3 codes.
+                weights = moe.quantize_expert_weights(weights)
+        self.w = weights
         self.layer = moe.MoELayer(layer_config(cfg, self.T_max), self.w)
         self.device = device
 
@@ -120,10 +125,15 @@ def cfg_k(ref):
     return ref["idx"].shape[1]
 
 
+def host_weights(cfg):
+    hw = SD.HostWeights(cfg)
+    return O.FP4Weights(hw) if cfg.weight_format else hw
+
+
 def oracle_full(cfg, T=None, rows=None):
     """Oracle on the workload's inputs (all T rows routed; experts for ``rows``)."""
     T = cfg.T if T is None else T
-    hw = SD.HostWeights(cfg)
+    hw = host_weights(cfg)
     x = SD.host_rows(cfg, "x", range(T), T=T)
     r = SD.host_rows(cfg, "residual", range(T), T=T)
     ids = W.host_token_ids(cfg, T)

@@ -26,7 +26,8 @@ def torch_cuda():
 
 
 @pytest.mark.parametrize("name,splits", [("tiny", 7), ("fine_grained", 4), ("skew_hash", 3),
-                                         ("fine_grained_situ", 5), ("latent_situ", 4)])
+                                         ("fine_grained_situ", 5), ("latent_situ", 4),
+                                         ("tiny_fp8", 6), ("fine_grained_fp8", 4)])
 def test_splits_permutation_repeats(torch_cuda, name, splits):
     torch = torch_cuda
     cfg = W.CONFIGS[name]
@@ -67,3 +68,19 @@ def test_repeat_runs_same_bits_v3_shape_small(torch_cuda):
     ws = torch.empty(run.layer.invariance_workspace_size(cfg.T), dtype=torch.uint8, device="cuda")
     perm = torch.from_numpy(W.token_permutation(cfg.T, salt=3).astype(np.int32)).cuda()
     assert run.layer.check_invariance(x, r, ws, token_ids=ids, n_splits=5, perm=perm, repeats=1) == 0
+
+
+def test_fp8_decode_sweep_matches_full_batch(torch_cuda):
+    """FP4 expert weights: every decode batch reproduces its rows of the
+    8192-row run bit for bit (the per-row E4M3 scales are row-local)."""
+    torch = torch_cuda
+    cfg = W.C2F.with_T(W.C4_SOURCE_T)
+    run = Run(cfg, T_max=W.C4_SOURCE_T)
+    x, r, ids = run.inputs()
+    full = run.forward(x, r, ids)
+    for T in W.C4_T:
+        rows = W.decode_subset(T)
+        ri = torch.from_numpy(rows).cuda()
+        out = run.forward(x[ri].contiguous(), r[ri].contiguous(), ids[ri].contiguous())
+        for key in ("out_norm", "out_residual"):
+            assert torch.equal(out[key].view(torch.int16), full[key][ri].view(torch.int16)), (T, key)
