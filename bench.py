@@ -45,7 +45,7 @@ sys.path.insert(0, ROOT)
 METRIC = "MoE layer tokens/sec at 1 B200; % bf16 TC peak (prefill) / % HBM BW (decode)"
 UNIT = "tokens/s"
 GATEUP_STAGE = 5
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic_gemm_gateup_swiglu_fine_grained.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic_gemm_gateup.json")
 GEMM_SOURCES = [os.path.join(ROOT, "deterministic_expert_b200", "csrc", n)
                 for n in ("grouped_gemm.cu", "common.cuh", "moe_internal.h")]
 
@@ -104,9 +104,11 @@ def ncu_traffic(cfg):
         return None
     with open(TRAFFIC_FILE) as f:
         d = json.load(f)
-    if d.get("source_sha256") != gemm_source_hash() or d.get("T") != cfg.T or d.get("workload") != cfg.name:
-        return None
-    return d.get("dram_bytes_per_launch")
+    sha = gemm_source_hash()
+    for e in d.get("entries", []):
+        if e.get("source_sha256") == sha and e.get("T") == cfg.T and e.get("workload") == cfg.name:
+            return e.get("dram_bytes_per_launch")
+    return None
 
 
 # ------------------------------------------------------------------ clocks
