@@ -51,6 +51,7 @@ namespace moe {
 namespace {
 
 constexpr uint32_t kTmemCols = 512;
+constexpr int kMaxGroups = 256 + 8;   // routed experts + shared experts (checked by moe_init)
 constexpr int kRingBytes = kStages * (kSmemA + kSmemBMax);  // shared memory of the stage ring
 constexpr int kRingMax = 12;                                // most stages any variant uses
 constexpr int kBarBytes = 512;                              // mbarrier region after the ring
@@ -76,8 +77,11 @@ struct Tile {
   int nt;
 };
 
+// tile_start lives in shared memory (copied once per CTA), so the search costs
+// a few shared-memory reads instead of a chain of dependent global loads at
+// every tile boundary.
 template <int CG>
-__device__ __forceinline__ void decode_tile(const GemmArgs& a, int t, Tile& ti) {
+__device__ __forceinline__ void decode_tile(const GemmArgs& a, const int* tile_start, int t, Tile& ti) {
   int local = t;
   if (a.tile_start == nullptr) {
     // One dense group of T rows (router, latent projections) of kind dense_kind.
@@ -87,9 +91,9 @@ __device__ __forceinline__ void decode_tile(const GemmArgs& a, int t, Tile& ti) 
   int lo = 0, hi = a.G;
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
-    if (a.tile_start[mid] <= t) lo = mid; else hi = mid;
+    if (tile_start[mid] <= t) lo = mid; else hi = mid;
   }
-  local = t - a.tile_start[lo];
+  local = t - tile_start[lo];
   if (lo < a.E) {
     const int o0 = a.offsets[lo];
     ti.kind = 0; ti.idx = lo; ti.rows = a.offsets[lo + 1] - o0; ti.a_row0 = o0;
@@ -179,6 +183,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
   uint8_t* epi = reinterpret_cast<uint8_t*>(bars) + kBarBytes;  // kEpiWarps x kEpiBytes
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
+  __shared__ int s_tile_start[kMaxGroups + 1];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = CG == 2 ? cluster_ctarank() : 0;   // 0 = the MMA-issuing CTA
@@ -204,9 +209,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
   // of the stream before reading the tile list or any operand.
   griddep_wait();
   griddep_launch();
+  if (a.tile_start != nullptr)
+    for (int i = threadIdx.x; i <= a.G; i += blockDim.x) s_tile_start[i] = a.tile_start[i];
+  __syncthreads();
 
   const int cluster_id = blockIdx.x / CG, n_clusters = gridDim.x / CG;
-  const int total = (a.tile_start == nullptr) ? a.router_tiles : a.tile_start[a.G];
+  const int total = (a.tile_start == nullptr) ? a.router_tiles : s_tile_start[a.G];
   const int BN = a.BN;                                    // output columns per tile (per matrix)
   const int n_mma = MODE == kGateUp ? 2 * BN : BN;        // N of one MMA
   // B rows each CTA loads per stage, per matrix (gate and up each for gate/up).
@@ -227,7 +235,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
       bool ok = true;
       for (int t = cluster_id; ok && t < total; t += n_clusters) {
         Tile ti;
-        decode_tile<CG>(a, t, ti);
+        decode_tile<CG>(a, s_tile_start, t, ti);
         const int nkb = a.k_kind[ti.kind] / KE;
         // A: this CTA's rows of the tile (128, or 64 in a 128-row pair tile,
         // loaded with the 64-row box so no unused rows cross into shared memory).
@@ -291,7 +299,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
       bool ok = true;
       for (int t = cluster_id; ok && t < total; t += n_clusters) {
         Tile ti;
-        decode_tile<CG>(a, t, ti);
+        decode_tile<CG>(a, s_tile_start, t, ti);
         const int nkb = a.k_kind[ti.kind] / KE;
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort, a.err, a.timeout_ns)) break;
         tc_fence_after();
@@ -354,7 +362,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
     uint32_t xph = 0;  // phase of this warp's exchange channel (swapped gate/up tiles)
     for (int t = cluster_id; t < total; t += n_clusters) {
       Tile ti;
-      decode_tile<CG>(a, t, ti);
+      decode_tile<CG>(a, s_tile_start, t, ti);
       bool ok = mbar_wait(&tfull[acc], acc_phase, abort, a.err, a.timeout_ns);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
