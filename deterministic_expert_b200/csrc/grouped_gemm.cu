@@ -178,8 +178,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
   uint64_t* tfull = bars + 2 * kRingMax;
   uint64_t* tempty = tfull + 2;
   uint64_t* tdone = tempty + 2;
-  uint64_t* xfull = tdone + 1;   // [4] swapped gate/up tiles: up values staged for the gate warp
-  uint64_t* xempty = xfull + 4;  // [4] ... and read back
+  // Swapped gate/up tiles: per warp pair, up values staged for the gate warp
+  // (xfull / xempty) and gate values staged for the up warp (gfull / gempty).
+  uint64_t* xfull = tdone + 1;   // [4]
+  uint64_t* xempty = xfull + 4;  // [4]
+  uint64_t* gfull = xempty + 4;  // [4]
+  uint64_t* gempty = gfull + 4;  // [4]
   uint8_t* epi = reinterpret_cast<uint8_t*>(bars) + kBarBytes;  // kEpiWarps x kEpiBytes
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
@@ -192,7 +196,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
     for (int s = 0; s < S; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
     for (int b = 0; b < 2; ++b) { mbar_init(&tfull[b], 1); mbar_init(&tempty[b], CG * kEpiWarps); }
     mbar_init(tdone, 1);
-    for (int p = 0; p < 4; ++p) { mbar_init(&xfull[p], 1); mbar_init(&xempty[p], 1); }
+    for (int p = 0; p < 4; ++p) {
+      mbar_init(&xfull[p], 1); mbar_init(&xempty[p], 1);
+      mbar_init(&gfull[p], 1); mbar_init(&gempty[p], 1);
+    }
     abort_flag = 0;
     fence_barrier_init();
   }
@@ -375,13 +382,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
         const int trow0 = ti.m * C::kTileM;
         if (MODE == kGateUp) {
           // Lanes 0-63 hold the gate rows and lanes 64-127 the up rows of the CTA's
-          // 64 output columns; TMEM columns are tokens.  The up warp of each lane
-          // quarter pair stages its values in its buffer (4-byte word j of lane l
-          // at l * 32 + (j ^ l): conflict-free both ways) and the gate warp of the
-          // same columns reads them, both under bounded mbarrier waits.
+          // 64 output columns; TMEM columns are tokens.  A gate warp (lane quarter
+          // 0 or 1) and the up warp of the same columns (quarter 2 or 3) split
+          // each 32-token block: the gate warp computes tokens 0-15 and the up
+          // warp tokens 16-31, each receiving the other branch's values for its
+          // half through shared memory (word j of lane l at j * 32 + l: lane l
+          // of both warps is the same column, so both sides are conflict-free),
+          // every hand-over under bounded mbarrier waits.  Both warps' SMSPs do
+          // half of the unit's arithmetic.
           const bool gate_warp = q < 2;
           const int pch = (q & 1) + 2 * half;  // exchange channel of this warp pair
-          uint32_t* xbuf = reinterpret_cast<uint32_t*>(gate_warp ? stage_w - 2 * kEpiBytes : stage_w);
+          uint32_t* sendb = reinterpret_cast<uint32_t*>(stage_w);   // this warp's buffer
+          uint32_t* recvb = reinterpret_cast<uint32_t*>(gate_warp ? stage_w - 2 * kEpiBytes
+                                                                  : stage_w + 2 * kEpiBytes);
+          uint64_t* my_full = gate_warp ? &gfull[pch] : &xfull[pch];
+          uint64_t* my_empty = gate_warp ? &gempty[pch] : &xempty[pch];
+          uint64_t* their_full = gate_warp ? &xfull[pch] : &gfull[pch];
+          uint64_t* their_empty = gate_warp ? &xempty[pch] : &gempty[pch];
+          const int base = gate_warp ? 0 : 16;  // first token of this warp's half
           const int col = ti.n * BN + static_cast<int>(rank) * (BN / 2) + 32 * (q & 1) + lane;
           uint16_t* outb = static_cast<uint16_t*>(a.out[ti.kind]);
           const size_t ld = static_cast<size_t>(a.ld_out[ti.kind]);
@@ -390,42 +408,50 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
             uint32_t v[32];
             tmem_ld32(tb + c, v);
             tmem_ld_wait();
-            if (!gate_warp) {
-              ok = mbar_wait(&xempty[pch], xph ^ 1u, abort, a.err, a.timeout_ns);
-              if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+            ok = mbar_wait(my_empty, xph ^ 1u, abort, a.err, a.timeout_ns);
+            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+            // Hand over the partner's half: the gate warp sends tokens 16-31,
+            // the up warp tokens 0-15.
+            if (gate_warp) {
 #pragma unroll
-              for (int j = 0; j < 32; ++j) xbuf[lane * 32 + (j ^ lane)] = v[j];
-              __syncwarp();
-              if (lane == 0) mbar_arrive(&xfull[pch]);
+              for (int jj = 0; jj < 16; ++jj) sendb[jj * 32 + lane] = v[16 + jj];
             } else {
-              ok = mbar_wait(&xfull[pch], xph, abort, a.err, a.timeout_ns);
-              if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-              uint32_t u[32];
 #pragma unroll
-              for (int j = 0; j < 32; ++j) u[j] = xbuf[lane * 32 + (j ^ lane)];
-              __syncwarp();
-              if (lane == 0) mbar_arrive(&xempty[pch]);
-              // fp8: token c + lane's row scale, handed to every lane per token.
-              float my_sc = 1.f;
-              if (F8 && c + lane < r) my_sc = exp2_int(a.a_exp[ti.kind][ti.a_row0 + trow0 + c + lane]);
+              for (int jj = 0; jj < 16; ++jj) sendb[jj * 32 + lane] = v[jj];
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(my_full);
+            ok = mbar_wait(their_full, xph, abort, a.err, a.timeout_ns);
+            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+            uint32_t o[16];
 #pragma unroll
-              for (int j = 0; j < 32; ++j) {
-                const float sc = F8 ? __shfl_sync(0xffffffffu, my_sc, j) : 1.f;
-                if (c + j < r) {
-                  float gv = __uint_as_float(v[j]), uv = __uint_as_float(u[j]);
-                  if (F8) { gv = __fmul_rn(gv, sc); uv = __fmul_rn(uv, sc); }
-                  const float hv = glu_unit<ACT>(gv, uv, a);
-                  outb[static_cast<size_t>(orow0 + c + j) * ld + col] =
-                      static_cast<uint16_t>(pack_bf16x2(hv, 0.f) & 0xFFFFu);
-                }
+            for (int jj = 0; jj < 16; ++jj) o[jj] = recvb[jj * 32 + lane];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(their_empty);
+            // fp8: token c + lane's row scale, handed to every lane per token.
+            float my_sc = 1.f;
+            if (F8 && c + lane < r) my_sc = exp2_int(a.a_exp[ti.kind][ti.a_row0 + trow0 + c + lane]);
+#pragma unroll
+            for (int jj = 0; jj < 16; ++jj) {
+              const int j = base + jj;
+              const float sc = F8 ? __shfl_sync(0xffffffffu, my_sc, j) : 1.f;
+              // Gate warp: own gate values v[jj], received up values o[jj];
+              // up warp: received gate values o[jj], own up values v[16 + jj].
+              float gv = __uint_as_float(gate_warp ? v[jj] : o[jj]);
+              float uv = __uint_as_float(gate_warp ? o[jj] : v[16 + jj]);
+              if (c + j < r) {
+                if (F8) { gv = __fmul_rn(gv, sc); uv = __fmul_rn(uv, sc); }
+                const float hv = glu_unit<ACT>(gv, uv, a);
+                outb[static_cast<size_t>(orow0 + c + j) * ld + col] =
+                    static_cast<uint16_t>(pack_bf16x2(hv, 0.f) & 0xFFFFu);
               }
             }
             xph ^= 1u;
           }
-          // The up warp's buffer is its own staging area in row tiles: do not
-          // leave the tile before the gate warp has read the last block.
-          if (!gate_warp && ok) {
-            ok = mbar_wait(&xempty[pch], xph ^ 1u, abort, a.err, a.timeout_ns);
+          // Each warp's buffer is its own staging area in row tiles: do not
+          // leave the tile before the partner has read the last block from it.
+          if (ok) {
+            ok = mbar_wait(my_empty, xph ^ 1u, abort, a.err, a.timeout_ns);
             ok = __all_sync(0xffffffffu, ok);
           }
         } else {
