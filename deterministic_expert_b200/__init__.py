@@ -42,7 +42,8 @@ class moe_config(ctypes.Structure):
                 ("routed_scale", ctypes.c_float), ("gate_clamp_max", ctypes.c_float),
                 ("up_clamp", ctypes.c_float), ("eps", ctypes.c_float), ("hash_mult", ctypes.c_uint32),
                 ("activation", ctypes.c_int), ("situ_beta_gate", ctypes.c_float),
-                ("situ_beta_up", ctypes.c_float), ("latent", ctypes.c_int), ("weight_format", ctypes.c_int)]
+                ("situ_beta_up", ctypes.c_float), ("latent", ctypes.c_int), ("weight_format", ctypes.c_int),
+                ("ep_world", ctypes.c_int), ("ep_rank", ctypes.c_int)]
 
 
 class moe_weights(ctypes.Structure):
@@ -137,13 +138,15 @@ class LayerConfig:
     situ_beta_up: float = 25.0
     latent: int = 0
     weight_format: int = WEIGHTS_BF16
+    ep_world: int = 0
+    ep_rank: int = 0
 
     def to_c(self) -> moe_config:
         return moe_config(self.D, self.E, self.k, self.I, self.n_shared,
                           self.I_shared if self.n_shared else self.I, self.T_max, self.router,
                           self.renormalize, self.routed_scale, self.gate_clamp_max, self.up_clamp,
                           self.eps, self.hash_mult, self.activation, self.situ_beta_gate,
-                          self.situ_beta_up, self.latent, self.weight_format)
+                          self.situ_beta_up, self.latent, self.weight_format, self.ep_world, self.ep_rank)
 
 
 def _check_weight_sizes(cfg: LayerConfig, weights: dict) -> None:
@@ -151,8 +154,9 @@ def _check_weight_sizes(cfg: LayerConfig, weights: dict) -> None:
     configuration, so a tensor of another size must be refused here."""
     L = cfg.latent or cfg.D
     S, Is = cfg.n_shared, (cfg.I_shared if cfg.n_shared else cfg.I)
-    want = {"w_router": cfg.E * L, "router_bias": cfg.E, "w_gate": cfg.E * cfg.I * L,
-            "w_up": cfg.E * cfg.I * L, "w_down": cfg.E * L * cfg.I, "ws_gate": S * Is * cfg.D,
+    El = cfg.E // cfg.ep_world if cfg.ep_world > 1 else cfg.E   # routed experts held here
+    want = {"w_router": cfg.E * L, "router_bias": cfg.E, "w_gate": El * cfg.I * L,
+            "w_up": El * cfg.I * L, "w_down": El * L * cfg.I, "ws_gate": S * Is * cfg.D,
             "ws_up": S * Is * cfg.D, "ws_down": S * cfg.D * Is, "g_in": cfg.D, "g_out": cfg.D,
             "w_proj_down": cfg.latent * cfg.D, "w_proj_up": cfg.D * cfg.latent}
     for name, n in want.items():
@@ -501,6 +505,218 @@ class TPAllReduceNorm:
 
     def close(self) -> None:
         """Collective: unmap the peers' memory, then free this rank's."""
+        import torch
+        import torch.distributed as dist
+        if self._closed:
+            return
+        torch.cuda.synchronize()
+        dist.barrier(group=self.group)
+        for a in self._opened:
+            peer_close(a)
+        dist.barrier(group=self.group)
+        peer_free(self._base)
+        self._closed = True
+
+
+# ------------------------------------------------------------ expert parallelism
+class moe_ep_peers(ctypes.Structure):
+    _fields_ = [("xbuf", ctypes.c_void_p * 8)]
+
+
+def expert_range(E: int, world: int, rank: int):
+    """Routed experts [e0, e1) held by ``rank`` of ``world`` (contiguous blocks)."""
+    if world < 1 or E % world:
+        raise ValueError("the expert count must divide evenly over the ranks")
+    n = E // world
+    return rank * n, (rank + 1) * n
+
+
+def shard_expert_weights(weights: dict, world: int, rank: int) -> dict:
+    """The moe_weights dict of one expert-parallel rank: its block of routed
+    experts (views of the full tensors, first axis = expert), everything else
+    whole."""
+    out = dict(weights)
+    for n in ("w_gate", "w_up", "w_down"):
+        t = weights[n]
+        e0, e1 = expert_range(int(t.shape[0]), world, rank)
+        out[n] = t[e0:e1]
+    return out
+
+
+def _ep_call(name, *args):
+    L = lib()
+    fn = getattr(L, name)
+    _check(fn(*args), name)
+
+
+class _EPRank:
+    """One expert-parallel rank: its handle, workspace and exchange buffer."""
+
+    def __init__(self, cfg: LayerConfig, weights: dict, rank: int, world: int, device):
+        import dataclasses
+
+        import torch
+        self.rank = rank
+        self.cfg = dataclasses.replace(cfg, ep_world=world, ep_rank=rank)
+        self.layer = MoELayer(self.cfg, shard_expert_weights(weights, world, rank))
+        L = lib()
+        L.moe_ep_exchange_size.restype = ctypes.c_size_t
+        L.moe_ep_exchange_size.argtypes = [ctypes.c_void_p]
+        self.xbytes = int(L.moe_ep_exchange_size(self.layer.handle))
+        self.ws = torch.empty(max(self.layer.workspace_size(cfg.T_max), 256), dtype=torch.uint8, device=device)
+        self.device = device
+
+    def route(self, x, token_ids, xbuf, stream=None):
+        L = lib()
+        L.moe_ep_route.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
+                                   ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
+        _check(L.moe_ep_route(self.layer.handle, int(x.shape[0]), _ptr(x), _ptr(token_ids), xbuf,
+                              _ptr(self.ws), self.ws.numel(), _stream(stream)), "moe_ep_route")
+
+    def send(self, T, peers, stream=None):
+        L = lib()
+        L.moe_ep_send.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.POINTER(moe_ep_peers), ctypes.c_void_p,
+                                  ctypes.c_size_t, ctypes.c_void_p]
+        _check(L.moe_ep_send(self.layer.handle, T, ctypes.byref(peers), _ptr(self.ws), self.ws.numel(),
+                             _stream(stream)), "moe_ep_send")
+
+    def experts(self, T, peers, stream=None):
+        L = lib()
+        L.moe_ep_experts.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.POINTER(moe_ep_peers), ctypes.c_void_p,
+                                     ctypes.c_size_t, ctypes.c_void_p]
+        _check(L.moe_ep_experts(self.layer.handle, T, ctypes.byref(peers), _ptr(self.ws), self.ws.numel(),
+                                _stream(stream)), "moe_ep_experts")
+
+    def combine(self, residual, xbuf, out_norm, out_residual, out_idx=None, out_w=None, stream=None):
+        L = lib()
+        vp = ctypes.c_void_p
+        L.moe_ep_combine.argtypes = [vp, ctypes.c_int, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
+        _check(L.moe_ep_combine(self.layer.handle, int(residual.shape[0]), _ptr(residual), xbuf, _ptr(out_norm),
+                                _ptr(out_residual), _ptr(out_idx), _ptr(out_w), _ptr(self.ws), self.ws.numel(),
+                                _stream(stream)), "moe_ep_combine")
+
+    def device_error(self, stream=None) -> int:
+        return self.layer.device_error(self.ws, stream)
+
+
+class VirtualEP:
+    """``world`` expert-parallel ranks sharing one device and one stream: each
+    rank has its own handle (its block of routed experts), workspace and
+    exchange buffer, and a step runs every rank's route, then every rank's
+    send, experts and combine in stream order, so no kernel waits on another.
+    Each rank's outputs are bit for bit those of the single-device layer on
+    its tokens.  ``weights`` holds all E routed experts."""
+
+    def __init__(self, cfg: LayerConfig, weights: dict, world: int, device="cuda"):
+        import torch
+        if world < 2 or world > 8:
+            raise ValueError("2 .. 8 ranks")
+        self.world = world
+        self.ranks = [_EPRank(cfg, weights, r, world, device) for r in range(world)]
+        self.xbuf = [torch.zeros(max(rk.xbytes, 256), dtype=torch.uint8, device=device) for rk in self.ranks]
+        self.peers = moe_ep_peers()
+        for r in range(world):
+            self.peers.xbuf[r] = _ptr(self.xbuf[r])
+
+    def forward(self, xs, residuals, token_ids=None, stream=None):
+        """xs, residuals: one [T_r, D] bf16 tensor per rank; returns per rank
+        (out_norm, out_residual, topk_idx, topk_w)."""
+        import torch
+        ids = token_ids if token_ids is not None else [None] * self.world
+        for r, rk in enumerate(self.ranks):
+            rk.route(xs[r], ids[r], _ptr(self.xbuf[r]), stream)
+        for r, rk in enumerate(self.ranks):
+            rk.send(int(xs[r].shape[0]), self.peers, stream)
+        for r, rk in enumerate(self.ranks):
+            rk.experts(int(xs[r].shape[0]), self.peers, stream)
+        outs = []
+        for r, rk in enumerate(self.ranks):
+            T = int(xs[r].shape[0])
+            k = rk.cfg.k
+            on = torch.empty_like(residuals[r])
+            orr = torch.empty_like(residuals[r])
+            idx = torch.empty((T, k), dtype=torch.int32, device=on.device)
+            w = torch.empty((T, k), dtype=torch.float32, device=on.device)
+            rk.combine(residuals[r], _ptr(self.xbuf[r]), on, orr, idx, w, stream)
+            outs.append((on, orr, idx, w))
+        return outs
+
+    def device_errors(self):
+        return [rk.device_error() for rk in self.ranks]
+
+
+class EPMoELayer:
+    """Expert parallelism across processes, one GPU each (torch.distributed
+    group of ``world`` ranks): this rank's handle with its block of routed
+    experts, and one exported allocation holding its barrier flags and its
+    exchange buffer, mapped by every other rank (moe_peer_open; handles travel
+    over the process group).  A step is the four phases on the caller's
+    stream with a device barrier (bounded; ``check()`` reports a time-out)
+    after route, send and experts.  ``weights`` holds all E routed experts (only
+    this rank's block is kept).  ``close()`` (collective) releases the memory."""
+
+    _FLAGS = 4096
+
+    def __init__(self, cfg: LayerConfig, weights: dict, group=None, device=None, barrier_timeout_ms: int = 5000):
+        import torch
+        import torch.distributed as dist
+        self.group = group
+        self.world = dist.get_world_size(group)
+        self.rank = dist.get_rank(group)
+        dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+        self.me = _EPRank(cfg, weights, self.rank, self.world, dev)
+        self.limit_us = barrier_timeout_ms * 1000
+        with torch.cuda.device(dev):
+            self._base, handle = peer_alloc(self._FLAGS + self.me.xbytes)
+        info = [None] * self.world
+        dist.all_gather_object(info, (handle, self.me.xbytes), group=group)
+        if any(x[1] != self.me.xbytes for x in info):
+            raise ValueError("ranks disagree on the exchange buffer size (configurations differ)")
+        self._opened, self._closed = [], False
+        bases = []
+        with torch.cuda.device(dev):
+            for r in range(self.world):
+                if r == self.rank:
+                    bases.append(self._base)
+                else:
+                    bases.append(peer_open(info[r][0]))
+                    self._opened.append(bases[-1])
+        self._flags = bases
+        self.peers = moe_ep_peers()
+        for r in range(self.world):
+            self.peers.xbuf[r] = bases[r] + self._FLAGS
+        self.err = torch.zeros(1, dtype=torch.int32, device=dev)
+        self._epoch = 0
+
+    def _barrier(self, stream):
+        self._epoch += 1
+        peer_barrier(self._flags, self.rank, self._epoch, self.err, self.limit_us, stream)
+
+    def forward(self, x, residual, token_ids=None, stream=None):
+        import torch
+        T = int(x.shape[0])
+        mine = self.peers.xbuf[self.rank]
+        self.me.route(x, token_ids, mine, stream)
+        self._barrier(stream)          # every rank's counts are out
+        self.me.send(T, self.peers, stream)
+        self._barrier(stream)          # every row has reached its owner
+        self.me.experts(T, self.peers, stream)
+        self._barrier(stream)          # every result row is back home
+        on, orr = torch.empty_like(residual), torch.empty_like(residual)
+        idx = torch.empty((T, self.me.cfg.k), dtype=torch.int32, device=on.device)
+        w = torch.empty((T, self.me.cfg.k), dtype=torch.float32, device=on.device)
+        self.me.combine(residual, mine, on, orr, idx, w, stream)
+        return on, orr, idx, w
+
+    def check(self) -> None:
+        e = int(self.err.item())
+        self.err.zero_()
+        if e:
+            raise MoEError(MOE_ETIMEOUT, "EPMoELayer barrier")
+        if self.me.device_error() != MOE_OK:
+            raise MoEError(MOE_ETIMEOUT, "EPMoELayer device wait")
+
+    def close(self) -> None:
         import torch
         import torch.distributed as dist
         if self._closed:

@@ -479,11 +479,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
               const float sc = F8 ? __shfl_sync(0xffffffffu, my_sc, j) : 1.f;
               if (c + j < r) {
                 const float val = F8 ? __fmul_rn(__uint_as_float(v[j]), sc) : __uint_as_float(v[j]);
-                if (a.out_bf16)
+                if (a.out_bf16) {
                   outh[static_cast<size_t>(orow) * ld + col] =
                       static_cast<uint16_t>(pack_bf16x2(val, 0.f) & 0xFFFFu);
-                else
+                } else if (scatter && a.ep) {
+                  // Expert parallelism: the row lives in its source rank's buffer.
+                  a.out_rank[orow >> 24][static_cast<size_t>(orow & 0xFFFFFF) * ld + col] = val;
+                } else {
                   outb[static_cast<size_t>(orow) * ld + col] = val;
+                }
               }
             }
           }
@@ -600,15 +604,26 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
               const int drow = __shfl_sync(0xffffffffu, my_dest, r);
               if (r < nvalid) {
                 const uint4 val = *reinterpret_cast<const uint4*>(stage_w + r * 128 + ((sc ^ (r & 7)) << 4));
-                const size_t orow = scatter ? static_cast<size_t>(drow) : static_cast<size_t>(orow0 + r);
-                *reinterpret_cast<uint4*>(out0 + orow * ld + c + 4 * sc) = val;
+                float* ob = out0;
+                size_t orow = scatter ? static_cast<size_t>(drow) : static_cast<size_t>(orow0 + r);
+                if (scatter && a.ep) {
+                  // Expert parallelism: the row lives in its source rank's buffer.
+                  ob = a.out_rank[drow >> 24] + ti.n * BN + colhalf * (BN / 2);
+                  orow = static_cast<size_t>(drow & 0xFFFFFF);
+                }
+                *reinterpret_cast<uint4*>(ob + orow * ld + c + 4 * sc) = val;
               }
             }
             __syncwarp();
           } else if (lane < nvalid) {
             // Narrow tail (router with fewer than 32 columns left): direct stores.
-            const size_t orow = scatter ? static_cast<size_t>(my_dest) : static_cast<size_t>(orow0 + lane);
-            float4* dst = reinterpret_cast<float4*>(out0 + orow * ld + c);
+            float* ob = out0;
+            size_t orow = scatter ? static_cast<size_t>(my_dest) : static_cast<size_t>(orow0 + lane);
+            if (scatter && a.ep) {
+              ob = a.out_rank[my_dest >> 24] + ti.n * BN + colhalf * (BN / 2);
+              orow = static_cast<size_t>(my_dest & 0xFFFFFF);
+            }
+            float4* dst = reinterpret_cast<float4*>(ob + orow * ld + c);
             const int nq = (ncols - c) / 4;
 #pragma unroll
             for (int i = 0; i < 8; ++i)

@@ -20,6 +20,9 @@ struct moe_handle {
   int S = 0, G = 0, E_pad = 0, bn_gu = 0, bn_dn = 0, num_sms = 0, device = 0, max_pairs = 0;
   int L = 0;                          // width the router and routed experts read (latent or D)
   bool fp8 = false;                   // MOE_WEIGHTS_FP8: E4M3 expert GEMMs
+  int ep_world = 1, ep_rank = 0;      // expert parallelism (1: none)
+  int E_loc = 0;                      // routed experts held here (E / ep_world)
+  long long cap = 0;                  // rows a rank can receive: ep_world * T_max * k
   int bn_pd = 0, bn_pu = 0;           // N tiles of the latent down / up projections
   uint16_t* w_router_pad = nullptr;  // [E_pad, L], rows >= E zero
   CUtensorMap map_router, map_wg, map_wu, map_wd, map_wsg, map_wsu, map_wsd, map_pd, map_pu;
@@ -39,7 +42,8 @@ size_t align256(size_t b) { return (b + 255) & ~static_cast<size_t>(255); }
 
 struct Layout {
   size_t err, xn, logits, tidx, tw, bcount, counts, offsets, tiles_gu, tiles_dn, dest, src,
-      xp, h, hs, y, ys, z, agg, ylat, xq, xqe, xpe, hq, hqs, he, hse, total;
+      xp, h, hs, y, ys, z, agg, ylat, xq, xqe, xpe, hq, hqs, he, hse,
+      hr, hqr, her, epoff, eptg, eptd, eprows, total;   // hr..eprows: expert parallelism
 };
 
 Layout layout(const moe_handle* h, int T) {
@@ -62,10 +66,12 @@ Layout layout(const moe_handle* h, int T) {
   L.src = take(Tz * c.k * 4);
   const size_t Lw = static_cast<size_t>(h->L);
   const size_t eb = h->fp8 ? 1 : 2;   // bytes per element of the expert GEMMs' inputs
-  L.xp = take(Tz * c.k * Lw * eb);
-  L.h = take(Tz * c.k * c.I * 2);
+  const bool ep = h->ep_world > 1;    // routed rows live in the exchange buffers
+  const size_t rt = ep ? 0 : 1;
+  L.xp = take(rt * Tz * c.k * Lw * eb);
+  L.h = take(rt * Tz * c.k * c.I * 2);
   L.hs = take(static_cast<size_t>(h->S) * Tz * c.I_shared * 2);
-  L.y = take(Tz * c.k * Lw * 4);
+  L.y = take(rt * Tz * c.k * Lw * 4);
   L.ys = take(static_cast<size_t>(h->S) * Tz * c.D * 4);
   const bool lat = c.latent > 0;
   L.z = take(lat ? Tz * Lw * 2 : 0);
@@ -75,13 +81,43 @@ Layout layout(const moe_handle* h, int T) {
   const size_t f = h->fp8 ? 1 : 0;
   L.xq = take(f * Tz * c.D);
   L.xqe = take(f * Tz);
-  L.xpe = take(f * Tz * c.k);
-  L.hq = take(f * Tz * c.k * c.I);
+  L.xpe = take(rt * f * Tz * c.k);
+  L.hq = take(rt * f * Tz * c.k * c.I);
   L.hqs = take(f * static_cast<size_t>(h->S) * Tz * c.I_shared);
-  L.he = take(f * Tz * c.k);
+  L.he = take(rt * f * Tz * c.k);
   L.hse = take(f * static_cast<size_t>(h->S) * Tz);
+  // Expert parallelism: h of the received rows, the owner's plan.
+  const size_t cap = ep ? static_cast<size_t>(h->cap) : 0;
+  const size_t gl = static_cast<size_t>(h->E_loc + h->S + 1);
+  L.hr = take(cap * c.I * 2);
+  L.hqr = take(f * cap * c.I);
+  L.her = take(f * cap);
+  L.epoff = take(ep ? static_cast<size_t>(h->E_loc + 1) * 4 : 0);
+  L.eptg = take(ep ? gl * 4 : 0);
+  L.eptd = take(ep ? gl * 4 : 0);
+  L.eprows = take(ep ? 4 : 0);
   L.total = off;
   return L;
+}
+
+// Expert parallelism: the exchange buffer every rank exposes to the others.
+struct XLayout {
+  size_t board, recv, recv_exp, meta, y, total;
+};
+
+XLayout xlayout(const moe_handle* h) {
+  const moe_config& c = h->cfg;
+  const size_t cap = static_cast<size_t>(h->cap), rowb = static_cast<size_t>(h->L) * (h->fp8 ? 1 : 2);
+  XLayout X;
+  size_t off = 0;
+  auto take = [&](size_t bytes) { const size_t o = off; off += align256(bytes); return o; };
+  X.board = take(static_cast<size_t>(c.E) * 4);
+  X.recv = take(cap * rowb);
+  X.recv_exp = take(h->fp8 ? cap : 0);
+  X.meta = take(cap * 4);
+  X.y = take(static_cast<size_t>(c.T_max) * c.k * h->L * 4);
+  X.total = off;
+  return X;
 }
 
 struct InvLayout {
@@ -155,6 +191,11 @@ int validate_config(const moe_config* c, const moe_weights* w) {
     return MOE_EINVAL;
   if (c->D % 64 || c->I % 64 || (c->n_shared > 0 && c->I_shared % 64)) return MOE_EUNSUPPORTED;
   if (c->weight_format != MOE_WEIGHTS_BF16 && c->weight_format != MOE_WEIGHTS_FP8) return MOE_EINVAL;
+  if (c->ep_world < 0 || c->ep_world > 8 || c->ep_rank < 0 || (c->ep_world > 1 && c->ep_rank >= c->ep_world))
+    return MOE_EINVAL;
+  if (c->ep_world > 1 && (c->E % c->ep_world || c->latent > 0)) return MOE_EUNSUPPORTED;
+  if (c->ep_world > 1 && static_cast<long long>(c->ep_world) * c->T_max * c->k >= (1ll << 24))
+    return MOE_EUNSUPPORTED;   // return addresses keep the row in 24 bits
   if (c->weight_format == MOE_WEIGHTS_FP8 &&
       (c->D % 128 || c->I % 128 || (c->n_shared > 0 && c->I_shared % 128) || c->latent > 0))
     return MOE_EUNSUPPORTED;
@@ -224,10 +265,12 @@ int pair_grid(const moe_handle* h, int tiles_bound) {
   return 2 * std::max(1, std::min(h->max_pairs, tiles_bound));
 }
 
+// The layer forward.  front_only (expert parallelism): stop after the grouping
+// (stages 0-3), with the per-expert counts written to counts_dst.
 int forward_impl(moe_handle* h, int T, const uint16_t* x, const uint16_t* residual,
                  const int32_t* token_ids, uint16_t* out_norm, uint16_t* out_residual,
                  int32_t* out_idx, float* out_w, int32_t* out_counts, uint8_t* ws,
-                 cudaStream_t s) {
+                 cudaStream_t s, bool front_only = false, int32_t* counts_dst = nullptr) {
   const moe_config& c = h->cfg;
   const Layout L = layout(h, T);
   int* err = reinterpret_cast<int*>(ws + L.err);
@@ -340,7 +383,7 @@ int forward_impl(moe_handle* h, int T, const uint16_t* x, const uint16_t* residu
   DispatchArgs da;
   da.idx = tidx; da.T = T; da.k = c.k; da.E = c.E; da.S = h->S;
   da.block_counts = bcount; da.E4 = E4;
-  da.counts = reinterpret_cast<int32_t*>(ws + L.counts);
+  da.counts = counts_dst != nullptr ? counts_dst : reinterpret_cast<int32_t*>(ws + L.counts);
   da.offsets = offsets; da.user_counts = out_counts; da.tiles_gu = tiles_gu; da.tiles_dn = tiles_dn;
   da.gu_ntiles_routed = c.I / h->bn_gu;
   da.gu_ntiles_shared = h->S > 0 ? c.I_shared / h->bn_gu : 0;
@@ -351,6 +394,7 @@ int forward_impl(moe_handle* h, int T, const uint16_t* x, const uint16_t* residu
   prof.begin(3);
   MOE_TRY(launch_dispatch(da, s));
   prof.end(3);
+  if (front_only) return MOE_OK;
 
   // 4. grouped A rows of the routed experts
   prof.begin(4);
@@ -396,7 +440,7 @@ int forward_impl(moe_handle* h, int T, const uint16_t* x, const uint16_t* residu
   // 5b. E4M3: h rows (routed and shared) to E4M3 with their row exponents
   if (f8) {
     prof.begin(11);
-    MOE_TRY(launch_quant_rows(hb, TK, c.I, hq, he, hsb, h->S * T, c.I_shared, hqs, hse, s));
+    MOE_TRY(launch_quant_rows(hb, TK, c.I, hq, he, hsb, h->S * T, c.I_shared, hqs, hse, nullptr, s));
     prof.end(11);
   }
 
@@ -462,6 +506,7 @@ int check_forward_args(const moe_handle* h, int T, const void* x, const void* re
                        const void* token_ids, const void* out_norm, const void* out_residual,
                        const void* workspace, size_t ws_bytes, size_t need) {
   if (!h || T < 0) return MOE_EINVAL;
+  if (h->ep_world > 1) return MOE_EINVAL;   // expert-parallel handles run the moe_ep_* phases
   if (T > h->cfg.T_max) return MOE_ETOOBIG;
   if (T == 0) return MOE_OK;
   if (!x || !residual || !out_norm || !out_residual || !workspace) return MOE_EINVAL;
@@ -495,6 +540,10 @@ int moe_init(const moe_config* cfg, const moe_weights* w, moe_handle** out) {
   // bn_gu / 2 up rows) or half of a down tile (bn_dn / 2 rows).
   h->L = cfg->latent > 0 ? cfg->latent : cfg->D;
   h->fp8 = cfg->weight_format == MOE_WEIGHTS_FP8;
+  h->ep_world = cfg->ep_world > 1 ? cfg->ep_world : 1;
+  h->ep_rank = cfg->ep_world > 1 ? cfg->ep_rank : 0;
+  h->E_loc = cfg->E / h->ep_world;
+  h->cap = h->ep_world > 1 ? static_cast<long long>(h->ep_world) * cfg->T_max * cfg->k : 0;
   h->bn_gu = (cfg->I % 128 == 0 && h->cfg.I_shared % 128 == 0) ? 128 : 64;
   // The down GEMM's routed groups have N = L, its shared groups N = D.
   auto bn_for = [](int n) { return n % 256 == 0 ? 256 : (n % 128 == 0 ? 128 : 64); };
@@ -518,9 +567,9 @@ int moe_init(const moe_config* cfg, const moe_weights* w, moe_handle** out) {
   }
   const int eb = h->fp8 ? 1 : 2;   // expert weights: E4M3 or bf16
   bool ok = make_map(&h->map_router, h->w_router_pad, h->L, h->w_router_pad ? h->E_pad : 0, h->E_pad) &&
-            make_map(&h->map_wg, w->w_gate, h->L, static_cast<uint64_t>(c.E) * c.I, h->bn_gu / 2, eb) &&
-            make_map(&h->map_wu, w->w_up, h->L, static_cast<uint64_t>(c.E) * c.I, h->bn_gu / 2, eb) &&
-            make_map(&h->map_wd, w->w_down, c.I, static_cast<uint64_t>(c.E) * h->L, h->bn_dn / 2, eb) &&
+            make_map(&h->map_wg, w->w_gate, h->L, static_cast<uint64_t>(h->E_loc) * c.I, h->bn_gu / 2, eb) &&
+            make_map(&h->map_wu, w->w_up, h->L, static_cast<uint64_t>(h->E_loc) * c.I, h->bn_gu / 2, eb) &&
+            make_map(&h->map_wd, w->w_down, c.I, static_cast<uint64_t>(h->E_loc) * h->L, h->bn_dn / 2, eb) &&
             make_map(&h->map_wsg, w->ws_gate, c.D, static_cast<uint64_t>(h->S) * c.I_shared, h->bn_gu / 2, eb) &&
             make_map(&h->map_wsu, w->ws_up, c.D, static_cast<uint64_t>(h->S) * c.I_shared, h->bn_gu / 2, eb) &&
             make_map(&h->map_wsd, w->ws_down, c.I_shared, static_cast<uint64_t>(h->S) * c.D, h->bn_dn / 2, eb) &&
@@ -606,7 +655,8 @@ int moe_check_invariance(moe_handle* h, int T, const moe_bf16* x, const moe_bf16
                          const int32_t* token_ids, int n_splits, const int32_t* perm, int repeats,
                          void* workspace, size_t ws_bytes, unsigned long long* out_mismatched_elems,
                          void* stream) {
-  if (!h || !out_mismatched_elems || T <= 0 || n_splits < 0 || repeats < 0) return MOE_EINVAL;
+  if (!h || !out_mismatched_elems || T <= 0 || n_splits < 0 || repeats < 0 || h->ep_world > 1)
+    return MOE_EINVAL;
   if (T > h->cfg.T_max) return MOE_ETOOBIG;
   if (n_splits > T || 2 + n_splits + repeats > kMaxInvRuns) return MOE_EINVAL;
   if (!x || !residual || !workspace) return MOE_EINVAL;
@@ -758,6 +808,217 @@ int moe_selftest_wait_timeout(int limit_us, void* stream) {
     res = host[1] == kDevTimeout ? MOE_ETIMEOUT : MOE_OK;
   cudaFree(buf);
   return res;
+}
+
+// ---------------------------------------------------------------- expert parallelism
+namespace {
+
+int ep_check(const moe_handle* h, int T, const void* workspace, size_t ws_bytes) {
+  if (!h || h->ep_world <= 1 || T < 0 || !workspace) return MOE_EINVAL;
+  if (T > h->cfg.T_max) return MOE_ETOOBIG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MOE_EINVAL;
+  if (T > 0 && ws_bytes < layout(h, T).total) return MOE_EWORKSPACE;
+  return MOE_OK;
+}
+
+int ep_peers_ok(const moe_handle* h, const moe_ep_peers* p) {
+  if (!p) return MOE_EINVAL;
+  for (int r = 0; r < h->ep_world; ++r)
+    if (!p->xbuf[r] || (reinterpret_cast<uintptr_t>(p->xbuf[r]) & 255u) != 0) return MOE_EINVAL;
+  return MOE_OK;
+}
+
+}  // namespace
+
+size_t moe_ep_exchange_size(const moe_handle* h) {
+  if (!h || h->ep_world <= 1) return 0;
+  return xlayout(h).total;
+}
+
+int moe_ep_route(moe_handle* h, int T, const moe_bf16* x, const int32_t* token_ids, void* xbuf_self,
+                 void* workspace, size_t ws_bytes, void* stream) {
+  const int v = ep_check(h, T, workspace, ws_bytes);
+  if (v != MOE_OK) return v;
+  if (!xbuf_self || (reinterpret_cast<uintptr_t>(xbuf_self) & 255u) != 0) return MOE_EINVAL;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int32_t* board = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(xbuf_self) + xlayout(h).board);
+  if (T == 0) return cudaMemsetAsync(board, 0, static_cast<size_t>(h->cfg.E) * 4, s) == cudaSuccess ? MOE_OK
+                                                                                                   : MOE_ECUDA;
+  if (!x || !aligned16(x) || (h->cfg.router == MOE_ROUTER_HASH && !token_ids)) return MOE_EINVAL;
+  return forward_impl(h, T, x, nullptr, token_ids, nullptr, nullptr, nullptr, nullptr, nullptr,
+                      static_cast<uint8_t*>(workspace), s, true, board);
+}
+
+int moe_ep_send(moe_handle* h, int T, const moe_ep_peers* peers, void* workspace, size_t ws_bytes,
+                void* stream) {
+  int v = ep_check(h, T, workspace, ws_bytes);
+  if (v == MOE_OK) v = ep_peers_ok(h, peers);
+  if (v != MOE_OK || T == 0) return v;
+  const moe_config& c = h->cfg;
+  const Layout L = layout(h, T);
+  const XLayout X = xlayout(h);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  EpSendArgs a;
+  std::memset(&a, 0, sizeof(a));
+  for (int r = 0; r < h->ep_world; ++r) {
+    uint8_t* xb = static_cast<uint8_t*>(peers->xbuf[r]);
+    a.boards[r] = reinterpret_cast<const int32_t*>(xb + X.board);
+    a.recv[r] = xb + X.recv;
+    a.recv_exp[r] = h->fp8 ? reinterpret_cast<int8_t*>(xb + X.recv_exp) : nullptr;
+    a.meta[r] = reinterpret_cast<int32_t*>(xb + X.meta);
+  }
+  a.src_rows = h->fp8 ? ws + L.xq : ws + L.xn;
+  a.src_exp = h->fp8 ? reinterpret_cast<const int8_t*>(ws + L.xqe) : nullptr;
+  a.offsets = reinterpret_cast<const int32_t*>(ws + L.offsets);
+  a.src_token = reinterpret_cast<const int32_t*>(ws + L.src);
+  a.dest_row = reinterpret_cast<const int32_t*>(ws + L.dest);
+  a.rows = T * c.k;
+  a.row_bytes = h->L * (h->fp8 ? 1 : 2);
+  a.E = c.E; a.E_loc = h->E_loc; a.world = h->ep_world; a.rank = h->ep_rank;
+  const int grid = std::max(1, std::min((a.rows + 7) / 8, 4 * h->num_sms));
+  return launch_ep_send(a, grid, static_cast<cudaStream_t>(stream)) == cudaSuccess ? MOE_OK : MOE_ECUDA;
+}
+
+int moe_ep_experts(moe_handle* h, int T, const moe_ep_peers* peers, void* workspace, size_t ws_bytes,
+                   void* stream) {
+  int v = ep_check(h, T, workspace, ws_bytes);
+  if (v == MOE_OK) v = ep_peers_ok(h, peers);
+  if (v != MOE_OK) return v;
+  if (T == 0 && h->S > 0) return MOE_EINVAL;   // shared experts need this rank's tokens
+  const moe_config& c = h->cfg;
+  const Layout L = layout(h, std::max(T, 1));
+  const XLayout X = xlayout(h);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const bool f8 = h->fp8;
+  const int eb = f8 ? 1 : 2;
+  uint8_t* self = static_cast<uint8_t*>(peers->xbuf[h->ep_rank]);
+  int* err = reinterpret_cast<int*>(ws + L.err);
+  int32_t* off = reinterpret_cast<int32_t*>(ws + L.epoff);
+  int32_t* tg = reinterpret_cast<int32_t*>(ws + L.eptg);
+  int32_t* td = reinterpret_cast<int32_t*>(ws + L.eptd);
+  int32_t* nrows = reinterpret_cast<int32_t*>(ws + L.eprows);
+  const int nt_gu = c.I / h->bn_gu, nt_gus = h->S > 0 ? c.I_shared / h->bn_gu : 0;
+  const int nt_dn = h->L / h->bn_dn, nt_dns = c.D / h->bn_dn;
+  // 1. The owner's plan from every rank's counts.
+  EpPlanArgs pa;
+  std::memset(&pa, 0, sizeof(pa));
+  for (int r = 0; r < h->ep_world; ++r)
+    pa.boards[r] = reinterpret_cast<const int32_t*>(static_cast<uint8_t*>(peers->xbuf[r]) + X.board);
+  pa.world = h->ep_world; pa.rank = h->ep_rank; pa.E_loc = h->E_loc; pa.S = h->S; pa.T_self = T;
+  pa.offsets = off; pa.tiles_gu = tg; pa.tiles_dn = td; pa.rows_received = nrows;
+  pa.gu_ntiles_routed = nt_gu; pa.gu_ntiles_shared = nt_gus; pa.dn_ntiles = nt_dn; pa.dn_ntiles_shared = nt_dns;
+  pa.tile_m = kPairTileM;
+  MOE_TRY(launch_ep_plan(pa, s));
+  const long long cap = h->cap;
+  const int G = h->E_loc + h->S;
+  // Tiles at most: sum over local experts of ceil(rows / 256) <= cap / 256 + E_loc.
+  auto bound = [&](int nt_r, int nt_s) {
+    const long long b = (cap / kPairTileM + h->E_loc) * nt_r +
+                        static_cast<long long>(h->S) * ((T + kPairTileM - 1) / kPairTileM) * nt_s;
+    return static_cast<int>(std::min<long long>(b, 1 << 29));
+  };
+  const uint8_t* recv = self + X.recv;
+  const int8_t* recv_exp = f8 ? reinterpret_cast<const int8_t*>(self + X.recv_exp) : nullptr;
+  uint16_t* xn = reinterpret_cast<uint16_t*>(ws + L.xn);
+  uint16_t* hr = reinterpret_cast<uint16_t*>(ws + L.hr);
+  uint16_t* hsb = reinterpret_cast<uint16_t*>(ws + L.hs);
+  float* ys = reinterpret_cast<float*>(ws + L.ys);
+  // 2. gate/up: routed groups read the received rows, shared groups this rank's xn.
+  {
+    GemmArgs g;
+    std::memset(&g, 0, sizeof(g));
+    const void* xs = f8 ? static_cast<const void*>(ws + L.xq) : static_cast<const void*>(xn);
+    if (!make_map(&g.mapA[0], recv, h->L, cap, kBM, eb) || !make_map(&g.mapA64[0], recv, h->L, cap, kBM / 2, eb) ||
+        !make_map(&g.mapA16[0], recv, h->L, cap, 16, eb))
+      return MOE_ECUDA;
+    if (h->S > 0 && T > 0 &&
+        (!make_map(&g.mapA[1], xs, c.D, T, kBM, eb) || !make_map(&g.mapA64[1], xs, c.D, T, kBM / 2, eb) ||
+         !make_map(&g.mapA16[1], xs, c.D, T, 16, eb)))
+      return MOE_ECUDA;
+    g.mapB[0] = h->map_wg; g.mapB[1] = h->map_wu; g.mapB[2] = h->map_wsg; g.mapB[3] = h->map_wsu;
+    g.offsets = off; g.tile_start = tg; g.G = G; g.E = h->E_loc; g.T = T;
+    g.n_kind[0] = c.I; g.n_kind[1] = c.I_shared;
+    g.k_kind[0] = h->L; g.k_kind[1] = c.D;
+    g.BN = h->bn_gu;
+    g.swap_ok = h->bn_gu == 128;
+    g.shared_a_stride = 0;
+    g.out[0] = hr; g.ld_out[0] = c.I;
+    g.out[1] = hsb; g.ld_out[1] = c.I_shared;
+    g.shared_out_stride = T;
+    g.gate_clamp = c.gate_clamp_max; g.up_clamp = c.up_clamp;
+    g.act = c.activation; g.beta_g = c.situ_beta_gate; g.beta_u = c.situ_beta_up;
+    g.inv_beta_g = 1.0f / c.situ_beta_gate; g.inv_beta_u = 1.0f / c.situ_beta_up;
+    g.fp8 = f8;
+    g.a_exp[0] = recv_exp; g.a_exp[1] = reinterpret_cast<const int8_t*>(ws + L.xqe);
+    g.err = err; g.timeout_ns = h->timeout_ns;
+    MOE_TRY(launch_grouped_gemm(kGateUp, g, pair_grid(h, bound(nt_gu, nt_gus)), s));
+  }
+  // 3. E4M3: the received rows' h (only the first rows_received are real) and the shared h.
+  uint8_t* hqr = ws + L.hqr;
+  int8_t* her = reinterpret_cast<int8_t*>(ws + L.her);
+  uint8_t* hqs = ws + L.hqs;
+  int8_t* hse = reinterpret_cast<int8_t*>(ws + L.hse);
+  if (f8)
+    MOE_TRY(launch_quant_rows(hr, static_cast<int>(cap), c.I, hqr, her, hsb, h->S * T, c.I_shared, hqs, hse,
+                              nrows, s));
+  // 4. down: routed rows go back to their source rank's slot rows, shared rows stay here.
+  {
+    GemmArgs g;
+    std::memset(&g, 0, sizeof(g));
+    const void* ar = f8 ? static_cast<const void*>(hqr) : static_cast<const void*>(hr);
+    const void* as = f8 ? static_cast<const void*>(hqs) : static_cast<const void*>(hsb);
+    const uint64_t srows = static_cast<uint64_t>(h->S) * T;
+    if (!make_map(&g.mapA[0], ar, c.I, cap, kBM, eb) || !make_map(&g.mapA64[0], ar, c.I, cap, kBM / 2, eb) ||
+        !make_map(&g.mapA16[0], ar, c.I, cap, 16, eb))
+      return MOE_ECUDA;
+    if (h->S > 0 && T > 0 &&
+        (!make_map(&g.mapA[1], as, c.I_shared, srows, kBM, eb) ||
+         !make_map(&g.mapA64[1], as, c.I_shared, srows, kBM / 2, eb) ||
+         !make_map(&g.mapA16[1], as, c.I_shared, srows, 16, eb)))
+      return MOE_ECUDA;
+    g.mapB[0] = h->map_wd; g.mapB[2] = h->map_wsd;
+    g.offsets = off; g.tile_start = td; g.G = G; g.E = h->E_loc; g.T = T;
+    g.n_kind[0] = h->L; g.n_kind[1] = c.D;
+    g.k_kind[0] = c.I; g.k_kind[1] = c.I_shared;
+    g.BN = h->bn_dn;
+    g.swap_ok = h->bn_dn == 256;
+    g.shared_a_stride = T;
+    g.out[0] = nullptr; g.ld_out[0] = h->L;
+    g.out[1] = ys; g.ld_out[1] = c.D;
+    g.shared_out_stride = T;
+    g.dest_row = reinterpret_cast<const int32_t*>(self + X.meta);
+    g.ep = 1;
+    for (int r = 0; r < h->ep_world; ++r)
+      g.out_rank[r] = reinterpret_cast<float*>(static_cast<uint8_t*>(peers->xbuf[r]) + X.y);
+    g.fp8 = f8;
+    g.a_exp[0] = her; g.a_exp[1] = hse;
+    g.err = err; g.timeout_ns = h->timeout_ns;
+    MOE_TRY(launch_grouped_gemm(kDown, g, pair_grid(h, bound(nt_dn, nt_dns)), s));
+  }
+  return MOE_OK;
+}
+
+int moe_ep_combine(moe_handle* h, int T, const moe_bf16* residual, void* xbuf_self, moe_bf16* out_norm,
+                   moe_bf16* out_residual, int32_t* out_topk_idx, float* out_topk_w, void* workspace,
+                   size_t ws_bytes, void* stream) {
+  const int v = ep_check(h, T, workspace, ws_bytes);
+  if (v != MOE_OK || T == 0) return v;
+  if (!residual || !out_norm || !out_residual || !xbuf_self || !aligned16(residual) || !aligned16(out_norm) ||
+      !aligned16(out_residual))
+    return MOE_EINVAL;
+  const moe_config& c = h->cfg;
+  const Layout L = layout(h, T);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const float* y = reinterpret_cast<const float*>(static_cast<uint8_t*>(xbuf_self) + xlayout(h).y);
+  const float* tw = reinterpret_cast<const float*>(ws + L.tw);
+  MOE_TRY(launch_combine_norm(y, tw, reinterpret_cast<const float*>(ws + L.ys), c.k, h->S, residual, h->w.g_out,
+                              out_norm, out_residual, T, c.D, c.eps, s));
+  const size_t tk = static_cast<size_t>(T) * c.k * 4;
+  if (out_topk_idx) MOE_TRY(cudaMemcpyAsync(out_topk_idx, ws + L.tidx, tk, cudaMemcpyDeviceToDevice, s));
+  if (out_topk_w) MOE_TRY(cudaMemcpyAsync(out_topk_w, ws + L.tw, tk, cudaMemcpyDeviceToDevice, s));
+  return MOE_OK;
 }
 
 int moe_quantize_weights_fp4(const moe_bf16* w, uint8_t* w8, int8_t* block_exp, long long rows, int K,

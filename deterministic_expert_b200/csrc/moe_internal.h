@@ -75,6 +75,8 @@ struct GemmArgs {
   int dense_kind;         // kind of the single group when tile_start is NULL
   int out_bf16;           // down-mode output as bf16 instead of fp32 (latent projection)
   int fp8;                // expert GEMMs: A and B are E4M3 codes (kind::f8f6f4)
+  int ep;                 // down, routed: dest_row = rank << 24 | row, stored at out_rank[rank]
+  float* out_rank[8];     // ep: each rank's slot-row output base (addresses on this rank)
   const int8_t* a_exp[2]; // fp8: per kind, power-of-two exponent of each A row; the
                           // accumulator of row r is multiplied by 2^a_exp[kind][r]
   void* out[2];           // output base per kind
@@ -100,9 +102,11 @@ cudaError_t launch_rmsnorm_rows(const uint16_t* x, const uint16_t* g, uint16_t* 
                                 float eps, int* err_to_clear, int32_t* zero, int zero_words,
                                 uint8_t* yq, int8_t* yq_exp, cudaStream_t s);
 // bf16 rows -> E4M3 rows + per-row exponents, two segments.
+// rows0_dev != NULL: only the first *rows0_dev of the rows0 rows of segment 0
+// are real (the rest are skipped).
 cudaError_t launch_quant_rows(const uint16_t* a0, int rows0, int w0, uint8_t* q0, int8_t* e0,
                               const uint16_t* a1, int rows1, int w1, uint8_t* q1, int8_t* e1,
-                              cudaStream_t s);
+                              const int32_t* rows0_dev, cudaStream_t s);
 // FP4 (E2M1, power-of-two scale per 32-element block) -> E4M3 weights.
 cudaError_t launch_quant_weights_fp4(const uint16_t* w, uint8_t* w8, int8_t* block_exp, long long nblocks,
                                      cudaStream_t s);
@@ -173,6 +177,32 @@ struct DispatchArgs {
 cudaError_t launch_dispatch(const DispatchArgs& a, cudaStream_t s);
 cudaError_t launch_gather_rows(const void* src, const int32_t* src_row, int rows, int row_bytes, void* dst,
                                const int8_t* src_exp, int8_t* dst_exp, cudaStream_t s);
+
+// ------------------------------------------------------- expert parallelism
+struct EpSendArgs {
+  const int32_t* boards[8];  // per rank: its [E] expert counts (addresses on this rank)
+  uint8_t* recv[8];          // per rank: received input rows
+  int8_t* recv_exp[8];       // per rank: their E4M3 exponents (E4M3 rows only)
+  int32_t* meta[8];          // per rank: return address (source rank << 24 | token * k + slot)
+  const uint8_t* src_rows;   // this rank's input rows (xn bf16 or xq E4M3)
+  const int8_t* src_exp;     // their exponents, or NULL for bf16 rows
+  const int32_t* offsets;    // [E + 1] this rank's grouped rows per expert
+  const int32_t* src_token;  // [rows] grouped row -> token
+  const int32_t* dest_row;   // [rows] grouped row -> token * k + slot
+  int rows, row_bytes, E, E_loc, world, rank;
+};
+cudaError_t launch_ep_send(const EpSendArgs& a, int grid, cudaStream_t s);
+
+struct EpPlanArgs {
+  const int32_t* boards[8];
+  int world, rank, E_loc, S, T_self;
+  int32_t* offsets;          // [E_loc + 1] received rows per local expert
+  int32_t* tiles_gu;         // [E_loc + S + 1]
+  int32_t* tiles_dn;         // [E_loc + S + 1]
+  int32_t* rows_received;    // [1]
+  int gu_ntiles_routed, gu_ntiles_shared, dn_ntiles, dn_ntiles_shared, tile_m;
+};
+cudaError_t launch_ep_plan(const EpPlanArgs& a, cudaStream_t s);
 
 // ------------------------------------------------------------ self test
 cudaError_t launch_wait_selftest(int* flag, int* err, unsigned long long limit_ns,

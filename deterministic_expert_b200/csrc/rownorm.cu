@@ -180,12 +180,14 @@ __global__ void __launch_bounds__(kRowThreads) k_rmsnorm_rows(const uint16_t* __
 __global__ void __launch_bounds__(256) k_quant_rows(const uint16_t* __restrict__ a0, int rows0, int w0,
                                                     uint8_t* __restrict__ q0, int8_t* __restrict__ e0,
                                                     const uint16_t* __restrict__ a1, int rows1, int w1,
-                                                    uint8_t* __restrict__ q1, int8_t* __restrict__ e1) {
+                                                    uint8_t* __restrict__ q1, int8_t* __restrict__ e1,
+                                                    const int32_t* __restrict__ rows0_dev) {
   griddep_wait();
   griddep_launch();
   const int r0 = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   const bool first = r0 < rows0;
   if (!first && r0 >= rows0 + rows1) return;
+  if (first && rows0_dev != nullptr && r0 >= *rows0_dev) return;
   const int r = first ? r0 : r0 - rows0;
   const int w = first ? w0 : w1;
   const uint16_t* ar = (first ? a0 : a1) + static_cast<size_t>(r) * w;
@@ -438,11 +440,11 @@ cudaError_t launch_rmsnorm_rows(const uint16_t* x, const uint16_t* g, uint16_t* 
 
 cudaError_t launch_quant_rows(const uint16_t* a0, int rows0, int w0, uint8_t* q0, int8_t* e0,
                               const uint16_t* a1, int rows1, int w1, uint8_t* q1, int8_t* e1,
-                              cudaStream_t s) {
+                              const int32_t* rows0_dev, cudaStream_t s) {
   const int rows = rows0 + rows1;
   if (rows <= 0) return cudaSuccess;
   return launch_k(k_quant_rows, dim3((rows + 7) / 8), dim3(256), 0, s, false, a0, rows0, w0, q0, e0, a1,
-                  rows1, w1, q1, e1);
+                  rows1, w1, q1, e1, rows0_dev);
 }
 
 cudaError_t launch_combine_norm(const float* y_slot, const float* topk_w, const float* y_shared,

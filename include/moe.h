@@ -126,6 +126,12 @@ typedef struct moe_config {
                           experts stay at width D (linux.do post on MoE variants,
                           "潜在MoE (Latent MoE)" and K3's Stable Latent MoE)          */
   int weight_format;   /* moe_weight_format of the routed and shared expert weights     */
+  int ep_world;        /* expert parallelism over this many ranks (0 or 1 = none; at most
+                          8, dividing E): rank r owns routed experts [r E/ep_world,
+                          (r+1) E/ep_world) and its w_gate / w_up / w_down hold only
+                          those; router and shared experts are whole on every rank.
+                          Such a handle runs the moe_ep_* phases, not moe_layer_forward */
+  int ep_rank;         /* this rank, 0 <= ep_rank < ep_world                             */
 } moe_config;
 
 typedef struct moe_weights {      /* device pointers, caller-owned; L = latent if
@@ -327,6 +333,60 @@ int moe_layer_forward_noalloc(moe_handle* h, int T, const moe_bf16* x, const moe
  * multiple of 32), MOE_ECUDA (launch). */
 int moe_quantize_weights_fp4(const moe_bf16* w, uint8_t* w8, int8_t* block_exp, long long rows, int K,
                              void* stream);
+
+/* ------------------------------------------------------------------------
+ * Expert parallelism (DeepSeek V4 infra notes, §6.1: dispatch -> compute ->
+ * combine, with tokens sent to the rank that holds their expert and results
+ * sent back; the Fireworks parity post, Trap 3 and its case study: the k
+ * contributions of a token are added in fp32, in slot order, on the token's
+ * own rank, never in bf16 or in arrival order).
+ *
+ * Every rank holds its own T tokens (T may differ between ranks, each at most
+ * T_max) and one exchange buffer of moe_ep_exchange_size bytes that the other
+ * ranks can address (moe_peer_alloc / moe_peer_open across processes, or plain
+ * device memory when several ranks share one device and one process).  A step
+ * is four calls on each rank, in this order, with every rank's call of one
+ * phase complete before any rank's call of the next phase reads what it wrote
+ * (a device barrier such as moe_peer_barrier between phases, or stream order
+ * when the ranks share a stream):
+ *   moe_ep_route    RMSNorm, router, top-k, the stable grouping of the rank's
+ *                   (token, slot) rows by expert; its per-expert counts go to
+ *                   its own exchange buffer.
+ *   moe_ep_send     from every rank's counts, the row each (token, slot) takes at
+ *                   its expert's owner (owner's experts in order; inside an
+ *                   expert, source ranks in order; inside a source rank, tokens
+ *                   in order, then slots); the input row (bf16, or E4M3 and its
+ *                   exponent) and its return address are stored there.
+ *   moe_ep_experts  the owner's routed experts over the rows it received and the
+ *                   shared experts over its own tokens; each routed output row
+ *                   (fp32) is stored into its source rank's exchange buffer at
+ *                   that token's slot row.
+ *   moe_ep_combine  the fixed slot-order combine + residual + RMSNorm of the
+ *                   rank's own tokens (as moe_layer_forward).
+ * Each (token, slot) row goes through the same full-K GEMMs as in
+ * moe_layer_forward, whose bits do not depend on which rows share a tile, so
+ * every rank's outputs are bit for bit those of moe_layer_forward on its
+ * tokens with all experts on one device.
+ * `peers` lists the exchange buffer of every rank (index = rank) as addresses
+ * valid on this rank.  `workspace` is this rank's (moe_workspace_size for its
+ * T), kept across the four calls.  Errors: MOE_EINVAL (NULL, wrong rank
+ * count, not an EP handle), MOE_ETOOBIG, MOE_EWORKSPACE, MOE_ECUDA.  No call
+ * synchronises.
+ * ------------------------------------------------------------------------ */
+typedef struct moe_ep_peers {
+  void* xbuf[8];
+} moe_ep_peers;
+
+size_t moe_ep_exchange_size(const moe_handle* h);
+int moe_ep_route(moe_handle* h, int T, const moe_bf16* x, const int32_t* token_ids, void* xbuf_self,
+                 void* workspace, size_t ws_bytes, void* stream);
+int moe_ep_send(moe_handle* h, int T, const moe_ep_peers* peers, void* workspace, size_t ws_bytes,
+                void* stream);
+int moe_ep_experts(moe_handle* h, int T, const moe_ep_peers* peers, void* workspace, size_t ws_bytes,
+                   void* stream);
+int moe_ep_combine(moe_handle* h, int T, const moe_bf16* residual, void* xbuf_self, moe_bf16* out_norm,
+                   moe_bf16* out_residual, int32_t* out_topk_idx, float* out_topk_w, void* workspace,
+                   size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
  * Peer memory for the tensor-parallel epilogue (one process per GPU).
