@@ -466,28 +466,37 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
             uint32_t v[32];
             tmem_ld32(tb + c, v);
             tmem_ld_wait();
-            const int my_tok = c + lane;  // this lane fetches the output row of token c + lane
+            // Lane j resolves the output row of token c + j once (its scattered
+            // slot row, in its source rank's buffer under expert parallelism);
+            // the stores below take it by shuffle.
+            const int my_tok = c + lane;
             int my_row = 0;
+            float* my_ptr = outb;
             float my_sc = 1.f;
             if (my_tok < r) {
               my_row = scatter ? a.dest_row[ti.a_row0 + trow0 + my_tok] : orow0 + my_tok;
+              if (scatter && a.ep) my_ptr = a.out_rank[my_row >> 24] + static_cast<size_t>(my_row & 0xFFFFFF) * ld;
+              else my_ptr = outb + static_cast<size_t>(my_row) * ld;
               if (F8) my_sc = exp2_int(a.a_exp[ti.kind][ti.a_row0 + trow0 + my_tok]);
             }
+            if (a.out_bf16) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const int orow = __shfl_sync(0xffffffffu, my_row, j);
-              const float sc = F8 ? __shfl_sync(0xffffffffu, my_sc, j) : 1.f;
-              if (c + j < r) {
-                const float val = F8 ? __fmul_rn(__uint_as_float(v[j]), sc) : __uint_as_float(v[j]);
-                if (a.out_bf16) {
+              for (int j = 0; j < 32; ++j) {
+                const int orow = __shfl_sync(0xffffffffu, my_row, j);
+                const float sc = F8 ? __shfl_sync(0xffffffffu, my_sc, j) : 1.f;
+                if (c + j < r) {
+                  const float val = F8 ? __fmul_rn(__uint_as_float(v[j]), sc) : __uint_as_float(v[j]);
                   outh[static_cast<size_t>(orow) * ld + col] =
                       static_cast<uint16_t>(pack_bf16x2(val, 0.f) & 0xFFFFu);
-                } else if (scatter && a.ep) {
-                  // Expert parallelism: the row lives in its source rank's buffer.
-                  a.out_rank[orow >> 24][static_cast<size_t>(orow & 0xFFFFFF) * ld + col] = val;
-                } else {
-                  outb[static_cast<size_t>(orow) * ld + col] = val;
                 }
+              }
+            } else {
+              const unsigned long long my_addr = reinterpret_cast<unsigned long long>(my_ptr);
+#pragma unroll
+              for (int j = 0; j < 32; ++j) {
+                float* rowp = reinterpret_cast<float*>(__shfl_sync(0xffffffffu, my_addr, j));
+                const float sc = F8 ? __shfl_sync(0xffffffffu, my_sc, j) : 1.f;
+                if (c + j < r) rowp[col] = F8 ? __fmul_rn(__uint_as_float(v[j]), sc) : __uint_as_float(v[j]);
               }
             }
           }
