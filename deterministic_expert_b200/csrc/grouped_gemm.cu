@@ -61,8 +61,6 @@ template <int CG>
 struct Cfg {
   static constexpr int kTileM = 128 * CG;                                 // rows per tile (pair)
   static constexpr int kSmemB = CG == 1 ? 256 * kBK * 2 : 128 * kBK * 2;  // B bytes per CTA stage
-  static constexpr int kStage = kSmemA + kSmemB;
-  static constexpr int kStagesN = kRingBytes / kStage;  // 4 or 6
 };
 
 struct Tile {
