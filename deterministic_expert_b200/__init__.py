@@ -567,6 +567,7 @@ class _EPRank:
         self.device = device
 
     def route(self, x, token_ids, xbuf, stream=None):
+        # A rank with no tokens still publishes its (zero) counts.
         L = lib()
         L.moe_ep_route.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
                                    ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]

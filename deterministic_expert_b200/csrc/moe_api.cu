@@ -842,8 +842,13 @@ int moe_ep_route(moe_handle* h, int T, const moe_bf16* x, const int32_t* token_i
   if (!xbuf_self || (reinterpret_cast<uintptr_t>(xbuf_self) & 255u) != 0) return MOE_EINVAL;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int32_t* board = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(xbuf_self) + xlayout(h).board);
-  if (T == 0) return cudaMemsetAsync(board, 0, static_cast<size_t>(h->cfg.E) * 4, s) == cudaSuccess ? MOE_OK
-                                                                                                   : MOE_ECUDA;
+  if (T == 0) {
+    // No tokens: publish zero counts and clear the device error word (which the
+    // input RMSNorm clears otherwise).
+    MOE_TRY(cudaMemsetAsync(board, 0, static_cast<size_t>(h->cfg.E) * 4, s));
+    MOE_TRY(cudaMemsetAsync(workspace, 0, 4, s));
+    return MOE_OK;
+  }
   if (!x || !aligned16(x) || (h->cfg.router == MOE_ROUTER_HASH && !token_ids)) return MOE_EINVAL;
   return forward_impl(h, T, x, nullptr, token_ids, nullptr, nullptr, nullptr, nullptr, nullptr,
                       static_cast<uint8_t*>(workspace), s, true, board);
@@ -884,7 +889,8 @@ int moe_ep_experts(moe_handle* h, int T, const moe_ep_peers* peers, void* worksp
   int v = ep_check(h, T, workspace, ws_bytes);
   if (v == MOE_OK) v = ep_peers_ok(h, peers);
   if (v != MOE_OK) return v;
-  if (T == 0 && h->S > 0) return MOE_EINVAL;   // shared experts need this rank's tokens
+  // T == 0: this rank has no tokens (no shared-expert tiles) but still serves
+  // its routed experts for the other ranks.
   const moe_config& c = h->cfg;
   const Layout L = layout(h, std::max(T, 1));
   const XLayout X = xlayout(h);

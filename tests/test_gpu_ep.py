@@ -29,6 +29,7 @@ CASES = {
     "tiny_w2": (W.C1, 2, [37, 100]),
     "tiny_w4": (W.C1, 4, [1, 64, 129, 30]),
     "tiny_w8": (W.C1, 8, [5, 17, 33, 1, 64, 2, 90, 11]),
+    "tiny_w4_empty_rank": (W.C1, 4, [40, 0, 70, 25]),
     "tiny_fp8_w4": (W.C1F, 4, [50, 7, 200, 64]),
     "hash_w2": (dataclasses.replace(W.C1, router=W.ROUTER_HASH, k=3, name="hash_small"), 2, [77, 120]),
     "situ_w2": (dataclasses.replace(W.C1, activation=1, name="tiny_situ"), 2, [90, 40]),
