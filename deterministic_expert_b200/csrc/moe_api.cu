@@ -3,6 +3,7 @@
 // layer forward.  Everything here runs on the host; every step of the layer
 // runs in the kernels of the other translation units.
 #include <cudaTypedefs.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <algorithm>
 #include <cstring>
@@ -227,15 +228,25 @@ int gemm_grid(const moe_handle* h, int tiles_bound) {
   return std::max(1, std::min(h->num_sms, tiles_bound));
 }
 
+// Stage names as moe_profile_read numbers them; each stage's launch is also an
+// NVTX range of that name (host-side markers for a timeline tool; a no-op
+// when none is attached).
+const char* const kStageNames[MOE_NUM_STAGES] = {
+    "moe.rmsnorm_in", "moe.router_gemm", "moe.router_topk", "moe.dispatch", "moe.gather_rows",
+    "moe.gemm_gateup", "moe.gemm_down", "moe.combine_norm", "moe.latent_down", "moe.latent_combine",
+    "moe.latent_up", "moe.quant_h"};
+
 struct Prof {
   moe_handle* h;
   cudaStream_t s;
   int f;
   bool on(int stage) const { return f >= 0 && ((h->prof_mask >> stage) & 1); }
   void begin(int stage) {
+    nvtxRangePushA(kStageNames[stage]);
     if (on(stage)) cudaEventRecord(h->ev[(static_cast<size_t>(f) * MOE_NUM_STAGES + stage) * 2], s);
   }
   void end(int stage) {
+    nvtxRangePop();
     if (on(stage)) {
       cudaEventRecord(h->ev[(static_cast<size_t>(f) * MOE_NUM_STAGES + stage) * 2 + 1], s);
       h->prof_launches[stage] += 1;

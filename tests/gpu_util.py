@@ -43,12 +43,16 @@ class Run:
         import torch
         T = int(x.shape[0])
         if ws is None:
-            ws = torch.empty(max(self.layer.workspace_size(T), 256), dtype=torch.uint8, device=self.device)
-        on = torch.empty((T, self.cfg.D), dtype=torch.bfloat16, device=self.device)
-        orr = torch.empty_like(on)
-        idx = torch.empty((T, self.cfg.k), dtype=torch.int32, device=self.device)
-        tw = torch.empty((T, self.cfg.k), dtype=torch.float32, device=self.device)
-        cnt = torch.empty(self.cfg.E, dtype=torch.int32, device=self.device)
+            # The workspace starts as 0xFF bytes (NaN for every float view, -1
+            # for every int view): no stage may read what it did not write.
+            ws = torch.full((max(self.layer.workspace_size(T), 256),), 0xFF, dtype=torch.uint8, device=self.device)
+        # Outputs start poisoned (NaN, -1), so an element the layer leaves
+        # unwritten fails every comparison instead of passing on stale memory.
+        on = torch.full((T, self.cfg.D), float("nan"), dtype=torch.bfloat16, device=self.device)
+        orr = torch.full_like(on, float("nan"))
+        idx = torch.full((T, self.cfg.k), -1, dtype=torch.int32, device=self.device)
+        tw = torch.full((T, self.cfg.k), float("nan"), dtype=torch.float32, device=self.device)
+        cnt = torch.full((self.cfg.E,), -1, dtype=torch.int32, device=self.device)
         self.layer.forward(x, r, on, orr, ws, token_ids=ids, out_topk_idx=idx, out_topk_w=tw,
                            out_counts=cnt)
         torch.cuda.synchronize()
