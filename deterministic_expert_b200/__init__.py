@@ -15,11 +15,14 @@ import os
 from dataclasses import dataclass
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libmoe.so")
+# MOE_LIBRARY=checked loads the build with device-side index checks
+# (MOE_CHECK_BOUNDS: an out-of-range index skips its access and the forward
+# reports MOE_EINDEX); anything else loads the regular build.
+LIB_PATH = os.path.join(_HERE, "libmoe_checked.so" if os.environ.get("MOE_LIBRARY") == "checked" else "libmoe.so")
 HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "moe.h")
 
-MOE_OK, MOE_EINVAL, MOE_ETOOBIG, MOE_EWORKSPACE, MOE_EUNSUPPORTED, MOE_ECUDA, MOE_ETIMEOUT = (
-    0, -1, -2, -3, -4, -5, -6)
+MOE_OK, MOE_EINVAL, MOE_ETOOBIG, MOE_EWORKSPACE, MOE_EUNSUPPORTED, MOE_ECUDA, MOE_ETIMEOUT, MOE_EINDEX = (
+    0, -1, -2, -3, -4, -5, -6, -7)
 ROUTER_SOFTMAX, ROUTER_SIGMOID_BIAS, ROUTER_HASH = 0, 1, 2
 ACT_SWIGLU, ACT_SITU_GLU = 0, 1
 WEIGHTS_BF16, WEIGHTS_FP8 = 0, 1

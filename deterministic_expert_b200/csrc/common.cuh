@@ -11,7 +11,23 @@ namespace moe {
 
 // ------------------------------------------------------------------ errors
 // Device error word values (first word of every forward's workspace).
-enum : int { kDevOk = 0, kDevTimeout = 1, kDevBadTile = 2 };
+enum : int { kDevOk = 0, kDevTimeout = 1, kDevBadTile = 2, kDevBadIndex = 3 };
+
+// Index checks of a build with -DMOE_CHECK_BOUNDS: every index a kernel
+// computes from device data (expert ids, grouped rows, tile coordinates,
+// scatter destinations, rows sent to other ranks) is tested against the
+// extent of the buffer it addresses; a failing index skips its access and
+// records kDevBadIndex in the device error word.  Without the flag the checks
+// compile to nothing.
+__device__ __forceinline__ bool index_fail(int* err) {
+  if (err != nullptr) atomicExch(err, kDevBadIndex);
+  return false;
+}
+#ifdef MOE_CHECK_BOUNDS
+#define MOE_INDEX_OK(cond, err) ((cond) ? true : ::moe::index_fail(err))
+#else
+#define MOE_INDEX_OK(cond, err) true
+#endif
 
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;

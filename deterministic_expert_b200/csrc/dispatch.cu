@@ -108,14 +108,19 @@ __global__ void __launch_bounds__(kDispatchRows) k_dispatch(const DispatchArgs a
 
   const int t = b * kDispatchRows + tid;
   if (t < a.T)
-    for (int j = 0; j < a.k; ++j) atomicOr(&mask[a.idx[t * a.k + j]][tid >> 5], 1u << (tid & 31));
+    for (int j = 0; j < a.k; ++j) {
+      const int e = a.idx[t * a.k + j];
+      if (MOE_INDEX_OK(e >= 0 && e < a.E, a.err)) atomicOr(&mask[e][tid >> 5], 1u << (tid & 31));
+    }
   __syncthreads();
   if (t < a.T) {
     for (int j = 0; j < a.k; ++j) {
       const int e = a.idx[t * a.k + j];
+      if (!MOE_INDEX_OK(e >= 0 && e < a.E, a.err)) continue;
       int rank = __popc(mask[e][tid >> 5] & ((1u << (tid & 31)) - 1u));
       for (int w = 0; w < (tid >> 5); ++w) rank += __popc(mask[e][w]);
       const int p = offs[e] + before[e] + rank;
+      if (!MOE_INDEX_OK(p >= 0 && p < a.T * a.k, a.err)) continue;
       a.dest_row[p] = t * a.k + j;
       a.src_token[p] = t;
     }
@@ -147,14 +152,15 @@ __global__ void __launch_bounds__(kDispatchRows) k_dispatch(const DispatchArgs a
 // dst[p] = src[src_row[p]], one warp per row, 16-byte vectors.
 // Row p of dst = row src_row[p] of src (row_bytes each, a multiple of 16: bf16
 // rows or E4M3 rows), and with E4M3 rows also their exponents.
-__global__ void k_gather_rows(const uint8_t* __restrict__ src, const int32_t* __restrict__ src_row,
+__global__ void k_gather_rows(const uint8_t* __restrict__ src, int src_rows, const int32_t* __restrict__ src_row,
                               int rows, int row_bytes, uint8_t* __restrict__ dst,
-                              const int8_t* __restrict__ src_exp, int8_t* __restrict__ dst_exp) {
+                              const int8_t* __restrict__ src_exp, int8_t* __restrict__ dst_exp, int* err) {
   griddep_wait();
   griddep_launch();
   const int p = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   if (p >= rows) return;
   const int from = src_row[p];
+  if (!MOE_INDEX_OK(from >= 0 && from < src_rows, err)) return;
   const uint4* s = reinterpret_cast<const uint4*>(src + static_cast<size_t>(from) * row_bytes);
   uint4* d = reinterpret_cast<uint4*>(dst + static_cast<size_t>(p) * row_bytes);
   for (int c = lane; c < row_bytes / 16; c += 32) d[c] = s[c];
@@ -168,13 +174,13 @@ cudaError_t launch_dispatch(const DispatchArgs& a, cudaStream_t s) {
   return launch_k(k_dispatch, dim3(nb), dim3(kDispatchRows), 0, s, false, a);
 }
 
-cudaError_t launch_gather_rows(const void* src, const int32_t* src_row, int rows, int row_bytes, void* dst,
-                               const int8_t* src_exp, int8_t* dst_exp, cudaStream_t s) {
+cudaError_t launch_gather_rows(const void* src, int src_rows, const int32_t* src_row, int rows, int row_bytes,
+                               void* dst, const int8_t* src_exp, int8_t* dst_exp, int* err, cudaStream_t s) {
   if (rows <= 0) return cudaSuccess;
   const int warps_per_block = 8;
   return launch_k(k_gather_rows, dim3((rows + warps_per_block - 1) / warps_per_block),
-                  dim3(32 * warps_per_block), 0, s, false, static_cast<const uint8_t*>(src), src_row, rows,
-                  row_bytes, static_cast<uint8_t*>(dst), src_exp, dst_exp);
+                  dim3(32 * warps_per_block), 0, s, false, static_cast<const uint8_t*>(src), src_rows, src_row,
+                  rows, row_bytes, static_cast<uint8_t*>(dst), src_exp, dst_exp, err);
 }
 
 }  // namespace moe

@@ -61,6 +61,7 @@ __global__ void __launch_bounds__(256) k_ep_send(const EpSendArgs a) {
     const int e = lo, owner = e / a.E_loc;
     const int row = dst[e] + (p - offs[e]);
     const int tok = a.src_token[p];
+    if (!MOE_INDEX_OK(owner < a.world && row >= 0 && row < a.cap && tok >= 0, a.err)) continue;
     const uint4* s = reinterpret_cast<const uint4*>(a.src_rows + static_cast<size_t>(tok) * a.row_bytes);
     uint4* d = reinterpret_cast<uint4*>(a.recv[owner] + static_cast<size_t>(row) * a.row_bytes);
     for (int c = lane; c < a.row_bytes / 16; c += 32) d[c] = s[c];

@@ -373,7 +373,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
       tc_fence_after();
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                           static_cast<uint32_t>(acc) * acc_stride;
-      if (CG == 2 && ti.swap) {
+      // Index check (MOE_CHECK_BOUNDS builds): the group's rows lie in its A tensor.
+      const bool tile_ok = a.a_rows[ti.kind] == 0 ||
+                           MOE_INDEX_OK(ti.rows >= 0 && ti.a_row0 >= 0 && ti.a_row0 + ti.rows <= a.a_rows[ti.kind],
+                                        a.err);
+      if (!tile_ok) {
+        // out-of-range group: nothing is stored
+      } else if (CG == 2 && ti.swap) {
         // Operand-swapped tile: TMEM lanes are output columns, TMEM columns are
         // the tile's tokens (rows m * 256 + j of the group, j < r valid).
         const int r = min(256, ti.rows - ti.m * C::kTileM);
@@ -476,6 +482,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
               if (scatter && a.ep) my_ptr = a.out_rank[my_row >> 24] + static_cast<size_t>(my_row & 0xFFFFFF) * ld;
               else my_ptr = outb + static_cast<size_t>(my_row) * ld;
               if (F8) my_sc = exp2_int(a.a_exp[ti.kind][ti.a_row0 + trow0 + my_tok]);
+#ifdef MOE_CHECK_BOUNDS
+              const bool in_range = (scatter && a.ep)
+                                        ? ((my_row >> 24) < a.ep_world && (my_row & 0xFFFFFF) < a.out_rows[0])
+                                        : (my_row >= 0 && my_row < a.out_rows[ti.kind]);
+              if (!MOE_INDEX_OK(in_range, a.err)) my_ptr = nullptr;
+#endif
             }
             if (a.out_bf16) {
 #pragma unroll
@@ -494,6 +506,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
               for (int j = 0; j < 32; ++j) {
                 float* rowp = reinterpret_cast<float*>(__shfl_sync(0xffffffffu, my_addr, j));
                 const float sc = F8 ? __shfl_sync(0xffffffffu, my_sc, j) : 1.f;
+#ifdef MOE_CHECK_BOUNDS
+                if (rowp == nullptr) continue;
+#endif
                 if (c + j < r) rowp[col] = F8 ? __fmul_rn(__uint_as_float(v[j]), sc) : __uint_as_float(v[j]);
               }
             }
@@ -618,6 +633,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
                   ob = a.out_rank[drow >> 24] + ti.n * BN + colhalf * (BN / 2);
                   orow = static_cast<size_t>(drow & 0xFFFFFF);
                 }
+#ifdef MOE_CHECK_BOUNDS
+                {
+                  const bool in_range = (scatter && a.ep)
+                                            ? ((drow >> 24) < a.ep_world && orow < static_cast<size_t>(a.out_rows[0]))
+                                            : (orow < static_cast<size_t>(a.out_rows[ti.kind]));
+                  if (a.out_rows[ti.kind] != 0 && !MOE_INDEX_OK(in_range, a.err)) continue;
+                }
+#endif
                 *reinterpret_cast<uint4*>(ob + orow * ld + c + 4 * sc) = val;
               }
             }

@@ -400,7 +400,7 @@ int forward_impl(moe_handle* h, int T, const uint16_t* x, const uint16_t* residu
   da.gu_ntiles_shared = h->S > 0 ? c.I_shared / h->bn_gu : 0;
   da.dn_ntiles = LW / h->bn_dn;
   da.dn_ntiles_shared = c.D / h->bn_dn;
-  da.dest_row = dest; da.src_token = src;
+  da.dest_row = dest; da.src_token = src; da.err = err;
   da.tile_m = kPairTileM;
   prof.begin(3);
   MOE_TRY(launch_dispatch(da, s));
@@ -409,8 +409,8 @@ int forward_impl(moe_handle* h, int T, const uint16_t* x, const uint16_t* residu
 
   // 4. grouped A rows of the routed experts
   prof.begin(4);
-  if (f8) MOE_TRY(launch_gather_rows(xq, src, TK, LW, xp, xqe, xpe, s));
-  else MOE_TRY(launch_gather_rows(xe, src, TK, LW * 2, xp, nullptr, nullptr, s));
+  if (f8) MOE_TRY(launch_gather_rows(xq, T, src, TK, LW, xp, xqe, xpe, err, s));
+  else MOE_TRY(launch_gather_rows(xe, T, src, TK, LW * 2, xp, nullptr, nullptr, err, s));
   prof.end(4);
 
   // 5. gate/up + SwiGLU(+clamp): routed groups read xp, shared groups read xn
@@ -427,6 +427,8 @@ int forward_impl(moe_handle* h, int T, const uint16_t* x, const uint16_t* residu
     if (h->S > 0 && !make_map(&g.mapA16[1], xs, c.D, T, 16, eb)) return MOE_ECUDA;
     g.fp8 = f8;
     g.a_exp[0] = xpe; g.a_exp[1] = xqe;
+    g.a_rows[0] = TK; g.a_rows[1] = T;
+    g.out_rows[0] = TK; g.out_rows[1] = h->S * T;
     g.mapB[0] = h->map_wg; g.mapB[1] = h->map_wu; g.mapB[2] = h->map_wsg; g.mapB[3] = h->map_wsu;
     g.offsets = offsets; g.tile_start = tiles_gu; g.G = h->G; g.E = c.E; g.T = T;
     g.n_kind[0] = c.I; g.n_kind[1] = c.I_shared;
@@ -470,6 +472,8 @@ int forward_impl(moe_handle* h, int T, const uint16_t* x, const uint16_t* residu
     if (h->S > 0 && !make_map(&g.mapA16[1], as, c.I_shared, srows, 16, eb)) return MOE_ECUDA;
     g.fp8 = f8;
     g.a_exp[0] = he; g.a_exp[1] = hse;
+    g.a_rows[0] = TK; g.a_rows[1] = h->S * T;
+    g.out_rows[0] = TK; g.out_rows[1] = h->S * T;
     g.mapB[0] = h->map_wd; g.mapB[2] = h->map_wsd;
     g.offsets = offsets; g.tile_start = tiles_dn; g.G = h->G; g.E = c.E; g.T = T;
     g.n_kind[0] = LW; g.n_kind[1] = c.D;
@@ -615,7 +619,8 @@ int moe_get_device_error(moe_handle* h, void* workspace, void* stream) {
   if (cudaMemcpyAsync(&e, workspace, 4, cudaMemcpyDeviceToHost, s) != cudaSuccess) return MOE_ECUDA;
   if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ECUDA;
   if (cudaMemsetAsync(workspace, 0, 4, s) != cudaSuccess) return MOE_ECUDA;
-  return e == kDevOk ? MOE_OK : MOE_ETIMEOUT;
+  if (e == kDevOk) return MOE_OK;
+  return e == kDevBadIndex ? MOE_EINDEX : MOE_ETIMEOUT;
 }
 
 int moe_reduce_partials_rows(int P, const moe_bf16* const* partials, const moe_bf16* residual,
@@ -891,6 +896,7 @@ int moe_ep_send(moe_handle* h, int T, const moe_ep_peers* peers, void* workspace
   a.rows = T * c.k;
   a.row_bytes = h->L * (h->fp8 ? 1 : 2);
   a.E = c.E; a.E_loc = h->E_loc; a.world = h->ep_world; a.rank = h->ep_rank;
+  a.cap = h->cap; a.err = reinterpret_cast<int*>(ws + L.err);
   const int grid = std::max(1, std::min((a.rows + 7) / 8, 4 * h->num_sms));
   return launch_ep_send(a, grid, static_cast<cudaStream_t>(stream)) == cudaSuccess ? MOE_OK : MOE_ECUDA;
 }
@@ -968,6 +974,8 @@ int moe_ep_experts(moe_handle* h, int T, const moe_ep_peers* peers, void* worksp
     g.inv_beta_g = 1.0f / c.situ_beta_gate; g.inv_beta_u = 1.0f / c.situ_beta_up;
     g.fp8 = f8;
     g.a_exp[0] = recv_exp; g.a_exp[1] = reinterpret_cast<const int8_t*>(ws + L.xqe);
+    g.a_rows[0] = static_cast<int>(cap); g.a_rows[1] = T;
+    g.out_rows[0] = static_cast<int>(cap); g.out_rows[1] = h->S * T;
     g.err = err; g.timeout_ns = h->timeout_ns;
     MOE_TRY(launch_grouped_gemm(kGateUp, g, pair_grid(h, bound(nt_gu, nt_gus)), s));
   }
@@ -1006,6 +1014,9 @@ int moe_ep_experts(moe_handle* h, int T, const moe_ep_peers* peers, void* worksp
     g.shared_out_stride = T;
     g.dest_row = reinterpret_cast<const int32_t*>(self + X.meta);
     g.ep = 1;
+    g.ep_world = h->ep_world;
+    g.a_rows[0] = static_cast<int>(cap); g.a_rows[1] = h->S * T;
+    g.out_rows[0] = c.T_max * c.k; g.out_rows[1] = h->S * T;
     for (int r = 0; r < h->ep_world; ++r)
       g.out_rank[r] = reinterpret_cast<float*>(static_cast<uint8_t*>(peers->xbuf[r]) + X.y);
     g.fp8 = f8;
@@ -1124,6 +1135,7 @@ const char* moe_status_string(int status) {
     case MOE_EUNSUPPORTED: return "unsupported shape";
     case MOE_ECUDA: return "CUDA error";
     case MOE_ETIMEOUT: return "device wait timed out";
+    case MOE_EINDEX: return "device index out of range (bounds-checked build)";
     default: return "unknown status";
   }
 }

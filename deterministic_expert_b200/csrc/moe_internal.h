@@ -76,6 +76,9 @@ struct GemmArgs {
   int out_bf16;           // down-mode output as bf16 instead of fp32 (latent projection)
   int fp8;                // expert GEMMs: A and B are E4M3 codes (kind::f8f6f4)
   int ep;                 // down, routed: dest_row = rank << 24 | row, stored at out_rank[rank]
+  int ep_world;           // ep: ranks
+  int a_rows[2];          // rows of each kind's A tensor (index checks; 0 = unchecked)
+  int out_rows[2];        // rows of each kind's output (per rank under ep)
   float* out_rank[8];     // ep: each rank's slot-row output base (addresses on this rank)
   const int8_t* a_exp[2]; // fp8: per kind, power-of-two exponent of each A row; the
                           // accumulator of row r is multiplied by 2^a_exp[kind][r]
@@ -173,10 +176,11 @@ struct DispatchArgs {
   int tile_m;             // rows per expert-GEMM tile (256: a CTA pair)
   int32_t* dest_row;      // [T * k]
   int32_t* src_token;     // [T * k]
+  int* err;               // device error word (index checks)
 };
 cudaError_t launch_dispatch(const DispatchArgs& a, cudaStream_t s);
-cudaError_t launch_gather_rows(const void* src, const int32_t* src_row, int rows, int row_bytes, void* dst,
-                               const int8_t* src_exp, int8_t* dst_exp, cudaStream_t s);
+cudaError_t launch_gather_rows(const void* src, int src_rows, const int32_t* src_row, int rows, int row_bytes,
+                               void* dst, const int8_t* src_exp, int8_t* dst_exp, int* err, cudaStream_t s);
 
 // ------------------------------------------------------- expert parallelism
 struct EpSendArgs {
@@ -190,6 +194,8 @@ struct EpSendArgs {
   const int32_t* src_token;  // [rows] grouped row -> token
   const int32_t* dest_row;   // [rows] grouped row -> token * k + slot
   int rows, row_bytes, E, E_loc, world, rank;
+  long long cap;             // rows of each rank's receive buffers
+  int* err;                  // device error word (index checks)
 };
 cudaError_t launch_ep_send(const EpSendArgs& a, int grid, cudaStream_t s);
 

@@ -63,7 +63,9 @@ typedef enum {
   MOE_EWORKSPACE = -3,    /* workspace smaller than moe_workspace_size()            */
   MOE_EUNSUPPORTED = -4,  /* shape outside the limits above                         */
   MOE_ECUDA = -5,         /* a CUDA runtime call failed (launch, copy, allocation)  */
-  MOE_ETIMEOUT = -6       /* a device-side wait gave up (see moe_get_device_error)  */
+  MOE_ETIMEOUT = -6,      /* a device-side wait gave up (see moe_get_device_error)  */
+  MOE_EINDEX = -7         /* a device-side index check failed (only in a library
+                             built with MOE_CHECK_BOUNDS; see moe_get_device_error)  */
 } moe_status;
 
 typedef enum {

@@ -22,6 +22,18 @@ def test_every_declared_symbol_is_exported():
         assert hasattr(lib, n), n
 
 
+def test_bounds_checked_build_exports_the_same_symbols():
+    """The MOE_CHECK_BOUNDS build (libmoe_checked.so) is the same ABI."""
+    import os
+    path = os.path.join(os.path.dirname(moe.LIB_PATH), "libmoe_checked.so")
+    assert os.path.exists(path), "build libmoe_checked.so with __graft_entry__.build()"
+    checked = ctypes.CDLL(path)
+    for n in declared_functions():
+        assert hasattr(checked, n), n
+    checked.moe_status_string.restype = ctypes.c_char_p
+    assert b"index" in checked.moe_status_string(moe.MOE_EINDEX)
+
+
 def test_status_strings():
     assert moe.status_string(0) == "ok"
     assert "timed out" in moe.status_string(moe.MOE_ETIMEOUT)
