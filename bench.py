@@ -5,7 +5,8 @@
                     [--workload NAME] [--T TOKENS] [--no-cpu-baseline]
 
 --workload picks another workload (v3_shaped, skew_zipf, skew_hash,
-fine_grained_situ, latent_situ, fine_grained_fp8, tiny, tiny_fp8, or skew_epilogue for the 8-partial
+fine_grained_situ, latent_situ, fine_grained_fp8, latent_situ_fp8, tiny, tiny_fp8,
+or skew_epilogue for the 8-partial
 reduce + residual + RMSNorm); --T overrides the batch size (the decode sweep
 is --T 1, 8, 64, 128, 512 on the fine-grained weights).
 

@@ -44,7 +44,7 @@ size_t align256(size_t b) { return (b + 255) & ~static_cast<size_t>(255); }
 struct Layout {
   size_t err, xn, logits, tidx, tw, bcount, counts, offsets, tiles_gu, tiles_dn, dest, src,
       xp, h, hs, y, ys, z, agg, ylat, xq, xqe, xpe, hq, hqs, he, hse,
-      hr, hqr, her, epoff, eptg, eptd, eprows, total;   // hr..eprows: expert parallelism
+      hr, hqr, her, epoff, eptg, eptd, eprows, zq, zqe, total;   // hr..eprows: expert parallelism
 };
 
 Layout layout(const moe_handle* h, int T) {
@@ -97,6 +97,9 @@ Layout layout(const moe_handle* h, int T) {
   L.eptg = take(ep ? gl * 4 : 0);
   L.eptd = take(ep ? gl * 4 : 0);
   L.eprows = take(ep ? 4 : 0);
+  // E4M3 copy of the latent input z (latent width with E4M3 experts).
+  L.zq = take(lat ? f * Tz * Lw : 0);
+  L.zqe = take(lat ? f * Tz : 0);
   L.total = off;
   return L;
 }
@@ -198,7 +201,7 @@ int validate_config(const moe_config* c, const moe_weights* w) {
   if (c->ep_world > 1 && static_cast<long long>(c->ep_world) * c->T_max * c->k >= (1ll << 24))
     return MOE_EUNSUPPORTED;   // return addresses keep the row in 24 bits
   if (c->weight_format == MOE_WEIGHTS_FP8 &&
-      (c->D % 128 || c->I % 128 || (c->n_shared > 0 && c->I_shared % 128) || c->latent > 0))
+      (c->D % 128 || c->I % 128 || (c->n_shared > 0 && c->I_shared % 128) || c->latent % 128))
     return MOE_EUNSUPPORTED;
   if (c->D > 16384 || c->E > 256 || c->k > c->E || c->k > 16 || c->n_shared > 8 || c->T_max > (1 << 20))
     return MOE_EUNSUPPORTED;
@@ -354,6 +357,10 @@ int forward_impl(moe_handle* h, int T, const uint16_t* x, const uint16_t* residu
     prof.begin(8);
     const int r = dense_gemm(xn, c.D, h->map_pd, LW, h->bn_pd, zb, 1);
     if (r != MOE_OK) return r;
+    // E4M3 experts read z as E4M3 rows with their exponents, like xn.
+    if (f8)
+      MOE_TRY(launch_quant_rows(zb, T, LW, ws + L.zq, reinterpret_cast<int8_t*>(ws + L.zqe), nullptr, 0, 0,
+                                nullptr, nullptr, nullptr, s));
     prof.end(8);
     xe = zb;
   }
@@ -409,7 +416,9 @@ int forward_impl(moe_handle* h, int T, const uint16_t* x, const uint16_t* residu
 
   // 4. grouped A rows of the routed experts
   prof.begin(4);
-  if (f8) MOE_TRY(launch_gather_rows(xq, T, src, TK, LW, xp, xqe, xpe, err, s));
+  if (f8 && lat)
+    MOE_TRY(launch_gather_rows(ws + L.zq, T, src, TK, LW, xp, reinterpret_cast<int8_t*>(ws + L.zqe), xpe, err, s));
+  else if (f8) MOE_TRY(launch_gather_rows(xq, T, src, TK, LW, xp, xqe, xpe, err, s));
   else MOE_TRY(launch_gather_rows(xe, T, src, TK, LW * 2, xp, nullptr, nullptr, err, s));
   prof.end(4);
 
@@ -806,7 +815,8 @@ int moe_forward_launch_count(const moe_handle* h, int T) {
   if (!h || T < 0) return -1;
   if (T == 0) return 0;
   const int base = 8 + (h->cfg.latent > 0 ? 3 : 0)   // latent: two projections and the latent sum
-                   + (h->fp8 ? 1 : 0);                // E4M3: quantisation of h
+                   + (h->fp8 ? 1 : 0)                 // E4M3: quantisation of h
+                   + (h->fp8 && h->cfg.latent > 0 ? 1 : 0);   // ... and of z
   return h->cfg.router == MOE_ROUTER_HASH ? base - 1 : base;  // hash routing: no router GEMM
 }
 

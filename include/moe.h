@@ -99,8 +99,9 @@ typedef enum moe_weight_format {
                             code = E4M3 round-to-nearest-even of value / 2^e; the
                             row's accumulators are multiplied by 2^e.  The gate/up
                             input is xn (after its bf16 rounding), the down input
-                            is h.  The router GEMM stays bf16.  Needs D, I and
-                            I_shared multiples of 128 and latent == 0.              */
+                            is h (with a latent width, the routed experts' input
+                            is z).  The router GEMM and the latent projections stay
+                            bf16.  Needs D, I, I_shared and latent multiples of 128. */
 } moe_weight_format;
 
 typedef struct moe_config {

@@ -105,7 +105,9 @@ EPILOGUE_T = 16384
 EPILOGUE_D = 4096
 EPILOGUE_SIGMA = 1.0 / 8.0
 
-CONFIGS = {c.name: c for c in (C1, C2, C3, C5, C5H, C2S, C6, C1F, C2F)}
+# The latent workload with FP4 expert weights (routed and shared).
+C6F = dataclasses.replace(C6, name="latent_situ_fp8", weight_format=1)
+CONFIGS = {c.name: c for c in (C1, C2, C3, C5, C5H, C2S, C6, C1F, C2F, C6F)}
 
 _ZIPF_FILE = os.path.join(os.path.dirname(os.path.abspath(__file__)), "zipf_beta.json")
 ZIPF_S = 1.2
@@ -251,5 +253,5 @@ def pretty(cfg: MoEConfig) -> str:
             f"shared={cfg.n_shared}x{cfg.I_shared}{act}")
 
 
-__all__ = ["MoEConfig", "C1", "C1F", "C2", "C2F", "C2S", "C3", "C4_T", "C5", "C5H", "C6", "CONFIGS", "STREAM", "SEED",
+__all__ = ["MoEConfig", "C1", "C1F", "C2", "C2F", "C2S", "C3", "C4_T", "C5", "C5H", "C6", "C6F", "CONFIGS", "STREAM", "SEED",
            "host_bf16", "host_router_bias", "host_token_ids", "moe_flops", "math"]

@@ -204,3 +204,12 @@ def test_fp8_situ_parity(torch_cuda):
     same = check_routing(out, ref)
     check_outputs(out, ref, same_rows=same)
     _fp8_stage_checks(run, out, ref, hw, torch_cuda)
+
+
+def test_fp8_latent_situ_parity(torch_cuda):
+    """FP4 expert weights with a latent width (the routed experts read z as E4M3
+    rows, the shared expert xn) and SiTU-GLU units, on a 512-token batch."""
+    from test_gpu_layer import _latent_parity
+    cfg = dataclasses.replace(W.C6F, T=512)
+    run = Run(cfg)
+    _latent_parity(run, cfg, torch_cuda)

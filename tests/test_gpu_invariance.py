@@ -27,7 +27,7 @@ def torch_cuda():
 
 @pytest.mark.parametrize("name,splits", [("tiny", 7), ("fine_grained", 4), ("skew_hash", 3),
                                          ("fine_grained_situ", 5), ("latent_situ", 4),
-                                         ("tiny_fp8", 6), ("fine_grained_fp8", 4)])
+                                         ("tiny_fp8", 6), ("fine_grained_fp8", 4), ("latent_situ_fp8", 3)])
 def test_splits_permutation_repeats(torch_cuda, name, splits):
     torch = torch_cuda
     cfg = W.CONFIGS[name]
