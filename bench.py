@@ -313,7 +313,7 @@ def run_epilogue(a):
     stream = torch.cuda.current_stream()
     # N > 1 (N dividing 8): tensor parallel, as in the Fireworks parity post
     # (Trap 1, one reduction order on every rank).  Rank r holds
-    # partials r*8/N .. (r+1)*8/N - 1 in symmetric memory; each step is one
+    # partials r*8/N .. (r+1)*8/N - 1 in exported peer memory; each step is one
     # TPAllReduceNorm call (device barrier, one kernel reducing this rank's rows
     # over every rank's partials and storing them to every rank, barrier).
     tp = None
