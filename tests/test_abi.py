@@ -95,3 +95,42 @@ def test_weight_size_mismatch_is_refused():
     w = {"router_bias": torch.empty(8, dtype=torch.bfloat16)}
     with pytest.raises(ValueError):
         moe.MoELayer(cfg, w)
+
+
+def test_header_is_plain_c_and_links(tmp_path):
+    """include/moe.h compiles as C99 and a C program links against libmoe.so
+    and calls entry points that need no GPU (status strings, argument
+    checks): the boundary is a real C ABI, not a Python-only one."""
+    import os
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "abi.c"
+    src.write_text(r'''
+#include <stdio.h>
+#include <string.h>
+#include "moe.h"
+int main(void) {
+  moe_config cfg;
+  moe_weights w;
+  moe_handle* h = 0;
+  memset(&cfg, 0, sizeof cfg);
+  memset(&w, 0, sizeof w);
+  if (strcmp(moe_status_string(MOE_OK), "ok") != 0) return 1;
+  if (moe_init(&cfg, &w, &h) != MOE_EINVAL || h != 0) return 2;       /* D = 0: refused before CUDA */
+  if (moe_workspace_size(0, 16) != 0) return 3;
+  if (moe_ep_exchange_size(0) != 0) return 4;
+  if (moe_quantize_weights_fp4(0, 0, 0, 1, 32, 0) != MOE_EINVAL) return 5;
+  printf("%s\n", moe_status_string(MOE_EINDEX));
+  return 0;
+}
+''')
+    lib_dir = os.path.dirname(moe.LIB_PATH)
+    inc = os.path.dirname(moe.HEADER_PATH)
+    exe = tmp_path / "abi"
+    subprocess.check_call(["gcc", "-std=c99", "-Wall", "-Werror", "-I", inc, str(src), "-o", str(exe),
+                           "-L", lib_dir, "-l:libmoe.so", "-Wl,-rpath," + lib_dir])
+    out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert out.returncode == 0, (out.returncode, out.stderr)
+    assert "index" in out.stdout
