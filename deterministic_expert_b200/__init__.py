@@ -553,15 +553,20 @@ def _ep_call(name, *args):
 
 
 class _EPRank:
-    """One expert-parallel rank: its handle, workspace and exchange buffer."""
+    """One expert-parallel rank: its handle, workspace and exchange buffer.
+    ``own_copy``: keep a private copy of this rank's expert block (so the full
+    weight tensors can be freed) instead of views into them."""
 
-    def __init__(self, cfg: LayerConfig, weights: dict, rank: int, world: int, device):
+    def __init__(self, cfg: LayerConfig, weights: dict, rank: int, world: int, device, own_copy: bool = False):
         import dataclasses
 
         import torch
         self.rank = rank
         self.cfg = dataclasses.replace(cfg, ep_world=world, ep_rank=rank)
-        self.layer = MoELayer(self.cfg, shard_expert_weights(weights, world, rank))
+        shard = shard_expert_weights(weights, world, rank)
+        if own_copy:
+            shard = {n: (t.clone() if n in ("w_gate", "w_up", "w_down") else t) for n, t in shard.items()}
+        self.layer = MoELayer(self.cfg, shard)
         L = lib()
         L.moe_ep_exchange_size.restype = ctypes.c_size_t
         L.moe_ep_exchange_size.argtypes = [ctypes.c_void_p]
@@ -656,8 +661,9 @@ class EPMoELayer:
     exchange buffer, mapped by every other rank (moe_peer_open; handles travel
     over the process group).  A step is the four phases on the caller's
     stream with a device barrier (bounded; ``check()`` reports a time-out)
-    after route, send and experts.  ``weights`` holds all E routed experts (only
-    this rank's block is kept).  ``close()`` (collective) releases the memory."""
+    after route, send and experts.  ``weights`` holds all E routed experts; the
+    rank keeps its own copy of its block, so the caller may free the rest.
+    ``close()`` (collective) releases the memory."""
 
     _FLAGS = 4096
 
@@ -668,7 +674,7 @@ class EPMoELayer:
         self.world = dist.get_world_size(group)
         self.rank = dist.get_rank(group)
         dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
-        self.me = _EPRank(cfg, weights, self.rank, self.world, dev)
+        self.me = _EPRank(cfg, weights, self.rank, self.world, dev, own_copy=True)
         self.limit_us = barrier_timeout_ms * 1000
         with torch.cuda.device(dev):
             self._base, handle = peer_alloc(self._FLAGS + self.me.xbytes)
@@ -713,12 +719,15 @@ class EPMoELayer:
         return on, orr, idx, w
 
     def check(self) -> None:
+        """Raise MoEError if a barrier wait gave up or a kernel reported a device
+        error (a bounded wait, or an index check in the checked build)."""
         e = int(self.err.item())
         self.err.zero_()
         if e:
             raise MoEError(MOE_ETIMEOUT, "EPMoELayer barrier")
-        if self.me.device_error() != MOE_OK:
-            raise MoEError(MOE_ETIMEOUT, "EPMoELayer device wait")
+        st = self.me.device_error()
+        if st != MOE_OK:
+            raise MoEError(st, "EPMoELayer device error")
 
     def close(self) -> None:
         import torch
