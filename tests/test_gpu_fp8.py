@@ -213,3 +213,25 @@ def test_fp8_latent_situ_parity(torch_cuda):
     cfg = dataclasses.replace(W.C6F, T=512)
     run = Run(cfg)
     _latent_parity(run, cfg, torch_cuda)
+
+
+@pytest.mark.parametrize("variant", ["hash", "sigmoid_clamp", "no_shared"])
+def test_fp8_layer_variants(torch_cuda, variant):
+    """E4M3 experts under the other router variants: hash routing, sigmoid
+    scores with a selection bias and tight SwiGLU clamps, no shared expert.
+    (A V3-shaped case is left out: the oracle's FP4 quantisation of its
+    7168 x 2048 expert matrices in fp64 takes tens of minutes.)"""
+    base = dataclasses.replace(W.C1F, T=300)
+    cfg = {
+        "hash": dataclasses.replace(base, router=W.ROUTER_HASH, k=3, name="tiny_fp8_hash"),
+        "sigmoid_clamp": dataclasses.replace(base, router=W.ROUTER_SIGMOID_BIAS, renormalize=1, routed_scale=2.5,
+                                             gate_clamp_max=0.05, up_clamp=0.05, bias="normal", bias_sigma=0.01,
+                                             name="tiny_fp8_sigmoid"),
+        "no_shared": dataclasses.replace(base, n_shared=0, name="tiny_fp8_noshared"),
+    }[variant]
+    run = Run(cfg)
+    out = run.forward(*run.inputs())
+    ref, hw = oracle_full(cfg)
+    same = check_routing(out, ref)
+    check_outputs(out, ref, same_rows=same)
+    _fp8_stage_checks(run, out, ref, hw, torch_cuda)
