@@ -24,6 +24,16 @@
  *   r0..r7 reduction ... same post, Trap 1 (the uniform r0 + r1 + ... + r7 order, fp32)
  *   full-K GEMMs ....... Meituan LongCat parity article, "为什么会不一致" (a full-K
  *                        computation instead of summing split partial results)
+ * Variants (moe_config fields):
+ *   activation ......... SiTU-GLU units instead of SwiGLU (linux.do post, "SiTU-GLU")
+ *   latent ............. router and routed experts at a latent width l, their sum
+ *                        projected back (linux.do post, "潜在MoE (Latent MoE)")
+ *   weight_format ...... FP4-valued expert weights stored as E4M3, E4M3 x E4M3 expert
+ *                        GEMMs (DeepSeek V4 infra notes, §6.2 FP4 QAT)
+ *   ep_world, ep_rank .. expert parallelism over ranks, phases moe_ep_* (§6.1 there:
+ *                        dispatch -> compute -> combine)
+ * Multi-GPU epilogue: moe_reduce_partials_rows over peer memory (moe_peer_*) is the
+ * tensor-parallel all-reduce + residual + RMSNorm in the fixed r0..r7 order.
  *
  * Determinism contract.  For every row t, out_norm[t], out_residual[t],
  * out_topk_idx[t] and out_topk_w[t] are bit-identical whatever T is, where
