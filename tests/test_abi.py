@@ -9,7 +9,8 @@ import deterministic_expert_b200 as moe
 
 
 def declared_functions():
-    src = open(moe.HEADER_PATH).read()
+    with open(moe.HEADER_PATH) as f:
+        src = f.read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
     return sorted(set(re.findall(r"^\s*(?:int|size_t|const char\*)\s+(moe_\w+)\s*\(", src, flags=re.M)))
 

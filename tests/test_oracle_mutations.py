@@ -88,7 +88,8 @@ MUTATIONS = {
 
 def mutated_module(name):
     old, new = MUTATIONS[name]
-    src = open(SRC).read()
+    with open(SRC) as f:
+        src = f.read()
     assert src.count(old) == 1, f"mutation {name}: anchor not found once in the oracle"
     mod = types.ModuleType(f"oracle_mutant_{name}")
     exec(compile(src.replace(old, new), f"<mutant {name}>", "exec"), mod.__dict__)
