@@ -394,6 +394,35 @@ def fp4_weights_as_fp8(w, block: int = FP4_BLOCK) -> np.ndarray:
     return dequantize_fp4(*quantize_weights_fp4(w, block), block)
 
 
+def e2m1_codes(q) -> np.ndarray:
+    """4-bit E2M1 code of FP4 values (sign bit 3, then the index of the
+    magnitude in E2M1_GRID: exponent bits 2-1, mantissa bit 0)."""
+    q = np.asarray(q, np.float64)
+    mag = np.abs(q)
+    idx = np.searchsorted(E2M1_GRID, mag)
+    if not np.array_equal(E2M1_GRID[np.minimum(idx, 7)], mag):
+        raise ValueError("not E2M1 values")
+    return (idx | np.where(np.signbit(q), 8, 0)).astype(np.uint8)
+
+
+def pack_fp4(q, s):
+    """Storage form of FP4 weights: two E2M1 codes per byte along the last axis
+    (element 2i in the low nibble, 2i + 1 in the high nibble) and the block
+    exponents s as int8.  Returns (packed uint8 [..., K / 2], s int8)."""
+    c = e2m1_codes(q)
+    return (c[..., 0::2] | (c[..., 1::2] << 4)).astype(np.uint8), np.asarray(s).astype(np.int8)
+
+
+def unpack_fp4(packed, s, block: int = FP4_BLOCK) -> np.ndarray:
+    """Inverse of pack_fp4 followed by dequantize_fp4: the FP8 values."""
+    packed = np.asarray(packed, np.uint8)
+    codes = np.empty(packed.shape[:-1] + (2 * packed.shape[-1],), np.uint8)
+    codes[..., 0::2] = packed & 0xF
+    codes[..., 1::2] = packed >> 4
+    q = np.where(codes & 8, -1.0, 1.0) * E2M1_GRID[codes & 7]
+    return dequantize_fp4(q, np.asarray(s, np.int64), block)
+
+
 def round_e4m3(x) -> np.ndarray:
     """Nearest E4M3 value (1 sign, 4 exponent bits with bias 7, 3 mantissa
     bits; subnormals m/8 * 2^-6; largest finite 448), ties to even; magnitudes

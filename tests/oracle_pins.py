@@ -613,6 +613,27 @@ def pin_fp4_weight_blocks(O):
     assert np.all(np.abs(wr - w8) <= step)   # worst gap on the grid is 2 units (between 4 and 6)
 
 
+def pin_fp4_packed_storage(O):
+    """The packed FP4 form: codes from the E2M1 bit layout (sign in bit 3,
+    exponent in bits 2-1 with bias 1, mantissa in bit 0), a hand-packed pair,
+    and the round trip master -> (packed, exponents) -> FP8 values."""
+    # Codes rebuilt from the bit layout, against the oracle's grid order.
+    for code in range(16):
+        sign, e, m = code >> 3, (code >> 1) & 3, code & 1
+        val = (m / 2.0) if e == 0 else (1.0 + m / 2.0) * 2.0 ** (e - 1)
+        val = -val if sign else val
+        assert int(O.e2m1_codes(np.array([val]))[0]) == (code if val != 0 or not sign else 8), code
+    # [1.5, -6, 0.5, 3]: codes 3, 15, 1, 5 -> bytes 0xF3, 0x51 (low nibble first).
+    packed, _ = O.pack_fp4(np.array([[1.5, -6.0, 0.5, 3.0]]), np.array([[0]]))
+    assert packed.tolist() == [[0xF3, 0x51]]
+    rng = np.random.default_rng(12)
+    w = rng.standard_normal((3, 96)) * 0.03
+    q, s_ = O.quantize_weights_fp4(w)
+    packed, s8 = O.pack_fp4(q, s_)
+    assert packed.shape == (3, 48) and s8.dtype == np.int8
+    assert np.array_equal(O.unpack_fp4(packed, s8), O.fp4_weights_as_fp8(w))
+
+
 def pin_fp8_activation_rows(O):
     """Hand-derived per-row activation scales and E4M3 codes, the scale being
     the smallest power of two that brings the row into +-448."""

@@ -81,6 +81,10 @@ MUTATIONS = {
     "down_input_not_quantised": ("return h, (qh @ Wd.T) * np.exp2(eh)[:, None]", "return h, h @ Wd.T"),
     "fp8_path_ignored": ("return expert_ffn_fp8 if int(getattr(cfg, \"weight_format\", WEIGHTS_BF16)) == WEIGHTS_FP8 else expert_ffn",
                          "return expert_ffn"),
+    "fp4_nibbles_swapped": ("return (c[..., 0::2] | (c[..., 1::2] << 4)).astype(np.uint8), np.asarray(s).astype(np.int8)",
+                            "return (c[..., 1::2] | (c[..., 0::2] << 4)).astype(np.uint8), np.asarray(s).astype(np.int8)"),
+    "fp4_sign_in_wrong_bit": ("return (idx | np.where(np.signbit(q), 8, 0)).astype(np.uint8)",
+                              "return (idx | np.where(np.signbit(q), 4, 0)).astype(np.uint8)"),
     "histogram_off_by_one": ("return np.bincount(np.asarray(idx).ravel(), minlength=E).astype(np.int64)",
                              "return np.bincount(np.asarray(idx).ravel() % max(E - 1, 1), minlength=E).astype(np.int64)"),
 }
