@@ -163,3 +163,28 @@ def test_ctypes_structs_match_the_c_layout(tmp_path):
         assert got[(cname, "size")] == ctypes.sizeof(ct), cname
         for fname, _ in ct._fields_:
             assert got[(cname, fname)] == getattr(ct, fname).offset, (cname, fname)
+
+
+def test_binding_argument_counts_match_the_header():
+    """Every ctypes argtypes list in the binding has as many entries as the
+    header declares parameters for that entry point."""
+    import inspect
+    with open(moe.HEADER_PATH) as f:
+        hdr = re.sub(r"/\*.*?\*/", "", f.read(), flags=re.S)
+    decl = {}
+    for m in re.finditer(r"^\s*(?:int|size_t|const char\*)\s+(moe_\w+)\s*\(([^;]*?)\)\s*;", hdr, flags=re.M | re.S):
+        decl[m.group(1)] = len([p for p in m.group(2).split(",") if p.strip() and p.strip() != "void"])
+    src = inspect.getsource(moe)
+    # "L.moe_x.argtypes = [...]" and "fn = L.moe_x" followed by "fn.argtypes = [...]"
+    found = {}
+    for m in re.finditer(r"\.(moe_\w+)\.argtypes\s*=\s*\[|fn = L\.(moe_\w+)\n(?:.*\n){0,3}?\s*fn\.argtypes\s*=\s*\[", src):
+        name = m.group(1) or m.group(2)
+        i, depth = m.end(), 1
+        while depth:
+            depth += {"[": 1, "]": -1}.get(src[i], 0)
+            i += 1
+        body = src[m.end():i - 1]
+        found[name] = len([x for x in re.split(r",(?![^\[]*\])", body) if x.strip()])
+    assert len(found) >= 25
+    for name, n in found.items():
+        assert decl.get(name) == n, (name, n, decl.get(name))
