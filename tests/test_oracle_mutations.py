@@ -6,6 +6,7 @@ the real oracle is never modified.
 import os
 import types
 
+import numpy as np
 import pytest
 
 import oracle_pins as P
@@ -106,7 +107,8 @@ def test_planted_mistake_is_caught(name):
     caught = []
     for pin in P.ALL_PINS:
         try:
-            pin(M)
+            with np.errstate(over="ignore", invalid="ignore", divide="ignore"):  # mutants may overflow
+                pin(M)
         except Exception as e:  # AssertionError, or a shape error from a wrong operand
             caught.append((pin.__name__, type(e).__name__))
     assert caught, f"no pin caught the planted mistake {name}"
