@@ -98,6 +98,26 @@ def test_weight_size_mismatch_is_refused():
         moe.MoELayer(cfg, w)
 
 
+def test_weight_format_and_expert_shard_checks():
+    """E4M3 expert weights must be byte tensors (bf16 ones are refused, and
+    E4M3 bytes under a bf16 configuration too); an expert-parallel rank's
+    routed matrices hold E / ep_world experts, the router all E."""
+    import torch
+    import deterministic_expert_b200 as moe
+    D, E, I = 256, 8, 128
+    fp8 = moe.LayerConfig(D=D, E=E, k=2, I=I, weight_format=moe.WEIGHTS_FP8)
+    with pytest.raises(ValueError):
+        moe.MoELayer(fp8, {"w_gate": torch.empty(E * I * D, dtype=torch.bfloat16)})
+    bf16 = moe.LayerConfig(D=D, E=E, k=2, I=I)
+    with pytest.raises(ValueError):
+        moe.MoELayer(bf16, {"w_gate": torch.empty(E * I * D, dtype=torch.uint8)})
+    ep = moe.LayerConfig(D=D, E=E, k=2, I=I, ep_world=4, ep_rank=1)
+    with pytest.raises(ValueError):   # all 8 experts given to a rank that holds 2
+        moe.MoELayer(ep, {"w_gate": torch.empty(E * I * D, dtype=torch.bfloat16)})
+    with pytest.raises(ValueError):   # the router is whole on every rank
+        moe.MoELayer(ep, {"w_router": torch.empty(2 * D, dtype=torch.bfloat16)})
+
+
 def test_header_is_plain_c_and_links(tmp_path):
     """include/moe.h compiles as C99 and a C program links against libmoe.so
     and calls entry points that need no GPU (status strings, argument
