@@ -143,7 +143,9 @@ typedef struct moe_config {
                           8, dividing E): rank r owns routed experts [r E/ep_world,
                           (r+1) E/ep_world) and its w_gate / w_up / w_down hold only
                           those; router and shared experts are whole on every rank.
-                          Such a handle runs the moe_ep_* phases, not moe_layer_forward */
+                          Such a handle runs the moe_ep_* phases, not moe_layer_forward.
+                          Not combined with a latent width (MOE_EUNSUPPORTED), and
+                          ep_world * T_max * k must stay below 2^24                   */
   int ep_rank;         /* this rank, 0 <= ep_rank < ep_world                             */
 } moe_config;
 
