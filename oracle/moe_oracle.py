@@ -50,11 +50,16 @@ The layer, in order:
 Precision.  Every floating-point step runs in fp64, on the bf16-rounded values
 the GPU path reads (x, residual, weights, xn between steps 1 and 2/6, h between
 the two expert matmuls).  Rounding to bf16 is done directly from fp64 (round to
-nearest, ties to even), never through fp32.  Two exceptions: step 9, whose
+nearest, ties to even), never through fp32.  One exception: step 9, whose
 precision the pages fix (both all-reduce orders accumulate in FP32, [FW] Trap
-1), is emulated in IEEE fp32 left to right; and the bf16 code of xn, which
-decides the routing (an integer), is decided in the kernel's precision
-(``rmsnorm_bf16_code``).
+1), is emulated in IEEE fp32 left to right.
+
+Forced routing.  ``moe_layer`` can take the top-k indices from the caller
+(``force_idx``) instead of choosing them, with the weights still computed from
+the oracle's own scores of those experts.  A token whose top-k is decided by a
+near tie (or by an xn element that sits on a bf16 rounding boundary) may
+legitimately route differently on another implementation; with its indices
+forced, the rest of the layer for that token can still be checked.
 
 Readings of points the pages leave open (each is also listed in the design
 notes): epsilon inside the square root; gains g_in = g_out = 1 unless given;
@@ -118,21 +123,11 @@ def rmsnorm(x, g, eps: float) -> np.ndarray:
     return np.asarray(g, dtype=np.float64) * (x / np.sqrt(ms + eps))
 
 
-def rmsnorm_bf16_code(x, g, eps: float) -> np.ndarray:
-    """xn = bf16(RMSNorm(x) * g), with the bf16 code decided in the kernel's
-    precision.  The code of xn decides the routing (an integer), so both
-    sides decide it the same way: the mean of squares in fp64 (exact to
-    ~2^-52 for bf16 inputs), the scale s = 1/sqrt(mean + eps) rounded once to
-    fp32, then y = (x * s) * g with two fp32 products (round to nearest), then
-    round to nearest even bf16.  eps is the fp32 value the kernel receives.
-    Away from bf16 rounding boundaries this equals round_bf16(rmsnorm(...)),
-    the plain fp64 definition ([LD] "RMSNorm before up-projection")."""
-    x = np.asarray(x, np.float64)
-    ms = np.mean(x * x, axis=-1, keepdims=True)
-    s = (1.0 / np.sqrt(ms + float(np.float32(eps)))).astype(np.float32)
-    y = np.multiply(x.astype(np.float32), s, dtype=np.float32)
-    y = np.multiply(y, np.asarray(g, np.float64).astype(np.float32), dtype=np.float32)
-    return round_bf16(y.astype(np.float64))
+def xn_bf16(x, g, eps: float) -> np.ndarray:
+    """xn = bf16(g * x / sqrt(mean(x^2) + eps)): the input RMSNorm of [LD]
+    "RMSNorm before up-projection" in fp64, rounded once to bf16 (the
+    activation the router and the expert matmuls read)."""
+    return round_bf16(rmsnorm(x, g, eps))
 
 
 # ------------------------------------------------------- 2-3. router, top-k
@@ -162,36 +157,38 @@ def sigmoid(z) -> np.ndarray:
     return 1.0 / (1.0 + np.exp(-np.asarray(z, np.float64)))
 
 
-def route_softmax(logits, k: int, renormalize: bool, routed_scale: float, logit_bias=None):
+def route_softmax(logits, k: int, renormalize: bool, routed_scale: float, logit_bias=None, idx=None):
     """Softmax router ([V4] §2.2: Linear -> logits -> softmax weights -> top-k).
 
     Optional logit bias b (a per-expert offset added to the logits, used for
     the skewed workload).  Keys are the probabilities p; weights are p_j,
     divided by the sum over the chosen k when ``renormalize``, times
-    ``routed_scale``.  Returns (idx [T,k], w [T,k], keys [T,E]).
+    ``routed_scale``.  ``idx`` (optional, [T,k]) replaces the top-k choice.
+    Returns (idx [T,k], w [T,k], keys [T,E]).
     """
     z = np.asarray(logits, np.float64)
     if logit_bias is not None:
         z = z + np.asarray(logit_bias, np.float64)
     p = softmax(z)
-    idx = topk_desc(p, k)
+    idx = topk_desc(p, k) if idx is None else np.asarray(idx, np.int64)
     w = np.take_along_axis(p, idx, axis=-1)
     if renormalize:
         w = w / np.sum(w, axis=-1, keepdims=True)
     return idx, w * routed_scale, p
 
 
-def route_sigmoid_bias(logits, bias, k: int, renormalize: bool, routed_scale: float):
+def route_sigmoid_bias(logits, bias, k: int, renormalize: bool, routed_scale: float, idx=None):
     """Sigmoid scores with a per-expert balancing bias ([DS] §6.3: upper layers
     keep "sigmoid + balance"; [LD] "QuantileBalancing": expert e enters token
     t's top-k when s_{t,e} + b_e exceeds the boundary).
 
     The bias only selects: keys are s + b, weights are the unbiased s_j,
     normalised over the chosen k when ``renormalize``, times ``routed_scale``.
+    ``idx`` (optional, [T,k]) replaces the top-k choice.
     """
     s = sigmoid(logits)
     keys = s + (0.0 if bias is None else np.asarray(bias, np.float64))
-    idx = topk_desc(keys, k)
+    idx = topk_desc(keys, k) if idx is None else np.asarray(idx, np.int64)
     w = np.take_along_axis(s, idx, axis=-1)
     if renormalize:
         w = w / np.sum(w, axis=-1, keepdims=True)
@@ -215,14 +212,17 @@ def route_hash(token_ids, E: int, k: int, mult: int, routed_scale: float):
     return idx.astype(np.int64), w, None
 
 
-def route(cfg, logits, bias, token_ids):
-    """Dispatch on the router variant; returns (idx, w, keys)."""
+def route(cfg, logits, bias, token_ids, force_idx=None):
+    """Dispatch on the router variant; returns (idx, w, keys).  ``force_idx``
+    ([T,k], optional) replaces the top-k choice; the weights are then those
+    the router gives the forced experts."""
     if cfg.router == ROUTER_SOFTMAX:
-        return route_softmax(logits, cfg.k, bool(cfg.renormalize), cfg.routed_scale, bias)
+        return route_softmax(logits, cfg.k, bool(cfg.renormalize), cfg.routed_scale, bias, force_idx)
     if cfg.router == ROUTER_SIGMOID_BIAS:
-        return route_sigmoid_bias(logits, bias, cfg.k, bool(cfg.renormalize), cfg.routed_scale)
+        return route_sigmoid_bias(logits, bias, cfg.k, bool(cfg.renormalize), cfg.routed_scale, force_idx)
     if cfg.router == ROUTER_HASH:
-        return route_hash(token_ids, cfg.E, cfg.k, cfg.hash_mult, cfg.routed_scale)
+        idx, w, keys = route_hash(token_ids, cfg.E, cfg.k, cfg.hash_mult, cfg.routed_scale)
+        return (idx if force_idx is None else np.asarray(force_idx, np.int64)), w, keys
     raise ValueError(f"unknown router {cfg.router}")
 
 
@@ -620,7 +620,7 @@ class FP4Weights:
         return self._q(("s", int(s)), self._master.shared(s))
 
 
-def moe_layer(cfg, W, x, residual, token_ids=None, rows=None) -> dict:
+def moe_layer(cfg, W, x, residual, token_ids=None, rows=None, force_idx=None) -> dict:
     """The whole layer.  Routing, histogram and permutation are computed for
     every token; the experts, combine and epilogue for ``rows`` (all tokens
     when None).  ``cfg`` carries D, E, k, I, n_shared, I_shared, router,
@@ -630,6 +630,10 @@ def moe_layer(cfg, W, x, residual, token_ids=None, rows=None) -> dict:
     weight_format (WEIGHTS_FP8: the expert weights in ``W`` are FP8 values, as
     fp4_weights_as_fp8 gives, and the experts run expert_ffn_fp8).
 
+    ``force_idx`` ([T,k] expert indices, optional) replaces the top-k choice
+    of every token; the weights are still the router's own for those experts,
+    and ``margin`` stays that of the oracle's own choice.
+
     Latent MoE ([LD] "潜在MoE" and its K3 flow): the router and the routed
     experts read z = latent_down(xn) (width l), the routed experts' weighted sum
     is projected back by latent_up, and the shared experts keep the full width
@@ -637,13 +641,13 @@ def moe_layer(cfg, W, x, residual, token_ids=None, rows=None) -> dict:
     x = np.asarray(x, np.float64)
     T = x.shape[0]
     rows = np.arange(T) if rows is None else np.asarray(rows, np.int64)
-    xn = rmsnorm_bf16_code(x, W.g_in, cfg.eps)
+    xn = xn_bf16(x, W.g_in, cfg.eps)
     lat = int(getattr(cfg, "latent", 0) or 0)
     xe = latent_down(xn, W.w_proj_down) if lat else xn   # what the router and routed experts read
     logits = None
     if cfg.router != ROUTER_HASH:
         logits = router_logits(xe, W.w_router)
-    idx, w, keys = route(cfg, logits, W.router_bias, token_ids)
+    idx, w, keys = route(cfg, logits, W.router_bias, token_ids, force_idx)
     margin = topk_margin(keys, cfg.k)
     counts = expert_histogram(idx, cfg.E)
     offsets, perm_token, perm_slot, pos = stable_permute(idx, cfg.E)
@@ -679,17 +683,18 @@ def moe_layer(cfg, W, x, residual, token_ids=None, rows=None) -> dict:
                 out_norm=out_norm, out_residual=out_residual)
 
 
-def moe_layer_dense_masked(cfg, W, x, residual, token_ids=None) -> dict:
+def moe_layer_dense_masked(cfg, W, x, residual, token_ids=None, force_idx=None) -> dict:
     """Cross-check of the routed path: run every expert on every token, weight
     each output by the token's routing weight for that expert (0 when not
-    chosen) and sum over all experts.  Mathematically equal to ``moe_layer``."""
+    chosen) and sum over all experts.  Mathematically equal to ``moe_layer``
+    (up to the order of the routed sum)."""
     x = np.asarray(x, np.float64)
     T = x.shape[0]
-    xn = rmsnorm_bf16_code(x, W.g_in, cfg.eps)
+    xn = xn_bf16(x, W.g_in, cfg.eps)
     lat = int(getattr(cfg, "latent", 0) or 0)
     xe = latent_down(xn, W.w_proj_down) if lat else xn
     logits = None if cfg.router == ROUTER_HASH else router_logits(xe, W.w_router)
-    idx, w, _ = route(cfg, logits, W.router_bias, token_ids)
+    idx, w, _ = route(cfg, logits, W.router_bias, token_ids, force_idx)
     mask = np.zeros((T, cfg.E))
     np.put_along_axis(mask, idx, w, axis=-1)
     acc = np.zeros((T, lat or cfg.D))

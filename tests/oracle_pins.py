@@ -86,26 +86,75 @@ def pin_rmsnorm_scale_invariance(O):
     assert np.allclose(np.sqrt(np.mean(a * a, axis=-1)), 1.0, rtol=1e-13)
 
 
-def pin_rmsnorm_bf16_code(O):
+def pin_xn_bf16_by_hand(O):
     # By hand: [3,4], eps 1e-6: 3/sqrt(12.5) = 0.848528 -> 434 * 2^-9; 4/sqrt(12.5) = 1.131371 -> 145 * 2^-7.
-    assert np.array_equal(O.rmsnorm_bf16_code(np.array([[3.0, 4.0]]), np.ones(2), 1e-6)[0],
+    assert np.array_equal(O.xn_bf16(np.array([[3.0, 4.0]]), np.ones(2), 1e-6)[0],
                           [434 * 2.0 ** -9, 145 * 2.0 ** -7])
     # eps = 1 sits inside the root: 3/sqrt(13.5) = 0.816497 -> 418 * 2^-9; 4/sqrt(13.5) = 1.088662 -> 139 * 2^-7.
-    assert np.array_equal(O.rmsnorm_bf16_code(np.array([[3.0, 4.0]]), np.ones(2), 1.0)[0],
+    assert np.array_equal(O.xn_bf16(np.array([[3.0, 4.0]]), np.ones(2), 1.0)[0],
                           [418 * 2.0 ** -9, 139 * 2.0 ** -7])
     # Gains after the scale: 2 * 0.848528 = 1.697056 -> 217 * 2^-7; -0.5 * 1.131371 = -0.565685 -> -290 * 2^-9.
-    assert np.array_equal(O.rmsnorm_bf16_code(np.array([[3.0, 4.0]]), np.array([2.0, -0.5]), 0.0)[0],
+    assert np.array_equal(O.xn_bf16(np.array([[3.0, 4.0]]), np.array([2.0, -0.5]), 0.0)[0],
                           [217 * 2.0 ** -7, -290 * 2.0 ** -9])
-    # Random rows: equal to the plain fp64 definition rounded once, except for
-    # rare values next to a bf16 rounding boundary, which differ by one bf16 step.
-    rng = np.random.default_rng(11)
-    x = O.round_bf16(rng.standard_normal((64, 2048)))
-    g = O.round_bf16(1 + 0.1 * rng.standard_normal(2048))
-    a = O.rmsnorm_bf16_code(x, g, 1e-6)
-    b = O.round_bf16(O.rmsnorm(x, g, float(np.float32(1e-6))))
-    d = a != b
-    assert d.mean() < 1e-3
-    assert np.all(np.abs(a[d] - b[d]) <= np.abs(b[d]) * 2.0 ** -7 * 1.0001)
+
+
+def _bf16_mag_value(m):
+    """Exact value (a Fraction) of the non-negative bf16 whose magnitude bits are m."""
+    from fractions import Fraction
+    return Fraction(float(np.array([m << 16], np.uint32).view(np.float32)[0]))
+
+
+def _is_correct_bf16(c, gx, S):
+    """Is the bf16 value c the round-to-nearest-even of v = gx / sqrt(S)?
+    Decided in exact rational arithmetic: v lies between the midpoints
+    m- < v < m+ around c  <=>  (m-)^2 S < gx^2 < (m+)^2 S (signs apart), and a
+    value exactly on a midpoint goes to the even code."""
+    from fractions import Fraction
+    bits = int(np.array([c], np.float32).view(np.uint32)[0] >> 16)
+    mag, neg = bits & 0x7FFF, bool(bits & 0x8000)
+    if gx == 0:
+        return mag == 0
+    if (gx < 0) != neg:
+        return False
+    lo = (_bf16_mag_value(mag - 1) + _bf16_mag_value(mag)) / 2 if mag > 0 else Fraction(0)
+    hi = (_bf16_mag_value(mag) + _bf16_mag_value(mag + 1)) / 2
+    a2 = gx * gx
+    even = mag % 2 == 0
+    below = lo * lo * S
+    above = hi * hi * S
+    ok_lo = a2 > below or (a2 == below and even)
+    ok_hi = a2 < above or (a2 == above and even)
+    return ok_lo and ok_hi
+
+
+def pin_xn_bf16_exact_at_rounding_boundaries(O):
+    """xn = bf16(g x / sqrt(mean(x^2) + eps)) rounded once from the exact value
+    ([LD] "RMSNorm before up-projection").  Rows are screened for elements that
+    lie within 2^-16 of a bf16 quantum from a rounding midpoint -- where any
+    intermediate rounding to fp32 (of the scale or of a product) can move the
+    value across the midpoint -- and every element of those rows is checked in
+    exact rational arithmetic."""
+    from fractions import Fraction
+    rng = np.random.default_rng(2024)
+    D, n = 256, 3000
+    x = O.round_bf16(rng.standard_normal((n, D)))
+    g = O.round_bf16(1 + 0.1 * rng.standard_normal(D))
+    eps = 1e-6
+    # Screen in fp64: distance from the nearest midpoint in units of the quantum.
+    v = g * x / np.sqrt(np.mean(x * x, axis=1, keepdims=True) + eps)
+    _, e = np.frexp(v)
+    t = np.ldexp(v, -(e.astype(np.int64) - 8))          # v in units of its bf16 quantum
+    dist = np.abs(t - np.floor(t) - 0.5)
+    rows = np.unique(np.nonzero(dist < 2.0 ** -16)[0])
+    assert len(rows) >= 8, len(rows)                     # enough boundary cases to test
+    xn = O.xn_bf16(x[rows], g, eps)
+    eps_q = Fraction(eps)
+    gq = [Fraction(float(gi)) for gi in g]
+    for ri, r in enumerate(rows):
+        xr = [Fraction(float(xi)) for xi in x[r]]
+        S = sum(xi * xi for xi in xr) / D + eps_q
+        for d in range(D):
+            assert _is_correct_bf16(xn[ri, d], gq[d] * xr[d], S), (int(r), d)
 
 
 # ------------------------------------------------------------------ SwiGLU
@@ -368,6 +417,37 @@ def pin_closed_form_layer(O):
     assert np.array_equal(out["out_norm"][0], _torch_bf16(r / rms))
     # Counts / permutation of the single routed row.
     assert list(out["counts"]) == [0, 1] and list(out["offsets"]) == [0, 0, 1]
+
+
+def pin_forced_routing(O):
+    """Forced indices replace the top-k choice; the weights stay the router's
+    own scores of the forced experts (worked by hand on the closed-form case)."""
+    cfg, W, x, residual = closed_form_case()
+    out = O.moe_layer(cfg, W, x, residual, force_idx=np.array([[0]]))
+    xn0, xn1 = 434 * 2.0 ** -9, 145 * 2.0 ** -7
+    # Expert 0 (all-zero weights) instead of expert 1: its output is 0; its
+    # weight is p_0 = 1/(1 + e^(xn1 - xn0)).
+    assert out["idx"][0, 0] == 0
+    assert abs(out["w"][0, 0] - 1.0 / (1.0 + math.exp(xn1 - xn0))) < 1e-15
+    silu = lambda a: a / (1.0 + math.exp(-a))  # noqa: E731
+    hs0 = float(_torch_bf16(silu(xn1) * xn0))
+    assert np.allclose(out["r"][0], [0.5, hs0 - 0.25], rtol=1e-15, atol=1e-16)
+    assert list(out["counts"]) == [1, 0]
+    # The margin still describes the oracle's own choice (expert 1 over 0).
+    p1 = 1.0 / (1.0 + math.exp(-(xn1 - xn0)))
+    assert abs(out["margin"][0] - (p1 - (1 - p1))) < 1e-15
+    # Forcing the oracle's own choice changes nothing; forcing the reversed
+    # slot order reverses the weights and reorders only the routed sum.
+    for router, extra in [(0, {}), (1, {"renormalize": 1, "routed_scale": 2.5}), (2, {})]:
+        cfg, W, xr, res, ids = small_random_case(O, router=router, **extra)
+        a = O.moe_layer(cfg, W, xr, res, ids)
+        b = O.moe_layer(cfg, W, xr, res, ids, force_idx=a["idx"])
+        assert np.array_equal(a["out_norm"], b["out_norm"]) and np.array_equal(a["w"], b["w"])
+        c = O.moe_layer(cfg, W, xr, res, ids, force_idx=a["idx"][:, ::-1])
+        assert np.array_equal(c["idx"], a["idx"][:, ::-1])
+        if router != 2:
+            assert np.array_equal(c["w"], a["w"][:, ::-1])
+        assert np.allclose(c["r"], a["r"], rtol=1e-12, atol=1e-12)
 
 
 # ---------------------------------------------------------- dense cross-check

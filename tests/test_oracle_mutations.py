@@ -18,10 +18,19 @@ MUTATIONS = {
     "eps_outside_sqrt": ("x / np.sqrt(ms + eps)", "x / (np.sqrt(ms) + eps)"),
     "gain_dropped": ("return np.asarray(g, dtype=np.float64) * (x / np.sqrt(ms + eps))",
                      "return (x / np.sqrt(ms + eps))"),
-    "code_eps_outside_sqrt": ("s = (1.0 / np.sqrt(ms + float(np.float32(eps)))).astype(np.float32)",
-                              "s = (1.0 / (np.sqrt(ms) + float(np.float32(eps)))).astype(np.float32)"),
-    "code_gain_dropped": ("    y = np.multiply(y, np.asarray(g, np.float64).astype(np.float32), dtype=np.float32)\n",
-                          ""),
+    # xn decided in a GPU kernel's fp32 precision (an fp32 scale and two fp32
+    # products before the bf16 rounding) instead of the fp64 definition.
+    "xn_kernel_precision": ("    return round_bf16(rmsnorm(x, g, eps))\n",
+                            "    x = np.asarray(x, np.float64)\n"
+                            "    s = (1.0 / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps)).astype(np.float32)\n"
+                            "    y = np.multiply(x.astype(np.float32), s, dtype=np.float32)\n"
+                            "    y = np.multiply(y, np.asarray(g, np.float64).astype(np.float32), dtype=np.float32)\n"
+                            "    return round_bf16(y.astype(np.float64))\n"),
+    "xn_not_rounded": ("    return round_bf16(rmsnorm(x, g, eps))\n", "    return rmsnorm(x, g, eps)\n"),
+    "forced_routing_ignored": ("idx = topk_desc(p, k) if idx is None else np.asarray(idx, np.int64)",
+                               "idx = topk_desc(p, k)"),
+    "forced_weights_of_natural_choice": ("    idx = topk_desc(p, k) if idx is None else np.asarray(idx, np.int64)\n    w = np.take_along_axis(p, idx, axis=-1)",
+                                         "    w = np.take_along_axis(p, topk_desc(p, k), axis=-1)\n    idx = topk_desc(p, k) if idx is None else np.asarray(idx, np.int64)"),
     "double_rounding_via_fp32": ("a = np.asarray(a, dtype=np.float64)\n    _, e",
                                  "a = np.asarray(a, dtype=np.float64).astype(np.float32).astype(np.float64)\n    _, e"),
     "topk_ascending": ("neg = np.where(np.isnan(keys), np.inf, -keys)",
