@@ -11,7 +11,7 @@ namespace moe {
 
 // ------------------------------------------------------------------ errors
 // Device error word values (first word of every forward's workspace).
-enum : int { kDevOk = 0, kDevTimeout = 1, kDevBadTile = 2, kDevBadIndex = 3 };
+enum : int { kDevOk = 0, kDevTimeout = 1, kDevBadIndex = 3 };
 
 // Index checks of a build with -DMOE_CHECK_BOUNDS: every index a kernel
 // computes from device data (expert ids, grouped rows, tile coordinates,
@@ -83,9 +83,9 @@ __device__ __forceinline__ float block_sum_fixed(float v, float* smem_warps /*[k
 }
 
 // The same fixed tree in fp64 (used for the input RMSNorm's sum of squares,
-// whose bf16 output feeds the router: with an fp64 sum the fp32 scale is the
-// correctly rounded value of 1/sqrt(mean + eps) whatever the summation order,
-// so the bf16 code of every element is decided from a well-defined fp32 scale).
+// whose bf16 output feeds the router: an fp64 sum of the exact squares of bf16
+// values is itself exact to ~2^-52, so the bf16 code of every element of xn
+// follows the exact value of the definition).
 __device__ __forceinline__ double block_sum_fixed_f64(double v, double* smem_warps) {
   v += __shfl_xor_sync(0xffffffffu, v, 16);
   v += __shfl_xor_sync(0xffffffffu, v, 8);

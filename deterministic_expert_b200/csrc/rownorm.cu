@@ -8,10 +8,12 @@
 // parity post (Chinese translation), Trap 2, says must not change with the
 // launch shape.  Nothing here depends on T.
 //
-//   rmsnorm_rows     (also zeroes the routing histogram) xn = bf16((x * s) * g), s = fp32(1 / sqrt(mean(x^2) + eps)) from an
-//                    fp64 sum of squares (same fixed tree) so that the bf16 code of
-//                    xn, which decides the routing, is fixed by a well-defined fp32
-//                    scale (linux.do post on MoE variants, "RMSNorm before up-projection")
+//   rmsnorm_rows     (also zeroes the routing histogram) xn = bf16(g x / sqrt(mean(x^2) + eps))
+//                    (linux.do post on MoE variants, "RMSNorm before up-projection"),
+//                    evaluated in fp64 (sum of squares over the same fixed tree, scale
+//                    and products) and rounded once to bf16, so the bf16 code of xn,
+//                    which decides the routing, is that of the exact value except
+//                    within ~2^-52 of a rounding midpoint
 //                    (with FP8 expert weights also an E4M3 copy of xn with one
 //                    power-of-two scale per row; quant_rows does the same for h)
 //   combine_norm     acc = sum_j w_j y_j (slot order) + sum_s y_s; r = acc + residual;
@@ -76,6 +78,26 @@ __device__ __forceinline__ float inv_rms(float ss, int D, float eps) {
   return 1.0f / sqrtf(ss / static_cast<float>(D) + eps);
 }
 
+// bf16 code of an fp64 value, round to nearest, ties to even, in one step
+// (rounding to fp32 first could land a value exactly on a bf16 midpoint and
+// round it a second time).  Normal range: keep the top 7 of the 52 fraction
+// bits with the usual add-half-minus-one-plus-lsb carry, then move the
+// exponent bias from 1023 to 127; overflow gives infinity.  Below 2^-126 the
+// bf16 spacing is 2^-133, so the code is the magnitude in units of 2^-133
+// rounded to an integer (an exact scaling, then rint, which rounds half to even).
+__device__ __forceinline__ uint32_t f64_to_bf16_rne(double v) {
+  const unsigned long long b = static_cast<unsigned long long>(__double_as_longlong(v));
+  const uint32_t sign = static_cast<uint32_t>(b >> 48) & 0x8000u;
+  const unsigned long long mag = b & 0x7FFFFFFFFFFFFFFFull;
+  if (mag > 0x7FF0000000000000ull) return 0x7FC0u;          // NaN
+  if ((mag >> 52) >= 897ull) {                                // |v| >= 2^-126
+    const unsigned long long r = (mag + 0xFFFFFFFFFFFull + ((mag >> 45) & 1ull)) >> 45;
+    const unsigned long long code = r - (896ull << 7);
+    return sign | static_cast<uint32_t>(code >= 0x7F80ull ? 0x7F80ull : code);
+  }
+  return sign | static_cast<uint32_t>(rint(fabs(v) * 0x1p133));
+}
+
 // Largest value of amax over the block (max is exact, so any order gives the
 // same result); every thread receives it.
 __device__ __forceinline__ float block_max(float amax, float* redf) {
@@ -134,11 +156,11 @@ __global__ void __launch_bounds__(kRowThreads) k_rmsnorm_rows(const uint16_t* __
         ss = fma(static_cast<double>(v[i].v[q]), static_cast<double>(v[i].v[q]), ss);
     }
   }
-  // The squares of bf16 values are exact in fp64 and the fp64 sum is exact to
-  // ~2^-52, so the scale below is the correctly rounded fp32 value of
-  // 1 / sqrt(mean(x^2) + eps); xn = bf16((x * scale) * g) in fp32.
+  // The squares of bf16 values are exact in fp64 and their fp64 sum is exact
+  // to ~2^-52 relative; the scale and both products are fp64 too, and the
+  // result is rounded once to bf16.
   const double ms = block_sum_fixed_f64(ss, red) / static_cast<double>(D);
-  const float inv = static_cast<float>(1.0 / sqrt(ms + static_cast<double>(eps)));
+  const double inv = 1.0 / sqrt(ms + static_cast<double>(eps));
   uint16_t* yr = y + row * D;
   float amax = 0.f;
 #pragma unroll
@@ -146,15 +168,18 @@ __global__ void __launch_bounds__(kRowThreads) k_rmsnorm_rows(const uint16_t* __
     const int c = threadIdx.x + i * kRowThreads;
     if (c < nch) {
       const f8 gg = ld_bf16x8(g + 8 * c);
-      float o[8];
+      uint32_t o[8];
 #pragma unroll
-      for (int q = 0; q < 8; ++q) o[q] = v[i].v[q] * inv * gg.v[q];
-      st_bf16x8(yr + 8 * c, o);
+      for (int q = 0; q < 8; ++q)
+        o[q] = f64_to_bf16_rne(__dmul_rn(__dmul_rn(static_cast<double>(v[i].v[q]), inv),
+                                         static_cast<double>(gg.v[q])));
+      *reinterpret_cast<uint4*>(yr + 8 * c) =
+          make_uint4(o[0] | (o[1] << 16), o[2] | (o[3] << 16), o[4] | (o[5] << 16), o[6] | (o[7] << 16));
       if (yq != nullptr) {
         // Keep the bf16 values (what the expert GEMMs read) for the E4M3 copy.
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
-          v[i].v[q] = bf16_lo(pack_bf16x2(o[q], 0.f));
+          v[i].v[q] = bf16_lo(o[q]);
           amax = fmaxf(amax, fabsf(v[i].v[q]));
         }
       }
