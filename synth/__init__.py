@@ -53,6 +53,7 @@ def _h():
         lib.syn_draw.argtypes = [u64, u64]
         lib.syn_normal_bf16.argtypes = [u64, u64, u64, f32, vp]
         lib.syn_normal_f32.argtypes = [u64, u64, u64, f32, vp]
+        lib.syn_normal_bf16_as_f64.argtypes = [u64, u64, u64, f32, vp]
         lib.syn_uniform_int.argtypes = [u64, u64, u64, ctypes.c_uint32, vp]
         lib.syn_splitmix64_sequence.argtypes = [u64, u64, vp]
         _host = lib
@@ -94,6 +95,14 @@ def normal_bf16(k: int, start: int, count: int, sigma: float) -> np.ndarray:
 def normal_f32(k: int, start: int, count: int, sigma: float) -> np.ndarray:
     out = np.empty(count, np.float32)
     _h().syn_normal_f32(k, start, count, sigma, out.ctypes.data)
+    return out
+
+
+def normal_bf16_as_f64(k: int, start: int, count: int, sigma: float) -> np.ndarray:
+    """The draws of normal_bf16, each bf16 value widened exactly to float64."""
+    out = np.empty(count, np.float64)
+    if count:
+        _h().syn_normal_bf16_as_f64(k, start, count, sigma, out.ctypes.data)
     return out
 
 

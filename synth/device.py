@@ -115,7 +115,7 @@ class HostWeights:
 
     def _slice(self, name, index, rows, cols):
         n = rows * cols
-        return f64(W.host_bf16(self.cfg, name, start=index * n, count=n)).reshape(rows, cols)
+        return W.host_f64(self.cfg, name, start=index * n, count=n).reshape(rows, cols)
 
     def routed(self, e):
         key = ("r", int(e))
@@ -143,6 +143,6 @@ def host_rows(cfg, name, rows, T=None):
     D = cfg.D
     rows = np.asarray(rows, np.int64)
     if len(rows) and np.all(np.diff(rows) == 1):
-        return f64(W.host_bf16(cfg, name, start=int(rows[0]) * D, count=len(rows) * D, T=T)).reshape(-1, D)
-    return np.stack([f64(W.host_bf16(cfg, name, start=int(r) * D, count=D, T=T)) for r in rows]) \
+        return W.host_f64(cfg, name, start=int(rows[0]) * D, count=len(rows) * D, T=T).reshape(-1, D)
+    return np.stack([W.host_f64(cfg, name, start=int(r) * D, count=D, T=T) for r in rows]) \
         if len(rows) else np.zeros((0, D))

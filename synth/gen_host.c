@@ -82,6 +82,19 @@ void syn_normal_bf16(uint64_t key, uint64_t start, uint64_t count, float sigma,
     out[j] = syn_f32_to_bf16_rne(syn_z(key, start + (uint64_t)j) * sigma);
 }
 
+/* The same bf16 draws, each widened exactly to double (a storage format only:
+ * the bf16 value placed in the upper half of an fp32 pattern, then converted). */
+void syn_normal_bf16_as_f64(uint64_t key, uint64_t start, uint64_t count, float sigma,
+                            double *out) {
+#pragma omp parallel for schedule(static)
+  for (int64_t j = 0; j < (int64_t)count; ++j) {
+    uint32_t u = (uint32_t)syn_f32_to_bf16_rne(syn_z(key, start + (uint64_t)j) * sigma) << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    out[j] = (double)f;
+  }
+}
+
 void syn_normal_f32(uint64_t key, uint64_t start, uint64_t count, float sigma,
                     float *out) {
 #pragma omp parallel for schedule(static)

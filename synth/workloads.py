@@ -16,7 +16,7 @@ import os
 
 import numpy as np
 
-from . import key, normal_bf16, normal_f32, uniform_int, _h  # noqa: F401
+from . import key, normal_bf16, normal_bf16_as_f64, normal_f32, uniform_int, _h  # noqa: F401
 
 SEED = 0
 
@@ -150,6 +150,17 @@ def host_bf16(cfg: MoEConfig, name: str, start: int = 0, count: int | None = Non
     cnt = n - start if count is None else count
     out = normal_bf16(k_(name), start, cnt, sigma)
     return out.reshape(shape) if (start == 0 and count is None) else out
+
+
+def host_f64(cfg: MoEConfig, name: str, start: int = 0, count: int | None = None,
+             T: int | None = None) -> np.ndarray:
+    """The values of host_bf16 widened to float64 (flat)."""
+    n = int(np.prod(tensor_shape(cfg, name, T)))
+    cnt = n - start if count is None else count
+    if name in ("g_in", "g_out"):
+        return np.ones(cnt)
+    sigma = cfg.x_sigma if name in ("x", "residual") else cfg.weight_sigma
+    return normal_bf16_as_f64(k_(name), start, cnt, sigma)
 
 
 def host_router_bias(cfg: MoEConfig) -> np.ndarray | None:

@@ -23,13 +23,12 @@ import dataclasses, numpy as np, torch
 import deterministic_expert_b200 as moe
 assert moe.LIB_PATH.endswith("libmoe_checked.so"), moe.LIB_PATH
 import sys; sys.path.insert(0, "tests")
-from gpu_util import Run, check_outputs, check_routing, oracle_full
+from gpu_util import Run, verify
 from synth import device as SD, workloads as W
 for cfg in (W.C1, W.C1F, dataclasses.replace(W.C1, T=129, n_shared=0)):
     run = Run(cfg)
     out = run.forward(*run.inputs())          # asserts device_error == 0
-    ref, _ = oracle_full(cfg)
-    check_outputs(out, ref, same_rows=check_routing(out, ref))
+    verify(run, out)
 cfg = W.C1.with_T(300)
 w = SD.device_weights(cfg)
 x, r, ids = SD.device_inputs(cfg, T=300)
@@ -63,9 +62,17 @@ for q, rk in enumerate(ep.ranks):
     rk.route(xs[q], None, moe._ptr(ep.xbuf[q]))
 torch.cuda.synchronize()
 # Rank 1 publishes impossible counts (its board is the first E int32 of its
-# exchange buffer): every other rank's destination rows for the experts after
-# the first of each owner now lie far past the receive buffers.
-ep.xbuf[1][:4 * cfg.E].view(torch.int32).fill_(1 << 16)
+# exchange buffer): 200 rows for every expert, where a rank has 100 (token,
+# slot) rows in all.  The destination rows computed from them run past each
+# owner's 400-row receive buffer, to row 487 at most on this routing (about
+# 380 expected from the other ranks' counts); every row stays inside the
+# owner's own exchange allocation (receive rows, their return addresses, then
+# the 100 KB of slot rows), so a send path whose check went missing would
+# overwrite memory this process owns instead of faulting the GPU.
+exch = ep.xbuf[1].numel()
+rows_in_alloc = exch // (cfg.D * 2)
+assert rows_in_alloc > 487 + 8, rows_in_alloc
+ep.xbuf[1][:4 * cfg.E].view(torch.int32).fill_(200)
 for q, rk in enumerate(ep.ranks):
     rk.send(50, ep.peers)
 torch.cuda.synchronize()                      # no CUDA error: the bad rows were skipped

@@ -2,9 +2,13 @@
 
 Inputs are the seeded synthetic workloads (both sides draw them from the same
 counter-based generator).  Floating-point outputs must satisfy
-max |gpu - oracle| / max(1, |oracle|) <= 2e-2 and a mean of the same <= 4e-3;
-integer stages (routing, histogram, permutation) must match exactly except on
-tokens whose top-k margin is below 1e-5 in the oracle's key space.
+max |gpu - oracle| / max(1, |oracle|) <= 2e-2 and a mean of the same <= 4e-3
+on every token; xn may differ from the oracle's by one bf16 step on at most
+1e-4 of its elements; integer stages (routing, histogram, permutation) must
+match exactly except on tokens whose top-k margin is below 1e-5 in the
+oracle's key space (near ties) or whose routing the oracle reproduces from the
+GPU's own xn (rounding-boundary flips).  Tokens routed differently are
+value-checked on the oracle with the GPU's indices forced.
 """
 import dataclasses
 
@@ -12,16 +16,10 @@ import numpy as np
 import pytest
 
 import oracle as O
-from gpu_util import Run, check_outputs, check_routing, np64, oracle_full, rel_err
+from gpu_util import Run, host_weights, np64, rel_err, verify
 from synth import workloads as W
 
 pytestmark = pytest.mark.gpu
-
-# Routing weights (in [0, 1]) inherit the logit differences of xn elements that
-# the fp32 kernel and the fp64 oracle round to neighbouring bf16 values: one
-# bf16 ulp (<= 2^-7 relative) times a router weight (|w| ~ 0.02 * 6 sigma)
-# per flipped element moves a logit by ~1e-3 at most, and a weight by less.
-W_TOL = 2e-3
 
 
 @pytest.fixture(scope="module")
@@ -62,13 +60,10 @@ def _views_np(run, T, ws, torch):
 
 
 def _stage_checks(run, out, ref, hw, torch):
-    """Intermediate stages against the oracle's own intermediates."""
+    """Intermediate stages against the oracle's own intermediates (xn itself is
+    checked by verify)."""
     c, T = run.cfg, run.T
     v = _views_np(run, T, out["ws"], torch)
-    # xn: the bf16 code is decided in the same precision on both sides
-    # (fp64 mean of squares, one fp32 scale, fp32 products), so it matches bit
-    # for bit.
-    assert np.array_equal(np64(v["xn"]), ref["xn"])
     if "logits" in v:
         e = np.abs(np64(v["logits"]) - ref["logits"])
         assert e.max() < 5e-3 * (1 + np.abs(ref["logits"]).max()), e.max()
@@ -101,12 +96,8 @@ def test_tiny_layer_parity_with_stages(torch_cuda):
     cfg = W.C1
     run = Run(cfg)
     out = run.forward(*run.inputs())
-    ref, hw = oracle_full(cfg)
-    same = check_routing(out, ref)
-    assert np.array_equal(out["counts"].cpu().numpy(), O.expert_histogram(out["idx"].cpu().numpy(), cfg.E))
-    check_outputs(out, ref, same_rows=same)
-    w = out["w"].cpu().numpy().astype(np.float64)
-    assert np.abs(w[same] - ref["w"][same]).max() < W_TOL
+    hw = host_weights(cfg)
+    ref, same, _ = verify(run, out, hw=hw)
     _stage_checks(run, out, ref, hw, torch_cuda)
 
 
@@ -114,11 +105,9 @@ def test_fine_grained_layer_parity(torch_cuda):
     cfg = W.C2
     run = Run(cfg)
     out = run.forward(*run.inputs())
-    ref, hw = oracle_full(cfg)
-    same = check_routing(out, ref)
-    check_outputs(out, ref, same_rows=same)
+    hw = host_weights(cfg)
+    ref, same, rep = verify(run, out, hw=hw)
     w = out["w"].cpu().numpy().astype(np.float64)
-    assert np.abs(w[same] - ref["w"][same]).max() < W_TOL
     assert np.allclose(w.sum(1), 1.0, atol=1e-5)  # renormalised
     _stage_checks(run, out, ref, hw, torch_cuda)
 
@@ -127,10 +116,7 @@ def test_fine_grained_layer_parity(torch_cuda):
 def test_ragged_and_tiny_batches(torch_cuda, T):
     cfg = dataclasses.replace(W.C1, T=T)
     run = Run(cfg)
-    out = run.forward(*run.inputs())
-    ref, _ = oracle_full(cfg)
-    same = check_routing(out, ref)
-    check_outputs(out, ref, same_rows=same)
+    verify(run, run.forward(*run.inputs()))
 
 
 @pytest.mark.parametrize("variant", ["all_experts", "no_shared", "hash_small", "sigmoid_clamp", "k1",
@@ -155,50 +141,23 @@ def test_layer_variants(torch_cuda, variant):
                                                situ_beta_up=0.5, name="situ_tight"),
     }[variant]
     run = Run(cfg)
-    out = run.forward(*run.inputs())
-    ref, _ = oracle_full(cfg)
-    same = check_routing(out, ref)
-    check_outputs(out, ref, same_rows=same)
+    verify(run, run.forward(*run.inputs()))
 
 
 def test_fine_grained_situ_parity(torch_cuda):
     """SiTU-GLU experts on the fine-grained shapes (a 512-token batch)."""
     cfg = dataclasses.replace(W.C2S, T=512)
     run = Run(cfg)
-    out = run.forward(*run.inputs())
-    ref, _ = oracle_full(cfg)
-    same = check_routing(out, ref)
-    check_outputs(out, ref, same_rows=same)
+    verify(run, run.forward(*run.inputs()))
 
 
 def _latent_parity(run, cfg, torch):
     """Latent layers: z = bf16(xn W_down^T) is rounded from fp32 on the GPU and
-    from fp64 in the oracle, so an element may land one bf16 step apart; the
-    routing is therefore checked against the oracle's router run on the GPU's
-    own z (the step's input), and the rest of the layer against the oracle."""
+    from fp64 in the oracle (verify allows single bf16 steps on under 1 % of
+    z); routing differences are classified on the GPU's own z, and every token
+    is value-checked."""
     out = run.forward(*run.inputs())
-    ref, hw = oracle_full(cfg)
-    T, c = cfg.T, cfg
-    v = run.layer.views(T, out["ws"])
-    ws = out["ws"]
-    off = v.z - ws.data_ptr()
-    z = ws[off:off + T * c.latent * 2].view(torch.bfloat16).reshape(T, c.latent)
-    zg = np64(z)
-    # Differences are single bf16 steps of the larger of the two values, or,
-    # where the dot product cancels to a tiny z, within the fp32 accumulation
-    # error of its terms (|x| ~ 1, |w| ~ 0.02, K = D).
-    dz = np.abs(zg - ref["z"])
-    big = np.maximum(np.abs(zg), np.abs(ref["z"]))
-    ulp = 2.0 ** (np.floor(np.log2(np.maximum(big, 1e-30))) - 7)
-    assert np.all(dz <= np.maximum(ulp * 1.0000001, 2.0 ** -16)), float(dz.max())
-    # The tensor cores' fp32 accumulation of the K = D products rounds about
-    # 0.1 % of z to the neighbouring bf16 value of the fp64 result.
-    print(f"z elements one bf16 step from the oracle's: {(dz > 0).mean():.2e}")
-    assert (dz > 0).mean() < 1e-2, (dz > 0).mean()
-    logits = O.router_logits(zg, hw.w_router)
-    _, _, keys = O.route(c, logits, hw.router_bias, W.host_token_ids(c, T))
-    same = check_routing(out, dict(ref, keys=keys))
-    check_outputs(out, ref, same_rows=same)
+    ref, same, rep = verify(run, out)
     return out, ref
 
 

@@ -60,3 +60,11 @@ def test_zipf_bias_frozen():
     r = W.zipf_ranks(128)
     assert sorted(r) == list(range(1, 129))
     assert b[np.argmin(r)] == 0.0 and np.all(np.diff(b[np.argsort(r)]) < 0)
+
+
+def test_f64_widening_matches_bf16_bits():
+    """normal_bf16_as_f64 is the bf16 draws widened exactly (a storage format)."""
+    k = synth.key(0, 77)
+    bits = synth.normal_bf16(k, 1000, 50000, 0.7)
+    wide = synth.normal_bf16_as_f64(k, 1000, 50000, 0.7)
+    assert np.array_equal(synth.bf16_bits_to_f32(bits).astype(np.float64), wide)
