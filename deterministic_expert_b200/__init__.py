@@ -220,6 +220,9 @@ class MoELayer:
                "moe_layer_forward")
 
     def device_error(self, workspace, stream=None) -> int:
+        """moe_get_device_error: read and clear the device error word of the
+        last forward on ``workspace`` (None: the no-allocation forward's static
+        scratch on the current device)."""
         return int(lib().moe_get_device_error(self.handle, _ptr(workspace), _stream(stream)))
 
     def check_invariance(self, x, residual, workspace, token_ids=None, n_splits=0, perm=None,
@@ -254,6 +257,87 @@ class MoELayer:
 
     def launch_count(self, T: int) -> int:
         return int(lib().moe_forward_launch_count(self.handle, T))
+
+
+class HostPipeline:
+    """Layer forwards of batches held in pinned host memory, end to end.
+
+    Each step copies its batch (x, residual and, for hash routing, the token
+    ids) from pinned host memory to the device, runs the layer forward, and
+    copies out_norm and out_residual back to pinned host memory.  Three streams
+    (copy-in, compute, copy-out) and two sets of device buffers let the copy-in
+    of step i + 1 and the copy-out of step i - 1 run while step i computes, so
+    the steady state costs max(compute, copy-in, copy-out) per step instead of
+    their sum.  ``chunks`` > 1 also splits every batch into that many row
+    blocks, each its own forward: a row's outputs do not depend on the rest of
+    its batch, so the bits are those of one call over the whole batch.
+
+    Only copies and stream ordering happen here; every step of the layer runs
+    in the library's kernels."""
+
+    def __init__(self, layer: "MoELayer", T: int, chunks: int = 1, device=None):
+        import torch
+        self.layer, self.T = layer, int(T)
+        self.chunks = max(1, min(int(chunks), self.T))
+        cfg = layer.cfg
+        dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+        self.device = dev
+        bounds = [self.T * c // self.chunks for c in range(self.chunks + 1)]
+        self.blocks = [(bounds[c], bounds[c + 1]) for c in range(self.chunks) if bounds[c + 1] > bounds[c]]
+        tmax = max(b - a for a, b in self.blocks)
+        mk = lambda: torch.empty((self.T, cfg.D), dtype=torch.bfloat16, device=dev)  # noqa: E731
+        self.x = [mk(), mk()]
+        self.r = [mk(), mk()]
+        self.on = [mk(), mk()]
+        self.orr = [mk(), mk()]
+        self.ids = [torch.empty(self.T, dtype=torch.int32, device=dev) for _ in range(2)]
+        self.ws = torch.empty(max(layer.workspace_size(tmax), 256), dtype=torch.uint8, device=dev)
+        self.s_in, self.s_comp, self.s_out = (torch.cuda.Stream(device=dev) for _ in range(3))
+        ev = lambda: [torch.cuda.Event(), torch.cuda.Event()]  # noqa: E731
+        self.in_done, self.comp_done, self.out_done = ev(), ev(), ev()
+        self._used = [False, False]
+
+    def run(self, xs, residuals, outs_norm, outs_residual, token_ids=None) -> None:
+        """Forward every batch i: xs[i], residuals[i] (pinned host [T, D] bf16)
+        -> outs_norm[i], outs_residual[i] (pinned host [T, D] bf16).
+        ``token_ids`` (list of pinned host [T] int32) is required for hash
+        routing.  Returns once the work is queued; synchronise the device (or
+        ``self.s_out``) before reading the outputs."""
+        import torch
+        hashr = self.layer.cfg.router == ROUTER_HASH
+        if hashr and token_ids is None:
+            raise ValueError("hash routing needs token_ids")
+        cur = torch.cuda.current_stream(self.device)
+        # Work queued on the caller's stream before this call comes first.
+        for s in (self.s_in, self.s_comp, self.s_out):
+            s.wait_stream(cur)
+        for i in range(len(xs)):
+            b = i & 1
+            if self._used[b]:
+                # Buffer set b is free for new inputs once step i - 2 has computed.
+                self.s_in.wait_event(self.comp_done[b])
+            with torch.cuda.stream(self.s_in):
+                self.x[b].copy_(xs[i], non_blocking=True)
+                self.r[b].copy_(residuals[i], non_blocking=True)
+                if hashr:
+                    self.ids[b].copy_(token_ids[i], non_blocking=True)
+                self.in_done[b].record(self.s_in)
+            self.s_comp.wait_event(self.in_done[b])
+            if self._used[b]:
+                # ... and its outputs may be overwritten once step i - 2 was copied out.
+                self.s_comp.wait_event(self.out_done[b])
+            for a, e in self.blocks:
+                self.layer.forward(self.x[b][a:e], self.r[b][a:e], self.on[b][a:e], self.orr[b][a:e], self.ws,
+                                   token_ids=self.ids[b][a:e] if hashr else None, stream=self.s_comp)
+            self.comp_done[b].record(self.s_comp)
+            self.s_out.wait_event(self.comp_done[b])
+            with torch.cuda.stream(self.s_out):
+                outs_norm[i].copy_(self.on[b], non_blocking=True)
+                outs_residual[i].copy_(self.orr[b], non_blocking=True)
+                self.out_done[b].record(self.s_out)
+            self._used[b] = True
+        # The caller's stream continues after the last copy-out.
+        cur.wait_stream(self.s_out)
 
 
 def reduce_partials(partials, residual, g, out_norm, out_residual, eps: float = 1e-6,

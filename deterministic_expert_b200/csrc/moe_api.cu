@@ -37,6 +37,10 @@ struct moe_handle {
 
 namespace {
 
+// Device address of the no-allocation forward's static scratch on the current
+// device (defined with that entry point at the end of this file).
+void* noalloc_scratch();
+
 constexpr int kProfFwd = 256;
 
 size_t align256(size_t b) { return (b + 255) & ~static_cast<size_t>(255); }
@@ -622,14 +626,21 @@ int moe_layer_forward(moe_handle* h, int T, const moe_bf16* x, const moe_bf16* r
 }
 
 int moe_get_device_error(moe_handle* h, void* workspace, void* stream) {
-  if (!h || !workspace) return MOE_EINVAL;
+  if (!h) return MOE_EINVAL;
+  // NULL: the error word of moe_layer_forward_noalloc's static scratch.
+  if (!workspace) workspace = noalloc_scratch();
+  if (!workspace) return MOE_ECUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int e = 0;
   if (cudaMemcpyAsync(&e, workspace, 4, cudaMemcpyDeviceToHost, s) != cudaSuccess) return MOE_ECUDA;
   if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ECUDA;
   if (cudaMemsetAsync(workspace, 0, 4, s) != cudaSuccess) return MOE_ECUDA;
-  if (e == kDevOk) return MOE_OK;
-  return e == kDevBadIndex ? MOE_EINDEX : MOE_ETIMEOUT;
+  switch (e) {
+    case kDevOk: return MOE_OK;
+    case kDevTimeout: return MOE_ETIMEOUT;
+    case kDevBadIndex: return MOE_EINDEX;
+    default: return MOE_ECUDA;   // a value no kernel writes: the word itself was overwritten
+  }
 }
 
 int moe_reduce_partials_rows(int P, const moe_bf16* const* partials, const moe_bf16* residual,

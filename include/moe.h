@@ -210,8 +210,11 @@ int moe_layer_forward(moe_handle* h, int T, const moe_bf16* x, const moe_bf16* r
                       void* workspace, size_t ws_bytes, void* stream);
 
 /* Read and clear the device error word the last forward on `workspace` left:
- * MOE_OK, or MOE_ETIMEOUT when a bounded device wait gave up.  Synchronises
- * `stream`. */
+ * MOE_OK; MOE_ETIMEOUT when a bounded device wait gave up; MOE_EINDEX when a
+ * device-side index check failed (bounds-checked library only); MOE_ECUDA when
+ * the copy failed or the word holds a value no kernel writes.  workspace NULL
+ * reads the error word of moe_layer_forward_noalloc's static scratch on the
+ * current device.  Synchronises `stream`. */
 int moe_get_device_error(moe_handle* h, void* workspace, void* stream);
 
 /* The tensor-parallel epilogue on one GPU (Fireworks parity post, Trap 1 + 2):
@@ -325,8 +328,10 @@ int moe_selftest_wait_timeout(int limit_us, void* stream);
  * only value that must start at zero (the device error word) is cleared by
  * the call's first kernel.  Calls whose kernels overlap on the GPU (other
  * streams, or another thread's call) race on the array: serialise them.
- * A device-side wait time-out is recorded in the array's error word and is
- * not reported to the caller. */
+ * A device-side wait time-out (or, in the bounds-checked library, an index
+ * fault) is recorded in the array's error word, which the call itself does
+ * not read: moe_get_device_error(h, NULL, stream) reads and clears it on the
+ * current device. */
 #define MOE_NOALLOC_SCRATCH_BYTES (32u << 20)
 int moe_layer_forward_noalloc(moe_handle* h, int T, const moe_bf16* x, const moe_bf16* residual,
                               const int32_t* token_ids, moe_bf16* out_norm,
