@@ -2,31 +2,37 @@
 """Throughput of the batch-invariant MoE layer forward on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl b200|reference]
-                    [--workload NAME] [--T TOKENS] [--no-cpu-baseline]
+                    [--workload NAME] [--T TOKENS] [--no-cpu-baseline] [--no-sweeps]
 
---workload picks another workload (v3_shaped, skew_zipf, skew_hash,
-fine_grained_situ, latent_situ, fine_grained_fp8, latent_situ_fp8, tiny, tiny_fp8,
-or skew_epilogue for the 8-partial
-reduce + residual + RMSNorm); --T overrides the batch size (the decode sweep
-is --T 1, 8, 64, 128, 512 on the fine-grained weights).
-
-One step is one full layer forward (all eight kernels: RMSNorm, router GEMM,
-top-k with the expert histogram, offsets + stable scatter, row gather,
-gate/up + SwiGLU GEMM, down GEMM, fixed-order combine + residual + RMSNorm) over one batch of the
-fine-grained workload (T=4096 tokens, D=2048, 64 experts top-6 softmax
-renormalised, I=1408, 2 shared experts of 1408) with seeded synthetic inputs
-and random weights of that architecture.  The L2 cache is flushed (a 512 MiB
-write) before every timed step; each step is timed with CUDA events on the
-launching stream.  N > 1 (torchrun, one rank per GPU) runs independent
+One step is one full layer forward (RMSNorm, router GEMM, top-k with the
+expert histogram, offsets + stable scatter, row gather, gate/up + SwiGLU GEMM,
+down GEMM, fixed-order combine + residual + RMSNorm) over one batch of the
+DeepSeek-V3-shaped workload (T=8192 tokens, D=7168, 256 experts top-8 sigmoid
+scores with a selection bias, normalised over the chosen 8, routed scale 2.5,
+SwiGLU clamp 10, I=2048, one shared expert of 2048) with seeded synthetic
+inputs and random weights of that architecture.  The L2 cache is flushed (a
+512 MiB write) before every timed step; each step is timed with CUDA events
+on the launching stream.  N > 1 (torchrun, one rank per GPU) runs independent
 replicas on disjoint token batches: the layer shards by token with no data
 exchange, so scaling is weak and `value` = all ranks' tokens / the slowest
 rank's time.
 
-Printed by rank 0 as one JSON line: tokens/s, the roofline of the dominant
-kernel (the gate/up + SwiGLU grouped GEMM, tensor-bound), the end-to-end
-number through the public API with host buffers, SM clocks sampled during the
-timed region, and the fp64 CPU oracle timed on a bounded sample
-(`cpu_baseline`).  `--impl reference` times only that oracle.
+Printed by rank 0 as one JSON line: tokens/s; the roofline of the dominant
+kernel (the gate/up + SwiGLU grouped GEMM, tensor-bound) against the measured
+peak (and, as `frac_of_nominal`, against the nominal dense bf16 peak); the
+end-to-end number through the public API with pinned host buffers (copies in
+and out every step, pipelined across steps by HostPipeline); SM clocks sampled
+during the timed region; the fine-grained workload (T=4096, D=2048, 64 experts
+top-6) as a sub-object; the decode sweep (T = 1, 8, 64, 128, 512 on the
+fine-grained weights, HBM-bound) as a sub-object; and the fp64 CPU oracle
+timed on a bounded sample (`cpu_baseline`) with the GPU's outputs on that
+sample compared against it (`parity`).
+
+--workload picks another headline workload (fine_grained, skew_zipf,
+skew_hash, fine_grained_situ, latent_situ, fine_grained_fp8, latent_situ_fp8,
+tiny, tiny_fp8, or skew_epilogue for the 8-partial reduce + residual +
+RMSNorm); --T overrides its batch size; --no-sweeps drops the two
+sub-objects.  `--impl reference` times only the oracle.
 """
 from __future__ import annotations
 
@@ -45,10 +51,16 @@ sys.path.insert(0, ROOT)
 
 METRIC = "MoE layer tokens/sec at 1 B200; % bf16 TC peak (prefill) / % HBM BW (decode)"
 UNIT = "tokens/s"
+DEFAULT_WORKLOAD = "v3_shaped"
 GATEUP_STAGE = 5
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic_gemm_gateup.json")
 GEMM_SOURCES = [os.path.join(ROOT, "deterministic_expert_b200", "csrc", n)
                 for n in ("grouped_gemm.cu", "common.cuh", "moe_internal.h")]
+# Nominal B200 figures (dense bf16 tensor peak; HBM3e bandwidth as the
+# spec target states it), reported beside the measured-peak fractions.
+NOMINAL_BF16_TFLOPS = 2250.0
+NOMINAL_HBM_GBS = 8000.0
+L2_NOTE = "flushed before every step (512 MiB write, untimed)"
 
 
 def parse():
@@ -57,9 +69,10 @@ def parse():
     p.add_argument("--steps", type=int, default=20)
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", default="b200", choices=["b200", "reference"])
-    p.add_argument("--workload", default="fine_grained")
+    p.add_argument("--workload", default=DEFAULT_WORKLOAD)
     p.add_argument("--T", type=int, default=None, help="override the workload's batch size")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-sweeps", action="store_true", help="skip the fine-grained and decode sub-objects")
     a = p.parse_args()
     a.warmup = max(a.warmup, 3)
     return a
@@ -81,13 +94,27 @@ def describe(cfg):
             "expert_weights": "FP4 values as E4M3 (E4M3 x E4M3 GEMMs)" if cfg.weight_format else "bf16"}
 
 
+def bench_config(cfg, world):
+    """The `config` object both arms print for a workload."""
+    return {**describe(cfg), "l2": L2_NOTE, "parallelism": f"replicas x{world} (token-sharded, no collective)"}
+
+
 def peaks():
+    """Measured peaks (MEASURED_PEAKS.json) or the machine's fallback figures."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
         with open(path) as f:
             d = json.load(f)
-        return d["bf16_tflops"], d["hbm_gbs"], "measured"
-    return 1590.0, 6650.0, "fallback"
+        return {"tc": d["bf16_tflops"], "tc_sustained": d.get("bf16_tflops_sustained"), "hbm": d["hbm_gbs"],
+                "kind": "measured"}
+    return {"tc": 1590.0, "tc_sustained": 1400.0, "hbm": 6650.0, "kind": "fallback"}
+
+
+def host_threads():
+    """Threads the oracle's BLAS uses, and the host's usable cores."""
+    from threadpoolctl import threadpool_info
+    blas = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    return blas, len(os.sched_getaffinity(0))
 
 
 def gemm_source_hash():
@@ -154,83 +181,142 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ oracle
-def oracle_sample(cfg, budget_s=12.0, chunk=256):
-    """Time the fp64 oracle (as it stands) on chunks of the workload's tokens
-    until about budget_s of CPU work has run.  Weight generation is not timed."""
+class TimedWeights:
+    """The workload's host weights (fp64 arrays of the bf16 values, regenerated
+    from the seeded generator) with the time spent regenerating experts
+    recorded, so the oracle can be timed without its input generation."""
+
+    def __init__(self, cfg, cache_experts):
+        import oracle as O
+        from synth import device as SD
+        self.base = SD.HostWeights(cfg, cache_experts=cache_experts)
+        self.gen_s = 0.0
+        for n in ("w_router", "router_bias", "g_in", "g_out", "w_proj_down", "w_proj_up"):
+            setattr(self, n, getattr(self.base, n, None))
+        # FP4 experts: the oracle's own FP4 quantisation of the master weights (part of its work).
+        self.view = O.FP4Weights(self) if cfg.weight_format else self
+
+    def _timed(self, fn, i):
+        t0 = time.perf_counter()
+        out = fn(i)
+        self.gen_s += time.perf_counter() - t0
+        return out
+
+    def routed(self, e):
+        return self._timed(self.base.routed, e)
+
+    def shared(self, s):
+        return self._timed(self.base.shared, s)
+
+
+def _cache_for(cfg, budget_bytes=8 << 30):
+    """Experts kept in fp64 at once: all of them when they fit the budget."""
+    from synth import workloads as W
+    per = 3 * (cfg.latent or cfg.D) * cfg.I * 8
+    return max(2, min(cfg.E + cfg.n_shared, budget_bytes // per)), per * cfg.E <= budget_bytes
+
+
+def oracle_run(cfg, rows, tw, x_all=None):
+    """The oracle on rows of the workload's batch; returns (ref, oracle seconds
+    without weight regeneration)."""
     import numpy as np
-    from threadpoolctl import threadpool_info
 
     import oracle as O
     from synth import device as SD
-    hw = SD.HostWeights(cfg)
-    if cfg.weight_format:
-        hw = O.FP4Weights(hw)   # the oracle's own FP4 quantisation of the master weights
-    for e in range(cfg.E):
-        hw.routed(e)
-    for s in range(cfg.n_shared):
-        hw.shared(s)
     from synth import workloads as W
-    tokens, spent, chunks = 0, 0.0, 0
-    while spent < budget_s and tokens < cfg.T:
+    x = SD.host_rows(cfg, "x", rows, T=cfg.T)
+    r = SD.host_rows(cfg, "residual", rows, T=cfg.T)
+    ids = W.host_token_ids(cfg, cfg.T)[np.asarray(rows)]
+    g0 = tw.gen_s
+    t0 = time.perf_counter()
+    ref = O.moe_layer(cfg, tw.view, x, r, ids)
+    return ref, (time.perf_counter() - t0) - (tw.gen_s - g0)
+
+
+def oracle_sample(cfg, budget_s=12.0, wall_s=90.0):
+    """Time the fp64 oracle (as it stands) on consecutive chunks of the
+    workload's tokens until about budget_s of oracle time (or wall_s of wall
+    time, weight regeneration included) has passed.  Expert weights are
+    regenerated on the host from the seeded generator; that time is not
+    counted.  Returns (cpu_baseline dict, [(rows, ref), ...])."""
+    import numpy as np
+    cache, all_fit = _cache_for(cfg)
+    tw = TimedWeights(cfg, cache)
+    chunk = 256 if all_fit else 16
+    tokens, spent, chunks, refs = 0, 0.0, 0, []
+    w0 = time.perf_counter()
+    while spent < budget_s and tokens < cfg.T and time.perf_counter() - w0 < wall_s:
         rows = np.arange(tokens, min(cfg.T, tokens + chunk))
-        x = SD.host_rows(cfg, "x", rows, T=cfg.T)
-        r = SD.host_rows(cfg, "residual", rows, T=cfg.T)
-        ids = W.host_token_ids(cfg, cfg.T)[rows]
-        t0 = time.perf_counter()
-        O.moe_layer(cfg, hw, x, r, ids)
-        spent += time.perf_counter() - t0
+        ref, dt = oracle_run(cfg, rows, tw)
+        spent += dt
         tokens += len(rows)
         chunks += 1
-    cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
-    return {"value": tokens / spent, "unit": UNIT, "cores": cores, "kind": "oracle",
-            "sample": f"{tokens} of {cfg.T} tokens ({chunks} chunks of {chunk}), full layer in fp64, "
-                      f"{spent:.1f} s of oracle time; weight generation not timed"}
+        refs.append((rows, ref))
+    blas, ncpu = host_threads()
+    return ({"value": round(tokens / spent, 2), "unit": UNIT, "cores": blas, "host_cores": ncpu,
+             "kind": "oracle",
+             "sample": f"tokens 0..{tokens - 1} of the {cfg.T}-token batch ({chunks} chunks of {chunk}), full "
+                       f"layer in fp64, {spent:.1f} s of oracle time; regenerating the expert weights on the "
+                       f"host ({tw.gen_s:.1f} s) not timed"}, refs)
+
+
+def parity_readout(refs, out_norm, out_residual, idx):
+    """The GPU's outputs on the oracle sample's tokens against the oracle
+    (tokens routed differently are counted, not value-compared here; the
+    test suite classifies and value-checks them)."""
+    import numpy as np
+    import torch
+    gi = idx.cpu().numpy()
+    on = out_norm.to(torch.float32).cpu().numpy().astype(np.float64)
+    orr = out_residual.to(torch.float32).cpu().numpy().astype(np.float64)
+    alike, differ, emax, esum, n = 0, 0, 0.0, 0.0, 0
+    for rows, ref in refs:
+        same = np.all(gi[rows] == ref["idx"], axis=1)
+        alike += int(same.sum())
+        differ += int((~same).sum())
+        for g, o in ((on[rows][same], ref["out_norm"][same]), (orr[rows][same], ref["out_residual"][same])):
+            e = np.abs(g - o) / np.maximum(1.0, np.abs(o))
+            if e.size:
+                emax = max(emax, float(e.max()))
+                esum += float(e.sum())
+                n += e.size
+    return {"tokens": alike + differ, "routed_like_oracle": alike, "routed_differently": differ,
+            "max_rel_err": round(emax, 6), "mean_rel_err": round(esum / max(n, 1), 7),
+            "tolerance": {"max": 2e-2, "mean": 4e-3}}
 
 
 def run_reference(a):
-    """--impl reference: the oracle on the same workload, rank 0 only."""
+    """--impl reference: the oracle on the same workload, rank 0 only.  Every
+    step times the oracle on the same bounded sample of the batch (its first
+    tokens), as every GPU step runs the same batch; the weights of the experts
+    it touches are regenerated once, untimed."""
     rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", str(a.gpus)))
     if rank != 0:
         return
-    cfg = workload(a)
     import numpy as np
-    from threadpoolctl import threadpool_info
-
-    import oracle as O
-    from synth import device as SD
-    from synth import workloads as W
-    hw = SD.HostWeights(cfg)
-    if cfg.weight_format:
-        hw = O.FP4Weights(hw)   # the oracle's own FP4 quantisation of the master weights
-    for e in range(cfg.E):
-        hw.routed(e)
-    for s in range(cfg.n_shared):
-        hw.shared(s)
-    chunk = 128
-    ids_all = W.host_token_ids(cfg, cfg.T)
+    cfg = workload(a)
+    cache, all_fit = _cache_for(cfg)
+    n = 128 if all_fit else 2
+    rows = np.arange(min(n, cfg.T))
+    tw = TimedWeights(cfg, max(cache, cfg.k * n + cfg.n_shared + 1))
     times = []
     for step in range(a.warmup + a.steps):
-        r0 = (step * chunk) % cfg.T
-        rows = np.arange(r0, min(cfg.T, r0 + chunk))
-        x = SD.host_rows(cfg, "x", rows, T=cfg.T)
-        r = SD.host_rows(cfg, "residual", rows, T=cfg.T)
-        t0 = time.perf_counter()
-        O.moe_layer(cfg, hw, x, r, ids_all[rows])
-        dt = time.perf_counter() - t0
+        _, dt = oracle_run(cfg, rows, tw)
         if step >= a.warmup:
-            times.append((dt, len(rows)))
-    secs = sum(t for t, _ in times)
-    toks = sum(n for _, n in times)
-    value = toks / secs
-    cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+            times.append(dt)
+    secs = sum(times)
+    value = len(rows) * len(times) / secs
+    blas, ncpu = host_threads()
     print(json.dumps({
-        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": a.gpus,
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": a.steps, "warmup": a.warmup, "ms_per_step": 1e3 * secs / len(times),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded counter-based generator; random weights of the workload's shape)",
-        "config": describe(cfg),
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
-                         "sample": f"each step: {chunk} tokens of the {cfg.T}-token batch, full layer in fp64"},
+        "config": bench_config(cfg, world),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas, "host_cores": ncpu, "kind": "oracle",
+                         "sample": f"each step: tokens 0..{len(rows) - 1} of the {cfg.T}-token batch, full layer "
+                                   f"in fp64; expert weight regeneration ({tw.gen_s:.1f} s) not timed"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }), flush=True)
 
@@ -239,7 +325,6 @@ def epilogue_oracle_sample(budget_s, chunk=256):
     """The oracle's fixed-order reduce + residual + RMSNorm on consecutive
     256-row chunks of the epilogue workload until ``budget_s`` has passed."""
     import numpy as np
-    from threadpoolctl import threadpool_info
 
     import oracle as O
     from synth import device as SD
@@ -258,8 +343,8 @@ def epilogue_oracle_sample(budget_s, chunk=256):
         secs += time.perf_counter() - t0
         rows += n
         r0 = (r0 + n) % T
-    cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
-    return {"value": round(rows / secs, 1), "unit": UNIT, "cores": cores, "kind": "oracle",
+    cores, ncpu = host_threads()
+    return {"value": round(rows / secs, 1), "unit": UNIT, "cores": cores, "host_cores": ncpu, "kind": "oracle",
             "sample": f"{rows} rows of the {T}-row epilogue in {chunk}-row chunks, fp32 fixed-order sum, fp64 norm"}
 
 
@@ -378,7 +463,8 @@ def run_epilogue(a):
                "h2d_bytes_per_step": (P + 1) * T * D * 2, "d2h_bytes_per_step": 2 * T * D * 2}
     cpu = None if (rank != 0 or a.no_cpu_baseline) else epilogue_oracle_sample(budget_s=12.0)
     if rank == 0:
-        _, hbm_peak, peak_kind = peaks()
+        pk = peaks()
+        hbm_peak, peak_kind = pk["hbm"], pk["kind"]
         wl = (f"skewed workload epilogue: {P} partial buffers [T={T}, D={D}] bf16 "
               f"N(0,1)/8, fixed r0..r{P - 1} order + residual + RMSNorm")
         if tp is None:
@@ -417,6 +503,127 @@ def run_epilogue(a):
         dist.destroy_process_group()
 
 
+def timed_steps(layer, x, r, on, orr, ws, ids, steps, flush, stream, cnt=None, profile=None):
+    """Run `steps` layer forwards, L2 flushed before each, each bracketed by a
+    CUDA event pair on the launching stream; returns the per-step ms and, with
+    ``profile`` (stage indices), the per-stage average ms over the steps."""
+    import torch
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    if profile is not None:
+        layer.profile_enable(profile)
+    for e0, e1 in evs:
+        flush.fill_(1)
+        e0.record(stream)
+        layer.forward(x, r, on, orr, ws, token_ids=ids, out_counts=cnt, stream=stream)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    stage = None
+    if profile is not None:
+        ms, n = layer.profile_read()
+        layer.profile_enable([])
+        stage = [ms[i] / n[i] if n[i] else None for i in range(len(ms))]
+    return [e0.elapsed_time(e1) for e0, e1 in evs], stage
+
+
+def gemm_roofline(cfg, gate_ms, pk, traffic):
+    from synth import workloads as W
+    tc = pk["tc"] * (2.0 if cfg.weight_format else 1.0)
+    nominal = NOMINAL_BF16_TFLOPS * (2.0 if cfg.weight_format else 1.0)
+    fl = W.moe_flops(cfg)["gateup"]
+    achieved = fl / (gate_ms / 1e3) / 1e12
+    src = f"{pk['kind']} bf16 (burst)"
+    if cfg.weight_format:
+        # E4M3 x E4M3: the bf16 peak times the nominal dense ratio of the two formats (4.5 / 2.25 PFLOP/s).
+        src += " x 2, nominal E4M3 / bf16 ratio"
+    return {"bound": "tensor", "kernel": "gemm_gateup_swiglu", "achieved": round(achieved, 1), "peak": tc,
+            "unit": "TFLOP/s", "frac": round(achieved / tc, 4), "traffic": traffic, "peak_source": src,
+            "frac_of_nominal": round(achieved / nominal, 4), "nominal_peak": nominal,
+            "flops_per_launch": fl, "avg_launch_ms": round(gate_ms, 4)}
+
+
+def layer_numbers(cfg, T, ms, distinct, pk):
+    from synth import workloads as W
+    tc = pk["tc"] * (2.0 if cfg.weight_format else 1.0)
+    nominal = NOMINAL_BF16_TFLOPS * (2.0 if cfg.weight_format else 1.0)
+    fl = W.moe_flops(cfg, T)["total"]
+    tf = fl / (ms / 1e3) / 1e12
+    nbytes = W.layer_bytes(cfg, T, distinct)
+    gbs = nbytes / (ms / 1e3) / 1e9
+    return {"tflops": round(tf, 1), "frac_of_tc_peak": round(tf / tc, 4), "frac_of_nominal_tc": round(tf / nominal, 4),
+            "flops_per_step": fl, "distinct_experts": distinct, "algorithmic_bytes": nbytes,
+            "hbm_gbs": round(gbs, 1), "frac_of_hbm": round(gbs / pk["hbm"], 4),
+            "frac_of_nominal_hbm": round(gbs / NOMINAL_HBM_GBS, 4)}
+
+
+def fine_grained_object(a, dev, flush, stream, pk):
+    """The fine-grained workload (T=4096, D=2048, 64 experts top-6 softmax
+    renormalised, I=1408, 2 shared) timed as the headline is."""
+    import torch
+
+    import deterministic_expert_b200 as moe
+    from synth import device as SD
+    from synth import workloads as W
+    cfg = W.C2
+    w = SD.device_weights(cfg, device=dev)
+    x, r, _ = SD.device_inputs(cfg, device=dev)
+    layer = moe.MoELayer(SD.layer_config(cfg, cfg.T), w)
+    ws = torch.empty(layer.workspace_size(cfg.T), dtype=torch.uint8, device=dev)
+    on, orr = torch.empty_like(x), torch.empty_like(x)
+    cnt = torch.empty(cfg.E, dtype=torch.int32, device=dev)
+    timed_steps(layer, x, r, on, orr, ws, None, a.warmup, flush, stream)
+    ms_steps, stage = timed_steps(layer, x, r, on, orr, ws, None, a.steps, flush, stream, cnt=cnt,
+                                  profile=[GATEUP_STAGE])
+    if layer.device_error(ws) != moe.MOE_OK:
+        raise RuntimeError("device wait timed out (fine-grained)")
+    ms = sum(ms_steps) / len(ms_steps)
+    out = {"workload": W.pretty(cfg), "ms_per_step": round(ms, 4), "value": round(cfg.T / (ms / 1e3), 1),
+           "unit": UNIT, "steps": a.steps,
+           "layer": layer_numbers(cfg, cfg.T, ms, int((cnt > 0).sum().item()), pk),
+           "roofline": gemm_roofline(cfg, stage[GATEUP_STAGE], pk, ncu_traffic(cfg)),
+           "gpu_launches": a.steps * layer.launch_count(cfg.T)}
+    layer.close()
+    return out, w
+
+
+def decode_object(a, dev, flush, stream, pk, w):
+    """The decode sweep: batches of T = 1, 8, 64, 128, 512 tokens (the first T
+    rows of an 8192-row input) on the fine-grained weights; HBM-bound, so the
+    figure is algorithmic bytes (the weights of the experts actually routed to,
+    shared and router weights, activations) over the time per forward."""
+    import torch
+
+    import deterministic_expert_b200 as moe
+    from synth import device as SD
+    from synth import workloads as W
+    cfg = W.C2
+    xa, ra, _ = SD.device_inputs(cfg, T=W.C4_SOURCE_T, device=dev)
+    tmax = max(W.C4_T)
+    layer = moe.MoELayer(SD.layer_config(cfg, tmax), w)
+    ws = torch.empty(layer.workspace_size(tmax), dtype=torch.uint8, device=dev)
+    cnt = torch.empty(cfg.E, dtype=torch.int32, device=dev)
+    rows = []
+    launches = 0
+    for T in W.C4_T:
+        x, r = xa[:T].contiguous(), ra[:T].contiguous()
+        on, orr = torch.empty_like(x), torch.empty_like(x)
+        timed_steps(layer, x, r, on, orr, ws, None, a.warmup, flush, stream)
+        ms_steps, _ = timed_steps(layer, x, r, on, orr, ws, None, a.steps, flush, stream, cnt=cnt)
+        ms = sum(ms_steps) / len(ms_steps)
+        distinct = int((cnt > 0).sum().item())
+        nb = W.layer_bytes(cfg, T, distinct)
+        gbs = nb / (ms / 1e3) / 1e9
+        rows.append({"T": T, "us_per_forward": round(ms * 1e3, 2), "tokens_per_s": round(T / (ms / 1e3), 1),
+                     "distinct_experts": distinct, "algorithmic_bytes": nb, "hbm_gbs": round(gbs, 1),
+                     "frac_of_hbm": round(gbs / pk["hbm"], 4), "frac_of_nominal_hbm": round(gbs / NOMINAL_HBM_GBS, 4)})
+        launches += a.steps * layer.launch_count(T)
+    if layer.device_error(ws) != moe.MOE_OK:
+        raise RuntimeError("device wait timed out (decode)")
+    layer.close()
+    return {"weights": W.pretty(cfg), "source_batch": f"first T rows of a {W.C4_SOURCE_T}-row input",
+            "bound": "hbm", "peak_gbs": pk["hbm"], "nominal_gbs": NOMINAL_HBM_GBS, "steps": a.steps,
+            "sweep": rows, "gpu_launches": launches}
+
+
 def main():
     a = parse()
     if a.impl == "reference":
@@ -444,11 +651,11 @@ def main():
     dev = torch.device("cuda", local)
     if world > 1:
         import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=dev)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     cfg = workload(a)
     T = cfg.T
     stream = torch.cuda.current_stream()
+    pk = peaks()
 
     w = SD.device_weights(cfg, device=dev)
     if cfg.weight_format:
@@ -461,46 +668,29 @@ def main():
     x, r, ids = (xa[rank * T:(rank + 1) * T].contiguous(), ra[rank * T:(rank + 1) * T].contiguous(),
                  ida[rank * T:(rank + 1) * T].contiguous())
     del xa, ra, ida
-    lc = SD.layer_config(cfg, T_max=T)
-    layer = moe.MoELayer(lc, w)
+    layer = moe.MoELayer(SD.layer_config(cfg, T_max=T), w)
     ws = torch.empty(layer.workspace_size(T), dtype=torch.uint8, device=dev)
     on = torch.empty((T, cfg.D), dtype=torch.bfloat16, device=dev)
     orr = torch.empty_like(on)
     cnt = torch.empty(cfg.E, dtype=torch.int32, device=dev)
+    idx = torch.empty((T, cfg.k), dtype=torch.int32, device=dev)
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
     use_ids = ids if cfg.router == W.ROUTER_HASH else None
 
-    def step(timed_events=None):
-        flush.fill_(1)
-        if timed_events:
-            timed_events[0].record(stream)
-        layer.forward(x, r, on, orr, ws, token_ids=use_ids, out_counts=cnt, stream=stream)
-        if timed_events:
-            timed_events[1].record(stream)
-
-    for _ in range(a.warmup):
-        step()
-    torch.cuda.synchronize()
+    timed_steps(layer, x, r, on, orr, ws, use_ids, a.warmup, flush, stream)
     if layer.device_error(ws) != moe.MOE_OK:
         raise RuntimeError("device wait timed out during warm-up")
 
     # ------------------------------------------------ timed region (value)
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(a.steps)]
     clocks = ClockSampler(local) if rank == 0 else None
-    layer.profile_enable([GATEUP_STAGE])
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    for i in range(a.steps):
-        step(evs[i])
-    torch.cuda.synchronize()
+    ms_steps, stage = timed_steps(layer, x, r, on, orr, ws, use_ids, a.steps, flush, stream, cnt=cnt,
+                                  profile=[GATEUP_STAGE])
     if world > 1:
         dist.barrier()
     clk = clocks.stop() if clocks else None
-    ms_steps = [e0.elapsed_time(e1) for e0, e1 in evs]
-    stage_ms, stage_n = layer.profile_read()
-    layer.profile_enable([])
     if layer.device_error(ws) != moe.MOE_OK:
         raise RuntimeError("device wait timed out in the timed region")
     ms_total = torch.tensor([sum(ms_steps)], dtype=torch.float64, device=dev)
@@ -509,95 +699,83 @@ def main():
     ms_per_step = float(ms_total.item()) / a.steps
     value = world * T / (ms_per_step / 1e3)
     distinct = int((cnt > 0).sum().item())
+    gate_ms = stage[GATEUP_STAGE]
 
     # --------------------------------------------- per-stage breakdown (untimed)
-    layer.profile_enable(None)
-    for _ in range(3):
-        step()
-    all_ms, all_n = layer.profile_read()
-    layer.profile_enable([])
-    stage_avg = {moe.STAGE_NAMES[i]: round(all_ms[i] / all_n[i] * 1e3, 2) if all_n[i] else None
-                 for i in range(moe.NUM_STAGES)}
+    _, all_stage = timed_steps(layer, x, r, on, orr, ws, use_ids, 3, flush, stream, profile=list(range(moe.NUM_STAGES)))
+    stage_avg = {moe.STAGE_NAMES[i]: round(v * 1e3, 2) if v else None for i, v in enumerate(all_stage)}
+    # The GPU's outputs (and routing) of the batch, for the parity readout.
+    layer.forward(x, r, on, orr, ws, token_ids=use_ids, out_topk_idx=idx, stream=stream)
+    torch.cuda.synchronize()
 
     # ------------------------------------------------------- e2e (host buffers)
-    xh, rh = x.cpu().pin_memory(), r.cpu().pin_memory()
-    idh = ids.cpu().pin_memory()
-    onh = torch.empty(on.shape, dtype=on.dtype).pin_memory()
-    orh = torch.empty_like(onh).pin_memory()
-    h2d = xh.numel() * 2 + rh.numel() * 2 + (idh.numel() * 4 if use_ids is not None else 0)
-    d2h = onh.numel() * 2 + orh.numel() * 2
+    # Through the public API: HostPipeline copies every step's inputs in from
+    # pinned host memory and both outputs back, overlapping the copies of
+    # neighbouring steps with each step's forward.
+    hx, hr = x.cpu().pin_memory(), r.cpu().pin_memory()
+    hid = ids.cpu().pin_memory() if use_ids is not None else None
+    hon = [torch.empty(on.shape, dtype=on.dtype).pin_memory() for _ in range(2)]
+    hor = [torch.empty(on.shape, dtype=on.dtype).pin_memory() for _ in range(2)]
+    pipe = moe.HostPipeline(layer, T, device=dev)
+    h2d = hx.numel() * 2 + hr.numel() * 2 + (hid.numel() * 4 if hid is not None else 0)
+    d2h = 2 * on.numel() * 2
 
-    def e2e_step(ev=None):
-        flush.fill_(1)
-        if ev:
-            ev[0].record(stream)
-        x.copy_(xh, non_blocking=True)
-        r.copy_(rh, non_blocking=True)
-        if use_ids is not None:
-            ids.copy_(idh, non_blocking=True)
-        layer.forward(x, r, on, orr, ws, token_ids=use_ids, stream=stream)
-        onh.copy_(on, non_blocking=True)
-        orh.copy_(orr, non_blocking=True)
-        if ev:
-            ev[1].record(stream)
+    def e2e(n):
+        pipe.run([hx] * n, [hr] * n, [hon[i & 1] for i in range(n)], [hor[i & 1] for i in range(n)],
+                 token_ids=None if hid is None else [hid] * n)
 
-    for _ in range(a.warmup):
-        e2e_step()
-    ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(a.steps)]
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    for i in range(a.steps):
-        e2e_step(ev2[i])
+    e2e(a.warmup)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    e2e_ms = torch.tensor([sum(e0.elapsed_time(e1) for e0, e1 in ev2)], dtype=torch.float64, device=dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    e2e(a.steps)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    if layer.device_error(pipe.ws) != moe.MOE_OK:
+        raise RuntimeError("device wait timed out (end to end)")
+    e2e_ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
-    e2e_value = world * T / (float(e2e_ms.item()) / a.steps / 1e3)
+    e2e_value = world * T * a.steps / (float(e2e_ms.item()) / 1e3)
+    e2e_bits = torch.equal(hon[(a.steps - 1) & 1].view(torch.int16), on.cpu().view(torch.int16))
+    del pipe
+
+    sub = {}
+    if not a.no_sweeps and cfg.name == DEFAULT_WORKLOAD and not a.T:
+        fg, w2 = fine_grained_object(a, dev, flush, stream, pk)
+        sub["fine_grained"] = fg
+        sub["decode"] = decode_object(a, dev, flush, stream, pk, w2)
+        del w2
 
     if rank == 0:
-        tc_peak, hbm_peak, peak_kind = peaks()
-        peak_src = f"{peak_kind} bf16 (burst)"
-        if cfg.weight_format:
-            # E4M3 x E4M3: the measured bf16 peak times the nominal dense ratio
-            # of the two formats (4.5 / 2.25 PFLOP/s).
-            tc_peak, peak_src = 2.0 * tc_peak, f"{peak_kind} bf16 (burst) x 2, nominal E4M3 / bf16 ratio"
-        fl = W.moe_flops(cfg)
-        gate_ms = stage_ms[GATEUP_STAGE] / max(stage_n[GATEUP_STAGE], 1)
-        achieved = fl["gateup"] / (gate_ms / 1e3) / 1e12
-        traffic = ncu_traffic(cfg)
-        roof = {"bound": "tensor", "kernel": "gemm_gateup_swiglu", "achieved": round(achieved, 1),
-                "peak": tc_peak, "unit": "TFLOP/s", "frac": round(achieved / tc_peak, 4),
-                "traffic": traffic, "peak_source": peak_src,
-                "flops_per_launch": fl["gateup"], "avg_launch_ms": round(gate_ms, 4)}
-        layer_tflops = fl["total"] / (ms_per_step / 1e3) / 1e12
-        cpu = None
+        cpu = par = None
         if world == 1 and not a.no_cpu_baseline:
-            cpu = oracle_sample(cfg)
+            cpu, refs = oracle_sample(cfg)
+            par = parity_readout(refs, on, orr, idx)
         line = {
             "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
             "steps": a.steps, "warmup": a.warmup, "ms_per_step": round(ms_per_step, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "e4m3" if cfg.weight_format else "bf16",
             "data": "synthetic (seeded counter-based generator; random weights of the workload's shape)",
-            "config": {**describe(cfg), "l2": "flushed before every step (512 MiB write, untimed)",
-                       "parallelism": f"replicas x{world} (token-sharded, no collective)"},
-            "roofline": roof,
-            "layer": {"tflops": round(layer_tflops, 1), "frac_of_tc_peak": round(layer_tflops / tc_peak, 4),
-                      "flops_per_step": fl["total"], "distinct_experts": distinct,
-                      "algorithmic_bytes": W.layer_bytes(cfg, T, distinct),
-                      "hbm_gbs": round(W.layer_bytes(cfg, T, distinct) / (ms_per_step / 1e3) / 1e9, 1),
-                      "frac_of_hbm": round(W.layer_bytes(cfg, T, distinct) / (ms_per_step / 1e3) / 1e9
-                                           / hbm_peak, 4)},
+            "config": bench_config(cfg, world),
+            "roofline": gemm_roofline(cfg, gate_ms, pk, ncu_traffic(cfg)),
+            "layer": layer_numbers(cfg, T, ms_per_step, distinct, pk),
             "stage_us": stage_avg,
             "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h},
+                    "d2h_bytes_per_step": d2h, "api": "HostPipeline (copy-in, compute and copy-out streams, "
+                                                       "two buffer sets, steps overlapped)",
+                    "outputs_bit_equal_to_device_forward": bool(e2e_bits)},
             "gpu_launches": a.steps * layer.launch_count(T),
             "clocks": clk,
+            **sub,
             "cpu_baseline": cpu,
+            "parity": par,
         }
         print(json.dumps(line), flush=True)
     layer.close()

@@ -84,3 +84,37 @@ def test_fp8_decode_sweep_matches_full_batch(torch_cuda):
         out = run.forward(x[ri].contiguous(), r[ri].contiguous(), ids[ri].contiguous())
         for key in ("out_norm", "out_residual"):
             assert torch.equal(out[key].view(torch.int16), full[key][ri].view(torch.int16)), (T, key)
+
+
+@pytest.mark.parametrize("name,chunks", [("fine_grained", 1), ("fine_grained", 3), ("skew_hash", 2)])
+def test_host_pipeline_matches_single_calls(torch_cuda, name, chunks):
+    """End-to-end forwards through HostPipeline (pinned host batches copied in,
+    outputs copied out, neighbouring steps overlapped on three streams, each
+    batch optionally split into row blocks) give the bits of one device
+    forward per batch."""
+    import deterministic_expert_b200 as moe
+    torch = torch_cuda
+    cfg = W.CONFIGS[name]
+    T = 1024
+    run = Run(cfg.with_T(T), T_max=T)
+    xa, ra, ida = run.inputs(3 * T)
+    batches = [(xa[i * T:(i + 1) * T].contiguous(), ra[i * T:(i + 1) * T].contiguous(),
+                ida[i * T:(i + 1) * T].contiguous()) for i in range(3)]
+    want = [run.forward(*b) for b in batches]
+    pipe = moe.HostPipeline(run.layer, T, chunks=chunks)
+    hx = [b[0].cpu().pin_memory() for b in batches]
+    hr = [b[1].cpu().pin_memory() for b in batches]
+    hid = [b[2].cpu().pin_memory() for b in batches]
+    hon = [torch.full((T, cfg.D), float("nan"), dtype=torch.bfloat16).pin_memory() for _ in range(3)]
+    hor = [torch.full((T, cfg.D), float("nan"), dtype=torch.bfloat16).pin_memory() for _ in range(3)]
+    # Five steps over the three batches: buffer sets are reused across steps.
+    order = [0, 1, 2, 1, 0]
+    outs_n = [hon[i] for i in order]
+    outs_r = [hor[i] for i in order]
+    pipe.run([hx[i] for i in order], [hr[i] for i in order], outs_n, outs_r,
+             token_ids=[hid[i] for i in order] if cfg.router == W.ROUTER_HASH else None)
+    torch.cuda.synchronize()
+    assert run.layer.device_error(pipe.ws) == 0
+    for i in range(3):
+        assert torch.equal(hon[i].view(torch.int16), want[i]["out_norm"].cpu().view(torch.int16)), i
+        assert torch.equal(hor[i].view(torch.int16), want[i]["out_residual"].cpu().view(torch.int16)), i
