@@ -81,7 +81,11 @@ struct Tile {
 template <int CG>
 __device__ __forceinline__ void decode_tile(const GemmArgs& a, const int* tile_start, int t, Tile& ti) {
   int local = t;
-  if (a.tile_start == nullptr) {
+  if (a.tile_start == nullptr && a.shared_only_tiles > 0) {
+    // The shared groups alone (each T rows, the same tiles per group).
+    ti.kind = 1; ti.idx = t / a.shared_only_tiles; ti.rows = a.T; ti.a_row0 = ti.idx * a.shared_a_stride;
+    local = t - ti.idx * a.shared_only_tiles;
+  } else if (a.tile_start == nullptr) {
     // One dense group of T rows (router, latent projections) of kind dense_kind.
     ti.kind = a.dense_kind; ti.idx = 0; ti.rows = a.T; ti.a_row0 = 0;
   } else {
@@ -99,9 +103,17 @@ __device__ __forceinline__ void decode_tile(const GemmArgs& a, const int* tile_s
     ti.kind = 1; ti.idx = lo - a.E; ti.rows = a.T; ti.a_row0 = ti.idx * a.shared_a_stride;
   }
   }
-  const int mt = (ti.rows + Cfg<CG>::kTileM - 1) / Cfg<CG>::kTileM;
-  ti.n = local / mt;
-  ti.m = local - ti.n * mt;
+  // Tiles of a group are numbered M-major: (m, n) = (local / nt, local % nt).
+  // Pairs take tiles t, t + n_clusters, ...; numbered N-major instead, a group
+  // with two M-tiles would put its full tiles on even and its small last tiles
+  // on odd tile indices, so with an even number of pairs every full tile
+  // would land on the even pairs.  M-major keeps the tiles that share A rows
+  // (one M-tile, all N-tiles) and the tiles that share weights (one N-tile,
+  // the group's M-tiles) within a few tiles of each other, so both still
+  // meet in L2.
+  const int nt = a.n_kind[ti.kind] / a.BN;
+  ti.m = local / nt;
+  ti.n = local - ti.m * nt;
   const int r = ti.rows - ti.m * Cfg<CG>::kTileM;
   ti.swap = CG == 2 && a.swap_ok && r < 256;
   ti.nt = ti.swap ? (r + 15) & ~15 : 0;

@@ -28,6 +28,13 @@ struct moe_handle {
   uint16_t* w_router_pad = nullptr;  // [E_pad, L], rows >= E zero
   CUtensorMap map_router, map_wg, map_wu, map_wd, map_wsg, map_wsu, map_wsd, map_pd, map_pu;
   unsigned long long timeout_ns = 2000ull * 1000 * 1000;
+  // Decode-sized batches run the shared experts (which need no routing) on an
+  // auxiliary stream while the routing front end runs on the caller's stream;
+  // the mutex keeps concurrent forwards on one handle from interleaving their
+  // event records.
+  cudaStream_t aux = nullptr;
+  cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
+  std::mutex fork_mu;
   // Per-stage timing (moe_profile_*).
   int prof_mask = 0;
   int prof_fwd = 0;
@@ -283,6 +290,20 @@ int pair_grid(const moe_handle* h, int tiles_bound) {
   return 2 * std::max(1, std::min(h->max_pairs, tiles_bound));
 }
 
+// Shared-expert tiles of the gate/up GEMM for T rows.
+int shared_gateup_tiles(const moe_handle* h, int T) {
+  return h->S * ((T + kPairTileM - 1) / kPairTileM) * (h->cfg.I_shared / h->bn_gu);
+}
+
+// Whether a forward of T rows runs the shared experts on the auxiliary stream:
+// only when their gate/up tiles occupy at most two thirds of the CTA pairs, so
+// the routing front end and the routed experts keep SMs to run on.  (At
+// prefill sizes the shared tiles would hold every SM and gain nothing.)
+bool fork_shared(const moe_handle* h, int T) {
+  return h->S > 0 && h->aux != nullptr && h->ep_world == 1 &&
+         3 * shared_gateup_tiles(h, T) <= 2 * h->max_pairs;
+}
+
 // The layer forward.  front_only (expert parallelism): stop after the grouping
 // (stages 0-3), with the per-expert counts written to counts_dst.
 int forward_impl(moe_handle* h, int T, const uint16_t* x, const uint16_t* residual,
@@ -355,6 +376,123 @@ int forward_impl(moe_handle* h, int T, const uint16_t* x, const uint16_t* residu
                               f8 ? xqe : nullptr, s));
   prof.end(0);
 
+  // 5-6. gate/up + SwiGLU(+clamp) (routed groups read xp, shared groups read
+  // xn), the E4M3 quantisation of h, and down (routed rows scatter to their
+  // (token, slot) row of y).  `part` selects the groups: all of them, the
+  // routed ones, or the shared ones (each group's tiles are the same in every
+  // case, so the bits are too).
+  enum Part { kAllGroups, kRoutedGroups, kSharedGroups };
+  auto expert_gemms = [&](Part part, cudaStream_t st) -> int {
+    const bool routed = part != kSharedGroups, shared = part != kRoutedGroups && h->S > 0;
+    const bool timed = st == s;   // stage timing covers the caller's stream only
+    const int mt_shared = (T + kPairTileM - 1) / kPairTileM;
+    // Which groups a launch walks: the device tile list (all groups, or its
+    // routed prefix), or the shared groups alone.
+    auto select = [&](GemmArgs& g, int32_t* tiles, int nt_routed, int nt_shared) {
+      if (part == kSharedGroups) {
+        g.tile_start = nullptr;
+        g.shared_only_tiles = mt_shared * nt_shared;
+        g.router_tiles = h->S * g.shared_only_tiles;
+        return g.router_tiles;
+      }
+      g.tile_start = tiles;
+      g.G = part == kAllGroups ? h->G : c.E;
+      return expert_tile_bound(h, T, nt_routed, part == kAllGroups ? nt_shared : 0);
+    };
+    {
+      GemmArgs g;
+      std::memset(&g, 0, sizeof(g));
+      // E4M3: the routed rows are the gathered E4M3 rows, the shared rows xq.
+      const void* xs = f8 ? static_cast<const void*>(xq) : static_cast<const void*>(xn);
+      if (!make_map(&g.mapA[0], xp, LW, TK, kBM, eb)) return MOE_ECUDA;
+      if (!make_map(&g.mapA64[0], xp, LW, TK, kBM / 2, eb)) return MOE_ECUDA;
+      if (!make_map(&g.mapA16[0], xp, LW, TK, 16, eb)) return MOE_ECUDA;
+      if (h->S > 0 && !make_map(&g.mapA[1], xs, c.D, T, kBM, eb)) return MOE_ECUDA;
+      if (h->S > 0 && !make_map(&g.mapA64[1], xs, c.D, T, kBM / 2, eb)) return MOE_ECUDA;
+      if (h->S > 0 && !make_map(&g.mapA16[1], xs, c.D, T, 16, eb)) return MOE_ECUDA;
+      g.fp8 = f8;
+      g.a_exp[0] = xpe; g.a_exp[1] = xqe;
+      g.a_rows[0] = TK; g.a_rows[1] = T;
+      g.out_rows[0] = TK; g.out_rows[1] = h->S * T;
+      g.mapB[0] = h->map_wg; g.mapB[1] = h->map_wu; g.mapB[2] = h->map_wsg; g.mapB[3] = h->map_wsu;
+      g.offsets = offsets; g.G = h->G; g.E = c.E; g.T = T;
+      g.n_kind[0] = c.I; g.n_kind[1] = c.I_shared;
+      g.k_kind[0] = LW; g.k_kind[1] = c.D;
+      g.BN = h->bn_gu;
+      g.swap_ok = h->bn_gu == 128;
+      g.a_stage_bytes = g.swap_ok ? small_batch_a_bytes(T) : 0;
+      g.shared_a_stride = 0;
+      g.out[0] = hb; g.ld_out[0] = c.I;
+      g.out[1] = hsb; g.ld_out[1] = c.I_shared;
+      g.shared_out_stride = T;
+      g.gate_clamp = c.gate_clamp_max; g.up_clamp = c.up_clamp;
+      g.act = c.activation; g.beta_g = c.situ_beta_gate; g.beta_u = c.situ_beta_up;
+      g.inv_beta_g = 1.0f / c.situ_beta_gate; g.inv_beta_u = 1.0f / c.situ_beta_up;
+      g.err = err; g.timeout_ns = h->timeout_ns;
+      const int bound = select(g, tiles_gu, c.I / h->bn_gu, h->S > 0 ? c.I_shared / h->bn_gu : 0);
+      if (timed) prof.begin(5);
+      if (launch_grouped_gemm(kGateUp, g, pair_grid(h, bound), st) != cudaSuccess) return MOE_ECUDA;
+      if (timed) prof.end(5);
+    }
+    // 5b. E4M3: h rows (routed and / or shared) to E4M3 with their row exponents
+    if (f8) {
+      if (timed) prof.begin(11);
+      if (launch_quant_rows(hb, routed ? TK : 0, c.I, hq, he, hsb, shared ? h->S * T : 0, c.I_shared, hqs, hse,
+                            nullptr, st) != cudaSuccess)
+        return MOE_ECUDA;
+      if (timed) prof.end(11);
+    }
+    {
+      GemmArgs g;
+      std::memset(&g, 0, sizeof(g));
+      const void* ar = f8 ? static_cast<const void*>(hq) : static_cast<const void*>(hb);
+      const void* as = f8 ? static_cast<const void*>(hqs) : static_cast<const void*>(hsb);
+      const uint64_t srows = static_cast<uint64_t>(h->S) * T;
+      if (!make_map(&g.mapA[0], ar, c.I, TK, kBM, eb)) return MOE_ECUDA;
+      if (!make_map(&g.mapA64[0], ar, c.I, TK, kBM / 2, eb)) return MOE_ECUDA;
+      if (!make_map(&g.mapA16[0], ar, c.I, TK, 16, eb)) return MOE_ECUDA;
+      if (h->S > 0 && !make_map(&g.mapA[1], as, c.I_shared, srows, kBM, eb)) return MOE_ECUDA;
+      if (h->S > 0 && !make_map(&g.mapA64[1], as, c.I_shared, srows, kBM / 2, eb)) return MOE_ECUDA;
+      if (h->S > 0 && !make_map(&g.mapA16[1], as, c.I_shared, srows, 16, eb)) return MOE_ECUDA;
+      g.fp8 = f8;
+      g.a_exp[0] = he; g.a_exp[1] = hse;
+      g.a_rows[0] = TK; g.a_rows[1] = h->S * T;
+      g.out_rows[0] = TK; g.out_rows[1] = h->S * T;
+      g.mapB[0] = h->map_wd; g.mapB[2] = h->map_wsd;
+      g.offsets = offsets; g.G = h->G; g.E = c.E; g.T = T;
+      g.n_kind[0] = LW; g.n_kind[1] = c.D;
+      g.k_kind[0] = c.I; g.k_kind[1] = c.I_shared;
+      g.BN = h->bn_dn;
+      g.swap_ok = h->bn_dn == 256;
+      g.a_stage_bytes = g.swap_ok ? small_batch_a_bytes(T) : 0;
+      g.shared_a_stride = T;
+      g.out[0] = y; g.ld_out[0] = LW;
+      g.out[1] = ys; g.ld_out[1] = c.D;
+      g.shared_out_stride = T;
+      g.dest_row = dest;
+      g.err = err; g.timeout_ns = h->timeout_ns;
+      const int bound = select(g, tiles_dn, LW / h->bn_dn, c.D / h->bn_dn);
+      if (timed) prof.begin(6);
+      if (launch_grouped_gemm(kDown, g, pair_grid(h, bound), st) != cudaSuccess) return MOE_ECUDA;
+      if (timed) prof.end(6);
+    }
+    return MOE_OK;
+  };
+
+  // Decode-sized batches: the shared experts need only xn, so they start now
+  // on the auxiliary stream and run beside the routing front end; the caller's
+  // stream joins them before the combine.
+  const bool fork = !front_only && fork_shared(h, T);
+  std::unique_lock<std::mutex> fork_lock(h->fork_mu, std::defer_lock);
+  if (fork) {
+    fork_lock.lock();
+    MOE_TRY(cudaEventRecord(h->ev_fork, s));
+    MOE_TRY(cudaStreamWaitEvent(h->aux, h->ev_fork, 0));
+    const int r = expert_gemms(kSharedGroups, h->aux);
+    if (r != MOE_OK) return r;
+    MOE_TRY(cudaEventRecord(h->ev_join, h->aux));
+  }
+
   // Latent MoE: the router and the routed experts read z = bf16(xn W_down^T).
   const uint16_t* xe = xn;
   if (lat) {
@@ -426,84 +564,14 @@ int forward_impl(moe_handle* h, int T, const uint16_t* x, const uint16_t* residu
   else MOE_TRY(launch_gather_rows(xe, T, src, TK, LW * 2, xp, nullptr, nullptr, err, s));
   prof.end(4);
 
-  // 5. gate/up + SwiGLU(+clamp): routed groups read xp, shared groups read xn
-  {
-    GemmArgs g;
-    std::memset(&g, 0, sizeof(g));
-    // E4M3: the routed rows are the gathered E4M3 rows, the shared rows xq.
-    const void* xs = f8 ? static_cast<const void*>(xq) : static_cast<const void*>(xn);
-    if (!make_map(&g.mapA[0], xp, LW, TK, kBM, eb)) return MOE_ECUDA;
-    if (!make_map(&g.mapA64[0], xp, LW, TK, kBM / 2, eb)) return MOE_ECUDA;
-    if (!make_map(&g.mapA16[0], xp, LW, TK, 16, eb)) return MOE_ECUDA;
-    if (h->S > 0 && !make_map(&g.mapA[1], xs, c.D, T, kBM, eb)) return MOE_ECUDA;
-    if (h->S > 0 && !make_map(&g.mapA64[1], xs, c.D, T, kBM / 2, eb)) return MOE_ECUDA;
-    if (h->S > 0 && !make_map(&g.mapA16[1], xs, c.D, T, 16, eb)) return MOE_ECUDA;
-    g.fp8 = f8;
-    g.a_exp[0] = xpe; g.a_exp[1] = xqe;
-    g.a_rows[0] = TK; g.a_rows[1] = T;
-    g.out_rows[0] = TK; g.out_rows[1] = h->S * T;
-    g.mapB[0] = h->map_wg; g.mapB[1] = h->map_wu; g.mapB[2] = h->map_wsg; g.mapB[3] = h->map_wsu;
-    g.offsets = offsets; g.tile_start = tiles_gu; g.G = h->G; g.E = c.E; g.T = T;
-    g.n_kind[0] = c.I; g.n_kind[1] = c.I_shared;
-    g.k_kind[0] = LW; g.k_kind[1] = c.D;
-    g.BN = h->bn_gu;
-    g.swap_ok = h->bn_gu == 128;
-    g.a_stage_bytes = g.swap_ok ? small_batch_a_bytes(T) : 0;
-    g.shared_a_stride = 0;
-    g.out[0] = hb; g.ld_out[0] = c.I;
-    g.out[1] = hsb; g.ld_out[1] = c.I_shared;
-    g.shared_out_stride = T;
-    g.gate_clamp = c.gate_clamp_max; g.up_clamp = c.up_clamp;
-    g.act = c.activation; g.beta_g = c.situ_beta_gate; g.beta_u = c.situ_beta_up;
-    g.inv_beta_g = 1.0f / c.situ_beta_gate; g.inv_beta_u = 1.0f / c.situ_beta_up;
-    g.err = err; g.timeout_ns = h->timeout_ns;
-    const int bound = expert_tile_bound(h, T, da.gu_ntiles_routed, da.gu_ntiles_shared);
-    prof.begin(5);
-    MOE_TRY(launch_grouped_gemm(kGateUp, g, pair_grid(h, bound), s));
-    prof.end(5);
-  }
-
-  // 5b. E4M3: h rows (routed and shared) to E4M3 with their row exponents
-  if (f8) {
-    prof.begin(11);
-    MOE_TRY(launch_quant_rows(hb, TK, c.I, hq, he, hsb, h->S * T, c.I_shared, hqs, hse, nullptr, s));
-    prof.end(11);
-  }
-
-  // 6. down: routed rows scatter to their (token, slot) row of y
-  {
-    GemmArgs g;
-    std::memset(&g, 0, sizeof(g));
-    const void* ar = f8 ? static_cast<const void*>(hq) : static_cast<const void*>(hb);
-    const void* as = f8 ? static_cast<const void*>(hqs) : static_cast<const void*>(hsb);
-    const uint64_t srows = static_cast<uint64_t>(h->S) * T;
-    if (!make_map(&g.mapA[0], ar, c.I, TK, kBM, eb)) return MOE_ECUDA;
-    if (!make_map(&g.mapA64[0], ar, c.I, TK, kBM / 2, eb)) return MOE_ECUDA;
-    if (!make_map(&g.mapA16[0], ar, c.I, TK, 16, eb)) return MOE_ECUDA;
-    if (h->S > 0 && !make_map(&g.mapA[1], as, c.I_shared, srows, kBM, eb)) return MOE_ECUDA;
-    if (h->S > 0 && !make_map(&g.mapA64[1], as, c.I_shared, srows, kBM / 2, eb)) return MOE_ECUDA;
-    if (h->S > 0 && !make_map(&g.mapA16[1], as, c.I_shared, srows, 16, eb)) return MOE_ECUDA;
-    g.fp8 = f8;
-    g.a_exp[0] = he; g.a_exp[1] = hse;
-    g.a_rows[0] = TK; g.a_rows[1] = h->S * T;
-    g.out_rows[0] = TK; g.out_rows[1] = h->S * T;
-    g.mapB[0] = h->map_wd; g.mapB[2] = h->map_wsd;
-    g.offsets = offsets; g.tile_start = tiles_dn; g.G = h->G; g.E = c.E; g.T = T;
-    g.n_kind[0] = LW; g.n_kind[1] = c.D;
-    g.k_kind[0] = c.I; g.k_kind[1] = c.I_shared;
-    g.BN = h->bn_dn;
-    g.swap_ok = h->bn_dn == 256;
-    g.a_stage_bytes = g.swap_ok ? small_batch_a_bytes(T) : 0;
-    g.shared_a_stride = T;
-    g.out[0] = y; g.ld_out[0] = LW;
-    g.out[1] = ys; g.ld_out[1] = c.D;
-    g.shared_out_stride = T;
-    g.dest_row = dest;
-    g.err = err; g.timeout_ns = h->timeout_ns;
-    const int bound = expert_tile_bound(h, T, da.dn_ntiles, da.dn_ntiles_shared);
-    prof.begin(6);
-    MOE_TRY(launch_grouped_gemm(kDown, g, pair_grid(h, bound), s));
-    prof.end(6);
+  if (fork) {
+    // The shared experts were started on the auxiliary stream after step 0.
+    const int r = expert_gemms(kRoutedGroups, s);
+    if (r != MOE_OK) return r;
+    MOE_TRY(cudaStreamWaitEvent(s, h->ev_join, 0));
+  } else {
+    const int r = expert_gemms(kAllGroups, s);
+    if (r != MOE_OK) return r;
   }
 
   // 7. fixed-order combine + residual + RMSNorm
@@ -585,6 +653,11 @@ int moe_init(const moe_config* cfg, const moe_weights* w, moe_handle** out) {
   gemm_prepare();
   h->max_pairs = gemm_max_pairs();
   if (h->max_pairs <= 0) h->max_pairs = h->num_sms / 2;
+  if (h->S > 0 && h->ep_world == 1 &&
+      (cudaStreamCreateWithFlags(&h->aux, cudaStreamNonBlocking) != cudaSuccess ||
+       cudaEventCreateWithFlags(&h->ev_fork, cudaEventDisableTiming) != cudaSuccess ||
+       cudaEventCreateWithFlags(&h->ev_join, cudaEventDisableTiming) != cudaSuccess))
+    return fail(MOE_ECUDA);
   const moe_config& c = h->cfg;
   if (c.router != MOE_ROUTER_HASH) {
     const size_t row = static_cast<size_t>(h->L) * 2;
@@ -825,8 +898,10 @@ int moe_profile_read(moe_handle* h, float* ms, int* launches) {
 int moe_forward_launch_count(const moe_handle* h, int T) {
   if (!h || T < 0) return -1;
   if (T == 0) return 0;
+  const bool fork = fork_shared(h, T);
   const int base = 8 + (h->cfg.latent > 0 ? 3 : 0)   // latent: two projections and the latent sum
-                   + (h->fp8 ? 1 : 0)                 // E4M3: quantisation of h
+                   + (fork ? 2 : 0)                   // shared experts' two GEMMs on their own
+                   + (h->fp8 ? (fork ? 2 : 1) : 0)    // E4M3: quantisation of h (routed, shared)
                    + (h->fp8 && h->cfg.latent > 0 ? 1 : 0);   // ... and of z
   return h->cfg.router == MOE_ROUTER_HASH ? base - 1 : base;  // hash routing: no router GEMM
 }
@@ -1142,6 +1217,9 @@ int moe_destroy(moe_handle* h) {
   if (!h) return MOE_EINVAL;
   for (auto& e : h->ev)
     if (e) cudaEventDestroy(e);
+  if (h->ev_fork) cudaEventDestroy(h->ev_fork);
+  if (h->ev_join) cudaEventDestroy(h->ev_join);
+  if (h->aux) cudaStreamDestroy(h->aux);
   if (h->w_router_pad) cudaFree(h->w_router_pad);
   delete h;
   return MOE_OK;

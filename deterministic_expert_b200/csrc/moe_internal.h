@@ -73,6 +73,8 @@ struct GemmArgs {
   int shared_a_stride;    // A rows between consecutive shared experts (0: all read row 0..T)
   int router_tiles;       // tile count when tile_start is NULL (M-tiles x N-tiles)
   int dense_kind;         // kind of the single group when tile_start is NULL
+  int shared_only_tiles;  // > 0 with tile_start NULL: only the shared groups (each of T rows),
+                          // this many tiles per group, group s at tiles [s * n, (s + 1) * n)
   int out_bf16;           // down-mode output as bf16 instead of fp32 (latent projection)
   int fp8;                // expert GEMMs: A and B are E4M3 codes (kind::f8f6f4)
   int ep;                 // down, routed: dest_row = rank << 24 | row, stored at out_rank[rank]

@@ -107,7 +107,10 @@ EPILOGUE_SIGMA = 1.0 / 8.0
 
 # The latent workload with FP4 expert weights (routed and shared).
 C6F = dataclasses.replace(C6, name="latent_situ_fp8", weight_format=1)
-CONFIGS = {c.name: c for c in (C1, C2, C3, C5, C5H, C2S, C6, C1F, C2F, C6F)}
+# A small case of the V3-shaped kernels for profiler captures (a few GB on the
+# device): the same D, I, top-8 and about 256 rows per expert, with 32 experts.
+C3P = dataclasses.replace(C3, name="v3_shaped_e32", T=1024, E=32)
+CONFIGS = {c.name: c for c in (C1, C2, C3, C5, C5H, C2S, C6, C1F, C2F, C6F, C3P)}
 
 _ZIPF_FILE = os.path.join(os.path.dirname(os.path.abspath(__file__)), "zipf_beta.json")
 ZIPF_S = 1.2
