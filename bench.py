@@ -585,9 +585,10 @@ def fine_grained_object(a, dev, flush, stream, pk):
     return out, w
 
 
-def decode_object(a, dev, flush, stream, pk, w):
+def decode_object(a, dev, flush, stream, pk, w, cfg=None):
     """The decode sweep: batches of T = 1, 8, 64, 128, 512 tokens (the first T
-    rows of an 8192-row input) on the fine-grained weights; HBM-bound, so the
+    rows of an 8192-row input) on the fine-grained weights (bf16, or their FP4
+    storage form with cfg = the fine_grained_fp4 workload); HBM-bound, so the
     figure is algorithmic bytes (the weights of the experts actually routed to,
     shared and router weights, activations) over the time per forward."""
     import torch
@@ -595,7 +596,7 @@ def decode_object(a, dev, flush, stream, pk, w):
     import deterministic_expert_b200 as moe
     from synth import device as SD
     from synth import workloads as W
-    cfg = W.C2
+    cfg = W.C2 if cfg is None else cfg
     xa, ra, _ = SD.device_inputs(cfg, T=W.C4_SOURCE_T, device=dev)
     tmax = max(W.C4_T)
     layer = moe.MoELayer(SD.layer_config(cfg, tmax), w)
@@ -658,10 +659,14 @@ def main():
     pk = peaks()
 
     w = SD.device_weights(cfg, device=dev)
-    if cfg.weight_format:
+    if cfg.weight_format == 1:
         # FP4 expert weights: the library's quantiser turns the bf16 master
         # weights into their E4M3 codes once, before anything is timed.
         w = moe.quantize_expert_weights(w)
+        torch.cuda.synchronize()
+    elif cfg.weight_format == 2:
+        # ... or into their storage form (packed E2M1 codes and block exponents).
+        w = moe.pack_expert_weights_fp4(w)
         torch.cuda.synchronize()
     # Each rank takes its own T rows of a world*T-row batch (disjoint tokens).
     xa, ra, ida = SD.device_inputs(cfg, T=T * world, device=dev)
@@ -750,6 +755,9 @@ def main():
         fg, w2 = fine_grained_object(a, dev, flush, stream, pk)
         sub["fine_grained"] = fg
         sub["decode"] = decode_object(a, dev, flush, stream, pk, w2)
+        # The same sweep with the FP4 experts in their storage form (half a
+        # byte per weight plus block exponents, expanded to E4M3 on chip).
+        sub["decode_fp4"] = decode_object(a, dev, flush, stream, pk, moe.pack_expert_weights_fp4(w2), cfg=W.C2P)
         del w2
 
     if rank == 0:

@@ -25,11 +25,14 @@ MOE_OK, MOE_EINVAL, MOE_ETOOBIG, MOE_EWORKSPACE, MOE_EUNSUPPORTED, MOE_ECUDA, MO
     0, -1, -2, -3, -4, -5, -6, -7)
 ROUTER_SOFTMAX, ROUTER_SIGMOID_BIAS, ROUTER_HASH = 0, 1, 2
 ACT_SWIGLU, ACT_SITU_GLU = 0, 1
-WEIGHTS_BF16, WEIGHTS_FP8 = 0, 1
+WEIGHTS_BF16, WEIGHTS_FP8, WEIGHTS_FP4 = 0, 1, 2
 NUM_STAGES = 12
 STAGE_NAMES = ("rmsnorm_in", "router_gemm", "router_topk", "dispatch", "gather_rows",
                "gemm_gateup_swiglu", "gemm_down", "combine_norm", "latent_down", "latent_combine",
                "latent_up", "quant_h")
+
+
+EXPERT_WEIGHTS = ("w_gate", "w_up", "w_down", "ws_gate", "ws_up", "ws_down")
 
 
 class MoEError(RuntimeError):
@@ -52,7 +55,8 @@ class moe_config(ctypes.Structure):
 class moe_weights(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in ("w_router", "router_bias", "w_gate", "w_up", "w_down",
                                                "ws_gate", "ws_up", "ws_down", "g_in", "g_out",
-                                               "w_proj_down", "w_proj_up")]
+                                               "w_proj_down", "w_proj_up", "w_gate_exp", "w_up_exp",
+                                               "w_down_exp", "ws_gate_exp", "ws_up_exp", "ws_down_exp")]
 
 
 class moe_views(ctypes.Structure):
@@ -162,6 +166,12 @@ def _check_weight_sizes(cfg: LayerConfig, weights: dict) -> None:
             "w_up": El * cfg.I * L, "w_down": El * L * cfg.I, "ws_gate": S * Is * cfg.D,
             "ws_up": S * Is * cfg.D, "ws_down": S * cfg.D * Is, "g_in": cfg.D, "g_out": cfg.D,
             "w_proj_down": cfg.latent * cfg.D, "w_proj_up": cfg.D * cfg.latent}
+    fp4 = cfg.weight_format == WEIGHTS_FP4
+    if fp4:
+        # Packed codes: half a byte per weight; one exponent word per row per 128 of K.
+        for n in EXPERT_WEIGHTS:
+            want[n + "_exp"] = want[n] // 128
+            want[n] //= 2
     for name, n in want.items():
         t = weights.get(name)
         if t is None:
@@ -171,8 +181,10 @@ def _check_weight_sizes(cfg: LayerConfig, weights: dict) -> None:
                              f"got {t.numel()} (contiguous={t.is_contiguous()})")
         import torch
         dtype = torch.float32 if name == "router_bias" else torch.bfloat16
-        if cfg.weight_format == WEIGHTS_FP8 and name in ("w_gate", "w_up", "w_down", "ws_gate", "ws_up", "ws_down"):
-            dtype = torch.uint8   # E4M3 codes
+        if cfg.weight_format != WEIGHTS_BF16 and name in EXPERT_WEIGHTS:
+            dtype = torch.uint8   # E4M3 codes, or packed E2M1 codes
+        if name.endswith("_exp"):
+            dtype = torch.int32   # four int8 block exponents a word
         if t.dtype != dtype:
             raise ValueError(f"weight {name}: expected {dtype}, got {t.dtype}")
 
@@ -366,7 +378,6 @@ def quantize_weights_fp4(w, w8, block_exp=None, stream=None) -> None:
            "moe_quantize_weights_fp4")
 
 
-EXPERT_WEIGHTS = ("w_gate", "w_up", "w_down", "ws_gate", "ws_up", "ws_down")
 
 
 def quantize_expert_weights(weights: dict, stream=None) -> dict:
@@ -382,6 +393,45 @@ def quantize_expert_weights(weights: dict, stream=None) -> dict:
         q = torch.empty(t.shape, dtype=torch.uint8, device=t.device)
         quantize_weights_fp4(t, q, stream=stream)
         out[n] = q
+    return out
+
+
+def quantize_weights_fp4_packed(w, packed, exps, stream=None) -> None:
+    """moe_quantize_weights_fp4_packed: bf16 master weights [..., K] -> their FP4
+    storage form: ``packed`` uint8 [..., K / 2] (two E2M1 codes a byte, low nibble
+    first) and ``exps`` int32 [K / 128, rows] (four int8 block exponents a word)."""
+    L = lib()
+    K = int(w.shape[-1])
+    rows = w.numel() // K if K else 0
+    if packed.numel() * 2 != w.numel() or packed.dtype.itemsize != 1:
+        raise ValueError("packed must be a byte tensor with half as many elements as w")
+    if exps.numel() * 128 != w.numel() or exps.dtype.itemsize != 4:
+        raise ValueError("exps must be a 4-byte tensor with one word per 128 elements of w")
+    L.moe_quantize_weights_fp4_packed.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                                  ctypes.c_longlong, ctypes.c_int, ctypes.c_void_p]
+    _check(L.moe_quantize_weights_fp4_packed(_ptr(w), _ptr(packed), _ptr(exps), rows, K, _stream(stream)),
+           "moe_quantize_weights_fp4_packed")
+
+
+def pack_expert_weights_fp4(weights: dict, stream=None) -> dict:
+    """A copy of a moe_weights dict whose expert matrices (bf16 master weights)
+    are replaced by their FP4 storage form from quantize_weights_fp4_packed
+    (packed codes under the matrix's name, exponent words under name + "_exp"),
+    for a layer configured with weight_format=WEIGHTS_FP4.  Other entries are
+    shared."""
+    import torch
+    out = dict(weights)
+    for n in EXPERT_WEIGHTS:
+        t = weights.get(n)
+        if t is None:
+            continue
+        K = int(t.shape[-1])
+        rows = t.numel() // K
+        p = torch.empty(t.shape[:-1] + (K // 2,), dtype=torch.uint8, device=t.device)
+        x = torch.empty((K // 128, rows), dtype=torch.int32, device=t.device)
+        quantize_weights_fp4_packed(t, p, x, stream=stream)
+        out[n] = p
+        out[n + "_exp"] = x
     return out
 
 
@@ -625,8 +675,14 @@ def shard_expert_weights(weights: dict, world: int, rank: int) -> dict:
     out = dict(weights)
     for n in ("w_gate", "w_up", "w_down"):
         t = weights[n]
-        e0, e1 = expert_range(int(t.shape[0]), world, rank)
+        E = int(t.shape[0])
+        e0, e1 = expert_range(E, world, rank)
         out[n] = t[e0:e1]
+        x = weights.get(n + "_exp")
+        if x is not None:
+            # FP4 exponent words [K / 128, E * rows]: this rank's columns, made contiguous.
+            per = x.shape[1] // E
+            out[n + "_exp"] = x[:, e0 * per:e1 * per].contiguous()
     return out
 
 

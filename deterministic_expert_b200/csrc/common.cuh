@@ -140,6 +140,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait with acquire semantics at cluster scope (pairs with a cluster-scope
+// release arrive, mbar_arrive_release_cluster).
+__device__ __forceinline__ bool mbar_try_wait_acq_cluster(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait for the phase with the given parity to complete, for at most
 // limit_ns nanoseconds.  On time-out it raises *abort (shared by the CTA's
 // roles) and the device error word, and returns false; it also returns
@@ -150,6 +164,25 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 63u) == 0) {
+      if (*abort) return false;
+      if (globaltimer_ns() - t0 > limit_ns) {
+        *abort = 1;
+        atomicExch(err, kDevTimeout);
+        return false;
+      }
+    }
+  }
+}
+
+// mbar_wait with a cluster-scope acquire (for phases completed by arrivals
+// from the other CTA of a pair that publish its shared-memory writes).
+__device__ __forceinline__ bool mbar_wait_acq_cluster(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                                      int* err, uint64_t limit_ns) {
+  if (mbar_try_wait_acq_cluster(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait_acq_cluster(bar, parity)) return true;
     if ((it & 63u) == 0) {
       if (*abort) return false;
       if (globaltimer_ns() - t0 > limit_ns) {
@@ -204,6 +237,19 @@ __device__ __forceinline__ uint32_t mapa_shared(const void* p, uint32_t rank) {
 
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+// Arrive with release semantics at cluster scope (the arriving thread's
+// earlier shared-memory writes are visible to a cluster-scope acquire of the
+// phase), on an mbarrier of this CTA or of another CTA of the cluster.
+__device__ __forceinline__ void mbar_arrive_release_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+// Make this thread's generic-proxy shared-memory writes visible to the async
+// proxy (the tensor core's operand reads).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 // 2D tiled load into this CTA's shared memory whose completion is counted on

@@ -163,7 +163,14 @@ __global__ void k_gather_rows(const uint8_t* __restrict__ src, int src_rows, con
   if (!MOE_INDEX_OK(from >= 0 && from < src_rows, err)) return;
   const uint4* s = reinterpret_cast<const uint4*>(src + static_cast<size_t>(from) * row_bytes);
   uint4* d = reinterpret_cast<uint4*>(dst + static_cast<size_t>(p) * row_bytes);
-  for (int c = lane; c < row_bytes / 16; c += 32) d[c] = s[c];
+  // Four 16-byte loads in flight per lane before their stores.
+  const int n = row_bytes / 16;
+  int c = lane;
+  for (; c + 96 < n; c += 128) {
+    const uint4 v0 = s[c], v1 = s[c + 32], v2 = s[c + 64], v3 = s[c + 96];
+    d[c] = v0; d[c + 32] = v1; d[c + 64] = v2; d[c + 96] = v3;
+  }
+  for (; c < n; c += 32) d[c] = s[c];
   if (dst_exp != nullptr && lane == 0) dst_exp[p] = src_exp[from];
 }
 

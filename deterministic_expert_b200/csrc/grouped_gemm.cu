@@ -110,7 +110,8 @@ __device__ __forceinline__ void decode_tile(const GemmArgs& a, const int* tile_s
   // would land on the even pairs.  M-major keeps the tiles that share A rows
   // (one M-tile, all N-tiles) and the tiles that share weights (one N-tile,
   // the group's M-tiles) within a few tiles of each other, so both still
-  // meet in L2.
+  // meet in L2.  (Measured on the V3-shaped layer: N-major with an odd pair
+  // count read 10 % more DRAM in gate/up.)
   const int nt = a.n_kind[ti.kind] / a.BN;
   ti.m = local / nt;
   ti.n = local - ti.m * nt;
@@ -158,9 +159,64 @@ __device__ __forceinline__ float glu_unit(float g, float u, const GemmArgs& a) {
   return silu_clamped_product(g, u, a.gate_clamp, a.up_clamp);
 }
 
-template <int MODE, int CG, int ACT, int F8>
-__global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_constant__ GemmArgs a) {
+// FP4 weights (F4, with F8): expand one converter warp's 32 weight rows of a
+// stage's B slot in place.  The warp's rows r = 32 w + lane own the E4M3 bytes
+// [4096 w, 4096 w + 4096) of the slot (row r at 128 r, its 16-byte chunk c at
+// chunk position c ^ (r & 7): the layout a 128-byte-swizzled TMA load of E4M3
+// rows leaves); their packed E2M1 codes (64 bytes a row) were loaded to
+// 4096 w + 2048 and their exponent words to 4096 w + 1024, inside that span.
+// Every lane reads all of its input before any lane writes (__syncwarp), then
+// writes byte code * 2^s: the magnitude from the exponent's 8-entry table
+// (lut[s + 8], E4M3 codes of 0, 0.5, 1, 1.5, 2, 3, 4, 6 times 2^s) picked by
+// prmt, the sign bit from bit 3 of the code.
+// prmt.b32 in its default mode: byte n of the result is byte (c >> 4n) & 7 of
+// {b, a} (a = bytes 0-3), or, when bit 3 of that selector nibble is set, that
+// byte's top bit replicated over all 8 bits.
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+// Four E2M1 codes (the low four nibbles of codes16) -> four E4M3 bytes.
+__device__ __forceinline__ uint32_t e2m1x4_to_e4m3(uint32_t codes16, uint32_t lut_lo, uint32_t lut_hi) {
+  const uint32_t mag = prmt(lut_lo, lut_hi, codes16 & 0x7777u);
+  // Sign set: selector nibble 8 replicates the top bit of byte 0 of 0x80 ->
+  // 0xFF; sign clear: selector nibble 1 picks byte 1, 0x00.
+  const uint32_t t = codes16 & 0x8888u;
+  const uint32_t neg = prmt(0x80u, 0u, t | ((t >> 3) ^ 0x1111u));
+  return mag | (neg & 0x80808080u);
+}
+
+__device__ __forceinline__ void fp4_expand_rows(uint8_t* slot, int w, int lane, const uint32_t (*lut)[2]) {
+  const uint8_t* in = slot + 4096 * w + 2048 + 64 * lane;
+  uint4 p[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) p[j] = *reinterpret_cast<const uint4*>(in + 16 * j);
+  const uint32_t ex = *reinterpret_cast<const uint32_t*>(slot + 4096 * w + 1024 + 4 * lane);
+  __syncwarp();
+  const int r = 32 * w + lane;
+  uint8_t* out = slot + 128 * r;
+  const uint32_t words[16] = {p[0].x, p[0].y, p[0].z, p[0].w, p[1].x, p[1].y, p[1].z, p[1].w,
+                              p[2].x, p[2].y, p[2].z, p[2].w, p[3].x, p[3].y, p[3].z, p[3].w};
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    // Chunk c: elements 16c .. 16c + 15, in block c / 2 (exponent byte c / 2).
+    // s in [-8, 6] by construction; the clamp keeps any other byte inside the table.
+    const int sb = min(max(static_cast<int>(static_cast<int8_t>((ex >> (8 * (c >> 1))) & 0xFFu)) + 8, 0), 14);
+    const uint32_t lo = lut[sb][0], hi = lut[sb][1];
+    const uint32_t w0 = words[2 * c], w1 = words[2 * c + 1];
+    const uint4 v = make_uint4(e2m1x4_to_e4m3(w0, lo, hi), e2m1x4_to_e4m3(w0 >> 16, lo, hi),
+                               e2m1x4_to_e4m3(w1, lo, hi), e2m1x4_to_e4m3(w1 >> 16, lo, hi));
+    *reinterpret_cast<uint4*>(out + ((c ^ (r & 7)) << 4)) = v;
+  }
+}
+
+template <int MODE, int CG, int ACT, int F8, int F4 = 0>
+__global__ void __launch_bounds__(F4 ? kGemmThreadsF4 : kGemmThreads, 1)
+    k_grouped_gemm(const __grid_constant__ GemmArgs a) {
   using C = Cfg<CG>;
+  static_assert(!F4 || (F8 && MODE != kRouter && CG == 2), "FP4 weights: the expert GEMMs' E4M3 pair kernels");
   // K elements per 128-byte operand row of a stage: 64 bf16 or 128 E4M3.  Every
   // byte count below (stage slots, TMA boxes, descriptor steps) is the same for
   // both; an E4M3 MMA walks 32 elements where a bf16 one walks 16.
@@ -194,16 +250,37 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
   uint64_t* xempty = xfull + 4;  // [4]
   uint64_t* gfull = xempty + 4;  // [4]
   uint64_t* gempty = gfull + 4;  // [4]
+  // FP4: each CTA's own TMA loads of a stage complete lfull; full then counts
+  // the converter warps of both CTAs (the expanded tile is what the MMA reads).
+  uint64_t* lfull = gempty + 4;  // [kRingMax]
   uint8_t* epi = reinterpret_cast<uint8_t*>(bars) + kBarBytes;  // kEpiWarps x kEpiBytes
   __shared__ uint32_t tmem_slot;
+  __shared__ uint32_t s_lut[F4 ? 15 : 1][2];
   __shared__ int abort_flag;
   __shared__ int s_tile_start[kMaxGroups + 1];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = CG == 2 ? cluster_ctarank() : 0;   // 0 = the MMA-issuing CTA
   const bool leader = rank == 0;
+  if (F4 && threadIdx.x < 15) {
+    // E4M3 codes of the 8 E2M1 magnitudes times 2^s, s = threadIdx.x - 8 (exact products).
+    const float mags[8] = {0.f, 0.5f, 1.f, 1.5f, 2.f, 3.f, 4.f, 6.f};
+    const float sc = exp2_int(static_cast<int>(threadIdx.x) - 8);
+    uint32_t lo = 0, hi = 0;
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      lo |= e4m3_rn(__fmul_rn(mags[m], sc)) << (8 * m);
+      hi |= e4m3_rn(__fmul_rn(mags[m + 4], sc)) << (8 * m);
+    }
+    s_lut[threadIdx.x][0] = lo;
+    s_lut[threadIdx.x][1] = hi;
+  }
   if (threadIdx.x == 0) {
-    for (int s = 0; s < S; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], F4 ? CG * kCvtWarps : 1);
+      mbar_init(&empty[s], 1);
+      if (F4) mbar_init(&lfull[s], 1);
+    }
     for (int b = 0; b < 2; ++b) { mbar_init(&tfull[b], 1); mbar_init(&tempty[b], CG * kEpiWarps); }
     mbar_init(tdone, 1);
     for (int p = 0; p < 4; ++p) {
@@ -275,7 +352,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort, a.err, a.timeout_ns)) { ok = false; break; }
           uint8_t* b0 = sB + stage * sb_bytes;
-          if (CG == 1) {
+          if (F4) {
+            // This CTA's A rows, and for each converter warp w its 32 weight rows
+            // as packed E2M1 codes (64 bytes a row, to 4096 w + 2048 of the slot)
+            // with their exponent words (to 4096 w + 1024); gate/up: warps 0-1
+            // gate rows, 2-3 up rows.  All counted on this CTA's lfull.
+            mbar_arrive_expect_tx(&lfull[stage], static_cast<uint32_t>(box) * 128 + kCvtWarps * (32 * 64 + 32 * 4));
+            tma_load_2d(sA + stage * sa_bytes, amap, kb * KE, a_y, &lfull[stage]);
+#pragma unroll
+            for (int w = 0; w < kCvtWarps; ++w) {
+              const int mat = (MODE == kGateUp && w >= 2) ? 1 : 0;
+              const int row = b_y + 32 * (MODE == kGateUp ? (w & 1) : w);
+              tma_load_2d(b0 + 4096 * w + 2048, &a.mapBp[ti.kind * 2 + mat], kb * 64, row, &lfull[stage]);
+              tma_load_2d(b0 + 4096 * w + 1024, &a.mapBx[ti.kind * 2 + mat], row, kb, &lfull[stage]);
+            }
+          } else if (CG == 1) {
             mbar_arrive_expect_tx(&full[stage], tx);
             tma_load_2d(sA + stage * sa_bytes, amap, kb * KE, a_y, &full[stage]);
             tma_load_2d(b0, bmap, kb * KE, b_y, &full[stage]);
@@ -293,10 +384,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
           if (++stage == S) { stage = 0; phase ^= 1u; }
         }
       }
-      if (!ok && (CG == 1 || leader)) {
+      if (!ok && (F4 || CG == 1 || leader)) {
         // Let the copies already in flight land before the CTA goes away.
         for (int s = 0; s < S; ++s)
-          if (issued[s] >= 0) mbar_wait_drain(&full[s], static_cast<uint32_t>(issued[s]), kDrainNs);
+          if (issued[s] >= 0) mbar_wait_drain(F4 ? &lfull[s] : &full[s], static_cast<uint32_t>(issued[s]), kDrainNs);
       }
     }
   } else if (warp == 1) {
@@ -325,7 +416,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
         // (gate/up: the 64 gate rows then the 64 up rows of its output columns).
         const uint32_t idesc = ti.swap ? idesc_of(256, ti.nt) : (ti.small ? idesc_small : idesc_full);
         for (int kb = 0; kb < nkb; ++kb) {
-          if (!mbar_wait(&full[stage], phase, abort, a.err, a.timeout_ns)) { ok = false; break; }
+          // FP4: full completes on the converter warps' cluster-scope release arrivals.
+          const bool got = F4 ? mbar_wait_acq_cluster(&full[stage], phase, abort, a.err, a.timeout_ns)
+                              : mbar_wait(&full[stage], phase, abort, a.err, a.timeout_ns);
+          if (!got) { ok = false; break; }
           tc_fence_after();
           // A swapped tile reads the weight rows as its A operand and the token
           // rows as its B operand (the same K order, so the same bits per element).
@@ -359,6 +453,29 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_grouped_gemm(const __grid_c
       if (CG == 2) umma_commit_pair_mc(tdone, 0x1);
       else umma_commit(tdone);
       mbar_wait_drain(tdone, 0, kDrainNs);
+    }
+  } else if (F4 && warp >= 2 + kEpiWarps) {
+    // ----------------------------------------------------- FP4 converters
+    // Warp w expands its 32 weight rows of every stage in the order the
+    // producer fills them, then releases the stage to the MMA issuer.
+    const int w = warp - 2 - kEpiWarps;
+    const uint32_t full0c = CG == 2 ? mapa_shared(full, 0) : smem_u32(full);
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int t = cluster_id; ok && t < total; t += n_clusters) {
+      Tile ti;
+      decode_tile<CG>(a, s_tile_start, t, ti);
+      const int nkb = a.k_kind[ti.kind] / KE;
+      for (int kb = 0; kb < nkb; ++kb) {
+        ok = mbar_wait(&lfull[stage], phase, abort, a.err, a.timeout_ns);
+        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+        fp4_expand_rows(sB + stage * sb_bytes, w, lane, s_lut);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_release_cluster(full0c + 8 * stage);
+        if (++stage == S) { stage = 0; phase ^= 1u; }
+      }
     }
   } else {
     // --------------------------------------------------------- epilogue
@@ -712,9 +829,10 @@ cudaLaunchConfig_t pair_config(int grid, cudaStream_t s, cudaLaunchAttribute* at
   return cfg;
 }
 
-template <int MODE, int CG, int ACT = MOE_ACT_SWIGLU, int F8 = 0>
+template <int MODE, int CG, int ACT = MOE_ACT_SWIGLU, int F8 = 0, int F4 = 0>
 cudaError_t launch_one(const GemmArgs& a, int grid, cudaStream_t s) {
-  return launch_k(k_grouped_gemm<MODE, CG, ACT, F8>, dim3(grid), dim3(kGemmThreads), kGemmSmem, s, CG == 2, a);
+  return launch_k(k_grouped_gemm<MODE, CG, ACT, F8, F4>, dim3(grid), dim3(F4 ? kGemmThreadsF4 : kGemmThreads),
+                  kGemmSmem, s, CG == 2, a);
 }
 
 int g_pair_clusters[64] = {0};
@@ -734,6 +852,9 @@ void gemm_prepare() {
   cudaFuncSetAttribute(k_grouped_gemm<kDown, 2, 0, 0>, smem_attr, kGemmSmem);
   cudaFuncSetAttribute(k_grouped_gemm<kDown, 2, 0, 1>, smem_attr, kGemmSmem);
   cudaFuncSetAttribute(k_grouped_gemm<kRouter, 1, 0, 0>, smem_attr, kGemmSmem);
+  cudaFuncSetAttribute(k_grouped_gemm<kGateUp, 2, MOE_ACT_SWIGLU, 1, 1>, smem_attr, kGemmSmem);
+  cudaFuncSetAttribute(k_grouped_gemm<kGateUp, 2, MOE_ACT_SITU_GLU, 1, 1>, smem_attr, kGemmSmem);
+  cudaFuncSetAttribute(k_grouped_gemm<kDown, 2, 0, 1, 1>, smem_attr, kGemmSmem);
   // How many CTA pairs fit on the device at once: the persistent pair grid is
   // never larger, so no pair waits for another to finish before it starts.
   cudaLaunchAttribute attr[1];
@@ -750,6 +871,10 @@ void gemm_prepare() {
   occ(reinterpret_cast<const void*>(k_grouped_gemm<kGateUp, 2, 1, 1>));
   occ(reinterpret_cast<const void*>(k_grouped_gemm<kDown, 2, 0, 0>));
   occ(reinterpret_cast<const void*>(k_grouped_gemm<kDown, 2, 0, 1>));
+  cfg.blockDim = dim3(kGemmThreadsF4, 1, 1);
+  occ(reinterpret_cast<const void*>(k_grouped_gemm<kGateUp, 2, 0, 1, 1>));
+  occ(reinterpret_cast<const void*>(k_grouped_gemm<kGateUp, 2, 1, 1, 1>));
+  occ(reinterpret_cast<const void*>(k_grouped_gemm<kDown, 2, 0, 1, 1>));
   cudaGetLastError();
   if (dev >= 0 && dev < 64) g_pair_clusters[dev] = n;
   done_dev = dev;
@@ -764,6 +889,15 @@ int gemm_max_pairs() {
 cudaError_t launch_grouped_gemm(int mode, const GemmArgs& a, int grid, cudaStream_t s) {
   if (grid <= 0) return cudaSuccess;
   const bool f8 = a.fp8 != 0;
+  if (a.fp4 != 0) {
+    switch (mode) {
+      case kGateUp:
+        return a.act == MOE_ACT_SITU_GLU ? launch_one<kGateUp, 2, MOE_ACT_SITU_GLU, 1, 1>(a, grid, s)
+                                         : launch_one<kGateUp, 2, MOE_ACT_SWIGLU, 1, 1>(a, grid, s);
+      case kDown: return launch_one<kDown, 2, 0, 1, 1>(a, grid, s);
+      default: return cudaErrorInvalidValue;   // the router GEMM stays bf16
+    }
+  }
   switch (mode) {
     case kGateUp:
       if (a.act == MOE_ACT_SITU_GLU)

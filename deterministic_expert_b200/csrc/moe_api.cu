@@ -20,13 +20,17 @@ struct moe_handle {
   moe_weights w;
   int S = 0, G = 0, E_pad = 0, bn_gu = 0, bn_dn = 0, num_sms = 0, device = 0, max_pairs = 0;
   int L = 0;                          // width the router and routed experts read (latent or D)
-  bool fp8 = false;                   // MOE_WEIGHTS_FP8: E4M3 expert GEMMs
+  bool fp8 = false;                   // MOE_WEIGHTS_FP8 or _FP4: E4M3 expert GEMMs
+  bool fp4 = false;                   // MOE_WEIGHTS_FP4: packed E2M1 weights expanded on chip
   int ep_world = 1, ep_rank = 0;      // expert parallelism (1: none)
   int E_loc = 0;                      // routed experts held here (E / ep_world)
   long long cap = 0;                  // rows a rank can receive: ep_world * T_max * k
   int bn_pd = 0, bn_pu = 0;           // N tiles of the latent down / up projections
   uint16_t* w_router_pad = nullptr;  // [E_pad, L], rows >= E zero
   CUtensorMap map_router, map_wg, map_wu, map_wd, map_wsg, map_wsu, map_wsd, map_pd, map_pu;
+  // MOE_WEIGHTS_FP4: the expert matrices as packed codes and their exponent words.
+  CUtensorMap pmap_wg, pmap_wu, pmap_wd, pmap_wsg, pmap_wsu, pmap_wsd;
+  CUtensorMap xmap_wg, xmap_wu, xmap_wd, xmap_wsg, xmap_wsu, xmap_wsd;
   unsigned long long timeout_ns = 2000ull * 1000 * 1000;
   // Decode-sized batches run the shared experts (which need no routing) on an
   // auxiliary stream while the routing front end runs on the caller's stream;
@@ -185,6 +189,39 @@ bool make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t rows, ui
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// MOE_WEIGHTS_FP4: a [rows, K] expert matrix stored as packed E2M1 codes
+// (uint8 [rows, K/2]): boxes of 64 bytes (128 codes, one stage of K) x 32 rows,
+// no swizzle (a converter warp's rows, 64 bytes apart).
+bool make_packed_map(CUtensorMap* m, const void* ptr, uint64_t K, uint64_t rows) {
+  std::memset(m, 0, sizeof(*m));
+  if (rows == 0 || ptr == nullptr) return true;
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {K / 2, rows};
+  cuuint64_t strides[1] = {K / 2};
+  cuuint32_t box[2] = {64, 32};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ... and its exponent words (uint32 [K/128, rows]): boxes of 32 words (32 rows)
+// x 1 chunk of K.
+bool make_exp_map(CUtensorMap* m, const void* ptr, uint64_t K, uint64_t rows) {
+  std::memset(m, 0, sizeof(*m));
+  if (rows == 0 || ptr == nullptr) return true;
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {rows, K / 128};
+  cuuint64_t strides[1] = {rows * 4};
+  cuuint32_t box[2] = {32, 1};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int validate_config(const moe_config* c, const moe_weights* w) {
@@ -205,15 +242,27 @@ int validate_config(const moe_config* c, const moe_weights* w) {
         c->situ_beta_up < 3.0e38f))
     return MOE_EINVAL;
   if (c->D % 64 || c->I % 64 || (c->n_shared > 0 && c->I_shared % 64)) return MOE_EUNSUPPORTED;
-  if (c->weight_format != MOE_WEIGHTS_BF16 && c->weight_format != MOE_WEIGHTS_FP8) return MOE_EINVAL;
+  if (c->weight_format != MOE_WEIGHTS_BF16 && c->weight_format != MOE_WEIGHTS_FP8 &&
+      c->weight_format != MOE_WEIGHTS_FP4)
+    return MOE_EINVAL;
   if (c->ep_world < 0 || c->ep_world > 8 || c->ep_rank < 0 || (c->ep_world > 1 && c->ep_rank >= c->ep_world))
     return MOE_EINVAL;
   if (c->ep_world > 1 && (c->E % c->ep_world || c->latent > 0)) return MOE_EUNSUPPORTED;
   if (c->ep_world > 1 && static_cast<long long>(c->ep_world) * c->T_max * c->k >= (1ll << 24))
     return MOE_EUNSUPPORTED;   // return addresses keep the row in 24 bits
-  if (c->weight_format == MOE_WEIGHTS_FP8 &&
+  if (c->weight_format != MOE_WEIGHTS_BF16 &&
       (c->D % 128 || c->I % 128 || (c->n_shared > 0 && c->I_shared % 128) || c->latent % 128))
     return MOE_EUNSUPPORTED;
+  // FP4: every CTA of a pair expands 128 weight rows a stage (four converter
+  // warps of 32), so gate/up tiles of 128 columns and down tiles of 256.
+  if (c->weight_format == MOE_WEIGHTS_FP4 && (c->D % 256 || c->latent % 256)) return MOE_EUNSUPPORTED;
+  if (c->weight_format == MOE_WEIGHTS_FP4) {
+    if (!w->w_gate_exp || !w->w_up_exp || !w->w_down_exp) return MOE_EINVAL;
+    if (c->n_shared > 0 && (!w->ws_gate_exp || !w->ws_up_exp || !w->ws_down_exp)) return MOE_EINVAL;
+    const void* ep[] = {w->w_gate_exp, w->w_up_exp, w->w_down_exp, w->ws_gate_exp, w->ws_up_exp, w->ws_down_exp};
+    for (const void* p : ep)
+      if (p && !aligned16(p)) return MOE_EINVAL;
+  }
   if (c->D > 16384 || c->E > 256 || c->k > c->E || c->k > 16 || c->n_shared > 8 || c->T_max > (1 << 20))
     return MOE_EUNSUPPORTED;
   const long long rows = static_cast<long long>(c->T_max) * std::max(c->k, c->n_shared);
@@ -415,6 +464,9 @@ int forward_impl(moe_handle* h, int T, const uint16_t* x, const uint16_t* residu
       g.a_rows[0] = TK; g.a_rows[1] = T;
       g.out_rows[0] = TK; g.out_rows[1] = h->S * T;
       g.mapB[0] = h->map_wg; g.mapB[1] = h->map_wu; g.mapB[2] = h->map_wsg; g.mapB[3] = h->map_wsu;
+      g.fp4 = h->fp4;
+      g.mapBp[0] = h->pmap_wg; g.mapBp[1] = h->pmap_wu; g.mapBp[2] = h->pmap_wsg; g.mapBp[3] = h->pmap_wsu;
+      g.mapBx[0] = h->xmap_wg; g.mapBx[1] = h->xmap_wu; g.mapBx[2] = h->xmap_wsg; g.mapBx[3] = h->xmap_wsu;
       g.offsets = offsets; g.G = h->G; g.E = c.E; g.T = T;
       g.n_kind[0] = c.I; g.n_kind[1] = c.I_shared;
       g.k_kind[0] = LW; g.k_kind[1] = c.D;
@@ -459,6 +511,9 @@ int forward_impl(moe_handle* h, int T, const uint16_t* x, const uint16_t* residu
       g.a_rows[0] = TK; g.a_rows[1] = h->S * T;
       g.out_rows[0] = TK; g.out_rows[1] = h->S * T;
       g.mapB[0] = h->map_wd; g.mapB[2] = h->map_wsd;
+      g.fp4 = h->fp4;
+      g.mapBp[0] = h->pmap_wd; g.mapBp[2] = h->pmap_wsd;
+      g.mapBx[0] = h->xmap_wd; g.mapBx[2] = h->xmap_wsd;
       g.offsets = offsets; g.G = h->G; g.E = c.E; g.T = T;
       g.n_kind[0] = LW; g.n_kind[1] = c.D;
       g.k_kind[0] = c.I; g.k_kind[1] = c.I_shared;
@@ -635,7 +690,8 @@ int moe_init(const moe_config* cfg, const moe_weights* w, moe_handle** out) {
   // on CTA pairs: each CTA loads half of a gate/up tile (bn_gu / 2 gate rows and
   // bn_gu / 2 up rows) or half of a down tile (bn_dn / 2 rows).
   h->L = cfg->latent > 0 ? cfg->latent : cfg->D;
-  h->fp8 = cfg->weight_format == MOE_WEIGHTS_FP8;
+  h->fp8 = cfg->weight_format == MOE_WEIGHTS_FP8 || cfg->weight_format == MOE_WEIGHTS_FP4;
+  h->fp4 = cfg->weight_format == MOE_WEIGHTS_FP4;
   h->ep_world = cfg->ep_world > 1 ? cfg->ep_world : 1;
   h->ep_rank = cfg->ep_world > 1 ? cfg->ep_rank : 0;
   h->E_loc = cfg->E / h->ep_world;
@@ -676,6 +732,18 @@ int moe_init(const moe_config* cfg, const moe_weights* w, moe_handle** out) {
             make_map(&h->map_wsd, w->ws_down, c.I_shared, static_cast<uint64_t>(h->S) * c.D, h->bn_dn / 2, eb) &&
             make_map(&h->map_pd, c.latent > 0 ? w->w_proj_down : nullptr, c.D, c.latent, h->bn_pd / 2) &&
             make_map(&h->map_pu, c.latent > 0 ? w->w_proj_up : nullptr, h->L, c.D, h->bn_pu / 2);
+  if (ok && h->fp4) {
+    const uint64_t rg = static_cast<uint64_t>(h->E_loc) * c.I, rd = static_cast<uint64_t>(h->E_loc) * h->L;
+    const uint64_t rsg = static_cast<uint64_t>(h->S) * c.I_shared, rsd = static_cast<uint64_t>(h->S) * c.D;
+    ok = make_packed_map(&h->pmap_wg, w->w_gate, h->L, rg) && make_packed_map(&h->pmap_wu, w->w_up, h->L, rg) &&
+         make_packed_map(&h->pmap_wd, w->w_down, c.I, rd) && make_packed_map(&h->pmap_wsg, w->ws_gate, c.D, rsg) &&
+         make_packed_map(&h->pmap_wsu, w->ws_up, c.D, rsg) &&
+         make_packed_map(&h->pmap_wsd, w->ws_down, c.I_shared, rsd) &&
+         make_exp_map(&h->xmap_wg, w->w_gate_exp, h->L, rg) && make_exp_map(&h->xmap_wu, w->w_up_exp, h->L, rg) &&
+         make_exp_map(&h->xmap_wd, w->w_down_exp, c.I, rd) && make_exp_map(&h->xmap_wsg, w->ws_gate_exp, c.D, rsg) &&
+         make_exp_map(&h->xmap_wsu, w->ws_up_exp, c.D, rsg) &&
+         make_exp_map(&h->xmap_wsd, w->ws_down_exp, c.I_shared, rsd);
+  }
   if (!ok) return fail(MOE_ECUDA);
   *out = h;
   return MOE_OK;
@@ -1056,6 +1124,9 @@ int moe_ep_experts(moe_handle* h, int T, const moe_ep_peers* peers, void* worksp
          !make_map(&g.mapA16[1], xs, c.D, T, 16, eb)))
       return MOE_ECUDA;
     g.mapB[0] = h->map_wg; g.mapB[1] = h->map_wu; g.mapB[2] = h->map_wsg; g.mapB[3] = h->map_wsu;
+    g.fp4 = h->fp4;
+    g.mapBp[0] = h->pmap_wg; g.mapBp[1] = h->pmap_wu; g.mapBp[2] = h->pmap_wsg; g.mapBp[3] = h->pmap_wsu;
+    g.mapBx[0] = h->xmap_wg; g.mapBx[1] = h->xmap_wu; g.mapBx[2] = h->xmap_wsg; g.mapBx[3] = h->xmap_wsu;
     g.offsets = off; g.tile_start = tg; g.G = G; g.E = h->E_loc; g.T = T;
     g.n_kind[0] = c.I; g.n_kind[1] = c.I_shared;
     g.k_kind[0] = h->L; g.k_kind[1] = c.D;
@@ -1099,6 +1170,9 @@ int moe_ep_experts(moe_handle* h, int T, const moe_ep_peers* peers, void* worksp
          !make_map(&g.mapA16[1], as, c.I_shared, srows, 16, eb)))
       return MOE_ECUDA;
     g.mapB[0] = h->map_wd; g.mapB[2] = h->map_wsd;
+    g.fp4 = h->fp4;
+    g.mapBp[0] = h->pmap_wd; g.mapBp[2] = h->pmap_wsd;
+    g.mapBx[0] = h->xmap_wd; g.mapBx[2] = h->xmap_wsd;
     g.offsets = off; g.tile_start = td; g.G = G; g.E = h->E_loc; g.T = T;
     g.n_kind[0] = h->L; g.n_kind[1] = c.D;
     g.k_kind[0] = c.I; g.k_kind[1] = c.I_shared;
@@ -1149,6 +1223,17 @@ int moe_quantize_weights_fp4(const moe_bf16* w, uint8_t* w8, int8_t* block_exp, 
                              void* stream) {
   if (!w || !w8 || rows < 0 || K <= 0 || K % 32 || !aligned16(w) || !aligned16(w8)) return MOE_EINVAL;
   return launch_quant_weights_fp4(w, w8, block_exp, rows * (K / 32), static_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess
+             ? MOE_OK
+             : MOE_ECUDA;
+}
+
+int moe_quantize_weights_fp4_packed(const moe_bf16* w, uint8_t* packed, uint32_t* exps, long long rows, int K,
+                                    void* stream) {
+  if (!w || !packed || !exps || rows < 0 || K <= 0 || K % 128 || !aligned16(w) || !aligned16(packed) ||
+      !aligned16(exps))
+    return MOE_EINVAL;
+  return launch_quant_weights_fp4_packed(w, packed, exps, rows, K, static_cast<cudaStream_t>(stream)) ==
                  cudaSuccess
              ? MOE_OK
              : MOE_ECUDA;

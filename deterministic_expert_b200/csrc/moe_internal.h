@@ -47,6 +47,8 @@ constexpr int kBK = 64;
 constexpr int kStages = 4;
 constexpr int kEpiWarps = 8;       // two per TMEM lane quarter, splitting the columns
 constexpr int kGemmThreads = 64 + 32 * kEpiWarps;  // warp 0: TMA, warp 1: MMA, warps 2-9: epilogue
+constexpr int kCvtWarps = 4;                        // FP4 weights: warps 10-13 expand them to E4M3
+constexpr int kGemmThreadsF4 = kGemmThreads + 32 * kCvtWarps;
 constexpr int kSmemA = kBM * kBK * 2;
 constexpr int kSmemBMax = 256 * kBK * 2;
 constexpr int kEpiBytes = 32 * 128;  // per epilogue warp: 32 rows x 128 B, XOR-swizzled
@@ -60,6 +62,9 @@ struct GemmArgs {
   CUtensorMap mapA16[2];  // ... and a 16-row box (swapped tiles of up to 32 tokens)
   CUtensorMap mapB[4];    // B operands: [kind * 2 + 0] first (gate / down / router),
                           //             [kind * 2 + 1] second (up; gate/up only)
+  CUtensorMap mapBp[4];   // fp4: the same B operands as packed E2M1 codes (uint8 [rows, K/2],
+                          //      64-byte x 32-row boxes, no swizzle)
+  CUtensorMap mapBx[4];   // fp4: their block exponents (uint32 [K/128, rows], 32-word boxes)
   const int* offsets;     // [E + 1] grouped-row offsets of the routed groups
   const int* tile_start;  // [G + 1] first tile of each group; NULL: one group of T rows
   int G, E, T;
@@ -77,6 +82,8 @@ struct GemmArgs {
                           // this many tiles per group, group s at tiles [s * n, (s + 1) * n)
   int out_bf16;           // down-mode output as bf16 instead of fp32 (latent projection)
   int fp8;                // expert GEMMs: A and B are E4M3 codes (kind::f8f6f4)
+  int fp4;                // fp8 with B stored as packed E2M1 + block exponents (expanded
+                          // to E4M3 in shared memory by the converter warps)
   int ep;                 // down, routed: dest_row = rank << 24 | row, stored at out_rank[rank]
   int ep_world;           // ep: ranks
   int a_rows[2];          // rows of each kind's A tensor (index checks; 0 = unchecked)
@@ -115,6 +122,10 @@ cudaError_t launch_quant_rows(const uint16_t* a0, int rows0, int w0, uint8_t* q0
 // FP4 (E2M1, power-of-two scale per 32-element block) -> E4M3 weights.
 cudaError_t launch_quant_weights_fp4(const uint16_t* w, uint8_t* w8, int8_t* block_exp, long long nblocks,
                                      cudaStream_t s);
+// The same quantisation in storage form: packed E2M1 codes [rows, K/2] and the
+// block exponents as uint32 [K/128, rows] (four int8 per word).
+cudaError_t launch_quant_weights_fp4_packed(const uint16_t* w, uint8_t* packed, uint32_t* exps, long long rows,
+                                            int K, cudaStream_t s);
 // topk_w == NULL: every slot weighs 1.
 cudaError_t launch_combine_norm(const float* y_slot, const float* topk_w, const float* y_shared,
                                 int k, int S, const uint16_t* residual, const uint16_t* g,

@@ -81,7 +81,74 @@ __global__ void __launch_bounds__(256) k_quant_weights_fp4(const uint16_t* __res
   if (block_exp != nullptr) block_exp[b] = static_cast<int8_t>(s);
 }
 
+// Index of the nearest E2M1 magnitude to x >= 0 in 0, 0.5, 1, 1.5, 2, 3, 4, 6
+// (the same thresholds and ties as e2m1_rn).
+__device__ __forceinline__ uint32_t e2m1_index_rn(float x) {
+  if (x <= 0.25f) return 0;
+  if (x < 0.75f) return 1;
+  if (x <= 1.25f) return 2;
+  if (x < 1.75f) return 3;
+  if (x <= 2.5f) return 4;
+  if (x < 3.5f) return 5;
+  if (x <= 5.f) return 6;
+  return 7;
+}
+
+// The storage form: one thread per 32-element block writes its 16 bytes of
+// packed E2M1 codes and its exponent byte (word [c, row] of exps, byte kb % 4).
+__global__ void __launch_bounds__(256) k_quant_weights_fp4_packed(const uint16_t* __restrict__ w,
+                                                                  uint8_t* __restrict__ packed,
+                                                                  uint8_t* __restrict__ exps_bytes,
+                                                                  long long nblocks, int kblocks,
+                                                                  long long rows) {
+  const long long b = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (b >= nblocks) return;
+  const uint4* src = reinterpret_cast<const uint4*>(w + b * kFp4Block);
+  float v[kFp4Block];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint4 u = src[i];
+    const uint32_t word[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      v[8 * i + 2 * j] = bf16_lo(word[j]);
+      v[8 * i + 2 * j + 1] = bf16_hi(word[j]);
+    }
+  }
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < kFp4Block; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  const int s = fp4_block_exp(amax);
+  const float down = exp2_int(-s);
+  uint32_t out[kFp4Block / 8];
+#pragma unroll
+  for (int i = 0; i < kFp4Block / 8; ++i) {
+    uint32_t word = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float x = v[8 * i + j];
+      const uint32_t code = e2m1_index_rn(__fmul_rn(fabsf(x), down)) | (signbit(x) ? 8u : 0u);
+      word |= code << (4 * j);
+    }
+    out[i] = word;
+  }
+  *reinterpret_cast<uint4*>(packed + b * (kFp4Block / 2)) = make_uint4(out[0], out[1], out[2], out[3]);
+  const long long row = b / kblocks, kb = b - row * kblocks;
+  exps_bytes[((kb >> 2) * rows + row) * 4 + (kb & 3)] = static_cast<uint8_t>(static_cast<int8_t>(s));
+}
+
 }  // namespace
+
+cudaError_t launch_quant_weights_fp4_packed(const uint16_t* w, uint8_t* packed, uint32_t* exps, long long rows,
+                                            int K, cudaStream_t s) {
+  const long long nblocks = rows * (K / kFp4Block);
+  if (nblocks <= 0) return cudaSuccess;
+  const long long grid = (nblocks + 255) / 256;
+  if (grid > 0x7FFFFFFFll) return cudaErrorInvalidValue;
+  k_quant_weights_fp4_packed<<<static_cast<unsigned>(grid), 256, 0, s>>>(
+      w, packed, reinterpret_cast<uint8_t*>(exps), nblocks, K / kFp4Block, rows);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_quant_weights_fp4(const uint16_t* w, uint8_t* w8, int8_t* block_exp, long long nblocks,
                                      cudaStream_t s) {

@@ -124,7 +124,7 @@ __device__ __forceinline__ uint2 e4m3x8(const float (&v)[8], float inv_scale) {
 }
 
 template <int NC>
-__global__ void __launch_bounds__(kRowThreads) k_rmsnorm_rows(const uint16_t* __restrict__ x,
+__global__ void __launch_bounds__(kRowThreads, NC <= 4 ? 6 : 1) k_rmsnorm_rows(const uint16_t* __restrict__ x,
                                                               const uint16_t* __restrict__ g,
                                                               uint16_t* __restrict__ y, int D,
                                                               float eps, int* err, int32_t* zero,
@@ -140,20 +140,25 @@ __global__ void __launch_bounds__(kRowThreads) k_rmsnorm_rows(const uint16_t* __
   const size_t row = blockIdx.x;
   const int nch = D / 8;
   const uint16_t* xr = x + row * D;
-  f8 v[NC];
+  // The row stays in registers as packed bf16 (4 words per 8-element chunk),
+  // half the registers of unpacked floats, so more rows fit on an SM.
+  uint4 v[NC];
   double ss = 0.0;
 #pragma unroll
   for (int i = 0; i < NC; ++i) {
     const int c = threadIdx.x + i * kRowThreads;
-    if (c < nch) v[i] = ld_bf16x8(xr + 8 * c);
+    if (c < nch) v[i] = *reinterpret_cast<const uint4*>(xr + 8 * c);
   }
 #pragma unroll
   for (int i = 0; i < NC; ++i) {
     const int c = threadIdx.x + i * kRowThreads;
     if (c < nch) {
+      const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
 #pragma unroll
-      for (int q = 0; q < 8; ++q)
-        ss = fma(static_cast<double>(v[i].v[q]), static_cast<double>(v[i].v[q]), ss);
+      for (int q = 0; q < 8; ++q) {
+        const double e = static_cast<double>(q & 1 ? bf16_hi(w[q >> 1]) : bf16_lo(w[q >> 1]));
+        ss = fma(e, e, ss);
+      }
     }
   }
   // The squares of bf16 values are exact in fp64 and their fp64 sum is exact
@@ -168,20 +173,19 @@ __global__ void __launch_bounds__(kRowThreads) k_rmsnorm_rows(const uint16_t* __
     const int c = threadIdx.x + i * kRowThreads;
     if (c < nch) {
       const f8 gg = ld_bf16x8(g + 8 * c);
+      const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
       uint32_t o[8];
 #pragma unroll
-      for (int q = 0; q < 8; ++q)
-        o[q] = f64_to_bf16_rne(__dmul_rn(__dmul_rn(static_cast<double>(v[i].v[q]), inv),
-                                         static_cast<double>(gg.v[q])));
-      *reinterpret_cast<uint4*>(yr + 8 * c) =
-          make_uint4(o[0] | (o[1] << 16), o[2] | (o[3] << 16), o[4] | (o[5] << 16), o[6] | (o[7] << 16));
+      for (int q = 0; q < 8; ++q) {
+        const float xv = q & 1 ? bf16_hi(w[q >> 1]) : bf16_lo(w[q >> 1]);
+        o[q] = f64_to_bf16_rne(__dmul_rn(__dmul_rn(static_cast<double>(xv), inv), static_cast<double>(gg.v[q])));
+      }
+      v[i] = make_uint4(o[0] | (o[1] << 16), o[2] | (o[3] << 16), o[4] | (o[5] << 16), o[6] | (o[7] << 16));
+      *reinterpret_cast<uint4*>(yr + 8 * c) = v[i];
       if (yq != nullptr) {
-        // Keep the bf16 values (what the expert GEMMs read) for the E4M3 copy.
+        // The E4M3 copy below reads these bf16 values (what the expert GEMMs read).
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          v[i].v[q] = bf16_lo(o[q]);
-          amax = fmaxf(amax, fabsf(v[i].v[q]));
-        }
+        for (int q = 0; q < 8; ++q) amax = fmaxf(amax, fabsf(bf16_lo(o[q])));
       }
     }
   }
@@ -193,7 +197,12 @@ __global__ void __launch_bounds__(kRowThreads) k_rmsnorm_rows(const uint16_t* __
 #pragma unroll
   for (int i = 0; i < NC; ++i) {
     const int c = threadIdx.x + i * kRowThreads;
-    if (c < nch) *reinterpret_cast<uint2*>(qr + 8 * c) = e4m3x8(v[i].v, inv_scale);
+    if (c < nch) {
+      float o[8];
+      o[0] = bf16_lo(v[i].x); o[1] = bf16_hi(v[i].x); o[2] = bf16_lo(v[i].y); o[3] = bf16_hi(v[i].y);
+      o[4] = bf16_lo(v[i].z); o[5] = bf16_hi(v[i].z); o[6] = bf16_lo(v[i].w); o[7] = bf16_hi(v[i].w);
+      *reinterpret_cast<uint2*>(qr + 8 * c) = e4m3x8(o, inv_scale);
+    }
   }
   if (threadIdx.x == 0) yq_exp[row] = static_cast<int8_t>(e);
 }

@@ -101,7 +101,7 @@ typedef enum moe_activation {
  * FP8, and the experts run FP8 x FP8 GEMMs). */
 typedef enum moe_weight_format {
   MOE_WEIGHTS_BF16 = 0,  /* bf16 weights, bf16 x bf16 GEMMs                          */
-  MOE_WEIGHTS_FP8 = 1    /* E4M3 bytes (as moe_quantize_weights_fp4 writes them),
+  MOE_WEIGHTS_FP8 = 1,   /* E4M3 bytes (as moe_quantize_weights_fp4 writes them),
                             E4M3 x E4M3 GEMMs with fp32 accumulation.  Each expert
                             GEMM's input rows are E4M3 with one power-of-two scale
                             per row: e = the smallest integer with max|row| <=
@@ -112,6 +112,20 @@ typedef enum moe_weight_format {
                             is h (with a latent width, the routed experts' input
                             is z).  The router GEMM and the latent projections stay
                             bf16.  Needs D, I, I_shared and latent multiples of 128. */
+  MOE_WEIGHTS_FP4 = 2    /* FP4 storage: each expert matrix [rows, K] is held as packed
+                            E2M1 codes, uint8 [rows, K / 2] (element 2i in the low
+                            nibble of byte i, 2i + 1 in the high nibble; bit 3 of a code
+                            is the sign, bits 0-2 the index of the magnitude in
+                            0, 0.5, 1, 1.5, 2, 3, 4, 6), plus its block exponents
+                            (moe_weights.*_exp): one power-of-two scale 2^s per 32
+                            consecutive elements of a row, s in [-8, 6].  The GEMMs
+                            expand each weight tile to the E4M3 values code * 2^s in
+                            shared memory (exact: every such product is an E4M3 value)
+                            and then compute exactly as MOE_WEIGHTS_FP8 does, so the
+                            results are bit for bit those of the E4M3 weights that
+                            moe_quantize_weights_fp4 writes for the same master weights.
+                            Half a byte per weight (plus 1/32 byte of exponent) instead
+                            of one.  Same shape limits as MOE_WEIGHTS_FP8.            */
 } moe_weight_format;
 
 typedef struct moe_config {
@@ -151,7 +165,8 @@ typedef struct moe_config {
 
 typedef struct moe_weights {      /* device pointers, caller-owned; L = latent if
                                      latent > 0, else D.  The six expert matrices are
-                                     bf16 or E4M3 bytes, as weight_format says.       */
+                                     bf16, E4M3 bytes or packed E2M1 codes ([rows, K/2]
+                                     bytes), as weight_format says.                   */
   const moe_bf16* w_router;       /* [E, L]      (unused for hash routing)            */
   const float* router_bias;       /* [E] fp32 or NULL: logit bias (softmax) or
                                      selection bias (sigmoid)                         */
@@ -165,6 +180,18 @@ typedef struct moe_weights {      /* device pointers, caller-owned; L = latent i
   const moe_bf16* g_out;          /* [D] output RMSNorm gain                          */
   const moe_bf16* w_proj_down;    /* [latent, D] latent down-projection (latent > 0)  */
   const moe_bf16* w_proj_up;      /* [D, latent] latent up-projection (latent > 0)    */
+  /* MOE_WEIGHTS_FP4 only (else NULL): the block exponents of the six expert
+   * matrices, as moe_quantize_weights_fp4_packed writes them: for a matrix of
+   * R rows (all experts stacked: E*I for w_gate / w_up, E*L for w_down, S*I_shared
+   * for ws_gate / ws_up, S*D for ws_down) and K columns, uint32 [K / 128, R]:
+   * word [c, r] holds the four int8 exponents of row r's 32-element blocks
+   * 4c .. 4c + 3, block 4c in the lowest byte. */
+  const uint32_t* w_gate_exp;
+  const uint32_t* w_up_exp;
+  const uint32_t* w_down_exp;
+  const uint32_t* ws_gate_exp;
+  const uint32_t* ws_up_exp;
+  const uint32_t* ws_down_exp;
 } moe_weights;
 
 typedef struct moe_handle moe_handle;
@@ -353,6 +380,20 @@ int moe_layer_forward_noalloc(moe_handle* h, int T, const moe_bf16* x, const moe
  * multiple of 32), MOE_ECUDA (launch). */
 int moe_quantize_weights_fp4(const moe_bf16* w, uint8_t* w8, int8_t* block_exp, long long rows, int K,
                              void* stream);
+
+/* The same FP4 quantisation (DeepSeek V4 infra notes, §6.2: FP4 (E2M1) weights
+ * with one scale per block) written in its storage form for
+ * MOE_WEIGHTS_FP4: `packed` uint8 [rows, K / 2], two E2M1 codes per byte (element
+ * 2i in the low nibble; sign in bit 3, magnitude index in bits 0-2; a value that
+ * rounds to zero keeps its sign), and `exps` uint32 [K / 128, rows], word [c, r]
+ * holding the int8 exponents s of row r's blocks 4c .. 4c + 3 (block 4c in the
+ * lowest byte).  Block scale and rounding exactly as moe_quantize_weights_fp4, so
+ * code * 2^s is the E4M3 value that function writes.  K must be a multiple of
+ * 128; all pointers 16-byte aligned device memory.  Asynchronous on `stream`.
+ * Errors: MOE_EINVAL (NULL, misaligned, rows < 0, K not a positive multiple of
+ * 128), MOE_ECUDA (launch). */
+int moe_quantize_weights_fp4_packed(const moe_bf16* w, uint8_t* packed, uint32_t* exps, long long rows,
+                                    int K, void* stream);
 
 /* ------------------------------------------------------------------------
  * Expert parallelism (DeepSeek V4 infra notes, §6.1: dispatch -> compute ->

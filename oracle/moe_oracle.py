@@ -335,7 +335,10 @@ def expert_ffn(xn_rows, w_gate, w_up, w_down, gate_clamp_max=np.inf, up_clamp=np
 # scale per row (row-local, so batch-invariant); products accumulate exactly
 # and the row scale is applied to the sum.  Every quantisation step divides by
 # a power of two (exact) and rounds to nearest, ties to even.
-WEIGHTS_BF16, WEIGHTS_FP8 = 0, 1
+# WEIGHTS_FP4 is the storage form of the same FP4 weights ([DS] §6.2: FP4 with
+# a scale per block, dequantised losslessly to FP8): its GEMMs read the same FP8
+# values, so the oracle computes it exactly as WEIGHTS_FP8.
+WEIGHTS_BF16, WEIGHTS_FP8, WEIGHTS_FP4 = 0, 1, 2
 E2M1_GRID = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])   # magnitudes, code order
 FP4_BLOCK = 32
 FP4_SCALE_MIN, FP4_SCALE_MAX = -8, 6     # 2^s keeps every q * 2^s an E4M3 value
@@ -492,7 +495,8 @@ def expert_ffn_fp8(xn_rows, w8_gate, w8_up, w8_down, gate_clamp_max=np.inf, up_c
 
 def expert_fn(cfg):
     """expert_ffn or expert_ffn_fp8, by the configuration's weight format."""
-    return expert_ffn_fp8 if int(getattr(cfg, "weight_format", WEIGHTS_BF16)) == WEIGHTS_FP8 else expert_ffn
+    fmt = int(getattr(cfg, "weight_format", WEIGHTS_BF16))
+    return expert_ffn_fp8 if fmt in (WEIGHTS_FP8, WEIGHTS_FP4) else expert_ffn
 
 
 # ------------------------------------------------------------ latent MoE

@@ -61,7 +61,8 @@ class MoEConfig:
     situ_beta_gate: float = 4.0
     situ_beta_up: float = 25.0
     latent: int = 0                 # latent MoE width (0: none)
-    weight_format: int = 0          # 0 bf16 experts, 1 FP4-valued experts stored as E4M3
+    weight_format: int = 0          # 0 bf16 experts, 1 FP4-valued experts stored as E4M3,
+                                    # 2 the same experts stored as packed E2M1 + block exponents
 
     def with_T(self, T: int) -> "MoEConfig":
         return dataclasses.replace(self, T=T)
@@ -107,10 +108,15 @@ EPILOGUE_SIGMA = 1.0 / 8.0
 
 # The latent workload with FP4 expert weights (routed and shared).
 C6F = dataclasses.replace(C6, name="latent_situ_fp8", weight_format=1)
+# The same FP4 experts in their storage form (packed E2M1 codes, half a byte a
+# weight, plus block exponents), expanded to E4M3 on chip by the GEMMs.
+C1P = dataclasses.replace(C1, name="tiny_fp4", weight_format=2)
+C2P = dataclasses.replace(C2, name="fine_grained_fp4", weight_format=2)
+C6P = dataclasses.replace(C6, name="latent_situ_fp4", weight_format=2)
 # A small case of the V3-shaped kernels for profiler captures (a few GB on the
 # device): the same D, I, top-8 and about 256 rows per expert, with 32 experts.
 C3P = dataclasses.replace(C3, name="v3_shaped_e32", T=1024, E=32)
-CONFIGS = {c.name: c for c in (C1, C2, C3, C5, C5H, C2S, C6, C1F, C2F, C6F, C3P)}
+CONFIGS = {c.name: c for c in (C1, C2, C3, C5, C5H, C2S, C6, C1F, C2F, C6F, C3P, C1P, C2P, C6P)}
 
 _ZIPF_FILE = os.path.join(os.path.dirname(os.path.abspath(__file__)), "zipf_beta.json")
 ZIPF_S = 1.2
@@ -237,19 +243,20 @@ def moe_flops(cfg: MoEConfig, T: int | None = None) -> dict:
             "total": routed + shared + router + proj, "gateup": gateup, "down": routed + shared - gateup}
 
 
-def weight_elem_bytes(cfg: MoEConfig) -> int:
-    """Bytes per expert weight element as the GEMMs read them (bf16 or E4M3)."""
-    return 1 if cfg.weight_format else 2
+def weight_bytes(cfg: MoEConfig, n: int) -> int:
+    """HBM bytes of n expert weights as the GEMMs read them: bf16 (2), E4M3 (1),
+    or packed E2M1 (1/2) plus one 4-byte exponent word per 128 weights (1/32)."""
+    return {0: 2 * n, 1: n, 2: n * 17 // 32}[cfg.weight_format]
 
 
 def expert_bytes(cfg: MoEConfig) -> int:
-    return 3 * (cfg.latent or cfg.D) * cfg.I * weight_elem_bytes(cfg)
+    return weight_bytes(cfg, 3 * (cfg.latent or cfg.D) * cfg.I)
 
 
 def layer_bytes(cfg: MoEConfig, T: int, distinct_experts: int) -> int:
     """Algorithmic HBM bytes: the touched routed experts, shared and router
     weights, x and residual in, two bf16 outputs."""
-    w = distinct_experts * expert_bytes(cfg) + cfg.n_shared * 3 * cfg.D * cfg.I_shared * weight_elem_bytes(cfg)
+    w = distinct_experts * expert_bytes(cfg) + weight_bytes(cfg, cfg.n_shared * 3 * cfg.D * cfg.I_shared)
     if cfg.router != ROUTER_HASH:
         w += cfg.E * (cfg.latent or cfg.D) * 2
     w += 2 * cfg.D * cfg.latent * 2   # latent projections
@@ -261,11 +268,14 @@ def pretty(cfg: MoEConfig) -> str:
     r = {0: "softmax", 1: "sigmoid+bias", 2: "hash"}[cfg.router]
     act = "" if cfg.activation == 0 else f" SiTU-GLU({cfg.situ_beta_gate:g},{cfg.situ_beta_up:g})"
     lat = f" latent={cfg.latent}" if cfg.latent else ""
-    if cfg.weight_format:
-        act += " FP4 weights (E4M3 x E4M3 GEMMs)"
+    if cfg.weight_format == 1:
+        act += " FP4 weights as E4M3 bytes (E4M3 x E4M3 GEMMs)"
+    elif cfg.weight_format == 2:
+        act += " FP4 weights packed (E2M1 + block exponents, expanded on chip; E4M3 x E4M3 GEMMs)"
     return (f"{cfg.name}: T={cfg.T} D={cfg.D}{lat} E={cfg.E} top-{cfg.k} {r} I={cfg.I} "
             f"shared={cfg.n_shared}x{cfg.I_shared}{act}")
 
 
-__all__ = ["MoEConfig", "C1", "C1F", "C2", "C2F", "C2S", "C3", "C4_T", "C5", "C5H", "C6", "C6F", "CONFIGS", "STREAM", "SEED",
+__all__ = ["MoEConfig", "C1", "C1F", "C1P", "C2", "C2F", "C2P", "C2S", "C3", "C4_T", "C5", "C5H", "C6", "C6F", "C6P",
+           "CONFIGS", "STREAM", "SEED",
            "host_bf16", "host_router_bias", "host_token_ids", "moe_flops", "math"]

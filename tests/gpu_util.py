@@ -29,9 +29,12 @@ class Run:
         self.T_max = T_max or max(self.T, 1)
         if weights is None:
             weights = SD.device_weights(cfg, device=device)
-            if cfg.weight_format:
+            if cfg.weight_format == 1:
                 # FP4 expert weights: the library's own quantiser writes their E4M3 codes.
                 weights = moe.quantize_expert_weights(weights)
+            elif cfg.weight_format == 2:
+                # ... or their storage form (packed E2M1 codes and exponent words).
+                weights = moe.pack_expert_weights_fp4(weights)
         self.w = weights
         self.layer = moe.MoELayer(layer_config(cfg, self.T_max), self.w)
         self.device = device

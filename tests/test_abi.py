@@ -116,6 +116,14 @@ def test_weight_format_and_expert_shard_checks():
         moe.MoELayer(ep, {"w_gate": torch.empty(E * I * D, dtype=torch.bfloat16)})
     with pytest.raises(ValueError):   # the router is whole on every rank
         moe.MoELayer(ep, {"w_router": torch.empty(2 * D, dtype=torch.bfloat16)})
+    # Packed FP4 storage: half a byte per weight, one int32 exponent word per 128.
+    fp4 = moe.LayerConfig(D=D, E=E, k=2, I=I, weight_format=moe.WEIGHTS_FP4)
+    with pytest.raises(ValueError):   # E4M3 bytes (one per weight) are not the packed form
+        moe.MoELayer(fp4, {"w_gate": torch.empty(E * I * D, dtype=torch.uint8)})
+    with pytest.raises(ValueError):   # exponent words of the wrong count
+        moe.MoELayer(fp4, {"w_gate_exp": torch.empty(E * I * D // 64, dtype=torch.int32)})
+    with pytest.raises(ValueError):   # ... or type
+        moe.MoELayer(fp4, {"w_gate_exp": torch.empty(E * I * D // 128, dtype=torch.uint8)})
 
 
 def test_header_is_plain_c_and_links(tmp_path):

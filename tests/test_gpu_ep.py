@@ -35,6 +35,7 @@ CASES = {
     "situ_w2": (dataclasses.replace(W.C1, activation=1, name="tiny_situ"), 2, [90, 40]),
     "fine_grained_w4": (W.C2, 4, [512, 300, 1, 1024]),
     "fine_grained_fp8_w2": (W.C2F, 2, [700, 333]),
+    "tiny_fp4_w4": (W.C1P, 4, [50, 7, 200, 64]),
 }
 
 
@@ -46,8 +47,10 @@ def test_virtual_ep_matches_single_device(torch_cuda, case):
     T = sum(Ts)
     cfg = base.with_T(T)
     weights = SD.device_weights(cfg)
-    if cfg.weight_format:
+    if cfg.weight_format == 1:
         weights = moe.quantize_expert_weights(weights)
+    elif cfg.weight_format == 2:
+        weights = moe.pack_expert_weights_fp4(weights)
     x, r, ids = SD.device_inputs(cfg, T=T)
     # The single-device layer over all T tokens.
     single = moe.MoELayer(SD.layer_config(cfg, T), weights)

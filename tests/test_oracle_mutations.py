@@ -89,7 +89,7 @@ MUTATIONS = {
     "act_scale_not_applied": ("h = round_bf16(glu_unit((qx @ Wg.T) * sx, (qx @ Wu.T) * sx,",
                               "h = round_bf16(glu_unit((qx @ Wg.T), (qx @ Wu.T),"),
     "down_input_not_quantised": ("return h, (qh @ Wd.T) * np.exp2(eh)[:, None]", "return h, h @ Wd.T"),
-    "fp8_path_ignored": ("return expert_ffn_fp8 if int(getattr(cfg, \"weight_format\", WEIGHTS_BF16)) == WEIGHTS_FP8 else expert_ffn",
+    "fp8_path_ignored": ("return expert_ffn_fp8 if fmt in (WEIGHTS_FP8, WEIGHTS_FP4) else expert_ffn",
                          "return expert_ffn"),
     "fp4_nibbles_swapped": ("return (c[..., 0::2] | (c[..., 1::2] << 4)).astype(np.uint8), np.asarray(s).astype(np.int8)",
                             "return (c[..., 1::2] | (c[..., 0::2] << 4)).astype(np.uint8), np.asarray(s).astype(np.int8)"),
