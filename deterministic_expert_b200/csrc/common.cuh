@@ -246,6 +246,20 @@ __device__ __forceinline__ void mbar_arrive_release_cluster(uint32_t cluster_add
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
+// Bulk copy of `bytes` (a multiple of 16, 16-byte aligned ends) from this
+// CTA's shared memory to shared memory of a CTA of the cluster, completing
+// that many transaction bytes on the mbarrier at `bar_cluster` (in the
+// destination CTA) when the data has landed.  An async-proxy operation: it is
+// ordered after this thread's earlier fence.proxy.async.
+__device__ __forceinline__ void bulk_copy_s2cluster(uint32_t dst_cluster, const void* src, uint32_t bytes,
+                                                    uint32_t bar_cluster) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          dst_cluster),
+      "r"(smem_u32(src)), "r"(bytes), "r"(bar_cluster)
+      : "memory");
+}
+
 // Make this thread's generic-proxy shared-memory writes visible to the async
 // proxy (the tensor core's operand reads).
 __device__ __forceinline__ void fence_proxy_async_smem() {

@@ -54,7 +54,7 @@ constexpr uint32_t kTmemCols = 512;
 constexpr int kMaxGroups = 256 + 8;   // routed experts + shared experts (checked by moe_init)
 constexpr int kRingBytes = kStages * (kSmemA + kSmemBMax);  // shared memory of the stage ring
 constexpr int kRingMax = 12;                                // most stages any variant uses
-constexpr int kBarBytes = 512;                              // mbarrier region after the ring
+constexpr int kBarBytes = kGemmBarBytes;                    // mbarrier region after the ring
 constexpr unsigned long long kDrainNs = 200ull * 1000 * 1000;  // 200 ms
 
 template <int CG>
@@ -163,12 +163,14 @@ __device__ __forceinline__ float glu_unit(float g, float u, const GemmArgs& a) {
 // stage's B slot in place.  The warp's rows r = 32 w + lane own the E4M3 bytes
 // [4096 w, 4096 w + 4096) of the slot (row r at 128 r, its 16-byte chunk c at
 // chunk position c ^ (r & 7): the layout a 128-byte-swizzled TMA load of E4M3
-// rows leaves); their packed E2M1 codes (64 bytes a row) were loaded to
-// 4096 w + 2048 and their exponent words to 4096 w + 1024, inside that span.
-// Every lane reads all of its input before any lane writes (__syncwarp), then
-// writes byte code * 2^s: the magnitude from the exponent's 8-entry table
-// (lut[s + 8], E4M3 codes of 0, 0.5, 1, 1.5, 2, 3, 4, 6 times 2^s) picked by
-// prmt, the sign bit from bit 3 of the code.
+// rows leaves).  Their packed E2M1 codes (64 bytes a row) arrive in two
+// 64-row boxes, rows 0-63 at byte 2048 and rows 64-127 at byte 10240 of the
+// slot, which puts every warp's input inside its own 4 KB span; the lane's
+// exponent word (its row's four 32-element blocks of this stage) comes in a
+// register.  Every lane reads all of its input before any lane writes
+// (__syncwarp), then writes byte code * 2^s: the magnitude from the
+// exponent's 8-entry table (lut[s + 8], E4M3 codes of 0, 0.5, 1, 1.5, 2, 3, 4,
+// 6 times 2^s) picked by prmt, the sign bit from bit 3 of the code.
 // prmt.b32 in its default mode: byte n of the result is byte (c >> 4n) & 7 of
 // {b, a} (a = bytes 0-3), or, when bit 3 of that selector nibble is set, that
 // byte's top bit replicated over all 8 bits.
@@ -188,12 +190,12 @@ __device__ __forceinline__ uint32_t e2m1x4_to_e4m3(uint32_t codes16, uint32_t lu
   return mag | (neg & 0x80808080u);
 }
 
-__device__ __forceinline__ void fp4_expand_rows(uint8_t* slot, int w, int lane, const uint32_t (*lut)[2]) {
-  const uint8_t* in = slot + 4096 * w + 2048 + 64 * lane;
+__device__ __forceinline__ void fp4_expand_rows(uint8_t* slot, int w, int lane, uint32_t ex,
+                                                const uint32_t (*lut)[2]) {
+  const uint8_t* in = slot + 2048 + 8192 * (w >> 1) + 64 * (32 * (w & 1) + lane);
   uint4 p[4];
 #pragma unroll
   for (int j = 0; j < 4; ++j) p[j] = *reinterpret_cast<const uint4*>(in + 16 * j);
-  const uint32_t ex = *reinterpret_cast<const uint32_t*>(slot + 4096 * w + 1024 + 4 * lane);
   __syncwarp();
   const int r = 32 * w + lane;
   uint8_t* out = slot + 128 * r;
@@ -253,9 +255,11 @@ __global__ void __launch_bounds__(F4 ? kGemmThreadsF4 : kGemmThreads, 1)
   // FP4: each CTA's own TMA loads of a stage complete lfull; full then counts
   // the converter warps of both CTAs (the expanded tile is what the MMA reads).
   uint64_t* lfull = gempty + 4;  // [kRingMax]
+
   uint8_t* epi = reinterpret_cast<uint8_t*>(bars) + kBarBytes;  // kEpiWarps x kEpiBytes
   __shared__ uint32_t tmem_slot;
   __shared__ uint32_t s_lut[F4 ? 15 : 1][2];
+  __shared__ __align__(16) uint32_t s_signal[4];   // FP4: source and target of the odd CTA's signal copies
   __shared__ int abort_flag;
   __shared__ int s_tile_start[kMaxGroups + 1];
 
@@ -277,7 +281,9 @@ __global__ void __launch_bounds__(F4 ? kGemmThreadsF4 : kGemmThreads, 1)
   }
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
-      mbar_init(&full[s], F4 ? CG * kCvtWarps : 1);
+      // FP4: the even CTA's producer (expecting the odd CTA's converter
+      // signals as transaction bytes) and its converter warps.
+      mbar_init(&full[s], F4 ? 1 + kCvtWarps : 1);
       mbar_init(&empty[s], 1);
       if (F4) mbar_init(&lfull[s], 1);
     }
@@ -353,19 +359,21 @@ __global__ void __launch_bounds__(F4 ? kGemmThreadsF4 : kGemmThreads, 1)
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort, a.err, a.timeout_ns)) { ok = false; break; }
           uint8_t* b0 = sB + stage * sb_bytes;
           if (F4) {
-            // This CTA's A rows, and for each converter warp w its 32 weight rows
-            // as packed E2M1 codes (64 bytes a row, to 4096 w + 2048 of the slot)
-            // with their exponent words (to 4096 w + 1024); gate/up: warps 0-1
-            // gate rows, 2-3 up rows.  All counted on this CTA's lfull.
-            mbar_arrive_expect_tx(&lfull[stage], static_cast<uint32_t>(box) * 128 + kCvtWarps * (32 * 64 + 32 * 4));
+            // This CTA's A rows and its 128 weight rows as packed E2M1 codes in
+            // two 64-row boxes (gate/up: the gate rows, then the up rows;
+            // down: rows 0-63, then 64-127), to bytes 2048 and 10240 of the
+            // slot.  All counted on this CTA's lfull.
+            mbar_arrive_expect_tx(&lfull[stage], static_cast<uint32_t>(box) * 128 + 2 * 64 * 64);
+            // The even CTA's full also expects the odd CTA's converter warps'
+            // 16-byte signal copies (one per warp per stage).
+            if (CG == 2 && leader) mbar_arrive_expect_tx(&full[stage], kCvtWarps * 16);
+            else if (CG == 1) mbar_arrive(&full[stage]);
             tma_load_2d(sA + stage * sa_bytes, amap, kb * KE, a_y, &lfull[stage]);
-#pragma unroll
-            for (int w = 0; w < kCvtWarps; ++w) {
-              const int mat = (MODE == kGateUp && w >= 2) ? 1 : 0;
-              const int row = b_y + 32 * (MODE == kGateUp ? (w & 1) : w);
-              tma_load_2d(b0 + 4096 * w + 2048, &a.mapBp[ti.kind * 2 + mat], kb * 64, row, &lfull[stage]);
-              tma_load_2d(b0 + 4096 * w + 1024, &a.mapBx[ti.kind * 2 + mat], row, kb, &lfull[stage]);
-            }
+            tma_load_2d(b0 + 2048, &a.mapBp[ti.kind * 2], kb * 64, b_y, &lfull[stage]);
+            if (MODE == kGateUp)
+              tma_load_2d(b0 + 10240, &a.mapBp[ti.kind * 2 + 1], kb * 64, b_y, &lfull[stage]);
+            else
+              tma_load_2d(b0 + 10240, &a.mapBp[ti.kind * 2], kb * 64, b_y + 64, &lfull[stage]);
           } else if (CG == 1) {
             mbar_arrive_expect_tx(&full[stage], tx);
             tma_load_2d(sA + stage * sa_bytes, amap, kb * KE, a_y, &full[stage]);
@@ -385,9 +393,14 @@ __global__ void __launch_bounds__(F4 ? kGemmThreadsF4 : kGemmThreads, 1)
         }
       }
       if (!ok && (F4 || CG == 1 || leader)) {
-        // Let the copies already in flight land before the CTA goes away.
+        // Let the copies already in flight land before the CTA goes away
+        // (FP4: this CTA's loads on lfull, and on the even CTA's full the odd
+        // CTA's signal copies, bounded like every other wait).
         for (int s = 0; s < S; ++s)
-          if (issued[s] >= 0) mbar_wait_drain(F4 ? &lfull[s] : &full[s], static_cast<uint32_t>(issued[s]), kDrainNs);
+          if (issued[s] >= 0) {
+            mbar_wait_drain(F4 ? &lfull[s] : &full[s], static_cast<uint32_t>(issued[s]), kDrainNs);
+            if (F4 && leader) mbar_wait_drain(&full[s], static_cast<uint32_t>(issued[s]), kDrainNs);
+          }
       }
     }
   } else if (warp == 1) {
@@ -457,9 +470,18 @@ __global__ void __launch_bounds__(F4 ? kGemmThreadsF4 : kGemmThreads, 1)
   } else if (F4 && warp >= 2 + kEpiWarps) {
     // ----------------------------------------------------- FP4 converters
     // Warp w expands its 32 weight rows of every stage in the order the
-    // producer fills them, then releases the stage to the MMA issuer.
+    // producer fills them, then hands the stage to the MMA issuer: each lane
+    // fences its writes into the async proxy, and after __syncwarp lane 0 of
+    // an even-CTA warp arrives on full, while lane 0 of an odd-CTA warp
+    // issues a 16-byte bulk copy to the even CTA that completes its bytes on
+    // full (an async-proxy signal, ordered after the fenced writes, that
+    // leaves the warp free to go on).  Each lane's exponent words are read
+    // from global memory two stages ahead.
     const int w = warp - 2 - kEpiWarps;
-    const uint32_t full0c = CG == 2 ? mapa_shared(full, 0) : smem_u32(full);
+    const uint32_t full0c = mapa_shared(full, 0);
+    const uint32_t sig0c = mapa_shared(s_signal, 0);
+    const int mat = (MODE == kGateUp && w >= 2) ? 1 : 0;
+    const int row_in = MODE == kGateUp ? 32 * (w & 1) + lane : 32 * w + lane;
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
@@ -467,13 +489,23 @@ __global__ void __launch_bounds__(F4 ? kGemmThreadsF4 : kGemmThreads, 1)
       Tile ti;
       decode_tile<CG>(a, s_tile_start, t, ti);
       const int nkb = a.k_kind[ti.kind] / KE;
+      const int sel = ti.kind * 2 + mat;
+      const int row = ti.idx * a.n_kind[ti.kind] + ti.n * BN + static_cast<int>(rank) * (BN / 2) + row_in;
+      const uint32_t* xp = a.bexp[sel] + row;
+      const size_t xstride = static_cast<size_t>(a.bexp_rows[sel]);
+      uint32_t ex0 = __ldg(xp), ex1 = nkb > 1 ? __ldg(xp + xstride) : 0u;
       for (int kb = 0; kb < nkb; ++kb) {
         ok = mbar_wait(&lfull[stage], phase, abort, a.err, a.timeout_ns);
         if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-        fp4_expand_rows(sB + stage * sb_bytes, w, lane, s_lut);
+        fp4_expand_rows(sB + stage * sb_bytes, w, lane, ex0, s_lut);
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive_release_cluster(full0c + 8 * stage);
+        if (lane == 0) {
+          if (leader) mbar_arrive(&full[stage]);
+          else bulk_copy_s2cluster(sig0c, s_signal, 16, full0c + 8 * stage);
+        }
+        ex0 = ex1;
+        if (kb + 2 < nkb) ex1 = __ldg(xp + static_cast<size_t>(kb + 2) * xstride);
         if (++stage == S) { stage = 0; phase ^= 1u; }
       }
     }

@@ -30,7 +30,6 @@ struct moe_handle {
   CUtensorMap map_router, map_wg, map_wu, map_wd, map_wsg, map_wsu, map_wsd, map_pd, map_pu;
   // MOE_WEIGHTS_FP4: the expert matrices as packed codes and their exponent words.
   CUtensorMap pmap_wg, pmap_wu, pmap_wd, pmap_wsg, pmap_wsu, pmap_wsd;
-  CUtensorMap xmap_wg, xmap_wu, xmap_wd, xmap_wsg, xmap_wsu, xmap_wsd;
   unsigned long long timeout_ns = 2000ull * 1000 * 1000;
   // Decode-sized batches run the shared experts (which need no routing) on an
   // auxiliary stream while the routing front end runs on the caller's stream;
@@ -190,8 +189,8 @@ bool make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t rows, ui
 }
 
 // MOE_WEIGHTS_FP4: a [rows, K] expert matrix stored as packed E2M1 codes
-// (uint8 [rows, K/2]): boxes of 64 bytes (128 codes, one stage of K) x 32 rows,
-// no swizzle (a converter warp's rows, 64 bytes apart).
+// (uint8 [rows, K/2]): boxes of 64 bytes (128 codes, one stage of K) x 64 rows,
+// no swizzle (rows 64 bytes apart).
 bool make_packed_map(CUtensorMap* m, const void* ptr, uint64_t K, uint64_t rows) {
   std::memset(m, 0, sizeof(*m));
   if (rows == 0 || ptr == nullptr) return true;
@@ -199,26 +198,10 @@ bool make_packed_map(CUtensorMap* m, const void* ptr, uint64_t K, uint64_t rows)
   if (!fn) return false;
   cuuint64_t dims[2] = {K / 2, rows};
   cuuint64_t strides[1] = {K / 2};
-  cuuint32_t box[2] = {64, 32};
+  cuuint32_t box[2] = {64, 64};
   cuuint32_t estr[2] = {1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-// ... and its exponent words (uint32 [K/128, rows]): boxes of 32 words (32 rows)
-// x 1 chunk of K.
-bool make_exp_map(CUtensorMap* m, const void* ptr, uint64_t K, uint64_t rows) {
-  std::memset(m, 0, sizeof(*m));
-  if (rows == 0 || ptr == nullptr) return true;
-  auto fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[2] = {rows, K / 128};
-  cuuint64_t strides[1] = {rows * 4};
-  cuuint32_t box[2] = {32, 1};
-  cuuint32_t estr[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void*>(ptr), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -281,6 +264,23 @@ int validate_config(const moe_config* c, const moe_weights* w) {
 // tile with at most ceil(T rounded up to 16 / 2) token rows per CTA; the GEMM
 // then sizes its stages' A slot to the TMA box that covers them (16, 64 or 128
 // rows).  0: the default 16 KB slot.
+// MOE_WEIGHTS_FP4: the exponent words the expert GEMM's converter warps read
+// (base and rows of each B operand, as mapB orders them).
+void fp4_exponents(const moe_handle* h, GemmArgs& g, bool gateup) {
+  if (!h->fp4) return;
+  const moe_config& c = h->cfg;
+  if (gateup) {
+    g.bexp[0] = h->w.w_gate_exp; g.bexp[1] = h->w.w_up_exp;
+    g.bexp[2] = h->w.ws_gate_exp; g.bexp[3] = h->w.ws_up_exp;
+    g.bexp_rows[0] = g.bexp_rows[1] = h->E_loc * c.I;
+    g.bexp_rows[2] = g.bexp_rows[3] = h->S * c.I_shared;
+  } else {
+    g.bexp[0] = h->w.w_down_exp; g.bexp[2] = h->w.ws_down_exp;
+    g.bexp_rows[0] = h->E_loc * h->L;
+    g.bexp_rows[2] = h->S * c.D;
+  }
+}
+
 int small_batch_a_bytes(int T) {
   if (T >= 256) return 0;
   const int rows = ((T + 15) / 16 * 16) / 2;
@@ -466,7 +466,7 @@ int forward_impl(moe_handle* h, int T, const uint16_t* x, const uint16_t* residu
       g.mapB[0] = h->map_wg; g.mapB[1] = h->map_wu; g.mapB[2] = h->map_wsg; g.mapB[3] = h->map_wsu;
       g.fp4 = h->fp4;
       g.mapBp[0] = h->pmap_wg; g.mapBp[1] = h->pmap_wu; g.mapBp[2] = h->pmap_wsg; g.mapBp[3] = h->pmap_wsu;
-      g.mapBx[0] = h->xmap_wg; g.mapBx[1] = h->xmap_wu; g.mapBx[2] = h->xmap_wsg; g.mapBx[3] = h->xmap_wsu;
+      fp4_exponents(h, g, true);
       g.offsets = offsets; g.G = h->G; g.E = c.E; g.T = T;
       g.n_kind[0] = c.I; g.n_kind[1] = c.I_shared;
       g.k_kind[0] = LW; g.k_kind[1] = c.D;
@@ -513,7 +513,7 @@ int forward_impl(moe_handle* h, int T, const uint16_t* x, const uint16_t* residu
       g.mapB[0] = h->map_wd; g.mapB[2] = h->map_wsd;
       g.fp4 = h->fp4;
       g.mapBp[0] = h->pmap_wd; g.mapBp[2] = h->pmap_wsd;
-      g.mapBx[0] = h->xmap_wd; g.mapBx[2] = h->xmap_wsd;
+      fp4_exponents(h, g, false);
       g.offsets = offsets; g.G = h->G; g.E = c.E; g.T = T;
       g.n_kind[0] = LW; g.n_kind[1] = c.D;
       g.k_kind[0] = c.I; g.k_kind[1] = c.I_shared;
@@ -738,11 +738,7 @@ int moe_init(const moe_config* cfg, const moe_weights* w, moe_handle** out) {
     ok = make_packed_map(&h->pmap_wg, w->w_gate, h->L, rg) && make_packed_map(&h->pmap_wu, w->w_up, h->L, rg) &&
          make_packed_map(&h->pmap_wd, w->w_down, c.I, rd) && make_packed_map(&h->pmap_wsg, w->ws_gate, c.D, rsg) &&
          make_packed_map(&h->pmap_wsu, w->ws_up, c.D, rsg) &&
-         make_packed_map(&h->pmap_wsd, w->ws_down, c.I_shared, rsd) &&
-         make_exp_map(&h->xmap_wg, w->w_gate_exp, h->L, rg) && make_exp_map(&h->xmap_wu, w->w_up_exp, h->L, rg) &&
-         make_exp_map(&h->xmap_wd, w->w_down_exp, c.I, rd) && make_exp_map(&h->xmap_wsg, w->ws_gate_exp, c.D, rsg) &&
-         make_exp_map(&h->xmap_wsu, w->ws_up_exp, c.D, rsg) &&
-         make_exp_map(&h->xmap_wsd, w->ws_down_exp, c.I_shared, rsd);
+         make_packed_map(&h->pmap_wsd, w->ws_down, c.I_shared, rsd);
   }
   if (!ok) return fail(MOE_ECUDA);
   *out = h;
@@ -1126,7 +1122,7 @@ int moe_ep_experts(moe_handle* h, int T, const moe_ep_peers* peers, void* worksp
     g.mapB[0] = h->map_wg; g.mapB[1] = h->map_wu; g.mapB[2] = h->map_wsg; g.mapB[3] = h->map_wsu;
     g.fp4 = h->fp4;
     g.mapBp[0] = h->pmap_wg; g.mapBp[1] = h->pmap_wu; g.mapBp[2] = h->pmap_wsg; g.mapBp[3] = h->pmap_wsu;
-    g.mapBx[0] = h->xmap_wg; g.mapBx[1] = h->xmap_wu; g.mapBx[2] = h->xmap_wsg; g.mapBx[3] = h->xmap_wsu;
+    fp4_exponents(h, g, true);
     g.offsets = off; g.tile_start = tg; g.G = G; g.E = h->E_loc; g.T = T;
     g.n_kind[0] = c.I; g.n_kind[1] = c.I_shared;
     g.k_kind[0] = h->L; g.k_kind[1] = c.D;
@@ -1172,7 +1168,7 @@ int moe_ep_experts(moe_handle* h, int T, const moe_ep_peers* peers, void* worksp
     g.mapB[0] = h->map_wd; g.mapB[2] = h->map_wsd;
     g.fp4 = h->fp4;
     g.mapBp[0] = h->pmap_wd; g.mapBp[2] = h->pmap_wsd;
-    g.mapBx[0] = h->xmap_wd; g.mapBx[2] = h->xmap_wsd;
+    fp4_exponents(h, g, false);
     g.offsets = off; g.tile_start = td; g.G = G; g.E = h->E_loc; g.T = T;
     g.n_kind[0] = h->L; g.n_kind[1] = c.D;
     g.k_kind[0] = c.I; g.k_kind[1] = c.I_shared;

@@ -52,7 +52,8 @@ constexpr int kGemmThreadsF4 = kGemmThreads + 32 * kCvtWarps;
 constexpr int kSmemA = kBM * kBK * 2;
 constexpr int kSmemBMax = 256 * kBK * 2;
 constexpr int kEpiBytes = 32 * 128;  // per epilogue warp: 32 rows x 128 B, XOR-swizzled
-constexpr int kGemmSmem = 1024 + kStages * (kSmemA + kSmemBMax) + 512 + kEpiWarps * kEpiBytes;
+constexpr int kGemmBarBytes = 512;  // the GEMM's mbarriers, after its stage ring
+constexpr int kGemmSmem = 1024 + kStages * (kSmemA + kSmemBMax) + kGemmBarBytes + kEpiWarps * kEpiBytes;
 
 enum GemmMode : int { kGateUp = 0, kDown = 1, kRouter = 2 };
 
@@ -63,8 +64,9 @@ struct GemmArgs {
   CUtensorMap mapB[4];    // B operands: [kind * 2 + 0] first (gate / down / router),
                           //             [kind * 2 + 1] second (up; gate/up only)
   CUtensorMap mapBp[4];   // fp4: the same B operands as packed E2M1 codes (uint8 [rows, K/2],
-                          //      64-byte x 32-row boxes, no swizzle)
-  CUtensorMap mapBx[4];   // fp4: their block exponents (uint32 [K/128, rows], 32-word boxes)
+                          //      64-byte x 64-row boxes, no swizzle)
+  const uint32_t* bexp[4];// fp4: their block exponent words, uint32 [K/128, bexp_rows[i]]
+  int bexp_rows[4];
   const int* offsets;     // [E + 1] grouped-row offsets of the routed groups
   const int* tile_start;  // [G + 1] first tile of each group; NULL: one group of T rows
   int G, E, T;
