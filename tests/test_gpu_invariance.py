@@ -118,3 +118,16 @@ def test_host_pipeline_matches_single_calls(torch_cuda, name, chunks):
     for i in range(3):
         assert torch.equal(hon[i].view(torch.int16), want[i]["out_norm"].cpu().view(torch.int16)), i
         assert torch.equal(hor[i].view(torch.int16), want[i]["out_residual"].cpu().view(torch.int16)), i
+
+
+def test_v3_full_batch_with_wide_tiles_matches_splits(torch_cuda):
+    """The V3-shaped batch (T=8192: about 256 rows per expert, so the GEMMs run
+    wide tiles for experts with 257-320 rows) against four 2048-token splits
+    (64 rows per expert: no wide tiles) and a permuted order: the same bits."""
+    torch = torch_cuda
+    cfg = W.C3
+    run = Run(cfg)
+    x, r, ids = run.inputs()
+    perm = torch.from_numpy(W.token_permutation(cfg.T, salt=7).astype(np.int32)).cuda()
+    ws = torch.empty(run.layer.invariance_workspace_size(cfg.T), dtype=torch.uint8, device="cuda")
+    assert run.layer.check_invariance(x, r, ws, token_ids=ids, n_splits=4, perm=perm, repeats=1) == 0
