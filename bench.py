@@ -625,6 +625,48 @@ def decode_object(a, dev, flush, stream, pk, w, cfg=None):
             "sweep": rows, "gpu_launches": launches}
 
 
+def ep_waves_object(a, dev, flush, stream, w, world=8, T_rank=512, waves=(1, 2, 4)):
+    """Expert parallelism over ``world`` virtual ranks on this one device
+    (VirtualEP, fine-grained weights, T_rank tokens per rank): the step time
+    with the four phases in one stream (waves = 1) and with the experts in
+    waves, the sends of wave w + 1 on a second stream beside the GEMMs of wave
+    w.  Every wave count must give the same bits.  On one device the sends are
+    copies inside HBM, a small share of the step, so this measures what the
+    wave split costs (more, smaller GEMM launches), not what it hides on links."""
+    import torch
+
+    import deterministic_expert_b200 as moe
+    from synth import device as SD
+    from synth import workloads as W
+    cfg = W.C2.with_T(world * T_rank)
+    x, r, _ = SD.device_inputs(cfg, device=dev)
+    ep = moe.VirtualEP(SD.layer_config(cfg, T_rank), w, world, device=dev)
+    xs = [x[q * T_rank:(q + 1) * T_rank].contiguous() for q in range(world)]
+    rs = [r[q * T_rank:(q + 1) * T_rank].contiguous() for q in range(world)]
+    rows, ref = [], None
+    with torch.cuda.stream(stream):
+        for n in waves:
+            times = []
+            for i in range(a.warmup + a.steps):
+                flush.fill_(i & 0xFF)
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                outs = ep.forward(xs, rs, stream=stream, waves=n)
+                e1.record(stream)
+                torch.cuda.synchronize()
+                if i >= a.warmup:
+                    times.append(e0.elapsed_time(e1))
+            got = torch.cat([o[0] for o in outs]).view(torch.int16)
+            ref = got.clone() if ref is None else ref
+            ms = sum(times) / len(times)
+            rows.append({"waves": n, "ms_per_step": round(ms, 4), "tokens_per_s": round(world * T_rank / (ms / 1e3), 1),
+                         "bits_equal_one_wave": bool(torch.equal(got, ref))})
+    if ep.device_errors() != [moe.MOE_OK] * world:
+        raise RuntimeError("device error (virtual expert parallelism)")
+    return {"workload": f"{W.pretty(cfg)}; {world} virtual expert-parallel ranks of {T_rank} tokens on one device",
+            "steps": a.steps, "sweep": rows}
+
+
 def main():
     a = parse()
     if a.impl == "reference":
@@ -758,6 +800,7 @@ def main():
         # The same sweep with the FP4 experts in their storage form (half a
         # byte per weight plus block exponents, expanded to E4M3 on chip).
         sub["decode_fp4"] = decode_object(a, dev, flush, stream, pk, moe.pack_expert_weights_fp4(w2), cfg=W.C2P)
+        sub["ep_waves"] = ep_waves_object(a, dev, flush, stream, w2)
         del w2
 
     if rank == 0:

@@ -124,6 +124,17 @@ def _stream(stream) -> int | None:
     return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
 
 
+def _torch_stream(stream, device):
+    """The caller's stream as a torch stream (None: the current one; a raw
+    cudaStream_t handle is wrapped), for recording and waiting on events."""
+    import torch
+    if stream is None:
+        return torch.cuda.current_stream(device)
+    if hasattr(stream, "cuda_stream"):
+        return stream
+    return torch.cuda.ExternalStream(int(stream), device=device)
+
+
 @dataclass
 class LayerConfig:
     D: int
@@ -722,19 +733,34 @@ class _EPRank:
         _check(L.moe_ep_route(self.layer.handle, int(x.shape[0]), _ptr(x), _ptr(token_ids), xbuf,
                               _ptr(self.ws), self.ws.numel(), _stream(stream)), "moe_ep_route")
 
-    def send(self, T, peers, stream=None):
+    def send(self, T, peers, stream=None, wave=None, n_waves=1):
+        """The whole send (wave None), or the rows of wave ``wave`` of ``n_waves``."""
         L = lib()
-        L.moe_ep_send.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.POINTER(moe_ep_peers), ctypes.c_void_p,
-                                  ctypes.c_size_t, ctypes.c_void_p]
-        _check(L.moe_ep_send(self.layer.handle, T, ctypes.byref(peers), _ptr(self.ws), self.ws.numel(),
-                             _stream(stream)), "moe_ep_send")
+        if wave is None:
+            L.moe_ep_send.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.POINTER(moe_ep_peers), ctypes.c_void_p,
+                                      ctypes.c_size_t, ctypes.c_void_p]
+            _check(L.moe_ep_send(self.layer.handle, T, ctypes.byref(peers), _ptr(self.ws), self.ws.numel(),
+                                 _stream(stream)), "moe_ep_send")
+            return
+        L.moe_ep_send_wave.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.POINTER(moe_ep_peers), ctypes.c_int,
+                                       ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
+        _check(L.moe_ep_send_wave(self.layer.handle, T, ctypes.byref(peers), wave, n_waves, _ptr(self.ws),
+                                  self.ws.numel(), _stream(stream)), "moe_ep_send_wave")
 
-    def experts(self, T, peers, stream=None):
+    def experts(self, T, peers, stream=None, wave=None, n_waves=1):
+        """All of the rank's experts (wave None), or those of wave ``wave`` of ``n_waves``."""
         L = lib()
-        L.moe_ep_experts.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.POINTER(moe_ep_peers), ctypes.c_void_p,
-                                     ctypes.c_size_t, ctypes.c_void_p]
-        _check(L.moe_ep_experts(self.layer.handle, T, ctypes.byref(peers), _ptr(self.ws), self.ws.numel(),
-                                _stream(stream)), "moe_ep_experts")
+        if wave is None:
+            L.moe_ep_experts.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.POINTER(moe_ep_peers),
+                                         ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
+            _check(L.moe_ep_experts(self.layer.handle, T, ctypes.byref(peers), _ptr(self.ws), self.ws.numel(),
+                                    _stream(stream)), "moe_ep_experts")
+            return
+        L.moe_ep_experts_wave.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.POINTER(moe_ep_peers),
+                                          ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t,
+                                          ctypes.c_void_p]
+        _check(L.moe_ep_experts_wave(self.layer.handle, T, ctypes.byref(peers), wave, n_waves, _ptr(self.ws),
+                                     self.ws.numel(), _stream(stream)), "moe_ep_experts_wave")
 
     def combine(self, residual, xbuf, out_norm, out_residual, out_idx=None, out_w=None, stream=None):
         L = lib()
@@ -749,12 +775,17 @@ class _EPRank:
 
 
 class VirtualEP:
-    """``world`` expert-parallel ranks sharing one device and one stream: each
-    rank has its own handle (its block of routed experts), workspace and
-    exchange buffer, and a step runs every rank's route, then every rank's
-    send, experts and combine in stream order, so no kernel waits on another.
-    Each rank's outputs are bit for bit those of the single-device layer on
-    its tokens.  ``weights`` holds all E routed experts."""
+    """``world`` expert-parallel ranks sharing one device: each rank has its own
+    handle (its block of routed experts), workspace and exchange buffer.  With
+    ``waves`` = 1 a step runs every rank's route, send, experts and combine in
+    the order of one stream.  With ``waves`` = n > 1 (wave scheduling, DeepSeek
+    V4 infra notes §6.1 "MegaMoE") the experts are split into n waves: every
+    rank's sends run on a communication stream, wave after wave, and every
+    rank's expert GEMMs on a compute stream, wave w after the event that closes
+    wave w's sends, so the rows of wave w + 1 travel while wave w computes.
+    Ordering is by stream order and events only: no kernel waits on another.
+    Either way each rank's outputs are bit for bit those of the single-device
+    layer on its tokens.  ``weights`` holds all E routed experts."""
 
     def __init__(self, cfg: LayerConfig, weights: dict, world: int, device="cuda"):
         import torch
@@ -762,22 +793,45 @@ class VirtualEP:
             raise ValueError("2 .. 8 ranks")
         self.world = world
         self.ranks = [_EPRank(cfg, weights, r, world, device) for r in range(world)]
+        self.E_loc = cfg.E // world
         self.xbuf = [torch.zeros(max(rk.xbytes, 256), dtype=torch.uint8, device=device) for rk in self.ranks]
         self.peers = moe_ep_peers()
         for r in range(world):
             self.peers.xbuf[r] = _ptr(self.xbuf[r])
+        self._comm = torch.cuda.Stream(device=device)
+        self._comp = torch.cuda.Stream(device=device)
 
-    def forward(self, xs, residuals, token_ids=None, stream=None):
+    def forward(self, xs, residuals, token_ids=None, stream=None, waves: int = 1):
         """xs, residuals: one [T_r, D] bf16 tensor per rank; returns per rank
-        (out_norm, out_residual, topk_idx, topk_w)."""
+        (out_norm, out_residual, topk_idx, topk_w).  ``waves``: 1 .. E / world."""
         import torch
+        if waves < 1 or waves > self.E_loc:
+            raise ValueError(f"waves must be in 1 .. {self.E_loc}")
         ids = token_ids if token_ids is not None else [None] * self.world
+        Ts = [int(x.shape[0]) for x in xs]
         for r, rk in enumerate(self.ranks):
             rk.route(xs[r], ids[r], _ptr(self.xbuf[r]), stream)
-        for r, rk in enumerate(self.ranks):
-            rk.send(int(xs[r].shape[0]), self.peers, stream)
-        for r, rk in enumerate(self.ranks):
-            rk.experts(int(xs[r].shape[0]), self.peers, stream)
+        if waves == 1:
+            for r, rk in enumerate(self.ranks):
+                rk.send(Ts[r], self.peers, stream)
+            for r, rk in enumerate(self.ranks):
+                rk.experts(Ts[r], self.peers, stream)
+        else:
+            main = _torch_stream(stream, self.xbuf[0].device)
+            routed = torch.cuda.Event()
+            routed.record(main)
+            self._comm.wait_event(routed)
+            self._comp.wait_event(routed)
+            for w in range(waves):
+                for r, rk in enumerate(self.ranks):
+                    rk.send(Ts[r], self.peers, self._comm, wave=w, n_waves=waves)
+                sent = torch.cuda.Event()
+                sent.record(self._comm)
+                self._comp.wait_event(sent)
+                for r, rk in enumerate(self.ranks):
+                    rk.experts(Ts[r], self.peers, self._comp, wave=w, n_waves=waves)
+            main.wait_stream(self._comm)
+            main.wait_stream(self._comp)
         outs = []
         for r, rk in enumerate(self.ranks):
             T = int(xs[r].shape[0])
@@ -837,21 +891,51 @@ class EPMoELayer:
             self.peers.xbuf[r] = bases[r] + self._FLAGS
         self.err = torch.zeros(1, dtype=torch.int32, device=dev)
         self._epoch = 0
+        self._comm = self._comp = None
 
     def _barrier(self, stream):
         self._epoch += 1
         peer_barrier(self._flags, self.rank, self._epoch, self.err, self.limit_us, stream)
 
-    def forward(self, x, residual, token_ids=None, stream=None):
+    def forward(self, x, residual, token_ids=None, stream=None, waves: int = 1):
+        """One step.  ``waves`` = n > 1: the experts in n waves, every rank's
+        send of wave w followed by a barrier on a communication stream, and the
+        expert GEMMs of wave w on a compute stream after that barrier, so the
+        rows of wave w + 1 cross the links while wave w computes.  Every rank
+        must pass the same ``waves``: the barriers' epochs follow the same
+        order on every rank (route, the waves' sends, the results)."""
         import torch
         T = int(x.shape[0])
+        E_loc = self.me.cfg.E // self.world
+        if waves < 1 or waves > E_loc:
+            raise ValueError(f"waves must be in 1 .. {E_loc}")
         mine = self.peers.xbuf[self.rank]
         self.me.route(x, token_ids, mine, stream)
         self._barrier(stream)          # every rank's counts are out
-        self.me.send(T, self.peers, stream)
-        self._barrier(stream)          # every row has reached its owner
-        self.me.experts(T, self.peers, stream)
-        self._barrier(stream)          # every result row is back home
+        if waves == 1:
+            self.me.send(T, self.peers, stream)
+            self._barrier(stream)      # every row has reached its owner
+            self.me.experts(T, self.peers, stream)
+            self._barrier(stream)      # every result row is back home
+        else:
+            dev = self.err.device
+            if self._comm is None:
+                self._comm, self._comp = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+            main = _torch_stream(stream, dev)
+            routed = torch.cuda.Event()
+            routed.record(main)
+            self._comm.wait_event(routed)
+            self._comp.wait_event(routed)
+            for w in range(waves):
+                self.me.send(T, self.peers, self._comm, wave=w, n_waves=waves)
+                self._barrier(self._comm)      # wave w's rows have reached their owners
+                arrived = torch.cuda.Event()
+                arrived.record(self._comm)
+                self._comp.wait_event(arrived)
+                self.me.experts(T, self.peers, self._comp, wave=w, n_waves=waves)
+            self._barrier(self._comp)          # every result row is back home
+            main.wait_stream(self._comm)
+            main.wait_stream(self._comp)
         on, orr = torch.empty_like(residual), torch.empty_like(residual)
         idx = torch.empty((T, self.me.cfg.k), dtype=torch.int32, device=on.device)
         w = torch.empty((T, self.me.cfg.k), dtype=torch.float32, device=on.device)

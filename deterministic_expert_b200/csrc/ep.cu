@@ -14,6 +14,14 @@
 //   ep_plan  the owner's per-expert row offsets and the tile lists of its two
 //            expert GEMMs (its E / world routed groups, then its shared groups
 //            over its own tokens).
+//
+// Waves (the wave scheduling of §6.1 there: each wave covers a few experts, and
+// the rows of wave w + 1 travel while the GEMMs of wave w run): both kernels can
+// be limited to local experts [wave_lo, wave_hi) of every owner.  A wave's send
+// writes exactly the rows, addresses and bytes that the whole send writes for
+// those experts, and the wave's plan lists only their tiles (plus the shared
+// experts' in the wave that carries them), so the waves together do the same
+// arithmetic on the same rows as one pass.
 // Stores to other ranks are plain 16-byte stores to peer-mapped memory.
 #include "common.cuh"
 #include "moe_internal.h"
@@ -27,6 +35,7 @@ __global__ void __launch_bounds__(256) k_ep_send(const EpSendArgs a) {
   __shared__ int offs[kEpMaxE + 1];
   __shared__ int dst[kEpMaxE];
   __shared__ int tot[kEpMaxE];
+  __shared__ int seg_start[9], seg_pre[9];
   griddep_wait();
   griddep_launch();
   const int tid = threadIdx.x;
@@ -48,10 +57,26 @@ __global__ void __launch_bounds__(256) k_ep_send(const EpSendArgs a) {
     for (int f = (e / a.E_loc) * a.E_loc; f < e; ++f) base += tot[f];
     dst[e] += base;
   }
+  // This wave's rows: for each owner o, the grouped rows of its experts
+  // o * E_loc + [wave_lo, wave_hi), contiguous in this rank's grouping.
+  if (tid == 0) {
+    int pre = 0;
+    for (int o = 0; o < a.world; ++o) {
+      seg_start[o] = offs[o * a.E_loc + a.wave_lo];
+      seg_pre[o] = pre;
+      pre += offs[o * a.E_loc + a.wave_hi] - seg_start[o];
+    }
+    seg_pre[a.world] = pre;
+  }
   __syncthreads();
+  const int n = seg_pre[a.world];
   const int warp = tid >> 5, lane = tid & 31;
   const int nw = blockDim.x >> 5;
-  for (int p = blockIdx.x * nw + warp; p < a.rows; p += gridDim.x * nw) {
+  for (int q = blockIdx.x * nw + warp; q < n; q += gridDim.x * nw) {
+    int o = 0;
+    while (o + 1 < a.world && seg_pre[o + 1] <= q) ++o;
+    const int p = seg_start[o] + (q - seg_pre[o]);
+    if (!MOE_INDEX_OK(p >= 0 && p < a.rows, a.err)) continue;
     // Expert of grouped row p: the largest e with offs[e] <= p.
     int lo = 0, hi = a.E;
     while (hi - lo > 1) {
@@ -87,19 +112,25 @@ __global__ void __launch_bounds__(256) k_ep_plan(const EpPlanArgs a) {
   if (tid == 0) {
     // At most 264 groups: plain serial scans.
     int o = 0;
-    for (int e = 0; e < a.E_loc; ++e) { a.offsets[e] = o; o += cnt[e]; }
+    for (int e = 0; e < a.E_loc; ++e) {
+      a.offsets[e] = o;
+      if (e == a.wave_lo) a.rows_received[1] = o;
+      if (e == a.wave_hi) a.rows_received[0] = o;
+      o += cnt[e];
+    }
     a.offsets[a.E_loc] = o;
-    *a.rows_received = o;
+    if (a.wave_hi == a.E_loc) a.rows_received[0] = o;
     const int mt_shared = (a.T_self + a.tile_m - 1) / a.tile_m;
     int tg = 0, td = 0;
     for (int g = 0; g < G; ++g) {
       a.tiles_gu[g] = tg;
       a.tiles_dn[g] = td;
       if (g < a.E_loc) {
+        if (g < a.wave_lo || g >= a.wave_hi) continue;
         const int mt = (cnt[g] + a.tile_m - 1) / a.tile_m;
         tg += mt * a.gu_ntiles_routed;
         td += mt * a.dn_ntiles;
-      } else {
+      } else if (a.with_shared) {
         tg += mt_shared * a.gu_ntiles_shared;
         td += mt_shared * a.dn_ntiles_shared;
       }

@@ -110,7 +110,7 @@ Layout layout(const moe_handle* h, int T) {
   L.epoff = take(ep ? static_cast<size_t>(h->E_loc + 1) * 4 : 0);
   L.eptg = take(ep ? gl * 4 : 0);
   L.eptd = take(ep ? gl * 4 : 0);
-  L.eprows = take(ep ? 4 : 0);
+  L.eprows = take(ep ? 8 : 0);
   // E4M3 copy of the latent input z (latent width with E4M3 experts).
   L.zq = take(lat ? f * Tz * Lw : 0);
   L.zqe = take(lat ? f * Tz : 0);
@@ -1004,6 +1004,14 @@ int ep_peers_ok(const moe_handle* h, const moe_ep_peers* p) {
   return MOE_OK;
 }
 
+// Local experts of wave `wave` of `n_waves`: [wave * E_loc / n, (wave + 1) * E_loc / n).
+bool ep_wave(const moe_handle* h, int wave, int n_waves, int* lo, int* hi) {
+  if (n_waves < 1 || n_waves > h->E_loc || wave < 0 || wave >= n_waves) return false;
+  *lo = static_cast<int>(static_cast<long long>(wave) * h->E_loc / n_waves);
+  *hi = static_cast<int>(static_cast<long long>(wave + 1) * h->E_loc / n_waves);
+  return true;
+}
+
 }  // namespace
 
 size_t moe_ep_exchange_size(const moe_handle* h) {
@@ -1032,8 +1040,15 @@ int moe_ep_route(moe_handle* h, int T, const moe_bf16* x, const int32_t* token_i
 
 int moe_ep_send(moe_handle* h, int T, const moe_ep_peers* peers, void* workspace, size_t ws_bytes,
                 void* stream) {
+  return moe_ep_send_wave(h, T, peers, 0, 1, workspace, ws_bytes, stream);
+}
+
+int moe_ep_send_wave(moe_handle* h, int T, const moe_ep_peers* peers, int wave, int n_waves, void* workspace,
+                     size_t ws_bytes, void* stream) {
   int v = ep_check(h, T, workspace, ws_bytes);
   if (v == MOE_OK) v = ep_peers_ok(h, peers);
+  int wlo = 0, whi = 0;
+  if (v == MOE_OK && !ep_wave(h, wave, n_waves, &wlo, &whi)) v = MOE_EINVAL;
   if (v != MOE_OK || T == 0) return v;
   const moe_config& c = h->cfg;
   const Layout L = layout(h, T);
@@ -1057,15 +1072,24 @@ int moe_ep_send(moe_handle* h, int T, const moe_ep_peers* peers, void* workspace
   a.row_bytes = h->L * (h->fp8 ? 1 : 2);
   a.E = c.E; a.E_loc = h->E_loc; a.world = h->ep_world; a.rank = h->ep_rank;
   a.cap = h->cap; a.err = reinterpret_cast<int*>(ws + L.err);
+  a.wave_lo = wlo; a.wave_hi = whi;
   const int grid = std::max(1, std::min((a.rows + 7) / 8, 4 * h->num_sms));
   return launch_ep_send(a, grid, static_cast<cudaStream_t>(stream)) == cudaSuccess ? MOE_OK : MOE_ECUDA;
 }
 
 int moe_ep_experts(moe_handle* h, int T, const moe_ep_peers* peers, void* workspace, size_t ws_bytes,
                    void* stream) {
+  return moe_ep_experts_wave(h, T, peers, 0, 1, workspace, ws_bytes, stream);
+}
+
+int moe_ep_experts_wave(moe_handle* h, int T, const moe_ep_peers* peers, int wave, int n_waves,
+                        void* workspace, size_t ws_bytes, void* stream) {
   int v = ep_check(h, T, workspace, ws_bytes);
   if (v == MOE_OK) v = ep_peers_ok(h, peers);
+  int wlo = 0, whi = 0;
+  if (v == MOE_OK && !ep_wave(h, wave, n_waves, &wlo, &whi)) v = MOE_EINVAL;
   if (v != MOE_OK) return v;
+  const bool with_shared = wave == 0;   // the shared experts run with the first wave
   // T == 0: this rank has no tokens (no shared-expert tiles) but still serves
   // its routed experts for the other ranks.
   const moe_config& c = h->cfg;
@@ -1092,6 +1116,7 @@ int moe_ep_experts(moe_handle* h, int T, const moe_ep_peers* peers, void* worksp
   pa.offsets = off; pa.tiles_gu = tg; pa.tiles_dn = td; pa.rows_received = nrows;
   pa.gu_ntiles_routed = nt_gu; pa.gu_ntiles_shared = nt_gus; pa.dn_ntiles = nt_dn; pa.dn_ntiles_shared = nt_dns;
   pa.tile_m = kPairTileM;
+  pa.wave_lo = wlo; pa.wave_hi = whi; pa.with_shared = with_shared ? 1 : 0;
   MOE_TRY(launch_ep_plan(pa, s));
   const long long cap = h->cap;
   const int G = h->E_loc + h->S;
@@ -1142,14 +1167,14 @@ int moe_ep_experts(moe_handle* h, int T, const moe_ep_peers* peers, void* worksp
     g.err = err; g.timeout_ns = h->timeout_ns;
     MOE_TRY(launch_grouped_gemm(kGateUp, g, pair_grid(h, bound(nt_gu, nt_gus)), s));
   }
-  // 3. E4M3: the received rows' h (only the first rows_received are real) and the shared h.
+  // 3. E4M3: the wave's received rows' h and the shared h.
   uint8_t* hqr = ws + L.hqr;
   int8_t* her = reinterpret_cast<int8_t*>(ws + L.her);
   uint8_t* hqs = ws + L.hqs;
   int8_t* hse = reinterpret_cast<int8_t*>(ws + L.hse);
   if (f8)
-    MOE_TRY(launch_quant_rows(hr, static_cast<int>(cap), c.I, hqr, her, hsb, h->S * T, c.I_shared, hqs, hse,
-                              nrows, s));
+    MOE_TRY(launch_quant_rows(hr, static_cast<int>(cap), c.I, hqr, her, hsb, with_shared ? h->S * T : 0,
+                              c.I_shared, hqs, hse, nrows, s));
   // 4. down: routed rows go back to their source rank's slot rows, shared rows stay here.
   {
     GemmArgs g;

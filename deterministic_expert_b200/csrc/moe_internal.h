@@ -116,8 +116,8 @@ cudaError_t launch_rmsnorm_rows(const uint16_t* x, const uint16_t* g, uint16_t* 
                                 float eps, int* err_to_clear, int32_t* zero, int zero_words,
                                 uint8_t* yq, int8_t* yq_exp, cudaStream_t s);
 // bf16 rows -> E4M3 rows + per-row exponents, two segments.
-// rows0_dev != NULL: only the first *rows0_dev of the rows0 rows of segment 0
-// are real (the rest are skipped).
+// rows0_dev != NULL: only rows [rows0_dev[1], rows0_dev[0]) of the rows0 rows
+// of segment 0 are quantised (the rest are skipped).
 cudaError_t launch_quant_rows(const uint16_t* a0, int rows0, int w0, uint8_t* q0, int8_t* e0,
                               const uint16_t* a1, int rows1, int w1, uint8_t* q1, int8_t* e1,
                               const int32_t* rows0_dev, cudaStream_t s);
@@ -210,6 +210,7 @@ struct EpSendArgs {
   const int32_t* dest_row;   // [rows] grouped row -> token * k + slot
   int rows, row_bytes, E, E_loc, world, rank;
   long long cap;             // rows of each rank's receive buffers
+  int wave_lo, wave_hi;      // rows of every owner's local experts [wave_lo, wave_hi) only
   int* err;                  // device error word (index checks)
 };
 cudaError_t launch_ep_send(const EpSendArgs& a, int grid, cudaStream_t s);
@@ -220,8 +221,10 @@ struct EpPlanArgs {
   int32_t* offsets;          // [E_loc + 1] received rows per local expert
   int32_t* tiles_gu;         // [E_loc + S + 1]
   int32_t* tiles_dn;         // [E_loc + S + 1]
-  int32_t* rows_received;    // [1]
+  int32_t* rows_received;    // [2]: end and start of the wave's received rows
   int gu_ntiles_routed, gu_ntiles_shared, dn_ntiles, dn_ntiles_shared, tile_m;
+  int wave_lo, wave_hi;      // tiles of local experts [wave_lo, wave_hi) only
+  int with_shared;           // and of the shared experts
 };
 cudaError_t launch_ep_plan(const EpPlanArgs& a, cudaStream_t s);
 

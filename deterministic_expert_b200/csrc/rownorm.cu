@@ -221,7 +221,7 @@ __global__ void __launch_bounds__(256) k_quant_rows(const uint16_t* __restrict__
   const int r0 = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   const bool first = r0 < rows0;
   if (!first && r0 >= rows0 + rows1) return;
-  if (first && rows0_dev != nullptr && r0 >= *rows0_dev) return;
+  if (first && rows0_dev != nullptr && (r0 >= rows0_dev[0] || r0 < rows0_dev[1])) return;
   const int r = first ? r0 : r0 - rows0;
   const int w = first ? w0 : w1;
   const uint16_t* ar = (first ? a0 : a1) + static_cast<size_t>(r) * w;

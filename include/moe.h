@@ -449,6 +449,32 @@ int moe_ep_combine(moe_handle* h, int T, const moe_bf16* residual, void* xbuf_se
                    moe_bf16* out_residual, int32_t* out_topk_idx, float* out_topk_w, void* workspace,
                    size_t ws_bytes, void* stream);
 
+/* Waves (DeepSeek V4 infra notes, §6.1 "MegaMoE": the experts are scheduled in
+ * waves, each covering a few of them, so that the rows of the next wave travel
+ * while the current wave computes).  Wave w of n (1 <= n <= E / ep_world,
+ * 0 <= w < n) covers local experts [w * E_loc / n, (w + 1) * E_loc / n) of
+ * every owner, E_loc = E / ep_world; the shared experts run in wave 0.
+ *   moe_ep_send_wave     the part of moe_ep_send whose rows go to the wave's
+ *                        experts: the same rows, return addresses and bytes at
+ *                        the same places.
+ *   moe_ep_experts_wave  moe_ep_experts over the wave's experts only (their
+ *                        received rows, which the wave's send of every rank
+ *                        must have completed), plus the shared experts in wave 0.
+ * moe_ep_send and moe_ep_experts are wave 0 of 1.  Running every wave's send
+ * and experts (in any interleaving that keeps each wave's experts after every
+ * rank's send of that wave, and one rank's experts calls in wave order) stores
+ * the same bits as the two whole calls, because every (token, slot) row still
+ * meets the same weights in the same full-K GEMM and lands in the same slot
+ * row.  The point of the split: the send of wave w + 1 may run on another
+ * stream while the GEMMs of wave w run.  A rank's workspace holds the plan of
+ * one wave at a time, so its experts calls must not overlap one another.
+ * Errors: as moe_ep_send / moe_ep_experts, and MOE_EINVAL for a wave outside
+ * [0, n) or n outside [1, E_loc]. */
+int moe_ep_send_wave(moe_handle* h, int T, const moe_ep_peers* peers, int wave, int n_waves, void* workspace,
+                     size_t ws_bytes, void* stream);
+int moe_ep_experts_wave(moe_handle* h, int T, const moe_ep_peers* peers, int wave, int n_waves,
+                        void* workspace, size_t ws_bytes, void* stream);
+
 /* ------------------------------------------------------------------------
  * Peer memory for the tensor-parallel epilogue (one process per GPU).
  *

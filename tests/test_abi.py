@@ -82,6 +82,8 @@ def test_calls_reject_null_handles():
     assert L.moe_reduce_partials(1, arr, 1 << 20, 1 << 20, 1 << 20, 1 << 20, 4, 100, 1e-6, None) \
         == moe.MOE_EUNSUPPORTED
     assert L.moe_selftest_wait_timeout(0, None) == moe.MOE_EINVAL
+    assert L.moe_ep_send_wave(None, 4, None, 0, 1, None, 0, None) == moe.MOE_EINVAL
+    assert L.moe_ep_experts_wave(None, 4, None, 0, 1, None, 0, None) == moe.MOE_EINVAL
 
 
 def test_weight_size_mismatch_is_refused():

@@ -39,11 +39,54 @@ CASES = {
 }
 
 
+# Wave scheduling (§6.1 "MegaMoE": experts in waves, the next wave's rows in
+# flight while the current wave computes): the same batches split into n
+# waves, sends and GEMMs on two streams, must still give the single-device bits.
+WAVE_CASES = {
+    "tiny_w2_waves2": (W.C1, 2, [37, 100], 2),
+    "tiny_w2_one_expert_per_wave": (W.C1, 2, [129, 64], 4),
+    "tiny_w4_empty_rank_waves2": (W.C1, 4, [40, 0, 70, 25], 2),
+    "tiny_fp8_w2_uneven_waves": (W.C1F, 2, [50, 200], 3),
+    "tiny_fp4_w2_waves2": (W.C1P, 2, [50, 200], 2),
+    "hash_w2_waves2": (dataclasses.replace(W.C1, router=W.ROUTER_HASH, k=3, name="hash_small"), 2, [77, 120], 2),
+    "fine_grained_w4_waves4": (W.C2, 4, [512, 300, 1, 1024], 4),
+    "fine_grained_w8_waves8": (W.C2, 8, [256, 100, 1, 512, 64, 300, 7, 128], 8),
+    "fine_grained_fp8_w2_waves2": (W.C2F, 2, [700, 333], 2),
+}
+
+
 @pytest.mark.parametrize("case", sorted(CASES))
 def test_virtual_ep_matches_single_device(torch_cuda, case):
-    torch = torch_cuda
-    import deterministic_expert_b200 as moe
     base, world, Ts = CASES[case]
+    _check_against_single_device(torch_cuda, base, world, Ts, waves=1)
+
+
+@pytest.mark.parametrize("case", sorted(WAVE_CASES))
+def test_virtual_ep_waves_match_single_device(torch_cuda, case):
+    base, world, Ts, waves = WAVE_CASES[case]
+    _check_against_single_device(torch_cuda, base, world, Ts, waves=waves)
+
+
+def test_virtual_ep_rejects_bad_wave_counts(torch_cuda):
+    import deterministic_expert_b200 as moe
+    cfg = W.C1.with_T(64)
+    ep = moe.VirtualEP(SD.layer_config(cfg, 32), SD.device_weights(cfg), 2)
+    x, r, _ = SD.device_inputs(cfg, T=64)
+    for waves in (0, cfg.E // 2 + 1):
+        with pytest.raises(ValueError):
+            ep.forward([x[:32].contiguous(), x[32:].contiguous()], [r[:32].contiguous(), r[32:].contiguous()],
+                       waves=waves)
+    # The C ABI refuses a wave outside [0, n) and n outside [1, E / world].
+    rk = ep.ranks[0]
+    for wave, n in ((1, 1), (-1, 2), (0, cfg.E // 2 + 1), (0, 0)):
+        with pytest.raises(moe.MoEError):
+            rk.send(32, ep.peers, wave=wave, n_waves=n)
+        with pytest.raises(moe.MoEError):
+            rk.experts(32, ep.peers, wave=wave, n_waves=n)
+
+
+def _check_against_single_device(torch, base, world, Ts, waves):
+    import deterministic_expert_b200 as moe
     T = sum(Ts)
     cfg = base.with_T(T)
     weights = SD.device_weights(cfg)
@@ -65,7 +108,7 @@ def test_virtual_ep_matches_single_device(torch_cuda, case):
     cut = np.concatenate([[0], np.cumsum(Ts)])
     sl = [slice(int(cut[q]), int(cut[q + 1])) for q in range(world)]
     outs = ep.forward([x[s].contiguous() for s in sl], [r[s].contiguous() for s in sl],
-                      [ids[s].contiguous() for s in sl])
+                      [ids[s].contiguous() for s in sl], waves=waves)
     torch.cuda.synchronize()
     assert ep.device_errors() == [0] * world
     assert single.device_error(ws) == 0
