@@ -140,20 +140,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// try_wait with acquire semantics at cluster scope (pairs with a cluster-scope
-// release arrive, mbar_arrive_release_cluster).
-__device__ __forceinline__ bool mbar_try_wait_acq_cluster(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}\n"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
 // Wait for the phase with the given parity to complete, for at most
 // limit_ns nanoseconds.  On time-out it raises *abort (shared by the CTA's
 // roles) and the device error word, and returns false; it also returns
@@ -164,25 +150,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 0) {
-      if (*abort) return false;
-      if (globaltimer_ns() - t0 > limit_ns) {
-        *abort = 1;
-        atomicExch(err, kDevTimeout);
-        return false;
-      }
-    }
-  }
-}
-
-// mbar_wait with a cluster-scope acquire (for phases completed by arrivals
-// from the other CTA of a pair that publish its shared-memory writes).
-__device__ __forceinline__ bool mbar_wait_acq_cluster(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                                      int* err, uint64_t limit_ns) {
-  if (mbar_try_wait_acq_cluster(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait_acq_cluster(bar, parity)) return true;
     if ((it & 63u) == 0) {
       if (*abort) return false;
       if (globaltimer_ns() - t0 > limit_ns) {
@@ -239,29 +206,8 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
-// Arrive with release semantics at cluster scope (the arriving thread's
-// earlier shared-memory writes are visible to a cluster-scope acquire of the
-// phase), on an mbarrier of this CTA or of another CTA of the cluster.
-__device__ __forceinline__ void mbar_arrive_release_cluster(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
-}
-
-// Bulk copy of `bytes` (a multiple of 16, 16-byte aligned ends) from this
-// CTA's shared memory to shared memory of a CTA of the cluster, completing
-// that many transaction bytes on the mbarrier at `bar_cluster` (in the
-// destination CTA) when the data has landed.  An async-proxy operation: it is
-// ordered after this thread's earlier fence.proxy.async.
-__device__ __forceinline__ void bulk_copy_s2cluster(uint32_t dst_cluster, const void* src, uint32_t bytes,
-                                                    uint32_t bar_cluster) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-          dst_cluster),
-      "r"(smem_u32(src)), "r"(bytes), "r"(bar_cluster)
-      : "memory");
-}
-
 // Make this thread's generic-proxy shared-memory writes visible to the async
-// proxy (the tensor core's operand reads).
+// proxy (tensor-core operand reads, tcgen05.cp).
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
@@ -344,6 +290,51 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
 // 128-byte swizzled row, as the bf16 form's 16).
 __host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
   return (1u << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// Block scales (kind::mxf8f6f4.block_scale, one UE8M0 scale per 32 K elements
+// of every row of A and of B).  The scales of a 128-row operand for one 128-wide
+// K stage form a 512-byte atom in shared memory: 16-byte row l holds the 4-byte
+// words of rows l, l + 32, l + 64, l + 96, byte j of a word being the scale of
+// K block j.  tcgen05.cp .32x128b.warpx4 puts the atom in 4 TMEM columns (the
+// 32 rows into every lane quarter); an MMA over K block j names byte j through
+// the scale ids of its instruction descriptor.  For a CTA pair, the even CTA's
+// copy moves each CTA's own atom (same shared-memory offset) into its own TMEM.
+// Source descriptor: no swizzle, K-major, 8-row x 16-byte core matrices 128
+// bytes apart (stride byte offset 128), version 1.
+__device__ __forceinline__ uint64_t sf_atom_desc(uint32_t smem_addr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((smem_addr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>(128u >> 4) << 16;
+  d |= static_cast<uint64_t>(128u >> 4) << 32;
+  d |= static_cast<uint64_t>(1u) << 46;
+  return d;
+}
+
+__device__ __forceinline__ void tmem_cp_sf_pair(uint32_t taddr, uint64_t src_desc) {
+  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(src_desc) : "memory");
+}
+
+// Instruction descriptor, kind::mxf8f6f4 with block scales: A E2M1 (type 5 at
+// bits 7-9: the FP4 weights), B E4M3 (type 0 at bits 10-12: the tokens), both
+// K-major, N >> 3 at bits 17-22, UE8M0 scales (bit 23), M >> 4 at bits 24-28,
+// scale ids of B at bits 4-5 and of A at bits 29-30 (the K block within the
+// scale words); the accumulator is fp32.
+__host__ __device__ constexpr uint32_t idesc_e2m1_e4m3_bs(int M, int N, int sf_id) {
+  return (static_cast<uint32_t>(sf_id) << 4) | (5u << 7) | (static_cast<uint32_t>(N >> 3) << 17) | (1u << 23) |
+         (static_cast<uint32_t>(M >> 4) << 24) | (static_cast<uint32_t>(sf_id) << 29);
+}
+
+// The block-scaled pair MMA: one M x N x 32 step, scales read from TMEM at
+// sfa (A's rows) and sfb (B's rows).
+__device__ __forceinline__ void umma_bs_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %6, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%4], [%5], p;\n\t}\n" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate)
+      : "memory");
 }
 
 // D[tmem] (+)= A[smem] * B[smem]^T, one M x N x 16 step, issued by one thread.

@@ -40,6 +40,13 @@
 //             thread; two warps per lane quarter split the columns), apply
 //             SwiGLU or scatter, store to global memory
 // Two accumulator buffers let the epilogue of tile i overlap the MMAs of i+1.
+// FP4 weights (packed E2M1 codes with one power-of-two scale per 32 K
+// elements; DeepSeek V4 infra notes, §6.2 FP4 QAT) go to the tensor core as
+// they are: TMA spreads each 8 bytes of codes over a 16-byte chunk (the operand
+// form kind::mxf8f6f4 reads), the block scales travel as UE8M0 atoms with each
+// stage and are copied into TMEM, and every tile is an operand-swapped
+// block-scaled pair MMA (weights the M = 256 operand with their scales, the
+// E4M3 tokens the N <= 128 operand with scale 1).
 // Every mbarrier wait is bounded in time; on time-out the CTA records an error
 // word, drains its own TMA copies and MMAs (bounded), frees TMEM and exits.
 #include <algorithm>
@@ -115,9 +122,11 @@ __device__ __forceinline__ void decode_tile(const GemmArgs& a, const int* tile_s
   const int nt = a.n_kind[ti.kind] / a.BN;
   ti.m = local / nt;
   ti.n = local - ti.m * nt;
-  const int r = ti.rows - ti.m * Cfg<CG>::kTileM;
-  ti.swap = CG == 2 && a.swap_ok && r < 256;
-  ti.nt = ti.swap ? (r + 15) & ~15 : 0;
+  // FP4: tiles of kF4TileTokens token rows, every one swapped.
+  const int tm = a.fp4 ? kF4TileTokens : Cfg<CG>::kTileM;
+  const int r = ti.rows - ti.m * tm;
+  ti.swap = CG == 2 && (a.fp4 || (a.swap_ok && r < 256));
+  ti.nt = ti.swap ? (min(r, tm) + 15) & ~15 : 0;
   ti.small = CG == 2 && !ti.swap && r <= 128;
 }
 
@@ -159,63 +168,14 @@ __device__ __forceinline__ float glu_unit(float g, float u, const GemmArgs& a) {
   return silu_clamped_product(g, u, a.gate_clamp, a.up_clamp);
 }
 
-// FP4 weights (F4, with F8): expand one converter warp's 32 weight rows of a
-// stage's B slot in place.  The warp's rows r = 32 w + lane own the E4M3 bytes
-// [4096 w, 4096 w + 4096) of the slot (row r at 128 r, its 16-byte chunk c at
-// chunk position c ^ (r & 7): the layout a 128-byte-swizzled TMA load of E4M3
-// rows leaves).  Their packed E2M1 codes (64 bytes a row) arrive in two
-// 64-row boxes, rows 0-63 at byte 2048 and rows 64-127 at byte 10240 of the
-// slot, which puts every warp's input inside its own 4 KB span; the lane's
-// exponent word (its row's four 32-element blocks of this stage) comes in a
-// register.  Every lane reads all of its input before any lane writes
-// (__syncwarp), then writes byte code * 2^s: the magnitude from the
-// exponent's 8-entry table (lut[s + 8], E4M3 codes of 0, 0.5, 1, 1.5, 2, 3, 4,
-// 6 times 2^s) picked by prmt, the sign bit from bit 3 of the code.
-// prmt.b32 in its default mode: byte n of the result is byte (c >> 4n) & 7 of
-// {b, a} (a = bytes 0-3), or, when bit 3 of that selector nibble is set, that
-// byte's top bit replicated over all 8 bits.
-__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t c) {
-  uint32_t d;
-  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
-  return d;
-}
-
-// Four E2M1 codes (the low four nibbles of codes16) -> four E4M3 bytes.
-__device__ __forceinline__ uint32_t e2m1x4_to_e4m3(uint32_t codes16, uint32_t lut_lo, uint32_t lut_hi) {
-  const uint32_t mag = prmt(lut_lo, lut_hi, codes16 & 0x7777u);
-  // Sign set: selector nibble 8 replicates the top bit of byte 0 of 0x80 ->
-  // 0xFF; sign clear: selector nibble 1 picks byte 1, 0x00.
-  const uint32_t t = codes16 & 0x8888u;
-  const uint32_t neg = prmt(0x80u, 0u, t | ((t >> 3) ^ 0x1111u));
-  return mag | (neg & 0x80808080u);
-}
-
-__device__ __forceinline__ void fp4_expand_rows(uint8_t* slot, int w, int lane, uint32_t ex,
-                                                const uint32_t (*lut)[2]) {
-  const uint8_t* in = slot + 2048 + 8192 * (w >> 1) + 64 * (32 * (w & 1) + lane);
-  uint4 p[4];
-#pragma unroll
-  for (int j = 0; j < 4; ++j) p[j] = *reinterpret_cast<const uint4*>(in + 16 * j);
-  __syncwarp();
-  const int r = 32 * w + lane;
-  uint8_t* out = slot + 128 * r;
-  const uint32_t words[16] = {p[0].x, p[0].y, p[0].z, p[0].w, p[1].x, p[1].y, p[1].z, p[1].w,
-                              p[2].x, p[2].y, p[2].z, p[2].w, p[3].x, p[3].y, p[3].z, p[3].w};
-#pragma unroll
-  for (int c = 0; c < 8; ++c) {
-    // Chunk c: elements 16c .. 16c + 15, in block c / 2 (exponent byte c / 2).
-    // s in [-8, 6] by construction; the clamp keeps any other byte inside the table.
-    const int sb = min(max(static_cast<int>(static_cast<int8_t>((ex >> (8 * (c >> 1))) & 0xFFu)) + 8, 0), 14);
-    const uint32_t lo = lut[sb][0], hi = lut[sb][1];
-    const uint32_t w0 = words[2 * c], w1 = words[2 * c + 1];
-    const uint4 v = make_uint4(e2m1x4_to_e4m3(w0, lo, hi), e2m1x4_to_e4m3(w0 >> 16, lo, hi),
-                               e2m1x4_to_e4m3(w1, lo, hi), e2m1x4_to_e4m3(w1 >> 16, lo, hi));
-    *reinterpret_cast<uint4*>(out + ((c ^ (r & 7)) << 4)) = v;
-  }
-}
+// TMEM columns (FP4): the two accumulators take [0, 256); four rotating scale
+// buffers of the weights (4 columns each) follow, then the tokens' constant scales.
+constexpr uint32_t kSfCol = 2 * kF4TileTokens;
+constexpr uint32_t kSfOneCol = kSfCol + 16;
+constexpr int kSfAtomBytes = 512;
 
 template <int MODE, int CG, int ACT, int F8, int F4 = 0>
-__global__ void __launch_bounds__(F4 ? kGemmThreadsF4 : kGemmThreads, 1)
+__global__ void __launch_bounds__(kGemmThreads, 1)
     k_grouped_gemm(const __grid_constant__ GemmArgs a) {
   using C = Cfg<CG>;
   static_assert(!F4 || (F8 && MODE != kRouter && CG == 2), "FP4 weights: the expert GEMMs' E4M3 pair kernels");
@@ -233,13 +193,18 @@ __global__ void __launch_bounds__(F4 ? kGemmThreadsF4 : kGemmThreads, 1)
   // bytes in flight per SM).  No stage layout changes a result.
   const int sa_bytes = (MODE != kRouter && a.a_stage_bytes > 0) ? a.a_stage_bytes : kSmemA;
   const int sb_bytes = MODE == kRouter ? a.BN * kBK * 2 : C::kSmemB;
+  // FP4: each stage also carries its scale atom, and the ring ends with the
+  // tokens' constant atom.
+  const int sf_bytes = F4 ? kSfAtomBytes : 0;
   const int S = MODE == kRouter ? min(8, kRingBytes / (kSmemA + sb_bytes))
-                                : min(kRingMax, kRingBytes / (sa_bytes + sb_bytes));
+                                : min(kRingMax, (kRingBytes - sf_bytes) / (sa_bytes + sb_bytes + sf_bytes));
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sA = smem;                              // S x sa_bytes
   uint8_t* sB = smem + S * sa_bytes;               // S x sb_bytes
+  uint8_t* sSF = sB + S * sb_bytes;                // FP4: S x 512-byte scale atoms
+  uint32_t* s_sf_one = reinterpret_cast<uint32_t*>(sSF + S * sf_bytes);  // FP4: atom of ones (UE8M0 127)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kRingBytes);
   uint64_t* full = bars;
   uint64_t* empty = bars + kRingMax;
@@ -252,40 +217,23 @@ __global__ void __launch_bounds__(F4 ? kGemmThreadsF4 : kGemmThreads, 1)
   uint64_t* xempty = xfull + 4;  // [4]
   uint64_t* gfull = xempty + 4;  // [4]
   uint64_t* gempty = gfull + 4;  // [4]
-  // FP4: each CTA's own TMA loads of a stage complete lfull; full then counts
-  // the converter warps of both CTAs (the expanded tile is what the MMA reads).
-  uint64_t* lfull = gempty + 4;  // [kRingMax]
 
   uint8_t* epi = reinterpret_cast<uint8_t*>(bars) + kBarBytes;  // kEpiWarps x kEpiBytes
   __shared__ uint32_t tmem_slot;
-  __shared__ uint32_t s_lut[F4 ? 15 : 1][2];
-  __shared__ __align__(16) uint32_t s_signal[4];   // FP4: source and target of the odd CTA's signal copies
   __shared__ int abort_flag;
   __shared__ int s_tile_start[kMaxGroups + 1];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = CG == 2 ? cluster_ctarank() : 0;   // 0 = the MMA-issuing CTA
   const bool leader = rank == 0;
-  if (F4 && threadIdx.x < 15) {
-    // E4M3 codes of the 8 E2M1 magnitudes times 2^s, s = threadIdx.x - 8 (exact products).
-    const float mags[8] = {0.f, 0.5f, 1.f, 1.5f, 2.f, 3.f, 4.f, 6.f};
-    const float sc = exp2_int(static_cast<int>(threadIdx.x) - 8);
-    uint32_t lo = 0, hi = 0;
-#pragma unroll
-    for (int m = 0; m < 4; ++m) {
-      lo |= e4m3_rn(__fmul_rn(mags[m], sc)) << (8 * m);
-      hi |= e4m3_rn(__fmul_rn(mags[m + 4], sc)) << (8 * m);
-    }
-    s_lut[threadIdx.x][0] = lo;
-    s_lut[threadIdx.x][1] = hi;
+  if (F4) {
+    for (int i = threadIdx.x; i < 128; i += blockDim.x) s_sf_one[i] = 0x7F7F7F7Fu;
+    fence_proxy_async_smem();   // read by tcgen05.cp (async proxy) after the cluster barrier below
   }
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
-      // FP4: the even CTA's producer (expecting the odd CTA's converter
-      // signals as transaction bytes) and its converter warps.
-      mbar_init(&full[s], F4 ? 1 + kCvtWarps : 1);
+      mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
-      if (F4) mbar_init(&lfull[s], 1);
     }
     for (int b = 0; b < 2; ++b) { mbar_init(&tfull[b], 1); mbar_init(&tempty[b], CG * kEpiWarps); }
     mbar_init(tdone, 1);
@@ -320,7 +268,8 @@ __global__ void __launch_bounds__(F4 ? kGemmThreadsF4 : kGemmThreads, 1)
   // B rows each CTA loads per stage, per matrix (gate and up each for gate/up).
   const uint32_t b_rows = static_cast<uint32_t>(BN / CG);
   const uint32_t stage_bytes = kSmemA + b_rows * kBK * 2 * (MODE == kGateUp ? 2 : 1);
-  const uint32_t acc_stride = static_cast<uint32_t>(n_mma);  // TMEM columns per buffer
+  // TMEM columns per accumulator buffer (FP4: swapped tiles of at most 128 tokens).
+  const uint32_t acc_stride = F4 ? static_cast<uint32_t>(kF4TileTokens) : static_cast<uint32_t>(n_mma);
   // Barriers the pair shares live in the even CTA.
   const uint32_t full0 = CG == 2 ? mapa_shared(full, 0) : 0;
   const uint32_t tempty0 = CG == 2 ? mapa_shared(tempty, 0) : 0;
@@ -341,7 +290,7 @@ __global__ void __launch_bounds__(F4 ? kGemmThreadsF4 : kGemmThreads, 1)
         // loaded with the 64-row box so no unused rows cross into shared memory).
         // Swapped tile: this CTA's nt / 2 token rows (the B operand's half).
         const int a_rows = ti.swap ? ti.nt / 2 : (ti.small ? 64 : 128);
-        const int a_y = ti.a_row0 + ti.m * C::kTileM + static_cast<int>(rank) * a_rows;
+        const int a_y = ti.a_row0 + ti.m * (F4 ? kF4TileTokens : C::kTileM) + static_cast<int>(rank) * a_rows;
         // Rows of A the MMA uses: a_rows (pairs), or the router tile's valid rows.
         const int need = CG == 2 ? a_rows : min(128, ti.rows - ti.m * 128);
         const int box = need <= 16 ? 16 : (need <= 64 ? 64 : 128);
@@ -355,25 +304,30 @@ __global__ void __launch_bounds__(F4 ? kGemmThreadsF4 : kGemmThreads, 1)
         // each accumulator lane holds matching gate and up columns); down - rows
         // [r*BN/2, (r+1)*BN/2) of the tile's output columns.
         if (CG == 2) b_y += static_cast<int>(rank) * (BN / 2);
+        // The host sizes the A slot for the largest token box a tile can need;
+        // a box that would overrun it is reported and nothing is loaded.
+        if (MODE != kRouter && box * kBK * 2 > sa_bytes) {
+          atomicExch(a.err, kDevBadIndex);
+          *abort = 1;
+          ok = false;
+          break;
+        }
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort, a.err, a.timeout_ns)) { ok = false; break; }
           uint8_t* b0 = sB + stage * sb_bytes;
           if (F4) {
-            // This CTA's A rows and its 128 weight rows as packed E2M1 codes in
-            // two 64-row boxes (gate/up: the gate rows, then the up rows;
-            // down: rows 0-63, then 64-127), to bytes 2048 and 10240 of the
-            // slot.  All counted on this CTA's lfull.
-            mbar_arrive_expect_tx(&lfull[stage], static_cast<uint32_t>(box) * 128 + 2 * 64 * 64);
-            // The even CTA's full also expects the odd CTA's converter warps'
-            // 16-byte signal copies (one per warp per stage).
-            if (CG == 2 && leader) mbar_arrive_expect_tx(&full[stage], kCvtWarps * 16);
-            else if (CG == 1) mbar_arrive(&full[stage]);
-            tma_load_2d(sA + stage * sa_bytes, amap, kb * KE, a_y, &lfull[stage]);
-            tma_load_2d(b0 + 2048, &a.mapBp[ti.kind * 2], kb * 64, b_y, &lfull[stage]);
-            if (MODE == kGateUp)
-              tma_load_2d(b0 + 10240, &a.mapBp[ti.kind * 2 + 1], kb * 64, b_y, &lfull[stage]);
-            else
-              tma_load_2d(b0 + 10240, &a.mapBp[ti.kind * 2], kb * 64, b_y + 64, &lfull[stage]);
+            // This CTA's token rows, its 128 weight rows as E2M1 codes (gate/up:
+            // the 64 gate rows, then the 64 up rows; down: 128 rows) and their
+            // scale atom (half h = b_y / (BN / 2) of the kind, stage kb), all
+            // counted on the even CTA's full.  A 4-bit load counts the bytes it
+            // reads (64 a row), not the 128 it fills in shared memory.
+            const uint32_t txf = static_cast<uint32_t>(box) * kBK * 2 + 128 * 64 + kSfAtomBytes;
+            if (leader) mbar_arrive_expect_tx(&full[stage], 2 * txf);
+            const uint32_t fb = full0 + 8 * stage;
+            tma_load_2d_pair(sA + stage * sa_bytes, amap, kb * KE, a_y, fb);
+            tma_load_2d_pair(b0, &a.mapBp[ti.kind * 2], kb * KE, b_y, fb);
+            if (MODE == kGateUp) tma_load_2d_pair(b0 + 64 * 128, &a.mapBp[ti.kind * 2 + 1], kb * KE, b_y, fb);
+            tma_load_2d_pair(sSF + stage * kSfAtomBytes, &a.mapSF[ti.kind], 0, (b_y / (BN / 2)) * nkb + kb, fb);
           } else if (CG == 1) {
             mbar_arrive_expect_tx(&full[stage], tx);
             tma_load_2d(sA + stage * sa_bytes, amap, kb * KE, a_y, &full[stage]);
@@ -392,15 +346,11 @@ __global__ void __launch_bounds__(F4 ? kGemmThreadsF4 : kGemmThreads, 1)
           if (++stage == S) { stage = 0; phase ^= 1u; }
         }
       }
-      if (!ok && (F4 || CG == 1 || leader)) {
+      if (!ok && (CG == 1 || leader)) {
         // Let the copies already in flight land before the CTA goes away
-        // (FP4: this CTA's loads on lfull, and on the even CTA's full the odd
-        // CTA's signal copies, bounded like every other wait).
+        // (bounded like every other wait).
         for (int s = 0; s < S; ++s)
-          if (issued[s] >= 0) {
-            mbar_wait_drain(F4 ? &lfull[s] : &full[s], static_cast<uint32_t>(issued[s]), kDrainNs);
-            if (F4 && leader) mbar_wait_drain(&full[s], static_cast<uint32_t>(issued[s]), kDrainNs);
-          }
+          if (issued[s] >= 0) mbar_wait_drain(&full[s], static_cast<uint32_t>(issued[s]), kDrainNs);
       }
     }
   } else if (warp == 1) {
@@ -418,6 +368,11 @@ __global__ void __launch_bounds__(F4 ? kGemmThreadsF4 : kGemmThreads, 1)
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
+      // FP4: the tokens' scales (all 1) once, and a rotating buffer of 4 TMEM
+      // column groups for the weights' per-stage atoms (tcgen05 operations of
+      // this thread run in issue order, so a copy never overtakes an earlier MMA).
+      uint32_t sf_buf = 0;
+      if (F4) tmem_cp_sf_pair(tmem_base + kSfOneCol, sf_atom_desc(smem_u32(s_sf_one)));
       for (int t = cluster_id; ok && t < total; t += n_clusters) {
         Tile ti;
         decode_tile<CG>(a, s_tile_start, t, ti);
@@ -429,10 +384,7 @@ __global__ void __launch_bounds__(F4 ? kGemmThreadsF4 : kGemmThreads, 1)
         // (gate/up: the 64 gate rows then the 64 up rows of its output columns).
         const uint32_t idesc = ti.swap ? idesc_of(256, ti.nt) : (ti.small ? idesc_small : idesc_full);
         for (int kb = 0; kb < nkb; ++kb) {
-          // FP4: full completes on the converter warps' cluster-scope release arrivals.
-          const bool got = F4 ? mbar_wait_acq_cluster(&full[stage], phase, abort, a.err, a.timeout_ns)
-                              : mbar_wait(&full[stage], phase, abort, a.err, a.timeout_ns);
-          if (!got) { ok = false; break; }
+          if (!mbar_wait(&full[stage], phase, abort, a.err, a.timeout_ns)) { ok = false; break; }
           tc_fence_after();
           // A swapped tile reads the weight rows as its A operand and the token
           // rows as its B operand (the same K order, so the same bits per element).
@@ -440,8 +392,19 @@ __global__ void __launch_bounds__(F4 ? kGemmThreadsF4 : kGemmThreads, 1)
           const uint32_t w_addr = smem_u32(sB + stage * sb_bytes);
           const uint32_t a_addr = ti.swap ? w_addr : tok_addr;
           const uint32_t b_addr = ti.swap ? tok_addr : w_addr;
+          if (F4) {
+            // Block-scaled: K block kk of the stage takes byte kk of the scale words.
+            const uint32_t sfa = tmem_base + kSfCol + 4 * sf_buf;
+            tmem_cp_sf_pair(sfa, sf_atom_desc(smem_u32(sSF + stage * kSfAtomBytes)));
 #pragma unroll
-          for (int kk = 0; kk < kBK / 16; ++kk) {
+            for (int kk = 0; kk < kBK / 16; ++kk)
+              umma_bs_pair(d0, sw128_kmajor_desc(a_addr + kk * 32), sw128_kmajor_desc(b_addr + kk * 32),
+                           idesc_e2m1_e4m3_bs(256, ti.nt, kk), sfa, tmem_base + kSfOneCol,
+                           (kb | kk) != 0 ? 1u : 0u);
+            sf_buf = (sf_buf + 1) & 3u;
+          }
+#pragma unroll
+          for (int kk = 0; kk < (F4 ? 0 : kBK / 16); ++kk) {
             const uint64_t ad = sw128_kmajor_desc(a_addr + kk * 32);
             const uint64_t bd = sw128_kmajor_desc(b_addr + kk * 32);
             const uint32_t accum = (kb | kk) != 0 ? 1u : 0u;
@@ -466,48 +429,6 @@ __global__ void __launch_bounds__(F4 ? kGemmThreadsF4 : kGemmThreads, 1)
       if (CG == 2) umma_commit_pair_mc(tdone, 0x1);
       else umma_commit(tdone);
       mbar_wait_drain(tdone, 0, kDrainNs);
-    }
-  } else if (F4 && warp >= 2 + kEpiWarps) {
-    // ----------------------------------------------------- FP4 converters
-    // Warp w expands its 32 weight rows of every stage in the order the
-    // producer fills them, then hands the stage to the MMA issuer: each lane
-    // fences its writes into the async proxy, and after __syncwarp lane 0 of
-    // an even-CTA warp arrives on full, while lane 0 of an odd-CTA warp
-    // issues a 16-byte bulk copy to the even CTA that completes its bytes on
-    // full (an async-proxy signal, ordered after the fenced writes, that
-    // leaves the warp free to go on).  Each lane's exponent words are read
-    // from global memory two stages ahead.
-    const int w = warp - 2 - kEpiWarps;
-    const uint32_t full0c = mapa_shared(full, 0);
-    const uint32_t sig0c = mapa_shared(s_signal, 0);
-    const int mat = (MODE == kGateUp && w >= 2) ? 1 : 0;
-    const int row_in = MODE == kGateUp ? 32 * (w & 1) + lane : 32 * w + lane;
-    int stage = 0;
-    uint32_t phase = 0;
-    bool ok = true;
-    for (int t = cluster_id; ok && t < total; t += n_clusters) {
-      Tile ti;
-      decode_tile<CG>(a, s_tile_start, t, ti);
-      const int nkb = a.k_kind[ti.kind] / KE;
-      const int sel = ti.kind * 2 + mat;
-      const int row = ti.idx * a.n_kind[ti.kind] + ti.n * BN + static_cast<int>(rank) * (BN / 2) + row_in;
-      const uint32_t* xp = a.bexp[sel] + row;
-      const size_t xstride = static_cast<size_t>(a.bexp_rows[sel]);
-      uint32_t ex0 = __ldg(xp), ex1 = nkb > 1 ? __ldg(xp + xstride) : 0u;
-      for (int kb = 0; kb < nkb; ++kb) {
-        ok = mbar_wait(&lfull[stage], phase, abort, a.err, a.timeout_ns);
-        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-        fp4_expand_rows(sB + stage * sb_bytes, w, lane, ex0, s_lut);
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          if (leader) mbar_arrive(&full[stage]);
-          else bulk_copy_s2cluster(sig0c, s_signal, 16, full0c + 8 * stage);
-        }
-        ex0 = ex1;
-        if (kb + 2 < nkb) ex1 = __ldg(xp + static_cast<size_t>(kb + 2) * xstride);
-        if (++stage == S) { stage = 0; phase ^= 1u; }
-      }
     }
   } else {
     // --------------------------------------------------------- epilogue
@@ -543,8 +464,9 @@ __global__ void __launch_bounds__(F4 ? kGemmThreadsF4 : kGemmThreads, 1)
       } else if (CG == 2 && ti.swap) {
         // Operand-swapped tile: TMEM lanes are output columns, TMEM columns are
         // the tile's tokens (rows m * 256 + j of the group, j < r valid).
-        const int r = min(256, ti.rows - ti.m * C::kTileM);
-        const int trow0 = ti.m * C::kTileM;
+        const int tm = F4 ? kF4TileTokens : C::kTileM;
+        const int r = min(tm, ti.rows - ti.m * tm);
+        const int trow0 = ti.m * tm;
         if (MODE == kGateUp) {
           // Lanes 0-63 hold the gate rows and lanes 64-127 the up rows of the CTA's
           // 64 output columns; TMEM columns are tokens.  A gate warp (lane quarter
@@ -863,7 +785,7 @@ cudaLaunchConfig_t pair_config(int grid, cudaStream_t s, cudaLaunchAttribute* at
 
 template <int MODE, int CG, int ACT = MOE_ACT_SWIGLU, int F8 = 0, int F4 = 0>
 cudaError_t launch_one(const GemmArgs& a, int grid, cudaStream_t s) {
-  return launch_k(k_grouped_gemm<MODE, CG, ACT, F8, F4>, dim3(grid), dim3(F4 ? kGemmThreadsF4 : kGemmThreads),
+  return launch_k(k_grouped_gemm<MODE, CG, ACT, F8, F4>, dim3(grid), dim3(kGemmThreads),
                   kGemmSmem, s, CG == 2, a);
 }
 
@@ -903,7 +825,6 @@ void gemm_prepare() {
   occ(reinterpret_cast<const void*>(k_grouped_gemm<kGateUp, 2, 1, 1>));
   occ(reinterpret_cast<const void*>(k_grouped_gemm<kDown, 2, 0, 0>));
   occ(reinterpret_cast<const void*>(k_grouped_gemm<kDown, 2, 0, 1>));
-  cfg.blockDim = dim3(kGemmThreadsF4, 1, 1);
   occ(reinterpret_cast<const void*>(k_grouped_gemm<kGateUp, 2, 0, 1, 1>));
   occ(reinterpret_cast<const void*>(k_grouped_gemm<kGateUp, 2, 1, 1, 1>));
   occ(reinterpret_cast<const void*>(k_grouped_gemm<kDown, 2, 0, 1, 1>));

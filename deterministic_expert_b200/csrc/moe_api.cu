@@ -21,7 +21,7 @@ struct moe_handle {
   int S = 0, G = 0, E_pad = 0, bn_gu = 0, bn_dn = 0, num_sms = 0, device = 0, max_pairs = 0;
   int L = 0;                          // width the router and routed experts read (latent or D)
   bool fp8 = false;                   // MOE_WEIGHTS_FP8 or _FP4: E4M3 expert GEMMs
-  bool fp4 = false;                   // MOE_WEIGHTS_FP4: packed E2M1 weights expanded on chip
+  bool fp4 = false;                   // MOE_WEIGHTS_FP4: packed E2M1 weights, block-scaled MMAs
   int ep_world = 1, ep_rank = 0;      // expert parallelism (1: none)
   int E_loc = 0;                      // routed experts held here (E / ep_world)
   long long cap = 0;                  // rows a rank can receive: ep_world * T_max * k
@@ -30,6 +30,10 @@ struct moe_handle {
   CUtensorMap map_router, map_wg, map_wu, map_wd, map_wsg, map_wsu, map_wsd, map_pd, map_pu;
   // MOE_WEIGHTS_FP4: the expert matrices as packed codes and their exponent words.
   CUtensorMap pmap_wg, pmap_wu, pmap_wd, pmap_wsg, pmap_wsu, pmap_wsd;
+  // FP4: the block scales as the GEMMs' UE8M0 atoms (built at init, owned here)
+  // and their maps: routed gate/up, routed down, shared gate/up, shared down.
+  uint32_t* sf_atoms[4] = {nullptr, nullptr, nullptr, nullptr};
+  CUtensorMap smap[4];
   unsigned long long timeout_ns = 2000ull * 1000 * 1000;
   // Decode-sized batches run the shared experts (which need no routing) on an
   // auxiliary stream while the routing front end runs on the caller's stream;
@@ -189,18 +193,37 @@ bool make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t rows, ui
 }
 
 // MOE_WEIGHTS_FP4: a [rows, K] expert matrix stored as packed E2M1 codes
-// (uint8 [rows, K/2]): boxes of 64 bytes (128 codes, one stage of K) x 64 rows,
-// no swizzle (rows 64 bytes apart).
-bool make_packed_map(CUtensorMap* m, const void* ptr, uint64_t K, uint64_t rows) {
+// (uint8 [rows, K/2], two codes a byte, low nibble first), loaded as 4-bit
+// elements that TMA spreads 16 to a 16-byte chunk (8 bytes of codes, 8 unused:
+// the layout the tensor core reads E2M1 operands in), 128-byte swizzled, boxes
+// of 128 codes (one K stage) x box_rows rows.  Needs a 32-byte aligned base,
+// K a multiple of 128 and rows K/2 bytes apart (a multiple of 32).
+bool make_packed_map(CUtensorMap* m, const void* ptr, uint64_t K, uint64_t rows, uint32_t box_rows) {
   std::memset(m, 0, sizeof(*m));
   if (rows == 0 || ptr == nullptr) return true;
   auto fn = encode_fn();
   if (!fn) return false;
-  cuuint64_t dims[2] = {K / 2, rows};
+  cuuint64_t dims[2] = {K, rows};
   cuuint64_t strides[1] = {K / 2};
-  cuuint32_t box[2] = {64, 64};
+  cuuint32_t box[2] = {128, box_rows};
   cuuint32_t estr[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// MOE_WEIGHTS_FP4: n 512-byte scale atoms as a [n, 128] uint32 tensor, one
+// atom per box.
+bool make_sf_map(CUtensorMap* m, const void* ptr, uint64_t n) {
+  std::memset(m, 0, sizeof(*m));
+  if (n == 0 || ptr == nullptr) return true;
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {128, n};
+  cuuint64_t strides[1] = {512};
+  cuuint32_t box[2] = {128, 1};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void*>(ptr), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -236,8 +259,8 @@ int validate_config(const moe_config* c, const moe_weights* w) {
   if (c->weight_format != MOE_WEIGHTS_BF16 &&
       (c->D % 128 || c->I % 128 || (c->n_shared > 0 && c->I_shared % 128) || c->latent % 128))
     return MOE_EUNSUPPORTED;
-  // FP4: every CTA of a pair expands 128 weight rows a stage (four converter
-  // warps of 32), so gate/up tiles of 128 columns and down tiles of 256.
+  // FP4: every CTA of a pair holds 128 weight rows with one scale atom a
+  // stage, so gate/up tiles of 128 columns and down tiles of 256.
   if (c->weight_format == MOE_WEIGHTS_FP4 && (c->D % 256 || c->latent % 256)) return MOE_EUNSUPPORTED;
   if (c->weight_format == MOE_WEIGHTS_FP4) {
     if (!w->w_gate_exp || !w->w_up_exp || !w->w_down_exp) return MOE_EINVAL;
@@ -245,6 +268,10 @@ int validate_config(const moe_config* c, const moe_weights* w) {
     const void* ep[] = {w->w_gate_exp, w->w_up_exp, w->w_down_exp, w->ws_gate_exp, w->ws_up_exp, w->ws_down_exp};
     for (const void* p : ep)
       if (p && !aligned16(p)) return MOE_EINVAL;
+    // 4-bit TMA loads need 32-byte aligned packed weights.
+    const void* pw[] = {w->w_gate, w->w_up, w->w_down, w->ws_gate, w->ws_up, w->ws_down};
+    for (const void* p : pw)
+      if (p && (reinterpret_cast<uintptr_t>(p) & 31u) != 0) return MOE_EINVAL;
   }
   if (c->D > 16384 || c->E > 256 || c->k > c->E || c->k > 16 || c->n_shared > 8 || c->T_max > (1 << 20))
     return MOE_EUNSUPPORTED;
@@ -264,27 +291,30 @@ int validate_config(const moe_config* c, const moe_weights* w) {
 // tile with at most ceil(T rounded up to 16 / 2) token rows per CTA; the GEMM
 // then sizes its stages' A slot to the TMA box that covers them (16, 64 or 128
 // rows).  0: the default 16 KB slot.
-// MOE_WEIGHTS_FP4: the exponent words the expert GEMM's converter warps read
-// (base and rows of each B operand, as mapB orders them).
-void fp4_exponents(const moe_handle* h, GemmArgs& g, bool gateup) {
-  if (!h->fp4) return;
-  const moe_config& c = h->cfg;
-  if (gateup) {
-    g.bexp[0] = h->w.w_gate_exp; g.bexp[1] = h->w.w_up_exp;
-    g.bexp[2] = h->w.ws_gate_exp; g.bexp[3] = h->w.ws_up_exp;
-    g.bexp_rows[0] = g.bexp_rows[1] = h->E_loc * c.I;
-    g.bexp_rows[2] = g.bexp_rows[3] = h->S * c.I_shared;
-  } else {
-    g.bexp[0] = h->w.w_down_exp; g.bexp[2] = h->w.ws_down_exp;
-    g.bexp_rows[0] = h->E_loc * h->L;
-    g.bexp_rows[2] = h->S * c.D;
-  }
-}
-
 int small_batch_a_bytes(int T) {
   if (T >= 256) return 0;
   const int rows = ((T + 15) / 16 * 16) / 2;
   return (rows <= 16 ? 16 : (rows <= 64 ? 64 : 128)) * kBK * 2;
+}
+
+// MOE_WEIGHTS_FP4: the scale-atom maps of an expert GEMM (per kind: routed, shared).
+void fp4_exponents(const moe_handle* h, GemmArgs& g, bool gateup) {
+  if (!h->fp4) return;
+  g.mapSF[0] = h->smap[gateup ? 0 : 1];
+  g.mapSF[1] = h->smap[gateup ? 2 : 3];
+}
+
+// Rows per M-tile of the expert GEMMs (FP4: swapped tiles of at most 128 tokens).
+int tile_rows(const moe_handle* h) { return h->fp4 ? kF4TileTokens : kPairTileM; }
+
+// A bytes per stage of the expert GEMMs: FP4 tiles hold at most 64 token rows
+// per CTA; otherwise small batches size the slot to their TMA box.
+int expert_a_bytes(const moe_handle* h, int T, bool swap_ok) {
+  if (h->fp4) {
+    const int b = small_batch_a_bytes(T);
+    return (b == 0 || b > 64 * kBK * 2) ? 64 * kBK * 2 : b;
+  }
+  return swap_ok ? small_batch_a_bytes(T) : 0;
 }
 
 int gemm_grid(const moe_handle* h, int tiles_bound) {
@@ -328,9 +358,9 @@ struct Prof {
 int expert_tile_bound(const moe_handle* h, int T, int nt_routed, int nt_shared) {
   const moe_config& c = h->cfg;
   const long long tk = static_cast<long long>(T) * c.k;
-  const long long mt = (tk + kPairTileM - 1) / kPairTileM + std::min<long long>(c.E, tk);
-  const long long b = mt * nt_routed +
-                      static_cast<long long>(h->S) * ((T + kPairTileM - 1) / kPairTileM) * nt_shared;
+  const int tm = tile_rows(h);
+  const long long mt = (tk + tm - 1) / tm + std::min<long long>(c.E, tk);
+  const long long b = mt * nt_routed + static_cast<long long>(h->S) * ((T + tm - 1) / tm) * nt_shared;
   return static_cast<int>(std::min<long long>(b, 1 << 29));
 }
 
@@ -341,7 +371,7 @@ int pair_grid(const moe_handle* h, int tiles_bound) {
 
 // Shared-expert tiles of the gate/up GEMM for T rows.
 int shared_gateup_tiles(const moe_handle* h, int T) {
-  return h->S * ((T + kPairTileM - 1) / kPairTileM) * (h->cfg.I_shared / h->bn_gu);
+  return h->S * ((T + tile_rows(h) - 1) / tile_rows(h)) * (h->cfg.I_shared / h->bn_gu);
 }
 
 // Whether a forward of T rows runs the shared experts on the auxiliary stream:
@@ -434,7 +464,7 @@ int forward_impl(moe_handle* h, int T, const uint16_t* x, const uint16_t* residu
   auto expert_gemms = [&](Part part, cudaStream_t st) -> int {
     const bool routed = part != kSharedGroups, shared = part != kRoutedGroups && h->S > 0;
     const bool timed = st == s;   // stage timing covers the caller's stream only
-    const int mt_shared = (T + kPairTileM - 1) / kPairTileM;
+    const int mt_shared = (T + tile_rows(h) - 1) / tile_rows(h);
     // Which groups a launch walks: the device tile list (all groups, or its
     // routed prefix), or the shared groups alone.
     auto select = [&](GemmArgs& g, int32_t* tiles, int nt_routed, int nt_shared) {
@@ -472,7 +502,7 @@ int forward_impl(moe_handle* h, int T, const uint16_t* x, const uint16_t* residu
       g.k_kind[0] = LW; g.k_kind[1] = c.D;
       g.BN = h->bn_gu;
       g.swap_ok = h->bn_gu == 128;
-      g.a_stage_bytes = g.swap_ok ? small_batch_a_bytes(T) : 0;
+      g.a_stage_bytes = expert_a_bytes(h, T, g.swap_ok);
       g.shared_a_stride = 0;
       g.out[0] = hb; g.ld_out[0] = c.I;
       g.out[1] = hsb; g.ld_out[1] = c.I_shared;
@@ -519,7 +549,7 @@ int forward_impl(moe_handle* h, int T, const uint16_t* x, const uint16_t* residu
       g.k_kind[0] = c.I; g.k_kind[1] = c.I_shared;
       g.BN = h->bn_dn;
       g.swap_ok = h->bn_dn == 256;
-      g.a_stage_bytes = g.swap_ok ? small_batch_a_bytes(T) : 0;
+      g.a_stage_bytes = expert_a_bytes(h, T, g.swap_ok);
       g.shared_a_stride = T;
       g.out[0] = y; g.ld_out[0] = LW;
       g.out[1] = ys; g.ld_out[1] = c.D;
@@ -605,7 +635,7 @@ int forward_impl(moe_handle* h, int T, const uint16_t* x, const uint16_t* residu
   da.dn_ntiles = LW / h->bn_dn;
   da.dn_ntiles_shared = c.D / h->bn_dn;
   da.dest_row = dest; da.src_token = src; da.err = err;
-  da.tile_m = kPairTileM;
+  da.tile_m = tile_rows(h);
   prof.begin(3);
   MOE_TRY(launch_dispatch(da, s));
   prof.end(3);
@@ -735,10 +765,26 @@ int moe_init(const moe_config* cfg, const moe_weights* w, moe_handle** out) {
   if (ok && h->fp4) {
     const uint64_t rg = static_cast<uint64_t>(h->E_loc) * c.I, rd = static_cast<uint64_t>(h->E_loc) * h->L;
     const uint64_t rsg = static_cast<uint64_t>(h->S) * c.I_shared, rsd = static_cast<uint64_t>(h->S) * c.D;
-    ok = make_packed_map(&h->pmap_wg, w->w_gate, h->L, rg) && make_packed_map(&h->pmap_wu, w->w_up, h->L, rg) &&
-         make_packed_map(&h->pmap_wd, w->w_down, c.I, rd) && make_packed_map(&h->pmap_wsg, w->ws_gate, c.D, rsg) &&
-         make_packed_map(&h->pmap_wsu, w->ws_up, c.D, rsg) &&
-         make_packed_map(&h->pmap_wsd, w->ws_down, c.I_shared, rsd);
+    ok = make_packed_map(&h->pmap_wg, w->w_gate, h->L, rg, 64) && make_packed_map(&h->pmap_wu, w->w_up, h->L, rg, 64) &&
+         make_packed_map(&h->pmap_wd, w->w_down, c.I, rd, 128) &&
+         make_packed_map(&h->pmap_wsg, w->ws_gate, c.D, rsg, 64) &&
+         make_packed_map(&h->pmap_wsu, w->ws_up, c.D, rsg, 64) &&
+         make_packed_map(&h->pmap_wsd, w->ws_down, c.I_shared, rsd, 128);
+    // The scale atoms: gate/up halves of 64 + 64 rows, down halves of 128 rows.
+    struct Src { const uint32_t* first; const uint32_t* second; uint64_t rows; int KC; };
+    const Src src[4] = {{w->w_gate_exp, w->w_up_exp, rg, h->L / 128},
+                        {w->w_down_exp, nullptr, rd, c.I / 128},
+                        {w->ws_gate_exp, w->ws_up_exp, rsg, c.D / 128},
+                        {w->ws_down_exp, nullptr, rsd, c.I_shared / 128}};
+    for (int i = 0; ok && i < 4; ++i) {
+      if (src[i].rows == 0) continue;
+      const uint64_t atoms = src[i].rows / (src[i].second ? 64 : 128) * static_cast<uint64_t>(src[i].KC);
+      ok = cudaMalloc(&h->sf_atoms[i], atoms * 512) == cudaSuccess &&
+           launch_fp4_scale_atoms(src[i].first, src[i].second, static_cast<long long>(src[i].rows), src[i].KC,
+                                  h->sf_atoms[i], nullptr) == cudaSuccess &&
+           make_sf_map(&h->smap[i], h->sf_atoms[i], atoms);
+    }
+    ok = ok && cudaDeviceSynchronize() == cudaSuccess;
   }
   if (!ok) return fail(MOE_ECUDA);
   *out = h;
@@ -1115,15 +1161,15 @@ int moe_ep_experts_wave(moe_handle* h, int T, const moe_ep_peers* peers, int wav
   pa.world = h->ep_world; pa.rank = h->ep_rank; pa.E_loc = h->E_loc; pa.S = h->S; pa.T_self = T;
   pa.offsets = off; pa.tiles_gu = tg; pa.tiles_dn = td; pa.rows_received = nrows;
   pa.gu_ntiles_routed = nt_gu; pa.gu_ntiles_shared = nt_gus; pa.dn_ntiles = nt_dn; pa.dn_ntiles_shared = nt_dns;
-  pa.tile_m = kPairTileM;
+  pa.tile_m = tile_rows(h);
   pa.wave_lo = wlo; pa.wave_hi = whi; pa.with_shared = with_shared ? 1 : 0;
   MOE_TRY(launch_ep_plan(pa, s));
   const long long cap = h->cap;
   const int G = h->E_loc + h->S;
   // Tiles at most: sum over local experts of ceil(rows / 256) <= cap / 256 + E_loc.
   auto bound = [&](int nt_r, int nt_s) {
-    const long long b = (cap / kPairTileM + h->E_loc) * nt_r +
-                        static_cast<long long>(h->S) * ((T + kPairTileM - 1) / kPairTileM) * nt_s;
+    const int tm = tile_rows(h);
+    const long long b = (cap / tm + h->E_loc) * nt_r + static_cast<long long>(h->S) * ((T + tm - 1) / tm) * nt_s;
     return static_cast<int>(std::min<long long>(b, 1 << 29));
   };
   const uint8_t* recv = self + X.recv;
@@ -1153,6 +1199,9 @@ int moe_ep_experts_wave(moe_handle* h, int T, const moe_ep_peers* peers, int wav
     g.k_kind[0] = h->L; g.k_kind[1] = c.D;
     g.BN = h->bn_gu;
     g.swap_ok = h->bn_gu == 128;
+    // FP4: the owner's groups hold rows from every rank, so tiles reach 128
+    // tokens whatever this rank's T: the full 64-row A slot.
+    g.a_stage_bytes = h->fp4 ? 64 * kBK * 2 : 0;
     g.shared_a_stride = 0;
     g.out[0] = hr; g.ld_out[0] = c.I;
     g.out[1] = hsb; g.ld_out[1] = c.I_shared;
@@ -1199,6 +1248,7 @@ int moe_ep_experts_wave(moe_handle* h, int T, const moe_ep_peers* peers, int wav
     g.k_kind[0] = c.I; g.k_kind[1] = c.I_shared;
     g.BN = h->bn_dn;
     g.swap_ok = h->bn_dn == 256;
+    g.a_stage_bytes = h->fp4 ? 64 * kBK * 2 : 0;
     g.shared_a_stride = T;
     g.out[0] = nullptr; g.ld_out[0] = h->L;
     g.out[1] = ys; g.ld_out[1] = c.D;
@@ -1327,6 +1377,8 @@ int moe_destroy(moe_handle* h) {
   if (h->ev_join) cudaEventDestroy(h->ev_join);
   if (h->aux) cudaStreamDestroy(h->aux);
   if (h->w_router_pad) cudaFree(h->w_router_pad);
+  for (auto* p : h->sf_atoms)
+    if (p) cudaFree(p);
   delete h;
   return MOE_OK;
 }

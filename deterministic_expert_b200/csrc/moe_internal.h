@@ -47,8 +47,10 @@ constexpr int kBK = 64;
 constexpr int kStages = 4;
 constexpr int kEpiWarps = 8;       // two per TMEM lane quarter, splitting the columns
 constexpr int kGemmThreads = 64 + 32 * kEpiWarps;  // warp 0: TMA, warp 1: MMA, warps 2-9: epilogue
-constexpr int kCvtWarps = 4;                        // FP4 weights: warps 10-13 expand them to E4M3
-constexpr int kGemmThreadsF4 = kGemmThreads + 32 * kCvtWarps;
+// FP4 expert weights: every tile is operand-swapped with at most this many
+// token rows (the weights are the M = 256 operand, the tokens N <= 128), so
+// the two accumulators take 2 x 128 TMEM columns and the block scales fit beside.
+constexpr int kF4TileTokens = 128;
 constexpr int kSmemA = kBM * kBK * 2;
 constexpr int kSmemBMax = 256 * kBK * 2;
 constexpr int kEpiBytes = 32 * 128;  // per epilogue warp: 32 rows x 128 B, XOR-swizzled
@@ -63,10 +65,12 @@ struct GemmArgs {
   CUtensorMap mapA16[2];  // ... and a 16-row box (swapped tiles of up to 32 tokens)
   CUtensorMap mapB[4];    // B operands: [kind * 2 + 0] first (gate / down / router),
                           //             [kind * 2 + 1] second (up; gate/up only)
-  CUtensorMap mapBp[4];   // fp4: the same B operands as packed E2M1 codes (uint8 [rows, K/2],
-                          //      64-byte x 64-row boxes, no swizzle)
-  const uint32_t* bexp[4];// fp4: their block exponent words, uint32 [K/128, bexp_rows[i]]
-  int bexp_rows[4];
+  CUtensorMap mapBp[4];   // fp4: the same weight operands as packed E2M1 codes, loaded as
+                          //      16U4_ALIGN16B (16 codes per 16-byte chunk) with 128-byte
+                          //      swizzling: 128 codes x 64 rows (gate/up) or 128 rows (down)
+  CUtensorMap mapSF[2];   // fp4, per kind: the weights' block scales as UE8M0 scale atoms
+                          //      (512 bytes each: a CTA's 128 weight rows x one 128-wide
+                          //      K stage), atom (h, kc) at row h * K/128 + kc, one per box
   const int* offsets;     // [E + 1] grouped-row offsets of the routed groups
   const int* tile_start;  // [G + 1] first tile of each group; NULL: one group of T rows
   int G, E, T;
@@ -84,8 +88,8 @@ struct GemmArgs {
                           // this many tiles per group, group s at tiles [s * n, (s + 1) * n)
   int out_bf16;           // down-mode output as bf16 instead of fp32 (latent projection)
   int fp8;                // expert GEMMs: A and B are E4M3 codes (kind::f8f6f4)
-  int fp4;                // fp8 with B stored as packed E2M1 + block exponents (expanded
-                          // to E4M3 in shared memory by the converter warps)
+  int fp4;                // fp8 with the weights stored as packed E2M1 + block scales:
+                          // block-scaled MMAs (kind::mxf8f6f4), every tile swapped
   int ep;                 // down, routed: dest_row = rank << 24 | row, stored at out_rank[rank]
   int ep_world;           // ep: ranks
   int a_rows[2];          // rows of each kind's A tensor (index checks; 0 = unchecked)
@@ -126,6 +130,15 @@ cudaError_t launch_quant_weights_fp4(const uint16_t* w, uint8_t* w8, int8_t* blo
                                      cudaStream_t s);
 // The same quantisation in storage form: packed E2M1 codes [rows, K/2] and the
 // block exponents as uint32 [K/128, rows] (four int8 per word).
+// FP4 block scales in the order the expert GEMMs read them: for every half h
+// (a CTA's weight rows of a tile) and 128-wide K stage kc, a 512-byte atom whose
+// 16-byte lane row l holds the UE8M0 words (exponent + 127 per 32-element block)
+// of rows l, l + 32, l + 64, l + 96 of the half.  Gate/up halves are 64 rows of
+// `first` (gate) then 64 rows of `second` (up); down halves (second = NULL) are
+// 128 rows of `first`.  exps: uint32 [KC, rows] as moe_quantize_weights_fp4_packed
+// writes them; atoms: [rows_total / half_rows][KC][128] words.
+cudaError_t launch_fp4_scale_atoms(const uint32_t* first, const uint32_t* second, long long rows, int KC,
+                                   uint32_t* atoms, cudaStream_t s);
 cudaError_t launch_quant_weights_fp4_packed(const uint16_t* w, uint8_t* packed, uint32_t* exps, long long rows,
                                             int K, cudaStream_t s);
 // topk_w == NULL: every slot weighs 1.

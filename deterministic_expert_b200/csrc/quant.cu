@@ -1,6 +1,8 @@
 // FP4 expert weights (DeepSeek V4 infra notes, §6.2 FP4 QAT: master weights are
 // quantised to FP4 (E2M1) with one scale factor per block; FP4 -> FP8 is
 // lossless because every E2M1 value times the block's scale is an FP8 value).
+// The storage form (packed codes + exponents) and the scale atoms the
+// block-scaled expert GEMMs read are built here too.
 // One thread per block of 32 consecutive elements along a row (the GEMM's
 // contraction axis): the block's power-of-two scale, each element's nearest
 // E2M1 value, and the E4M3 code of their product, which the expert GEMMs read.
@@ -137,7 +139,43 @@ __global__ void __launch_bounds__(256) k_quant_weights_fp4_packed(const uint16_t
   exps_bytes[((kb >> 2) * rows + row) * 4 + (kb & 3)] = static_cast<uint8_t>(static_cast<int8_t>(s));
 }
 
+// Scale atoms for the block-scaled expert GEMMs: thread (atom, word i) writes
+// word i = 4 l + w of atom (h, kc), the UE8M0 bytes (exponent + 127, per byte)
+// of one weight row's four 32-element blocks of stage kc.  Gate/up halves
+// (second != NULL): w = 0, 1 -> first (gate) rows 64 h + 32 w + l, w = 2, 3 ->
+// second (up) rows 64 h + 32 (w - 2) + l; down halves: rows 128 h + 32 w + l.
+__global__ void __launch_bounds__(256) k_fp4_scale_atoms(const uint32_t* __restrict__ first,
+                                                         const uint32_t* __restrict__ second, long long rows,
+                                                         int KC, uint32_t* __restrict__ atoms, long long words) {
+  const long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (t >= words) return;
+  const int i = static_cast<int>(t & 127);
+  const long long atom = t >> 7;
+  const long long h = atom / KC;
+  const int kc = static_cast<int>(atom - h * KC);
+  const int l = i >> 2, w = i & 3;
+  const uint32_t* src = first;
+  long long row;
+  if (second != nullptr) {
+    if (w >= 2) src = second;
+    row = 64 * h + 32 * (w & 1) + l;
+  } else {
+    row = 128 * h + 32 * w + l;
+  }
+  atoms[t] = __vadd4(src[static_cast<long long>(kc) * rows + row], 0x7F7F7F7Fu);
+}
+
 }  // namespace
+
+cudaError_t launch_fp4_scale_atoms(const uint32_t* first, const uint32_t* second, long long rows, int KC,
+                                   uint32_t* atoms, cudaStream_t s) {
+  const long long words = rows / (second ? 64 : 128) * KC * 128;
+  if (words <= 0) return cudaSuccess;
+  const long long grid = (words + 255) / 256;
+  if (grid > 0x7FFFFFFFll) return cudaErrorInvalidValue;
+  k_fp4_scale_atoms<<<static_cast<unsigned>(grid), 256, 0, s>>>(first, second, rows, KC, atoms, words);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_quant_weights_fp4_packed(const uint16_t* w, uint8_t* packed, uint32_t* exps, long long rows,
                                             int K, cudaStream_t s) {

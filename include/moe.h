@@ -118,14 +118,20 @@ typedef enum moe_weight_format {
                             is the sign, bits 0-2 the index of the magnitude in
                             0, 0.5, 1, 1.5, 2, 3, 4, 6), plus its block exponents
                             (moe_weights.*_exp): one power-of-two scale 2^s per 32
-                            consecutive elements of a row, s in [-8, 6].  The GEMMs
-                            expand each weight tile to the E4M3 values code * 2^s in
-                            shared memory (exact: every such product is an E4M3 value)
-                            and then compute exactly as MOE_WEIGHTS_FP8 does, so the
-                            results are bit for bit those of the E4M3 weights that
-                            moe_quantize_weights_fp4 writes for the same master weights.
-                            Half a byte per weight (plus 1/32 byte of exponent) instead
-                            of one.  Same shape limits as MOE_WEIGHTS_FP8.            */
+                            consecutive elements of a row, s in [-8, 6].  The expert
+                            GEMMs feed the codes to the tensor core's block-scaled
+                            E2M1 x E4M3 MMA (kind::mxf8f6f4, one UE8M0 scale 2^s per
+                            32 weights, the E4M3 activations with scale 1 and their
+                            row scale applied after), every tile operand-swapped with
+                            at most 128 tokens; moe_init copies the exponents into the
+                            order the GEMMs read them (device memory the handle owns,
+                            as many bytes as the exponents).  Each product code * 2^s
+                            is an E4M3 value, and on B200 the results are bit for bit
+                            those of the E4M3 weights that moe_quantize_weights_fp4
+                            writes for the same master weights.  Half a byte per
+                            weight (plus 1/32 byte of exponent) instead of one.  Same
+                            shape limits as MOE_WEIGHTS_FP8, D and latent multiples of
+                            256, and the packed matrices 32-byte aligned.            */
 } moe_weight_format;
 
 typedef struct moe_config {

@@ -1,16 +1,17 @@
 """FP4 expert weights in their storage form (DeepSeek V4 infra notes, §6.2 FP4
 QAT: FP4 (E2M1) weights with one scale per block, dequantised losslessly to
 FP8, FP8 x FP8 GEMMs).  The weights live in HBM as packed E2M1 codes (half a
-byte each) with their block exponents; the expert GEMMs expand every weight
-tile to its E4M3 values in shared memory and then compute exactly as with E4M3
-weights.
+byte each) with their block exponents; the expert GEMMs hand the codes to the
+tensor core's block-scaled E2M1 x E4M3 MMA with the exponents as UE8M0 block
+scales.  Every code times its scale is an E4M3 value, so the products are
+those of the E4M3 weights.
 
 * The packed quantiser writes, code for code and exponent for exponent, the
   oracle's FP4 storage form (pack_fp4 of quantize_weights_fp4).
 * A layer with packed weights gives, bit for bit, the outputs of the same layer
-  with the E4M3 weights of the same master weights (every shape of tile:
-  256-row, 128-row and operand-swapped; SwiGLU and SiTU-GLU; a latent width;
-  hash routing; no shared expert).
+  with the E4M3 weights of the same master weights (whose GEMMs use every shape
+  of tile: 256-row, 128-row and operand-swapped; SwiGLU and SiTU-GLU; a latent
+  width; hash routing; no shared expert).
 * It matches the oracle within the layer tolerances, and its decode batches
   reproduce their rows of the 8192-row batch bit for bit.
 """
