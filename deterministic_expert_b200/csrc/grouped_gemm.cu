@@ -293,9 +293,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int a_y = ti.a_row0 + ti.m * (F4 ? kF4TileTokens : C::kTileM) + static_cast<int>(rank) * a_rows;
         // Rows of A the MMA uses: a_rows (pairs), or the router tile's valid rows.
         const int need = CG == 2 ? a_rows : min(128, ti.rows - ti.m * 128);
-        const int box = need <= 16 ? 16 : (need <= 64 ? 64 : 128);
-        const CUtensorMap* amap =
-            box == 16 ? &a.mapA16[ti.kind] : (box == 64 ? &a.mapA64[ti.kind] : &a.mapA[ti.kind]);
+        const int box = need <= 16 ? 16 : (need <= 32 ? 32 : (need <= 64 ? 64 : 128));
+        const CUtensorMap* amap = box == 16   ? &a.mapA16[ti.kind]
+                                  : box == 32 ? &a.mapA32[ti.kind]
+                                  : box == 64 ? &a.mapA64[ti.kind]
+                                              : &a.mapA[ti.kind];
         const uint32_t tx = stage_bytes - kSmemA + static_cast<uint32_t>(box) * kBK * 2;
         int b_y = ti.idx * a.n_kind[ti.kind] + ti.n * BN;
         const CUtensorMap* bmap = &a.mapB[ti.kind * 2];

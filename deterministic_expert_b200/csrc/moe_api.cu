@@ -289,12 +289,12 @@ int validate_config(const moe_config* c, const moe_weights* w) {
 
 // With T < 256 no group reaches 256 rows, so every expert tile is a swapped
 // tile with at most ceil(T rounded up to 16 / 2) token rows per CTA; the GEMM
-// then sizes its stages' A slot to the TMA box that covers them (16, 64 or 128
-// rows).  0: the default 16 KB slot.
+// then sizes its stages' A slot to the TMA box that covers them (16, 32, 64 or
+// 128 rows).  0: the default 16 KB slot.
 int small_batch_a_bytes(int T) {
   if (T >= 256) return 0;
   const int rows = ((T + 15) / 16 * 16) / 2;
-  return (rows <= 16 ? 16 : (rows <= 64 ? 64 : 128)) * kBK * 2;
+  return (rows <= 16 ? 16 : (rows <= 32 ? 32 : (rows <= 64 ? 64 : 128))) * kBK * 2;
 }
 
 // MOE_WEIGHTS_FP4: the scale-atom maps of an expert GEMM (per kind: routed, shared).
@@ -429,7 +429,7 @@ int forward_impl(moe_handle* h, int T, const uint16_t* x, const uint16_t* residu
     GemmArgs g;
     std::memset(&g, 0, sizeof(g));
     if (!make_map(&g.mapA[1], A, K, T, kBM) || !make_map(&g.mapA64[1], A, K, T, kBM / 2) ||
-        !make_map(&g.mapA16[1], A, K, T, 16))
+        (!make_map(&g.mapA16[1], A, K, T, 16) || !make_map(&g.mapA32[1], A, K, T, 32)))
       return MOE_ECUDA;
     g.mapB[2] = B;
     g.T = T; g.G = 1; g.E = 0;
@@ -485,10 +485,12 @@ int forward_impl(moe_handle* h, int T, const uint16_t* x, const uint16_t* residu
       const void* xs = f8 ? static_cast<const void*>(xq) : static_cast<const void*>(xn);
       if (!make_map(&g.mapA[0], xp, LW, TK, kBM, eb)) return MOE_ECUDA;
       if (!make_map(&g.mapA64[0], xp, LW, TK, kBM / 2, eb)) return MOE_ECUDA;
-      if (!make_map(&g.mapA16[0], xp, LW, TK, 16, eb)) return MOE_ECUDA;
+      if (!make_map(&g.mapA16[0], xp, LW, TK, 16, eb) || !make_map(&g.mapA32[0], xp, LW, TK, 32, eb))
+        return MOE_ECUDA;
       if (h->S > 0 && !make_map(&g.mapA[1], xs, c.D, T, kBM, eb)) return MOE_ECUDA;
       if (h->S > 0 && !make_map(&g.mapA64[1], xs, c.D, T, kBM / 2, eb)) return MOE_ECUDA;
-      if (h->S > 0 && !make_map(&g.mapA16[1], xs, c.D, T, 16, eb)) return MOE_ECUDA;
+      if (h->S > 0 && (!make_map(&g.mapA16[1], xs, c.D, T, 16, eb) || !make_map(&g.mapA32[1], xs, c.D, T, 32, eb)))
+        return MOE_ECUDA;
       g.fp8 = f8;
       g.a_exp[0] = xpe; g.a_exp[1] = xqe;
       g.a_rows[0] = TK; g.a_rows[1] = T;
@@ -532,10 +534,13 @@ int forward_impl(moe_handle* h, int T, const uint16_t* x, const uint16_t* residu
       const uint64_t srows = static_cast<uint64_t>(h->S) * T;
       if (!make_map(&g.mapA[0], ar, c.I, TK, kBM, eb)) return MOE_ECUDA;
       if (!make_map(&g.mapA64[0], ar, c.I, TK, kBM / 2, eb)) return MOE_ECUDA;
-      if (!make_map(&g.mapA16[0], ar, c.I, TK, 16, eb)) return MOE_ECUDA;
+      if (!make_map(&g.mapA16[0], ar, c.I, TK, 16, eb) || !make_map(&g.mapA32[0], ar, c.I, TK, 32, eb))
+        return MOE_ECUDA;
       if (h->S > 0 && !make_map(&g.mapA[1], as, c.I_shared, srows, kBM, eb)) return MOE_ECUDA;
       if (h->S > 0 && !make_map(&g.mapA64[1], as, c.I_shared, srows, kBM / 2, eb)) return MOE_ECUDA;
-      if (h->S > 0 && !make_map(&g.mapA16[1], as, c.I_shared, srows, 16, eb)) return MOE_ECUDA;
+      if (h->S > 0 && (!make_map(&g.mapA16[1], as, c.I_shared, srows, 16, eb) ||
+                       !make_map(&g.mapA32[1], as, c.I_shared, srows, 32, eb)))
+        return MOE_ECUDA;
       g.fp8 = f8;
       g.a_exp[0] = he; g.a_exp[1] = hse;
       g.a_rows[0] = TK; g.a_rows[1] = h->S * T;
@@ -598,7 +603,7 @@ int forward_impl(moe_handle* h, int T, const uint16_t* x, const uint16_t* residu
     std::memset(&g, 0, sizeof(g));
     if (!make_map(&g.mapA[0], xe, LW, T, kBM)) return MOE_ECUDA;
     if (!make_map(&g.mapA64[0], xe, LW, T, kBM / 2)) return MOE_ECUDA;
-    if (!make_map(&g.mapA16[0], xe, LW, T, 16)) return MOE_ECUDA;
+    if (!make_map(&g.mapA16[0], xe, LW, T, 16) || !make_map(&g.mapA32[0], xe, LW, T, 32)) return MOE_ECUDA;
     g.mapB[0] = h->map_router;
     g.T = T;
     g.n_kind[0] = h->E_pad;
@@ -1184,11 +1189,11 @@ int moe_ep_experts_wave(moe_handle* h, int T, const moe_ep_peers* peers, int wav
     std::memset(&g, 0, sizeof(g));
     const void* xs = f8 ? static_cast<const void*>(ws + L.xq) : static_cast<const void*>(xn);
     if (!make_map(&g.mapA[0], recv, h->L, cap, kBM, eb) || !make_map(&g.mapA64[0], recv, h->L, cap, kBM / 2, eb) ||
-        !make_map(&g.mapA16[0], recv, h->L, cap, 16, eb))
+        (!make_map(&g.mapA16[0], recv, h->L, cap, 16, eb) || !make_map(&g.mapA32[0], recv, h->L, cap, 32, eb)))
       return MOE_ECUDA;
     if (h->S > 0 && T > 0 &&
         (!make_map(&g.mapA[1], xs, c.D, T, kBM, eb) || !make_map(&g.mapA64[1], xs, c.D, T, kBM / 2, eb) ||
-         !make_map(&g.mapA16[1], xs, c.D, T, 16, eb)))
+         (!make_map(&g.mapA16[1], xs, c.D, T, 16, eb) || !make_map(&g.mapA32[1], xs, c.D, T, 32, eb))))
       return MOE_ECUDA;
     g.mapB[0] = h->map_wg; g.mapB[1] = h->map_wu; g.mapB[2] = h->map_wsg; g.mapB[3] = h->map_wsu;
     g.fp4 = h->fp4;
@@ -1232,12 +1237,12 @@ int moe_ep_experts_wave(moe_handle* h, int T, const moe_ep_peers* peers, int wav
     const void* as = f8 ? static_cast<const void*>(hqs) : static_cast<const void*>(hsb);
     const uint64_t srows = static_cast<uint64_t>(h->S) * T;
     if (!make_map(&g.mapA[0], ar, c.I, cap, kBM, eb) || !make_map(&g.mapA64[0], ar, c.I, cap, kBM / 2, eb) ||
-        !make_map(&g.mapA16[0], ar, c.I, cap, 16, eb))
+        (!make_map(&g.mapA16[0], ar, c.I, cap, 16, eb) || !make_map(&g.mapA32[0], ar, c.I, cap, 32, eb)))
       return MOE_ECUDA;
     if (h->S > 0 && T > 0 &&
         (!make_map(&g.mapA[1], as, c.I_shared, srows, kBM, eb) ||
          !make_map(&g.mapA64[1], as, c.I_shared, srows, kBM / 2, eb) ||
-         !make_map(&g.mapA16[1], as, c.I_shared, srows, 16, eb)))
+         (!make_map(&g.mapA16[1], as, c.I_shared, srows, 16, eb) || !make_map(&g.mapA32[1], as, c.I_shared, srows, 32, eb))))
       return MOE_ECUDA;
     g.mapB[0] = h->map_wd; g.mapB[2] = h->map_wsd;
     g.fp4 = h->fp4;

@@ -63,6 +63,7 @@ struct GemmArgs {
   CUtensorMap mapA[2];    // A operand per group kind: 0 routed, 1 shared
   CUtensorMap mapA64[2];  // the same A operands with a 64-row box (128-row pair tiles)
   CUtensorMap mapA16[2];  // ... and a 16-row box (swapped tiles of up to 32 tokens)
+  CUtensorMap mapA32[2];  // ... and a 32-row box (swapped tiles of up to 64 tokens)
   CUtensorMap mapB[4];    // B operands: [kind * 2 + 0] first (gate / down / router),
                           //             [kind * 2 + 1] second (up; gate/up only)
   CUtensorMap mapBp[4];   // fp4: the same weight operands as packed E2M1 codes, loaded as
