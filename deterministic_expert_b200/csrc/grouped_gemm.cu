@@ -46,7 +46,7 @@
 // form kind::mxf8f6f4 reads), the block scales travel as UE8M0 atoms with each
 // stage and are copied into TMEM, and every tile is an operand-swapped
 // block-scaled pair MMA (weights the M = 256 operand with their scales, the
-// E4M3 tokens the N <= 128 operand with scale 1).
+// E4M3 tokens the N <= 240 operand with scale 1).
 // Every mbarrier wait is bounded in time; on time-out the CTA records an error
 // word, drains its own TMA copies and MMAs (bounded), frees TMEM and exits.
 #include <algorithm>
@@ -168,10 +168,11 @@ __device__ __forceinline__ float glu_unit(float g, float u, const GemmArgs& a) {
   return silu_clamped_product(g, u, a.gate_clamp, a.up_clamp);
 }
 
-// TMEM columns (FP4): the two accumulators take [0, 256); four rotating scale
-// buffers of the weights (4 columns each) follow, then the tokens' constant scales.
-constexpr uint32_t kSfCol = 2 * kF4TileTokens;
-constexpr uint32_t kSfOneCol = kSfCol + 16;
+// TMEM columns (FP4): the accumulators take [0, 240) and [256, 496); two
+// rotating scale buffers of the weights (4 columns each) follow, then the
+// tokens' constant scales (8 columns: N > 128 reads a second atom).
+constexpr uint32_t kSfCol = 496;
+constexpr uint32_t kSfOneCol = 504;
 constexpr int kSfAtomBytes = 512;
 
 template <int MODE, int CG, int ACT, int F8, int F4 = 0>
@@ -268,8 +269,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   // B rows each CTA loads per stage, per matrix (gate and up each for gate/up).
   const uint32_t b_rows = static_cast<uint32_t>(BN / CG);
   const uint32_t stage_bytes = kSmemA + b_rows * kBK * 2 * (MODE == kGateUp ? 2 : 1);
-  // TMEM columns per accumulator buffer (FP4: swapped tiles of at most 128 tokens).
-  const uint32_t acc_stride = F4 ? static_cast<uint32_t>(kF4TileTokens) : static_cast<uint32_t>(n_mma);
+  const uint32_t acc_stride = static_cast<uint32_t>(n_mma);  // TMEM columns per buffer
   // Barriers the pair shares live in the even CTA.
   const uint32_t full0 = CG == 2 ? mapa_shared(full, 0) : 0;
   const uint32_t tempty0 = CG == 2 ? mapa_shared(tempty, 0) : 0;
@@ -370,11 +370,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      // FP4: the tokens' scales (all 1) once, and a rotating buffer of 4 TMEM
-      // column groups for the weights' per-stage atoms (tcgen05 operations of
-      // this thread run in issue order, so a copy never overtakes an earlier MMA).
+      // FP4: the tokens' scales (all 1, two atoms for up to 256 tokens) once, and
+      // two rotating TMEM column groups for the weights' per-stage atoms
+      // (tcgen05 operations of this thread run in issue order, so a copy never
+      // overtakes an earlier MMA).
       uint32_t sf_buf = 0;
-      if (F4) tmem_cp_sf_pair(tmem_base + kSfOneCol, sf_atom_desc(smem_u32(s_sf_one)));
+      if (F4) {
+        tmem_cp_sf_pair(tmem_base + kSfOneCol, sf_atom_desc(smem_u32(s_sf_one)));
+        tmem_cp_sf_pair(tmem_base + kSfOneCol + 4, sf_atom_desc(smem_u32(s_sf_one)));
+      }
       for (int t = cluster_id; ok && t < total; t += n_clusters) {
         Tile ti;
         decode_tile<CG>(a, s_tile_start, t, ti);
@@ -403,7 +407,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               umma_bs_pair(d0, sw128_kmajor_desc(a_addr + kk * 32), sw128_kmajor_desc(b_addr + kk * 32),
                            idesc_e2m1_e4m3_bs(256, ti.nt, kk), sfa, tmem_base + kSfOneCol,
                            (kb | kk) != 0 ? 1u : 0u);
-            sf_buf = (sf_buf + 1) & 3u;
+            sf_buf ^= 1u;
           }
 #pragma unroll
           for (int kk = 0; kk < (F4 ? 0 : kBK / 16); ++kk) {

@@ -304,17 +304,14 @@ void fp4_exponents(const moe_handle* h, GemmArgs& g, bool gateup) {
   g.mapSF[1] = h->smap[gateup ? 2 : 3];
 }
 
-// Rows per M-tile of the expert GEMMs (FP4: swapped tiles of at most 128 tokens).
+// Rows per M-tile of the expert GEMMs (FP4: swapped tiles of at most 240 tokens).
 int tile_rows(const moe_handle* h) { return h->fp4 ? kF4TileTokens : kPairTileM; }
 
-// A bytes per stage of the expert GEMMs: FP4 tiles hold at most 64 token rows
-// per CTA; otherwise small batches size the slot to their TMA box.
+// A bytes per stage of the expert GEMMs: small batches size the slot to their
+// TMA box (FP4 tiles, every one swapped, hold at most 120 token rows per CTA,
+// within the default slot).
 int expert_a_bytes(const moe_handle* h, int T, bool swap_ok) {
-  if (h->fp4) {
-    const int b = small_batch_a_bytes(T);
-    return (b == 0 || b > 64 * kBK * 2) ? 64 * kBK * 2 : b;
-  }
-  return swap_ok ? small_batch_a_bytes(T) : 0;
+  return (swap_ok || h->fp4) ? small_batch_a_bytes(T) : 0;
 }
 
 int gemm_grid(const moe_handle* h, int tiles_bound) {
@@ -1204,9 +1201,9 @@ int moe_ep_experts_wave(moe_handle* h, int T, const moe_ep_peers* peers, int wav
     g.k_kind[0] = h->L; g.k_kind[1] = c.D;
     g.BN = h->bn_gu;
     g.swap_ok = h->bn_gu == 128;
-    // FP4: the owner's groups hold rows from every rank, so tiles reach 128
-    // tokens whatever this rank's T: the full 64-row A slot.
-    g.a_stage_bytes = h->fp4 ? 64 * kBK * 2 : 0;
+    // The owner's groups hold rows from every rank, so tiles reach their full
+    // height whatever this rank's T: the default A slot.
+    g.a_stage_bytes = 0;
     g.shared_a_stride = 0;
     g.out[0] = hr; g.ld_out[0] = c.I;
     g.out[1] = hsb; g.ld_out[1] = c.I_shared;
@@ -1253,7 +1250,7 @@ int moe_ep_experts_wave(moe_handle* h, int T, const moe_ep_peers* peers, int wav
     g.k_kind[0] = c.I; g.k_kind[1] = c.I_shared;
     g.BN = h->bn_dn;
     g.swap_ok = h->bn_dn == 256;
-    g.a_stage_bytes = h->fp4 ? 64 * kBK * 2 : 0;
+    g.a_stage_bytes = 0;
     g.shared_a_stride = T;
     g.out[0] = nullptr; g.ld_out[0] = h->L;
     g.out[1] = ys; g.ld_out[1] = c.D;

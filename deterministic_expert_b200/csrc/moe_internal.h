@@ -48,9 +48,10 @@ constexpr int kStages = 4;
 constexpr int kEpiWarps = 8;       // two per TMEM lane quarter, splitting the columns
 constexpr int kGemmThreads = 64 + 32 * kEpiWarps;  // warp 0: TMA, warp 1: MMA, warps 2-9: epilogue
 // FP4 expert weights: every tile is operand-swapped with at most this many
-// token rows (the weights are the M = 256 operand, the tokens N <= 128), so
-// the two accumulators take 2 x 128 TMEM columns and the block scales fit beside.
-constexpr int kF4TileTokens = 128;
+// token rows (the weights are the M = 256 operand, the tokens N <= 240), so
+// the two accumulators (columns [0, 240) and [256, 496)) leave 16 TMEM columns
+// for the block scales.
+constexpr int kF4TileTokens = 240;
 constexpr int kSmemA = kBM * kBK * 2;
 constexpr int kSmemBMax = 256 * kBK * 2;
 constexpr int kEpiBytes = 32 * 128;  // per epilogue warp: 32 rows x 128 B, XOR-swizzled

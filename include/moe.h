@@ -123,7 +123,7 @@ typedef enum moe_weight_format {
                             E2M1 x E4M3 MMA (kind::mxf8f6f4, one UE8M0 scale 2^s per
                             32 weights, the E4M3 activations with scale 1 and their
                             row scale applied after), every tile operand-swapped with
-                            at most 128 tokens; moe_init copies the exponents into the
+                            at most 240 tokens; moe_init copies the exponents into the
                             order the GEMMs read them (device memory the handle owns,
                             as many bytes as the exponents).  Each product code * 2^s
                             is an E4M3 value, and on B200 the results are bit for bit

@@ -3,7 +3,8 @@ kernel computes from device data is tested against its buffer before use.
 
 Each test runs in a child process started with MOE_LIBRARY=checked (the
 binding then loads the checked library), so the parent's regular library is
-untouched.  Clean runs must report no index error and give the bits of the
+untouched.  Clean runs (bf16, E4M3 and FP4 layers; an expert-parallel step in
+one pass and in waves) must report no index error and give the bits of the
 regular build's contract (oracle parity, EP == single device); a corrupted
 per-expert count handed between expert-parallel phases must be reported as
 MOE_EINDEX with every out-of-range row skipped (the send kernel writes only
@@ -25,7 +26,7 @@ assert moe.LIB_PATH.endswith("libmoe_checked.so"), moe.LIB_PATH
 import sys; sys.path.insert(0, "tests")
 from gpu_util import Run, verify
 from synth import device as SD, workloads as W
-for cfg in (W.C1, W.C1F, dataclasses.replace(W.C1, T=129, n_shared=0)):
+for cfg in (W.C1, W.C1F, dataclasses.replace(W.C1, T=129, n_shared=0), W.C1P, dataclasses.replace(W.C1P, T=300)):
     run = Run(cfg)
     out = run.forward(*run.inputs())          # asserts device_error == 0
     verify(run, out)
@@ -43,6 +44,12 @@ ws = torch.empty(single.workspace_size(277), dtype=torch.uint8, device="cuda")
 on = torch.empty((277, cfg.D), dtype=torch.bfloat16, device="cuda"); orr = torch.empty_like(on)
 single.forward(x[:277].contiguous(), r[:277].contiguous(), on, orr, ws)
 torch.cuda.synchronize()
+got = torch.cat([o[0] for o in outs])
+assert torch.equal(got.view(torch.int16), on.view(torch.int16))
+# The same step in two waves of experts (wave-limited send and expert phases).
+outs = ep.forward([x[cut[q]:cut[q + 1]] for q in range(4)], [r[cut[q]:cut[q + 1]] for q in range(4)], waves=2)
+torch.cuda.synchronize()
+assert ep.device_errors() == [0, 0, 0, 0], ep.device_errors()
 got = torch.cat([o[0] for o in outs])
 assert torch.equal(got.view(torch.int16), on.view(torch.int16))
 print("CLEAN-OK")
