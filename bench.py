@@ -91,7 +91,9 @@ def describe(cfg):
             "router": {0: "softmax", 1: "sigmoid+bias", 2: "hash"}[cfg.router],
             "renormalize": bool(cfg.renormalize),
             "activation": "SiTU-GLU" if cfg.activation == 1 else "SwiGLU", "latent": cfg.latent,
-            "expert_weights": "FP4 values as E4M3 (E4M3 x E4M3 GEMMs)" if cfg.weight_format else "bf16"}
+            "expert_weights": {0: "bf16", 1: "FP4 values as E4M3 (E4M3 x E4M3 GEMMs)",
+                               2: "FP4 packed E2M1 + UE8M0 block scales (block-scaled E2M1 x E4M3 GEMMs)"}[
+                                   cfg.weight_format]}
 
 
 def bench_config(cfg, world):
@@ -533,8 +535,9 @@ def gemm_roofline(cfg, gate_ms, pk, traffic):
     achieved = fl / (gate_ms / 1e3) / 1e12
     src = f"{pk['kind']} bf16 (burst)"
     if cfg.weight_format:
-        # E4M3 x E4M3: the bf16 peak times the nominal dense ratio of the two formats (4.5 / 2.25 PFLOP/s).
-        src += " x 2, nominal E4M3 / bf16 ratio"
+        # E4M3 x E4M3 and block-scaled E2M1 x E4M3 run at the FP8 rate: the bf16 peak times the
+        # nominal dense ratio of the two formats (4.5 / 2.25 PFLOP/s).
+        src += " x 2, nominal FP8 / bf16 ratio"
     return {"bound": "tensor", "kernel": "gemm_gateup_swiglu", "achieved": round(achieved, 1), "peak": tc,
             "unit": "TFLOP/s", "frac": round(achieved / tc, 4), "traffic": traffic, "peak_source": src,
             "frac_of_nominal": round(achieved / nominal, 4), "nominal_peak": nominal,
@@ -798,7 +801,7 @@ def main():
         sub["fine_grained"] = fg
         sub["decode"] = decode_object(a, dev, flush, stream, pk, w2)
         # The same sweep with the FP4 experts in their storage form (half a
-        # byte per weight plus block exponents, expanded to E4M3 on chip).
+        # byte per weight plus block exponents, block-scaled E2M1 x E4M3 GEMMs).
         sub["decode_fp4"] = decode_object(a, dev, flush, stream, pk, moe.pack_expert_weights_fp4(w2), cfg=W.C2P)
         sub["ep_waves"] = ep_waves_object(a, dev, flush, stream, w2)
         del w2
@@ -812,7 +815,7 @@ def main():
             "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
             "steps": a.steps, "warmup": a.warmup, "ms_per_step": round(ms_per_step, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "e4m3" if cfg.weight_format else "bf16",
+            "dtype": {0: "bf16", 1: "e4m3", 2: "e2m1 x e4m3"}[cfg.weight_format],
             "data": "synthetic (seeded counter-based generator; random weights of the workload's shape)",
             "config": bench_config(cfg, world),
             "roofline": gemm_roofline(cfg, gate_ms, pk, ncu_traffic(cfg)),

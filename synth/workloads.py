@@ -109,7 +109,7 @@ EPILOGUE_SIGMA = 1.0 / 8.0
 # The latent workload with FP4 expert weights (routed and shared).
 C6F = dataclasses.replace(C6, name="latent_situ_fp8", weight_format=1)
 # The same FP4 experts in their storage form (packed E2M1 codes, half a byte a
-# weight, plus block exponents), expanded to E4M3 on chip by the GEMMs.
+# weight, plus block exponents), read as they are by block-scaled GEMMs.
 C1P = dataclasses.replace(C1, name="tiny_fp4", weight_format=2)
 C2P = dataclasses.replace(C2, name="fine_grained_fp4", weight_format=2)
 C6P = dataclasses.replace(C6, name="latent_situ_fp4", weight_format=2)
@@ -271,7 +271,7 @@ def pretty(cfg: MoEConfig) -> str:
     if cfg.weight_format == 1:
         act += " FP4 weights as E4M3 bytes (E4M3 x E4M3 GEMMs)"
     elif cfg.weight_format == 2:
-        act += " FP4 weights packed (E2M1 + block exponents, expanded on chip; E4M3 x E4M3 GEMMs)"
+        act += " FP4 weights packed (E2M1 + block exponents; block-scaled E2M1 x E4M3 GEMMs)"
     return (f"{cfg.name}: T={cfg.T} D={cfg.D}{lat} E={cfg.E} top-{cfg.k} {r} I={cfg.I} "
             f"shared={cfg.n_shared}x{cfg.I_shared}{act}")
 
