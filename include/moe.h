@@ -213,8 +213,12 @@ typedef struct moe_handle moe_handle;
 #define MOE_NUM_STAGES 12
 
 /* Validate `cfg`, keep the weight pointers and build the weight TMA
- * descriptors on the current CUDA device.  Allocates one small handle-owned
- * device buffer (the router weights zero-padded to a multiple of 16 rows).
+ * descriptors on the current CUDA device.  Allocates handle-owned device
+ * memory: the router weights zero-padded to a multiple of 16 rows, and with
+ * MOE_WEIGHTS_FP4 the block exponents rearranged as the expert GEMMs read them
+ * (as many bytes as the exponents; built by a kernel on the legacy default
+ * stream, after which moe_init synchronises the device); the exponent arrays
+ * themselves are read only during moe_init.
  * Returns MOE_EINVAL / MOE_EUNSUPPORTED for bad configs (checked before any
  * CUDA call), MOE_ECUDA when a CUDA call fails.  *out is NULL on failure. */
 int moe_init(const moe_config* cfg, const moe_weights* w, moe_handle** out);
