@@ -558,16 +558,18 @@ def layer_numbers(cfg, T, ms, distinct, pk):
             "frac_of_nominal_hbm": round(gbs / NOMINAL_HBM_GBS, 4)}
 
 
-def fine_grained_object(a, dev, flush, stream, pk):
+def fine_grained_object(a, dev, flush, stream, pk, cfg=None, w=None):
     """The fine-grained workload (T=4096, D=2048, 64 experts top-6 softmax
-    renormalised, I=1408, 2 shared) timed as the headline is."""
+    renormalised, I=1408, 2 shared) timed as the headline is; with cfg / w the
+    same shapes in another weight format (the given weights)."""
     import torch
 
     import deterministic_expert_b200 as moe
     from synth import device as SD
     from synth import workloads as W
-    cfg = W.C2
-    w = SD.device_weights(cfg, device=dev)
+    cfg = W.C2 if cfg is None else cfg
+    if w is None:
+        w = SD.device_weights(cfg, device=dev)
     x, r, _ = SD.device_inputs(cfg, device=dev)
     layer = moe.MoELayer(SD.layer_config(cfg, cfg.T), w)
     ws = torch.empty(layer.workspace_size(cfg.T), dtype=torch.uint8, device=dev)
@@ -802,7 +804,11 @@ def main():
         sub["decode"] = decode_object(a, dev, flush, stream, pk, w2)
         # The same sweep with the FP4 experts in their storage form (half a
         # byte per weight plus block exponents, block-scaled E2M1 x E4M3 GEMMs).
-        sub["decode_fp4"] = decode_object(a, dev, flush, stream, pk, moe.pack_expert_weights_fp4(w2), cfg=W.C2P)
+        w4 = moe.pack_expert_weights_fp4(w2)
+        sub["decode_fp4"] = decode_object(a, dev, flush, stream, pk, w4, cfg=W.C2P)
+        # The prefill-sized batch with the FP4 storage form (block-scaled GEMMs).
+        sub["fine_grained_fp4"], _ = fine_grained_object(a, dev, flush, stream, pk, cfg=W.C2P, w=w4)
+        del w4
         sub["ep_waves"] = ep_waves_object(a, dev, flush, stream, w2)
         del w2
 
